@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Decode-step throughput of libckv on B200 (CommunityKV community-retrieval
+sparse decode, "CommunityKV: Efficient Long-Context Decoding via Graph
+Partitioning", Figure 1 step (3)).
+
+Workload: Qwen3-8B-shaped decode with query-group graphs -- batch 4, 32 query
+heads over 8 KV heads, head_dim 128, bf16 K/V, n = 131072 context tokens,
+communities of 16 (8192 per graph), 4 sinks, budget 4096, kappa 8; seeded
+synthetic clustered keys (long_context_decode_ckv_b200.synth).
+
+A step = ckv_decode_step + ckv_assign_update for all 32 graphs of one layer.
+The timed loop rotates over `--replicas` independent copies of the layer
+(separate K/V caches and community state, > 18 GB in total), so no step finds
+its working set in the 126 MB L2: inputs larger than L2, no flush.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle
+(test infrastructure; the only other code here that runs it is the
+cpu_baseline leg) on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_decode_ckv_b200 import synth  # noqa: E402
+
+CFG = synth.QWEN8B
+WORKLOAD = "qwen3_8b_shape_query_group_b4_h32kv8_d128_n131072_budget4096_k8_s4_bf16"
+METRIC = "decode steps/s"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def algorithmic_bytes(cfg, T):
+    """Bytes one step must move, per graph (T = member tokens kept):
+    centroids N_c*D*4, community offset+size N_c*8, member ids T*4, K and V
+    rows (T+S+1)*D*2*2, queries in and outputs out |H(g)|*D*(2+4)."""
+    Nc, D, S, hg = cfg.n_comm, cfg.head_dim, cfg.n_sinks, cfg.heads_per_graph
+    eb = 2 if cfg.bf16 else 4
+    return (Nc * D * 4 + Nc * 8 + T * 4 + (T + S + 1) * D * eb * 2 + hg * D * (eb + 4))
+
+
+def kernel_bytes(cfg, T):
+    """Algorithmic bytes of the two streaming kernels per graph."""
+    Nc, D, S, hg = cfg.n_comm, cfg.head_dim, cfg.n_sinks, cfg.heads_per_graph
+    eb = 2 if cfg.bf16 else 4
+    return {
+        "score": Nc * D * 4 + Nc * 4 + Nc * 4,                         # centroids, sizes, scores out
+        "attend": (T + S + 1) * D * eb * 2 + T * 4 + hg * D * (eb + 4),  # K/V rows, ids, q, out
+    }
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, index: int):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *exc):
+        time.sleep(0.15)
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in self.rows for k in range(4)
+                          if len(r) > 4 + k and r[4 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ oracle
+def run_oracle_steps(wl, n_steps, graphs=None):
+    """Time the CPU oracle (single thread) on `n_steps` decode steps of the
+    workload; returns (seconds, graph-steps done)."""
+    import oracle
+    cfg = wl.cfg
+    graphs = list(range(cfg.n_graphs)) if graphs is None else graphs
+    og = {}
+    for g in graphs:
+        b, kvh, _ = cfg.graph_heads(g)
+        og[g] = oracle.Graph(cfg.n_comm, cfg.head_dim, cfg.n_max)
+        og[g].init(cfg.n0, cfg.n_sinks, wl.labels[g], wl.K[b, kvh])
+    t0 = time.perf_counter()
+    for i in range(n_steps):
+        n = cfg.n0 + i + 1
+        for g in graphs:
+            b, kvh, heads = cfg.graph_heads(g)
+            oracle.decode_step(og[g], np.ascontiguousarray(wl.q[i, b, heads]), wl.K[b, kvh],
+                               wl.V[b, kvh], n, cfg.n_sinks, cfg.kappa, cfg.budget)
+    return time.perf_counter() - t0, n_steps * len(graphs)
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return 0
+    wl = synth.make_workload(CFG, workers=max(1, min(16, os.cpu_count() or 1)))
+    steps = args.warmup + args.steps
+    if steps > CFG.steps:
+        raise SystemExit(f"--impl reference supports at most {CFG.steps} steps")
+    import oracle
+    cfg = CFG
+    og = {}
+    for g in range(cfg.n_graphs):
+        b, kvh, _ = cfg.graph_heads(g)
+        og[g] = oracle.Graph(cfg.n_comm, cfg.head_dim, cfg.n_max)
+        og[g].init(cfg.n0, cfg.n_sinks, wl.labels[g], wl.K[b, kvh])
+
+    def one(i):
+        n = cfg.n0 + i + 1
+        for g in range(cfg.n_graphs):
+            b, kvh, heads = cfg.graph_heads(g)
+            oracle.decode_step(og[g], np.ascontiguousarray(wl.q[i, b, heads]), wl.K[b, kvh],
+                               wl.V[b, kvh], n, cfg.n_sinks, cfg.kappa, cfg.budget)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, steps):
+        one(i)
+    dt = time.perf_counter() - t0
+    v = args.steps / dt
+    sample = f"{args.steps} full decode steps (all 32 graphs) after {args.warmup} warm-up steps"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ckv", choices=["ckv", "reference"])
+    ap.add_argument("--replicas", type=int, default=0, help="layer copies rotated (0 = auto)")
+    ap.add_argument("--e2e-steps", type=int, default=40)
+    ap.add_argument("--cpu-steps", type=int, default=8)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    # host-side generation first (spawned pool, before any CUDA call)
+    workers = max(1, min(16, (os.cpu_count() or 1) // max(1, world)))
+    t_gen = time.perf_counter()
+    wl = synth.make_workload(CFG, workers=workers)
+    t_gen = time.perf_counter() - t_gen
+
+    import torch
+    import long_context_decode_ckv_b200 as ckv
+    from long_context_decode_ckv_b200 import build as ckv_build
+    ckv_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    cfg = CFG
+    total_steps = args.warmup + args.steps + args.e2e_steps
+    L = args.replicas or max(4, -(-total_steps // cfg.steps))
+    if -(-total_steps // L) > cfg.steps:
+        raise SystemExit("not enough decode tokens in the workload for these steps; raise --replicas")
+
+    def upload(a):
+        t = torch.from_numpy(a)
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).to(dev)
+
+    K0, V0, q = upload(wl.K), upload(wl.V), upload(wl.q)
+    reps = []
+    for r in range(L):
+        K = K0 if r == 0 else K0.clone()
+        V = V0 if r == 0 else V0.clone()
+        c = ckv.ckv_config()
+        c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, 128
+        c.n_max, c.max_communities, c.n_sinks = cfg.n_max, cfg.n_comm, cfg.n_sinks
+        c.kappa, c.budget, c.slack = cfg.kappa, cfg.budget, 16
+        c.kv_dtype, c.mode, c.device, c.pool_capacity = ckv.CKV_BF16, ckv.CKV_QUERY_GROUP, local, 0
+        ctx = ckv.ckv_create(c)
+        ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        reps.append({"ctx": ctx, "K": K, "V": V, "i": 0})
+    out = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sel_tok = np.zeros(cfg.n_graphs, np.int32)
+
+    def step(s):
+        r = reps[s % L]
+        i = r["i"]
+        n = cfg.n0 + i + 1
+        ckv.ckv_decode_step(r["ctx"], q[i], r["K"], r["V"], n, out, stream)
+        ckv.ckv_assign_update(r["ctx"], r["K"], n, stream)
+        r["i"] = i + 1
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize(dev)
+    for r in reps:
+        ckv.ckv_profile_begin(r["ctx"])
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with Clocks(local) as clk:
+        start.record(stream)
+        for s in range(args.warmup, args.warmup + args.steps):
+            step(s)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    ms = start.elapsed_time(end)
+    kern_ms, kern_steps = [0.0] * 4, 0
+    for r in reps:
+        m, k = ckv.ckv_profile_end(r["ctx"])
+        kern_ms = [a + b for a, b in zip(kern_ms, m)]
+        kern_steps += k
+    for r in reps:
+        assert ckv.ckv_last_error(r["ctx"]) == ckv.CKV_OK
+    ckv.ckv_get_step_debug(reps[(args.warmup + args.steps - 1) % L]["ctx"], n_tok_sel=sel_tok)
+    T_mean = float(sel_tok.mean())
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end-to-end through the host-buffer entry point: per step H2D of q and
+    # the new token's K/V rows from pinned memory, D2H of the output
+    e2e = None
+    if args.e2e_steps:
+        qh = torch.from_numpy(wl.q).pin_memory()
+        kh = torch.from_numpy(np.ascontiguousarray(wl.K[:, :, cfg.n0:])).pin_memory()
+        vh = torch.from_numpy(np.ascontiguousarray(wl.V[:, :, cfg.n0:])).pin_memory()
+        oh = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32).pin_memory()
+        kstep = [kh[:, :, i].contiguous() for i in range(cfg.steps)]
+        vstep = [vh[:, :, i].contiguous() for i in range(cfg.steps)]
+        s0 = args.warmup + args.steps
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(s0, s0 + args.e2e_steps):
+            r = reps[s % L]
+            i = r["i"]
+            ckv.ckv_decode_host(r["ctx"], qh[i], kstep[i], vstep[i], r["K"], r["V"], cfg.n0 + i + 1,
+                                oh, stream)
+            r["i"] = i + 1
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([ems], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ems = float(t.item())
+        eb = 2
+        e2e = {"value": world * args.e2e_steps / (ems / 1e3), "unit": "steps/s",
+               "h2d_bytes_per_step": cfg.batch * (cfg.n_q_heads + 2 * cfg.n_kv_heads) * 128 * eb,
+               "d2h_bytes_per_step": cfg.batch * cfg.n_q_heads * 128 * 4}
+
+    for r in reps:
+        ckv.ckv_destroy(r["ctx"])
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    steps_per_s = world * args.steps / (ms / 1e3)
+    per_graph = algorithmic_bytes(cfg, T_mean)
+    step_bytes = per_graph * cfg.n_graphs
+    gbs = step_bytes * args.steps / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    names = ["score", "select", "attend", "assign"]
+    avg = {nm: kern_ms[k] / max(1, kern_steps) for k, nm in enumerate(names)}
+    dom = max(("score", "attend"), key=lambda nm: avg[nm])
+    kb = kernel_bytes(cfg, T_mean)[dom] * cfg.n_graphs
+    achieved = kb / (avg[dom] / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                "traffic": None, "algorithmic_bytes_per_launch": kb,
+                "avg_launch_ms": avg[dom]}
+
+    cpu = None
+    if not args.no_cpu:
+        secs, gsteps = run_oracle_steps(wl, args.cpu_steps)
+        cpu = {"value": (gsteps / cfg.n_graphs) / secs, "unit": "steps/s", "cores": 1, "kind": "oracle",
+               "sample": f"{args.cpu_steps} decode steps x {cfg.n_graphs} graphs of the same workload, "
+                         f"single-threaded C oracle ({secs:.1f} s)"}
+    line = {
+        "metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "graphs": cfg.n_graphs, "layer_replicas": L,
+                   "l2": f"{L} layer replicas rotated (inputs larger than L2), no flush",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "hbm_gbs": gbs, "hbm_frac_of_8000": gbs / NOMINAL_HBM_GBS, "hbm_frac_of_measured": gbs / peak,
+        "algorithmic_bytes_per_step": step_bytes, "mean_tokens_kept": T_mean,
+        "kernel_ms_per_step": avg,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+        "gen_seconds": t_gen,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,215 @@
+/*
+ * ckv.h -- C ABI of libckv: CommunityKV community-retrieval sparse decode
+ * attention and prefill top-kappa graph construction for NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "CommunityKV: Efficient Long-Context Decoding via Graph
+ * Partitioning".  Figure 1's caption gives the three stages: (1) during
+ * prefill each query connects to its top-kappa keys of the attention matrix,
+ * sinks excluded; (2) the token graph is partitioned into communities (the
+ * Leiden partition arrives here as a label array) and each community gets a
+ * centroid; (3) at each decode step the query is scored against the
+ * centroids, the best communities up to a token budget are retrieved, exact
+ * attention runs over them plus the sink tokens, and the new token's
+ * top-kappa keys become its edges and assign it to a community in constant
+ * time (abstract: "a local update rule").  Table 1 gives the costs: O(d)
+ * update, O(sqrt(n) d) retrieval.
+ *
+ * Conventions for every call:
+ *  - Pointers named "host" are host memory; all other data pointers are
+ *    device memory on the context's device.  The caller owns every buffer it
+ *    passes; the context owns the community state and its scratch.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    asynchronous on it unless stated otherwise.
+ *  - Arguments are checked on the host before anything is launched; a bad
+ *    argument returns CKV_ERR_INVALID_ARG and launches nothing.
+ *  - Errors found on the device (label out of range, community storage
+ *    exhausted) set the context's error word.  They surface at the next
+ *    ckv_last_error(), and every later call of that context then returns
+ *    the same error until ckv_init_communities() or ckv_import_state().
+ *  - No call aborts, traps or prints.
+ *  - A context is not thread-safe; use one context per host thread.
+ */
+#ifndef CKV_H
+#define CKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CKV_OK = 0,
+    CKV_ERR_INVALID_ARG = 1,  /* a pointer, size or configuration is out of range        */
+    CKV_ERR_CAPACITY = 2,     /* community member storage of a graph is exhausted        */
+    CKV_ERR_OOM = 3,          /* device or host allocation failed                        */
+    CKV_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, copy, sync)         */
+    CKV_ERR_TIMEOUT = 5,      /* a bounded device wait ran out                           */
+    CKV_ERR_STATE = 6         /* call out of order (e.g. step before init, wrong n)      */
+} ckv_status;
+
+typedef enum { CKV_F32 = 0, CKV_BF16 = 1 } ckv_dtype;
+
+/* Graph aggregation (abstract: "one graph per query head" versus
+ * "query-group graph aggregation").  PER_HEAD: one graph per (batch, query
+ * head).  QUERY_GROUP: one graph per (batch, KV head), shared by the query
+ * heads of its group; the group's scores and edge weights are sums over
+ * its heads. */
+typedef enum { CKV_PER_HEAD = 0, CKV_QUERY_GROUP = 1 } ckv_graph_mode;
+
+typedef struct {
+    int batch;            /* B >= 1                                                   */
+    int n_q_heads;        /* H_q >= 1                                                 */
+    int n_kv_heads;       /* H_kv >= 1, H_q % H_kv == 0; QUERY_GROUP: H_q/H_kv in {1,2,4,8} */
+    int head_dim;         /* D; must be 128                                           */
+    int n_max;            /* rows of the caller's K/V caches per (batch, KV head)     */
+    int max_communities;  /* most communities a graph may have (>= 1)                 */
+    int n_sinks;          /* S >= 0: positions [0, S) are always attended            */
+    int kappa;            /* edges per new token, 1..32 (the pages default to 8)      */
+    int budget;           /* token budget T_b >= 1 for the retrieved communities     */
+    int slack;            /* spare member slots given to each community at init      */
+    ckv_dtype kv_dtype;   /* element type of q, K and V                                */
+    ckv_graph_mode mode;
+    int device;           /* CUDA device ordinal of every device pointer              */
+    int pool_capacity;    /* member slots per graph; 0 = automatic, enough for any
+                             sequence of steps up to n_max: 5*n_max +
+                             max_communities*(slack+32).  A smaller value bounds
+                             memory; running out is reported as CKV_ERR_CAPACITY.  */
+} ckv_config;
+
+typedef struct ckv_ctx ckv_ctx;   /* opaque; owns all community state and scratch */
+
+/* Number of graphs G of a configuration: B*H_kv (QUERY_GROUP) or B*H_q
+ * (PER_HEAD).  Returns -1 for an invalid mode. */
+int ckv_graph_count(const ckv_config* cfg);
+
+/* Allocate a context and all its device state for cfg (synchronous).
+ * Errors: CKV_ERR_INVALID_ARG (cfg out of range), CKV_ERR_OOM, CKV_ERR_CUDA. */
+ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out);
+
+/* Free a context (synchronises its device first).  NULL is ignored. */
+void ckv_destroy(ckv_ctx* ctx);
+
+/* Prefill graph construction -- Figure 1, step (1): for each head and each
+ * causal query row i of Q, z_ij = q_i.k_j / sqrt(D) for j <= i; the row's
+ * edges are its top-kappa keys j in [S, i-1] (sinks and self excluded) by
+ * (z desc, j asc), weighted by the softmax probability over j in [0, i].
+ * Q, K: [n_heads][n][D] bf16 (dtype must be CKV_BF16, D = 128), device.
+ * Outputs (caller-allocated, device):
+ *   row_ptr [n_heads][n+1] int64: offsets of row i within its head's edges,
+ *           row i holding min(kappa, max(0, i - S)) edges (closed form);
+ *   col     [n_heads][E] int32 and w [n_heads][E] float, E = row_ptr[h][n],
+ *           each row's edges in rank order.
+ * The n x n score matrix is never stored.  Stateless, asynchronous.
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_CUDA. */
+ckv_status ckv_build_graph(int n_heads, int n, int head_dim, int n_sinks, int kappa,
+                           ckv_dtype dtype, const void* Q, const void* K,
+                           int64_t* row_ptr, int32_t* col, float* w, void* stream);
+
+/* Initial partition -- Figure 1, step (2): community c of graph g holds the
+ * positions j in [S, n) with labels[g][j] == c (ascending); its centroid is
+ * the mean of those keys (float, summed in double).  labels: int32
+ * [G][n] (graph-major), host (labels_on_device = 0) or device memory.
+ * K: the caller's key cache [B][H_kv][n_max][D] with rows [0, n) filled.
+ * Resets the context: previous state, pending steps and errors are dropped.
+ * Synchronous (returns after the device work has finished).
+ * Errors: CKV_ERR_INVALID_ARG (a label outside [0, n_communities), n, or
+ * n_communities out of range), CKV_ERR_CAPACITY, CKV_ERR_OOM, CKV_ERR_CUDA. */
+ckv_status ckv_init_communities(ckv_ctx* ctx, const int32_t* labels, int labels_on_device,
+                                int n_communities, const void* K, int n, void* stream);
+
+/* Decode step, first half -- Figure 1, step (3): for every graph, score the
+ * query against every community centroid (QUERY_GROUP: summed over the
+ * group's heads), keep communities in (score desc, id asc) order while their
+ * sizes fit the budget (at least one), and run exact softmax attention of
+ * each query head over the sinks, the kept members and the new token.
+ * q: [B][H_q][D] (kv_dtype); K, V: caches [B][H_kv][n_max][D] whose row
+ * n-1 already holds the new token; n: cache length including the new token;
+ * it must be one more than after the previous step (or init).
+ * out: [B][H_q][D] float32, device.  Asynchronous.
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no init, wrong n, or the
+ * previous step's ckv_assign_update missing), sticky device errors. */
+ckv_status ckv_decode_step(ckv_ctx* ctx, const void* q, const void* K, const void* V, int n,
+                           float* out, void* stream);
+
+/* Decode step, second half -- Figure 1, step (3) end and Table 1's O(d)
+ * update: for every graph, rank the kept members by their attention weight
+ * (summed over the graph's heads) and record the top kappa as the new
+ * token's edges; assign the token to the community with the largest summed
+ * edge weight (ties to the lower id) and update that centroid's running
+ * mean mu + (k - mu) / (m + 1).  K and n as in the preceding
+ * ckv_decode_step.  Asynchronous.
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no preceding decode step),
+ * sticky device errors; community storage exhaustion is reported by the
+ * next ckv_last_error() as CKV_ERR_CAPACITY and leaves that graph's state
+ * as it was before the step. */
+ckv_status ckv_assign_update(ckv_ctx* ctx, const void* K, int n, void* stream);
+
+/* One whole decode step from host memory: copies the new token's key and
+ * value (k_new_host, v_new_host: [B][H_kv][D]) into row n-1 of the device
+ * caches K and V, copies q_host ([B][H_q][D]) to the device, runs
+ * ckv_decode_step and ckv_assign_update, copies the output to out_host
+ * ([B][H_q][D] float32) and synchronises the stream.  Host buffers should
+ * be page-locked for the copies to be asynchronous.
+ * Errors: as the two calls above, plus CKV_ERR_CUDA. */
+ckv_status ckv_decode_host(ckv_ctx* ctx, const void* q_host, const void* k_new_host,
+                           const void* v_new_host, void* K, void* V, int n, float* out_host,
+                           void* stream);
+
+/* Synchronise the context's device work and return its error word
+ * (CKV_OK if none). */
+ckv_status ckv_last_error(ckv_ctx* ctx);
+
+/* Read back the last completed step's decisions into host buffers (any may
+ * be NULL).  n_sel [G]; sel [G][max_communities] (kept community ids of
+ * each graph, ascending id); n_tok_sel [G] (member tokens kept); n_edges
+ * [G]; edges [G][kappa] (token ids, rank order); edge_w [G][kappa];
+ * assigned [G].  Synchronous. */
+ckv_status ckv_get_step_debug(ckv_ctx* ctx, int32_t* n_sel, int32_t* sel, int32_t* n_tok_sel,
+                              int32_t* n_edges, int32_t* edges, float* edge_w, int32_t* assigned);
+
+/* Per-kernel device time of the decode steps, in the spirit of the pages'
+ * Table 10 split of a step into retrieval and attention.  After
+ * ckv_profile_begin, every ckv_decode_step / ckv_assign_update records CUDA
+ * events on its stream around each of its kernels; ckv_profile_end
+ * synchronises, writes the summed milliseconds of the four kernels
+ * (ms[0] centroid scoring, ms[1] community selection, ms[2] gather +
+ * attention, ms[3] edges + assignment + update) and the number of steps
+ * they cover, and stops recording.  Both are host calls; begin is not
+ * allowed while a step is half done.  Errors: CKV_ERR_INVALID_ARG,
+ * CKV_ERR_STATE, CKV_ERR_CUDA. */
+ckv_status ckv_profile_begin(ckv_ctx* ctx);
+ckv_status ckv_profile_end(ckv_ctx* ctx, float* ms /* [4] */, int* steps);
+
+/* Checkpoint of the community state in a layout-free host format:
+ *   int32 header[9] = {0x31564B43 ("CKV1"), 1, G, n_communities, D, n_tok,
+ *                      S, kappa, n_init}
+ *   float   centroids [G][n_communities][D]
+ *   int32   sizes     [G][n_communities]
+ *   int32   members   [G][n_tok - S]  (community by community, ascending)
+ *   int32   deg       [G][n_tok - n_init]          decode-time edges of
+ *   int32   col       [G][n_tok - n_init][kappa]   positions n_init .. n_tok-1
+ *   float   w         [G][n_tok - n_init][kappa]
+ * n_tok = positions covered (sinks + assigned tokens).  Export: pass
+ * host_buf = NULL to get the size in *bytes; otherwise *bytes is the
+ * buffer's capacity on entry and the bytes written on return.  Import
+ * validates the record against the context and replaces the state.
+ * Both are synchronous.  Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no
+ * state yet), CKV_ERR_OOM, CKV_ERR_CUDA. */
+ckv_status ckv_export_state(ckv_ctx* ctx, void* host_buf, size_t* bytes);
+ckv_status ckv_import_state(ckv_ctx* ctx, const void* host_buf, size_t bytes);
+
+/* Auxiliary storage of the context (centroids, community index, member
+ * pool, decode-time edges; scratch excluded) and, for comparison, the bytes
+ * of the K and V caches it serves. */
+ckv_status ckv_aux_bytes(const ckv_ctx* ctx, size_t* aux_bytes, size_t* kv_bytes);
+
+/* Static description of a status code. */
+const char* ckv_status_string(ckv_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,211 @@
+"""Python binding of libckv: CommunityKV community-retrieval sparse decode
+attention for B200 (sm_100a).
+
+Argument marshalling only: every function below calls the C entry point of
+the same name in libckv.so (declared in include/ckv.h), passing device
+pointers of torch tensors and the raw CUDA stream.  No step of the method
+runs in Python.  If the compiled library is missing, the first call raises
+``RuntimeError`` -- there is no fallback.
+
+Method: "CommunityKV: Efficient Long-Context Decoding via Graph
+Partitioning" (Figure 1: graph construction, initial partitioning,
+incremental update).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libckv.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "ckv.h")
+
+CKV_OK, CKV_ERR_INVALID_ARG, CKV_ERR_CAPACITY, CKV_ERR_OOM = 0, 1, 2, 3
+CKV_ERR_CUDA, CKV_ERR_TIMEOUT, CKV_ERR_STATE = 4, 5, 6
+CKV_F32, CKV_BF16 = 0, 1
+CKV_PER_HEAD, CKV_QUERY_GROUP = 0, 1
+
+
+class ckv_config(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int) for name in (
+        "batch", "n_q_heads", "n_kv_heads", "head_dim", "n_max", "max_communities",
+        "n_sinks", "kappa", "budget", "slack", "kv_dtype", "mode", "device", "pool_capacity")]
+
+
+class CkvError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        self.status = status
+        super().__init__(f"{call} failed: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def declared_functions():
+    """Names of every function declared in include/ckv.h."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ckv_[a-z_0-9]+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libckv.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_int
+    sz = ctypes.c_size_t
+    L.ckv_graph_count.restype = I
+    L.ckv_graph_count.argtypes = [ctypes.POINTER(ckv_config)]
+    L.ckv_create.restype = st
+    L.ckv_create.argtypes = [ctypes.POINTER(ckv_config), ctypes.POINTER(P)]
+    L.ckv_destroy.restype = None
+    L.ckv_destroy.argtypes = [P]
+    L.ckv_build_graph.restype = st
+    L.ckv_build_graph.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P]
+    L.ckv_init_communities.restype = st
+    L.ckv_init_communities.argtypes = [P, P, I, I, P, I, P]
+    L.ckv_decode_step.restype = st
+    L.ckv_decode_step.argtypes = [P, P, P, P, I, P, P]
+    L.ckv_assign_update.restype = st
+    L.ckv_assign_update.argtypes = [P, P, I, P]
+    L.ckv_decode_host.restype = st
+    L.ckv_decode_host.argtypes = [P, P, P, P, P, P, I, P, P]
+    L.ckv_last_error.restype = st
+    L.ckv_last_error.argtypes = [P]
+    L.ckv_get_step_debug.restype = st
+    L.ckv_get_step_debug.argtypes = [P, P, P, P, P, P, P, P]
+    L.ckv_profile_begin.restype = st
+    L.ckv_profile_begin.argtypes = [P]
+    L.ckv_profile_end.restype = st
+    L.ckv_profile_end.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
+    L.ckv_export_state.restype = st
+    L.ckv_export_state.argtypes = [P, P, ctypes.POINTER(sz)]
+    L.ckv_import_state.restype = st
+    L.ckv_import_state.argtypes = [P, P, sz]
+    L.ckv_aux_bytes.restype = st
+    L.ckv_aux_bytes.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.ckv_status_string.restype = ctypes.c_char_p
+    L.ckv_status_string.argtypes = [I]
+    _lib = L
+    return L
+
+
+def _ptr(x) -> int | None:
+    """Device/host address of a torch tensor, numpy array, int or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if hasattr(x, "ctypes"):
+        return x.ctypes.data
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(call: str, status: int):
+    if status != CKV_OK:
+        raise CkvError(call, status)
+
+
+# ------------------------------------------------------------ entry points
+def status_string(status: int) -> str:
+    return lib().ckv_status_string(status).decode()
+
+
+def ckv_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def ckv_graph_count(cfg: ckv_config) -> int:
+    return lib().ckv_graph_count(ctypes.byref(cfg))
+
+
+def ckv_create(cfg: ckv_config) -> int:
+    h = ctypes.c_void_p()
+    _check("ckv_create", lib().ckv_create(ctypes.byref(cfg), ctypes.byref(h)))
+    return h.value
+
+
+def ckv_destroy(ctx: int) -> None:
+    lib().ckv_destroy(ctx)
+
+
+def ckv_build_graph(n_heads, n, head_dim, n_sinks, kappa, dtype, Q, K, row_ptr, col, w, stream=None):
+    _check("ckv_build_graph", lib().ckv_build_graph(
+        n_heads, n, head_dim, n_sinks, kappa, dtype, _ptr(Q), _ptr(K), _ptr(row_ptr), _ptr(col),
+        _ptr(w), _stream(stream)))
+
+
+def ckv_init_communities(ctx, labels, labels_on_device, n_communities, K, n, stream=None):
+    _check("ckv_init_communities", lib().ckv_init_communities(
+        ctx, _ptr(labels), int(labels_on_device), n_communities, _ptr(K), n, _stream(stream)))
+
+
+def ckv_decode_step(ctx, q, K, V, n, out, stream=None):
+    _check("ckv_decode_step", lib().ckv_decode_step(ctx, _ptr(q), _ptr(K), _ptr(V), n, _ptr(out),
+                                                    _stream(stream)))
+
+
+def ckv_assign_update(ctx, K, n, stream=None):
+    _check("ckv_assign_update", lib().ckv_assign_update(ctx, _ptr(K), n, _stream(stream)))
+
+
+def ckv_decode_host(ctx, q_host, k_new_host, v_new_host, K, V, n, out_host, stream=None):
+    _check("ckv_decode_host", lib().ckv_decode_host(
+        ctx, _ptr(q_host), _ptr(k_new_host), _ptr(v_new_host), _ptr(K), _ptr(V), n, _ptr(out_host),
+        _stream(stream)))
+
+
+def ckv_last_error(ctx) -> int:
+    return lib().ckv_last_error(ctx)
+
+
+def ckv_get_step_debug(ctx, n_sel=None, sel=None, n_tok_sel=None, n_edges=None, edges=None,
+                       edge_w=None, assigned=None):
+    _check("ckv_get_step_debug", lib().ckv_get_step_debug(
+        ctx, _ptr(n_sel), _ptr(sel), _ptr(n_tok_sel), _ptr(n_edges), _ptr(edges), _ptr(edge_w),
+        _ptr(assigned)))
+
+
+def ckv_profile_begin(ctx) -> None:
+    _check("ckv_profile_begin", lib().ckv_profile_begin(ctx))
+
+
+def ckv_profile_end(ctx):
+    """Summed device milliseconds of (score, select, attend, assign) and the
+    number of profiled steps."""
+    ms = (ctypes.c_float * 4)()
+    steps = ctypes.c_int(0)
+    _check("ckv_profile_end", lib().ckv_profile_end(ctx, ms, ctypes.byref(steps)))
+    return list(ms), steps.value
+
+
+def ckv_export_state(ctx) -> bytes:
+    n = ctypes.c_size_t(0)
+    _check("ckv_export_state", lib().ckv_export_state(ctx, None, ctypes.byref(n)))
+    buf = ctypes.create_string_buffer(n.value)
+    _check("ckv_export_state", lib().ckv_export_state(ctx, buf, ctypes.byref(n)))
+    return buf.raw[:n.value]
+
+
+def ckv_import_state(ctx, blob: bytes) -> None:
+    _check("ckv_import_state", lib().ckv_import_state(ctx, blob, len(blob)))
+
+
+def ckv_aux_bytes(ctx):
+    a, k = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("ckv_aux_bytes", lib().ckv_aux_bytes(ctx, ctypes.byref(a), ctypes.byref(k)))
+    return a.value, k.value

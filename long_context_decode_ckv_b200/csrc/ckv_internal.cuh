@@ -1,0 +1,98 @@
+// ckv_internal.cuh -- context layout and kernel launchers of libckv.
+//
+// Device memory of one context (G graphs, Nc = max_communities, D = 128,
+// NM = n_max rows, HG = query heads per graph):
+//   mu        float [G][Nc][D]     centroids (Figure 1, step (2): one per community)
+//   csize     int32 [G][Nc]        members per community
+//   coff,ccap int32 [G][Nc]        segment of the community in the member pool
+//   pool      int32 [G][P]         member positions, ascending within a segment
+//   pool_top  int32 [G]            first free pool slot (segments move up when full)
+//   tok_comm  int32 [G][NM]        community of each position (-1: sink / none)
+//   edges     int32/float [G][NM-n_init][kappa] + deg  decode-time token graph rows
+// Per-step scratch (reused every step):
+//   score     float [G][Nc]        centroid scores
+//   sel       int32 [G][Nc]        kept communities (ascending id), sel_pre prefix of sizes
+//   meta      int32 [G][META]      C, T, rows, ... of the step
+//   part      float [G][splits][HG][D+2]   split-K partial (m, l, o) per head
+//   zrow      float [G][NM][HG]    logits of the kept members (for the edges)
+//   rtok,rcomm int32 [G][NM]       token / community of each kept member row
+//   ml        float [G][HG][2]     final softmax max and sum per head
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ckv.h"
+
+namespace ckv {
+
+constexpr int kD = 128;          // head_dim the kernels are written for
+constexpr int kMaxKappa = 32;
+constexpr int kSelBins = 2048;   // bucket count of the selection passes
+constexpr int kSortCap = 1024;   // candidates sorted exactly in one CTA
+
+// meta slots per graph
+enum { M_C = 0, M_T = 1, M_ROWS = 2, M_NEDGE = 3, M_ASSIGNED = 4, M_COUNT = 8 };
+
+struct DevState {
+    float* mu;
+    int32_t* csize;
+    int32_t* coff;
+    int32_t* ccap;
+    int32_t* pool;
+    int32_t* pool_top;
+    int32_t* tok_comm;
+    int32_t* edge_col;
+    float* edge_w;
+    int32_t* edge_deg;
+    // scratch
+    float* score;
+    int32_t* sel;
+    int32_t* sel_pre;
+    int8_t* cstat;           // [G][Nc] selection status of each community
+    int32_t* meta;
+    unsigned int* counter;   // [G] arrivals of the attention kernel's CTAs
+    float* part;
+    float* zrow;
+    int32_t* rtok;
+    int32_t* rcomm;
+    float* ml;
+    int32_t* dbg_edges;      // [G][kappa]
+    float* dbg_w;            // [G][kappa]
+    int* err;                // sticky device error word (ckv_status)
+};
+
+struct Dims {
+    int B, Hq, Hkv, Gq, G, HG, Nc, NM, S, kappa, budget, mode, bf16;
+    int64_t P;               // pool capacity per graph
+    int splits;              // CTAs per graph of the attention kernel
+    int n_comm;              // communities in use (set at init)
+    int n_init;              // first decode position (edge store row 0)
+};
+
+// kernel launchers (k_decode.cu)
+cudaError_t launch_score(const DevState& s, const Dims& d, const void* q, cudaStream_t st);
+cudaError_t launch_select(const DevState& s, const Dims& d, int n, cudaStream_t st);
+cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const void* K,
+                          const void* V, int n, float* out, cudaStream_t st);
+cudaError_t launch_assign(const DevState& s, const Dims& d, const void* K, int n,
+                          cudaStream_t st);
+size_t select_smem_bytes();
+
+// init kernels (k_init.cu)
+cudaError_t launch_init_count(const DevState& s, const Dims& d, const int32_t* labels, int n,
+                              cudaStream_t st);
+cudaError_t launch_init_layout(const DevState& s, const Dims& d, int slack, cudaStream_t st);
+cudaError_t launch_init_fill(const DevState& s, const Dims& d, const int32_t* labels, int n,
+                             cudaStream_t st);
+cudaError_t launch_init_centroids(const DevState& s, const Dims& d, const void* K,
+                                  cudaStream_t st);
+
+// prefill (k_prefill.cu)
+cudaError_t launch_build_graph(int H, int n, int S, int kappa, const void* Q, const void* K,
+                               int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st);
+
+// device error word: first error wins
+__device__ __forceinline__ void set_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+}  // namespace ckv

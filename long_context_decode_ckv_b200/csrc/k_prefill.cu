@@ -1,0 +1,397 @@
+// k_prefill.cu -- prefill top-kappa token graph on the sm_100a tensor cores.
+//
+// "CommunityKV: Efficient Long-Context Decoding via Graph Partitioning",
+// Figure 1 caption, step (1) Graph Construction: during prefill each query
+// is connected to its top-kappa keys of the attention matrix, sink tokens
+// excluded from the pool; Table 10 times this "fused top-kappa selection"
+// inside prefill.  Here: for each head and causal row i, z_ij = q_i.k_j /
+// sqrt(D) over j <= i; edges = top-kappa of j in [S, i-1] by (z desc, j asc)
+// with weight softmax_j(z)_ij over [0, i].  The n x n matrix never leaves
+// the SM: a 128 x 128 tile of Q K^T lives in tensor memory only.
+//
+// One CTA per (head, 128-row query block), heaviest (longest causal row
+// range) blocks first.  Warp roles:
+//   warp 0      TMA producer: Q block once, then K tiles through a 4-stage
+//               ring (128-byte swizzled, the layout tcgen05 reads).
+//   warp 1      allocates 256 TMEM columns (two 128 x 128 fp32
+//               accumulators) and issues tcgen05.mma (kind::f16, bf16 in,
+//               fp32 accumulate, M = N = 128, K = 16 x 8) from one thread.
+//   warps 2..5  epilogue: thread = one query row (its TMEM lane); reads the
+//               row's 128 scores with tcgen05.ld, keeps the online softmax
+//               (max, sum of exp2) and a sorted register top-KM list.
+// Every mbarrier wait is bounded; a wait that runs out marks row_ptr[h][0]
+// = -1 (an impossible offset), every role leaves its loop, and the TMEM is
+// freed before the CTA exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include "ckv_internal.cuh"
+
+namespace ckv {
+
+namespace {
+
+constexpr int kBM = 128, kBN = 128;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kHalfBytes = kBM * 64 * 2;            // one 64-column half of a 128-row tile
+constexpr int kTileBytes = 2 * kHalfBytes;           // 32 KB
+constexpr unsigned kWaitLimit = 1u << 22;
+constexpr float kLog2eOverSqrtD = 0.12751743082459868f;   // log2(e) / sqrt(128)
+
+struct __align__(1024) PrefillSmem {
+    unsigned char q[kTileBytes];
+    unsigned char k[kStages][kTileBytes];
+    unsigned long long bar_q;
+    unsigned long long bar_kfull[kStages];
+    unsigned long long bar_kempty[kStages];
+    unsigned long long bar_afull[2];
+    unsigned long long bar_aempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* b, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* b, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* b)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+// bounded wait for the phase with the given parity to complete
+__device__ __forceinline__ bool mbar_wait(unsigned long long* b, unsigned parity, volatile int* abort)
+{
+    const uint32_t a = smem_u32(b);
+    for (unsigned it = 0; it < kWaitLimit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((it & 1023) == 1023 && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, unsigned long long* bar,
+                                            int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+          "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// UMMA shared-memory descriptor of a K-major, 128-byte-swizzled bf16 tile:
+// rows 128 B apart, 8-row groups 1024 B apart (SBO), version 1 (sm_100).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);          // start address
+    d |= (uint64_t)(16 >> 4) << 16;                   // leading byte offset (unused for SW128 K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset
+    d |= (uint64_t)1 << 46;                           // descriptor version
+    d |= (uint64_t)2 << 61;                           // layout: SWIZZLE_128B
+    return d;
+}
+
+// instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(unsigned long long* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// edges before row i: rows S+1 .. S+kappa have 1 .. kappa edges, later rows kappa
+__device__ __forceinline__ int64_t row_offset(int64_t i, int S, int kappa)
+{
+    const int64_t a = max((int64_t)0, min(i, (int64_t)S + kappa + 1) - S - 1);
+    return a * (a + 1) / 2 + max((int64_t)0, i - (S + kappa + 1)) * kappa;
+}
+
+template <int KM>
+__global__ void __launch_bounds__(kThreads, 1)
+k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int H, int n,
+               int S, int kappa, int64_t* __restrict__ row_ptr, int32_t* __restrict__ col,
+               float* __restrict__ w)
+{
+    extern __shared__ unsigned char smem_raw[];
+    PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nqb = (n + kBM - 1) / kBM;
+    const int qb = nqb - 1 - (int)(blockIdx.x / H);    // heaviest blocks first
+    const int h = (int)(blockIdx.x % H);
+    const int i0 = qb * kBM;
+    const int ntiles = qb + 1;
+    const int64_t E = row_offset(n, S, kappa);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_q, 1);
+        for (int s = 0; s < kStages; ++s) { mbar_init(&sm.bar_kfull[s], 1); mbar_init(&sm.bar_kempty[s], 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&sm.bar_afull[b], 1); mbar_init(&sm.bar_aempty[b], 4); }
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;"
+                     ::"r"(smem_u32(&sm.tmem_base)) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int* abort = &sm.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_expect_tx(&sm.bar_q, kTileBytes);
+            tma_load_3d(sm.q, &tmQ, &sm.bar_q, 0, i0, h);
+            tma_load_3d(sm.q + kHalfBytes, &tmQ, &sm.bar_q, 64, i0, h);
+            int issued = 0;
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % kStages;
+                if (!mbar_wait(&sm.bar_kempty[s], ((t / kStages) & 1) ^ 1, abort)) break;
+                mbar_expect_tx(&sm.bar_kfull[s], kTileBytes);
+                tma_load_3d(sm.k[s], &tmK, &sm.bar_kfull[s], 0, t * kBN, h);
+                tma_load_3d(sm.k[s] + kHalfBytes, &tmK, &sm.bar_kfull[s], 64, t * kBN, h);
+                issued = t + 1;
+            }
+            // do not leave with copies in flight: the last load of every stage has landed
+            for (int t = max(0, issued - kStages); t < issued; ++t)
+                mbar_wait(&sm.bar_kfull[t % kStages], (t / kStages) & 1, abort);
+            mbar_wait(&sm.bar_q, 0, abort);
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------- MMA
+        if (lane == 0) {
+            int committed = 0;
+            if (mbar_wait(&sm.bar_q, 0, abort)) {
+                const uint32_t qa = smem_u32(sm.q);
+                for (int t = 0; t < ntiles; ++t) {
+                    const int s = t % kStages, b = t & 1;
+                    if (!mbar_wait(&sm.bar_kfull[s], (t / kStages) & 1, abort)) break;
+                    if (!mbar_wait(&sm.bar_aempty[b], ((t >> 1) & 1) ^ 1, abort)) break;
+                    tc_fence_after();
+                    const uint32_t ka = smem_u32(sm.k[s]);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t off = c * kHalfBytes + k * 32;
+                            umma_bf16(tmem + b * kBN, umma_desc(qa + off), umma_desc(ka + off), (c | k) != 0);
+                        }
+                    umma_commit(&sm.bar_kempty[s]);
+                    umma_commit(&sm.bar_afull[b]);
+                    committed = t + 1;
+                }
+            }
+            // the tensor core has finished every issued tile before TMEM is freed
+            if (committed > 0) {
+                const int t = committed - 1;
+                mbar_wait(&sm.bar_afull[t & 1], (t >> 1) & 1, abort);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int quarter = warp & 3;                 // TMEM lanes this warp may read
+        const int r = quarter * 32 + lane;
+        const int i = i0 + r;
+        const bool row_ok = i < n;
+        float m2 = -INFINITY, l = 0.f;                // running max of z*log2e and sum of 2^(.)
+        float vals[KM];
+        int idx[KM];
+#pragma unroll
+        for (int k = 0; k < KM; ++k) { vals[k] = -INFINITY; idx[k] = -1; }
+        for (int t = 0; t < ntiles; ++t) {
+            const int b = t & 1;
+            if (!mbar_wait(&sm.bar_afull[b], (t >> 1) & 1, abort)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int ch = 0; ch < kBN / 32; ++ch) {
+                float v[32];
+                __syncwarp();   // tcgen05.ld is warp-collective
+                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + b * kBN + ch * 32, v);
+                const int j0 = t * kBN + ch * 32;
+                // causal mask (only the diagonal tile reaches past i)
+                float mc = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    if (j0 + k > i) v[k] = -INFINITY;
+                    mc = fmaxf(mc, v[k]);
+                }
+                if (!row_ok) continue;
+                const float mcs = mc * kLog2eOverSqrtD;
+                if (mcs > m2) {
+                    l *= ex2(m2 - mcs);
+                    m2 = mcs;
+                }
+                float ps = 0.f;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) ps += ex2(fmaf(v[k], kLog2eOverSqrtD, -m2));
+                l += ps;
+                // top-KM candidates j in [S, i-1], ranked by the raw score
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int j = j0 + k;
+                    const float a = v[k];
+                    if (a > vals[KM - 1] && j >= S && j < i) {
+#pragma unroll
+                        for (int p = KM - 1; p > 0; --p) {
+                            const float up = vals[p - 1];
+                            const int upi = idx[p - 1];
+                            const bool shift = up < a;
+                            const bool land = !shift && vals[p] < a;
+                            vals[p] = shift ? up : (land ? a : vals[p]);
+                            idx[p] = shift ? upi : (land ? j : idx[p]);
+                        }
+                        if (vals[0] < a) { vals[0] = a; idx[0] = j; }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.bar_aempty[b]);
+        }
+        if (row_ok && !*abort) {
+            const int64_t base = (int64_t)h * E + row_offset(i, S, kappa);
+            const int deg = (int)min((int64_t)kappa, max((int64_t)0, (int64_t)i - S));
+            const float inv_l = 1.f / l;
+#pragma unroll
+            for (int k = 0; k < KM; ++k) {
+                if (k < deg) {
+                    col[base + k] = idx[k];
+                    w[base + k] = ex2(fmaf(vals[k], kLog2eOverSqrtD, -m2)) * inv_l;
+                }
+            }
+            row_ptr[(int64_t)h * (n + 1) + i] = row_offset(i, S, kappa);
+            if (i == n - 1) row_ptr[(int64_t)h * (n + 1) + n] = E;
+        }
+    }
+    __syncthreads();
+    if (*abort && threadIdx.x == 0) row_ptr[(int64_t)h * (n + 1)] = -1;
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [H][n][128] bf16 viewed as a 3-D tensor, box = 64 columns x 128 rows x 1 head
+bool make_map(CUtensorMap* m, const void* base, int H, int n)
+{
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)n, (cuuint64_t)H};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)n * 128 * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KM>
+cudaError_t launch_km(const CUtensorMap& mq, const CUtensorMap& mk, int H, int n, int S, int kappa,
+                      int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st)
+{
+    const size_t smem = sizeof(PrefillSmem) + 1024;
+    auto kern = k_prefill_topk<KM>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int nqb = (n + kBM - 1) / kBM;
+    kern<<<H * nqb, kThreads, smem, st>>>(mq, mk, H, n, S, kappa, row_ptr, col, w);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_build_graph(int H, int n, int S, int kappa, const void* Q, const void* K, int64_t* row_ptr,
+                               int32_t* col, float* w, cudaStream_t st)
+{
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K)) & 15) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk;
+    if (!make_map(&mq, Q, H, n) || !make_map(&mk, K, H, n)) return cudaErrorInvalidValue;
+    if (kappa <= 8) return launch_km<8>(mq, mk, H, n, S, kappa, row_ptr, col, w, st);
+    if (kappa <= 16) return launch_km<16>(mq, mk, H, n, S, kappa, row_ptr, col, w, st);
+    return launch_km<32>(mq, mk, H, n, S, kappa, row_ptr, col, w, st);
+}
+
+}  // namespace ckv

@@ -212,18 +212,34 @@ class Workload:
     labels: np.ndarray   # [n_graphs][n0] int32
 
 
-def make_workload(cfg: DecodeConfig) -> Workload:
-    """Whole workload on the host (all slabs)."""
+def _slab_job(args):
+    cfg, b, kvh = args
+    s = make_slab(cfg, b, kvh)
+    return b, kvh, s.K, s.V, s.labels, make_queries(cfg, s, b, kvh)
+
+
+def make_workload(cfg: DecodeConfig, workers: int = 1) -> Workload:
+    """Whole workload on the host (all slabs).  workers > 1 draws the slabs
+    in a pool of spawned processes (same bytes as workers = 1)."""
     dt = np.uint16 if cfg.bf16 else np.float32
     K = np.empty((cfg.batch, cfg.n_kv_heads, cfg.n_max, cfg.head_dim), dt)
     V = np.empty_like(K)
     q = np.empty((cfg.steps, cfg.batch, cfg.n_q_heads, cfg.head_dim), dt)
     lab_kv = np.empty((cfg.batch, cfg.n_kv_heads, cfg.n0), np.int32)
-    for b in range(cfg.batch):
-        for kvh in range(cfg.n_kv_heads):
-            s = make_slab(cfg, b, kvh)
-            K[b, kvh], V[b, kvh], lab_kv[b, kvh] = s.K, s.V, s.labels
-            q[:, b, kvh * cfg.group:(kvh + 1) * cfg.group] = make_queries(cfg, s, b, kvh)
+    jobs = [(cfg, b, kvh) for b in range(cfg.batch) for kvh in range(cfg.n_kv_heads)]
+    if workers > 1 and len(jobs) > 1:
+        import multiprocessing as mp
+        from concurrent.futures import ProcessPoolExecutor
+        with ProcessPoolExecutor(min(workers, len(jobs)), mp_context=mp.get_context("spawn")) as ex:
+            results = ex.map(_slab_job, jobs)
+            for b, kvh, sk, sv, sl, sq in results:
+                K[b, kvh], V[b, kvh], lab_kv[b, kvh] = sk, sv, sl
+                q[:, b, kvh * cfg.group:(kvh + 1) * cfg.group] = sq
+    else:
+        for job in jobs:
+            b, kvh, sk, sv, sl, sq = _slab_job(job)
+            K[b, kvh], V[b, kvh], lab_kv[b, kvh] = sk, sv, sl
+            q[:, b, kvh * cfg.group:(kvh + 1) * cfg.group] = sq
     labels = np.empty((cfg.n_graphs, cfg.n0), np.int32)
     for g in range(cfg.n_graphs):
         b, kvh, _ = cfg.graph_heads(g)

@@ -1,0 +1,191 @@
+"""Lockstep parity checker: the CUDA library against the CPU oracle, step by
+step, on the same seeded workload.
+
+Per decode step and tracked graph it compares (rules of the north-star
+contract, readings listed in the design doc):
+
+* attention output: max |o_gpu - o_ref| / max |o_ref| <= 2e-3 per (batch, head);
+* kept communities, edge set and assigned community: bit-exact, except where
+  the oracle's float gap at the cutoff is below 1e-5 relative (a near-tie
+  where either choice is correct).  Such an exempt divergence is logged and
+  the GPU state is re-synchronised from the oracle's state;
+* edge weights: relative 2e-5 (float logits against the double oracle);
+* community state (centroids bit-exact, sizes, ascending members, edge rows)
+  through the library's checkpoint record.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+import oracle
+import long_context_decode_ckv_b200 as ckv
+from long_context_decode_ckv_b200 import state as ckv_state
+from long_context_decode_ckv_b200 import synth
+
+OUT_RTOL = 2e-3
+GAP_EXEMPT = 1e-5
+W_RTOL = 2e-5
+
+
+@dataclass
+class StepLog:
+    step: int
+    exempt: list = field(default_factory=list)      # (graph, what, gap)
+    max_out_err: float = 0.0
+
+
+def _torch_view(a, dev):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if a.dtype == np.uint16:
+        t = t.view(torch.bfloat16)
+    return t.to(dev)
+
+
+def config_for(cfg: synth.DecodeConfig, device: int = 0, slack: int = 16,
+               pool_capacity: int = 0) -> ckv.ckv_config:
+    c = ckv.ckv_config()
+    c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    c.n_max, c.max_communities, c.n_sinks = cfg.n_max, cfg.n_comm, cfg.n_sinks
+    c.kappa, c.budget, c.slack = cfg.kappa, cfg.budget, slack
+    c.kv_dtype = ckv.CKV_BF16 if cfg.bf16 else ckv.CKV_F32
+    c.mode = ckv.CKV_QUERY_GROUP if cfg.mode == synth.QUERY_GROUP else ckv.CKV_PER_HEAD
+    c.device = device
+    c.pool_capacity = pool_capacity
+    return c
+
+
+class Lockstep:
+    def __init__(self, wl: synth.Workload, tracked=None, device: int = 0, slack: int = 16):
+        import torch
+        self.wl, self.cfg = wl, wl.cfg
+        cfg = self.cfg
+        self.dev = torch.device("cuda", device)
+        self.K = _torch_view(wl.K, self.dev)
+        self.V = _torch_view(wl.V, self.dev)
+        self.q = _torch_view(wl.q, self.dev)
+        self.out = torch.empty((cfg.batch, cfg.n_q_heads, cfg.head_dim), dtype=torch.float32,
+                               device=self.dev)
+        self.ctx = ckv.ckv_create(config_for(cfg, device, slack))
+        ckv.ckv_init_communities(self.ctx, wl.labels, 0, cfg.n_comm, self.K, cfg.n0)
+        self.tracked = list(range(cfg.n_graphs)) if tracked is None else list(tracked)
+        self.og = {}
+        for g in self.tracked:
+            b, kvh, _ = cfg.graph_heads(g)
+            o = oracle.Graph(cfg.n_comm, cfg.head_dim, cfg.n_max)
+            o.init(cfg.n0, cfg.n_sinks, wl.labels[g], wl.K[b, kvh])
+            self.og[g] = o
+        self.oracle_edges = {g: [] for g in self.tracked}   # per decode row: (col, w)
+        self.n = cfg.n0
+        self.logs: list[StepLog] = []
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            ckv.ckv_destroy(self.ctx)
+            self.ctx = None
+
+    # ---------------------------------------------------------------- step
+    def step(self, i: int) -> StepLog:
+        import torch
+        cfg = self.cfg
+        n = self.n + 1
+        ckv.ckv_decode_step(self.ctx, self.q[i], self.K, self.V, n, self.out)
+        ckv.ckv_assign_update(self.ctx, self.K, n)
+        st = ckv.ckv_last_error(self.ctx)
+        assert st == ckv.CKV_OK, ckv.status_string(st)
+        G, Nc, kap = cfg.n_graphs, cfg.n_comm, cfg.kappa
+        n_sel = np.zeros(G, np.int32)
+        sel = np.zeros((G, Nc), np.int32)
+        n_edges = np.zeros(G, np.int32)
+        edges = np.zeros((G, kap), np.int32)
+        edge_w = np.zeros((G, kap), np.float32)
+        assigned = np.zeros(G, np.int32)
+        n_tok_sel = np.zeros(G, np.int32)
+        ckv.ckv_get_step_debug(self.ctx, n_sel, sel, n_tok_sel, n_edges, edges, edge_w, assigned)
+        out = self.out.cpu().numpy()
+        log = StepLog(i)
+        resync = False
+        for g in self.tracked:
+            b, kvh, heads = cfg.graph_heads(g)
+            r = oracle.decode_step(self.og[g], np.ascontiguousarray(self.wl.q[i, b, heads]),
+                                   self.wl.K[b, kvh], self.wl.V[b, kvh], n, cfg.n_sinks, kap,
+                                   cfg.budget)
+            self.oracle_edges[g].append((r.edge_col.copy(), r.edge_w.copy()))
+            gsel = set(sel[g, :n_sel[g]].tolist())
+            if gsel != set(r.sel.tolist()):
+                gap = min(r.cut_gap_lo, r.cut_gap_hi)
+                assert gap < GAP_EXEMPT, (
+                    f"step {i} graph {g}: kept communities differ (gap {gap:.3g} not a near-tie): "
+                    f"gpu-only {sorted(gsel - set(r.sel.tolist()))[:8]} "
+                    f"oracle-only {sorted(set(r.sel.tolist()) - gsel)[:8]}")
+                log.exempt.append((g, "select", gap))
+                resync = True
+                continue
+            assert n_tok_sel[g] == r.T
+            for h_i, h in enumerate(heads):
+                ref = r.out[h_i]
+                err = float(np.max(np.abs(out[b, h] - ref)) / max(np.max(np.abs(ref)), 1e-30))
+                log.max_out_err = max(log.max_out_err, err)
+                assert err <= OUT_RTOL, f"step {i} graph {g} head {h}: out rel err {err:.3g}"
+            E = int(n_edges[g])
+            ge, gw = edges[g, :E], edge_w[g, :E]
+            assert E == len(r.edge_col), f"step {i} graph {g}: {E} edges vs {len(r.edge_col)}"
+            if set(ge.tolist()) != set(r.edge_col.tolist()):
+                assert r.edge_gap < GAP_EXEMPT, (
+                    f"step {i} graph {g}: edges differ (gap {r.edge_gap:.3g}): gpu {ge} oracle {r.edge_col}")
+                log.exempt.append((g, "edges", r.edge_gap))
+                resync = True
+                continue
+            # weights per token, and the GPU's own order is (w desc, token asc)
+            ref_w = dict(zip(r.edge_col.tolist(), r.edge_w.tolist()))
+            for tk, wv in zip(ge.tolist(), gw.tolist()):
+                assert abs(wv - ref_w[tk]) <= W_RTOL * abs(ref_w[tk]) + 1e-12, (
+                    f"step {i} graph {g}: edge {tk} w {wv} vs {ref_w[tk]}")
+            for a in range(E - 1):
+                assert (gw[a] > gw[a + 1]) or (gw[a] == gw[a + 1] and ge[a] < ge[a + 1])
+            if int(assigned[g]) != r.assigned:
+                assert r.vote_gap < GAP_EXEMPT, (
+                    f"step {i} graph {g}: assigned {assigned[g]} vs {r.assigned} (gap {r.vote_gap:.3g})")
+                log.exempt.append((g, "assign", r.vote_gap))
+                resync = True
+        self.n = n
+        if resync:
+            self.resync()
+        self.logs.append(log)
+        return log
+
+    # ----------------------------------------------------------- state
+    def oracle_state_into(self, s: ckv_state.State) -> ckv_state.State:
+        """Replace the tracked graphs' part of a checkpoint by the oracle's."""
+        for g in self.tracked:
+            o = self.og[g]
+            s.centroids[g] = o.centroids()
+            s.sizes[g] = o.sizes()
+            s.members[g] = o.members()
+            for r_i, (col, w) in enumerate(self.oracle_edges[g]):
+                s.deg[g, r_i] = len(col)
+                s.col[g, r_i, :len(col)] = col
+                s.w[g, r_i, :len(col)] = w
+        return s
+
+    def resync(self):
+        s = ckv_state.parse(ckv.ckv_export_state(self.ctx))
+        ckv.ckv_import_state(self.ctx, ckv_state.pack(self.oracle_state_into(s)))
+
+    def compare_state(self):
+        """GPU checkpoint against the oracle for every tracked graph."""
+        s = ckv_state.parse(ckv.ckv_export_state(self.ctx))
+        assert s.n_tok == self.n
+        for g in self.tracked:
+            o = self.og[g]
+            np.testing.assert_array_equal(s.sizes[g], o.sizes(), err_msg=f"graph {g} sizes")
+            np.testing.assert_array_equal(s.members[g], o.members(), err_msg=f"graph {g} members")
+            assert np.array_equal(s.centroids[g].view(np.uint32), o.centroids().view(np.uint32)), (
+                f"graph {g}: centroids not bit-exact "
+                f"(max diff {np.max(np.abs(s.centroids[g] - o.centroids()))})")
+            for r_i, (col, w) in enumerate(self.oracle_edges[g]):
+                assert s.deg[g, r_i] == len(col)
+                assert set(s.col[g, r_i, :len(col)].tolist()) == set(col.tolist())
+        return s

@@ -1,0 +1,110 @@
+"""The C-ABI library builds, loads without a GPU, exports every symbol that
+include/ckv.h declares, and rejects bad configurations on the host."""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+
+import long_context_decode_ckv_b200 as ckv
+from long_context_decode_ckv_b200 import build as ckv_build
+from long_context_decode_ckv_b200 import state as ckv_state
+
+
+@pytest.fixture(scope="module")
+def L():
+    ckv_build.build()
+    return ckv.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = ckv.declared_functions()
+    assert len(names) >= 14
+    raw = ctypes.CDLL(ckv.LIB_PATH)
+    for name in names:
+        assert hasattr(raw, name), f"libckv.so does not export {name}"
+
+
+def test_exports_nothing_undeclared(L):
+    out = os.popen(f"nm -D --defined-only {ckv.LIB_PATH}").read().split("\n")
+    ours = {ln.split()[-1] for ln in out if " T ckv_" in ln}
+    assert ours == set(ckv.declared_functions())
+
+
+def good_config():
+    c = ckv.ckv_config()
+    c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim = 4, 32, 8, 128
+    c.n_max, c.max_communities, c.n_sinks = 131200, 8192, 4
+    c.kappa, c.budget, c.slack = 8, 4096, 16
+    c.kv_dtype, c.mode, c.device, c.pool_capacity = ckv.CKV_BF16, ckv.CKV_QUERY_GROUP, 0, 0
+    return c
+
+
+def test_graph_count_and_status_strings(L):
+    c = good_config()
+    assert ckv.ckv_graph_count(c) == 32
+    c.mode = ckv.CKV_PER_HEAD
+    assert ckv.ckv_graph_count(c) == 128
+    c.mode = 7
+    assert ckv.ckv_graph_count(c) == -1
+    for s in range(7):
+        assert ckv.status_string(s) and ckv.status_string(s) != "unknown status"
+    assert ckv.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("field,value", [
+    ("batch", 0), ("n_q_heads", 0), ("n_kv_heads", 3), ("head_dim", 64), ("n_max", 0),
+    ("max_communities", 0), ("n_sinks", -1), ("n_sinks", 131200), ("kappa", 0), ("kappa", 33),
+    ("budget", 0), ("slack", -1), ("kv_dtype", 5), ("mode", 2), ("device", -1),
+    ("pool_capacity", -1),
+])
+def test_bad_config_rejected_on_host(L, field, value):
+    c = good_config()
+    setattr(c, field, value)
+    h = ctypes.c_void_p()
+    assert L.ckv_create(ctypes.byref(c), ctypes.byref(h)) == ckv.CKV_ERR_INVALID_ARG
+    assert h.value is None
+
+
+def test_group_size_must_be_supported(L):
+    c = good_config()
+    c.n_q_heads, c.n_kv_heads = 48, 8          # group of 6
+    h = ctypes.c_void_p()
+    assert L.ckv_create(ctypes.byref(c), ctypes.byref(h)) == ckv.CKV_ERR_INVALID_ARG
+
+
+def test_null_arguments_rejected(L):
+    assert L.ckv_create(None, None) == ckv.CKV_ERR_INVALID_ARG
+    assert L.ckv_decode_step(None, None, None, None, 1, None, None) == ckv.CKV_ERR_INVALID_ARG
+    assert L.ckv_assign_update(None, None, 1, None) == ckv.CKV_ERR_INVALID_ARG
+    assert L.ckv_last_error(None) == ckv.CKV_ERR_INVALID_ARG
+    assert L.ckv_import_state(None, None, 0) == ckv.CKV_ERR_INVALID_ARG
+    assert L.ckv_build_graph(8, 64, 128, 4, 8, ckv.CKV_BF16, None, None, None, None, None, None) \
+        == ckv.CKV_ERR_INVALID_ARG
+    # prefill takes bf16 only, head_dim 128, kappa 1..32
+    p = ctypes.c_void_p(16)
+    assert L.ckv_build_graph(8, 64, 128, 4, 8, ckv.CKV_F32, p, p, p, p, p, None) == ckv.CKV_ERR_INVALID_ARG
+    assert L.ckv_build_graph(8, 64, 64, 4, 8, ckv.CKV_BF16, p, p, p, p, p, None) == ckv.CKV_ERR_INVALID_ARG
+    assert L.ckv_build_graph(8, 64, 128, 4, 40, ckv.CKV_BF16, p, p, p, p, p, None) == ckv.CKV_ERR_INVALID_ARG
+    ckv.ckv_destroy(None)   # ignored
+
+
+def test_checkpoint_record_roundtrip():
+    rng = np.random.default_rng(0)
+    G, Nc, D, S, kap, n_init, n_tok = 3, 5, 128, 4, 8, 40, 43
+    sizes = np.zeros((G, Nc), np.int32)
+    for g in range(G):
+        sizes[g] = np.bincount(rng.integers(0, Nc, n_tok - S), minlength=Nc)
+    s = ckv_state.State(G, Nc, D, n_tok, S, kap, n_init,
+                        rng.standard_normal((G, Nc, D)).astype(np.float32), sizes,
+                        np.tile(np.arange(S, n_tok, dtype=np.int32), (G, 1)),
+                        rng.integers(0, kap + 1, (G, n_tok - n_init)).astype(np.int32),
+                        rng.integers(0, n_tok, (G, n_tok - n_init, kap)).astype(np.int32),
+                        rng.random((G, n_tok - n_init, kap)).astype(np.float32))
+    blob = ckv_state.pack(s)
+    assert len(blob) == 36 + 4 * (G * Nc * D + G * Nc + G * (n_tok - S) + G * (n_tok - n_init) * (1 + 2 * kap))
+    t = ckv_state.parse(blob)
+    for f in ("centroids", "sizes", "members", "deg", "col", "w"):
+        np.testing.assert_array_equal(getattr(t, f), getattr(s, f))
+    with pytest.raises(ValueError):
+        ckv_state.parse(b"\0" * 64)

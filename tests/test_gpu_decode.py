@@ -1,0 +1,225 @@
+"""GPU parity of the decode path (ckv_init_communities, ckv_decode_step,
+ckv_assign_update) against the CPU oracle, through the C ABI.
+
+"CommunityKV: Efficient Long-Context Decoding via Graph Partitioning",
+Figure 1 caption steps (2)-(3).  The comparison rules are in lockstep.py.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import long_context_decode_ckv_b200 as ckv
+from long_context_decode_ckv_b200 import build as ckv_build
+from long_context_decode_ckv_b200 import state as ckv_state
+from long_context_decode_ckv_b200 import synth
+from tests.conftest import gpu_available
+from tests.lockstep import Lockstep, config_for, _torch_view
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]
+
+WORKERS = min(8, os.cpu_count() or 1)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    ckv_build.build()
+
+
+def run_lockstep(cfg, tracked=None, steps=None, compare_every=1, slack=16):
+    wl = synth.make_workload(cfg, workers=WORKERS)
+    ls = Lockstep(wl, tracked=tracked, slack=slack)
+    try:
+        ls.compare_state()
+        steps = cfg.steps if steps is None else steps
+        for i in range(steps):
+            ls.step(i)
+            if compare_every and (i + 1) % compare_every == 0:
+                ls.compare_state()
+        ls.compare_state()
+    finally:
+        ls.close()
+    n_ex = sum(len(l.exempt) for l in ls.logs)
+    print(f"{cfg.name}: {steps} steps, max out err "
+          f"{max(l.max_out_err for l in ls.logs):.3g}, exempt near-ties {n_ex}")
+    return ls
+
+
+def test_tiny_fp32_all_steps():
+    run_lockstep(synth.TINY)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(n0=1000, n_clusters=25, budget=200),          # ragged tiles, uneven clusters
+    dict(budget=8),                                     # no community fits: forced C = 1
+    dict(budget=10 ** 6),                               # every community kept: dense attention
+    dict(kappa=1), dict(kappa=32), dict(n_sinks=0), dict(n_sinks=17),
+    dict(n0=5, n_clusters=1, steps=6, comm_size=16),    # one community, a few members
+])
+def test_tiny_edge_cases(kw):
+    cfg = synth.scaled(synth.TINY, **kw)
+    run_lockstep(cfg)
+
+
+def test_small_slack_relocates_segments():
+    # slack 0: every append past the initial size moves the community segment
+    cfg = synth.scaled(synth.TINY, n0=512, n_clusters=2, steps=40)
+    run_lockstep(cfg, slack=0)
+
+
+@pytest.mark.parametrize("mode", [synth.PER_HEAD, synth.QUERY_GROUP])
+def test_small_gqa_both_modes(mode):
+    cfg = synth.scaled(synth.LLAMA, batch=2, n_q_heads=8, n_kv_heads=2, n0=4000, n_clusters=125,
+                       budget=300, steps=12, mode=mode)
+    run_lockstep(cfg)
+
+
+def test_llama_per_head_full():
+    run_lockstep(synth.LLAMA, compare_every=16)
+
+
+def test_qwen8b_query_group_full_size_sampled():
+    # full size, all 128 steps on the GPU; the oracle follows 4 of the 32 graphs
+    run_lockstep(synth.QWEN8B, tracked=[0, 9, 22, 31], compare_every=0)
+
+
+@pytest.mark.parametrize("n,budget", [(8192, 128), (8192, 4096), (32768, 512), (131072, 1024)])
+def test_sweep_points_sampled(n, budget):
+    cfg = synth.sweep_config(n, budget, steps=8)
+    run_lockstep(cfg, tracked=[0, 37, 127], compare_every=0)
+
+
+# ----------------------------------------------------------------- boundary
+def _small_ctx(slack=16, pool_capacity=0, cfg=None):
+    import torch
+    cfg = cfg or synth.scaled(synth.TINY, n0=256, n_clusters=8, steps=4)
+    wl = synth.make_workload(cfg)
+    dev = torch.device("cuda", 0)
+    K, V, q = _torch_view(wl.K, dev), _torch_view(wl.V, dev), _torch_view(wl.q, dev)
+    ctx = ckv.ckv_create(config_for(cfg, 0, slack, pool_capacity))
+    out = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
+    return cfg, wl, ctx, K, V, q, out
+
+
+def test_call_order_and_arguments_checked():
+    cfg, wl, ctx, K, V, q, out = _small_ctx()
+    try:
+        with pytest.raises(ckv.CkvError) as e:          # step before init
+            ckv.ckv_decode_step(ctx, q[0], K, V, cfg.n0 + 1, out)
+        assert e.value.status == ckv.CKV_ERR_STATE
+        bad = wl.labels.copy()
+        bad[0, 100] = cfg.n_comm                        # label out of range
+        with pytest.raises(ckv.CkvError) as e:
+            ckv.ckv_init_communities(ctx, bad, 0, cfg.n_comm, K, cfg.n0)
+        assert e.value.status == ckv.CKV_ERR_INVALID_ARG
+        ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        with pytest.raises(ckv.CkvError) as e:          # wrong n
+            ckv.ckv_decode_step(ctx, q[0], K, V, cfg.n0 + 2, out)
+        assert e.value.status == ckv.CKV_ERR_STATE
+        with pytest.raises(ckv.CkvError) as e:          # update without a step
+            ckv.ckv_assign_update(ctx, K, cfg.n0 + 1)
+        assert e.value.status == ckv.CKV_ERR_STATE
+        ckv.ckv_decode_step(ctx, q[0], K, V, cfg.n0 + 1, out)
+        with pytest.raises(ckv.CkvError) as e:          # second step before the update
+            ckv.ckv_decode_step(ctx, q[1], K, V, cfg.n0 + 2, out)
+        assert e.value.status == ckv.CKV_ERR_STATE
+        ckv.ckv_assign_update(ctx, K, cfg.n0 + 1)
+        assert ckv.ckv_last_error(ctx) == ckv.CKV_OK
+        with pytest.raises(ckv.CkvError):               # corrupt checkpoint
+            blob = bytearray(ckv.ckv_export_state(ctx))
+            blob[36 + 4 * cfg.n_comm * 128] = 0xFF      # first size -> negative
+            blob[36 + 4 * cfg.n_comm * 128 + 3] = 0xFF
+            ckv.ckv_import_state(ctx, bytes(blob))
+    finally:
+        ckv.ckv_destroy(ctx)
+
+
+def test_capacity_error_is_sticky_and_state_unchanged():
+    cfg = synth.scaled(synth.TINY, n0=256, n_clusters=1, steps=20)
+    # pool just large enough for the initial segments: the first relocation fails
+    cfg_, wl, ctx, K, V, q, out = _small_ctx(slack=0, pool_capacity=256, cfg=cfg)
+    try:
+        ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        before = ckv_state.parse(ckv.ckv_export_state(ctx))
+        ckv.ckv_decode_step(ctx, q[0], K, V, cfg.n0 + 1, out)
+        ckv.ckv_assign_update(ctx, K, cfg.n0 + 1)
+        assert ckv.ckv_last_error(ctx) == ckv.CKV_ERR_CAPACITY
+        with pytest.raises(ckv.CkvError) as e:          # sticky
+            ckv.ckv_decode_step(ctx, q[1], K, V, cfg.n0 + 2, out)
+        assert e.value.status == ckv.CKV_ERR_CAPACITY
+        ckv.ckv_import_state(ctx, ckv_state.pack(before))   # import clears it
+        assert ckv.ckv_last_error(ctx) == ckv.CKV_OK
+        after = ckv_state.parse(ckv.ckv_export_state(ctx))
+        np.testing.assert_array_equal(after.sizes, before.sizes)
+        np.testing.assert_array_equal(after.centroids, before.centroids)
+    finally:
+        ckv.ckv_destroy(ctx)
+
+
+def test_deterministic_and_checkpoint_roundtrip():
+    import torch
+    cfg = synth.scaled(synth.LLAMA, batch=1, n_q_heads=8, n_kv_heads=2, n0=3000, n_clusters=150,
+                       budget=256, steps=6, mode=synth.QUERY_GROUP)
+    wl = synth.make_workload(cfg)
+    dev = torch.device("cuda", 0)
+    K, V, q = _torch_view(wl.K, dev), _torch_view(wl.V, dev), _torch_view(wl.q, dev)
+    outs, blobs = [], []
+    for rep in range(2):
+        ctx = ckv.ckv_create(config_for(cfg))
+        o = torch.empty((1, 8, 128), dtype=torch.float32, device=dev)
+        ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        got = []
+        mid = None
+        for i in range(cfg.steps):
+            if i == 3:
+                mid = ckv.ckv_export_state(ctx)
+            ckv.ckv_decode_step(ctx, q[i], K, V, cfg.n0 + i + 1, o)
+            ckv.ckv_assign_update(ctx, K, cfg.n0 + i + 1)
+            got.append(o.cpu().numpy().copy())
+        blobs.append(ckv.ckv_export_state(ctx))
+        outs.append(np.stack(got))
+        # resume from the mid-run checkpoint and replay the last steps
+        ckv.ckv_import_state(ctx, mid)
+        for i in range(3, cfg.steps):
+            ckv.ckv_decode_step(ctx, q[i], K, V, cfg.n0 + i + 1, o)
+            ckv.ckv_assign_update(ctx, K, cfg.n0 + i + 1)
+            assert np.array_equal(o.cpu().numpy(), got[i])
+        assert ckv.ckv_export_state(ctx) == blobs[-1]
+        ckv.ckv_destroy(ctx)
+    assert np.array_equal(outs[0], outs[1])
+    assert blobs[0] == blobs[1]
+
+
+def test_host_buffer_step_matches_device_step():
+    import torch
+    cfg = synth.scaled(synth.LLAMA, batch=2, n_q_heads=8, n_kv_heads=2, n0=2000, n_clusters=100,
+                       budget=256, steps=5, mode=synth.QUERY_GROUP)
+    wl = synth.make_workload(cfg)
+    dev = torch.device("cuda", 0)
+    K, V, q = _torch_view(wl.K, dev), _torch_view(wl.V, dev), _torch_view(wl.q, dev)
+    K2 = K.clone()
+    V2 = V.clone()
+    K2[:, :, cfg.n0:] = 0                                   # the host path writes these rows
+    V2[:, :, cfg.n0:] = 0
+    a = ckv.ckv_create(config_for(cfg))
+    b = ckv.ckv_create(config_for(cfg))
+    try:
+        ckv.ckv_init_communities(a, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        ckv.ckv_init_communities(b, wl.labels, 0, cfg.n_comm, K2, cfg.n0)
+        o = torch.empty((2, 8, 128), dtype=torch.float32, device=dev)
+        oh = torch.empty((2, 8, 128), dtype=torch.float32).pin_memory()
+        for i in range(cfg.steps):
+            n = cfg.n0 + i + 1
+            ckv.ckv_decode_step(a, q[i], K, V, n, o)
+            ckv.ckv_assign_update(a, K, n)
+            qh = torch.from_numpy(wl.q[i].copy()).pin_memory()
+            kh = torch.from_numpy(np.ascontiguousarray(wl.K[:, :, n - 1])).pin_memory()
+            vh = torch.from_numpy(np.ascontiguousarray(wl.V[:, :, n - 1])).pin_memory()
+            ckv.ckv_decode_host(b, qh, kh, vh, K2, V2, n, oh)
+            assert np.array_equal(oh.numpy(), o.cpu().numpy())
+        assert torch.equal(K2, K) and torch.equal(V2, V)
+        assert ckv.ckv_export_state(a) == ckv.ckv_export_state(b)
+    finally:
+        ckv.ckv_destroy(a)
+        ckv.ckv_destroy(b)
