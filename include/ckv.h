@@ -201,6 +201,31 @@ ckv_status ckv_profile_end(ckv_ctx* ctx, float* ms /* [4] */, int* steps);
 ckv_status ckv_export_state(ckv_ctx* ctx, void* host_buf, size_t* bytes);
 ckv_status ckv_import_state(ckv_ctx* ctx, const void* host_buf, size_t bytes);
 
+/* Exact softmax attention with sinks over caller-chosen rows, without any
+ * device allocation.  The paper has no counterpart: this entry point exists
+ * for hosts that cannot call cudaMalloc where the attention runs (for
+ * example an inference engine's custom-op execute path that forbids device
+ * allocation after set-up and gives the op no workspace), so it needs no
+ * context.  For every graph g of cfg (only batch, heads, head_dim, n_max,
+ * n_sinks, kv_dtype, mode and device are read), each of the graph's query
+ * heads attends over the sinks [0, S), the positions rows_host[g][0 ..
+ * n_rows_host[g]) and the new token n-1 -- the attention of ckv_decode_step
+ * with the kept rows given instead of selected.  q, K, V, out as in
+ * ckv_decode_step (device); rows_host [G][max_rows] and n_rows_host [G] are
+ * host memory, each row in [S, n-1).
+ * Scratch: a 16 MiB file-scope device array that every GPU loading the
+ * library keeps until exit; a call needs about max_rows * (4 + 4 * heads
+ * per graph) bytes plus its split partials, so max_rows up to about 800,000
+ * for a group of 4 heads; a larger max_rows returns CKV_ERR_CAPACITY.
+ * Every call shares the array, so calls that overlap on the GPU race;
+ * serialise them.  The first call on a device looks up the array's device
+ * address; make it before any stream capture.  Asynchronous on `stream`.
+ * Errors: CKV_ERR_INVALID_ARG (bad pointer, size or row), CKV_ERR_CAPACITY,
+ * CKV_ERR_CUDA. */
+ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, const void* K, const void* V,
+                                  int n, const int32_t* rows_host, const int32_t* n_rows_host,
+                                  int max_rows, float* out, void* stream);
+
 /* Auxiliary storage of the context (centroids, community index, member
  * pool, decode-time edges; scratch excluded) and, for comparison, the bytes
  * of the K and V caches it serves. */

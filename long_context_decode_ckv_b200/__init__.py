@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
     L.ckv_import_state.argtypes = [P, P, sz]
     L.ckv_aux_bytes.restype = st
     L.ckv_aux_bytes.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.ckv_attend_rows_static.restype = st
+    L.ckv_attend_rows_static.argtypes = [ctypes.POINTER(ckv_config), P, P, P, I, P, P, I, P, P]
     L.ckv_status_string.restype = ctypes.c_char_p
     L.ckv_status_string.argtypes = [I]
     _lib = L
@@ -203,6 +205,15 @@ def ckv_export_state(ctx) -> bytes:
 
 def ckv_import_state(ctx, blob: bytes) -> None:
     _check("ckv_import_state", lib().ckv_import_state(ctx, blob, len(blob)))
+
+
+def ckv_attend_rows_static(cfg, q, K, V, n, rows_host, n_rows_host, max_rows, out, stream=None):
+    """Attention over caller-chosen rows with no device allocation (scratch
+    in the library's static device array); rows_host / n_rows_host are host
+    arrays."""
+    _check("ckv_attend_rows_static", lib().ckv_attend_rows_static(
+        ctypes.byref(cfg), _ptr(q), _ptr(K), _ptr(V), n, _ptr(rows_host), _ptr(n_rows_host), max_rows,
+        _ptr(out), _stream(stream)))
 
 
 def ckv_aux_bytes(ctx):
