@@ -188,6 +188,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--cpu-steps", type=int, default=8)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -244,27 +245,44 @@ def main():
     stream = torch.cuda.current_stream(dev)
     sel_tok = np.zeros(cfg.n_graphs, np.int32)
 
-    def step(s):
+    def step(s, st):
         r = reps[s % L]
         i = r["i"]
         n = cfg.n0 + i + 1
-        ckv.ckv_decode_step(r["ctx"], q[i], r["K"], r["V"], n, out, stream)
-        ckv.ckv_assign_update(r["ctx"], r["K"], n, stream)
+        ckv.ckv_decode_step(r["ctx"], q[i], r["K"], r["V"], n, out, st)
+        ckv.ckv_assign_update(r["ctx"], r["K"], n, st)
         r["i"] = i + 1
 
     for s in range(args.warmup):
-        step(s)
+        step(s, stream)
     torch.cuda.synchronize(dev)
     for r in reps:
         ckv.ckv_profile_begin(r["ctx"])
+    # The timed steps are captured once into a CUDA graph (the launches of a
+    # real decoder are), then replayed once: the device time is the steps'.
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+                cap = torch.cuda.current_stream(dev)
+                for s in range(args.warmup, args.warmup + args.steps):
+                    step(s, cap)
+        except Exception as exc:   # capture refused: time the same steps eagerly
+            print(f"CUDA graph capture failed ({exc}); timing eager launches", file=sys.stderr)
+            graph = None
+    launch_mode = "cuda-graph" if graph is not None else "eager"
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
     with Clocks(local) as clk:
         start.record(stream)
-        for s in range(args.warmup, args.warmup + args.steps):
-            step(s)
+        if graph is not None:
+            graph.replay()
+        else:
+            for s in range(args.warmup, args.warmup + args.steps):
+                step(s, stream)
         end.record(stream)
         torch.cuda.synchronize(dev)
     if pg:
@@ -272,7 +290,12 @@ def main():
     ms = start.elapsed_time(end)
     kern_ms, kern_steps = [0.0] * 4, 0
     for r in reps:
-        m, k = ckv.ckv_profile_end(r["ctx"])
+        try:
+            m, k = ckv.ckv_profile_end(r["ctx"])
+        except ckv.CkvError as exc:
+            print(f"per-kernel profile unavailable: {exc}", file=sys.stderr)
+            kern_ms, kern_steps = None, 0
+            break
         kern_ms = [a + b for a, b in zip(kern_ms, m)]
         kern_steps += k
     for r in reps:
@@ -318,6 +341,7 @@ def main():
                "h2d_bytes_per_step": cfg.batch * (cfg.n_q_heads + 2 * cfg.n_kv_heads) * 128 * eb,
                "d2h_bytes_per_step": cfg.batch * cfg.n_q_heads * 128 * 4}
 
+    del graph
     for r in reps:
         ckv.ckv_destroy(r["ctx"])
     if pg:
@@ -332,14 +356,16 @@ def main():
     gbs = step_bytes * args.steps / (ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     names = ["score", "select", "attend", "assign"]
-    avg = {nm: kern_ms[k] / max(1, kern_steps) for k, nm in enumerate(names)}
-    dom = max(("score", "attend"), key=lambda nm: avg[nm])
-    kb = kernel_bytes(cfg, T_mean)[dom] * cfg.n_graphs
-    achieved = kb / (avg[dom] / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": achieved, "peak": peak,
-                "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                "traffic": None, "algorithmic_bytes_per_launch": kb,
-                "avg_launch_ms": avg[dom]}
+    avg, roofline = None, None
+    if kern_ms is not None and kern_steps:
+        avg = {nm: kern_ms[k] / kern_steps for k, nm in enumerate(names)}
+        dom = max(("score", "attend"), key=lambda nm: avg[nm])
+        kb = kernel_bytes(cfg, T_mean)[dom] * cfg.n_graphs
+        achieved = kb / (avg[dom] / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": achieved, "peak": peak,
+                    "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                    "traffic": None, "algorithmic_bytes_per_launch": kb,
+                    "avg_launch_ms": avg[dom]}
 
     cpu = None
     if not args.no_cpu:
@@ -354,7 +380,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "graphs": cfg.n_graphs, "layer_replicas": L,
                    "l2": f"{L} layer replicas rotated (inputs larger than L2), no flush",
-                   "parallelism": "replicas" if world > 1 else "single"},
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "launch": launch_mode},
         "hbm_gbs": gbs, "hbm_frac_of_8000": gbs / NOMINAL_HBM_GBS, "hbm_frac_of_measured": gbs / peak,
         "algorithmic_bytes_per_step": step_bytes, "mean_tokens_kept": T_mean,
         "kernel_ms_per_step": avg,

@@ -65,7 +65,8 @@ typedef struct {
     int n_kv_heads;       /* H_kv >= 1, H_q % H_kv == 0; QUERY_GROUP: H_q/H_kv in {1,2,4,8} */
     int head_dim;         /* D; must be 128                                           */
     int n_max;            /* rows of the caller's K/V caches per (batch, KV head)     */
-    int max_communities;  /* most communities a graph may have (>= 1)                 */
+    int max_communities;  /* most communities a graph may have (1 .. 16384; the
+                             selection keeps one graph's scores in shared memory)    */
     int n_sinks;          /* S >= 0: positions [0, S) are always attended            */
     int kappa;            /* edges per new token, 1..32 (the pages default to 8)      */
     int budget;           /* token budget T_b >= 1 for the retrieved communities     */

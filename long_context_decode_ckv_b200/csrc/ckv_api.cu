@@ -77,7 +77,7 @@ bool valid_config(const ckv_config* c)
     if (c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1) return false;
     if (c->n_q_heads % c->n_kv_heads) return false;
     if (c->head_dim != ckv::kD) return false;
-    if (c->n_max < 1 || c->max_communities < 1) return false;
+    if (c->n_max < 1 || c->max_communities < 1 || c->max_communities > ckv::kMaxCommunities) return false;
     if (c->n_sinks < 0 || c->n_sinks >= c->n_max) return false;
     if (c->kappa < 1 || c->kappa > ckv::kMaxKappa) return false;
     if (c->budget < 1 || c->slack < 0 || c->slack > (1 << 20)) return false;
@@ -179,7 +179,9 @@ cudaError_t prof_mark(ckv_ctx* x, int slot, cudaStream_t st)
     cudaError_t r = next_event(x, &e);
     if (r != cudaSuccess) return r;
     x->ev_steps.back()[slot] = e;
-    return cudaEventRecord(e, st);
+    // external record: under stream capture it becomes an event-record node
+    // whose timestamps stay usable for cudaEventElapsedTime
+    return cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
 }
 
 }  // namespace
@@ -246,11 +248,10 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     // can never run out before n_max.
     d.P = cfg->pool_capacity > 0 ? (int64_t)cfg->pool_capacity
                                  : (int64_t)cfg->n_max * 5 + (int64_t)cfg->max_communities * (cfg->slack + 32);
-    // attention split: about 8 CTAs per SM in total, at least 32 rows each
-    const int rows_hint = d.S + cfg->budget + 1;
-    int splits = (sms * 8 + d.G - 1) / d.G;
-    splits = splits < (rows_hint + 31) / 32 ? splits : (rows_hint + 31) / 32;
-    d.splits = splits < 1 ? 1 : splits;
+    // the attention grid: as many CTAs as can be co-resident
+    d.nSM = sms;
+    d.nCTA = ckv::attend_grid(d, sms);
+    if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
     d.n_comm = 0;
     d.n_init = 0;
 
@@ -265,22 +266,22 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(pool, G * (size_t)d.P);
     ALLOC(pool_top, G);
     ALLOC(tok_comm, G * NM);
+    const size_t KC = d.nCTA, kap = d.kappa;
     ALLOC(score, G * Nc);
     ALLOC(sel, G * Nc);
-    ALLOC(sel_pre, G * (Nc + 1));
-    ALLOC(cstat, G * Nc);
     ALLOC(meta, G * ckv::M_COUNT);
-    ALLOC(counter, G);
-    ALLOC(part, G * (size_t)d.splits * HG * (ckv::kD + 2));
-    ALLOC(zrow, G * NM * HG);
     ALLOC(rtok, G * NM);
     ALLOC(rcomm, G * NM);
-    ALLOC(ml, G * HG * 2);
-    ALLOC(dbg_edges, G * (size_t)d.kappa);
-    ALLOC(dbg_w, G * (size_t)d.kappa);
+    ALLOC(zrow, G * NM * HG);
+    ALLOC(part_ml, G * KC * HG * 2);
+    ALLOC(part_o, G * KC * HG * ckv::kD);
+    ALLOC(bar, G * 2);
+    ALLOC(e_tok, G * kap);
+    ALLOC(e_w, G * kap);
+    ALLOC(e_comm, G * kap);
     ALLOC(err, 1);
 #undef ALLOC
-    if (e == cudaSuccess) e = cudaMemset(s.counter, 0, G * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemset(s.bar, 0, G * 2 * sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemset(s.err, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(s.meta, 0, G * ckv::M_COUNT * sizeof(int32_t));
     const size_t qb = (size_t)d.B * d.Hq * ckv::kD;
@@ -330,7 +331,7 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
     step(cudaMemsetAsync(s.coff, 0, G * d.Nc * sizeof(int32_t), st));
     step(cudaMemsetAsync(s.ccap, 0, G * d.Nc * sizeof(int32_t), st));
     step(cudaMemsetAsync(s.tok_comm, 0xff, G * d.NM * sizeof(int32_t), st));
-    step(cudaMemsetAsync(s.counter, 0, G * sizeof(unsigned), st));
+    step(cudaMemsetAsync(s.bar, 0, G * 2 * sizeof(unsigned), st));
     step(cudaMemsetAsync(s.mu, 0, G * d.Nc * ckv::kD * sizeof(float), st));
     step(ckv::launch_init_count(s, d, dlabels, n, st));
     int err = 0;
@@ -370,7 +371,7 @@ CKV_API ckv_status ckv_decode_step(ckv_ctx* x, const void* q, const void* K, con
     CKV_CUDA(prof_mark(x, 0, st));
     CKV_CUDA(ckv::launch_score(x->s, x->d, q, st));
     CKV_CUDA(prof_mark(x, 1, st));
-    CKV_CUDA(ckv::launch_select(x->s, x->d, n, st));
+    CKV_CUDA(ckv::launch_select(x->s, x->d, st));
     CKV_CUDA(prof_mark(x, 2, st));
     CKV_CUDA(ckv::launch_attend(x->s, x->d, q, K, V, n, out, st));
     CKV_CUDA(prof_mark(x, 3, st));
@@ -494,8 +495,8 @@ CKV_API ckv_status ckv_get_step_debug(ckv_ctx* x, int32_t* n_sel, int32_t* sel, 
         if (assigned) assigned[g] = m[ckv::M_ASSIGNED];
     }
     if (sel) CKV_CUDA(cudaMemcpy(sel, x->s.sel, (size_t)d.G * d.Nc * 4, cudaMemcpyDeviceToHost));
-    if (edges) CKV_CUDA(cudaMemcpy(edges, x->s.dbg_edges, (size_t)d.G * d.kappa * 4, cudaMemcpyDeviceToHost));
-    if (edge_w) CKV_CUDA(cudaMemcpy(edge_w, x->s.dbg_w, (size_t)d.G * d.kappa * 4, cudaMemcpyDeviceToHost));
+    if (edges) CKV_CUDA(cudaMemcpy(edges, x->s.e_tok, (size_t)d.G * d.kappa * 4, cudaMemcpyDeviceToHost));
+    if (edge_w) CKV_CUDA(cudaMemcpy(edge_w, x->s.e_w, (size_t)d.G * d.kappa * 4, cudaMemcpyDeviceToHost));
     return CKV_OK;
 }
 
@@ -652,7 +653,7 @@ CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t byt
         }
     }
     CKV_CUDA(cudaMemset(s.err, 0, sizeof(int)));
-    CKV_CUDA(cudaMemset(s.counter, 0, G * sizeof(unsigned)));
+    CKV_CUDA(cudaMemset(s.bar, 0, G * 2 * sizeof(unsigned)));
     CKV_CUDA(cudaDeviceSynchronize());
     d.n_comm = Nc;
     d.n_init = n_init;

@@ -9,14 +9,16 @@
 //   pool_top  int32 [G]            first free pool slot (segments move up when full)
 //   tok_comm  int32 [G][NM]        community of each position (-1: sink / none)
 //   edges     int32/float [G][NM-n_init][kappa] + deg  decode-time token graph rows
-// Per-step scratch (reused every step):
+// Per-step scratch (reused every step; KC = CTAs of the attention grid):
 //   score     float [G][Nc]        centroid scores
-//   sel       int32 [G][Nc]        kept communities (ascending id), sel_pre prefix of sizes
-//   meta      int32 [G][META]      C, T, rows, ... of the step
-//   part      float [G][splits][HG][D+2]   split-K partial (m, l, o) per head
-//   zrow      float [G][NM][HG]    logits of the kept members (for the edges)
+//   sel       int32 [G][Nc]        kept communities (ascending id)
+//   meta      int32 [G][META]      C, T, rows, edges, assigned of the step
 //   rtok,rcomm int32 [G][NM]       token / community of each kept member row
-//   ml        float [G][HG][2]     final softmax max and sum per head
+//   zrow      float [G][NM][HG]    logits of the kept members (for the edges)
+//   part_ml   float [G][KC][HG][2] per-CTA softmax max and sum per head
+//   part_o    float [G][KC][HG][D] per-CTA P.V per head, relative to its max
+//   bar       uint  [G][2]         arrivals of a graph's CTAs (slot 1)
+//   e_*       [G][kappa]           the step's edges (rank order) for the update
 #pragma once
 
 #include <cuda_runtime.h>
@@ -29,7 +31,7 @@ namespace ckv {
 constexpr int kD = 128;          // head_dim the kernels are written for
 constexpr int kMaxKappa = 32;
 constexpr int kSelBins = 2048;   // bucket count of the selection passes
-constexpr int kSortCap = 1024;   // candidates sorted exactly in one CTA
+constexpr int kSortCap = 1024;   // candidates ranked exactly in one CTA
 
 // meta slots per graph
 enum { M_C = 0, M_T = 1, M_ROWS = 2, M_NEDGE = 3, M_ASSIGNED = 4, M_COUNT = 8 };
@@ -48,36 +50,41 @@ struct DevState {
     // scratch
     float* score;
     int32_t* sel;
-    int32_t* sel_pre;
-    int8_t* cstat;           // [G][Nc] selection status of each community
     int32_t* meta;
-    unsigned int* counter;   // [G] arrivals of the attention kernel's CTAs
-    float* part;
-    float* zrow;
     int32_t* rtok;
     int32_t* rcomm;
-    float* ml;
-    int32_t* dbg_edges;      // [G][kappa]
-    float* dbg_w;            // [G][kappa]
+    float* zrow;
+    float* part_ml;
+    float* part_o;
+    unsigned int* bar;
+    int32_t* e_tok;
+    float* e_w;
+    int32_t* e_comm;
     int* err;                // sticky device error word (ckv_status)
 };
 
 struct Dims {
     int B, Hq, Hkv, Gq, G, HG, Nc, NM, S, kappa, budget, mode, bf16;
     int64_t P;               // pool capacity per graph
-    int splits;              // CTAs per graph of the attention kernel
+    int nCTA;                // CTAs of the (co-resident) attention grid
+    int nSM;                 // multiprocessors of the device
     int n_comm;              // communities in use (set at init)
     int n_init;              // first decode position (edge store row 0)
 };
 
 // kernel launchers (k_decode.cu)
 cudaError_t launch_score(const DevState& s, const Dims& d, const void* q, cudaStream_t st);
-cudaError_t launch_select(const DevState& s, const Dims& d, int n, cudaStream_t st);
+cudaError_t launch_select(const DevState& s, const Dims& d, cudaStream_t st);
 cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const void* K,
                           const void* V, int n, float* out, cudaStream_t st);
 cudaError_t launch_assign(const DevState& s, const Dims& d, const void* K, int n,
                           cudaStream_t st);
-size_t select_smem_bytes();
+size_t select_smem_bytes(int n_comm);
+// sets the kernels' shared-memory limits on the current device; then the
+// number of co-resident CTAs of the attention kernel (0 on error)
+cudaError_t prepare_kernels(const Dims& d);
+int attend_grid(const Dims& d, int sms);
+constexpr int kMaxCommunities = 16384;   // k_select keeps a graph's communities in shared memory
 
 // init kernels (k_init.cu)
 cudaError_t launch_init_count(const DevState& s, const Dims& d, const int32_t* labels, int n,

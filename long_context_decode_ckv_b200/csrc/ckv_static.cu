@@ -5,9 +5,10 @@
 // integrations (an inference engine's custom-op execute path, for example)
 // that forbid device allocation after set-up and hand the op no workspace.
 // For them ckv_attend_rows_static runs the library's gather-attention
-// kernel (the one ckv_decode_step uses) with its split-K scratch -- row
-// list, logits, per-split (m, l, o) partials, arrival counter -- in the
-// file-scope device array below instead of memory from a context.
+// kernel (the one ckv_decode_step uses) with its scratch -- row list,
+// logits, per-CTA softmax statistics and P.V partials, arrival counter,
+// edge ranking -- in the file-scope device array below instead of memory
+// from a context.
 //
 // The array is kStaticScratchBytes per device and stays resident on every
 // GPU that loads the library until the process exits.  Every call shares
@@ -98,32 +99,41 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     d.HG = HG;
     d.NM = cfg->n_max;
     d.S = cfg->n_sinks;
+    d.kappa = 1;          // the kernel also ranks one edge; this call discards it
     d.mode = CKV_QUERY_GROUP;
     d.bf16 = cfg->kv_dtype == CKV_BF16;
-    const int rows_hint = d.S + max_rows + 1;
-    d.splits = sms * 8 < (rows_hint + 31) / 32 ? sms * 8 : (rows_hint + 31) / 32;
-    if (d.splits < 1) d.splits = 1;
-    // scratch layout: meta | counter | err | ml | row list | logits | partials
+    const int grid = ckv::attend_grid(d, sms);
+    if (grid < 1) return CKV_ERR_CUDA;
+    // at most one CTA per 64 rows of the largest graph
+    const int64_t rows_max = (int64_t)d.S + max_rows + 1;
+    d.nCTA = (int)((rows_max + 63) / 64 < grid ? (rows_max + 63) / 64 : grid);
+    // scratch layout: meta | bar | err | edges | row list | logits | partials
+    const size_t KC = d.nCTA;
     size_t off = 0;
     const size_t o_meta = off;  off = align256(off + ckv::M_COUNT * 4);
-    const size_t o_cnt = off;   off = align256(off + 4);
+    const size_t o_bar = off;   off = align256(off + 2 * 4);
     const size_t o_err = off;   off = align256(off + 4);
-    const size_t o_ml = off;    off = align256(off + (size_t)HG * 2 * 4);
-    // (graph index 0 in every launch, so the row list and logits need
-    // max_rows entries, whatever the cache length)
+    const size_t o_e = off;     off = align256(off + 3 * 4);
+    // (graph index 0 in every launch: the row list holds max_rows entries and
+    // the spill logits rows_max rows, whatever the cache length)
     const size_t o_rtok = off;  off = align256(off + (size_t)max_rows * 4);
-    const size_t o_zrow = off;  off = align256(off + (size_t)max_rows * HG * 4);
-    const size_t o_part = off;  off = align256(off + (size_t)d.splits * HG * (kD + 2) * 4);
+    const size_t o_zrow = off;  off = align256(off + (size_t)rows_max * HG * 4);
+    const size_t o_pml = off;   off = align256(off + KC * HG * 2 * 4);
+    const size_t o_po = off;    off = align256(off + KC * HG * kD * 4);
     if (off > kStaticScratchBytes) return CKV_ERR_CAPACITY;   // max_rows too large for the array
     unsigned char* sb = static_cast<unsigned char*>(base);
     ckv::DevState s{};
     s.meta = reinterpret_cast<int32_t*>(sb + o_meta);
-    s.counter = reinterpret_cast<unsigned int*>(sb + o_cnt);
+    s.bar = reinterpret_cast<unsigned int*>(sb + o_bar);
     s.err = reinterpret_cast<int*>(sb + o_err);
-    s.ml = reinterpret_cast<float*>(sb + o_ml);
+    s.e_tok = reinterpret_cast<int32_t*>(sb + o_e);
+    s.e_w = reinterpret_cast<float*>(sb + o_e + 4);
+    s.e_comm = reinterpret_cast<int32_t*>(sb + o_e + 8);
     s.rtok = reinterpret_cast<int32_t*>(sb + o_rtok);
+    s.rcomm = s.rtok;     // community of a row: only read for the edges, which this call discards
     s.zrow = reinterpret_cast<float*>(sb + o_zrow);
-    s.part = reinterpret_cast<float*>(sb + o_part);
+    s.part_ml = reinterpret_cast<float*>(sb + o_pml);
+    s.part_o = reinterpret_cast<float*>(sb + o_po);
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t eb = d.bf16 ? 2 : 4;
@@ -142,7 +152,7 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
         e = cudaMemcpyAsync(s.meta, meta, sizeof meta, cudaMemcpyHostToDevice, st);
         if (e == cudaSuccess && T > 0)
             e = cudaMemcpyAsync(s.rtok, rows_host + (int64_t)g * max_rows, (size_t)T * 4, cudaMemcpyHostToDevice, st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(sb + o_cnt, 0, 256 + 256, st);   // counter and error word
+        if (e == cudaSuccess) e = cudaMemsetAsync(sb + o_bar, 0, 256 + 256, st);   // arrival counters, error word
         if (e == cudaSuccess) e = ckv::launch_attend(s, d, qg, Kg, Vg, n, og, st);
         if (e != cudaSuccess) return CKV_ERR_CUDA;
     }

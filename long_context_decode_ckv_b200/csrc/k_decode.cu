@@ -7,21 +7,21 @@
 // assign it to a community in constant time; Table 1: O(sqrt(n) d)
 // retrieval, O(d) update.
 //
-// Four kernels per step, all memory-bound:
-//   k_score   centroid GEMV, one warp per 32 communities, lane = 4 dims,
-//             32 partial dots reduced by a butterfly transpose (31 shuffles
-//             for 32 rows).
-//   k_select  one CTA per graph: exact budgeted top-C by bucket passes over
-//             the scores (a monotone linear bucketing, then radix windows of
-//             the order-preserving score bits, then of the id) and a final
-//             bitonic sort of <= 1024 candidates; writes the kept list, its
-//             size prefix and the kept member rows.
-//   k_attend  split-K gather attention: each CTA streams 32-row tiles of K
-//             and V (16-byte cp.async into an XOR-swizzled shared layout,
-//             double-buffered), all query heads of a graph share one gather;
-//             the last CTA of a graph merges the (m, l, o) partials.
-//   k_assign  one CTA per graph: edge weights from the logits, top-kappa,
-//             weighted-plurality vote, running-mean update, member append.
+// Four kernels per step:
+//   k_score   centroid GEMV (HBM-bound), one warp per 32 communities, lane =
+//             4 dims, the 32 partial dots reduced by a butterfly transpose.
+//   k_select  one CTA per graph, the graph's scores and sizes held in shared
+//             memory: exact budgeted top-C by bucket passes (a monotone
+//             linear bucketing, then radix windows of the order-preserving
+//             score bits, then of the id) and an exact rank of the last
+//             <= 1024 candidates; writes the kept list and the kept rows.
+//   k_attend  one CTA per SM, each a slice of one graph's rows; every warp
+//             streams its own run of rows (K and V together, 16-byte
+//             cp.async) with an online softmax; the last CTA of a graph
+//             merges the (m, l, o) partials exactly and ranks the kept
+//             members' edge weights from the logits spilled to L2.
+//   k_assign  one CTA per graph: vote, capacity check, running-mean
+//             update, member append, edge row.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -29,16 +29,15 @@
 #include <type_traits>
 
 #include "ckv_internal.cuh"
+#include "dev_async.cuh"
 
 namespace ckv {
 
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kTile = 32;          // rows per attention tile
-constexpr int kAttThreads = 256;
 constexpr int kSelThreads = 1024;
-constexpr int kAsgThreads = 256;
+constexpr int kAsgThreads = 128;
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -70,65 +69,121 @@ __device__ __forceinline__ uint32_t ord_u(float f)
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// (w desc, token asc) order of edge candidates
+__device__ __forceinline__ bool cand_better(float w, int t, float w2, int t2)
+{
+    return w > w2 || (w == w2 && t < t2);
+}
+
 // ---------------------------------------------------------------- k_score
+// Work unit = 32 consecutive communities of one graph (16 KB of centroids,
+// one bulk copy).  Each CTA owns a contiguous run of units in graph-major
+// order; its producer lane streams them through a ring, consumer warp c
+// takes local units c, c + 8, ...: lane = 4 dims, 32 partial dots reduced
+// by a butterfly transpose so lane r ends with row r's score.
+constexpr int kScoreCW = 8;
+constexpr int kScoreThreads = 32 * (1 + kScoreCW);
+constexpr int kScoreNST = 8;
+constexpr int kScoreStage = 32 * kD * 4;
+
+struct ScoreSmem {
+    unsigned char ring[kScoreNST][kScoreStage];
+    unsigned long long full[kScoreNST];
+    unsigned long long empty[kScoreNST];
+    int abort;
+};
+
 template <bool BF16>
-__global__ void __launch_bounds__(256) k_score(DevState s, Dims d, const void* __restrict__ q)
+__global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, const void* __restrict__ q)
 {
     if (*(volatile int*)s.err) return;
-    const int g = blockIdx.y;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int c0 = blockIdx.x * 256 + warp * 32;
-    if (c0 >= d.n_comm) return;
-    int b, h0, kvh;
-    graph_heads(d, g, b, h0, kvh);
-    const int hg = d.HG;
-    // Sum of the graph's query heads, 4 dims per lane (a group's score is
-    // the sum of its heads' scores).
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int upg = (d.n_comm + 31) / 32;                    // units per graph
+    const int64_t NU = (int64_t)d.G * upg;
+    const int64_t u0 = (int64_t)blockIdx.x * NU / gridDim.x, u1 = (int64_t)(blockIdx.x + 1) * NU / gridDim.x;
+    const int nu = (int)(u1 - u0);
+    if (tid == 0) {
+        for (int i = 0; i < kScoreNST; ++i) { mbar_init(&sm.full[i], 1); mbar_init(&sm.empty[i], 1); }
+        sm.abort = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    volatile int* abort_flag = &sm.abort;
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int u = 0; u < nu; ++u) {
+                const int st = u % kScoreNST;
+                if (!mbar_wait(&sm.empty[st], ((u / kScoreNST) & 1) ^ 1, abort_flag)) break;
+                const int64_t gu = u0 + u;
+                const int g = (int)(gu / upg), c0 = (int)(gu % upg) * 32;
+                const int rows = min(32, d.n_comm - c0);
+                mbar_expect_tx(&sm.full[st], rows * kD * 4);
+                bulk_g2s(sm.ring[st], s.mu + ((int64_t)g * d.Nc + c0) * kD, rows * kD * 4, &sm.full[st]);
+                issued = u + 1;
+            }
+            // nothing may still be landing when the CTA exits
+            for (int u = max(0, issued - kScoreNST); u < issued; ++u)
+                mbar_wait(&sm.full[u % kScoreNST], (u / kScoreNST) & 1, abort_flag);
+        }
+        return;
+    }
+    const int c = warp - 1;
+    int gq = -1;
     float qs[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int h = 0; h < hg; ++h) {
-        const int64_t base = ((int64_t)b * d.Hq + h0 + h) * kD + 4 * lane;
+    for (int u = c; u < nu; u += kScoreCW) {
+        const int64_t gu = u0 + u;
+        const int g = (int)(gu / upg), c0 = (int)(gu % upg) * 32;
+        if (g != gq) {   // sum of the graph's query heads, this lane's 4 dims
+            int b, h0, kvh;
+            graph_heads(d, g, b, h0, kvh);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) qs[k] += elem<BF16>(q, base + k);
-    }
-    const float4* mu = reinterpret_cast<const float4*>(s.mu + (int64_t)g * d.Nc * kD);
-    float part[32];
+            for (int k = 0; k < 4; ++k) qs[k] = 0.f;
+            for (int h = 0; h < d.HG; ++h) {
+                const int64_t base = ((int64_t)b * d.Hq + h0 + h) * kD + 4 * lane;
 #pragma unroll
-    for (int rb = 0; rb < 32; rb += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int c = c0 + rb + r;
-            v[r] = (c < d.n_comm) ? __ldcs(mu + (int64_t)c * (kD / 4) + lane)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 0; k < 4; ++k) qs[k] += elem<BF16>(q, base + k);
+            }
+            gq = g;
         }
+        const int st = u % kScoreNST;
+        const int64_t gi = (int64_t)g * d.Nc + c0 + lane;
+        const int sz = (c0 + lane < d.n_comm) ? s.csize[gi] : 0;
+        if (!mbar_wait(&sm.full[st], (u / kScoreNST) & 1, abort_flag)) break;
+        const int rows = min(32, d.n_comm - c0);
+        const float4* mu = reinterpret_cast<const float4*>(sm.ring[st]);
+        float part[32];
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
-            part[rb + r] = fmaf(qs[3], v[r].w, fmaf(qs[2], v[r].z, fmaf(qs[1], v[r].y, qs[0] * v[r].x)));
-    }
-    // butterfly transpose-reduce: afterwards lane L holds row c0 + L
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        const bool up = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < off; ++i) {
-            const float send = up ? part[i] : part[i + off];
-            const float keep = up ? part[i + off] : part[i];
-            part[i] = keep + __shfl_xor_sync(kFull, send, off);
+        for (int r = 0; r < 32; ++r) {
+            const float4 v = (r < rows) ? mu[r * (kD / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+            part[r] = fmaf(qs[3], v.w, fmaf(qs[2], v.z, fmaf(qs[1], v.y, qs[0] * v.x)));
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[st]);
+        // butterfly transpose-reduce: afterwards lane L holds row c0 + L
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int i = 0; i < off; ++i) {
+                const float send = up ? part[i] : part[i + off];
+                const float keep = up ? part[i + off] : part[i];
+                part[i] = keep + __shfl_xor_sync(kFull, send, off);
+            }
+        }
+        if (lane < rows) s.score[gi] = (sz > 0) ? part[0] : -INFINITY;
     }
-    const int c = c0 + lane;
-    if (c < d.n_comm) {
-        const int64_t gi = (int64_t)g * d.Nc + c;
-        s.score[gi] = (s.csize[gi] > 0) ? part[0] : -INFINITY;
-    }
+    if (*abort_flag && c == 0 && lane == 0) set_error(s.err, CKV_ERR_TIMEOUT);
 }
 
 // -------------------------------------------------------- block utilities
-// inclusive block scan of an int (kSelThreads threads); returns the block total
+// inclusive block scan of an int; returns the block total in `total`
 __device__ __forceinline__ int block_scan_incl(int v, int* warp_sums, int& total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = (int)(blockDim.x >> 5);
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         int t = __shfl_up_sync(kFull, v, o);
@@ -137,7 +192,7 @@ __device__ __forceinline__ int block_scan_incl(int v, int* warp_sums, int& total
     if (lane == 31) warp_sums[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+        int w = (lane < nw) ? warp_sums[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int t = __shfl_up_sync(kFull, w, o);
@@ -147,53 +202,24 @@ __device__ __forceinline__ int block_scan_incl(int v, int* warp_sums, int& total
     }
     __syncthreads();
     const int add = warp ? warp_sums[warp - 1] : 0;
-    total = warp_sums[(blockDim.x >> 5) - 1];
+    total = warp_sums[nw - 1];
     __syncthreads();
     return v + add;
 }
 
-__device__ __forceinline__ float block_reduce_max(float v, float* red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float r = -INFINITY;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) r = fmaxf(r, red[i]);
-    __syncthreads();
-    return r;
-}
-
-__device__ __forceinline__ uint32_t block_reduce_or_u(uint32_t v, uint32_t* red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) v |= __shfl_xor_sync(kFull, v, o);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    uint32_t r = 0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) r |= red[i];
-    __syncthreads();
-    return r;
-}
-
 // --------------------------------------------------------------- k_select
-// Status of a community during selection.
 enum : int8_t { ST_OUT = 0, ST_IN = 1, ST_CAND = 2 };
 
-struct SelShared {
-    int hist[kSelBins];
-    unsigned long long key[kSortCap];
-    int wt[kSortCap];
-    int warp_sums[32];
-    float redf[32];
-    uint32_t redu[32];
-    int bstar;          // boundary bin
-    int w_above;        // weight already kept
-    int n_cand;
-    int done;
+struct SelStats {
+    float lo, hi;
+    uint32_t uor, unand, ior, inand;
+    int cnt;
 };
+
+// shared memory (each region a multiple of 16 bytes):
+//   sc/pre [Nc+1] | wz/coffs [Nc] | hist, keys, weights / sel [max(Nc, 5120)] | st [Nc]
+__host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
+__host__ __device__ inline size_t sel_region3(int Nc) { return (size_t)(Nc > 5120 ? round4(Nc) : 5120); }
 
 // key of a candidate: (order-preserving score bits, inverted id): larger = kept first
 __device__ __forceinline__ unsigned long long sel_key(float sc, int c)
@@ -201,668 +227,805 @@ __device__ __forceinline__ unsigned long long sel_key(float sc, int c)
     return ((unsigned long long)ord_u(sc) << 32) | (unsigned long long)(~(uint32_t)c);
 }
 
-__global__ void __launch_bounds__(kSelThreads) k_select(DevState s, Dims d, int n)
+__global__ void __launch_bounds__(kSelThreads) k_select(DevState s, Dims d)
 {
     if (*(volatile int*)s.err) return;
-    __shared__ SelShared sh;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ int warp_sums[32];
+    __shared__ SelStats wst[32];
+    __shared__ int sh_bstar, sh_above, sh_wabove, sh_done, sh_ncand;
+    __shared__ SelStats sh_tot;
     const int g = blockIdx.x;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Nc = d.n_comm;
-    const float* sc = s.score + (int64_t)g * d.Nc;
-    const int32_t* csz = s.csize + (int64_t)g * d.Nc;
-    int8_t* stat = s.cstat + (int64_t)g * d.Nc;
-    // ---- pass 0: all non-empty communities are candidates
-    int wsum_local = 0;
+    float* sc = reinterpret_cast<float*>(smem);
+    int* pre = reinterpret_cast<int*>(smem);                 // reuses sc after the passes
+    int* wz = reinterpret_cast<int*>(sc + round4(Nc + 1));
+    int* coffs = wz;                                          // reuses wz after compaction
+    int* r3 = wz + round4(Nc);
+    int* hist = r3;                                           // [kSelBins]
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(r3 + kSelBins);   // [kSortCap]
+    int* wts = r3 + kSelBins + 2 * kSortCap;                  // [kSortCap]
+    int* sel_s = r3;                                          // reuses the above after ranking
+    int8_t* st = reinterpret_cast<int8_t*>(r3 + sel_region3(Nc));
+
+    // ---- load the graph's scores and sizes (coalesced, one round)
+    const float* gsc = s.score + (int64_t)g * d.Nc;
+    const int32_t* gsz = s.csize + (int64_t)g * d.Nc;
+    int wsum = 0;
     for (int c = tid; c < Nc; c += kSelThreads) {
-        const int w = csz[c];
-        stat[c] = (w > 0) ? ST_CAND : ST_OUT;
-        wsum_local += (w > 0) ? w : 0;
+        const float v = gsc[c];
+        const int w = gsz[c];
+        sc[c] = v;
+        wz[c] = w;
+        st[c] = (w > 0) ? ST_CAND : ST_OUT;
+        wsum += (w > 0) ? w : 0;
     }
     int total_w;
-    block_scan_incl(wsum_local, sh.warp_sums, total_w);
-    if (tid == 0) { sh.w_above = 0; sh.done = (total_w <= d.budget) ? 1 : 0; }
+    block_scan_incl(wsum, warp_sums, total_w);
+    if (tid == 0) { sh_wabove = 0; sh_done = (total_w <= d.budget); }
     __syncthreads();
-    if (sh.done) {   // every community fits the budget: keep them all
+    if (sh_done) {   // every community fits the budget: keep them all
         for (int c = tid; c < Nc; c += kSelThreads)
-            if (stat[c] == ST_CAND) stat[c] = ST_IN;
-        __syncthreads();
+            if (st[c] == ST_CAND) st[c] = ST_IN;
     }
 
-    // ---- bucket passes until <= kSortCap candidates remain
-    // pass kinds: 0 = linear in the float score over [lo, hi]; 1 = radix window
-    // of ord_u(score); 2 = radix window of the inverted id.
-    int kind = 0;
-    for (int pass = 0; pass < 12 && !sh.done; ++pass) {
-        // candidate statistics
-        float lo = INFINITY, hi = -INFINITY;
-        uint32_t uor = 0, uand = 0xffffffffu, ior = 0, iand = 0xffffffffu;
-        int cnt = 0;
+    // ---- bucket passes until <= kSortCap candidates remain.  Each thread
+    // owns communities tid, tid + 1024, ... so statuses need no barrier.
+    int kind = 0;   // 0 linear in the score over [lo, hi], 1 radix window of ord_u, 2 of the id
+    for (int pass = 0; pass < 12 && !sh_done; ++pass) {
+        SelStats a{INFINITY, -INFINITY, 0u, 0u, 0u, 0u, 0};
         for (int c = tid; c < Nc; c += kSelThreads) {
-            if (stat[c] != ST_CAND) continue;
+            if (st[c] != ST_CAND) continue;
             const float v = sc[c];
-            lo = fminf(lo, v);
-            hi = fmaxf(hi, v);
             const uint32_t u = ord_u(v), iv = ~(uint32_t)c;
-            uor |= u; uand &= u; ior |= iv; iand &= iv;
-            ++cnt;
+            a.lo = fminf(a.lo, v);
+            a.hi = fmaxf(a.hi, v);
+            a.uor |= u; a.unand |= ~u; a.ior |= iv; a.inand |= ~iv;
+            ++a.cnt;
         }
-        int ncand;
-        block_scan_incl(cnt, sh.warp_sums, ncand);
-        if (ncand <= kSortCap) break;
-        const float glo = -block_reduce_max(-lo, sh.redf);
-        const float ghi = block_reduce_max(hi, sh.redf);
-        // bits that differ among the candidates: OR of all & ~(AND of all)
-        const uint32_t udiff = block_reduce_or_u(uor, sh.redu) & block_reduce_or_u(~uand, sh.redu);
-        const uint32_t idiff = block_reduce_or_u(ior, sh.redu) & block_reduce_or_u(~iand, sh.redu);
-        int shift = 0;
-        if (kind == 0 && !(glo < ghi)) kind = 1;
-        if (kind == 1 && udiff == 0) kind = 2;
-        if (kind == 1) { const int top = 31 - __clz(udiff); shift = max(0, top - 10); }
-        if (kind == 2) { const int top = 31 - __clz(idiff); shift = max(0, top - 10); }
-        const double dlo = (double)glo, dscale = (double)kSelBins / ((double)ghi - (double)glo);
-        for (int i = tid; i < kSelBins; i += kSelThreads) sh.hist[i] = 0;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            a.lo = fminf(a.lo, __shfl_xor_sync(kFull, a.lo, o));
+            a.hi = fmaxf(a.hi, __shfl_xor_sync(kFull, a.hi, o));
+            a.uor |= __shfl_xor_sync(kFull, a.uor, o);
+            a.unand |= __shfl_xor_sync(kFull, a.unand, o);
+            a.ior |= __shfl_xor_sync(kFull, a.ior, o);
+            a.inand |= __shfl_xor_sync(kFull, a.inand, o);
+            a.cnt += __shfl_xor_sync(kFull, a.cnt, o);
+        }
+        if (lane == 0) wst[warp] = a;
+        for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0;
         __syncthreads();
-        for (int c = tid; c < Nc; c += kSelThreads) {
-            if (stat[c] != ST_CAND) continue;
-            const float v = sc[c];
-            int bin;
-            if (kind == 0) bin = max(0, min(kSelBins - 1, (int)(((double)v - dlo) * dscale)));
-            else if (kind == 1) bin = (int)((ord_u(v) >> shift) & (kSelBins - 1));
-            else bin = (int)((~(uint32_t)c >> shift) & (kSelBins - 1));
-            atomicAdd(&sh.hist[bin], csz[c]);
+        if (warp == 0) {
+            SelStats o = wst[lane];
+#pragma unroll
+            for (int x = 16; x; x >>= 1) {
+                o.lo = fminf(o.lo, __shfl_xor_sync(kFull, o.lo, x));
+                o.hi = fmaxf(o.hi, __shfl_xor_sync(kFull, o.hi, x));
+                o.uor |= __shfl_xor_sync(kFull, o.uor, x);
+                o.unand |= __shfl_xor_sync(kFull, o.unand, x);
+                o.ior |= __shfl_xor_sync(kFull, o.ior, x);
+                o.inand |= __shfl_xor_sync(kFull, o.inand, x);
+                o.cnt += __shfl_xor_sync(kFull, o.cnt, x);
+            }
+            if (lane == 0) sh_tot = o;
         }
+        __syncthreads();
+        const SelStats t = sh_tot;
+        if (t.cnt <= kSortCap) break;                       // uniform
+        // bits that differ among the candidates: OR of all & OR of complements
+        const uint32_t udiff = t.uor & t.unand, idiff = t.ior & t.inand;
+        if (kind == 0 && !(t.lo < t.hi)) kind = 1;
+        if (kind == 1 && udiff == 0) kind = 2;
+        int shift = 0;
+        if (kind == 1) shift = max(0, 31 - __clz(udiff) - 10);
+        if (kind == 2) shift = max(0, 31 - __clz(idiff) - 10);
+        const double dlo = (double)t.lo, dscale = (double)kSelBins / ((double)t.hi - (double)t.lo);
+        auto bin_of = [&](int c) -> int {
+            if (kind == 0) return max(0, min(kSelBins - 1, (int)(((double)sc[c] - dlo) * dscale)));
+            if (kind == 1) return (int)((ord_u(sc[c]) >> shift) & (kSelBins - 1));
+            return (int)((~(uint32_t)c >> shift) & (kSelBins - 1));
+        };
+        for (int c = tid; c < Nc; c += kSelThreads)
+            if (st[c] == ST_CAND) atomicAdd(&hist[bin_of(c)], wz[c]);
         __syncthreads();
         // boundary bin, scanning from the top bin down (2 bins per thread)
         const int rb0 = kSelBins - 1 - 2 * tid, rb1 = rb0 - 1;
-        const int h0v = sh.hist[rb0], h1v = sh.hist[rb1];
+        const int h0v = hist[rb0], h1v = hist[rb1];
         int tot;
-        const int incl = block_scan_incl(h0v + h1v, sh.warp_sums, tot);
-        const int before = sh.w_above + incl - (h0v + h1v);
-        if (tid == 0) sh.bstar = -1;
+        const int incl = block_scan_incl(h0v + h1v, warp_sums, tot);
+        const int w_above = sh_wabove;
+        const int before = w_above + incl - (h0v + h1v);
+        if (tid == 0) sh_bstar = -1;
         __syncthreads();
-        if (before <= d.budget && before + h0v > d.budget) sh.bstar = rb0;
-        else if (before + h0v <= d.budget && before + h0v + h1v > d.budget) sh.bstar = rb1;
-        __syncthreads();
-        const int bstar = sh.bstar;
-        // weight strictly above the boundary bin
-        int above_local = 0;
-        if (bstar >= 0) {
-            if (rb0 > bstar) above_local += h0v;
-            if (rb1 > bstar) above_local += h1v;
+        if (before <= d.budget && before + h0v > d.budget) { sh_bstar = rb0; sh_above = before - w_above; }
+        else if (before + h0v <= d.budget && before + h0v + h1v > d.budget) {
+            sh_bstar = rb1;
+            sh_above = before + h0v - w_above;
         }
-        int above;
-        block_scan_incl(above_local, sh.warp_sums, above);
+        __syncthreads();
+        const int bstar = sh_bstar;
         for (int c = tid; c < Nc; c += kSelThreads) {
-            if (stat[c] != ST_CAND) continue;
-            if (bstar < 0) { stat[c] = ST_IN; continue; }
-            const float v = sc[c];
-            int bin;
-            if (kind == 0) bin = max(0, min(kSelBins - 1, (int)(((double)v - dlo) * dscale)));
-            else if (kind == 1) bin = (int)((ord_u(v) >> shift) & (kSelBins - 1));
-            else bin = (int)((~(uint32_t)c >> shift) & (kSelBins - 1));
-            stat[c] = (bin > bstar) ? ST_IN : (bin < bstar ? ST_OUT : ST_CAND);
-        }
-        __syncthreads();
-        if (tid == 0) {
-            if (bstar < 0) sh.done = 1;
-            else sh.w_above += above;
+            if (st[c] != ST_CAND) continue;
+            if (bstar < 0) { st[c] = ST_IN; continue; }
+            const int bin = bin_of(c);
+            st[c] = (bin > bstar) ? ST_IN : (bin < bstar ? ST_OUT : ST_CAND);
         }
         if (kind == 0) kind = 1;   // the linear pass runs once, radix windows after
         __syncthreads();
+        if (tid == 0) {
+            if (bstar < 0) sh_done = 1;
+            else sh_wabove = w_above + sh_above;
+        }
+        __syncthreads();
     }
 
-    // ---- final exact pass: sort the remaining candidates by key
-    if (!sh.done) {
-        if (tid == 0) sh.n_cand = 0;
+    // ---- final exact pass: rank the remaining candidates by key
+    if (!sh_done) {
+        if (tid == 0) sh_ncand = 0;
         __syncthreads();
         for (int c = tid; c < Nc; c += kSelThreads) {
-            if (stat[c] != ST_CAND) continue;
-            const int slot = atomicAdd(&sh.n_cand, 1);
-            if (slot < kSortCap) { sh.key[slot] = sel_key(sc[c], c); sh.wt[slot] = csz[c]; }
+            if (st[c] != ST_CAND) continue;
+            const int slot = atomicAdd(&sh_ncand, 1);
+            if (slot < kSortCap) { keys[slot] = sel_key(sc[c], c); wts[slot] = wz[c]; }
         }
         __syncthreads();
-        const int m = min(sh.n_cand, kSortCap);
-        int m2 = 1;
-        while (m2 < m) m2 <<= 1;
-        for (int i = m + tid; i < m2; i += kSelThreads) { sh.key[i] = 0ull; sh.wt[i] = 0; }
-        __syncthreads();
-        // bitonic sort, descending keys
-        for (int k = 2; k <= m2; k <<= 1) {
-            for (int j = k >> 1; j > 0; j >>= 1) {
-                for (int i = tid; i < m2; i += kSelThreads) {
-                    const int p = i ^ j;
-                    if (p > i) {
-                        const bool desc = ((i & k) == 0);
-                        const unsigned long long a = sh.key[i], bb = sh.key[p];
-                        if (desc ? (a < bb) : (a > bb)) {
-                            sh.key[i] = bb; sh.key[p] = a;
-                            const int t = sh.wt[i]; sh.wt[i] = sh.wt[p]; sh.wt[p] = t;
-                        }
-                    }
-                }
-                __syncthreads();
-            }
+        const int m = min(sh_ncand, kSortCap);
+        int rank = 0;
+        unsigned long long mykey = 0ull;
+        int myw = 0;
+        if (tid < m) {
+            mykey = keys[tid];
+            myw = wts[tid];
+            for (int k = 0; k < m; ++k) rank += (keys[k] > mykey);   // keys are distinct
         }
-        // keep the prefix that fits (forced first when nothing is kept yet)
-        const int w_above = sh.w_above;
-        int local = (tid < m) ? sh.wt[tid] : 0;
+        __syncthreads();
+        // weights in rank order, then an inclusive prefix over them
+        if (tid < m) { wts[rank] = myw; keys[rank] = mykey; }
+        __syncthreads();
+        const int wr = (tid < m) ? wts[tid] : 0;
         int tot;
-        const int incl = block_scan_incl(local, sh.warp_sums, tot);
+        const int incl = block_scan_incl(wr, warp_sums, tot);
+        const int w_above = sh_wabove;
         if (tid < m) {
             const bool keep = (w_above + incl <= d.budget) || (w_above == 0 && tid == 0);
-            const int c = (int)(~(uint32_t)(sh.key[tid] & 0xffffffffull));
-            stat[c] = keep ? ST_IN : ST_OUT;
+            const int c = (int)(~(uint32_t)(keys[tid] & 0xffffffffull));
+            st[c] = keep ? ST_IN : ST_OUT;
         }
         __syncthreads();
     }
 
-    // ---- compaction in ascending id, prefix of sizes
-    int32_t* sel = s.sel + (int64_t)g * d.Nc;
-    int32_t* pre = s.sel_pre + (int64_t)g * (d.Nc + 1);
-    int carry_c = 0, carry_t = 0;
-    for (int base = 0; base < Nc; base += kSelThreads) {
-        const int c = base + tid;
-        const bool in = (c < Nc) && stat[c] == ST_IN;
-        const int w = in ? csz[c] : 0;
-        int tc, tw;
-        const int ic = block_scan_incl(in ? 1 : 0, sh.warp_sums, tc);
-        const int iw = block_scan_incl(w, sh.warp_sums, tw);
-        if (in) {
-            sel[carry_c + ic - 1] = c;
-            pre[carry_c + ic - 1] = carry_t + iw - w;
+    // ---- compaction in ascending id, prefix of sizes (pre reuses sc).
+    // Thread t owns the consecutive ids [t*per, (t+1)*per): two block scans
+    // (kept count, kept weight) place every thread's kept communities.
+    int32_t* gsel = s.sel + (int64_t)g * d.Nc;
+    const int per = (Nc + kSelThreads - 1) / kSelThreads;
+    const int c_lo = min(Nc, tid * per), c_hi = min(Nc, c_lo + per);
+    int my_c = 0, my_t = 0;
+    for (int c = c_lo; c < c_hi; ++c)
+        if (st[c] == ST_IN) { ++my_c; my_t += wz[c]; }
+    int tot_c, tot_t;
+    const int inc_c = block_scan_incl(my_c, warp_sums, tot_c);
+    const int inc_t = block_scan_incl(my_t, warp_sums, tot_t);
+    {
+        int pos = inc_c - my_c, acc = inc_t - my_t;
+        for (int c = c_lo; c < c_hi; ++c) {
+            if (st[c] != ST_IN) continue;
+            sel_s[pos] = c;
+            gsel[pos] = c;
+            pre[pos] = acc;
+            acc += wz[c];
+            ++pos;
         }
-        carry_c += tc;
-        carry_t += tw;
     }
+    const int C = tot_c, T = tot_t;
     if (tid == 0) {
-        pre[carry_c] = carry_t;
+        pre[C] = T;
         int32_t* meta = s.meta + (int64_t)g * M_COUNT;
-        meta[M_C] = carry_c;
-        meta[M_T] = carry_t;
-        meta[M_ROWS] = d.S + carry_t + 1;
+        meta[M_C] = C;
+        meta[M_T] = T;
+        meta[M_ROWS] = d.S + T + 1;
     }
     __syncthreads();
-    // ---- materialise the kept member rows: token and community of row r
-    const int32_t* coff = s.coff + (int64_t)g * d.Nc;
+    // ---- kept rows: segment starts of the kept communities (one round),
+    // then every row's token (one round)
+    const int32_t* gcoff = s.coff + (int64_t)g * d.Nc;
+    for (int k = tid; k < C; k += kSelThreads) coffs[k] = gcoff[sel_s[k]];
+    __syncthreads();
     const int32_t* pool = s.pool + (int64_t)g * d.P;
     int32_t* rtok = s.rtok + (int64_t)g * d.NM;
     int32_t* rcomm = s.rcomm + (int64_t)g * d.NM;
-    const int lane = tid & 31, warp = tid >> 5;
-    for (int k = warp; k < carry_c; k += kSelThreads / 32) {
-        const int c = sel[k];
-        const int off = coff[c];
-        const int sz = csz[c];
-        const int p0 = pre[k];
-        for (int i = lane; i < sz; i += 32) {
-            rtok[p0 + i] = pool[off + i];
-            rcomm[p0 + i] = c;
+    for (int base = 0; base < T; base += 4 * kSelThreads) {
+        int src[4], cc[4], idx[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            idx[u] = base + u * kSelThreads + tid;
+            src[u] = -1;
+            cc[u] = 0;
+            if (idx[u] < T) {
+                int lo = 0, hi = C - 1;          // last k with pre[k] <= idx
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (pre[mid] <= idx[u]) lo = mid; else hi = mid - 1;
+                }
+                src[u] = coffs[lo] + idx[u] - pre[lo];
+                cc[u] = sel_s[lo];
+            }
         }
+        int tk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tk[u] = (src[u] >= 0) ? pool[src[u]] : 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (src[u] >= 0) { rtok[idx[u]] = tk[u]; rcomm[idx[u]] = cc[u]; }
     }
-    (void)n;
 }
 
 // --------------------------------------------------------------- k_attend
-// shared layout: q[HG][128] f32 | tok[2][32] | K[2][32][RB] | V[2][32][RB] |
-//                zp[8][HG][32] | p[32][HG] | alpha[HG] | misc
+// Each warp owns a contiguous run of a graph slice's rows and streams them
+// through its own 3-buffer shared-memory pipeline: 8 rows per batch, K and
+// V of a row fetched together with 16-byte cp.async (the LSU gather path;
+// one bulk TMA copy per 256-byte row is far slower).  Per 4-row group the
+// lane's partial dots are reduced by a butterfly transpose; the warp keeps
+// an online softmax (running max, sum, P.V) per head and spills the logits
+// of the kept members to L2 for the edges.  The CTA combines its warps into
+// one (m, l, o) partial per head; the last CTA of a graph merges the
+// partials exactly, then ranks all kept members' edge weights.
+constexpr int kAttWarps = 16;
+constexpr int kAttNBuf = 3;        // batches per warp pipeline
+
 template <bool BF16, int HG>
 struct AttLayout {
-    static constexpr int RB = kD * (BF16 ? 2 : 4);       // bytes per K/V row
-    static constexpr int NCH = RB / 16;                  // 16-byte chunks per row
-    static constexpr int off_q = 0;
-    static constexpr int off_tok = off_q + HG * kD * 4;
-    static constexpr int off_k = off_tok + 2 * kTile * 4;
-    static constexpr int off_v = off_k + 2 * kTile * RB;
-    static constexpr int off_zp = off_v + 2 * kTile * RB;
-    static constexpr int off_p = off_zp + 8 * HG * kTile * 4;
-    static constexpr int off_alpha = off_p + kTile * HG * 4;
-    static constexpr int bytes_loop = off_alpha + 64;
-    // end-of-CTA reduction buffer (reuses the K/V region): [16][HG][128] f32
-    static constexpr int bytes_red = off_k + 16 * HG * kD * 4;
-    static constexpr int bytes = bytes_loop > bytes_red ? bytes_loop : bytes_red;
+    static constexpr int NB = BF16 ? 8 : 4;                      // rows per warp batch
+    static constexpr int RB = kD * (BF16 ? 2 : 4);               // bytes per K or V row
+    static constexpr int NCH = RB / 16;                          // 16-byte chunks per row
+    static constexpr int BATCH = NB * 2 * RB;                    // K and V of one batch
+    static constexpr int WBUF = kAttNBuf * BATCH;                // one warp's pipeline
+    static constexpr int off_buf = 0;
+    static constexpr int TOKW = 64;                              // row tokens a warp keeps at once
+    static constexpr int off_pz = off_buf + kAttWarps * WBUF;    // [warps][NB*HG] z / p exchange
+    static constexpr int off_tokw = off_pz + kAttWarps * NB * HG * 4;  // [warps][TOKW]
+    static constexpr int off_misc = off_tokw + kAttWarps * TOKW * 4;
+    static constexpr int bytes = off_misc + 512;
+    // end-of-slice reduction [warps][HG][RSTR] reuses the pipelines; a row is
+    // acc[0..D), m, l, padded to a multiple of 16 bytes for float4 stores
+    static constexpr int RSTR = kD + 4;
+    static_assert(kAttWarps * HG * RSTR * 4 <= kAttWarps * WBUF, "reduction must fit");
 };
-
-__device__ __forceinline__ int swz(int row, int ch) { return (ch & ~7) | ((ch ^ row) & 7); }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
 {
-    const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
-template <bool BF16, int HG>
-__global__ void __launch_bounds__(kAttThreads) k_attend(DevState s, Dims d, const void* __restrict__ q,
-                                                       const void* __restrict__ K,
-                                                       const void* __restrict__ V, int n,
-                                                       float* __restrict__ out)
+// Butterfly transpose-reduce of NV values per lane (NV a power of two
+// <= 32): afterwards every lane holds the warp-wide sum of value index
+// tr_index<NV>(lane); lanes that differ only in the bits below the last
+// halving offset hold the same value.
+template <int NV>
+__device__ __forceinline__ int tr_index(int lane)
+{
+    int idx = 0;
+#pragma unroll
+    for (int s = 0, len = NV; len > 1; ++s, len >>= 1)
+        idx += ((lane >> (4 - s)) & 1) * (len >> 1);
+    return idx;
+}
+
+template <int NV>
+__device__ __forceinline__ float transpose_reduce(float (&v)[NV], int lane)
+{
+#pragma unroll
+    for (int s = 0, len = NV; len > 1; ++s, len >>= 1) {
+        const int off = 16 >> s;
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < (len >> 1); ++i) {
+            const float send = up ? v[i] : v[i + (len >> 1)];
+            const float keep = up ? v[i + (len >> 1)] : v[i];
+            v[i] = keep + __shfl_xor_sync(kFull, send, off);
+        }
+    }
+    float r = v[0];
+    constexpr int levels = (NV >= 32) ? 5 : (NV >= 16) ? 4 : (NV >= 8) ? 3 : (NV >= 4) ? 2 : (NV >= 2) ? 1 : 0;
+#pragma unroll
+    for (int off = 16 >> levels; off >= 1 && levels < 5; off >>= 1) r += __shfl_xor_sync(kFull, r, off);
+    return r;
+}
+
+// A lane's sorted (w desc, token asc) list of its best KM candidates.
+template <int KM>
+struct TopList {
+    float w[KM];
+    int t[KM], x[KM];
+    __device__ __forceinline__ void clear()
+    {
+#pragma unroll
+        for (int i = 0; i < KM; ++i) { w[i] = -INFINITY; t[i] = 0x7fffffff; x[i] = -1; }
+    }
+    __device__ __forceinline__ void insert(float nw, int nt, int nx)
+    {
+        if (!cand_better(nw, nt, w[KM - 1], t[KM - 1])) return;
+#pragma unroll
+        for (int i = KM - 1; i > 0; --i) {
+            const bool shift = cand_better(nw, nt, w[i - 1], t[i - 1]);
+            const bool land = !shift && cand_better(nw, nt, w[i], t[i]);
+            w[i] = shift ? w[i - 1] : (land ? nw : w[i]);
+            t[i] = shift ? t[i - 1] : (land ? nt : t[i]);
+            x[i] = shift ? x[i - 1] : (land ? nx : x[i]);
+        }
+        if (cand_better(nw, nt, w[0], t[0])) { w[0] = nw; t[0] = nt; x[0] = nx; }
+    }
+    __device__ __forceinline__ void pop()
+    {
+#pragma unroll
+        for (int i = 0; i < KM - 1; ++i) { w[i] = w[i + 1]; t[i] = t[i + 1]; x[i] = x[i + 1]; }
+        w[KM - 1] = -INFINITY; t[KM - 1] = 0x7fffffff; x[KM - 1] = -1;
+    }
+};
+
+// Merge the 32 lanes' lists: the warp's top kappa (kappa <= KM) in rank
+// order, written by lane 0; returns how many (entries with w = -inf are
+// empty).
+template <int KM>
+__device__ __forceinline__ int warp_merge(TopList<KM>& L, int kappa, float* ow, int* ot, int* ox)
+{
+    const int lane = threadIdx.x & 31;
+    int nout = 0;
+    for (int k = 0; k < kappa; ++k) {
+        float bw = L.w[0];
+        int bt = L.t[0], bl = lane;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const float w2 = __shfl_xor_sync(kFull, bw, o);
+            const int t2 = __shfl_xor_sync(kFull, bt, o);
+            const int l2 = __shfl_xor_sync(kFull, bl, o);
+            if (cand_better(w2, t2, bw, bt) || (w2 == bw && t2 == bt && l2 < bl)) { bw = w2; bt = t2; bl = l2; }
+        }
+        if (bw == -INFINITY) break;
+        const int bx = __shfl_sync(kFull, L.x[0], bl);
+        if (lane == 0) { ow[k] = bw; ot[k] = bt; ox[k] = bx; }
+        if (lane == bl) L.pop();
+        ++nout;
+    }
+    return nout;
+}
+
+template <bool BF16, int HG, int KM>
+__global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d, const void* __restrict__ q,
+                                                             const void* __restrict__ K,
+                                                             const void* __restrict__ V, int n,
+                                                             float* __restrict__ out)
 {
     using L = AttLayout<BF16, HG>;
+    constexpr int NV = 4 * HG;                           // values per 4-row group: (row, head)
+    constexpr int RB = L::RB;
+    constexpr int NT = kAttWarps * 32;
+    constexpr int kAttNB = L::NB;
     if (*(volatile int*)s.err) return;
     extern __shared__ __align__(128) unsigned char smem[];
-    float* qf = reinterpret_cast<float*>(smem + L::off_q);
-    int* tok = reinterpret_cast<int*>(smem + L::off_tok);
-    unsigned char* Ks = smem + L::off_k;
-    unsigned char* Vs = smem + L::off_v;
-    float* zp = reinterpret_cast<float*>(smem + L::off_zp);
-    float* pt = reinterpret_cast<float*>(smem + L::off_p);
-    float* alpha = reinterpret_cast<float*>(smem + L::off_alpha);
-    __shared__ int s_last;
-
-    const int g = blockIdx.y, split = blockIdx.x;
+    float* sM = reinterpret_cast<float*>(smem + L::off_misc);          // [8]
+    float* sL = sM + 8;                                                // [8] 1 / L
+    float* mw = sL + 8;                                                // [warps] scratch
+    int* sidx = reinterpret_cast<int*>(mw + kAttWarps);
+    __shared__ int sh_seg[4];          // graph, slice, slices, last
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int b, h0, kvh;
-    graph_heads(d, g, b, h0, kvh);
-    const int R = s.meta[(int64_t)g * M_COUNT + M_ROWS];
-    const int T = R - d.S - 1;
-    const int per = (R + gridDim.x - 1) / gridDim.x;
-    const int r0 = min(R, split * per), r1 = min(R, r0 + per);
-    const int ntiles = (r1 - r0 + kTile - 1) / kTile;
-    const int t_new = n - 1;
-    const int64_t kvbase = ((int64_t)b * d.Hkv + kvh) * d.NM;     // row index base
-    const char* Kb = reinterpret_cast<const char*>(K) + kvbase * L::RB;
-    const char* Vb = reinterpret_cast<const char*>(V) + kvbase * L::RB;
-    const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
-    float* zrow = s.zrow + (int64_t)g * d.NM * HG;
+    const int nCTA = gridDim.x, bid = blockIdx.x;
+    const int G = d.G;
+    unsigned char* wbuf = smem + L::off_buf + warp * L::WBUF;
+    float* pz = reinterpret_cast<float*>(smem + L::off_pz) + warp * L::NB * HG;
 
-    for (int i = tid; i < HG * kD; i += kAttThreads) {
-        const int h = i / kD, dd = i % kD;
-        qf[i] = elem<BF16>(q, ((int64_t)b * d.Hq + h0 + h) * kD + dd);
+    // ---- which graph slice(s) this CTA owns.  G <= nCTA: every graph gets
+    // one CTA plus a share of the others proportional to its rows, and each
+    // CTA owns one contiguous slice of one graph.  G > nCTA: each CTA owns
+    // whole graphs.
+    int g_first, g_last;
+    if (G > nCTA) {
+        g_first = (int)((int64_t)bid * G / nCTA);
+        g_last = (int)((int64_t)(bid + 1) * G / nCTA);
+    } else {
+        // rows of every graph, staged once (one round of loads); warp 0 then
+        // forms their prefix and the first CTA of each graph,
+        // f(g) = g + floor(P_g * extra / R_tot)
+        int* sR = reinterpret_cast<int*>(smem + L::off_buf);
+        for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
+        __syncthreads();
+        if (warp == 0) {
+            const int extra = nCTA - G;
+            double R_tot = 0.0;
+            for (int g0 = 0; g0 < G; g0 += 32) {
+                const int g = g0 + lane;
+                R_tot += (g < G) ? (double)sR[g] : 0.0;
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) R_tot += __shfl_xor_sync(kFull, R_tot, o);
+            double carry = 0.0;
+            for (int g0 = 0; g0 < G; g0 += 32) {
+                const int g = g0 + lane;
+                const double R = (g < G) ? (double)sR[g] : 0.0;
+                double incl = R;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const double t = __shfl_up_sync(kFull, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const double P = carry + incl - R;
+                const int f = g + (int)floor(P * extra / R_tot);
+                const int f1 = g + 1 + (int)floor((P + R) * extra / R_tot);
+                if (g < G && bid >= f && bid < f1) {
+                    sh_seg[0] = g;
+                    sh_seg[1] = bid - f;
+                    sh_seg[2] = f1 - f;
+                }
+                carry += __shfl_sync(kFull, incl, 31);
+            }
+        }
+        __syncthreads();
+        g_first = sh_seg[0];
+        g_last = g_first + 1;
     }
 
-    auto row_token = [&](int r) -> int {
-        if (r < d.S) return r;
-        if (r == R - 1) return t_new;
-        return rtok[r - d.S];
-    };
-    auto issue = [&](int tile) {
-        const int buf = tile & 1;
-        const int rbase = r0 + tile * kTile;
-        if (tid < kTile) {
-            const int r = rbase + tid;
-            tok[buf * kTile + tid] = (r < r1) ? row_token(r) : -1;
-        }
-        __syncthreads();
-        // K and V: kTile rows x NCH chunks each
-        for (int i = tid; i < kTile * L::NCH; i += kAttThreads) {
-            const int row = i / L::NCH, ch = i % L::NCH;
-            const int tk = tok[buf * kTile + row];
-            if (tk < 0) continue;
-            const int dst = (buf * kTile + row) * L::RB + swz(row, ch) * 16;
-            cp_async16(Ks + dst, Kb + (int64_t)tk * L::RB + ch * 16);
-            cp_async16(Vs + dst, Vb + (int64_t)tk * L::RB + ch * 16);
-        }
-        cp_async_commit();
-    };
+    for (int g = g_first; g < g_last; ++g) {
+        const int k = (G > nCTA) ? 0 : sh_seg[1];
+        const int nc = (G > nCTA) ? 1 : sh_seg[2];
+        int b, h0, kvh;
+        graph_heads(d, g, b, h0, kvh);
+        const int R = s.meta[(int64_t)g * M_COUNT + M_ROWS];
+        const int T = R - d.S - 1;
+        const int r0 = (int)((int64_t)k * R / nc), r1 = (int)((int64_t)(k + 1) * R / nc);
+        const int nrows = r1 - r0;
+        // this warp's rows, in graph-row numbering: [a0, a1)
+        const int a0 = r0 + (int)((int64_t)warp * nrows / kAttWarps);
+        const int a1 = r0 + (int)((int64_t)(warp + 1) * nrows / kAttWarps);
+        const int nb = (a1 - a0 + kAttNB - 1) / kAttNB;
+        const int t_new = n - 1;
+        const int64_t kvbase = ((int64_t)b * d.Hkv + kvh) * d.NM;
+        const char* Kb = reinterpret_cast<const char*>(K) + kvbase * RB;
+        const char* Vb = reinterpret_cast<const char*>(V) + kvbase * RB;
+        const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
+        float* zrow = s.zrow + (int64_t)g * d.NM * HG;
+        auto row_token = [&](int r) -> int {
+            if (r < d.S) return r;
+            if (r == R - 1) return t_new;
+            return rtok[r - d.S];
+        };
 
-    // running softmax state, kept by warp h for head h
-    float m_run = -INFINITY, l_run = 0.f;
-    // PV accumulators: thread = (row group rg = tid/16, chunk c8 = tid%16): 8 dims x HG heads
-    const int c8 = tid & 15, rg = tid >> 4;
-    float acc[HG][8];
+        float qv[HG][4];
 #pragma unroll
-    for (int h = 0; h < HG; ++h)
+        for (int h = 0; h < HG; ++h)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[h][j] = 0.f;
+            for (int j = 0; j < 4; ++j)
+                qv[h][j] = elem<BF16>(q, ((int64_t)b * d.Hq + h0 + h) * kD + 4 * lane + j);
+        __syncthreads();   // the previous graph of this CTA is done with the buffers
 
-    const float scale = 0.08838834764831845f;   // 1 / sqrt(128), correctly rounded
-    if (ntiles > 0) issue(0);
-    for (int tile = 0; tile < ntiles; ++tile) {
-        const int buf = tile & 1;
-        if (tile + 1 < ntiles) { issue(tile + 1); cp_async_wait<1>(); }
-        else cp_async_wait<0>();
-        __syncthreads();
-        // ---- logits: warp e = dims [16e, 16e+16), lane = row
-        {
-            const int e = warp, r = lane;
-            float a[HG][8];
+        // row tokens of this warp, TOKW at a time (one round of loads each)
+        int* tokw = reinterpret_cast<int*>(smem + L::off_tokw) + warp * L::TOKW;
+        int tok_base = -L::TOKW;
+        auto tokens_from = [&](int r) {   // fill tokw with rows r .. r + TOKW - 1
+            __syncwarp();
+            int t0 = 0, t1 = 0;
+            if (r + lane < a1) t0 = row_token(r + lane);
+            if (r + 32 + lane < a1) t1 = row_token(r + 32 + lane);
+            tokw[lane] = t0;
+            tokw[32 + lane] = t1;
+            tok_base = r;
+            __syncwarp();
+        };
+        // batch bb's rows a0 + NB*bb .. : K rows at BATCH*buf, V rows after them
+        auto issue = [&](int bb) {
+            if (bb < nb) {
+                unsigned char* dst = wbuf + (bb % kAttNBuf) * L::BATCH;
+                const int rbase = a0 + bb * kAttNB;
+                if (rbase + kAttNB > tok_base + L::TOKW) tokens_from(rbase);
 #pragma unroll
-            for (int h = 0; h < HG; ++h)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) a[h][j] = 0.f;
-            const unsigned char* krow = Ks + (buf * kTile + r) * L::RB;
-            if (BF16) {
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int ch = 2 * e + cc;
-                    const uint4 w = *reinterpret_cast<const uint4*>(krow + swz(r, ch) * 16);
-                    float kv[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
-                                   bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
-#pragma unroll
-                    for (int h = 0; h < HG; ++h) {
-                        const float4 qa = *reinterpret_cast<const float4*>(qf + h * kD + ch * 8);
-                        const float4 qb = *reinterpret_cast<const float4*>(qf + h * kD + ch * 8 + 4);
-                        a[h][0] = fmaf(qa.x, kv[0], a[h][0]);
-                        a[h][1] = fmaf(qa.y, kv[1], a[h][1]);
-                        a[h][2] = fmaf(qa.z, kv[2], a[h][2]);
-                        a[h][3] = fmaf(qa.w, kv[3], a[h][3]);
-                        a[h][4] = fmaf(qb.x, kv[4], a[h][4]);
-                        a[h][5] = fmaf(qb.y, kv[5], a[h][5]);
-                        a[h][6] = fmaf(qb.z, kv[6], a[h][6]);
-                        a[h][7] = fmaf(qb.w, kv[7], a[h][7]);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int ch = 4 * e + cc;
-                    const float4 w = *reinterpret_cast<const float4*>(krow + swz(r, ch) * 16);
-#pragma unroll
-                    for (int h = 0; h < HG; ++h) {
-                        const float4 qa = *reinterpret_cast<const float4*>(qf + h * kD + ch * 4);
-                        const int j0 = (cc & 1) * 4;
-                        a[h][j0 + 0] = fmaf(qa.x, w.x, a[h][j0 + 0]);
-                        a[h][j0 + 1] = fmaf(qa.y, w.y, a[h][j0 + 1]);
-                        a[h][j0 + 2] = fmaf(qa.z, w.z, a[h][j0 + 2]);
-                        a[h][j0 + 3] = fmaf(qa.w, w.w, a[h][j0 + 3]);
+                for (int j = 0; j < kAttNB * L::NCH / 32; ++j) {
+                    const int e = j * 32 + lane;
+                    const int row = e / L::NCH, ch = e % L::NCH;
+                    const int tk = tokw[rbase - tok_base + row];
+                    if (rbase + row < a1) {
+                        cp_async16(dst + row * RB + ch * 16, Kb + (int64_t)tk * RB + ch * 16);
+                        cp_async16(dst + (kAttNB + row) * RB + ch * 16, Vb + (int64_t)tk * RB + ch * 16);
                     }
                 }
             }
+            cp_async_commit();
+        };
+
+        float m_run[HG], l_run[HG], acc[HG][4];
 #pragma unroll
-            for (int h = 0; h < HG; ++h)
-                zp[(e * HG + h) * kTile + r] =
-                    ((a[h][0] + a[h][1]) + (a[h][2] + a[h][3])) + ((a[h][4] + a[h][5]) + (a[h][6] + a[h][7]));
+        for (int h = 0; h < HG; ++h) {
+            m_run[h] = -INFINITY;
+            l_run[h] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
         }
-        __syncthreads();
-        // ---- softmax of the tile: warp h handles head h, lane = row
-        if (warp < HG) {
-            const int h = warp, r = lane;
-            const int gr = r0 + tile * kTile + r;
-            float z = -INFINITY;
-            if (gr < r1) {
-                float v[8];
+        issue(0);
+        issue(1);
+        for (int bb = 0; bb < nb; ++bb) {
+            issue(bb + 2);
+            cp_async_wait<kAttNBuf - 1>();
+            __syncwarp();
+            const unsigned char* kt = wbuf + (bb % kAttNBuf) * L::BATCH;
+            const unsigned char* vt = kt + kAttNB * RB;
+            const int rbase = a0 + bb * kAttNB;
+            const int rows_in = min(kAttNB, a1 - rbase);
+            // logits of the batch: two groups of 4 rows, a butterfly each
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = zp[(e * HG + h) * kTile + r];
-                z = (((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]))) * scale;
-                if (gr >= d.S && gr < d.S + T) zrow[(int64_t)(gr - d.S) * HG + h] = z;
+            for (int grp = 0; grp < kAttNB / 4; ++grp) {
+                float v[NV];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int rr = 4 * grp + r;
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (rr < rows_in) {
+                        if (BF16) {
+                            const uint2 w = *reinterpret_cast<const uint2*>(kt + rr * RB + 8 * lane);
+                            x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
+                        } else {
+                            const float4 w = *reinterpret_cast<const float4*>(kt + rr * RB + 16 * lane);
+                            x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
+                        }
+                    }
+#pragma unroll
+                    for (int h = 0; h < HG; ++h)
+                        v[r * HG + h] =
+                            fmaf(qv[h][3], x[3], fmaf(qv[h][2], x[2], fmaf(qv[h][1], x[1], qv[h][0] * x[0])));
+                }
+                const float z = transpose_reduce<NV>(v, lane) * 0.08838834764831845f;   // 1 / sqrt(128)
+                const int idx = tr_index<NV>(lane);
+                constexpr int lowmask = (NV >= 32) ? 0 : (32 / NV) - 1;
+                if ((lane & lowmask) == 0) {
+                    const int rr = 4 * grp + idx / HG;
+                    pz[rr * HG + idx % HG] = (rr < rows_in) ? z : -INFINITY;
+                    const int r = rbase + rr;
+                    if (rr < rows_in && r >= d.S && r < d.S + T) zrow[(int64_t)r * HG + idx % HG] = z;
+                }
             }
-            float mt = z;
+            __syncwarp();
+            // online softmax over the batch, then P . V
+            float pb[kAttNB][HG];
 #pragma unroll
-            for (int o = 16; o; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, o));
-            const float m_new = fmaxf(m_run, mt);
-            const float p = (gr < r1) ? __expf(z - m_new) : 0.f;
-            float ps = p;
+            for (int r = 0; r < kAttNB; ++r)
 #pragma unroll
-            for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(kFull, ps, o);
-            const float al = (m_run == -INFINITY) ? 0.f : __expf(m_run - m_new);
-            l_run = l_run * al + ps;
-            m_run = m_new;
-            pt[r * HG + h] = p;
-            if (lane == 0) alpha[h] = al;
-        }
-        __syncthreads();
-        // ---- PV: rows rg and rg + 16 of the tile (rows past the CTA's end
-        // hold stale shared memory and are skipped)
-        {
-            const int nvalid = min(kTile, r1 - (r0 + tile * kTile));
-            float al[HG];
+                for (int h = 0; h < HG; ++h) pb[r][h] = pz[r * HG + h];
 #pragma unroll
-            for (int h = 0; h < HG; ++h) al[h] = alpha[h];
+            for (int h = 0; h < HG; ++h) {
+                float mb = pb[0][h];
 #pragma unroll
-            for (int h = 0; h < HG; ++h)
+                for (int r = 1; r < kAttNB; ++r) mb = fmaxf(mb, pb[r][h]);
+                const float m_new = fmaxf(m_run[h], mb);
+                const float sc = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
+                l_run[h] *= sc;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[h][j] *= al[h];
+                for (int e = 0; e < 4; ++e) acc[h][e] *= sc;
+                m_run[h] = m_new;
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int r = rg + 16 * rr;
-                if (r >= nvalid) continue;
-                const unsigned char* vrow = Vs + (buf * kTile + r) * L::RB;
-                float vv[8];
+                for (int r = 0; r < kAttNB; ++r) {
+                    pb[r][h] = (pb[r][h] == -INFINITY) ? 0.f : __expf(pb[r][h] - m_new);
+                    l_run[h] += pb[r][h];
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kAttNB; ++r) {
+                if (r >= rows_in) break;
+                float x[4];
                 if (BF16) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(vrow + swz(r, c8) * 16);
-                    vv[0] = bf_lo(w.x); vv[1] = bf_hi(w.x); vv[2] = bf_lo(w.y); vv[3] = bf_hi(w.y);
-                    vv[4] = bf_lo(w.z); vv[5] = bf_hi(w.z); vv[6] = bf_lo(w.w); vv[7] = bf_hi(w.w);
+                    const uint2 w = *reinterpret_cast<const uint2*>(vt + r * RB + 8 * lane);
+                    x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
                 } else {
-                    const float4 w0 = *reinterpret_cast<const float4*>(vrow + swz(r, 2 * c8) * 16);
-                    const float4 w1 = *reinterpret_cast<const float4*>(vrow + swz(r, 2 * c8 + 1) * 16);
-                    vv[0] = w0.x; vv[1] = w0.y; vv[2] = w0.z; vv[3] = w0.w;
-                    vv[4] = w1.x; vv[5] = w1.y; vv[6] = w1.z; vv[7] = w1.w;
+                    const float4 w = *reinterpret_cast<const float4*>(vt + r * RB + 16 * lane);
+                    x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
                 }
 #pragma unroll
-                for (int h = 0; h < HG; ++h) {
-                    const float p = pt[r * HG + h];
+                for (int h = 0; h < HG; ++h)
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[h][j] = fmaf(p, vv[j], acc[h][j]);
-                }
+                    for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pb[r][h], x[e], acc[h][e]);
             }
+            __syncwarp();
+        }
+        cp_async_wait<0>();
+        __syncthreads();
+        // combine the warps: (m, l, acc) -> this slice's partial per head
+        float* red = reinterpret_cast<float*>(smem + L::off_buf);      // [warps][HG][RSTR]
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            float* rw = red + (warp * HG + h) * L::RSTR;
+            *reinterpret_cast<float4*>(rw + 4 * lane) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+            if (lane == 0) { rw[kD] = m_run[h]; rw[kD + 1] = l_run[h]; }
         }
         __syncthreads();
-    }
-
-    // ---- reduce the 16 row groups and write this CTA's partial
-    float* red = reinterpret_cast<float*>(smem + L::off_k);
-#pragma unroll
-    for (int h = 0; h < HG; ++h)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) red[(rg * HG + h) * kD + c8 * 8 + j] = acc[h][j];
-    __syncthreads();
-    float* part = s.part + ((int64_t)g * gridDim.x + split) * HG * (kD + 2);
-    for (int i = tid; i < HG * kD; i += kAttThreads) {
-        const int h = i / kD, dd = i % kD;
-        float o = 0.f;
-        for (int k = 0; k < 16; ++k) o += red[(k * HG + h) * kD + dd];
-        part[h * (kD + 2) + 2 + dd] = o;
-    }
-    if (warp < HG && lane == 0) {
-        part[warp * (kD + 2) + 0] = m_run;
-        part[warp * (kD + 2) + 1] = l_run;
-    }
-    // ---- last CTA of the graph merges
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned prev = atomicAdd(&s.counter[g], 1u);
-        s_last = (prev == gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    const int ns = gridDim.x;
-    const float* pg = s.part + (int64_t)g * ns * HG * (kD + 2);
-    float* ml = s.ml + (int64_t)g * HG * 2;
-    float* wgt = reinterpret_cast<float*>(smem + L::off_k);   // [ns][HG] merge weights
-    __shared__ float sM[8], sL[8];
-    if (warp < HG) {
-        const int h = warp;
-        float M = -INFINITY;
-        for (int k = lane; k < ns; k += 32) M = fmaxf(M, __ldcg(pg + ((int64_t)k * HG + h) * (kD + 2)));
-#pragma unroll
-        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-        float Lsum = 0.f;
-        for (int k = lane; k < ns; k += 32) {
-            const float mk = __ldcg(pg + ((int64_t)k * HG + h) * (kD + 2));
-            const float lk = __ldcg(pg + ((int64_t)k * HG + h) * (kD + 2) + 1);
-            const float wk = (mk == -INFINITY) ? 0.f : __expf(mk - M);
-            if ((int64_t)ns * HG * 4 <= (int64_t)(L::bytes - L::off_k)) wgt[k * HG + h] = wk;
-            Lsum += lk * wk;
-        }
-        // fixed-order sum over lanes
-#pragma unroll
-        for (int o = 16; o; o >>= 1) Lsum += __shfl_xor_sync(kFull, Lsum, o);
-        if (lane == 0) { sM[h] = M; sL[h] = Lsum; ml[h * 2] = M; ml[h * 2 + 1] = Lsum; }
-    }
-    __syncthreads();
-    const bool wgt_in_smem = (int64_t)ns * HG * 4 <= (int64_t)(L::bytes - L::off_k);
-    for (int i = tid; i < HG * kD; i += kAttThreads) {
-        const int h = i / kD, dd = i % kD;
-        float o = 0.f;
-        for (int k = 0; k < ns; ++k) {
-            float wk;
-            if (wgt_in_smem) wk = wgt[k * HG + h];
-            else {
-                const float mk = __ldcg(pg + ((int64_t)k * HG + h) * (kD + 2));
-                wk = (mk == -INFINITY) ? 0.f : __expf(mk - sM[h]);
+        float* po = s.part_o + ((int64_t)g * d.nCTA + k) * HG * kD;
+        float* pm = s.part_ml + ((int64_t)g * d.nCTA + k) * HG * 2;
+        for (int i = tid; i < HG * kD; i += NT) {
+            const int h = i / kD, dd = i % kD;
+            float M = -INFINITY;
+            for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, red[(w * HG + h) * L::RSTR + kD]);
+            float o = 0.f, l = 0.f;
+            for (int w = 0; w < kAttWarps; ++w) {
+                const float* rw = red + (w * HG + h) * L::RSTR;
+                const float f = (rw[kD] == -INFINITY) ? 0.f : __expf(rw[kD] - M);
+                o = fmaf(rw[dd], f, o);
+                l = fmaf(rw[kD + 1], f, l);
             }
-            if (wk != 0.f) o = fmaf(__ldcg(pg + ((int64_t)k * HG + h) * (kD + 2) + 2 + dd), wk, o);
+            po[i] = o;
+            if (dd == 0) { pm[h * 2] = M; pm[h * 2 + 1] = l; }
         }
-        out[((int64_t)b * d.Hq + h0 + h) * kD + dd] = o / sL[h];
+        // ---------------------------------------- last slice of the graph merges
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const unsigned prev = atomicAdd(&s.bar[g * 2 + 1], 1u);
+            sh_seg[3] = (prev == (unsigned)nc - 1);
+        }
+        __syncthreads();
+        if (!sh_seg[3]) continue;
+        __threadfence();
+        const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
+        const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
+        if (warp < HG) {   // exact softmax max and sum of the graph, per head
+            const int h = warp;
+            float M = -INFINITY;
+            for (int j = lane; j < nc; j += 32) M = fmaxf(M, __ldcg(pmg + ((int64_t)j * HG + h) * 2));
+#pragma unroll
+            for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+            float Ls = 0.f;
+            for (int j = lane; j < nc; j += 32) {
+                const float mj = __ldcg(pmg + ((int64_t)j * HG + h) * 2);
+                if (mj != -INFINITY) Ls += __ldcg(pmg + ((int64_t)j * HG + h) * 2 + 1) * __expf(mj - M);
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) Ls += __shfl_xor_sync(kFull, Ls, o);
+            if (lane == 0) { sM[h] = M; sL[h] = 1.f / Ls; }
+        }
+        __syncthreads();
+        for (int i = tid; i < HG * kD; i += NT) {
+            const int h = i / kD;
+            float o = 0.f;
+            for (int j0 = 0; j0 < nc; j0 += 8) {   // 8 slices' loads in flight at once
+                float mj[8], oj[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const bool ok = j0 + u < nc;
+                    mj[u] = ok ? __ldcg(pmg + ((int64_t)(j0 + u) * HG + h) * 2) : -INFINITY;
+                    oj[u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (mj[u] != -INFINITY) o = fmaf(oj[u], __expf(mj[u] - sM[h]), o);
+            }
+            out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o * sL[h];
+        }
+        // edges: top-kappa of w = sum_h exp(z - M_h) / L_h over the kept members
+        {
+            TopList<KM> tl;
+            tl.clear();
+            for (int j0 = tid; j0 < T; j0 += 8 * NT) {   // 8 rows' loads in flight at once
+                float zz[8][HG];
+                int tt[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int j = j0 + u * NT;
+                    const bool ok = j < T;
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) zz[u][h] = ok ? __ldcg(zrow + (int64_t)(d.S + j) * HG + h) : 0.f;
+                    tt[u] = ok ? __ldcg(rtok + j) : 0;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int j = j0 + u * NT;
+                    if (j >= T) break;
+                    float w = 0.f;
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) w += __expf(zz[u][h] - sM[h]) * sL[h];
+                    tl.insert(w, tt[u], j);
+                }
+            }
+            float* ew = reinterpret_cast<float*>(smem + L::off_buf);        // [warps][kMaxKappa]
+            int* et = reinterpret_cast<int*>(ew + kAttWarps * kMaxKappa);
+            int* ex = et + kAttWarps * kMaxKappa;
+            __syncthreads();    // the reduction buffer is free again
+            const int nw = warp_merge<KM>(tl, d.kappa, ew + warp * kMaxKappa, et + warp * kMaxKappa,
+                                          ex + warp * kMaxKappa);
+            if (lane == 0) sidx[warp] = nw;
+            __syncthreads();
+            if (warp == 0) {
+                TopList<KM> t2;
+                t2.clear();
+                for (int w = 0; w < kAttWarps; ++w)
+                    for (int e = lane; e < sidx[w]; e += 32)
+                        t2.insert(ew[w * kMaxKappa + e], et[w * kMaxKappa + e], ex[w * kMaxKappa + e]);
+                float* gw = s.e_w + (int64_t)g * d.kappa;
+                int* gt = s.e_tok + (int64_t)g * d.kappa;
+                int* gx = s.e_comm + (int64_t)g * d.kappa;   // row index first, community below
+                const int ne = warp_merge<KM>(t2, d.kappa, gw, gt, gx);
+                __syncwarp();
+                if (lane < ne) gx[lane] = s.rcomm[(int64_t)g * d.NM + gx[lane]];
+                if (lane == 0) {
+                    s.meta[(int64_t)g * M_COUNT + M_NEDGE] = ne;
+                    s.bar[g * 2 + 1] = 0u;
+                }
+            }
+        }
     }
-    if (tid == 0) s.counter[g] = 0u;
 }
 
 // --------------------------------------------------------------- k_assign
-template <bool BF16, int HG>
-__global__ void __launch_bounds__(kAsgThreads) k_assign(DevState s, Dims d, const void* __restrict__ K,
-                                                       int n)
+template <bool BF16>
+__global__ void __launch_bounds__(kAsgThreads) k_assign(DevState s, Dims d, const void* __restrict__ K, int n)
 {
     if (*(volatile int*)s.err) return;
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ float redw[32];
-    __shared__ int redt[32], redi[32];
-    __shared__ int e_tok[kMaxKappa], e_idx[kMaxKappa];
+    __shared__ int e_c[kMaxKappa];
     __shared__ float e_w[kMaxKappa];
-    __shared__ int s_c, s_ok, s_off, s_size;
-
+    __shared__ int s_c, s_ok, s_off, s_size, s_oldoff, s_E;
     const int g = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     int b, h0, kvh;
     graph_heads(d, g, b, h0, kvh);
-    const int32_t* meta = s.meta + (int64_t)g * M_COUNT;
-    const int T = meta[M_T];
     const int t = n - 1;
-    const float* zrow = s.zrow + (int64_t)g * d.NM * HG;
-    const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
-    const int32_t* rcomm = s.rcomm + (int64_t)g * d.NM;
-    float M[HG], invL[HG];
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-        M[h] = s.ml[((int64_t)g * HG + h) * 2];
-        invL[h] = 1.f / s.ml[((int64_t)g * HG + h) * 2 + 1];
+    // the new token's key (independent of the vote) and the step's edges
+    const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + t) * kD;
+    const double kv = (double)elem<BF16>(K, krow + tid);
+    const int E = s.meta[(int64_t)g * M_COUNT + M_NEDGE];
+    if (tid < E) {
+        e_c[tid] = s.e_comm[(int64_t)g * d.kappa + tid];
+        e_w[tid] = s.e_w[(int64_t)g * d.kappa + tid];
     }
-    // edge weights w_j = sum_h p_hj of the kept members (cached in shared
-    // memory when they fit, else recomputed per round)
-    float* ws = reinterpret_cast<float*>(smem);
-    int* ts = reinterpret_cast<int*>(smem) + kSortCap * 4;
-    const bool cached = (T <= kSortCap * 4);
-    auto weight = [&](int i) -> float {
-        float acc = 0.f;
-#pragma unroll
-        for (int h = 0; h < HG; ++h) acc += expf(zrow[(int64_t)i * HG + h] - M[h]) * invL[h];
-        return acc;
-    };
-    if (cached) {
-        for (int i = tid; i < T; i += kAsgThreads) { ws[i] = weight(i); ts[i] = rtok[i]; }
-        __syncthreads();
-    }
-    // ---- top-kappa by (w desc, token asc): kappa rounds of block argmax
-    // below the previous winner's key
-    const int E = min(d.kappa, T);
-    float pw = INFINITY;
-    int ptk = -1;
-    for (int k = 0; k < E; ++k) {
-        float bw = -INFINITY;
-        int bt = 0x7fffffff, bi = -1;
-        for (int i = tid; i < T; i += kAsgThreads) {
-            const float w = cached ? ws[i] : weight(i);
-            const int tk = cached ? ts[i] : rtok[i];
-            const bool below = (w < pw) || (w == pw && tk > ptk);
-            const bool better = (w > bw) || (w == bw && tk < bt);
-            if (below && better) { bw = w; bt = tk; bi = i; }
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            const float ow = __shfl_xor_sync(kFull, bw, o);
-            const int ot = __shfl_xor_sync(kFull, bt, o);
-            const int oi = __shfl_xor_sync(kFull, bi, o);
-            if (ow > bw || (ow == bw && ot < bt)) { bw = ow; bt = ot; bi = oi; }
-        }
-        if (lane == 0) { redw[warp] = bw; redt[warp] = bt; redi[warp] = bi; }
-        __syncthreads();
-        if (warp == 0) {
-            const int nw = kAsgThreads / 32;
-            bw = (lane < nw) ? redw[lane] : -INFINITY;
-            bt = (lane < nw) ? redt[lane] : 0x7fffffff;
-            bi = (lane < nw) ? redi[lane] : -1;
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                const float ow = __shfl_xor_sync(kFull, bw, o);
-                const int ot = __shfl_xor_sync(kFull, bt, o);
-                const int oi = __shfl_xor_sync(kFull, bi, o);
-                if (ow > bw || (ow == bw && ot < bt)) { bw = ow; bt = ot; bi = oi; }
-            }
-            if (lane == 0) { e_w[k] = bw; e_tok[k] = bt; e_idx[k] = bi; }
-        }
-        __syncthreads();
-        pw = e_w[k];
-        ptk = e_tok[k];
-    }
-    // ---- vote and capacity check (thread 0)
-    const int32_t* csz = s.csize + (int64_t)g * d.Nc;
+    __syncthreads();
+    int32_t* csz = s.csize + (int64_t)g * d.Nc;
     int32_t* coff = s.coff + (int64_t)g * d.Nc;
     int32_t* ccap = s.ccap + (int64_t)g * d.Nc;
     if (tid == 0) {
+        // weighted plurality in rank order, ties to the lower id
         int ids[kMaxKappa];
         double v[kMaxKappa];
         int nd = 0;
         for (int e = 0; e < E; ++e) {
-            const int c = rcomm[e_idx[e]];
             int k = 0;
-            while (k < nd && ids[k] != c) ++k;
-            if (k == nd) { ids[nd] = c; v[nd] = 0.0; ++nd; }
+            while (k < nd && ids[k] != e_c[e]) ++k;
+            if (k == nd) { ids[nd] = e_c[e]; v[nd] = 0.0; ++nd; }
             v[k] += (double)e_w[e];
         }
         int best = -1;
         for (int k = 0; k < nd; ++k)
             if (best < 0 || v[k] > v[best] || (v[k] == v[best] && ids[k] < ids[best])) best = k;
         const int c = (best < 0) ? 0 : ids[best];
-        const int size = csz[c], cp = ccap[c];
-        int ok = 1, off = coff[c];
-        if (size == cp) {
+        const int size = csz[c], cp = ccap[c], off0 = coff[c], top = s.pool_top[g];
+        int ok = 1, off = off0;
+        if (size == cp) {   // segment full: move it to the pool top with twice the room
             const int ncap = max(16, 2 * cp);
-            const int top = s.pool_top[g];
             if ((int64_t)top + ncap > d.P) ok = 0;
             else { s.pool_top[g] = top + ncap; off = top; }
         }
-        s_c = c; s_ok = ok; s_off = off; s_size = size;
+        s_c = c; s_ok = ok; s_off = off; s_size = size; s_oldoff = off0; s_E = E;
         if (!ok) set_error(s.err, CKV_ERR_CAPACITY);
     }
     __syncthreads();
     if (!s_ok) return;
-    const int c = s_c, size = s_size, off = s_off;
+    const int c = s_c, size = s_size, off = s_off, old_off = s_oldoff;
     int32_t* pool = s.pool + (int64_t)g * d.P;
-    const int old_off = coff[c];
-    if (off != old_off) {   // relocate the full segment
+    if (off != old_off)
         for (int i = tid; i < size; i += kAsgThreads) pool[off + i] = pool[old_off + i];
-    }
     // running-mean update of the assigned centroid, double math rounded once
-    const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + t) * kD;
     float* mu = s.mu + ((int64_t)g * d.Nc + c) * kD;
-    const double m1 = (double)(size + 1);
-    for (int i = tid; i < kD; i += kAsgThreads) {
-        const double mv = (double)mu[i];
-        const double kv = (double)elem<BF16>(K, krow + i);
-        mu[i] = __double2float_rn(__dadd_rn(mv, __ddiv_rn(__dsub_rn(kv, mv), m1)));
-    }
+    const double mv = (double)mu[tid];
+    mu[tid] = __double2float_rn(__dadd_rn(mv, __ddiv_rn(__dsub_rn(kv, mv), (double)(size + 1))));
     __syncthreads();
     if (tid == 0) {
         if (off != old_off) { coff[c] = off; ccap[c] = max(16, 2 * ccap[c]); }
         pool[off + size] = t;
-        s.csize[(int64_t)g * d.Nc + c] = size + 1;
+        csz[c] = size + 1;
         s.tok_comm[(int64_t)g * d.NM + t] = c;
-        int32_t* m = s.meta + (int64_t)g * M_COUNT;
-        m[M_NEDGE] = E;
-        m[M_ASSIGNED] = c;
-        const int64_t row = (int64_t)g * (d.NM - d.n_init) + (t - d.n_init);
-        s.edge_deg[row] = E;
-        for (int e = 0; e < E; ++e) {
-            s.edge_col[row * d.kappa + e] = e_tok[e];
-            s.edge_w[row * d.kappa + e] = e_w[e];
-            s.dbg_edges[(int64_t)g * d.kappa + e] = e_tok[e];
-            s.dbg_w[(int64_t)g * d.kappa + e] = e_w[e];
-        }
+        s.meta[(int64_t)g * M_COUNT + M_ASSIGNED] = c;
     }
-}
-
-template <typename F>
-cudaError_t dispatch_hg(int hg, F&& f)
-{
-    switch (hg) {
-        case 1: return f(std::integral_constant<int, 1>{});
-        case 2: return f(std::integral_constant<int, 2>{});
-        case 4: return f(std::integral_constant<int, 4>{});
-        case 8: return f(std::integral_constant<int, 8>{});
-        default: return cudaErrorInvalidValue;
+    const int64_t row = (int64_t)g * (d.NM - d.n_init) + (t - d.n_init);
+    if (tid == 0) s.edge_deg[row] = s_E;
+    if (tid < s_E) {
+        s.edge_col[row * d.kappa + tid] = s.e_tok[(int64_t)g * d.kappa + tid];
+        s.edge_w[row * d.kappa + tid] = e_w[tid];
     }
 }
 
@@ -878,67 +1041,128 @@ __global__ void k_append(const uint32_t* __restrict__ knew, const uint32_t* __re
     }
 }
 
+template <typename F>
+cudaError_t dispatch_hg(int hg, F&& f)
+{
+    switch (hg) {
+        case 1: return f(std::integral_constant<int, 1>{});
+        case 2: return f(std::integral_constant<int, 2>{});
+        case 4: return f(std::integral_constant<int, 4>{});
+        case 8: return f(std::integral_constant<int, 8>{});
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <bool BF16, int HG>
+void* attend_fn(int kappa)
+{
+    if (kappa <= 8) return reinterpret_cast<void*>(k_attend<BF16, HG, 8>);
+    if (kappa <= 16) return reinterpret_cast<void*>(k_attend<BF16, HG, 16>);
+    return reinterpret_cast<void*>(k_attend<BF16, HG, 32>);
+}
+
 }  // namespace
 
-size_t select_smem_bytes() { return sizeof(SelShared); }
-
-cudaError_t launch_append_rows(const Dims& d, const void* knew, const void* vnew, void* K, void* V,
-                               int row, cudaStream_t st)
+size_t select_smem_bytes(int n_comm)
 {
-    const int words = kD * (d.bf16 ? 2 : 4) / 4;
-    k_append<<<d.B * d.Hkv, 64, 0, st>>>(static_cast<const uint32_t*>(knew), static_cast<const uint32_t*>(vnew),
-                                         static_cast<uint32_t*>(K), static_cast<uint32_t*>(V), d.NM, row, words);
-    return cudaGetLastError();
+    return (size_t)4 * round4(n_comm + 1) + (size_t)4 * round4(n_comm) + 4 * sel_region3(n_comm) + (size_t)n_comm + 16;
 }
 
 cudaError_t launch_score(const DevState& s, const Dims& d, const void* q, cudaStream_t st)
 {
-    dim3 grid((d.n_comm + 255) / 256, d.G);
-    if (d.bf16) k_score<true><<<grid, 256, 0, st>>>(s, d, q);
-    else k_score<false><<<grid, 256, 0, st>>>(s, d, q);
+    const int units = d.G * ((d.n_comm + 31) / 32);
+    const int grid = units < d.nSM ? units : d.nSM;   // persistent: one CTA per SM
+    const size_t smem = sizeof(ScoreSmem);
+    if (d.bf16) k_score<true><<<grid, kScoreThreads, smem, st>>>(s, d, q);
+    else k_score<false><<<grid, kScoreThreads, smem, st>>>(s, d, q);
     return cudaGetLastError();
 }
 
-cudaError_t launch_select(const DevState& s, const Dims& d, int n, cudaStream_t st)
+cudaError_t launch_select(const DevState& s, const Dims& d, cudaStream_t st)
 {
-    k_select<<<d.G, kSelThreads, 0, st>>>(s, d, n);
+    k_select<<<d.G, kSelThreads, select_smem_bytes(d.n_comm), st>>>(s, d);
     return cudaGetLastError();
 }
 
-cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const void* K,
-                          const void* V, int n, float* out, cudaStream_t st)
+cudaError_t prepare_kernels(const Dims& d)
+{
+    // shared-memory limits are set once per device, before any launch (and
+    // so outside any stream capture)
+    cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)select_smem_bytes(kMaxCommunities));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_score<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScoreSmem));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_score<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScoreSmem));
+    if (e != cudaSuccess) return e;
+    return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
+        constexpr int HG = decltype(hgc)::value;
+        void* fn = d.bf16 ? attend_fn<true, HG>(d.kappa) : attend_fn<false, HG>(d.kappa);
+        const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
+        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    });
+}
+
+int attend_grid(const Dims& d, int sms)
+{
+    int occ = 0;
+    cudaError_t e = prepare_kernels(d);
+    if (e == cudaSuccess)
+        e = dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
+            constexpr int HG = decltype(hgc)::value;
+            void* fn = d.bf16 ? attend_fn<true, HG>(d.kappa) : attend_fn<false, HG>(d.kappa);
+            const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
+            return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kAttWarps * 32, bytes);
+        });
+    if (e != cudaSuccess || occ < 1) return 0;
+    return occ * sms;
+}
+
+cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const void* K, const void* V, int n,
+                          float* out, cudaStream_t st)
 {
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
-        dim3 grid(d.splits, d.G);
-        if (d.bf16) {
-            using L = AttLayout<true, HG>;
-            auto kern = k_attend<true, HG>;
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::bytes);
-            if (e != cudaSuccess) return e;
-            kern<<<grid, kAttThreads, L::bytes, st>>>(s, d, q, K, V, n, out);
-        } else {
-            using L = AttLayout<false, HG>;
-            auto kern = k_attend<false, HG>;
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::bytes);
-            if (e != cudaSuccess) return e;
-            kern<<<grid, kAttThreads, L::bytes, st>>>(s, d, q, K, V, n, out);
-        }
-        return cudaGetLastError();
+        void* fn = d.bf16 ? attend_fn<true, HG>(d.kappa) : attend_fn<false, HG>(d.kappa);
+        const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
+        // the slices of a graph wait for one another: all CTAs must be
+        // co-resident, which a cooperative launch guarantees (or refuses)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(d.nCTA);
+        cfg.blockDim = dim3(kAttWarps * 32);
+        cfg.dynamicSmemBytes = bytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        DevState ss = s;
+        Dims dd = d;
+        const void* qq = q;
+        const void* kk = K;
+        const void* vv = V;
+        int nn = n;
+        float* oo = out;
+        void* args[] = {&ss, &dd, &qq, &kk, &vv, &nn, &oo};
+        return cudaLaunchKernelExC(&cfg, fn, args);
     });
 }
 
 cudaError_t launch_assign(const DevState& s, const Dims& d, const void* K, int n, cudaStream_t st)
 {
-    const size_t smem = (size_t)kSortCap * 4 * 8;   // w (float) + token (int) of up to 4096 rows
-    return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
-        constexpr int HG = decltype(hgc)::value;
-        auto kern = d.bf16 ? k_assign<true, HG> : k_assign<false, HG>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<d.G, kAsgThreads, smem, st>>>(s, d, K, n);
-        return cudaGetLastError();
-    });
+    if (d.bf16) k_assign<true><<<d.G, kAsgThreads, 0, st>>>(s, d, K, n);
+    else k_assign<false><<<d.G, kAsgThreads, 0, st>>>(s, d, K, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_append_rows(const Dims& d, const void* knew, const void* vnew, void* K, void* V, int row,
+                               cudaStream_t st)
+{
+    const int words = kD * (d.bf16 ? 2 : 4) / 4;
+    k_append<<<d.B * d.Hkv, 64, 0, st>>>(static_cast<const uint32_t*>(knew), static_cast<const uint32_t*>(vnew),
+                                         static_cast<uint32_t*>(K), static_cast<uint32_t*>(V), d.NM, row, words);
+    return cudaGetLastError();
 }
 
 }  // namespace ckv
