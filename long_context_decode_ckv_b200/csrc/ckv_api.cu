@@ -179,9 +179,14 @@ cudaError_t prof_mark(ckv_ctx* x, int slot, cudaStream_t st)
     cudaError_t r = next_event(x, &e);
     if (r != cudaSuccess) return r;
     x->ev_steps.back()[slot] = e;
-    // external record: under stream capture it becomes an event-record node
-    // whose timestamps stay usable for cudaEventElapsedTime
-    return cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    // under stream capture an external record becomes an event-record node
+    // whose timestamps stay usable for cudaEventElapsedTime; the flag is
+    // only accepted while the stream is capturing
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    r = cudaStreamIsCapturing(st, &cap);
+    if (r != cudaSuccess) return r;
+    if (cap == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    return cudaEventRecord(e, st);
 }
 
 }  // namespace
@@ -276,6 +281,9 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(part_ml, G * KC * HG * 2);
     ALLOC(part_o, G * KC * HG * ckv::kD);
     ALLOC(bar, G * 2);
+    ALLOC(cand_w, G * KC * ckv::kAttWarps * kap);
+    ALLOC(cand_t, G * KC * ckv::kAttWarps * kap);
+    ALLOC(cand_x, G * KC * ckv::kAttWarps * kap);
     ALLOC(e_tok, G * kap);
     ALLOC(e_w, G * kap);
     ALLOC(e_comm, G * kap);

@@ -17,7 +17,9 @@
 //   zrow      float [G][NM][HG]    logits of the kept members (for the edges)
 //   part_ml   float [G][KC][HG][2] per-CTA softmax max and sum per head
 //   part_o    float [G][KC][HG][D] per-CTA P.V per head, relative to its max
-//   bar       uint  [G][2]         arrivals of a graph's CTAs (slot 1)
+//   bar       uint  [G][2]         arrivals of a graph's CTAs: partials published
+//                                  (slot 0), edge candidates published (slot 1)
+//   cand_*    [G][KC][W][kappa]    per-warp edge candidates (W = kAttWarps)
 //   e_*       [G][kappa]           the step's edges (rank order) for the update
 #pragma once
 
@@ -32,6 +34,7 @@ constexpr int kD = 128;          // head_dim the kernels are written for
 constexpr int kMaxKappa = 32;
 constexpr int kSelBins = 2048;   // bucket count of the selection passes
 constexpr int kSortCap = 1024;   // candidates ranked exactly in one CTA
+constexpr int kAttWarps = 8;     // warps of an attention CTA
 
 // meta slots per graph
 enum { M_C = 0, M_T = 1, M_ROWS = 2, M_NEDGE = 3, M_ASSIGNED = 4, M_COUNT = 8 };
@@ -57,6 +60,9 @@ struct DevState {
     float* part_ml;
     float* part_o;
     unsigned int* bar;
+    float* cand_w;           // per-warp edge candidates of each slice
+    int32_t* cand_t;
+    int32_t* cand_x;
     int32_t* e_tok;
     float* e_w;
     int32_t* e_comm;

@@ -16,10 +16,12 @@
 //             score bits, then of the id) and an exact rank of the last
 //             <= 1024 candidates; writes the kept list and the kept rows.
 //   k_attend  one CTA per SM, each a slice of one graph's rows; every warp
-//             streams its own run of rows (K and V together, 16-byte
-//             cp.async) with an online softmax; the last CTA of a graph
-//             merges the (m, l, o) partials exactly and ranks the kept
-//             members' edge weights from the logits spilled to L2.
+//             gathers its own run of K and V rows (16-byte cp.async) and,
+//             for bf16, runs both contractions on the tensor cores
+//             (mma.sync) with an online softmax; once a graph's slices have
+//             published their (m, l, o) partials, each merges its share of
+//             the output and ranks its own kept members' edge weights, and
+//             the last one merges the candidate lists.
 //   k_assign  one CTA per graph: vote, capacity check, running-mean
 //             update, member append, edge row.
 #include <cuda_runtime.h>
@@ -463,44 +465,104 @@ __global__ void __launch_bounds__(kSelThreads) k_select(DevState s, Dims d)
 }
 
 // --------------------------------------------------------------- k_attend
-// Each warp owns a contiguous run of a graph slice's rows and streams them
-// through its own 3-buffer shared-memory pipeline: 8 rows per batch, K and
-// V of a row fetched together with 16-byte cp.async (the LSU gather path;
-// one bulk TMA copy per 256-byte row is far slower).  Per 4-row group the
-// lane's partial dots are reduced by a butterfly transpose; the warp keeps
-// an online softmax (running max, sum, P.V) per head and spills the logits
-// of the kept members to L2 for the edges.  The CTA combines its warps into
-// one (m, l, o) partial per head; the last CTA of a graph merges the
-// partials exactly, then ranks all kept members' edge weights.
-constexpr int kAttWarps = 16;
+// One CTA per SM, each a slice of one graph's rows (or whole graphs when
+// there are more graphs than CTAs).  Every warp owns a contiguous run of the
+// slice's rows and streams it through its own 3-batch shared-memory
+// pipeline, K and V rows of a batch gathered together with 16-byte cp.async
+// (the LSU gather path; one bulk copy per 256-byte row is far slower).
+//
+// bf16 caches: a batch is 16 rows and both contractions run on the tensor
+// cores (mma.sync m16n8k16, fp32 accumulate): S^T = K_tile . Q^T with the
+// graph's heads as the 8 columns, then O^T += V_tile^T . P^T with P split
+// into a bf16 high and low part (two MMAs) so the weights keep ~16 bits.
+// Rows sit in shared memory with their 16-byte chunks XOR-swizzled by
+// (row mod 8), which makes every ldmatrix conflict-free.  fp32 caches:
+// 4-row batches on the CUDA cores (partial dots reduced by a butterfly).
+//
+// Each warp keeps an online softmax (running max and sum per head) and
+// spills the kept members' logits to L2.  The CTA combines its warps into
+// one (m, l, o) partial per head and publishes it; once all slices of the
+// graph have published (a per-graph arrival counter: the grid is
+// co-resident by cooperative launch, and the wait is bounded), every slice
+// derives the graph's exact softmax statistics, writes its share of the
+// output and ranks its own kept members' edge weights w_j; the last slice
+// to finish merges the slices' candidate lists into the top-kappa edges.
 constexpr int kAttNBuf = 3;        // batches per warp pipeline
 
 template <bool BF16, int HG>
 struct AttLayout {
-    static constexpr int NB = BF16 ? 8 : 4;                      // rows per warp batch
+    static constexpr int NB = BF16 ? 16 : 4;                     // rows per warp batch
     static constexpr int RB = kD * (BF16 ? 2 : 4);               // bytes per K or V row
-    static constexpr int NCH = RB / 16;                          // 16-byte chunks per row
-    static constexpr int BATCH = NB * 2 * RB;                    // K and V of one batch
+    static constexpr int BATCH = NB * 2 * RB;                    // K rows, then V rows
     static constexpr int WBUF = kAttNBuf * BATCH;                // one warp's pipeline
-    static constexpr int off_buf = 0;
     static constexpr int TOKW = 64;                              // row tokens a warp keeps at once
-    static constexpr int off_pz = off_buf + kAttWarps * WBUF;    // [warps][NB*HG] z / p exchange
-    static constexpr int off_tokw = off_pz + kAttWarps * NB * HG * 4;  // [warps][TOKW]
+    static constexpr int off_buf = 0;
+    static constexpr int off_pz = off_buf + kAttWarps * WBUF;    // fp32: [warps][NB*HG] z / p exchange
+    static constexpr int off_tokw = off_pz + (BF16 ? 0 : kAttWarps * NB * HG * 4);   // [warps][TOKW]
     static constexpr int off_misc = off_tokw + kAttWarps * TOKW * 4;
-    static constexpr int bytes = off_misc + 512;
+    static constexpr int bytes = off_misc + 256;
     // end-of-slice reduction [warps][HG][RSTR] reuses the pipelines; a row is
-    // acc[0..D), m, l, padded to a multiple of 16 bytes for float4 stores
+    // acc[0..D), m, l, padded to a multiple of 16 bytes for float4 access
     static constexpr int RSTR = kD + 4;
     static_assert(kAttWarps * HG * RSTR * 4 <= kAttWarps * WBUF, "reduction must fit");
+    static_assert(kAttWarps * kMaxKappa * 12 <= kAttWarps * WBUF, "edge lists must fit");
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
+// 16 bytes, or 16 zero bytes when !valid (nothing is read then)
+__device__ __forceinline__ void cp_async16z(uint32_t dst, const void* src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// four 8x8 b16 matrices; lanes 8i..8i+7 give the row addresses of matrix i
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// c += a . b  (16x16 bf16, row-major) x (16x8 bf16, column-major), fp32
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};\n"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// transpose of the warp's 8x8 b16 matrix held in fragment layout
+__device__ __forceinline__ uint32_t movtrans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+// (lo, hi) -> bf16 pair, round to nearest even; lo in the low half
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
 // Butterfly transpose-reduce of NV values per lane (NV a power of two
 // <= 32): afterwards every lane holds the warp-wide sum of value index
@@ -569,8 +631,8 @@ struct TopList {
 };
 
 // Merge the 32 lanes' lists: the warp's top kappa (kappa <= KM) in rank
-// order, written by lane 0; returns how many (entries with w = -inf are
-// empty).
+// order, written by lane 0 with w = -inf in the unused tail; returns how
+// many are real.
 template <int KM>
 __device__ __forceinline__ int warp_merge(TopList<KM>& L, int kappa, float* ow, int* ot, int* ox)
 {
@@ -592,7 +654,305 @@ __device__ __forceinline__ int warp_merge(TopList<KM>& L, int kappa, float* ow, 
         if (lane == bl) L.pop();
         ++nout;
     }
+    for (int k = nout + lane; k < kappa; k += 32) { ow[k] = -INFINITY; ot[k] = 0x7fffffff; ox[k] = -1; }
     return nout;
+}
+
+// Rows of one warp: [a0, a1) in the graph's row numbering (sinks, kept
+// members, the new token).
+struct WarpRows {
+    const char* Kb;          // this (batch, KV head)'s K cache
+    const char* Vb;
+    const int32_t* rtok;     // token of each kept-member row
+    float* zrow;             // logits of the kept members, [row][HG]
+    int a0, a1, S, T, R, t_new;
+};
+
+__device__ __forceinline__ int row_token(const WarpRows& a, int r)
+{
+    if (r < a.S) return r;
+    if (r == a.R - 1) return a.t_new;
+    return a.rtok[r - a.S];
+}
+
+// tokens of rows r .. r + TOKW - 1 of this warp into its smem window
+template <int TOKW>
+__device__ __forceinline__ void tokens_from(const WarpRows& a, int r, int* tokw, int lane)
+{
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < TOKW / 32; ++i) {
+        const int rr = r + 32 * i + lane;
+        tokw[32 * i + lane] = (rr < a.a1) ? row_token(a, rr) : 0;
+    }
+    __syncwarp();
+}
+
+// bf16 rows on the tensor cores; leaves the warp's (acc, m, l) per head in
+// red[warp][h][RSTR] (after a CTA barrier, as red overlays the pipelines)
+template <int HG>
+__device__ __forceinline__ void warp_rows_mma(const WarpRows& a, const uint32_t* __restrict__ q2,
+                                              unsigned char* wbuf, int* tokw, float* red)
+{
+    using L = AttLayout<true, HG>;
+    constexpr int NB = L::NB;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    // B operand Q^T (dims x heads): lane holds head gid, dims 16ks + 2tig (+1, +8, +9)
+    uint32_t qf[8][2];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        qf[ks][0] = (gid < HG) ? q2[(gid * kD + 16 * ks + 2 * tig) / 2] : 0u;
+        qf[ks][1] = (gid < HG) ? q2[(gid * kD + 16 * ks + 2 * tig + 8) / 2] : 0u;
+    }
+    const int nb = (a.a1 - a.a0 + NB - 1) / NB;
+    int tok_base = -L::TOKW;
+    auto issue = [&](int bb) {
+        if (bb < nb) {
+            const uint32_t dst = smem_u32(wbuf + (bb % kAttNBuf) * L::BATCH);
+            const int rbase = a.a0 + bb * NB;
+            if (rbase + NB > tok_base + L::TOKW) {
+                tokens_from<L::TOKW>(a, rbase, tokw, lane);
+                tok_base = rbase;
+            }
+            const int ch = lane & 15;
+#pragma unroll
+            for (int i = 0; i < NB / 2; ++i) {
+                const int row = 2 * i + (lane >> 4);
+                const bool ok = rbase + row < a.a1;
+                const int64_t src = ok ? (int64_t)tokw[rbase - tok_base + row] * 256 + ch * 16 : 0;
+                const uint32_t so = row * 256 + ((ch ^ (row & 7)) << 4);
+                cp_async16z(dst + so, a.Kb + src, ok);
+                cp_async16z(dst + NB * 256 + so, a.Vb + src, ok);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    float acc[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+    // ldmatrix row addresses of this lane: K tiles (A of S^T) and V tiles (A of O^T, transposed)
+    const int krow = (lane & 7) + ((lane >> 3) & 1) * 8, khi = lane >> 4;
+    const int vrow = (lane & 7) + (lane >> 4) * 8, vhi = (lane >> 3) & 1;
+    const bool h0ok = 2 * tig < HG, h1ok = 2 * tig + 1 < HG;
+
+    issue(0);
+    issue(1);
+    for (int bb = 0; bb < nb; ++bb) {
+        issue(bb + 2);
+        cp_async_wait<kAttNBuf - 1>();
+        __syncwarp();
+        const uint32_t kt = smem_u32(wbuf + (bb % kAttNBuf) * L::BATCH), vt = kt + NB * 256;
+        const int rbase = a.a0 + bb * NB;
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t fa[4];
+            ldsm4(kt + krow * 256 + (((2 * ks + khi) ^ (krow & 7)) << 4), fa);
+            mma_bf16(sc, fa, qf[ks][0], qf[ks][1]);
+        }
+        // logits of rows gid and gid + 8, heads 2tig and 2tig + 1
+        const int ra = rbase + gid, rb = ra + 8;
+        const bool va = ra < a.a1, vb = rb < a.a1;
+        const float kScale = 0.08838834764831845f;   // 1 / sqrt(128)
+        float z[4];
+        z[0] = (va && h0ok) ? sc[0] * kScale : -INFINITY;
+        z[1] = (va && h1ok) ? sc[1] * kScale : -INFINITY;
+        z[2] = (vb && h0ok) ? sc[2] * kScale : -INFINITY;
+        z[3] = (vb && h1ok) ? sc[3] * kScale : -INFINITY;
+        if (h0ok) {   // the kept members' logits, for the edge ranking
+            const bool ma = va && ra >= a.S && ra < a.S + a.T, mb = vb && rb >= a.S && rb < a.S + a.T;
+            if (HG == 1) {
+                if (ma) a.zrow[ra] = z[0];
+                if (mb) a.zrow[rb] = z[2];
+            } else {
+                if (ma) *reinterpret_cast<float2*>(a.zrow + (int64_t)ra * HG + 2 * tig) = make_float2(z[0], z[1]);
+                if (mb) *reinterpret_cast<float2*>(a.zrow + (int64_t)rb * HG + 2 * tig) = make_float2(z[2], z[3]);
+            }
+        }
+        // online softmax per head; the max is shared by the 8 lanes of a head column
+        float p[4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float t = fmaxf(z[j], z[2 + j]);
+            t = fmaxf(t, __shfl_xor_sync(kFull, t, 4));
+            t = fmaxf(t, __shfl_xor_sync(kFull, t, 8));
+            t = fmaxf(t, __shfl_xor_sync(kFull, t, 16));
+            const float mn = fmaxf(m[j], t);
+            const float al = (m[j] == -INFINITY) ? 0.f : __expf(m[j] - mn);
+            p[j] = (z[j] == -INFINITY) ? 0.f : __expf(z[j] - mn);
+            p[2 + j] = (z[2 + j] == -INFINITY) ? 0.f : __expf(z[2 + j] - mn);
+            l[j] = fmaf(l[j], al, p[j] + p[2 + j]);
+            m[j] = mn;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                acc[mt][j] *= al;
+                acc[mt][2 + j] *= al;
+            }
+        }
+        // P^T as the B operand, split into bf16 high + low parts
+        const uint32_t h01 = pack_bf16(p[0], p[1]), h23 = pack_bf16(p[2], p[3]);
+        const uint32_t l01 = pack_bf16(p[0] - bf_lo(h01), p[1] - bf_hi(h01));
+        const uint32_t l23 = pack_bf16(p[2] - bf_lo(h23), p[3] - bf_hi(h23));
+        const uint32_t bh0 = movtrans(h01), bh1 = movtrans(h23);
+        const uint32_t bl0 = movtrans(l01), bl1 = movtrans(l23);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            uint32_t fv[4];
+            ldsm4t(vt + vrow * 256 + (((2 * mt + vhi) ^ (vrow & 7)) << 4), fv);
+            mma_bf16(acc[mt], fv, bh0, bh1);
+            mma_bf16(acc[mt], fv, bl0, bl1);
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        l[j] += __shfl_xor_sync(kFull, l[j], 4);
+        l[j] += __shfl_xor_sync(kFull, l[j], 8);
+        l[j] += __shfl_xor_sync(kFull, l[j], 16);
+    }
+    __syncthreads();   // every warp is done with its pipeline: red overlays them
+    float* rw = red + warp * HG * L::RSTR;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int h = 2 * tig + j;
+        if (h < HG) {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                rw[h * L::RSTR + 16 * mt + gid] = acc[mt][j];
+                rw[h * L::RSTR + 16 * mt + gid + 8] = acc[mt][2 + j];
+            }
+            if (gid == 0) { rw[h * L::RSTR + kD] = m[j]; rw[h * L::RSTR + kD + 1] = l[j]; }
+        }
+    }
+}
+
+// fp32 rows on the CUDA cores: 4-row batches, lane = 4 dims
+template <int HG>
+__device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __restrict__ qg,
+                                              unsigned char* wbuf, int* tokw, float* pz, float* red)
+{
+    using L = AttLayout<false, HG>;
+    constexpr int NB = L::NB, RB = L::RB, NV = 4 * HG;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float qv[HG][4];
+#pragma unroll
+    for (int h = 0; h < HG; ++h)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) qv[h][j] = qg[h * kD + 4 * lane + j];
+    const int nb = (a.a1 - a.a0 + NB - 1) / NB;
+    int tok_base = -L::TOKW;
+    auto issue = [&](int bb) {
+        if (bb < nb) {
+            unsigned char* dst = wbuf + (bb % kAttNBuf) * L::BATCH;
+            const int rbase = a.a0 + bb * NB;
+            if (rbase + NB > tok_base + L::TOKW) {
+                tokens_from<L::TOKW>(a, rbase, tokw, lane);
+                tok_base = rbase;
+            }
+            constexpr int NCH = RB / 16;   // 16-byte chunks per row
+#pragma unroll
+            for (int j = 0; j < NB * NCH / 32; ++j) {
+                const int e = j * 32 + lane;
+                const int row = e / NCH, ch = e % NCH;
+                if (rbase + row < a.a1) {
+                    const int tk = tokw[rbase - tok_base + row];
+                    cp_async16(dst + row * RB + ch * 16, a.Kb + (int64_t)tk * RB + ch * 16);
+                    cp_async16(dst + (NB + row) * RB + ch * 16, a.Vb + (int64_t)tk * RB + ch * 16);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    float m_run[HG], l_run[HG], acc[HG][4];
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+        m_run[h] = -INFINITY;
+        l_run[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+    }
+    issue(0);
+    issue(1);
+    for (int bb = 0; bb < nb; ++bb) {
+        issue(bb + 2);
+        cp_async_wait<kAttNBuf - 1>();
+        __syncwarp();
+        const unsigned char* kt = wbuf + (bb % kAttNBuf) * L::BATCH;
+        const unsigned char* vt = kt + NB * RB;
+        const int rbase = a.a0 + bb * NB;
+        const int rows_in = min(NB, a.a1 - rbase);
+        {   // logits of the 4 rows: one butterfly
+            float v[NV];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+                if (r < rows_in) {
+                    const float4 w = *reinterpret_cast<const float4*>(kt + r * RB + 16 * lane);
+                    x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
+                }
+#pragma unroll
+                for (int h = 0; h < HG; ++h)
+                    v[r * HG + h] = fmaf(qv[h][3], x[3], fmaf(qv[h][2], x[2], fmaf(qv[h][1], x[1], qv[h][0] * x[0])));
+            }
+            const float z = transpose_reduce<NV>(v, lane) * 0.08838834764831845f;   // 1 / sqrt(128)
+            const int idx = tr_index<NV>(lane);
+            constexpr int lowmask = (NV >= 32) ? 0 : (32 / NV) - 1;
+            if ((lane & lowmask) == 0) {
+                const int rr = idx / HG;
+                pz[rr * HG + idx % HG] = (rr < rows_in) ? z : -INFINITY;
+                const int r = rbase + rr;
+                if (rr < rows_in && r >= a.S && r < a.S + a.T) a.zrow[(int64_t)r * HG + idx % HG] = z;
+            }
+        }
+        __syncwarp();
+        float pb[NB][HG];
+#pragma unroll
+        for (int r = 0; r < NB; ++r)
+#pragma unroll
+            for (int h = 0; h < HG; ++h) pb[r][h] = pz[r * HG + h];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            float mb = pb[0][h];
+#pragma unroll
+            for (int r = 1; r < NB; ++r) mb = fmaxf(mb, pb[r][h]);
+            const float m_new = fmaxf(m_run[h], mb);
+            const float sc = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
+            l_run[h] *= sc;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[h][e] *= sc;
+            m_run[h] = m_new;
+#pragma unroll
+            for (int r = 0; r < NB; ++r) {
+                pb[r][h] = (pb[r][h] == -INFINITY) ? 0.f : __expf(pb[r][h] - m_new);
+                l_run[h] += pb[r][h];
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < NB; ++r) {
+            if (r >= rows_in) break;
+            const float4 w = *reinterpret_cast<const float4*>(vt + r * RB + 16 * lane);
+            const float x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int h = 0; h < HG; ++h)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pb[r][h], x[e], acc[h][e]);
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+    __syncthreads();   // every warp is done with its pipeline: red overlays them
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+        float* rw = red + (warp * HG + h) * L::RSTR;
+        *reinterpret_cast<float4*>(rw + 4 * lane) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+        if (lane == 0) { rw[kD] = m_run[h]; rw[kD + 1] = l_run[h]; }
+    }
 }
 
 template <bool BF16, int HG, int KM>
@@ -602,22 +962,20 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
                                                              float* __restrict__ out)
 {
     using L = AttLayout<BF16, HG>;
-    constexpr int NV = 4 * HG;                           // values per 4-row group: (row, head)
     constexpr int RB = L::RB;
     constexpr int NT = kAttWarps * 32;
-    constexpr int kAttNB = L::NB;
     if (*(volatile int*)s.err) return;
     extern __shared__ __align__(128) unsigned char smem[];
-    float* sM = reinterpret_cast<float*>(smem + L::off_misc);          // [8]
-    float* sL = sM + 8;                                                // [8] 1 / L
-    float* mw = sL + 8;                                                // [warps] scratch
-    int* sidx = reinterpret_cast<int*>(mw + kAttWarps);
-    __shared__ int sh_seg[4];          // graph, slice, slices, last
+    float* sM = reinterpret_cast<float*>(smem + L::off_misc);          // [8] graph max per head
+    float* sL = sM + 8;                                                // [8] 1 / graph sum per head
+    int* sidx = reinterpret_cast<int*>(sL + 8);                        // [warps]
+    int* sh_seg = sidx + kAttWarps;                                    // graph, slice, slices, last, ok
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nCTA = gridDim.x, bid = blockIdx.x;
     const int G = d.G;
     unsigned char* wbuf = smem + L::off_buf + warp * L::WBUF;
-    float* pz = reinterpret_cast<float*>(smem + L::off_pz) + warp * L::NB * HG;
+    int* tokw = reinterpret_cast<int*>(smem + L::off_tokw) + warp * L::TOKW;
+    float* red = reinterpret_cast<float*>(smem + L::off_buf);          // [warps][HG][RSTR]
 
     // ---- which graph slice(s) this CTA owns.  G <= nCTA: every graph gets
     // one CTA plus a share of the others proportional to its rows, and each
@@ -628,9 +986,8 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         g_first = (int)((int64_t)bid * G / nCTA);
         g_last = (int)((int64_t)(bid + 1) * G / nCTA);
     } else {
-        // rows of every graph, staged once (one round of loads); warp 0 then
-        // forms their prefix and the first CTA of each graph,
-        // f(g) = g + floor(P_g * extra / R_tot)
+        // rows of every graph, staged once; warp 0 then forms their prefix
+        // and the first CTA of each graph, f(g) = g + floor(P_g * extra / R_tot)
         int* sR = reinterpret_cast<int*>(smem + L::off_buf);
         for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
         __syncthreads();
@@ -678,166 +1035,31 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         const int T = R - d.S - 1;
         const int r0 = (int)((int64_t)k * R / nc), r1 = (int)((int64_t)(k + 1) * R / nc);
         const int nrows = r1 - r0;
-        // this warp's rows, in graph-row numbering: [a0, a1)
-        const int a0 = r0 + (int)((int64_t)warp * nrows / kAttWarps);
-        const int a1 = r0 + (int)((int64_t)(warp + 1) * nrows / kAttWarps);
-        const int nb = (a1 - a0 + kAttNB - 1) / kAttNB;
-        const int t_new = n - 1;
         const int64_t kvbase = ((int64_t)b * d.Hkv + kvh) * d.NM;
-        const char* Kb = reinterpret_cast<const char*>(K) + kvbase * RB;
-        const char* Vb = reinterpret_cast<const char*>(V) + kvbase * RB;
         const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
         float* zrow = s.zrow + (int64_t)g * d.NM * HG;
-        auto row_token = [&](int r) -> int {
-            if (r < d.S) return r;
-            if (r == R - 1) return t_new;
-            return rtok[r - d.S];
-        };
-
-        float qv[HG][4];
-#pragma unroll
-        for (int h = 0; h < HG; ++h)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                qv[h][j] = elem<BF16>(q, ((int64_t)b * d.Hq + h0 + h) * kD + 4 * lane + j);
+        WarpRows a;
+        a.Kb = reinterpret_cast<const char*>(K) + kvbase * RB;
+        a.Vb = reinterpret_cast<const char*>(V) + kvbase * RB;
+        a.rtok = rtok;
+        a.zrow = zrow;
+        a.a0 = r0 + (int)((int64_t)warp * nrows / kAttWarps);
+        a.a1 = r0 + (int)((int64_t)(warp + 1) * nrows / kAttWarps);
+        a.S = d.S;
+        a.T = T;
+        a.R = R;
+        a.t_new = n - 1;
         __syncthreads();   // the previous graph of this CTA is done with the buffers
-
-        // row tokens of this warp, TOKW at a time (one round of loads each)
-        int* tokw = reinterpret_cast<int*>(smem + L::off_tokw) + warp * L::TOKW;
-        int tok_base = -L::TOKW;
-        auto tokens_from = [&](int r) {   // fill tokw with rows r .. r + TOKW - 1
-            __syncwarp();
-            int t0 = 0, t1 = 0;
-            if (r + lane < a1) t0 = row_token(r + lane);
-            if (r + 32 + lane < a1) t1 = row_token(r + 32 + lane);
-            tokw[lane] = t0;
-            tokw[32 + lane] = t1;
-            tok_base = r;
-            __syncwarp();
-        };
-        // batch bb's rows a0 + NB*bb .. : K rows at BATCH*buf, V rows after them
-        auto issue = [&](int bb) {
-            if (bb < nb) {
-                unsigned char* dst = wbuf + (bb % kAttNBuf) * L::BATCH;
-                const int rbase = a0 + bb * kAttNB;
-                if (rbase + kAttNB > tok_base + L::TOKW) tokens_from(rbase);
-#pragma unroll
-                for (int j = 0; j < kAttNB * L::NCH / 32; ++j) {
-                    const int e = j * 32 + lane;
-                    const int row = e / L::NCH, ch = e % L::NCH;
-                    const int tk = tokw[rbase - tok_base + row];
-                    if (rbase + row < a1) {
-                        cp_async16(dst + row * RB + ch * 16, Kb + (int64_t)tk * RB + ch * 16);
-                        cp_async16(dst + (kAttNB + row) * RB + ch * 16, Vb + (int64_t)tk * RB + ch * 16);
-                    }
-                }
-            }
-            cp_async_commit();
-        };
-
-        float m_run[HG], l_run[HG], acc[HG][4];
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-            m_run[h] = -INFINITY;
-            l_run[h] = 0.f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+        if constexpr (BF16) {
+            const uint32_t* q2 = reinterpret_cast<const uint32_t*>(q) + ((int64_t)b * d.Hq + h0) * kD / 2;
+            warp_rows_mma<HG>(a, q2, wbuf, tokw, red);
+        } else {
+            const float* qg = reinterpret_cast<const float*>(q) + ((int64_t)b * d.Hq + h0) * kD;
+            float* pz = reinterpret_cast<float*>(smem + L::off_pz) + warp * L::NB * HG;
+            warp_rows_fma<HG>(a, qg, wbuf, tokw, pz, red);
         }
-        issue(0);
-        issue(1);
-        for (int bb = 0; bb < nb; ++bb) {
-            issue(bb + 2);
-            cp_async_wait<kAttNBuf - 1>();
-            __syncwarp();
-            const unsigned char* kt = wbuf + (bb % kAttNBuf) * L::BATCH;
-            const unsigned char* vt = kt + kAttNB * RB;
-            const int rbase = a0 + bb * kAttNB;
-            const int rows_in = min(kAttNB, a1 - rbase);
-            // logits of the batch: two groups of 4 rows, a butterfly each
-#pragma unroll
-            for (int grp = 0; grp < kAttNB / 4; ++grp) {
-                float v[NV];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int rr = 4 * grp + r;
-                    float x[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (rr < rows_in) {
-                        if (BF16) {
-                            const uint2 w = *reinterpret_cast<const uint2*>(kt + rr * RB + 8 * lane);
-                            x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
-                        } else {
-                            const float4 w = *reinterpret_cast<const float4*>(kt + rr * RB + 16 * lane);
-                            x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
-                        }
-                    }
-#pragma unroll
-                    for (int h = 0; h < HG; ++h)
-                        v[r * HG + h] =
-                            fmaf(qv[h][3], x[3], fmaf(qv[h][2], x[2], fmaf(qv[h][1], x[1], qv[h][0] * x[0])));
-                }
-                const float z = transpose_reduce<NV>(v, lane) * 0.08838834764831845f;   // 1 / sqrt(128)
-                const int idx = tr_index<NV>(lane);
-                constexpr int lowmask = (NV >= 32) ? 0 : (32 / NV) - 1;
-                if ((lane & lowmask) == 0) {
-                    const int rr = 4 * grp + idx / HG;
-                    pz[rr * HG + idx % HG] = (rr < rows_in) ? z : -INFINITY;
-                    const int r = rbase + rr;
-                    if (rr < rows_in && r >= d.S && r < d.S + T) zrow[(int64_t)r * HG + idx % HG] = z;
-                }
-            }
-            __syncwarp();
-            // online softmax over the batch, then P . V
-            float pb[kAttNB][HG];
-#pragma unroll
-            for (int r = 0; r < kAttNB; ++r)
-#pragma unroll
-                for (int h = 0; h < HG; ++h) pb[r][h] = pz[r * HG + h];
-#pragma unroll
-            for (int h = 0; h < HG; ++h) {
-                float mb = pb[0][h];
-#pragma unroll
-                for (int r = 1; r < kAttNB; ++r) mb = fmaxf(mb, pb[r][h]);
-                const float m_new = fmaxf(m_run[h], mb);
-                const float sc = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
-                l_run[h] *= sc;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[h][e] *= sc;
-                m_run[h] = m_new;
-#pragma unroll
-                for (int r = 0; r < kAttNB; ++r) {
-                    pb[r][h] = (pb[r][h] == -INFINITY) ? 0.f : __expf(pb[r][h] - m_new);
-                    l_run[h] += pb[r][h];
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < kAttNB; ++r) {
-                if (r >= rows_in) break;
-                float x[4];
-                if (BF16) {
-                    const uint2 w = *reinterpret_cast<const uint2*>(vt + r * RB + 8 * lane);
-                    x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
-                } else {
-                    const float4 w = *reinterpret_cast<const float4*>(vt + r * RB + 16 * lane);
-                    x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
-                }
-#pragma unroll
-                for (int h = 0; h < HG; ++h)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pb[r][h], x[e], acc[h][e]);
-            }
-            __syncwarp();
-        }
-        cp_async_wait<0>();
         __syncthreads();
         // combine the warps: (m, l, acc) -> this slice's partial per head
-        float* red = reinterpret_cast<float*>(smem + L::off_buf);      // [warps][HG][RSTR]
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-            float* rw = red + (warp * HG + h) * L::RSTR;
-            *reinterpret_cast<float4*>(rw + 4 * lane) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-            if (lane == 0) { rw[kD] = m_run[h]; rw[kD + 1] = l_run[h]; }
-        }
-        __syncthreads();
         float* po = s.part_o + ((int64_t)g * d.nCTA + k) * HG * kD;
         float* pm = s.part_ml + ((int64_t)g * d.nCTA + k) * HG * 2;
         for (int i = tid; i < HG * kD; i += NT) {
@@ -854,16 +1076,21 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
             po[i] = o;
             if (dd == 0) { pm[h * 2] = M; pm[h * 2 + 1] = l; }
         }
-        // ---------------------------------------- last slice of the graph merges
+        // ---- wait until every slice of the graph has published
         __threadfence();
         __syncthreads();
         if (tid == 0) {
-            const unsigned prev = atomicAdd(&s.bar[g * 2 + 1], 1u);
-            sh_seg[3] = (prev == (unsigned)nc - 1);
+            atomicAdd(&s.bar[g * 2], 1u);
+            int ok = 0;
+            for (unsigned it = 0; it < kWaitLimit; ++it) {
+                if (ld_acquire(&s.bar[g * 2]) >= (unsigned)nc) { ok = 1; break; }
+                if ((it & 255) == 255 && *(volatile int*)s.err) break;
+            }
+            if (!ok) set_error(s.err, CKV_ERR_TIMEOUT);
+            sh_seg[4] = ok;
         }
         __syncthreads();
-        if (!sh_seg[3]) continue;
-        __threadfence();
+        if (!sh_seg[4]) return;
         const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
         const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
         if (warp < HG) {   // exact softmax max and sum of the graph, per head
@@ -882,62 +1109,71 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
             if (lane == 0) { sM[h] = M; sL[h] = 1.f / Ls; }
         }
         __syncthreads();
-        for (int i = tid; i < HG * kD; i += NT) {
-            const int h = i / kD;
-            float o = 0.f;
-            for (int j0 = 0; j0 < nc; j0 += 8) {   // 8 slices' loads in flight at once
-                float mj[8], oj[8];
+        {   // this slice's share of the output
+            const int i0 = (int)((int64_t)k * HG * kD / nc), i1 = (int)((int64_t)(k + 1) * HG * kD / nc);
+            for (int i = i0 + tid; i < i1; i += NT) {
+                const int h = i / kD;
+                float o = 0.f;
+                for (int j0 = 0; j0 < nc; j0 += 8) {   // 8 slices' loads in flight at once
+                    float mj[8], oj[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const bool ok = j0 + u < nc;
-                    mj[u] = ok ? __ldcg(pmg + ((int64_t)(j0 + u) * HG + h) * 2) : -INFINITY;
-                    oj[u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
+                    for (int u = 0; u < 8; ++u) {
+                        const bool ok = j0 + u < nc;
+                        mj[u] = ok ? __ldcg(pmg + ((int64_t)(j0 + u) * HG + h) * 2) : -INFINITY;
+                        oj[u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (mj[u] != -INFINITY) o = fmaf(oj[u], __expf(mj[u] - sM[h]), o);
                 }
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if (mj[u] != -INFINITY) o = fmaf(oj[u], __expf(mj[u] - sM[h]), o);
+                out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o * sL[h];
             }
-            out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o * sL[h];
         }
-        // edges: top-kappa of w = sum_h exp(z - M_h) / L_h over the kept members
+        // edge candidates of this slice: per warp the top kappa of
+        // w = sum_h exp(z - M_h) / L_h over the slice's kept members
+        const int64_t cbase = (int64_t)g * d.nCTA * kAttWarps * d.kappa;
         {
             TopList<KM> tl;
             tl.clear();
-            for (int j0 = tid; j0 < T; j0 += 8 * NT) {   // 8 rows' loads in flight at once
-                float zz[8][HG];
-                int tt[8];
+            const int js = max(r0, d.S) - d.S, je = min(r1, d.S + T) - d.S;
+            for (int j = js + tid; j < je; j += NT) {
+                const float* zr = zrow + (int64_t)(d.S + j) * HG;
+                float w = 0.f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = j0 + u * NT;
-                    const bool ok = j < T;
-#pragma unroll
-                    for (int h = 0; h < HG; ++h) zz[u][h] = ok ? __ldcg(zrow + (int64_t)(d.S + j) * HG + h) : 0.f;
-                    tt[u] = ok ? __ldcg(rtok + j) : 0;
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = j0 + u * NT;
-                    if (j >= T) break;
-                    float w = 0.f;
-#pragma unroll
-                    for (int h = 0; h < HG; ++h) w += __expf(zz[u][h] - sM[h]) * sL[h];
-                    tl.insert(w, tt[u], j);
-                }
+                for (int h = 0; h < HG; ++h) w += __expf(__ldcg(zr + h) - sM[h]) * sL[h];
+                tl.insert(w, __ldcg(rtok + j), j);
+            }
+            const int64_t o = cbase + ((int64_t)k * kAttWarps + warp) * d.kappa;
+            warp_merge<KM>(tl, d.kappa, s.cand_w + o, s.cand_t + o, s.cand_x + o);
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) sh_seg[3] = (atomicAdd(&s.bar[g * 2 + 1], 1u) == (unsigned)nc - 1);
+        __syncthreads();
+        if (!sh_seg[3]) continue;
+        // ---- the last slice: merge the graph's candidate lists
+        __threadfence();
+        {
+            TopList<KM> tl;
+            tl.clear();
+            const int ncand = nc * kAttWarps * d.kappa;
+            for (int e = tid; e < ncand; e += NT) {
+                const float w = __ldcg(s.cand_w + cbase + e);
+                if (w != -INFINITY) tl.insert(w, __ldcg(s.cand_t + cbase + e), __ldcg(s.cand_x + cbase + e));
             }
             float* ew = reinterpret_cast<float*>(smem + L::off_buf);        // [warps][kMaxKappa]
             int* et = reinterpret_cast<int*>(ew + kAttWarps * kMaxKappa);
             int* ex = et + kAttWarps * kMaxKappa;
-            __syncthreads();    // the reduction buffer is free again
-            const int nw = warp_merge<KM>(tl, d.kappa, ew + warp * kMaxKappa, et + warp * kMaxKappa,
-                                          ex + warp * kMaxKappa);
-            if (lane == 0) sidx[warp] = nw;
+            warp_merge<KM>(tl, d.kappa, ew + warp * kMaxKappa, et + warp * kMaxKappa, ex + warp * kMaxKappa);
             __syncthreads();
             if (warp == 0) {
                 TopList<KM> t2;
                 t2.clear();
-                for (int w = 0; w < kAttWarps; ++w)
-                    for (int e = lane; e < sidx[w]; e += 32)
-                        t2.insert(ew[w * kMaxKappa + e], et[w * kMaxKappa + e], ex[w * kMaxKappa + e]);
+                for (int e = lane; e < kAttWarps * d.kappa; e += 32) {
+                    const int w = e / d.kappa, i = e % d.kappa;
+                    const float v = ew[w * kMaxKappa + i];
+                    if (v != -INFINITY) t2.insert(v, et[w * kMaxKappa + i], ex[w * kMaxKappa + i]);
+                }
                 float* gw = s.e_w + (int64_t)g * d.kappa;
                 int* gt = s.e_tok + (int64_t)g * d.kappa;
                 int* gx = s.e_comm + (int64_t)g * d.kappa;   // row index first, community below
@@ -946,6 +1182,7 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
                 if (lane < ne) gx[lane] = s.rcomm[(int64_t)g * d.NM + gx[lane]];
                 if (lane == 0) {
                     s.meta[(int64_t)g * M_COUNT + M_NEDGE] = ne;
+                    s.bar[g * 2] = 0u;
                     s.bar[g * 2 + 1] = 0u;
                 }
             }

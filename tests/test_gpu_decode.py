@@ -223,3 +223,43 @@ def test_host_buffer_step_matches_device_step():
     finally:
         ckv.ckv_destroy(a)
         ckv.ckv_destroy(b)
+
+
+@pytest.mark.parametrize("captured", [False, True])
+def test_per_kernel_profile_eager_and_captured(captured):
+    """ckv_profile_begin/end time each kernel of eager and graph-captured steps;
+    profiling changes no result."""
+    import torch
+    cfg, wl, ctx, K, V, q, out = _small_ctx()
+    ref_ctx = ckv.ckv_create(config_for(cfg))
+    try:
+        ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        ckv.ckv_init_communities(ref_ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        ref = torch.empty_like(out)
+        ckv.ckv_profile_begin(ctx)
+        steps = range(cfg.steps)
+        if captured:
+            side = torch.cuda.Stream()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(side), torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+                for i in steps:
+                    ckv.ckv_decode_step(ctx, q[i], K, V, cfg.n0 + i + 1, out, side.cuda_stream)
+                    ckv.ckv_assign_update(ctx, K, cfg.n0 + i + 1, side.cuda_stream)
+            graph.replay()
+        else:
+            for i in steps:
+                ckv.ckv_decode_step(ctx, q[i], K, V, cfg.n0 + i + 1, out)
+                ckv.ckv_assign_update(ctx, K, cfg.n0 + i + 1)
+        torch.cuda.synchronize()
+        ms, n = ckv.ckv_profile_end(ctx)
+        assert n == cfg.steps
+        assert all(m > 0.0 for m in ms) and sum(ms) < 1000.0 * n
+        for i in steps:
+            ckv.ckv_decode_step(ref_ctx, q[i], K, V, cfg.n0 + i + 1, ref)
+            ckv.ckv_assign_update(ref_ctx, K, cfg.n0 + i + 1)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+        assert ckv.ckv_export_state(ctx) == ckv.ckv_export_state(ref_ctx)
+    finally:
+        ckv.ckv_destroy(ctx)
+        ckv.ckv_destroy(ref_ctx)
