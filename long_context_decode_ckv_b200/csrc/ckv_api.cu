@@ -281,9 +281,9 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(part_ml, G * KC * HG * 2);
     ALLOC(part_o, G * KC * HG * ckv::kD);
     ALLOC(bar, G * 2);
-    ALLOC(cand_w, G * KC * ckv::kAttWarps * kap);
-    ALLOC(cand_t, G * KC * ckv::kAttWarps * kap);
-    ALLOC(cand_x, G * KC * ckv::kAttWarps * kap);
+    ALLOC(cand_w, G * KC * kap);
+    ALLOC(cand_t, G * KC * kap);
+    ALLOC(cand_x, G * KC * kap);
     ALLOC(e_tok, G * kap);
     ALLOC(e_w, G * kap);
     ALLOC(e_comm, G * kap);

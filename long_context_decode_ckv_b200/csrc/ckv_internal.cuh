@@ -19,7 +19,7 @@
 //   part_o    float [G][KC][HG][D] per-CTA P.V per head, relative to its max
 //   bar       uint  [G][2]         arrivals of a graph's CTAs: partials published
 //                                  (slot 0), edge candidates published (slot 1)
-//   cand_*    [G][KC][W][kappa]    per-warp edge candidates (W = kAttWarps)
+//   cand_*    [G][KC][kappa]       each CTA's edge candidates (rank order)
 //   e_*       [G][kappa]           the step's edges (rank order) for the update
 #pragma once
 
@@ -60,7 +60,7 @@ struct DevState {
     float* part_ml;
     float* part_o;
     unsigned int* bar;
-    float* cand_w;           // per-warp edge candidates of each slice
+    float* cand_w;           // edge candidates of each attention CTA
     int32_t* cand_t;
     int32_t* cand_x;
     int32_t* e_tok;

@@ -120,7 +120,7 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     const size_t o_zrow = off;  off = align256(off + (size_t)rows_max * HG * 4);
     const size_t o_pml = off;   off = align256(off + KC * HG * 2 * 4);
     const size_t o_po = off;    off = align256(off + KC * HG * kD * 4);
-    const size_t o_cand = off;  off = align256(off + KC * ckv::kAttWarps * 3 * 4);   // kappa = 1
+    const size_t o_cand = off;  off = align256(off + KC * 3 * 4);   // kappa = 1
     if (off > kStaticScratchBytes) return CKV_ERR_CAPACITY;   // max_rows too large for the array
     unsigned char* sb = static_cast<unsigned char*>(base);
     ckv::DevState s{};
@@ -136,8 +136,8 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     s.part_ml = reinterpret_cast<float*>(sb + o_pml);
     s.part_o = reinterpret_cast<float*>(sb + o_po);
     s.cand_w = reinterpret_cast<float*>(sb + o_cand);
-    s.cand_t = reinterpret_cast<int32_t*>(sb + o_cand) + KC * ckv::kAttWarps;
-    s.cand_x = reinterpret_cast<int32_t*>(sb + o_cand) + 2 * KC * ckv::kAttWarps;
+    s.cand_t = reinterpret_cast<int32_t*>(sb + o_cand) + KC;
+    s.cand_x = reinterpret_cast<int32_t*>(sb + o_cand) + 2 * KC;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t eb = d.bf16 ? 2 : 4;

@@ -488,6 +488,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select(DevState s, Dims d)
 // output and ranks its own kept members' edge weights w_j; the last slice
 // to finish merges the slices' candidate lists into the top-kappa edges.
 constexpr int kAttNBuf = 3;        // batches per warp pipeline
+constexpr int kEdgeRows = 4;       // kept-member rows a thread holds for the edge ranking
+static_assert(kMaxKappa == 32, "edge lists give one slot per lane");
 
 template <bool BF16, int HG>
 struct AttLayout {
@@ -505,7 +507,7 @@ struct AttLayout {
     // acc[0..D), m, l, padded to a multiple of 16 bytes for float4 access
     static constexpr int RSTR = kD + 4;
     static_assert(kAttWarps * HG * RSTR * 4 <= kAttWarps * WBUF, "reduction must fit");
-    static_assert(kAttWarps * kMaxKappa * 12 <= kAttWarps * WBUF, "edge lists must fit");
+    static_assert(kAttWarps * 6 * (kMaxKappa + 128) * 4 <= kAttWarps * WBUF, "edge lists must fit");
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
@@ -599,63 +601,117 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[NV], int lane)
     return r;
 }
 
-// A lane's sorted (w desc, token asc) list of its best KM candidates.
-template <int KM>
-struct TopList {
-    float w[KM];
-    int t[KM], x[KM];
-    __device__ __forceinline__ void clear()
-    {
-#pragma unroll
-        for (int i = 0; i < KM; ++i) { w[i] = -INFINITY; t[i] = 0x7fffffff; x[i] = -1; }
-    }
-    __device__ __forceinline__ void insert(float nw, int nt, int nx)
-    {
-        if (!cand_better(nw, nt, w[KM - 1], t[KM - 1])) return;
-#pragma unroll
-        for (int i = KM - 1; i > 0; --i) {
-            const bool shift = cand_better(nw, nt, w[i - 1], t[i - 1]);
-            const bool land = !shift && cand_better(nw, nt, w[i], t[i]);
-            w[i] = shift ? w[i - 1] : (land ? nw : w[i]);
-            t[i] = shift ? t[i - 1] : (land ? nt : t[i]);
-            x[i] = shift ? x[i - 1] : (land ? nx : x[i]);
-        }
-        if (cand_better(nw, nt, w[0], t[0])) { w[0] = nw; t[0] = nt; x[0] = nx; }
-    }
-    __device__ __forceinline__ void pop()
-    {
-#pragma unroll
-        for (int i = 0; i < KM - 1; ++i) { w[i] = w[i + 1]; t[i] = t[i + 1]; x[i] = x[i + 1]; }
-        w[KM - 1] = -INFINITY; t[KM - 1] = 0x7fffffff; x[KM - 1] = -1;
-    }
+// Edge candidates of one warp in shared memory: a running list of the best
+// kappa (<= kMaxKappa) in slots [0, kMaxKappa) (w desc, token asc; w = -inf
+// marks an empty slot), new candidates in the block after it, and scratch
+// for the compaction.
+constexpr int kEdgeBlk = 128;                     // new candidates per selection round
+constexpr int kEdgeBuf = kMaxKappa + kEdgeBlk;
+static_assert(kEdgeRows * 32 <= kEdgeBlk, "a thread's rows fit one round");
+
+struct EdgeSlots {
+    float* w;
+    int* t;
+    int* x;
+    float* sw;
+    int* st;
+    int* sx;
 };
 
-// Merge the 32 lanes' lists: the warp's top kappa (kappa <= KM) in rank
-// order, written by lane 0 with w = -inf in the unused tail; returns how
-// many are real.
-template <int KM>
-__device__ __forceinline__ int warp_merge(TopList<KM>& L, int kappa, float* ow, int* ot, int* ox)
+__device__ __forceinline__ EdgeSlots edge_slots(unsigned char* base, int warp)
+{
+    float* f = reinterpret_cast<float*>(base) + warp * 6 * kEdgeBuf;
+    EdgeSlots e;
+    e.w = f;
+    e.t = reinterpret_cast<int*>(f + kEdgeBuf);
+    e.x = reinterpret_cast<int*>(f + 2 * kEdgeBuf);
+    e.sw = f + 3 * kEdgeBuf;
+    e.st = reinterpret_cast<int*>(f + 4 * kEdgeBuf);
+    e.sx = reinterpret_cast<int*>(f + 5 * kEdgeBuf);
+    return e;
+}
+
+__device__ __forceinline__ void edge_clear(const EdgeSlots& e, int lane)
+{
+    e.w[lane] = -INFINITY;   // kMaxKappa == 32 slots, one per lane
+    e.t[lane] = 0x7fffffff;
+    e.x[lane] = -1;
+}
+
+// list := the top kappa of the list and the block's nb candidates, by one
+// warp.  The kappa-th best of the lanes' best entries is a lower bound of
+// the answer (kappa distinct entries reach it), so only the entries at
+// least as good are compacted and ranked by counting.
+__device__ __forceinline__ void warp_select(const EdgeSlots& e, int nb, int kappa)
 {
     const int lane = threadIdx.x & 31;
-    int nout = 0;
-    for (int k = 0; k < kappa; ++k) {
-        float bw = L.w[0];
-        int bt = L.t[0], bl = lane;
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            const float w2 = __shfl_xor_sync(kFull, bw, o);
-            const int t2 = __shfl_xor_sync(kFull, bt, o);
-            const int l2 = __shfl_xor_sync(kFull, bl, o);
-            if (cand_better(w2, t2, bw, bt) || (w2 == bw && t2 == bt && l2 < bl)) { bw = w2; bt = t2; bl = l2; }
-        }
-        if (bw == -INFINITY) break;
-        const int bx = __shfl_sync(kFull, L.x[0], bl);
-        if (lane == 0) { ow[k] = bw; ot[k] = bt; ox[k] = bx; }
-        if (lane == bl) L.pop();
-        ++nout;
+    const int n = kMaxKappa + nb;
+    __syncwarp();
+    float bw = -INFINITY;
+    int bt = 0x7fffffff;
+    for (int i = lane; i < n; i += 32) {
+        const float w = e.w[i];
+        const int t = e.t[i];
+        if (w != -INFINITY && cand_better(w, t, bw, bt)) { bw = w; bt = t; }
     }
-    for (int k = nout + lane; k < kappa; k += 32) { ow[k] = -INFINITY; ot[k] = 0x7fffffff; ox[k] = -1; }
-    return nout;
+    float tw = -INFINITY;    // threshold (anything valid when fewer than kappa lanes hold one)
+    int tt = 0x7fffffff;
+    if (__popc(__ballot_sync(kFull, bw != -INFINITY)) >= kappa) {
+        int rank = 0;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const float w2 = __shfl_sync(kFull, bw, i);
+            const int t2 = __shfl_sync(kFull, bt, i);
+            rank += cand_better(w2, t2, bw, bt) ? 1 : 0;
+        }
+        const int src = __ffs(__ballot_sync(kFull, bw != -INFINITY && rank == kappa - 1)) - 1;
+        tw = __shfl_sync(kFull, bw, src);
+        tt = __shfl_sync(kFull, bt, src);
+    }
+    int c = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        float w = -INFINITY;
+        int t = 0x7fffffff, x = -1;
+        if (i < n) { w = e.w[i]; t = e.t[i]; x = e.x[i]; }
+        const bool ok = w != -INFINITY && !cand_better(tw, tt, w, t);
+        const unsigned bal = __ballot_sync(kFull, ok);
+        if (ok) {
+            const int p = c + __popc(bal & ((1u << lane) - 1u));
+            e.sw[p] = w;
+            e.st[p] = t;
+            e.sx[p] = x;
+        }
+        c += __popc(bal);
+    }
+    __syncwarp();
+    for (int i = lane; i < c; i += 32) {
+        const float w = e.sw[i];
+        const int t = e.st[i];
+        int r = 0;
+        for (int j = 0; j < c; ++j) r += cand_better(e.sw[j], e.st[j], w, t) ? 1 : 0;
+        if (r < kappa) { e.w[r] = w; e.t[r] = t; e.x[r] = e.sx[i]; }
+    }
+    for (int r = c + lane; r < kappa; r += 32) { e.w[r] = -INFINITY; e.t[r] = 0x7fffffff; e.x[r] = -1; }
+    __syncwarp();
+}
+
+// HG logits of one kept-member row (16-, 8- or 4-byte aligned by HG)
+template <int HG>
+__device__ __forceinline__ void load_logits(const float* p, float (&z)[HG])
+{
+    if constexpr (HG % 4 == 0) {
+#pragma unroll
+        for (int h = 0; h < HG; h += 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(p + h));
+            z[h] = v.x; z[h + 1] = v.y; z[h + 2] = v.z; z[h + 3] = v.w;
+        }
+    } else if constexpr (HG == 2) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(p));
+        z[0] = v.x; z[1] = v.y;
+    } else {
+        z[0] = __ldcg(p);
+    }
 }
 
 // Rows of one warp: [a0, a1) in the graph's row numbering (sinks, kept
@@ -955,7 +1011,7 @@ __device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __
     }
 }
 
-template <bool BF16, int HG, int KM>
+template <bool BF16, int HG>
 __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d, const void* __restrict__ q,
                                                              const void* __restrict__ K,
                                                              const void* __restrict__ V, int n,
@@ -1064,17 +1120,39 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         float* pm = s.part_ml + ((int64_t)g * d.nCTA + k) * HG * 2;
         for (int i = tid; i < HG * kD; i += NT) {
             const int h = i / kD, dd = i % kD;
+            float mw[kAttWarps];
             float M = -INFINITY;
-            for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, red[(w * HG + h) * L::RSTR + kD]);
+#pragma unroll
+            for (int w = 0; w < kAttWarps; ++w) {
+                mw[w] = red[(w * HG + h) * L::RSTR + kD];
+                M = fmaxf(M, mw[w]);
+            }
             float o = 0.f, l = 0.f;
+#pragma unroll
             for (int w = 0; w < kAttWarps; ++w) {
                 const float* rw = red + (w * HG + h) * L::RSTR;
-                const float f = (rw[kD] == -INFINITY) ? 0.f : __expf(rw[kD] - M);
+                const float f = (mw[w] == -INFINITY) ? 0.f : __expf(mw[w] - M);
                 o = fmaf(rw[dd], f, o);
                 l = fmaf(rw[kD + 1], f, l);
             }
             po[i] = o;
-            if (dd == 0) { pm[h * 2] = M; pm[h * 2 + 1] = l; }
+            if (dd == 0) *reinterpret_cast<float2*>(pm + h * 2) = make_float2(M, l);
+        }
+        // this thread's kept-member rows of the slice (logits written by this
+        // CTA's warps), loaded before the wait
+        const int js = max(r0, d.S) - d.S, je = min(r1, d.S + T) - d.S;
+        float zr[kEdgeRows][HG];
+        int tr[kEdgeRows];
+#pragma unroll
+        for (int u = 0; u < kEdgeRows; ++u) {
+            const int j = js + tid + u * NT;
+            tr[u] = 0;
+#pragma unroll
+            for (int h = 0; h < HG; ++h) zr[u][h] = -INFINITY;
+            if (j < je) {
+                load_logits<HG>(zrow + (int64_t)(d.S + j) * HG, zr[u]);
+                tr[u] = __ldcg(rtok + j);
+            }
         }
         // ---- wait until every slice of the graph has published
         __threadfence();
@@ -1093,93 +1171,133 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         if (!sh_seg[4]) return;
         const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
         const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
-        if (warp < HG) {   // exact softmax max and sum of the graph, per head
-            const int h = warp;
-            float M = -INFINITY;
-            for (int j = lane; j < nc; j += 32) M = fmaxf(M, __ldcg(pmg + ((int64_t)j * HG + h) * 2));
-#pragma unroll
-            for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-            float Ls = 0.f;
-            for (int j = lane; j < nc; j += 32) {
-                const float mj = __ldcg(pmg + ((int64_t)j * HG + h) * 2);
-                if (mj != -INFINITY) Ls += __ldcg(pmg + ((int64_t)j * HG + h) * 2 + 1) * __expf(mj - M);
+        if (warp >= kAttWarps - HG) {   // the graph's exact softmax max and 1 / sum per head
+            const int h = warp - (kAttWarps - HG);
+            float M = -INFINITY, Ls = 0.f;
+            for (int j = lane; j < nc; j += 32) {   // online over this lane's slices
+                const float2 ml = __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)j * HG + h) * 2));
+                if (ml.x != -INFINITY) {
+                    const float mn = fmaxf(M, ml.x);
+                    Ls = Ls * ((M == -INFINITY) ? 0.f : __expf(M - mn)) + ml.y * __expf(ml.x - mn);
+                    M = mn;
+                }
             }
 #pragma unroll
-            for (int o = 16; o; o >>= 1) Ls += __shfl_xor_sync(kFull, Ls, o);
+            for (int o = 16; o; o >>= 1) {
+                const float M2 = __shfl_xor_sync(kFull, M, o), L2 = __shfl_xor_sync(kFull, Ls, o);
+                const float mn = fmaxf(M, M2);
+                if (mn != -INFINITY)
+                    Ls = ((M == -INFINITY) ? 0.f : Ls * __expf(M - mn)) + ((M2 == -INFINITY) ? 0.f : L2 * __expf(M2 - mn));
+                M = mn;
+            }
             if (lane == 0) { sM[h] = M; sL[h] = 1.f / Ls; }
         }
-        __syncthreads();
-        {   // this slice's share of the output
+        {   // this slice's share of the output: each value merged online over the slices
             const int i0 = (int)((int64_t)k * HG * kD / nc), i1 = (int)((int64_t)(k + 1) * HG * kD / nc);
             for (int i = i0 + tid; i < i1; i += NT) {
                 const int h = i / kD;
-                float o = 0.f;
+                float M = -INFINITY, Ls = 0.f, o = 0.f;
                 for (int j0 = 0; j0 < nc; j0 += 8) {   // 8 slices' loads in flight at once
-                    float mj[8], oj[8];
+                    float2 mj[8];
+                    float oj[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const bool ok = j0 + u < nc;
-                        mj[u] = ok ? __ldcg(pmg + ((int64_t)(j0 + u) * HG + h) * 2) : -INFINITY;
+                        mj[u] = ok ? __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)(j0 + u) * HG + h) * 2))
+                                   : make_float2(-INFINITY, 0.f);
                         oj[u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
                     }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (mj[u] != -INFINITY) o = fmaf(oj[u], __expf(mj[u] - sM[h]), o);
+                    for (int u = 0; u < 8; ++u) {
+                        if (mj[u].x == -INFINITY) continue;
+                        const float mn = fmaxf(M, mj[u].x);
+                        const float a = (M == -INFINITY) ? 0.f : __expf(M - mn), c = __expf(mj[u].x - mn);
+                        o = o * a + oj[u] * c;
+                        Ls = Ls * a + mj[u].y * c;
+                        M = mn;
+                    }
                 }
-                out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o * sL[h];
+                out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o / Ls;
             }
         }
-        // edge candidates of this slice: per warp the top kappa of
-        // w = sum_h exp(z - M_h) / L_h over the slice's kept members
-        const int64_t cbase = (int64_t)g * d.nCTA * kAttWarps * d.kappa;
-        {
-            TopList<KM> tl;
-            tl.clear();
-            const int js = max(r0, d.S) - d.S, je = min(r1, d.S + T) - d.S;
-            for (int j = js + tid; j < je; j += NT) {
-                const float* zr = zrow + (int64_t)(d.S + j) * HG;
-                float w = 0.f;
+        __syncthreads();   // sM, sL
+        // ---- edge candidates: the slice's top kappa of w = sum_h exp(z - M_h) / L_h
+        const EdgeSlots es = edge_slots(smem + L::off_buf, warp);
+        edge_clear(es, lane);
 #pragma unroll
-                for (int h = 0; h < HG; ++h) w += __expf(__ldcg(zr + h) - sM[h]) * sL[h];
-                tl.insert(w, __ldcg(rtok + j), j);
-            }
-            const int64_t o = cbase + ((int64_t)k * kAttWarps + warp) * d.kappa;
-            warp_merge<KM>(tl, d.kappa, s.cand_w + o, s.cand_t + o, s.cand_x + o);
+        for (int u = 0; u < kEdgeRows; ++u) {
+            const int j = js + tid + u * NT;
+            float w = 0.f;
+#pragma unroll
+            for (int h = 0; h < HG; ++h) w += __expf(zr[u][h] - sM[h]) * sL[h];
+            es.w[kMaxKappa + u * 32 + lane] = (j < je) ? w : -INFINITY;
+            es.t[kMaxKappa + u * 32 + lane] = tr[u];
+            es.x[kMaxKappa + u * 32 + lane] = j;
         }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) sh_seg[3] = (atomicAdd(&s.bar[g * 2 + 1], 1u) == (unsigned)nc - 1);
-        __syncthreads();
-        if (!sh_seg[3]) continue;
-        // ---- the last slice: merge the graph's candidate lists
-        __threadfence();
-        {
-            TopList<KM> tl;
-            tl.clear();
-            const int ncand = nc * kAttWarps * d.kappa;
-            for (int e = tid; e < ncand; e += NT) {
-                const float w = __ldcg(s.cand_w + cbase + e);
-                if (w != -INFINITY) tl.insert(w, __ldcg(s.cand_t + cbase + e), __ldcg(s.cand_x + cbase + e));
-            }
-            float* ew = reinterpret_cast<float*>(smem + L::off_buf);        // [warps][kMaxKappa]
-            int* et = reinterpret_cast<int*>(ew + kAttWarps * kMaxKappa);
-            int* ex = et + kAttWarps * kMaxKappa;
-            warp_merge<KM>(tl, d.kappa, ew + warp * kMaxKappa, et + warp * kMaxKappa, ex + warp * kMaxKappa);
-            __syncthreads();
-            if (warp == 0) {
-                TopList<KM> t2;
-                t2.clear();
-                for (int e = lane; e < kAttWarps * d.kappa; e += 32) {
-                    const int w = e / d.kappa, i = e % d.kappa;
-                    const float v = ew[w * kMaxKappa + i];
-                    if (v != -INFINITY) t2.insert(v, et[w * kMaxKappa + i], ex[w * kMaxKappa + i]);
+        warp_select(es, kEdgeRows * 32, d.kappa);
+        for (int j0 = js + kEdgeRows * NT; j0 < je; j0 += kEdgeRows * NT) {   // slices longer than the registers hold
+            for (int u = 0; u < kEdgeRows; ++u) {
+                const int j = j0 + tid + u * NT;
+                float w = -INFINITY;
+                int t = 0;
+                if (j < je) {
+                    float z[HG];
+                    load_logits<HG>(zrow + (int64_t)(d.S + j) * HG, z);
+                    w = 0.f;
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) w += __expf(z[h] - sM[h]) * sL[h];
+                    t = __ldcg(rtok + j);
                 }
-                float* gw = s.e_w + (int64_t)g * d.kappa;
-                int* gt = s.e_tok + (int64_t)g * d.kappa;
-                int* gx = s.e_comm + (int64_t)g * d.kappa;   // row index first, community below
-                const int ne = warp_merge<KM>(t2, d.kappa, gw, gt, gx);
-                __syncwarp();
-                if (lane < ne) gx[lane] = s.rcomm[(int64_t)g * d.NM + gx[lane]];
+                es.w[kMaxKappa + u * 32 + lane] = w;
+                es.t[kMaxKappa + u * 32 + lane] = t;
+                es.x[kMaxKappa + u * 32 + lane] = j;
+            }
+            warp_select(es, kEdgeRows * 32, d.kappa);
+        }
+        __syncthreads();
+        const int64_t cbase = (int64_t)g * d.nCTA * d.kappa;
+        if (warp == 0) {   // the slice's list from its warps' lists
+            const int per = kEdgeBlk / d.kappa;   // whole lists per round
+            for (int w0 = 1; w0 < kAttWarps; w0 += per) {
+                const int nw = min(per, kAttWarps - w0);
+                for (int i = lane; i < nw * d.kappa; i += 32) {
+                    const EdgeSlots o = edge_slots(smem + L::off_buf, w0 + i / d.kappa);
+                    es.w[kMaxKappa + i] = o.w[i % d.kappa];
+                    es.t[kMaxKappa + i] = o.t[i % d.kappa];
+                    es.x[kMaxKappa + i] = o.x[i % d.kappa];
+                }
+                warp_select(es, nw * d.kappa, d.kappa);
+            }
+            if (lane < d.kappa) {
+                const int64_t o = cbase + (int64_t)k * d.kappa + lane;
+                s.cand_w[o] = es.w[lane];
+                s.cand_t[o] = es.t[lane];
+                s.cand_x[o] = es.x[lane];
+            }
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) last = (atomicAdd(&s.bar[g * 2 + 1], 1u) == (unsigned)nc - 1);
+            last = __shfl_sync(kFull, last, 0);
+            if (last) {   // the last slice: merge the slices' lists
+                __threadfence();
+                edge_clear(es, lane);
+                const int ncand = nc * d.kappa;
+                for (int e0 = 0; e0 < ncand; e0 += kEdgeBlk) {
+                    const int nb = min(kEdgeBlk, ncand - e0);
+                    for (int i = lane; i < nb; i += 32) {
+                        es.w[kMaxKappa + i] = __ldcg(s.cand_w + cbase + e0 + i);
+                        es.t[kMaxKappa + i] = __ldcg(s.cand_t + cbase + e0 + i);
+                        es.x[kMaxKappa + i] = __ldcg(s.cand_x + cbase + e0 + i);
+                    }
+                    warp_select(es, nb, d.kappa);
+                }
+                const int ne = __popc(__ballot_sync(kFull, lane < d.kappa && es.w[lane] != -INFINITY));
+                if (lane < ne) {
+                    s.e_w[(int64_t)g * d.kappa + lane] = es.w[lane];
+                    s.e_tok[(int64_t)g * d.kappa + lane] = es.t[lane];
+                    s.e_comm[(int64_t)g * d.kappa + lane] = s.rcomm[(int64_t)g * d.NM + es.x[lane]];
+                }
                 if (lane == 0) {
                     s.meta[(int64_t)g * M_COUNT + M_NEDGE] = ne;
                     s.bar[g * 2] = 0u;
@@ -1291,11 +1409,9 @@ cudaError_t dispatch_hg(int hg, F&& f)
 }
 
 template <bool BF16, int HG>
-void* attend_fn(int kappa)
+void* attend_fn()
 {
-    if (kappa <= 8) return reinterpret_cast<void*>(k_attend<BF16, HG, 8>);
-    if (kappa <= 16) return reinterpret_cast<void*>(k_attend<BF16, HG, 16>);
-    return reinterpret_cast<void*>(k_attend<BF16, HG, 32>);
+    return reinterpret_cast<void*>(k_attend<BF16, HG>);
 }
 
 }  // namespace
@@ -1334,7 +1450,7 @@ cudaError_t prepare_kernels(const Dims& d)
     if (e != cudaSuccess) return e;
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
-        void* fn = d.bf16 ? attend_fn<true, HG>(d.kappa) : attend_fn<false, HG>(d.kappa);
+        void* fn = d.bf16 ? attend_fn<true, HG>() : attend_fn<false, HG>();
         const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
         return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     });
@@ -1347,7 +1463,7 @@ int attend_grid(const Dims& d, int sms)
     if (e == cudaSuccess)
         e = dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
             constexpr int HG = decltype(hgc)::value;
-            void* fn = d.bf16 ? attend_fn<true, HG>(d.kappa) : attend_fn<false, HG>(d.kappa);
+            void* fn = d.bf16 ? attend_fn<true, HG>() : attend_fn<false, HG>();
             const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
             return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kAttWarps * 32, bytes);
         });
@@ -1360,7 +1476,7 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
 {
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
-        void* fn = d.bf16 ? attend_fn<true, HG>(d.kappa) : attend_fn<false, HG>(d.kappa);
+        void* fn = d.bf16 ? attend_fn<true, HG>() : attend_fn<false, HG>();
         const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
         // the slices of a graph wait for one another: all CTAs must be
         // co-resident, which a cooperative launch guarantees (or refuses)
