@@ -189,6 +189,8 @@ def main():
     ap.add_argument("--cpu-steps", type=int, default=8)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--profile-steps", type=int, default=40,
+                    help="further steps replayed with per-kernel events (0 = none)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -219,7 +221,7 @@ def main():
         pg = dist
 
     cfg = CFG
-    total_steps = args.warmup + args.steps + args.e2e_steps
+    total_steps = args.warmup + args.steps + args.profile_steps + args.e2e_steps
     L = args.replicas or max(4, -(-total_steps // cfg.steps))
     if -(-total_steps // L) > cfg.steps:
         raise SystemExit("not enough decode tokens in the workload for these steps; raise --replicas")
@@ -256,21 +258,36 @@ def main():
     for s in range(args.warmup):
         step(s, stream)
     torch.cuda.synchronize(dev)
-    for r in reps:
-        ckv.ckv_profile_begin(r["ctx"])
-    # The timed steps are captured once into a CUDA graph (the launches of a
-    # real decoder are), then replayed once: the device time is the steps'.
-    graph = None
-    if not args.no_graph:
+
+    def capture(first, count):
+        """The steps [first, first + count) captured into one CUDA graph (the
+        launches of a real decoder are), or None when capture is refused."""
+        if args.no_graph:
+            return None
+        saved = [r["i"] for r in reps]
         try:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
                 cap = torch.cuda.current_stream(dev)
-                for s in range(args.warmup, args.warmup + args.steps):
+                for s in range(first, first + count):
                     step(s, cap)
+            return g
         except Exception as exc:   # capture refused: time the same steps eagerly
             print(f"CUDA graph capture failed ({exc}); timing eager launches", file=sys.stderr)
-            graph = None
+            for r, i in zip(reps, saved):
+                r["i"] = i
+            return None
+
+    def run(first, count, g):
+        if g is not None:
+            g.replay()
+        else:
+            for s in range(first, first + count):
+                step(s, stream)
+
+    # timed steps: no profiling events inside
+    s_timed = args.warmup
+    graph = capture(s_timed, args.steps)
     launch_mode = "cuda-graph" if graph is not None else "eager"
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if pg:
@@ -278,26 +295,36 @@ def main():
     torch.cuda.synchronize(dev)
     with Clocks(local) as clk:
         start.record(stream)
-        if graph is not None:
-            graph.replay()
-        else:
-            for s in range(args.warmup, args.warmup + args.steps):
-                step(s, stream)
+        run(s_timed, args.steps, graph)
         end.record(stream)
         torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     ms = start.elapsed_time(end)
+    del graph
+
+    # per-kernel device time: the next steps again, with an event pair
+    # around every kernel (recorded on the launching stream)
+    s_prof = s_timed + args.steps
     kern_ms, kern_steps = [0.0] * 4, 0
-    for r in reps:
-        try:
-            m, k = ckv.ckv_profile_end(r["ctx"])
-        except ckv.CkvError as exc:
-            print(f"per-kernel profile unavailable: {exc}", file=sys.stderr)
-            kern_ms, kern_steps = None, 0
-            break
-        kern_ms = [a + b for a, b in zip(kern_ms, m)]
-        kern_steps += k
+    if args.profile_steps:
+        for r in reps:
+            ckv.ckv_profile_begin(r["ctx"])
+        pgraph = capture(s_prof, args.profile_steps)
+        run(s_prof, args.profile_steps, pgraph)
+        torch.cuda.synchronize(dev)
+        for r in reps:
+            try:
+                m, k = ckv.ckv_profile_end(r["ctx"])
+            except ckv.CkvError as exc:
+                print(f"per-kernel profile unavailable: {exc}", file=sys.stderr)
+                kern_ms, kern_steps = None, 0
+                break
+            kern_ms = [a + b for a, b in zip(kern_ms, m)]
+            kern_steps += k
+        del pgraph
+    else:
+        kern_ms = None
     for r in reps:
         assert ckv.ckv_last_error(r["ctx"]) == ckv.CKV_OK
     ckv.ckv_get_step_debug(reps[(args.warmup + args.steps - 1) % L]["ctx"], n_tok_sel=sel_tok)
@@ -317,7 +344,7 @@ def main():
         oh = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32).pin_memory()
         kstep = [kh[:, :, i].contiguous() for i in range(cfg.steps)]
         vstep = [vh[:, :, i].contiguous() for i in range(cfg.steps)]
-        s0 = args.warmup + args.steps
+        s0 = s_prof + args.profile_steps
         if pg:
             pg.barrier()
         torch.cuda.synchronize(dev)
@@ -341,7 +368,6 @@ def main():
                "h2d_bytes_per_step": cfg.batch * (cfg.n_q_heads + 2 * cfg.n_kv_heads) * 128 * eb,
                "d2h_bytes_per_step": cfg.batch * cfg.n_q_heads * 128 * 4}
 
-    del graph
     for r in reps:
         ckv.ckv_destroy(r["ctx"])
     if pg:

@@ -255,6 +255,12 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
                                  : (int64_t)cfg->n_max * 5 + (int64_t)cfg->max_communities * (cfg->slack + 32);
     // the attention grid: as many CTAs as can be co-resident
     d.nSM = sms;
+    {   // programmatic dependent launch between the decode kernels: off unless
+        // CKV_PDL is 1 (each kernel lets the next one launch at its start) or
+        // 2 (after its main work)
+        const char* v = getenv("CKV_PDL");
+        d.pdl = (v && (v[0] == '1' || v[0] == '2')) ? v[0] - '0' : 0;
+    }
     d.nCTA = ckv::attend_grid(d, sms);
     if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
     d.n_comm = 0;

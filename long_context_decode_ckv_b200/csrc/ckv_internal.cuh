@@ -33,7 +33,6 @@ namespace ckv {
 constexpr int kD = 128;          // head_dim the kernels are written for
 constexpr int kMaxKappa = 32;
 constexpr int kSelBins = 2048;   // bucket count of the selection passes
-constexpr int kSortCap = 1024;   // candidates ranked exactly in one CTA
 constexpr int kAttWarps = 8;     // warps of an attention CTA
 
 // meta slots per graph
@@ -76,6 +75,7 @@ struct Dims {
     int nSM;                 // multiprocessors of the device
     int n_comm;              // communities in use (set at init)
     int n_init;              // first decode position (edge store row 0)
+    int pdl;                 // programmatic dependent launch: 0 off, 1 trigger at kernel start, 2 after the main work
 };
 
 // kernel launchers (k_decode.cu)
@@ -85,12 +85,12 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
                           const void* V, int n, float* out, cudaStream_t st);
 cudaError_t launch_assign(const DevState& s, const Dims& d, const void* K, int n,
                           cudaStream_t st);
-size_t select_smem_bytes(int n_comm);
+size_t select_smem_bytes(int n_comm, int budget);
 // sets the kernels' shared-memory limits on the current device; then the
 // number of co-resident CTAs of the attention kernel (0 on error)
 cudaError_t prepare_kernels(const Dims& d);
 int attend_grid(const Dims& d, int sms);
-constexpr int kMaxCommunities = 16384;   // k_select keeps a graph's communities in shared memory
+constexpr int kMaxCommunities = 16384;   // k_select holds 16 of a graph's communities per thread
 
 // init kernels (k_init.cu)
 cudaError_t launch_init_count(const DevState& s, const Dims& d, const int32_t* labels, int n,

@@ -70,6 +70,13 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
         : "memory");
 }
 
+// Programmatic dependent launch.  pdl_wait blocks until the grid this one
+// was launched behind has completed and its memory is visible (a no-op for
+// an ordinary launch); pdl_trigger lets the grid launched behind this one
+// start its own launch (its CTAs still wait in pdl_wait before any work).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // barrier among `nthreads` threads (a multiple of 32) using hardware barrier `id` (1..15)
 __device__ __forceinline__ void named_sync(int id, int nthreads)
 {

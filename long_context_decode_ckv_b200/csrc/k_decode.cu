@@ -28,7 +28,9 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <type_traits>
+#include <utility>
 
 #include "ckv_internal.cuh"
 #include "dev_async.cuh"
@@ -38,7 +40,6 @@ namespace ckv {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kSelThreads = 1024;
 constexpr int kAsgThreads = 128;
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -98,6 +99,8 @@ struct ScoreSmem {
 template <bool BF16>
 __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, const void* __restrict__ q)
 {
+    pdl_wait();
+    if (d.pdl) pdl_trigger();
     if (*(volatile int*)s.err) return;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(smem_raw);
@@ -180,248 +183,266 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, 
     if (*abort_flag && c == 0 && lane == 0) set_error(s.err, CKV_ERR_TIMEOUT);
 }
 
-// -------------------------------------------------------- block utilities
-// inclusive block scan of an int; returns the block total in `total`
-__device__ __forceinline__ int block_scan_incl(int v, int* warp_sums, int& total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nw = (int)(blockDim.x >> 5);
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int t = __shfl_up_sync(kFull, v, o);
-        if (lane >= o) v += t;
-    }
-    if (lane == 31) warp_sums[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int w = (lane < nw) ? warp_sums[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int t = __shfl_up_sync(kFull, w, o);
-            if (lane >= o) w += t;
-        }
-        warp_sums[lane] = w;
-    }
-    __syncthreads();
-    const int add = warp ? warp_sums[warp - 1] : 0;
-    total = warp_sums[nw - 1];
-    __syncthreads();
-    return v + add;
-}
-
 // --------------------------------------------------------------- k_select
+// One CTA of 1024 threads per graph.  Thread t owns communities t, t + 1024,
+// ... (E of them, scores and sizes in registers); its status lives in
+// shared memory.  Exact budgeted top-C in (score desc, id asc) order:
+//   1. one round of loads; the score range and the total size;
+//   2. a size-weighted histogram over kSelBins bins, linear in the score
+//      (bins are monotone in the score, so every community of a higher bin
+//      ranks before every one of a lower bin); the boundary bin is where the
+//      size summed from the top first exceeds the budget;
+//   3. while the boundary bin holds more than kSelCand communities, radix
+//      passes over the composite key (score bits, inverted id) of those
+//      communities narrow it by 11 bits a pass;
+//   4. the boundary bin's communities are ranked exactly: each counts the
+//      size of the better ones, and is kept iff the sizes through it fit;
+//   5. the kept ids in ascending order with the prefix of their sizes, by
+//      ballots per 32 ids and one scan over the (round, warp) counts;
+//   6. each kept community's owner copies its members into the row list.
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelCand = 1024;     // boundary-bin communities ranked exactly
 enum : int8_t { ST_OUT = 0, ST_IN = 1, ST_CAND = 2 };
 
-struct SelStats {
-    float lo, hi;
-    uint32_t uor, unand, ior, inand;
-    int cnt;
-};
-
-// shared memory (each region a multiple of 16 bytes):
-//   sc/pre [Nc+1] | wz/coffs [Nc] | hist, keys, weights / sel [max(Nc, 5120)] | st [Nc]
-__host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
-__host__ __device__ inline size_t sel_region3(int Nc) { return (size_t)(Nc > 5120 ? round4(Nc) : 5120); }
-
-// key of a candidate: (order-preserving score bits, inverted id): larger = kept first
+// key of a community: (order-preserving score bits, inverted id): larger = kept first
 __device__ __forceinline__ unsigned long long sel_key(float sc, int c)
 {
-    return ((unsigned long long)ord_u(sc) << 32) | (unsigned long long)(~(uint32_t)c);
+    // -0 and +0 are the same score (adding +0 turns -0 into +0)
+    return ((unsigned long long)ord_u(sc + 0.0f) << 32) | (unsigned long long)(~(uint32_t)c);
 }
 
-__global__ void __launch_bounds__(kSelThreads) k_select(DevState s, Dims d)
+// inclusive prefix sum over the warp
+__device__ __forceinline__ int warp_incl(int x, int lane)
 {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+template <int E>
+__global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
+{
+    pdl_wait();
+    if (d.pdl == 1) pdl_trigger();
     if (*(volatile int*)s.err) return;
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ int warp_sums[32];
-    __shared__ SelStats wst[32];
-    __shared__ int sh_bstar, sh_above, sh_wabove, sh_done, sh_ncand;
-    __shared__ SelStats sh_tot;
+    extern __shared__ __align__(16) unsigned char smem_sel[];
+    int8_t* st = reinterpret_cast<int8_t*>(smem_sel);       // [Nc] status of each community
+    __shared__ float r_lo[kSelWarps], r_hi[kSelWarps];
+    __shared__ int r_w[kSelWarps];
+    __shared__ unsigned long long r_kmin[kSelWarps], r_kmax[kSelWarps];
+    __shared__ int off_c[E][kSelWarps], off_w[E][kSelWarps];
+    __shared__ int sh_b, sh_above, sh_n, sh_C, sh_T;
     const int g = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int Nc = d.n_comm;
-    float* sc = reinterpret_cast<float*>(smem);
-    int* pre = reinterpret_cast<int*>(smem);                 // reuses sc after the passes
-    int* wz = reinterpret_cast<int*>(sc + round4(Nc + 1));
-    int* coffs = wz;                                          // reuses wz after compaction
-    int* r3 = wz + round4(Nc);
-    int* hist = r3;                                           // [kSelBins]
-    unsigned long long* keys = reinterpret_cast<unsigned long long*>(r3 + kSelBins);   // [kSortCap]
-    int* wts = r3 + kSelBins + 2 * kSortCap;                  // [kSortCap]
-    int* sel_s = r3;                                          // reuses the above after ranking
-    int8_t* st = reinterpret_cast<int8_t*>(r3 + sel_region3(Nc));
+    const int Nc = d.n_comm, budget = d.budget;
 
-    // ---- load the graph's scores and sizes (coalesced, one round)
+    // ---- 1. scores and sizes (one round of loads), range and total size
     const float* gsc = s.score + (int64_t)g * d.Nc;
     const int32_t* gsz = s.csize + (int64_t)g * d.Nc;
+    float v[E];
+    int w[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int c = i * kSelThreads + tid;
+        w[i] = (c < Nc) ? gsz[c] : 0;
+        v[i] = (c < Nc) ? gsc[c] : 0.f;
+    }
+    float lo = INFINITY, hi = -INFINITY;
     int wsum = 0;
-    for (int c = tid; c < Nc; c += kSelThreads) {
-        const float v = gsc[c];
-        const int w = gsz[c];
-        sc[c] = v;
-        wz[c] = w;
-        st[c] = (w > 0) ? ST_CAND : ST_OUT;
-        wsum += (w > 0) ? w : 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int c = i * kSelThreads + tid;
+        if (w[i] > 0) {
+            lo = fminf(lo, v[i]);
+            hi = fmaxf(hi, v[i]);
+            wsum += w[i];
+        } else {
+            w[i] = 0;
+        }
+        if (c < Nc) st[c] = (w[i] > 0) ? ST_CAND : ST_OUT;
     }
-    int total_w;
-    block_scan_incl(wsum, warp_sums, total_w);
-    if (tid == 0) { sh_wabove = 0; sh_done = (total_w <= d.budget); }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(kFull, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, o));
+        wsum += __shfl_xor_sync(kFull, wsum, o);
+    }
+    if (lane == 0) { r_lo[warp] = lo; r_hi[warp] = hi; r_w[warp] = wsum; }
+    if (tid == 0) { sh_n = 0; sh_above = 0; }
     __syncthreads();
-    if (sh_done) {   // every community fits the budget: keep them all
-        for (int c = tid; c < Nc; c += kSelThreads)
-            if (st[c] == ST_CAND) st[c] = ST_IN;
+    lo = r_lo[lane];
+    hi = r_hi[lane];
+    wsum = r_w[lane];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(kFull, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, o));
+        wsum += __shfl_xor_sync(kFull, wsum, o);
     }
 
-    // ---- bucket passes until <= kSortCap candidates remain.  Each thread
-    // owns communities tid, tid + 1024, ... so statuses need no barrier.
-    int kind = 0;   // 0 linear in the score over [lo, hi], 1 radix window of ord_u, 2 of the id
-    for (int pass = 0; pass < 12 && !sh_done; ++pass) {
-        SelStats a{INFINITY, -INFINITY, 0u, 0u, 0u, 0u, 0};
-        for (int c = tid; c < Nc; c += kSelThreads) {
-            if (st[c] != ST_CAND) continue;
-            const float v = sc[c];
-            const uint32_t u = ord_u(v), iv = ~(uint32_t)c;
-            a.lo = fminf(a.lo, v);
-            a.hi = fmaxf(a.hi, v);
-            a.uor |= u; a.unand |= ~u; a.ior |= iv; a.inand |= ~iv;
-            ++a.cnt;
-        }
+    // shared memory after the statuses: the passes' histogram and boundary
+    // candidates, later (same bytes) the kept list
+    unsigned char* ub = smem_sel + ((Nc + 15) & ~15);
+    unsigned long long* ckey = reinterpret_cast<unsigned long long*>(ub);    // [kSelCand]
+    int* hist = reinterpret_cast<int*>(ckey + kSelCand);                      // [kSelBins]
+    int* cwt = hist + kSelBins;                                               // [kSelCand]
+    for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0;
+
+    if (wsum <= budget) {   // every community fits: keep them all
 #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            a.lo = fminf(a.lo, __shfl_xor_sync(kFull, a.lo, o));
-            a.hi = fmaxf(a.hi, __shfl_xor_sync(kFull, a.hi, o));
-            a.uor |= __shfl_xor_sync(kFull, a.uor, o);
-            a.unand |= __shfl_xor_sync(kFull, a.unand, o);
-            a.ior |= __shfl_xor_sync(kFull, a.ior, o);
-            a.inand |= __shfl_xor_sync(kFull, a.inand, o);
-            a.cnt += __shfl_xor_sync(kFull, a.cnt, o);
+        for (int i = 0; i < E; ++i) {
+            const int c = i * kSelThreads + tid;
+            if (w[i] > 0) st[c] = ST_IN;
         }
-        if (lane == 0) wst[warp] = a;
-        for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0;
-        __syncthreads();
-        if (warp == 0) {
-            SelStats o = wst[lane];
-#pragma unroll
-            for (int x = 16; x; x >>= 1) {
-                o.lo = fminf(o.lo, __shfl_xor_sync(kFull, o.lo, x));
-                o.hi = fmaxf(o.hi, __shfl_xor_sync(kFull, o.hi, x));
-                o.uor |= __shfl_xor_sync(kFull, o.uor, x);
-                o.unand |= __shfl_xor_sync(kFull, o.unand, x);
-                o.ior |= __shfl_xor_sync(kFull, o.ior, x);
-                o.inand |= __shfl_xor_sync(kFull, o.inand, x);
-                o.cnt += __shfl_xor_sync(kFull, o.cnt, x);
+    } else {
+        // ---- 2./3. bucket passes until the boundary bin is small
+        const float scale = (hi > lo) ? (float)kSelBins / (hi - lo) : 0.f;
+        int above = 0;      // size of the communities known to be kept
+        int shift = -1;     // -1: linear in the score; else radix window of the key
+        int m = 0;
+        __syncthreads();    // hist zeroed
+        for (int pass = 0;; ++pass) {
+            if (pass == 8) {   // 64 key bits take at most 6 radix passes: unreachable
+                if (tid == 0) set_error(s.err, CKV_ERR_STATE);
+                return;
             }
-            if (lane == 0) sh_tot = o;
+            auto bin_of = [&](int i, int c) -> int {
+                if (shift < 0) return min(kSelBins - 1, (int)((v[i] - lo) * scale));
+                return (int)((sel_key(v[i], c) >> shift) & (unsigned long long)(kSelBins - 1));
+            };
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int c = i * kSelThreads + tid;
+                if (c < Nc && st[c] == ST_CAND) atomicAdd(&hist[bin_of(i, c)], w[i]);
+            }
+            __syncthreads();
+            // boundary bin: the size summed from the top bin down first exceeds the budget
+            const int b0 = kSelBins - 1 - 2 * tid, b1 = b0 - 1;
+            const int h0 = hist[b0], h1 = hist[b1];
+            const int x = h0 + h1;
+            const int incl = warp_incl(x, lane);
+            if (lane == 31) r_w[warp] = incl;
+            __syncthreads();
+            int wpre = 0;
+            for (int j = 0; j < warp; ++j) wpre += r_w[j];
+            const int bef = above + wpre + incl - x;
+            if (bef <= budget && bef + h0 > budget) { sh_b = b0; sh_above = bef; }
+            else if (bef + h0 <= budget && bef + h0 + h1 > budget) { sh_b = b1; sh_above = bef + h0; }
+            __syncthreads();
+            const int bs = sh_b;
+            above = sh_above;
+            hist[b0] = 0;
+            hist[b1] = 0;
+            unsigned long long kmn = ~0ull, kmx = 0ull;
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int c = i * kSelThreads + tid;
+                if (c < Nc && st[c] == ST_CAND) {
+                    const int b = bin_of(i, c);
+                    if (b > bs) {
+                        st[c] = ST_IN;
+                    } else if (b < bs) {
+                        st[c] = ST_OUT;
+                    } else {
+                        const unsigned long long k = sel_key(v[i], c);
+                        kmn = min(kmn, k);
+                        kmx = max(kmx, k);
+                        const int slot = atomicAdd(&sh_n, 1);
+                        if (slot < kSelCand) { ckey[slot] = k; cwt[slot] = w[i]; }
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                kmn = min(kmn, __shfl_xor_sync(kFull, kmn, o));
+                kmx = max(kmx, __shfl_xor_sync(kFull, kmx, o));
+            }
+            if (lane == 0) { r_kmin[warp] = kmn; r_kmax[warp] = kmx; }
+            __syncthreads();
+            m = sh_n;
+            if (m <= kSelCand) break;                      // uniform
+            kmn = r_kmin[lane];
+            kmx = r_kmax[lane];
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                kmn = min(kmn, __shfl_xor_sync(kFull, kmn, o));
+                kmx = max(kmx, __shfl_xor_sync(kFull, kmx, o));
+            }
+            // the candidates share every key bit above the highest differing one
+            shift = max(0, 63 - __clzll((long long)(kmn ^ kmx)) - 10);
+            __syncthreads();                               // sh_n read by all
+            if (tid == 0) sh_n = 0;
         }
-        __syncthreads();
-        const SelStats t = sh_tot;
-        if (t.cnt <= kSortCap) break;                       // uniform
-        // bits that differ among the candidates: OR of all & OR of complements
-        const uint32_t udiff = t.uor & t.unand, idiff = t.ior & t.inand;
-        if (kind == 0 && !(t.lo < t.hi)) kind = 1;
-        if (kind == 1 && udiff == 0) kind = 2;
-        int shift = 0;
-        if (kind == 1) shift = max(0, 31 - __clz(udiff) - 10);
-        if (kind == 2) shift = max(0, 31 - __clz(idiff) - 10);
-        const double dlo = (double)t.lo, dscale = (double)kSelBins / ((double)t.hi - (double)t.lo);
-        auto bin_of = [&](int c) -> int {
-            if (kind == 0) return max(0, min(kSelBins - 1, (int)(((double)sc[c] - dlo) * dscale)));
-            if (kind == 1) return (int)((ord_u(sc[c]) >> shift) & (kSelBins - 1));
-            return (int)((~(uint32_t)c >> shift) & (kSelBins - 1));
-        };
-        for (int c = tid; c < Nc; c += kSelThreads)
-            if (st[c] == ST_CAND) atomicAdd(&hist[bin_of(c)], wz[c]);
-        __syncthreads();
-        // boundary bin, scanning from the top bin down (2 bins per thread)
-        const int rb0 = kSelBins - 1 - 2 * tid, rb1 = rb0 - 1;
-        const int h0v = hist[rb0], h1v = hist[rb1];
-        int tot;
-        const int incl = block_scan_incl(h0v + h1v, warp_sums, tot);
-        const int w_above = sh_wabove;
-        const int before = w_above + incl - (h0v + h1v);
-        if (tid == 0) sh_bstar = -1;
-        __syncthreads();
-        if (before <= d.budget && before + h0v > d.budget) { sh_bstar = rb0; sh_above = before - w_above; }
-        else if (before + h0v <= d.budget && before + h0v + h1v > d.budget) {
-            sh_bstar = rb1;
-            sh_above = before + h0v - w_above;
+        // ---- 4. exact rank of the boundary bin's communities
+        for (int j = tid; j < m; j += kSelThreads) {
+            const unsigned long long kj = ckey[j];
+            int pre = 0;
+            for (int t = 0; t < m; ++t) pre += (ckey[t] > kj) ? cwt[t] : 0;
+            const bool keep = (above + pre + cwt[j] <= budget) || (above == 0 && pre == 0);
+            st[(int)~(uint32_t)(kj & 0xffffffffull)] = keep ? ST_IN : ST_OUT;
         }
-        __syncthreads();
-        const int bstar = sh_bstar;
-        for (int c = tid; c < Nc; c += kSelThreads) {
-            if (st[c] != ST_CAND) continue;
-            if (bstar < 0) { st[c] = ST_IN; continue; }
-            const int bin = bin_of(c);
-            st[c] = (bin > bstar) ? ST_IN : (bin < bstar ? ST_OUT : ST_CAND);
-        }
-        if (kind == 0) kind = 1;   // the linear pass runs once, radix windows after
-        __syncthreads();
-        if (tid == 0) {
-            if (bstar < 0) sh_done = 1;
-            else sh_wabove = w_above + sh_above;
-        }
-        __syncthreads();
     }
+    __syncthreads();
 
-    // ---- final exact pass: rank the remaining candidates by key
-    if (!sh_done) {
-        if (tid == 0) sh_ncand = 0;
-        __syncthreads();
-        for (int c = tid; c < Nc; c += kSelThreads) {
-            if (st[c] != ST_CAND) continue;
-            const int slot = atomicAdd(&sh_ncand, 1);
-            if (slot < kSortCap) { keys[slot] = sel_key(sc[c], c); wts[slot] = wz[c]; }
-        }
-        __syncthreads();
-        const int m = min(sh_ncand, kSortCap);
-        int rank = 0;
-        unsigned long long mykey = 0ull;
-        int myw = 0;
-        if (tid < m) {
-            mykey = keys[tid];
-            myw = wts[tid];
-            for (int k = 0; k < m; ++k) rank += (keys[k] > mykey);   // keys are distinct
-        }
-        __syncthreads();
-        // weights in rank order, then an inclusive prefix over them
-        if (tid < m) { wts[rank] = myw; keys[rank] = mykey; }
-        __syncthreads();
-        const int wr = (tid < m) ? wts[tid] : 0;
-        int tot;
-        const int incl = block_scan_incl(wr, warp_sums, tot);
-        const int w_above = sh_wabove;
-        if (tid < m) {
-            const bool keep = (w_above + incl <= d.budget) || (w_above == 0 && tid == 0);
-            const int c = (int)(~(uint32_t)(keys[tid] & 0xffffffffull));
-            st[c] = keep ? ST_IN : ST_OUT;
-        }
-        __syncthreads();
+    // ---- 5. kept ids ascending with the prefix of their sizes: per round i
+    // a warp's 32 ids are consecutive, so ballots place them within the
+    // warp and one scan over the (round, warp) totals places the warps
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int c = i * kSelThreads + tid;
+        const bool kept = c < Nc && st[c] == ST_IN;
+        const unsigned bal = __ballot_sync(kFull, kept);
+        const int wt = bal ? (int)__reduce_add_sync(kFull, kept ? (unsigned)w[i] : 0u) : 0;
+        if (lane == 0) { off_c[i][warp] = __popc(bal); off_w[i][warp] = wt; }
     }
-
-    // ---- compaction in ascending id, prefix of sizes (pre reuses sc).
-    // Thread t owns the consecutive ids [t*per, (t+1)*per): two block scans
-    // (kept count, kept weight) place every thread's kept communities.
+    __syncthreads();
+    if (warp == 0) {   // exclusive offsets in (round, warp) order; lane owns E consecutive entries
+        int sc = 0, sw = 0;
+        for (int j = 0; j < E; ++j) {
+            const int e = lane * E + j;
+            sc += off_c[e / kSelWarps][e % kSelWarps];
+            sw += off_w[e / kSelWarps][e % kSelWarps];
+        }
+        const int ic = warp_incl(sc, lane), iw = warp_incl(sw, lane);
+        int pc = ic - sc, pw = iw - sw;
+        for (int j = 0; j < E; ++j) {
+            const int e = lane * E + j;
+            const int a = off_c[e / kSelWarps][e % kSelWarps], b = off_w[e / kSelWarps][e % kSelWarps];
+            off_c[e / kSelWarps][e % kSelWarps] = pc;
+            off_w[e / kSelWarps][e % kSelWarps] = pw;
+            pc += a;
+            pw += b;
+        }
+        if (lane == 31) { sh_C = ic; sh_T = iw; }
+    }
+    __syncthreads();
+    const int C = sh_C, T = sh_T;
+    // the kept list (overlays the passes' arrays): row start, id, segment start
+    int* pre = reinterpret_cast<int*>(ub);       // [C + 1]
+    int* cid = pre + C + 1;                      // [C]
+    int* cof = cid + C;                          // [C]
     int32_t* gsel = s.sel + (int64_t)g * d.Nc;
-    const int per = (Nc + kSelThreads - 1) / kSelThreads;
-    const int c_lo = min(Nc, tid * per), c_hi = min(Nc, c_lo + per);
-    int my_c = 0, my_t = 0;
-    for (int c = c_lo; c < c_hi; ++c)
-        if (st[c] == ST_IN) { ++my_c; my_t += wz[c]; }
-    int tot_c, tot_t;
-    const int inc_c = block_scan_incl(my_c, warp_sums, tot_c);
-    const int inc_t = block_scan_incl(my_t, warp_sums, tot_t);
-    {
-        int pos = inc_c - my_c, acc = inc_t - my_t;
-        for (int c = c_lo; c < c_hi; ++c) {
-            if (st[c] != ST_IN) continue;
-            sel_s[pos] = c;
+    const int32_t* gcoff = s.coff + (int64_t)g * d.Nc;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int c = i * kSelThreads + tid;
+        const bool kept = c < Nc && st[c] == ST_IN;
+        const unsigned bal = __ballot_sync(kFull, kept);
+        if (bal == 0u) continue;                                   // warp-uniform
+        const int wk = kept ? w[i] : 0;
+        const int wx = (bal & (bal - 1u)) ? warp_incl(wk, lane) - wk : 0;   // exclusive prefix
+        if (kept) {
+            const int pos = off_c[i][warp] + __popc(bal & ((1u << lane) - 1u));
+            pre[pos] = off_w[i][warp] + wx;
+            cid[pos] = c;
+            cof[pos] = gcoff[c];
             gsel[pos] = c;
-            pre[pos] = acc;
-            acc += wz[c];
-            ++pos;
         }
     }
-    const int C = tot_c, T = tot_t;
     if (tid == 0) {
         pre[C] = T;
         int32_t* meta = s.meta + (int64_t)g * M_COUNT;
@@ -429,38 +450,31 @@ __global__ void __launch_bounds__(kSelThreads) k_select(DevState s, Dims d)
         meta[M_T] = T;
         meta[M_ROWS] = d.S + T + 1;
     }
+    if (d.pdl == 2) pdl_trigger();
     __syncthreads();
-    // ---- kept rows: segment starts of the kept communities (one round),
-    // then every row's token (one round)
-    const int32_t* gcoff = s.coff + (int64_t)g * d.Nc;
-    for (int k = tid; k < C; k += kSelThreads) coffs[k] = gcoff[sel_s[k]];
-    __syncthreads();
+    // ---- 6. the kept members' rows: warp k copies kept communities k,
+    // k + 32, ... (contiguous segments, eight communities' loads in flight)
     const int32_t* pool = s.pool + (int64_t)g * d.P;
     int32_t* rtok = s.rtok + (int64_t)g * d.NM;
     int32_t* rcomm = s.rcomm + (int64_t)g * d.NM;
-    for (int base = 0; base < T; base += 4 * kSelThreads) {
-        int src[4], cc[4], idx[4];
+    for (int k0 = warp; k0 < C; k0 += 8 * kSelWarps) {
+        int tk[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            idx[u] = base + u * kSelThreads + tid;
-            src[u] = -1;
-            cc[u] = 0;
-            if (idx[u] < T) {
-                int lo = 0, hi = C - 1;          // last k with pre[k] <= idx
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (pre[mid] <= idx[u]) lo = mid; else hi = mid - 1;
-                }
-                src[u] = coffs[lo] + idx[u] - pre[lo];
-                cc[u] = sel_s[lo];
+        for (int u = 0; u < 8; ++u) {
+            const int k = k0 + u * kSelWarps;
+            tk[u] = (k < C && lane < pre[k + 1] - pre[k]) ? pool[cof[k] + lane] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int k = k0 + u * kSelWarps;
+            if (k >= C) break;
+            const int r0 = pre[k], sz = pre[k + 1] - r0, cc = cid[k];
+            if (lane < sz) { rtok[r0 + lane] = tk[u]; rcomm[r0 + lane] = cc; }
+            for (int j = 32 + lane; j < sz; j += 32) {   // communities longer than a warp
+                rtok[r0 + j] = pool[cof[k] + j];
+                rcomm[r0 + j] = cc;
             }
         }
-        int tk[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) tk[u] = (src[u] >= 0) ? pool[src[u]] : 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (src[u] >= 0) { rtok[idx[u]] = tk[u]; rcomm[idx[u]] = cc[u]; }
     }
 }
 
@@ -1020,6 +1034,8 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
     using L = AttLayout<BF16, HG>;
     constexpr int RB = L::RB;
     constexpr int NT = kAttWarps * 32;
+    pdl_wait();
+    if (d.pdl == 1) pdl_trigger();
     if (*(volatile int*)s.err) return;
     extern __shared__ __align__(128) unsigned char smem[];
     float* sM = reinterpret_cast<float*>(smem + L::off_misc);          // [8] graph max per head
@@ -1169,6 +1185,7 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         }
         __syncthreads();
         if (!sh_seg[4]) return;
+        if (d.pdl == 2) pdl_trigger();
         const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
         const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
         if (warp >= kAttWarps - HG) {   // the graph's exact softmax max and 1 / sum per head
@@ -1312,6 +1329,8 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
 template <bool BF16>
 __global__ void __launch_bounds__(kAsgThreads) k_assign(DevState s, Dims d, const void* __restrict__ K, int n)
 {
+    pdl_wait();
+    if (d.pdl) pdl_trigger();
     if (*(volatile int*)s.err) return;
     __shared__ int e_c[kMaxKappa];
     __shared__ float e_w[kMaxKappa];
@@ -1396,6 +1415,26 @@ __global__ void k_append(const uint32_t* __restrict__ knew, const uint32_t* __re
     }
 }
 
+// Launch with programmatic stream serialization (when d.pdl): the kernel may
+// begin launching while the previous kernel of the stream finishes; every
+// decode kernel starts with pdl_wait.  Cooperative when asked.
+template <typename... P, typename... A>
+cudaError_t launch_ex(const Dims& d, void (*fn)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      A&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = d.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, fn, std::forward<A>(args)...);
+}
+
 template <typename F>
 cudaError_t dispatch_hg(int hg, F&& f)
 {
@@ -1416,33 +1455,61 @@ void* attend_fn()
 
 }  // namespace
 
-size_t select_smem_bytes(int n_comm)
+size_t select_smem_bytes(int n_comm, int budget)
 {
-    return (size_t)4 * round4(n_comm + 1) + (size_t)4 * round4(n_comm) + 4 * sel_region3(n_comm) + (size_t)n_comm + 16;
-}
-
-cudaError_t launch_score(const DevState& s, const Dims& d, const void* q, cudaStream_t st)
+    // statuses, then the larger of the passes' arrays and the kept list
+    const size_t kept_cap = (size_t)std::min(n_comm, budget + 1);
+    const size_t passes = (size_t)8 * kSelCand + 4 * kSelBins + 4 * kSelCand;
+    return (size_t)((n_comm + 15) & ~15) + std::max(passes, 4 * (3 * kept_cap + 1));
+}template <int E>
+static cudaError_t launch_select_e(const DevState& s, const Dims& d, cudaStream_t st)
+{
+    return launch_ex(d, k_select<E>, dim3(d.G), dim3(kSelThreads), select_smem_bytes(d.n_comm, d.budget), st, s, d);
+}cudaError_t launch_score(const DevState& s, const Dims& d, const void* q, cudaStream_t st)
 {
     const int units = d.G * ((d.n_comm + 31) / 32);
     const int grid = units < d.nSM ? units : d.nSM;   // persistent: one CTA per SM
     const size_t smem = sizeof(ScoreSmem);
-    if (d.bf16) k_score<true><<<grid, kScoreThreads, smem, st>>>(s, d, q);
-    else k_score<false><<<grid, kScoreThreads, smem, st>>>(s, d, q);
-    return cudaGetLastError();
+    return launch_ex(d, d.bf16 ? k_score<true> : k_score<false>, dim3(grid), dim3(kScoreThreads), smem, st, s, d, q);
 }
 
 cudaError_t launch_select(const DevState& s, const Dims& d, cudaStream_t st)
 {
-    k_select<<<d.G, kSelThreads, select_smem_bytes(d.n_comm), st>>>(s, d);
-    return cudaGetLastError();
+    switch ((d.n_comm + kSelThreads - 1) / kSelThreads) {
+        case 0:
+        case 1: return launch_select_e<1>(s, d, st);
+        case 2: return launch_select_e<2>(s, d, st);
+        case 3: return launch_select_e<3>(s, d, st);
+        case 4: return launch_select_e<4>(s, d, st);
+        case 5: return launch_select_e<5>(s, d, st);
+        case 6: return launch_select_e<6>(s, d, st);
+        case 7: return launch_select_e<7>(s, d, st);
+        case 8: return launch_select_e<8>(s, d, st);
+        case 9: return launch_select_e<9>(s, d, st);
+        case 10: return launch_select_e<10>(s, d, st);
+        case 11: return launch_select_e<11>(s, d, st);
+        case 12: return launch_select_e<12>(s, d, st);
+        case 13: return launch_select_e<13>(s, d, st);
+        case 14: return launch_select_e<14>(s, d, st);
+        case 15: return launch_select_e<15>(s, d, st);
+        default: return launch_select_e<16>(s, d, st);
+    }
 }
 
 cudaError_t prepare_kernels(const Dims& d)
 {
     // shared-memory limits are set once per device, before any launch (and
     // so outside any stream capture)
-    cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)select_smem_bytes(kMaxCommunities));
+    const int sel_bytes = (int)select_smem_bytes(kMaxCommunities, kMaxCommunities);
+    cudaError_t e = cudaSuccess;
+    const void* sel_fns[] = {(const void*)k_select<1>,  (const void*)k_select<2>,  (const void*)k_select<3>,
+                             (const void*)k_select<4>,  (const void*)k_select<5>,  (const void*)k_select<6>,
+                             (const void*)k_select<7>,  (const void*)k_select<8>,  (const void*)k_select<9>,
+                             (const void*)k_select<10>, (const void*)k_select<11>, (const void*)k_select<12>,
+                             (const void*)k_select<13>, (const void*)k_select<14>, (const void*)k_select<15>,
+                             (const void*)k_select<16>};
+    for (const void* f : sel_fns)
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_bytes);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_score<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScoreSmem));
     if (e == cudaSuccess)
@@ -1485,11 +1552,13 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
         cfg.blockDim = dim3(kAttWarps * 32);
         cfg.dynamicSmemBytes = bytes;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = d.pdl ? 2 : 1;
         DevState ss = s;
         Dims dd = d;
         const void* qq = q;
@@ -1504,9 +1573,7 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
 
 cudaError_t launch_assign(const DevState& s, const Dims& d, const void* K, int n, cudaStream_t st)
 {
-    if (d.bf16) k_assign<true><<<d.G, kAsgThreads, 0, st>>>(s, d, K, n);
-    else k_assign<false><<<d.G, kAsgThreads, 0, st>>>(s, d, K, n);
-    return cudaGetLastError();
+    return launch_ex(d, d.bf16 ? k_assign<true> : k_assign<false>, dim3(d.G), dim3(kAsgThreads), 0, st, s, d, K, n);
 }
 
 cudaError_t launch_append_rows(const Dims& d, const void* knew, const void* vnew, void* K, void* V, int row,

@@ -62,6 +62,23 @@ def test_tiny_edge_cases(kw):
     run_lockstep(cfg)
 
 
+def test_tied_scores_take_the_radix_passes():
+    # a zero query scores every community 0: the boundary bin of the linear
+    # pass holds all 1500 communities, so the selection narrows it by radix
+    # passes down to the ids (equal scores keep the lower ids first)
+    cfg = synth.scaled(synth.TINY, n0=24000, n_clusters=1500, budget=6000, steps=3)
+    assert cfg.n_comm > 1024
+    wl = synth.make_workload(cfg, workers=WORKERS)
+    wl.q[:] = 0
+    ls = Lockstep(wl)
+    try:
+        for i in range(cfg.steps):
+            ls.step(i)
+        ls.compare_state()
+    finally:
+        ls.close()
+
+
 def test_small_slack_relocates_segments():
     # slack 0: every append past the initial size moves the community segment
     cfg = synth.scaled(synth.TINY, n0=512, n_clusters=2, steps=40)
