@@ -381,14 +381,14 @@ def main():
     step_bytes = per_graph * cfg.n_graphs
     gbs = step_bytes * args.steps / (ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
-    names = ["score", "select", "attend", "assign"]
+    names = ["score", "select", "attend_edges_update", "step_close"]
     avg, roofline = None, None
     if kern_ms is not None and kern_steps:
         avg = {nm: kern_ms[k] / kern_steps for k, nm in enumerate(names)}
-        dom = max(("score", "attend"), key=lambda nm: avg[nm])
-        kb = kernel_bytes(cfg, T_mean)[dom] * cfg.n_graphs
+        dom = max(("score", "attend_edges_update"), key=lambda nm: avg[nm])
+        kb = kernel_bytes(cfg, T_mean)["attend" if dom != "score" else "score"] * cfg.n_graphs
         achieved = kb / (avg[dom] / 1e3) / 1e9
-        roofline = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": achieved, "peak": peak,
+        roofline = {"bound": "hbm", "kernel": "k_score" if dom == "score" else "k_attend", "achieved": achieved, "peak": peak,
                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                     "traffic": None, "algorithmic_bytes_per_launch": kb,
                     "avg_launch_ms": avg[dom]}
@@ -412,7 +412,7 @@ def main():
         "algorithmic_bytes_per_step": step_bytes, "mean_tokens_kept": T_mean,
         "kernel_ms_per_step": avg,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+        "gpu_launches": 3 * args.steps, "clocks": clk.summary(),
         "gen_seconds": t_gen,
     }
     print(json.dumps(line), flush=True)

@@ -121,31 +121,32 @@ ckv_status ckv_build_graph(int n_heads, int n, int head_dim, int n_sinks, int ka
 ckv_status ckv_init_communities(ckv_ctx* ctx, const int32_t* labels, int labels_on_device,
                                 int n_communities, const void* K, int n, void* stream);
 
-/* Decode step, first half -- Figure 1, step (3): for every graph, score the
- * query against every community centroid (QUERY_GROUP: summed over the
- * group's heads), keep communities in (score desc, id asc) order while their
- * sizes fit the budget (at least one), and run exact softmax attention of
- * each query head over the sinks, the kept members and the new token.
+/* Decode step -- Figure 1, step (3): for every graph, score the query
+ * against every community centroid (QUERY_GROUP: summed over the group's
+ * heads), keep communities in (score desc, id asc) order while their sizes
+ * fit the budget (at least one), run exact softmax attention of each query
+ * head over the sinks, the kept members and the new token; then (Figure 1,
+ * step (3) end, and Table 1's O(d) update) rank the kept members by their
+ * attention weight summed over the graph's heads, record the top kappa as
+ * the new token's edges, assign the token to the community with the largest
+ * summed edge weight (ties to the lower id) and update that centroid's
+ * running mean mu + (k - mu) / (m + 1), k being row n-1 of K.
  * q: [B][H_q][D] (kv_dtype); K, V: caches [B][H_kv][n_max][D] whose row
  * n-1 already holds the new token; n: cache length including the new token;
  * it must be one more than after the previous step (or init).
  * out: [B][H_q][D] float32, device.  Asynchronous.
  * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no init, wrong n, or the
- * previous step's ckv_assign_update missing), sticky device errors. */
+ * previous step's ckv_assign_update missing), sticky device errors;
+ * community storage exhaustion is reported by the next ckv_last_error() as
+ * CKV_ERR_CAPACITY and leaves that graph's state as it was before the
+ * step. */
 ckv_status ckv_decode_step(ckv_ctx* ctx, const void* q, const void* K, const void* V, int n,
                            float* out, void* stream);
 
-/* Decode step, second half -- Figure 1, step (3) end and Table 1's O(d)
- * update: for every graph, rank the kept members by their attention weight
- * (summed over the graph's heads) and record the top kappa as the new
- * token's edges; assign the token to the community with the largest summed
- * edge weight (ties to the lower id) and update that centroid's running
- * mean mu + (k - mu) / (m + 1).  K and n as in the preceding
- * ckv_decode_step.  Asynchronous.
- * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no preceding decode step),
- * sticky device errors; community storage exhaustion is reported by the
- * next ckv_last_error() as CKV_ERR_CAPACITY and leaves that graph's state
- * as it was before the step. */
+/* Closes the decode step begun by ckv_decode_step with the same n (the
+ * edges, assignment and update already ran inside that call's last kernel;
+ * this call launches nothing).  K must be non-NULL.
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no preceding decode step). */
 ckv_status ckv_assign_update(ckv_ctx* ctx, const void* K, int n, void* stream);
 
 /* One whole decode step from host memory: copies the new token's key and
@@ -175,10 +176,11 @@ ckv_status ckv_get_step_debug(ckv_ctx* ctx, int32_t* n_sel, int32_t* sel, int32_
  * Table 10 split of a step into retrieval and attention.  After
  * ckv_profile_begin, every ckv_decode_step / ckv_assign_update records CUDA
  * events on its stream around each of its kernels; ckv_profile_end
- * synchronises, writes the summed milliseconds of the four kernels
- * (ms[0] centroid scoring, ms[1] community selection, ms[2] gather +
- * attention, ms[3] edges + assignment + update) and the number of steps
- * they cover, and stops recording.  Both are host calls; begin is not
+ * synchronises, writes the summed milliseconds of ms[0] centroid scoring,
+ * ms[1] community selection, ms[2] gather + attention + edges + assignment
+ * + update (one kernel) and ms[3] the rest of the step (ckv_assign_update,
+ * which launches nothing), and the number of steps they cover, and stops
+ * recording.  Both are host calls; begin is not
  * allowed while a step is half done.  Errors: CKV_ERR_INVALID_ARG,
  * CKV_ERR_STATE, CKV_ERR_CUDA. */
 ckv_status ckv_profile_begin(ckv_ctx* ctx);

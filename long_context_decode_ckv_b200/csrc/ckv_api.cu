@@ -255,6 +255,7 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
                                  : (int64_t)cfg->n_max * 5 + (int64_t)cfg->max_communities * (cfg->slack + 32);
     // the attention grid: as many CTAs as can be co-resident
     d.nSM = sms;
+    d.fuse_assign = 1;
     {   // programmatic dependent launch between the decode kernels: off unless
         // CKV_PDL is 1 (each kernel lets the next one launch at its start) or
         // 2 (after its main work)
@@ -287,9 +288,6 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(part_ml, G * KC * HG * 2);
     ALLOC(part_o, G * KC * HG * ckv::kD);
     ALLOC(bar, G * 2);
-    ALLOC(cand_w, G * KC * kap);
-    ALLOC(cand_t, G * KC * kap);
-    ALLOC(cand_x, G * KC * kap);
     ALLOC(e_tok, G * kap);
     ALLOC(e_w, G * kap);
     ALLOC(e_comm, G * kap);
@@ -402,8 +400,9 @@ CKV_API ckv_status ckv_assign_update(ckv_ctx* x, const void* K, int n, void* str
     if (!x->pending || n != x->pending_n) return CKV_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     CKV_CUDA(cudaSetDevice(x->cfg.device));
+    // the attention kernel of ckv_decode_step already assigned the token and
+    // updated its community (it reads the new key from the same K)
     CKV_CUDA(prof_mark(x, 4, st));
-    CKV_CUDA(ckv::launch_assign(x->s, x->d, K, n, st));
     CKV_CUDA(prof_mark(x, 5, st));
     x->pending = 0;
     x->n_tok = n;

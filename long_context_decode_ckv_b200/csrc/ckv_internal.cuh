@@ -17,9 +17,7 @@
 //   zrow      float [G][NM][HG]    logits of the kept members (for the edges)
 //   part_ml   float [G][KC][HG][2] per-CTA softmax max and sum per head
 //   part_o    float [G][KC][HG][D] per-CTA P.V per head, relative to its max
-//   bar       uint  [G][2]         arrivals of a graph's CTAs: partials published
-//                                  (slot 0), edge candidates published (slot 1)
-//   cand_*    [G][KC][kappa]       each CTA's edge candidates (rank order)
+//   bar       uint  [G][2]         arrivals of a graph's slices (slot 0)
 //   e_*       [G][kappa]           the step's edges (rank order) for the update
 #pragma once
 
@@ -59,9 +57,6 @@ struct DevState {
     float* part_ml;
     float* part_o;
     unsigned int* bar;
-    float* cand_w;           // edge candidates of each attention CTA
-    int32_t* cand_t;
-    int32_t* cand_x;
     int32_t* e_tok;
     float* e_w;
     int32_t* e_comm;
@@ -75,16 +70,16 @@ struct Dims {
     int nSM;                 // multiprocessors of the device
     int n_comm;              // communities in use (set at init)
     int n_init;              // first decode position (edge store row 0)
+    int fuse_assign;         // the attention kernel also assigns the new token and updates
     int pdl;                 // programmatic dependent launch: 0 off, 1 trigger at kernel start, 2 after the main work
 };
 
 // kernel launchers (k_decode.cu)
 cudaError_t launch_score(const DevState& s, const Dims& d, const void* q, cudaStream_t st);
 cudaError_t launch_select(const DevState& s, const Dims& d, cudaStream_t st);
+// attention, edges and (d.fuse_assign) the assignment and update of the step
 cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const void* K,
                           const void* V, int n, float* out, cudaStream_t st);
-cudaError_t launch_assign(const DevState& s, const Dims& d, const void* K, int n,
-                          cudaStream_t st);
 size_t select_smem_bytes(int n_comm, int budget);
 // sets the kernels' shared-memory limits on the current device; then the
 // number of co-resident CTAs of the attention kernel (0 on error)

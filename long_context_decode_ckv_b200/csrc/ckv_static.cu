@@ -107,7 +107,7 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     // at most one CTA per 64 rows of the largest graph
     const int64_t rows_max = (int64_t)d.S + max_rows + 1;
     d.nCTA = (int)((rows_max + 63) / 64 < grid ? (rows_max + 63) / 64 : grid);
-    // scratch layout: meta | bar | err | edges | row list | logits | partials | candidates
+    // scratch layout: meta | bar | err | edges | row list | logits | partials
     const size_t KC = d.nCTA;
     size_t off = 0;
     const size_t o_meta = off;  off = align256(off + ckv::M_COUNT * 4);
@@ -120,7 +120,6 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     const size_t o_zrow = off;  off = align256(off + (size_t)rows_max * HG * 4);
     const size_t o_pml = off;   off = align256(off + KC * HG * 2 * 4);
     const size_t o_po = off;    off = align256(off + KC * HG * kD * 4);
-    const size_t o_cand = off;  off = align256(off + KC * 3 * 4);   // kappa = 1
     if (off > kStaticScratchBytes) return CKV_ERR_CAPACITY;   // max_rows too large for the array
     unsigned char* sb = static_cast<unsigned char*>(base);
     ckv::DevState s{};
@@ -135,9 +134,6 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     s.zrow = reinterpret_cast<float*>(sb + o_zrow);
     s.part_ml = reinterpret_cast<float*>(sb + o_pml);
     s.part_o = reinterpret_cast<float*>(sb + o_po);
-    s.cand_w = reinterpret_cast<float*>(sb + o_cand);
-    s.cand_t = reinterpret_cast<int32_t*>(sb + o_cand) + KC;
-    s.cand_x = reinterpret_cast<int32_t*>(sb + o_cand) + 2 * KC;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t eb = d.bf16 ? 2 : 4;

@@ -7,23 +7,22 @@
 // assign it to a community in constant time; Table 1: O(sqrt(n) d)
 // retrieval, O(d) update.
 //
-// Four kernels per step:
-//   k_score   centroid GEMV (HBM-bound), one warp per 32 communities, lane =
-//             4 dims, the 32 partial dots reduced by a butterfly transpose.
-//   k_select  one CTA per graph, the graph's scores and sizes held in shared
-//             memory: exact budgeted top-C by bucket passes (a monotone
-//             linear bucketing, then radix windows of the order-preserving
-//             score bits, then of the id) and an exact rank of the last
-//             <= 1024 candidates; writes the kept list and the kept rows.
-//   k_attend  one CTA per SM, each a slice of one graph's rows; every warp
+// Three kernels per step:
+//   k_score   centroid GEMV (HBM-bound): a persistent TMA ring of 16 KB
+//             units (32 communities), lane = 4 dims, the 32 partial dots
+//             reduced by a butterfly transpose.
+//   k_select  one CTA per graph, each thread's communities in registers:
+//             exact budgeted top-C by a size-weighted histogram linear in
+//             the score (radix passes over (score bits, id) only when the
+//             boundary bin is crowded) and an exact rank of the boundary
+//             bin; writes the kept list and the kept rows.
+//   k_attend  the graphs' rows split evenly over one CTA per SM; every warp
 //             gathers its own run of K and V rows (16-byte cp.async) and,
 //             for bf16, runs both contractions on the tensor cores
-//             (mma.sync) with an online softmax; once a graph's slices have
-//             published their (m, l, o) partials, each merges its share of
-//             the output and ranks its own kept members' edge weights, and
-//             the last one merges the candidate lists.
-//   k_assign  one CTA per graph: vote, capacity check, running-mean
-//             update, member append, edge row.
+//             (mma.sync) with an online softmax; the last slice of a graph
+//             to finish merges the (m, l, o) partials, ranks the kept
+//             members' edge weights, assigns the new token by weighted
+//             plurality and updates that community's running mean.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -40,7 +39,6 @@ namespace ckv {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kAsgThreads = 128;
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -502,8 +500,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
 // output and ranks its own kept members' edge weights w_j; the last slice
 // to finish merges the slices' candidate lists into the top-kappa edges.
 constexpr int kAttNBuf = 3;        // batches per warp pipeline
-constexpr int kEdgeRows = 4;       // kept-member rows a thread holds for the edge ranking
-static_assert(kMaxKappa == 32, "edge lists give one slot per lane");
 
 template <bool BF16, int HG>
 struct AttLayout {
@@ -511,12 +507,12 @@ struct AttLayout {
     static constexpr int RB = kD * (BF16 ? 2 : 4);               // bytes per K or V row
     static constexpr int BATCH = NB * 2 * RB;                    // K rows, then V rows
     static constexpr int WBUF = kAttNBuf * BATCH;                // one warp's pipeline
-    static constexpr int TOKW = 64;                              // row tokens a warp keeps at once
+    static constexpr int TOKW = 128;                             // row tokens a warp keeps at once
     static constexpr int off_buf = 0;
     static constexpr int off_pz = off_buf + kAttWarps * WBUF;    // fp32: [warps][NB*HG] z / p exchange
     static constexpr int off_tokw = off_pz + (BF16 ? 0 : kAttWarps * NB * HG * 4);   // [warps][TOKW]
     static constexpr int off_misc = off_tokw + kAttWarps * TOKW * 4;
-    static constexpr int bytes = off_misc + 256;
+    static constexpr int bytes = off_misc + 1280;
     // end-of-slice reduction [warps][HG][RSTR] reuses the pipelines; a row is
     // acc[0..D), m, l, padded to a multiple of 16 bytes for float4 access
     static constexpr int RSTR = kD + 4;
@@ -573,12 +569,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p)
-{
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 
 // Butterfly transpose-reduce of NV values per lane (NV a power of two
 // <= 32): afterwards every lane holds the warp-wide sum of value index
@@ -615,101 +605,6 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[NV], int lane)
     return r;
 }
 
-// Edge candidates of one warp in shared memory: a running list of the best
-// kappa (<= kMaxKappa) in slots [0, kMaxKappa) (w desc, token asc; w = -inf
-// marks an empty slot), new candidates in the block after it, and scratch
-// for the compaction.
-constexpr int kEdgeBlk = 128;                     // new candidates per selection round
-constexpr int kEdgeBuf = kMaxKappa + kEdgeBlk;
-static_assert(kEdgeRows * 32 <= kEdgeBlk, "a thread's rows fit one round");
-
-struct EdgeSlots {
-    float* w;
-    int* t;
-    int* x;
-    float* sw;
-    int* st;
-    int* sx;
-};
-
-__device__ __forceinline__ EdgeSlots edge_slots(unsigned char* base, int warp)
-{
-    float* f = reinterpret_cast<float*>(base) + warp * 6 * kEdgeBuf;
-    EdgeSlots e;
-    e.w = f;
-    e.t = reinterpret_cast<int*>(f + kEdgeBuf);
-    e.x = reinterpret_cast<int*>(f + 2 * kEdgeBuf);
-    e.sw = f + 3 * kEdgeBuf;
-    e.st = reinterpret_cast<int*>(f + 4 * kEdgeBuf);
-    e.sx = reinterpret_cast<int*>(f + 5 * kEdgeBuf);
-    return e;
-}
-
-__device__ __forceinline__ void edge_clear(const EdgeSlots& e, int lane)
-{
-    e.w[lane] = -INFINITY;   // kMaxKappa == 32 slots, one per lane
-    e.t[lane] = 0x7fffffff;
-    e.x[lane] = -1;
-}
-
-// list := the top kappa of the list and the block's nb candidates, by one
-// warp.  The kappa-th best of the lanes' best entries is a lower bound of
-// the answer (kappa distinct entries reach it), so only the entries at
-// least as good are compacted and ranked by counting.
-__device__ __forceinline__ void warp_select(const EdgeSlots& e, int nb, int kappa)
-{
-    const int lane = threadIdx.x & 31;
-    const int n = kMaxKappa + nb;
-    __syncwarp();
-    float bw = -INFINITY;
-    int bt = 0x7fffffff;
-    for (int i = lane; i < n; i += 32) {
-        const float w = e.w[i];
-        const int t = e.t[i];
-        if (w != -INFINITY && cand_better(w, t, bw, bt)) { bw = w; bt = t; }
-    }
-    float tw = -INFINITY;    // threshold (anything valid when fewer than kappa lanes hold one)
-    int tt = 0x7fffffff;
-    if (__popc(__ballot_sync(kFull, bw != -INFINITY)) >= kappa) {
-        int rank = 0;
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-            const float w2 = __shfl_sync(kFull, bw, i);
-            const int t2 = __shfl_sync(kFull, bt, i);
-            rank += cand_better(w2, t2, bw, bt) ? 1 : 0;
-        }
-        const int src = __ffs(__ballot_sync(kFull, bw != -INFINITY && rank == kappa - 1)) - 1;
-        tw = __shfl_sync(kFull, bw, src);
-        tt = __shfl_sync(kFull, bt, src);
-    }
-    int c = 0;
-    for (int i0 = 0; i0 < n; i0 += 32) {
-        const int i = i0 + lane;
-        float w = -INFINITY;
-        int t = 0x7fffffff, x = -1;
-        if (i < n) { w = e.w[i]; t = e.t[i]; x = e.x[i]; }
-        const bool ok = w != -INFINITY && !cand_better(tw, tt, w, t);
-        const unsigned bal = __ballot_sync(kFull, ok);
-        if (ok) {
-            const int p = c + __popc(bal & ((1u << lane) - 1u));
-            e.sw[p] = w;
-            e.st[p] = t;
-            e.sx[p] = x;
-        }
-        c += __popc(bal);
-    }
-    __syncwarp();
-    for (int i = lane; i < c; i += 32) {
-        const float w = e.sw[i];
-        const int t = e.st[i];
-        int r = 0;
-        for (int j = 0; j < c; ++j) r += cand_better(e.sw[j], e.st[j], w, t) ? 1 : 0;
-        if (r < kappa) { e.w[r] = w; e.t[r] = t; e.x[r] = e.sx[i]; }
-    }
-    for (int r = c + lane; r < kappa; r += 32) { e.w[r] = -INFINITY; e.t[r] = 0x7fffffff; e.x[r] = -1; }
-    __syncwarp();
-}
-
 // HG logits of one kept-member row (16-, 8- or 4-byte aligned by HG)
 template <int HG>
 __device__ __forceinline__ void load_logits(const float* p, float (&z)[HG])
@@ -726,6 +621,146 @@ __device__ __forceinline__ void load_logits(const float* p, float (&z)[HG])
     } else {
         z[0] = __ldcg(p);
     }
+}
+
+// Edge ranking of one graph by a whole CTA.  The kept members go by in
+// rounds of FR rows per thread (one round of loads each); the running top
+// kappa (w desc, token asc) sits in shared memory and joins every round as
+// extra entries of threads 0 .. kappa-1.  Per round: tau = the kappa-th
+// best of the threads' best entries is a lower bound of the answer, and
+// only the kappa threads whose best reaches tau can hold entries at least
+// that good, so at most kappa * (FR + 1) entries are compacted and ranked
+// by counting.
+constexpr int kFinMaxRows = 16;                                  // rows per thread and round
+constexpr int kFinCand = kMaxKappa * (kFinMaxRows + 1);           // compacted entries, at most
+
+struct EdgeScratch {
+    float lw[kMaxKappa];       // running list
+    int lt[kMaxKappa];
+    int lx[kMaxKappa];
+    float ww[kAttWarps][kMaxKappa];   // each warp's best lane-bests
+    int wt[kAttWarps][kMaxKappa];
+    float tw;                   // threshold
+    int tt;
+    int m;                      // compacted entries
+    float cw[kFinCand];
+    int ct[kFinCand];
+    int cx[kFinCand];
+};
+
+template <int HG>
+struct EdgeRows {
+    static constexpr int FR = (64 / HG < kFinMaxRows) ? 64 / HG : kFinMaxRows;   // rows per thread and round
+    float z[FR][HG];
+    int t[FR];
+};
+
+// one round's logits and tokens of this thread: rows j0 + tid + u * NT
+template <int HG>
+__device__ __forceinline__ void edges_load(const Dims& d, const float* __restrict__ zrow,
+                                           const int32_t* __restrict__ rtok, int T, int j0, EdgeRows<HG>& r)
+{
+    constexpr int NT = kAttWarps * 32;
+#pragma unroll
+    for (int u = 0; u < EdgeRows<HG>::FR; ++u) {
+        const int j = j0 + threadIdx.x + u * NT;
+        r.t[u] = 0;
+        if (j < T) {
+            load_logits<HG>(zrow + (int64_t)(d.S + j) * HG, r.z[u]);
+            r.t[u] = __ldcg(rtok + j);
+        }
+    }
+}
+
+// r holds round 0 (edges_load with j0 = 0) on entry
+template <int HG>
+__device__ __forceinline__ void cta_edges(const Dims& d, const float* __restrict__ zrow,
+                                          const int32_t* __restrict__ rtok, int T, const float* sM,
+                                          const float* sL, EdgeScratch& e, EdgeRows<HG>& r)
+{
+    constexpr int NT = kAttWarps * 32;
+    constexpr int FR = EdgeRows<HG>::FR;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int kappa = d.kappa;
+    if (tid < kMaxKappa) { e.lw[tid] = -INFINITY; e.lt[tid] = 0x7fffffff; e.lx[tid] = -1; }
+    for (int j0 = 0; j0 < max(T, 1); j0 += FR * NT) {
+        if (j0 > 0) edges_load<HG>(d, zrow, rtok, T, j0, r);
+        float w[FR + 1];
+        int t[FR + 1];
+#pragma unroll
+        for (int u = 0; u < FR; ++u) {
+            const int j = j0 + tid + u * NT;
+            float sw = 0.f;
+#pragma unroll
+            for (int h = 0; h < HG; ++h) sw += __expf(r.z[u][h] - sM[h]) * sL[h];
+            w[u] = (j < T) ? sw : -INFINITY;
+            t[u] = r.t[u];
+        }
+        __syncthreads();   // the running list is complete
+        // the running list's entry `tid` joins as the thread's extra entry
+        w[FR] = (tid < kappa) ? e.lw[tid] : -INFINITY;
+        t[FR] = (tid < kappa) ? e.lt[tid] : 0x7fffffff;
+        const int xl = (tid < kappa) ? e.lx[tid] : -1;
+        float bw = -INFINITY;
+        int bt = 0x7fffffff;
+#pragma unroll
+        for (int u = 0; u <= FR; ++u)
+            if (w[u] != -INFINITY && cand_better(w[u], t[u], bw, bt)) { bw = w[u]; bt = t[u]; }
+        // each warp's best kappa lane-bests
+        int rank = 0;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const float w2 = __shfl_sync(kFull, bw, i);
+            const int t2 = __shfl_sync(kFull, bt, i);
+            rank += cand_better(w2, t2, bw, bt) ? 1 : 0;
+        }
+        if (lane < kappa) { e.ww[warp][lane] = -INFINITY; e.wt[warp][lane] = 0x7fffffff; }
+        __syncwarp();
+        if (rank < kappa && bw != -INFINITY) { e.ww[warp][rank] = bw; e.wt[warp][rank] = bt; }
+        if (tid == 0) { e.tw = -INFINITY; e.tt = 0x7fffffff; e.m = 0; }
+        __syncthreads();
+        // tau: the kappa-th best of the warps' lists (anything, when fewer exist)
+        if (tid < kAttWarps * kappa) {
+            const float mw = e.ww[tid / kappa][tid % kappa];
+            const int mt = e.wt[tid / kappa][tid % kappa];
+            if (mw != -INFINITY) {
+                int rr = 0;
+                for (int wi = 0; wi < kAttWarps; ++wi)
+                    for (int ki = 0; ki < kappa; ++ki) {
+                        const float w2 = e.ww[wi][ki];
+                        rr += (w2 != -INFINITY && cand_better(w2, e.wt[wi][ki], mw, mt)) ? 1 : 0;
+                    }
+                if (rr == kappa - 1) { e.tw = mw; e.tt = mt; }
+            }
+        }
+        __syncthreads();
+        // compact the entries at least as good as tau
+        const float tw = e.tw;
+        const int tt = e.tt;
+#pragma unroll
+        for (int u = 0; u <= FR; ++u) {
+            if (w[u] != -INFINITY && !cand_better(tw, tt, w[u], t[u])) {
+                const int slot = atomicAdd(&e.m, 1);
+                if (slot < kFinCand) {
+                    e.cw[slot] = w[u];
+                    e.ct[slot] = t[u];
+                    e.cx[slot] = (u < FR) ? j0 + tid + u * NT : xl;
+                }
+            }
+        }
+        __syncthreads();
+        // rank them; the first kappa become the running list
+        const int m = min(e.m, kFinCand);
+        for (int i = tid; i < m; i += NT) {
+            const float mw = e.cw[i];
+            const int mt = e.ct[i];
+            int rr = 0;
+            for (int j = 0; j < m; ++j) rr += cand_better(e.cw[j], e.ct[j], mw, mt) ? 1 : 0;
+            if (rr < kappa) { e.lw[rr] = mw; e.lt[rr] = mt; e.lx[rr] = e.cx[i]; }
+        }
+        for (int i = m + tid; i < kappa; i += NT) { e.lw[i] = -INFINITY; e.lt[i] = 0x7fffffff; e.lx[i] = -1; }
+    }
+    __syncthreads();
 }
 
 // Rows of one warp: [a0, a1) in the graph's row numbering (sinks, kept
@@ -1025,6 +1060,161 @@ __device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __
     }
 }
 
+// A graph's last slice to finish: merge the slices' partials, rank the
+// edges, and (when fused) assign the new token and update its community.
+// Runs with the whole CTA; red / smem scratch is free.
+template <int HG>
+__device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, int g, int nc, int R,
+                                             const void* __restrict__ K, int n, float* __restrict__ out,
+                                             unsigned char* scratch, float* sM, float* sL, int* sflag)
+{
+    constexpr int NT = kAttWarps * 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int b, h0, kvh;
+    graph_heads(d, g, b, h0, kvh);
+    const int T = R - d.S - 1;
+    const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
+    const float* zrow = s.zrow + (int64_t)g * d.NM * HG;
+    const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
+    const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
+
+    EdgeRows<HG> er;   // the first round of kept members, loaded under the output merge
+    edges_load<HG>(d, zrow, rtok, T, 0, er);
+    // ---- output: every value merged online over the slices; the thread of
+    // a head's first value also leaves that head's max and 1 / sum
+    for (int i = tid; i < HG * kD; i += NT) {
+        const int h = i / kD;
+        float M = -INFINITY, Ls = 0.f, o = 0.f;
+        for (int j0 = 0; j0 < nc; j0 += 8) {   // 8 slices' loads in flight at once
+            float2 mj[8];
+            float oj[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool ok = j0 + u < nc;
+                mj[u] = ok ? __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)(j0 + u) * HG + h) * 2))
+                           : make_float2(-INFINITY, 0.f);
+                oj[u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (mj[u].x == -INFINITY) continue;
+                const float mn = fmaxf(M, mj[u].x);
+                const float a = (M == -INFINITY) ? 0.f : __expf(M - mn), c = __expf(mj[u].x - mn);
+                o = o * a + oj[u] * c;
+                Ls = Ls * a + mj[u].y * c;
+                M = mn;
+            }
+        }
+        out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o / Ls;
+        if (i % kD == 0) { sM[h] = M; sL[h] = 1.f / Ls; }
+    }
+    __syncthreads();
+    // ---- edges: the top kappa of w = sum_h exp(z - M_h) / L_h over the kept members
+    EdgeScratch& es = *reinterpret_cast<EdgeScratch*>(scratch);
+    cta_edges<HG>(d, zrow, rtok, T, sM, sL, es, er);
+    if (warp == 0) {
+        const bool real = lane < d.kappa && es.lw[lane] != -INFINITY;
+        const int ne = __popc(__ballot_sync(kFull, real));
+        const int cm = real ? __ldcg(s.rcomm + (int64_t)g * d.NM + es.lx[lane]) : 0;
+        if (real) {
+            s.e_w[(int64_t)g * d.kappa + lane] = es.lw[lane];
+            s.e_tok[(int64_t)g * d.kappa + lane] = es.lt[lane];
+            s.e_comm[(int64_t)g * d.kappa + lane] = cm;
+        }
+        if (lane == 0) s.meta[(int64_t)g * M_COUNT + M_NEDGE] = ne;
+        if (d.fuse_assign) {
+            // every candidate community's counters, fetched under the vote
+            int32_t* csz = s.csize + (int64_t)g * d.Nc;
+            int32_t* coff = s.coff + (int64_t)g * d.Nc;
+            int32_t* ccap = s.ccap + (int64_t)g * d.Nc;
+            const int c_any = real ? cm : 0;
+            const int p_size = csz[c_any], p_cap = ccap[c_any], p_off = coff[c_any];
+            const int p_top = s.pool_top[g];
+            // weighted plurality of the edges' communities: each lane sums
+            // its community's weights in rank order (double), ties to the
+            // lower id
+            double v = 0.0;
+            for (int e = 0; e < ne; ++e) {
+                const int ce = __shfl_sync(kFull, cm, e);
+                const float we = __shfl_sync(kFull, es.lw[lane], e);
+                if (ce == cm) v += (double)we;
+            }
+            double bv = real ? v : -1.0;
+            int bc = real ? cm : 0x7fffffff;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const double v2 = __shfl_xor_sync(kFull, bv, o);
+                const int c2 = __shfl_xor_sync(kFull, bc, o);
+                if (v2 > bv || (v2 == bv && c2 < bc)) { bv = v2; bc = c2; }
+            }
+            const int c = (ne == 0) ? 0 : bc;
+            const int src = (ne == 0) ? 0 : __ffs(__ballot_sync(kFull, real && cm == c)) - 1;
+            const int size = __shfl_sync(kFull, p_size, src), cp = __shfl_sync(kFull, p_cap, src);
+            const int off0 = __shfl_sync(kFull, p_off, src), top = p_top;
+            if (lane == 0) {
+                int ok = 1, off = off0;
+                if (size == cp) {   // segment full: move it to the pool top with twice the room
+                    const int ncap = max(16, 2 * cp);
+                    if ((int64_t)top + ncap > d.P) ok = 0;
+                    else { s.pool_top[g] = top + ncap; off = top; }
+                }
+                if (!ok) set_error(s.err, CKV_ERR_CAPACITY);
+                sflag[0] = c; sflag[1] = ok; sflag[2] = off; sflag[3] = size; sflag[4] = off0; sflag[5] = ne;
+            }
+        }
+    }
+    if (!d.fuse_assign) return;
+    __syncthreads();
+    if (!sflag[1]) return;
+    const int c = sflag[0], off = sflag[2], size = sflag[3], old_off = sflag[4], ne = sflag[5];
+    const int t = n - 1;
+    int32_t* pool = s.pool + (int64_t)g * d.P;
+    if (off != old_off)
+        for (int i = tid; i < size; i += NT) pool[off + i] = pool[old_off + i];
+    // running-mean update of the assigned centroid, double math rounded once
+    if (tid < kD) {
+        const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + t) * kD;
+        const double kv = d.bf16 ? (double)elem<true>(K, krow + tid) : (double)elem<false>(K, krow + tid);
+        float* mu = s.mu + ((int64_t)g * d.Nc + c) * kD;
+        const double mv = (double)mu[tid];
+        mu[tid] = __double2float_rn(__dadd_rn(mv, __ddiv_rn(__dsub_rn(kv, mv), (double)(size + 1))));
+    }
+    __syncthreads();   // the segment copy is complete before the append
+    const int64_t row = (int64_t)g * (d.NM - d.n_init) + (t - d.n_init);
+    if (tid == 0) {
+        if (off != old_off) {
+            s.coff[(int64_t)g * d.Nc + c] = off;
+            s.ccap[(int64_t)g * d.Nc + c] = max(16, 2 * s.ccap[(int64_t)g * d.Nc + c]);
+        }
+        pool[off + size] = t;
+        s.csize[(int64_t)g * d.Nc + c] = size + 1;
+        s.tok_comm[(int64_t)g * d.NM + t] = c;
+        s.meta[(int64_t)g * M_COUNT + M_ASSIGNED] = c;
+        s.edge_deg[row] = ne;
+    }
+    if (tid < ne) {
+        s.edge_col[row * d.kappa + tid] = s.e_tok[(int64_t)g * d.kappa + tid];
+        s.edge_w[row * d.kappa + tid] = s.e_w[(int64_t)g * d.kappa + tid];
+    }
+}
+
+// CTA work: the graphs' rows laid end to end (graph-major, each graph's
+// rows in its own order) are split evenly over the CTAs; a CTA's share is
+// one or more pieces, each a contiguous run of one graph's rows.
+struct Piece {
+    int g, r0, r1;     // graph and its rows [r0, r1)
+    int k, nc;         // slice index of the piece among the graph's nc slices
+    int R;             // the graph's rows
+};
+constexpr int kMaxPieces = 32;
+
+// the CTA whose share holds global row x: shares are [lo(i), lo(i+1)) with
+// lo(i) = floor(i * tot / P), so the last i with lo(i) <= x
+__device__ __forceinline__ int share_of(long long x, long long tot, int P)
+{
+    return (int)(((x + 1) * P - 1) / tot);
+}
+
 template <bool BF16, int HG>
 __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d, const void* __restrict__ q,
                                                              const void* __restrict__ K,
@@ -1036,370 +1226,145 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
     constexpr int NT = kAttWarps * 32;
     pdl_wait();
     if (d.pdl == 1) pdl_trigger();
-    if (*(volatile int*)s.err) return;
     extern __shared__ __align__(128) unsigned char smem[];
     float* sM = reinterpret_cast<float*>(smem + L::off_misc);          // [8] graph max per head
     float* sL = sM + 8;                                                // [8] 1 / graph sum per head
-    int* sidx = reinterpret_cast<int*>(sL + 8);                        // [warps]
-    int* sh_seg = sidx + kAttWarps;                                    // graph, slice, slices, last, ok
+    int* sflag = reinterpret_cast<int*>(sL + 8);                       // [8]
+    int* snp = sflag + 8;                                              // [1] pieces of this CTA
+    int* snf = snp + 1;                                                // [1] graphs it finishes
+    Piece* sp = reinterpret_cast<Piece*>(snp + 4);                     // [kMaxPieces]
+    int* sfin = reinterpret_cast<int*>(sp + kMaxPieces);               // [kMaxPieces] their pieces
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nCTA = gridDim.x, bid = blockIdx.x;
     const int G = d.G;
     unsigned char* wbuf = smem + L::off_buf + warp * L::WBUF;
     int* tokw = reinterpret_cast<int*>(smem + L::off_tokw) + warp * L::TOKW;
     float* red = reinterpret_cast<float*>(smem + L::off_buf);          // [warps][HG][RSTR]
 
-    // ---- which graph slice(s) this CTA owns.  G <= nCTA: every graph gets
-    // one CTA plus a share of the others proportional to its rows, and each
-    // CTA owns one contiguous slice of one graph.  G > nCTA: each CTA owns
-    // whole graphs.
-    int g_first, g_last;
-    if (G > nCTA) {
-        g_first = (int)((int64_t)bid * G / nCTA);
-        g_last = (int)((int64_t)(bid + 1) * G / nCTA);
-    } else {
-        // rows of every graph, staged once; warp 0 then forms their prefix
-        // and the first CTA of each graph, f(g) = g + floor(P_g * extra / R_tot)
-        int* sR = reinterpret_cast<int*>(smem + L::off_buf);
-        for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
-        __syncthreads();
+    // ---- this CTA's pieces.  The graphs' rows and the error word in one
+    // round of loads; then warp 0 lists the pieces, kMaxPieces at a time
+    // (a later round reloads the rows: the staging area is reused)
+    int* sR = reinterpret_cast<int*>(smem + L::off_buf);
+    for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
+    const int errv = *(volatile int*)s.err;
+    __syncthreads();
+    if (errv) return;
+    for (int done = 0;; done += kMaxPieces) {
         if (warp == 0) {
-            const int extra = nCTA - G;
-            double R_tot = 0.0;
-            for (int g0 = 0; g0 < G; g0 += 32) {
-                const int g = g0 + lane;
-                R_tot += (g < G) ? (double)sR[g] : 0.0;
-            }
+            auto rows_of = [&](int g) -> int {
+                return done == 0 ? sR[g] : __ldcg(s.meta + (int64_t)g * M_COUNT + M_ROWS);
+            };
+            long long tot = 0;
+            for (int g0 = 0; g0 < G; g0 += 32) tot += (g0 + lane < G) ? rows_of(g0 + lane) : 0;
 #pragma unroll
-            for (int o = 16; o; o >>= 1) R_tot += __shfl_xor_sync(kFull, R_tot, o);
-            double carry = 0.0;
-            for (int g0 = 0; g0 < G; g0 += 32) {
+            for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(kFull, tot, o);
+            const int P = (int)min((long long)gridDim.x, tot);
+            const long long A = (long long)blockIdx.x * tot / P, B = (long long)(blockIdx.x + 1) * tot / P;
+            int np = 0;                            // pieces seen so far
+            long long carry = 0;
+            for (int g0 = 0; g0 < G && (int)blockIdx.x < P; g0 += 32) {
                 const int g = g0 + lane;
-                const double R = (g < G) ? (double)sR[g] : 0.0;
-                double incl = R;
+                const int R = (g < G) ? rows_of(g) : 0;
+                long long incl = R;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    const double t = __shfl_up_sync(kFull, incl, o);
+                    const long long t = __shfl_up_sync(kFull, incl, o);
                     if (lane >= o) incl += t;
                 }
-                const double P = carry + incl - R;
-                const int f = g + (int)floor(P * extra / R_tot);
-                const int f1 = g + 1 + (int)floor((P + R) * extra / R_tot);
-                if (g < G && bid >= f && bid < f1) {
-                    sh_seg[0] = g;
-                    sh_seg[1] = bid - f;
-                    sh_seg[2] = f1 - f;
+                const long long Pg = carry + incl - R;
+                const bool mine = g < G && Pg < B && Pg + R > A;
+                const unsigned bal = __ballot_sync(kFull, mine);
+                if (mine) {
+                    const int slot = np + __popc(bal & ((1u << lane) - 1u)) - done;
+                    if (slot >= 0 && slot < kMaxPieces) {
+                        Piece pc;
+                        pc.g = g;
+                        pc.r0 = (int)(max(A, Pg) - Pg);
+                        pc.r1 = (int)(min(B, Pg + R) - Pg);
+                        const int f = share_of(Pg, tot, P);
+                        pc.k = (int)blockIdx.x - f;
+                        pc.nc = share_of(Pg + R - 1, tot, P) - f + 1;
+                        pc.R = R;
+                        sp[slot] = pc;
+                    }
                 }
+                np += __popc(bal);
                 carry += __shfl_sync(kFull, incl, 31);
             }
+            if (lane == 0) { *snp = max(0, min(np - done, kMaxPieces)); *snf = 0; }
         }
         __syncthreads();
-        g_first = sh_seg[0];
-        g_last = g_first + 1;
-    }
-
-    for (int g = g_first; g < g_last; ++g) {
-        const int k = (G > nCTA) ? 0 : sh_seg[1];
-        const int nc = (G > nCTA) ? 1 : sh_seg[2];
-        int b, h0, kvh;
-        graph_heads(d, g, b, h0, kvh);
-        const int R = s.meta[(int64_t)g * M_COUNT + M_ROWS];
-        const int T = R - d.S - 1;
-        const int r0 = (int)((int64_t)k * R / nc), r1 = (int)((int64_t)(k + 1) * R / nc);
-        const int nrows = r1 - r0;
-        const int64_t kvbase = ((int64_t)b * d.Hkv + kvh) * d.NM;
-        const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
-        float* zrow = s.zrow + (int64_t)g * d.NM * HG;
-        WarpRows a;
-        a.Kb = reinterpret_cast<const char*>(K) + kvbase * RB;
-        a.Vb = reinterpret_cast<const char*>(V) + kvbase * RB;
-        a.rtok = rtok;
-        a.zrow = zrow;
-        a.a0 = r0 + (int)((int64_t)warp * nrows / kAttWarps);
-        a.a1 = r0 + (int)((int64_t)(warp + 1) * nrows / kAttWarps);
-        a.S = d.S;
-        a.T = T;
-        a.R = R;
-        a.t_new = n - 1;
-        __syncthreads();   // the previous graph of this CTA is done with the buffers
-        if constexpr (BF16) {
-            const uint32_t* q2 = reinterpret_cast<const uint32_t*>(q) + ((int64_t)b * d.Hq + h0) * kD / 2;
-            warp_rows_mma<HG>(a, q2, wbuf, tokw, red);
-        } else {
-            const float* qg = reinterpret_cast<const float*>(q) + ((int64_t)b * d.Hq + h0) * kD;
-            float* pz = reinterpret_cast<float*>(smem + L::off_pz) + warp * L::NB * HG;
-            warp_rows_fma<HG>(a, qg, wbuf, tokw, pz, red);
-        }
-        __syncthreads();
-        // combine the warps: (m, l, acc) -> this slice's partial per head
-        float* po = s.part_o + ((int64_t)g * d.nCTA + k) * HG * kD;
-        float* pm = s.part_ml + ((int64_t)g * d.nCTA + k) * HG * 2;
-        for (int i = tid; i < HG * kD; i += NT) {
-            const int h = i / kD, dd = i % kD;
-            float mw[kAttWarps];
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kAttWarps; ++w) {
-                mw[w] = red[(w * HG + h) * L::RSTR + kD];
-                M = fmaxf(M, mw[w]);
+        const int npieces = *snp;
+        for (int pi = 0; pi < npieces; ++pi) {
+            const Piece pc = sp[pi];
+            const int g = pc.g, k = pc.k, nc = pc.nc, R = pc.R;
+            int b, h0, kvh;
+            graph_heads(d, g, b, h0, kvh);
+            const int T = R - d.S - 1;
+            const int nrows = pc.r1 - pc.r0;
+            const int64_t kvbase = ((int64_t)b * d.Hkv + kvh) * d.NM;
+            WarpRows a;
+            a.Kb = reinterpret_cast<const char*>(K) + kvbase * RB;
+            a.Vb = reinterpret_cast<const char*>(V) + kvbase * RB;
+            a.rtok = s.rtok + (int64_t)g * d.NM;
+            a.zrow = s.zrow + (int64_t)g * d.NM * HG;
+            a.a0 = pc.r0 + (int)((int64_t)warp * nrows / kAttWarps);
+            a.a1 = pc.r0 + (int)((int64_t)(warp + 1) * nrows / kAttWarps);
+            a.S = d.S;
+            a.T = T;
+            a.R = R;
+            a.t_new = n - 1;
+            __syncthreads();   // the previous piece of this CTA is done with the buffers
+            if constexpr (BF16) {
+                const uint32_t* q2 = reinterpret_cast<const uint32_t*>(q) + ((int64_t)b * d.Hq + h0) * kD / 2;
+                warp_rows_mma<HG>(a, q2, wbuf, tokw, red);
+            } else {
+                const float* qg = reinterpret_cast<const float*>(q) + ((int64_t)b * d.Hq + h0) * kD;
+                float* pz = reinterpret_cast<float*>(smem + L::off_pz) + warp * L::NB * HG;
+                warp_rows_fma<HG>(a, qg, wbuf, tokw, pz, red);
             }
-            float o = 0.f, l = 0.f;
+            __syncthreads();
+            // combine the warps: (m, l, acc) -> this slice's partial per head
+            float* po = s.part_o + ((int64_t)g * d.nCTA + k) * HG * kD;
+            float* pm = s.part_ml + ((int64_t)g * d.nCTA + k) * HG * 2;
+            for (int i = tid; i < HG * kD; i += NT) {
+                const int h = i / kD, dd = i % kD;
+                float mw[kAttWarps];
+                float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kAttWarps; ++w) {
-                const float* rw = red + (w * HG + h) * L::RSTR;
-                const float f = (mw[w] == -INFINITY) ? 0.f : __expf(mw[w] - M);
-                o = fmaf(rw[dd], f, o);
-                l = fmaf(rw[kD + 1], f, l);
-            }
-            po[i] = o;
-            if (dd == 0) *reinterpret_cast<float2*>(pm + h * 2) = make_float2(M, l);
-        }
-        // this thread's kept-member rows of the slice (logits written by this
-        // CTA's warps), loaded before the wait
-        const int js = max(r0, d.S) - d.S, je = min(r1, d.S + T) - d.S;
-        float zr[kEdgeRows][HG];
-        int tr[kEdgeRows];
-#pragma unroll
-        for (int u = 0; u < kEdgeRows; ++u) {
-            const int j = js + tid + u * NT;
-            tr[u] = 0;
-#pragma unroll
-            for (int h = 0; h < HG; ++h) zr[u][h] = -INFINITY;
-            if (j < je) {
-                load_logits<HG>(zrow + (int64_t)(d.S + j) * HG, zr[u]);
-                tr[u] = __ldcg(rtok + j);
-            }
-        }
-        // ---- wait until every slice of the graph has published
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) {
-            atomicAdd(&s.bar[g * 2], 1u);
-            int ok = 0;
-            for (unsigned it = 0; it < kWaitLimit; ++it) {
-                if (ld_acquire(&s.bar[g * 2]) >= (unsigned)nc) { ok = 1; break; }
-                if ((it & 255) == 255 && *(volatile int*)s.err) break;
-            }
-            if (!ok) set_error(s.err, CKV_ERR_TIMEOUT);
-            sh_seg[4] = ok;
-        }
-        __syncthreads();
-        if (!sh_seg[4]) return;
-        if (d.pdl == 2) pdl_trigger();
-        const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
-        const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
-        if (warp >= kAttWarps - HG) {   // the graph's exact softmax max and 1 / sum per head
-            const int h = warp - (kAttWarps - HG);
-            float M = -INFINITY, Ls = 0.f;
-            for (int j = lane; j < nc; j += 32) {   // online over this lane's slices
-                const float2 ml = __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)j * HG + h) * 2));
-                if (ml.x != -INFINITY) {
-                    const float mn = fmaxf(M, ml.x);
-                    Ls = Ls * ((M == -INFINITY) ? 0.f : __expf(M - mn)) + ml.y * __expf(ml.x - mn);
-                    M = mn;
+                for (int w = 0; w < kAttWarps; ++w) {
+                    mw[w] = red[(w * HG + h) * L::RSTR + kD];
+                    M = fmaxf(M, mw[w]);
                 }
-            }
+                float o = 0.f, l = 0.f;
 #pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                const float M2 = __shfl_xor_sync(kFull, M, o), L2 = __shfl_xor_sync(kFull, Ls, o);
-                const float mn = fmaxf(M, M2);
-                if (mn != -INFINITY)
-                    Ls = ((M == -INFINITY) ? 0.f : Ls * __expf(M - mn)) + ((M2 == -INFINITY) ? 0.f : L2 * __expf(M2 - mn));
-                M = mn;
-            }
-            if (lane == 0) { sM[h] = M; sL[h] = 1.f / Ls; }
-        }
-        {   // this slice's share of the output: each value merged online over the slices
-            const int i0 = (int)((int64_t)k * HG * kD / nc), i1 = (int)((int64_t)(k + 1) * HG * kD / nc);
-            for (int i = i0 + tid; i < i1; i += NT) {
-                const int h = i / kD;
-                float M = -INFINITY, Ls = 0.f, o = 0.f;
-                for (int j0 = 0; j0 < nc; j0 += 8) {   // 8 slices' loads in flight at once
-                    float2 mj[8];
-                    float oj[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const bool ok = j0 + u < nc;
-                        mj[u] = ok ? __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)(j0 + u) * HG + h) * 2))
-                                   : make_float2(-INFINITY, 0.f);
-                        oj[u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        if (mj[u].x == -INFINITY) continue;
-                        const float mn = fmaxf(M, mj[u].x);
-                        const float a = (M == -INFINITY) ? 0.f : __expf(M - mn), c = __expf(mj[u].x - mn);
-                        o = o * a + oj[u] * c;
-                        Ls = Ls * a + mj[u].y * c;
-                        M = mn;
-                    }
+                for (int w = 0; w < kAttWarps; ++w) {
+                    const float* rw = red + (w * HG + h) * L::RSTR;
+                    const float f = (mw[w] == -INFINITY) ? 0.f : __expf(mw[w] - M);
+                    o = fmaf(rw[dd], f, o);
+                    l = fmaf(rw[kD + 1], f, l);
                 }
-                out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o / Ls;
+                po[i] = o;
+                if (dd == 0) *reinterpret_cast<float2*>(pm + h * 2) = make_float2(M, l);
             }
-        }
-        __syncthreads();   // sM, sL
-        // ---- edge candidates: the slice's top kappa of w = sum_h exp(z - M_h) / L_h
-        const EdgeSlots es = edge_slots(smem + L::off_buf, warp);
-        edge_clear(es, lane);
-#pragma unroll
-        for (int u = 0; u < kEdgeRows; ++u) {
-            const int j = js + tid + u * NT;
-            float w = 0.f;
-#pragma unroll
-            for (int h = 0; h < HG; ++h) w += __expf(zr[u][h] - sM[h]) * sL[h];
-            es.w[kMaxKappa + u * 32 + lane] = (j < je) ? w : -INFINITY;
-            es.t[kMaxKappa + u * 32 + lane] = tr[u];
-            es.x[kMaxKappa + u * 32 + lane] = j;
-        }
-        warp_select(es, kEdgeRows * 32, d.kappa);
-        for (int j0 = js + kEdgeRows * NT; j0 < je; j0 += kEdgeRows * NT) {   // slices longer than the registers hold
-            for (int u = 0; u < kEdgeRows; ++u) {
-                const int j = j0 + tid + u * NT;
-                float w = -INFINITY;
-                int t = 0;
-                if (j < je) {
-                    float z[HG];
-                    load_logits<HG>(zrow + (int64_t)(d.S + j) * HG, z);
-                    w = 0.f;
-#pragma unroll
-                    for (int h = 0; h < HG; ++h) w += __expf(z[h] - sM[h]) * sL[h];
-                    t = __ldcg(rtok + j);
-                }
-                es.w[kMaxKappa + u * 32 + lane] = w;
-                es.t[kMaxKappa + u * 32 + lane] = t;
-                es.x[kMaxKappa + u * 32 + lane] = j;
-            }
-            warp_select(es, kEdgeRows * 32, d.kappa);
-        }
-        __syncthreads();
-        const int64_t cbase = (int64_t)g * d.nCTA * d.kappa;
-        if (warp == 0) {   // the slice's list from its warps' lists
-            const int per = kEdgeBlk / d.kappa;   // whole lists per round
-            for (int w0 = 1; w0 < kAttWarps; w0 += per) {
-                const int nw = min(per, kAttWarps - w0);
-                for (int i = lane; i < nw * d.kappa; i += 32) {
-                    const EdgeSlots o = edge_slots(smem + L::off_buf, w0 + i / d.kappa);
-                    es.w[kMaxKappa + i] = o.w[i % d.kappa];
-                    es.t[kMaxKappa + i] = o.t[i % d.kappa];
-                    es.x[kMaxKappa + i] = o.x[i % d.kappa];
-                }
-                warp_select(es, nw * d.kappa, d.kappa);
-            }
-            if (lane < d.kappa) {
-                const int64_t o = cbase + (int64_t)k * d.kappa + lane;
-                s.cand_w[o] = es.w[lane];
-                s.cand_t[o] = es.t[lane];
-                s.cand_x[o] = es.x[lane];
-            }
+            // ---- the last slice of a graph to arrive finishes it
             __threadfence();
-            __syncwarp();
-            int last = 0;
-            if (lane == 0) last = (atomicAdd(&s.bar[g * 2 + 1], 1u) == (unsigned)nc - 1);
-            last = __shfl_sync(kFull, last, 0);
-            if (last) {   // the last slice: merge the slices' lists
-                __threadfence();
-                edge_clear(es, lane);
-                const int ncand = nc * d.kappa;
-                for (int e0 = 0; e0 < ncand; e0 += kEdgeBlk) {
-                    const int nb = min(kEdgeBlk, ncand - e0);
-                    for (int i = lane; i < nb; i += 32) {
-                        es.w[kMaxKappa + i] = __ldcg(s.cand_w + cbase + e0 + i);
-                        es.t[kMaxKappa + i] = __ldcg(s.cand_t + cbase + e0 + i);
-                        es.x[kMaxKappa + i] = __ldcg(s.cand_x + cbase + e0 + i);
-                    }
-                    warp_select(es, nb, d.kappa);
-                }
-                const int ne = __popc(__ballot_sync(kFull, lane < d.kappa && es.w[lane] != -INFINITY));
-                if (lane < ne) {
-                    s.e_w[(int64_t)g * d.kappa + lane] = es.w[lane];
-                    s.e_tok[(int64_t)g * d.kappa + lane] = es.t[lane];
-                    s.e_comm[(int64_t)g * d.kappa + lane] = s.rcomm[(int64_t)g * d.NM + es.x[lane]];
-                }
-                if (lane == 0) {
-                    s.meta[(int64_t)g * M_COUNT + M_NEDGE] = ne;
-                    s.bar[g * 2] = 0u;
-                    s.bar[g * 2 + 1] = 0u;
-                }
-            }
+            __syncthreads();
+            if (tid == 0 && atomicAdd(&s.bar[g * 2], 1u) == (unsigned)nc - 1) sfin[(*snf)++] = pi;
         }
-    }
-}
-
-// --------------------------------------------------------------- k_assign
-template <bool BF16>
-__global__ void __launch_bounds__(kAsgThreads) k_assign(DevState s, Dims d, const void* __restrict__ K, int n)
-{
-    pdl_wait();
-    if (d.pdl) pdl_trigger();
-    if (*(volatile int*)s.err) return;
-    __shared__ int e_c[kMaxKappa];
-    __shared__ float e_w[kMaxKappa];
-    __shared__ int s_c, s_ok, s_off, s_size, s_oldoff, s_E;
-    const int g = blockIdx.x;
-    const int tid = threadIdx.x;
-    int b, h0, kvh;
-    graph_heads(d, g, b, h0, kvh);
-    const int t = n - 1;
-    // the new token's key (independent of the vote) and the step's edges
-    const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + t) * kD;
-    const double kv = (double)elem<BF16>(K, krow + tid);
-    const int E = s.meta[(int64_t)g * M_COUNT + M_NEDGE];
-    if (tid < E) {
-        e_c[tid] = s.e_comm[(int64_t)g * d.kappa + tid];
-        e_w[tid] = s.e_w[(int64_t)g * d.kappa + tid];
-    }
-    __syncthreads();
-    int32_t* csz = s.csize + (int64_t)g * d.Nc;
-    int32_t* coff = s.coff + (int64_t)g * d.Nc;
-    int32_t* ccap = s.ccap + (int64_t)g * d.Nc;
-    if (tid == 0) {
-        // weighted plurality in rank order, ties to the lower id
-        int ids[kMaxKappa];
-        double v[kMaxKappa];
-        int nd = 0;
-        for (int e = 0; e < E; ++e) {
-            int k = 0;
-            while (k < nd && ids[k] != e_c[e]) ++k;
-            if (k == nd) { ids[nd] = e_c[e]; v[nd] = 0.0; ++nd; }
-            v[k] += (double)e_w[e];
+        // ---- graphs whose last slice this CTA was: finish them (after all
+        // of this CTA's pieces, so none of its slices waits behind a finish)
+        __syncthreads();
+        const int nfin = *snf;
+        if (nfin) __threadfence();
+        if (d.pdl == 2) pdl_trigger();
+        for (int f = 0; f < nfin; ++f) {
+            const Piece pc = sp[sfin[f]];
+            __syncthreads();   // the scratch is free
+            finish_graph<HG>(s, d, pc.g, pc.nc, pc.R, K, n, out, smem + L::off_buf, sM, sL, sflag);
+            if (tid == 0) s.bar[pc.g * 2] = 0u;
         }
-        int best = -1;
-        for (int k = 0; k < nd; ++k)
-            if (best < 0 || v[k] > v[best] || (v[k] == v[best] && ids[k] < ids[best])) best = k;
-        const int c = (best < 0) ? 0 : ids[best];
-        const int size = csz[c], cp = ccap[c], off0 = coff[c], top = s.pool_top[g];
-        int ok = 1, off = off0;
-        if (size == cp) {   // segment full: move it to the pool top with twice the room
-            const int ncap = max(16, 2 * cp);
-            if ((int64_t)top + ncap > d.P) ok = 0;
-            else { s.pool_top[g] = top + ncap; off = top; }
-        }
-        s_c = c; s_ok = ok; s_off = off; s_size = size; s_oldoff = off0; s_E = E;
-        if (!ok) set_error(s.err, CKV_ERR_CAPACITY);
-    }
-    __syncthreads();
-    if (!s_ok) return;
-    const int c = s_c, size = s_size, off = s_off, old_off = s_oldoff;
-    int32_t* pool = s.pool + (int64_t)g * d.P;
-    if (off != old_off)
-        for (int i = tid; i < size; i += kAsgThreads) pool[off + i] = pool[old_off + i];
-    // running-mean update of the assigned centroid, double math rounded once
-    float* mu = s.mu + ((int64_t)g * d.Nc + c) * kD;
-    const double mv = (double)mu[tid];
-    mu[tid] = __double2float_rn(__dadd_rn(mv, __ddiv_rn(__dsub_rn(kv, mv), (double)(size + 1))));
-    __syncthreads();
-    if (tid == 0) {
-        if (off != old_off) { coff[c] = off; ccap[c] = max(16, 2 * ccap[c]); }
-        pool[off + size] = t;
-        csz[c] = size + 1;
-        s.tok_comm[(int64_t)g * d.NM + t] = c;
-        s.meta[(int64_t)g * M_COUNT + M_ASSIGNED] = c;
-    }
-    const int64_t row = (int64_t)g * (d.NM - d.n_init) + (t - d.n_init);
-    if (tid == 0) s.edge_deg[row] = s_E;
-    if (tid < s_E) {
-        s.edge_col[row * d.kappa + tid] = s.e_tok[(int64_t)g * d.kappa + tid];
-        s.edge_w[row * d.kappa + tid] = e_w[tid];
+        if (npieces < kMaxPieces) break;
+        __syncthreads();   // every thread is done with this round's list
     }
 }
 
@@ -1543,38 +1508,15 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
 {
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
-        void* fn = d.bf16 ? attend_fn<true, HG>() : attend_fn<false, HG>();
         const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
-        // the slices of a graph wait for one another: all CTAs must be
-        // co-resident, which a cooperative launch guarantees (or refuses)
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(d.nCTA);
-        cfg.blockDim = dim3(kAttWarps * 32);
-        cfg.dynamicSmemBytes = bytes;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[2];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = d.pdl ? 2 : 1;
-        DevState ss = s;
-        Dims dd = d;
-        const void* qq = q;
-        const void* kk = K;
-        const void* vv = V;
-        int nn = n;
-        float* oo = out;
-        void* args[] = {&ss, &dd, &qq, &kk, &vv, &nn, &oo};
-        return cudaLaunchKernelExC(&cfg, fn, args);
+        if (d.bf16)
+            return launch_ex(d, k_attend<true, HG>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K, V, n,
+                             out);
+        return launch_ex(d, k_attend<false, HG>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K, V, n,
+                         out);
     });
 }
 
-cudaError_t launch_assign(const DevState& s, const Dims& d, const void* K, int n, cudaStream_t st)
-{
-    return launch_ex(d, d.bf16 ? k_assign<true> : k_assign<false>, dim3(d.G), dim3(kAsgThreads), 0, st, s, d, K, n);
-}
 
 cudaError_t launch_append_rows(const Dims& d, const void* knew, const void* vnew, void* K, void* V, int row,
                                cudaStream_t st)
