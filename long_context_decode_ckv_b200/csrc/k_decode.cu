@@ -70,11 +70,6 @@ __device__ __forceinline__ uint32_t ord_u(float f)
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// (w desc, token asc) order of edge candidates
-__device__ __forceinline__ bool cand_better(float w, int t, float w2, int t2)
-{
-    return w > w2 || (w == w2 && t < t2);
-}
 
 // ---------------------------------------------------------------- k_score
 // Work unit = 32 consecutive communities of one graph (16 KB of centroids,
@@ -634,17 +629,23 @@ __device__ __forceinline__ void load_logits(const float* p, float (&z)[HG])
 constexpr int kFinMaxRows = 16;                                  // rows per thread and round
 constexpr int kFinCand = kMaxKappa * (kFinMaxRows + 1);           // compacted entries, at most
 
+// 64-bit order-preserving key of an edge candidate: larger = ranked first
+// (w desc, token asc; w >= 0); 0 marks an empty slot
+__device__ __forceinline__ unsigned long long edge_key(float w, int t)
+{
+    return ((unsigned long long)__float_as_uint(w) << 32) | (unsigned long long)(~(uint32_t)t);
+}
+__device__ __forceinline__ float key_w(unsigned long long k) { return __uint_as_float((uint32_t)(k >> 32)); }
+__device__ __forceinline__ int key_t(unsigned long long k) { return (int)~(uint32_t)(k & 0xffffffffull); }
+
 struct EdgeScratch {
-    float lw[kMaxKappa];       // running list
-    int lt[kMaxKappa];
-    int lx[kMaxKappa];
-    float ww[kAttWarps][kMaxKappa];   // each warp's best lane-bests
-    int wt[kAttWarps][kMaxKappa];
-    float tw;                   // threshold
-    int tt;
-    int m;                      // compacted entries
-    float cw[kFinCand];
-    int ct[kFinCand];
+    unsigned long long lk[kMaxKappa];            // running list (rank order)
+    int lx[kMaxKappa];                           // kept-member row of each entry
+    int lc[kMaxKappa], lsz[kMaxKappa], lcap[kMaxKappa], loff[kMaxKappa];   // its community and counters
+    unsigned long long wk[kAttWarps][kMaxKappa]; // each warp's best lane-bests
+    unsigned long long tk;                       // threshold
+    int m;                                       // compacted entries
+    unsigned long long ck[kFinCand];
     int cx[kFinCand];
 };
 
@@ -672,78 +673,67 @@ __device__ __forceinline__ void edges_load(const Dims& d, const float* __restric
     }
 }
 
-// r holds round 0 (edges_load with j0 = 0) on entry
+// r holds round 0 (edges_load with j0 = 0) on entry.  With `counters`,
+// each ranked entry also fetches its community (rcomm) and that
+// community's size, capacity and segment start for the assignment.
 template <int HG>
-__device__ __forceinline__ void cta_edges(const Dims& d, const float* __restrict__ zrow,
+__device__ __forceinline__ void cta_edges(const DevState& st, const Dims& d, int g, const float* __restrict__ zrow,
                                           const int32_t* __restrict__ rtok, int T, const float* sM,
-                                          const float* sL, EdgeScratch& e, EdgeRows<HG>& r)
+                                          const float* sL, EdgeScratch& e, EdgeRows<HG>& r, bool counters)
 {
     constexpr int NT = kAttWarps * 32;
     constexpr int FR = EdgeRows<HG>::FR;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kappa = d.kappa;
-    if (tid < kMaxKappa) { e.lw[tid] = -INFINITY; e.lt[tid] = 0x7fffffff; e.lx[tid] = -1; }
+    if (tid < kMaxKappa) { e.lk[tid] = 0ull; e.lx[tid] = -1; }
     for (int j0 = 0; j0 < max(T, 1); j0 += FR * NT) {
         if (j0 > 0) edges_load<HG>(d, zrow, rtok, T, j0, r);
-        float w[FR + 1];
-        int t[FR + 1];
+        unsigned long long key[FR + 1];
 #pragma unroll
         for (int u = 0; u < FR; ++u) {
             const int j = j0 + tid + u * NT;
             float sw = 0.f;
 #pragma unroll
             for (int h = 0; h < HG; ++h) sw += __expf(r.z[u][h] - sM[h]) * sL[h];
-            w[u] = (j < T) ? sw : -INFINITY;
-            t[u] = r.t[u];
+            key[u] = (j < T) ? edge_key(sw, r.t[u]) : 0ull;
         }
         __syncthreads();   // the running list is complete
         // the running list's entry `tid` joins as the thread's extra entry
-        w[FR] = (tid < kappa) ? e.lw[tid] : -INFINITY;
-        t[FR] = (tid < kappa) ? e.lt[tid] : 0x7fffffff;
+        key[FR] = (tid < kappa) ? e.lk[tid] : 0ull;
         const int xl = (tid < kappa) ? e.lx[tid] : -1;
-        float bw = -INFINITY;
-        int bt = 0x7fffffff;
+        unsigned long long best = 0ull;
 #pragma unroll
-        for (int u = 0; u <= FR; ++u)
-            if (w[u] != -INFINITY && cand_better(w[u], t[u], bw, bt)) { bw = w[u]; bt = t[u]; }
+        for (int u = 0; u <= FR; ++u) best = max(best, key[u]);
         // each warp's best kappa lane-bests
         int rank = 0;
 #pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-            const float w2 = __shfl_sync(kFull, bw, i);
-            const int t2 = __shfl_sync(kFull, bt, i);
-            rank += cand_better(w2, t2, bw, bt) ? 1 : 0;
-        }
-        if (lane < kappa) { e.ww[warp][lane] = -INFINITY; e.wt[warp][lane] = 0x7fffffff; }
+        for (int i = 0; i < 32; ++i) rank += (__shfl_sync(kFull, best, i) > best) ? 1 : 0;
+        if (lane < kappa) e.wk[warp][lane] = 0ull;
         __syncwarp();
-        if (rank < kappa && bw != -INFINITY) { e.ww[warp][rank] = bw; e.wt[warp][rank] = bt; }
-        if (tid == 0) { e.tw = -INFINITY; e.tt = 0x7fffffff; e.m = 0; }
+        if (rank < kappa && best) e.wk[warp][rank] = best;
+        if (tid == 0) { e.tk = 0ull; e.m = 0; }
         __syncthreads();
         // tau: the kappa-th best of the warps' lists (anything, when fewer exist)
         if (tid < kAttWarps * kappa) {
-            const float mw = e.ww[tid / kappa][tid % kappa];
-            const int mt = e.wt[tid / kappa][tid % kappa];
-            if (mw != -INFINITY) {
+            const unsigned long long mk = e.wk[tid / kappa][tid % kappa];
+            if (mk) {
                 int rr = 0;
-                for (int wi = 0; wi < kAttWarps; ++wi)
-                    for (int ki = 0; ki < kappa; ++ki) {
-                        const float w2 = e.ww[wi][ki];
-                        rr += (w2 != -INFINITY && cand_better(w2, e.wt[wi][ki], mw, mt)) ? 1 : 0;
-                    }
-                if (rr == kappa - 1) { e.tw = mw; e.tt = mt; }
+                for (int wi = 0; wi < kAttWarps; ++wi) {
+#pragma unroll 8
+                    for (int ki = 0; ki < kappa; ++ki) rr += (e.wk[wi][ki] > mk) ? 1 : 0;
+                }
+                if (rr == kappa - 1) e.tk = mk;
             }
         }
         __syncthreads();
         // compact the entries at least as good as tau
-        const float tw = e.tw;
-        const int tt = e.tt;
+        const unsigned long long tk = e.tk;
 #pragma unroll
         for (int u = 0; u <= FR; ++u) {
-            if (w[u] != -INFINITY && !cand_better(tw, tt, w[u], t[u])) {
+            if (key[u] && key[u] >= tk) {
                 const int slot = atomicAdd(&e.m, 1);
                 if (slot < kFinCand) {
-                    e.cw[slot] = w[u];
-                    e.ct[slot] = t[u];
+                    e.ck[slot] = key[u];
                     e.cx[slot] = (u < FR) ? j0 + tid + u * NT : xl;
                 }
             }
@@ -752,13 +742,25 @@ __device__ __forceinline__ void cta_edges(const Dims& d, const float* __restrict
         // rank them; the first kappa become the running list
         const int m = min(e.m, kFinCand);
         for (int i = tid; i < m; i += NT) {
-            const float mw = e.cw[i];
-            const int mt = e.ct[i];
+            const unsigned long long mk = e.ck[i];
+            const int x = e.cx[i];
             int rr = 0;
-            for (int j = 0; j < m; ++j) rr += cand_better(e.cw[j], e.ct[j], mw, mt) ? 1 : 0;
-            if (rr < kappa) { e.lw[rr] = mw; e.lt[rr] = mt; e.lx[rr] = e.cx[i]; }
+#pragma unroll 8
+            for (int j = 0; j < m; ++j) rr += (e.ck[j] > mk) ? 1 : 0;
+            if (rr < kappa) {
+                e.lk[rr] = mk;
+                e.lx[rr] = x;
+                if (counters && j0 + FR * NT >= T) {   // last round: prefetch for the vote
+                    const int cm = __ldcg(st.rcomm + (int64_t)g * d.NM + x);
+                    const int64_t gi = (int64_t)g * d.Nc + cm;
+                    e.lc[rr] = cm;
+                    e.lsz[rr] = st.csize[gi];
+                    e.lcap[rr] = st.ccap[gi];
+                    e.loff[rr] = st.coff[gi];
+                }
+            }
         }
-        for (int i = m + tid; i < kappa; i += NT) { e.lw[i] = -INFINITY; e.lt[i] = 0x7fffffff; e.lx[i] = -1; }
+        for (int i = m + tid; i < kappa; i += NT) { e.lk[i] = 0ull; e.lx[i] = -1; }
     }
     __syncthreads();
 }
@@ -1111,32 +1113,27 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
     __syncthreads();
     // ---- edges: the top kappa of w = sum_h exp(z - M_h) / L_h over the kept members
     EdgeScratch& es = *reinterpret_cast<EdgeScratch*>(scratch);
-    cta_edges<HG>(d, zrow, rtok, T, sM, sL, es, er);
+    cta_edges<HG>(s, d, g, zrow, rtok, T, sM, sL, es, er, d.fuse_assign != 0);
     if (warp == 0) {
-        const bool real = lane < d.kappa && es.lw[lane] != -INFINITY;
+        const unsigned long long lk = (lane < d.kappa) ? es.lk[lane] : 0ull;
+        const bool real = lk != 0ull;
         const int ne = __popc(__ballot_sync(kFull, real));
-        const int cm = real ? __ldcg(s.rcomm + (int64_t)g * d.NM + es.lx[lane]) : 0;
+        const float lw = key_w(lk);
+        const int cm = !real ? 0 : d.fuse_assign ? es.lc[lane] : __ldcg(s.rcomm + (int64_t)g * d.NM + es.lx[lane]);
         if (real) {
-            s.e_w[(int64_t)g * d.kappa + lane] = es.lw[lane];
-            s.e_tok[(int64_t)g * d.kappa + lane] = es.lt[lane];
+            s.e_w[(int64_t)g * d.kappa + lane] = lw;
+            s.e_tok[(int64_t)g * d.kappa + lane] = key_t(lk);
             s.e_comm[(int64_t)g * d.kappa + lane] = cm;
         }
         if (lane == 0) s.meta[(int64_t)g * M_COUNT + M_NEDGE] = ne;
         if (d.fuse_assign) {
-            // every candidate community's counters, fetched under the vote
-            int32_t* csz = s.csize + (int64_t)g * d.Nc;
-            int32_t* coff = s.coff + (int64_t)g * d.Nc;
-            int32_t* ccap = s.ccap + (int64_t)g * d.Nc;
-            const int c_any = real ? cm : 0;
-            const int p_size = csz[c_any], p_cap = ccap[c_any], p_off = coff[c_any];
-            const int p_top = s.pool_top[g];
             // weighted plurality of the edges' communities: each lane sums
             // its community's weights in rank order (double), ties to the
             // lower id
             double v = 0.0;
             for (int e = 0; e < ne; ++e) {
                 const int ce = __shfl_sync(kFull, cm, e);
-                const float we = __shfl_sync(kFull, es.lw[lane], e);
+                const float we = __shfl_sync(kFull, lw, e);
                 if (ce == cm) v += (double)we;
             }
             double bv = real ? v : -1.0;
@@ -1147,11 +1144,17 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
                 const int c2 = __shfl_xor_sync(kFull, bc, o);
                 if (v2 > bv || (v2 == bv && c2 < bc)) { bv = v2; bc = c2; }
             }
-            const int c = (ne == 0) ? 0 : bc;
-            const int src = (ne == 0) ? 0 : __ffs(__ballot_sync(kFull, real && cm == c)) - 1;
-            const int size = __shfl_sync(kFull, p_size, src), cp = __shfl_sync(kFull, p_cap, src);
-            const int off0 = __shfl_sync(kFull, p_off, src), top = p_top;
             if (lane == 0) {
+                // the winner's counters were fetched with the ranking (no
+                // edges: community 0)
+                const int c = (ne == 0) ? 0 : bc;
+                int src = 0;
+                while (src < ne - 1 && es.lc[src] != c) ++src;
+                const int64_t gi = (int64_t)g * d.Nc + c;
+                const int size = ne ? es.lsz[src] : s.csize[gi];
+                const int cp = ne ? es.lcap[src] : s.ccap[gi];
+                const int off0 = ne ? es.loff[src] : s.coff[gi];
+                const int top = s.pool_top[g];
                 int ok = 1, off = off0;
                 if (size == cp) {   // segment full: move it to the pool top with twice the room
                     const int ncap = max(16, 2 * cp);
