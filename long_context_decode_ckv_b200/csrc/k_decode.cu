@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     __shared__ int r_w[kSelWarps];
     __shared__ unsigned long long r_kmin[kSelWarps], r_kmax[kSelWarps];
     __shared__ int off_c[E][kSelWarps], off_w[E][kSelWarps];
-    __shared__ int sh_b, sh_above, sh_n, sh_C, sh_T;
+    __shared__ int sh_b, sh_above, sh_n, sh_C, sh_T, sh_bn, sh_bt;
     const int g = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Nc = d.n_comm, budget = d.budget;
@@ -236,13 +236,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     // ---- 1. scores and sizes (one round of loads), range and total size
     const float* gsc = s.score + (int64_t)g * d.Nc;
     const int32_t* gsz = s.csize + (int64_t)g * d.Nc;
+    const int32_t* gco = s.coff + (int64_t)g * d.Nc;
     float v[E];
-    int w[E];
+    int w[E], co[E];   // score, size, segment start
 #pragma unroll
     for (int i = 0; i < E; ++i) {
         const int c = i * kSelThreads + tid;
         w[i] = (c < Nc) ? gsz[c] : 0;
         v[i] = (c < Nc) ? gsc[c] : 0.f;
+        co[i] = (c < Nc) ? gco[c] : 0;
     }
     float lo = INFINITY, hi = -INFINITY;
     int wsum = 0;
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
         wsum += __shfl_xor_sync(kFull, wsum, o);
     }
     if (lane == 0) { r_lo[warp] = lo; r_hi[warp] = hi; r_w[warp] = wsum; }
-    if (tid == 0) { sh_n = 0; sh_above = 0; }
+    if (tid == 0) { sh_n = 0; sh_above = 0; sh_bn = 0; sh_bt = 0; }
     __syncthreads();
     lo = r_lo[lane];
     hi = r_hi[lane];
@@ -283,6 +285,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     unsigned long long* ckey = reinterpret_cast<unsigned long long*>(ub);    // [kSelCand]
     int* hist = reinterpret_cast<int*>(ckey + kSelCand);                      // [kSelBins]
     int* cwt = hist + kSelBins;                                               // [kSelCand]
+    int* ccof = cwt + kSelCand;                                               // [kSelCand]
     for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0;
 
     if (wsum <= budget) {   // every community fits: keep them all
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
                         kmn = min(kmn, k);
                         kmx = max(kmx, k);
                         const int slot = atomicAdd(&sh_n, 1);
-                        if (slot < kSelCand) { ckey[slot] = k; cwt[slot] = w[i]; }
+                        if (slot < kSelCand) { ckey[slot] = k; cwt[slot] = w[i]; ccof[slot] = co[i]; }
                     }
                 }
             }
@@ -370,20 +373,28 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
             __syncthreads();                               // sh_n read by all
             if (tid == 0) sh_n = 0;
         }
-        // ---- 4. exact rank of the boundary bin's communities
-        for (int j = tid; j < m; j += kSelThreads) {
-            const unsigned long long kj = ckey[j];
-            int pre = 0;
-            for (int t = 0; t < m; ++t) pre += (ckey[t] > kj) ? cwt[t] : 0;
-            const bool keep = (above + pre + cwt[j] <= budget) || (above == 0 && pre == 0);
-            st[(int)~(uint32_t)(kj & 0xffffffffull)] = keep ? ST_IN : ST_OUT;
-        }
     }
-    __syncthreads();
-
-    // ---- 5. kept ids ascending with the prefix of their sizes: per round i
-    // a warp's 32 ids are consecutive, so ballots place them within the
-    // warp and one scan over the (round, warp) totals places the warps
+    // ---- 4./5. in one phase: the boundary bin's communities ranked exactly
+    // (each counts the better ones and their sizes; kept iff the sizes
+    // through it fit), and the surely kept ids placed in ascending order by
+    // ballots per 32 ids plus one scan over the (round, warp) totals.  The
+    // kept boundary communities follow the surely kept ones, in rank order.
+    const int m = (wsum <= budget) ? 0 : min(sh_n, kSelCand);
+    unsigned long long bkey = 0ull;
+    int brank = 0, bpre = 0, bw = 0, bco = 0;
+    bool bkeep = false;
+    if (tid < m) {
+        bkey = ckey[tid];
+        bw = cwt[tid];
+        bco = ccof[tid];
+        for (int t = 0; t < m; ++t) {
+            const bool better = ckey[t] > bkey;
+            brank += better ? 1 : 0;
+            bpre += better ? cwt[t] : 0;
+        }
+        bkeep = (sh_above + bpre + bw <= budget) || (sh_above == 0 && bpre == 0);
+        if (bkeep) { atomicAdd(&sh_bn, 1); atomicAdd(&sh_bt, bw); }
+    }
 #pragma unroll
     for (int i = 0; i < E; ++i) {
         const int c = i * kSelThreads + tid;
@@ -413,13 +424,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
         if (lane == 31) { sh_C = ic; sh_T = iw; }
     }
     __syncthreads();
-    const int C = sh_C, T = sh_T;
+    const int C0 = sh_C, T0 = sh_T;                // surely kept
+    const int C = C0 + sh_bn, T = T0 + sh_bt;
     // the kept list (overlays the passes' arrays): row start, id, segment start
     int* pre = reinterpret_cast<int*>(ub);       // [C + 1]
     int* cid = pre + C + 1;                      // [C]
     int* cof = cid + C;                          // [C]
     int32_t* gsel = s.sel + (int64_t)g * d.Nc;
-    const int32_t* gcoff = s.coff + (int64_t)g * d.Nc;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
         const int c = i * kSelThreads + tid;
@@ -432,9 +443,16 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
             const int pos = off_c[i][warp] + __popc(bal & ((1u << lane) - 1u));
             pre[pos] = off_w[i][warp] + wx;
             cid[pos] = c;
-            cof[pos] = gcoff[c];
+            cof[pos] = co[i];
             gsel[pos] = c;
         }
+    }
+    if (bkeep) {
+        const int pos = C0 + brank, c = (int)~(uint32_t)(bkey & 0xffffffffull);
+        pre[pos] = T0 + bpre;
+        cid[pos] = c;
+        cof[pos] = bco;
+        gsel[pos] = c;
     }
     if (tid == 0) {
         pre[C] = T;
@@ -1427,7 +1445,7 @@ size_t select_smem_bytes(int n_comm, int budget)
 {
     // statuses, then the larger of the passes' arrays and the kept list
     const size_t kept_cap = (size_t)std::min(n_comm, budget + 1);
-    const size_t passes = (size_t)8 * kSelCand + 4 * kSelBins + 4 * kSelCand;
+    const size_t passes = (size_t)8 * kSelCand + 4 * kSelBins + 8 * kSelCand;
     return (size_t)((n_comm + 15) & ~15) + std::max(passes, 4 * (3 * kept_cap + 1));
 }template <int E>
 static cudaError_t launch_select_e(const DevState& s, const Dims& d, cudaStream_t st)
