@@ -256,6 +256,10 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     // the attention grid: as many CTAs as can be co-resident
     d.nSM = sms;
     d.fuse_assign = 1;
+    {   // attention split: graph by graph unless CKV_ATT_SPLIT=rows
+        const char* v = getenv("CKV_ATT_SPLIT");
+        d.att_aligned = !(v && v[0] == 'r');
+    }
     {   // programmatic dependent launch between the decode kernels: off unless
         // CKV_PDL is 1 (each kernel lets the next one launch at its start) or
         // 2 (after its main work)

@@ -71,6 +71,7 @@ struct Dims {
     int n_comm;              // communities in use (set at init)
     int n_init;              // first decode position (edge store row 0)
     int fuse_assign;         // the attention kernel also assigns the new token and updates
+    int att_aligned;         // attention CTAs split graph by graph (else the rows evenly)
     int pdl;                 // programmatic dependent launch: 0 off, 1 trigger at kernel start, 2 after the main work
 };
 

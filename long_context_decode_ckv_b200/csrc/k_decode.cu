@@ -1280,9 +1280,14 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
             for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(kFull, tot, o);
             const int P = (int)min((long long)gridDim.x, tot);
             const long long A = (long long)blockIdx.x * tot / P, B = (long long)(blockIdx.x + 1) * tot / P;
+            // graph-aligned split (at least as many CTAs as graphs): graph g gets
+            // CTAs [f(g), f(g+1)), f(g) = g + floor(P_g * (P - G) / tot), and
+            // each of them one slice of it
+            const bool aligned = d.att_aligned && (int)gridDim.x >= G;
+            const int Pa = (int)gridDim.x;
             int np = 0;                            // pieces seen so far
             long long carry = 0;
-            for (int g0 = 0; g0 < G && (int)blockIdx.x < P; g0 += 32) {
+            for (int g0 = 0; g0 < G && (aligned || (int)blockIdx.x < P); g0 += 32) {
                 const int g = g0 + lane;
                 const int R = (g < G) ? rows_of(g) : 0;
                 long long incl = R;
@@ -1292,18 +1297,31 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
                     if (lane >= o) incl += t;
                 }
                 const long long Pg = carry + incl - R;
-                const bool mine = g < G && Pg < B && Pg + R > A;
+                int fa = 0, fb = 0;
+                if (aligned) {
+                    fa = g + (int)(Pg * (Pa - G) / tot);
+                    fb = g + 1 + (int)((Pg + R) * (Pa - G) / tot);
+                }
+                const bool mine = g < G && (aligned ? ((int)blockIdx.x >= fa && (int)blockIdx.x < fb)
+                                                    : (Pg < B && Pg + R > A));
                 const unsigned bal = __ballot_sync(kFull, mine);
                 if (mine) {
                     const int slot = np + __popc(bal & ((1u << lane) - 1u)) - done;
                     if (slot >= 0 && slot < kMaxPieces) {
                         Piece pc;
                         pc.g = g;
-                        pc.r0 = (int)(max(A, Pg) - Pg);
-                        pc.r1 = (int)(min(B, Pg + R) - Pg);
-                        const int f = share_of(Pg, tot, P);
-                        pc.k = (int)blockIdx.x - f;
-                        pc.nc = share_of(Pg + R - 1, tot, P) - f + 1;
+                        if (aligned) {
+                            pc.k = (int)blockIdx.x - fa;
+                            pc.nc = fb - fa;
+                            pc.r0 = (int)((int64_t)pc.k * R / pc.nc);
+                            pc.r1 = (int)((int64_t)(pc.k + 1) * R / pc.nc);
+                        } else {
+                            pc.r0 = (int)(max(A, Pg) - Pg);
+                            pc.r1 = (int)(min(B, Pg + R) - Pg);
+                            const int f = share_of(Pg, tot, P);
+                            pc.k = (int)blockIdx.x - f;
+                            pc.nc = share_of(Pg + R - 1, tot, P) - f + 1;
+                        }
                         pc.R = R;
                         sp[slot] = pc;
                     }
