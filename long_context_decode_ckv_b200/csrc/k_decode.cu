@@ -198,6 +198,14 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelCand = 1024;     // boundary-bin communities ranked exactly
 enum : int8_t { ST_OUT = 0, ST_IN = 1, ST_CAND = 2 };
 
+// asks L2 to fetch n ints from p on (one prefetch per 128-byte line)
+__device__ __forceinline__ void prefetch_l2_range(const int32_t* p, int n)
+{
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~(uintptr_t)127;
+    const uintptr_t a1 = reinterpret_cast<uintptr_t>(p + n);
+    for (uintptr_t a = a0; a < a1; a += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+}
+
 // key of a community: (order-preserving score bits, inverted id): larger = kept first
 __device__ __forceinline__ unsigned long long sel_key(float sc, int c)
 {
@@ -237,6 +245,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     const float* gsc = s.score + (int64_t)g * d.Nc;
     const int32_t* gsz = s.csize + (int64_t)g * d.Nc;
     const int32_t* gco = s.coff + (int64_t)g * d.Nc;
+    const int32_t* gpool = s.pool + (int64_t)g * d.P;
     float v[E];
     int w[E], co[E];   // score, size, segment start
 #pragma unroll
@@ -292,7 +301,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
 #pragma unroll
         for (int i = 0; i < E; ++i) {
             const int c = i * kSelThreads + tid;
-            if (w[i] > 0) st[c] = ST_IN;
+            if (w[i] > 0) {
+                st[c] = ST_IN;
+                prefetch_l2_range(gpool + co[i], w[i]);
+            }
         }
     } else {
         // ---- 2./3. bucket passes until the boundary bin is small
@@ -341,6 +353,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
                     const int b = bin_of(i, c);
                     if (b > bs) {
                         st[c] = ST_IN;
+                        prefetch_l2_range(gpool + co[i], w[i]);   // its members, for the row copy
                     } else if (b < bs) {
                         st[c] = ST_OUT;
                     } else {
@@ -349,6 +362,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
                         kmx = max(kmx, k);
                         const int slot = atomicAdd(&sh_n, 1);
                         if (slot < kSelCand) { ckey[slot] = k; cwt[slot] = w[i]; ccof[slot] = co[i]; }
+                        if (shift < 0) prefetch_l2_range(gpool + co[i], w[i]);   // likely kept too
                     }
                 }
             }
@@ -645,7 +659,7 @@ __device__ __forceinline__ void load_logits(const float* p, float (&z)[HG])
 // that good, so at most kappa * (FR + 1) entries are compacted and ranked
 // by counting.
 constexpr int kFinMaxRows = 16;                                  // rows per thread and round
-constexpr int kFinCand = kMaxKappa * (kFinMaxRows + 1);           // compacted entries, at most
+constexpr int kFinCand = kAttWarps * kMaxKappa * (kFinMaxRows + 1);   // compacted entries, at most
 
 // 64-bit order-preserving key of an edge candidate: larger = ranked first
 // (w desc, token asc; w >= 0); 0 marks an empty slot
@@ -661,7 +675,6 @@ struct EdgeScratch {
     int lx[kMaxKappa];                           // kept-member row of each entry
     int lc[kMaxKappa], lsz[kMaxKappa], lcap[kMaxKappa], loff[kMaxKappa];   // its community and counters
     unsigned long long wk[kAttWarps][kMaxKappa]; // each warp's best lane-bests
-    unsigned long long tk;                       // threshold
     int m;                                       // compacted entries
     unsigned long long ck[kFinCand];
     int cx[kFinCand];
@@ -722,30 +735,22 @@ __device__ __forceinline__ void cta_edges(const DevState& st, const Dims& d, int
         unsigned long long best = 0ull;
 #pragma unroll
         for (int u = 0; u <= FR; ++u) best = max(best, key[u]);
-        // each warp's best kappa lane-bests
+        // tau: every warp's kappa-th best lane-best is a lower bound of the
+        // answer (that warp holds kappa keys at least as good); their max
+        // bounds it best.  Entries >= tau come from at most kappa lanes per
+        // warp.
         int rank = 0;
 #pragma unroll 8
         for (int i = 0; i < 32; ++i) rank += (__shfl_sync(kFull, best, i) > best) ? 1 : 0;
-        if (lane < kappa) e.wk[warp][lane] = 0ull;
-        __syncwarp();
-        if (rank < kappa && best) e.wk[warp][rank] = best;
-        if (tid == 0) { e.tk = 0ull; e.m = 0; }
+        const unsigned tb = __ballot_sync(kFull, best != 0ull && rank == kappa - 1);
+        const unsigned long long tw = tb ? __shfl_sync(kFull, best, __ffs(tb) - 1) : 1ull;   // tb is warp-uniform
+        if (lane == 0) e.wk[warp][0] = tw;
+        if (tid == 0) e.m = 0;
         __syncthreads();
-        // tau: the kappa-th best of the warps' lists (anything, when fewer exist)
-        if (tid < kAttWarps * kappa) {
-            const unsigned long long mk = e.wk[tid / kappa][tid % kappa];
-            if (mk) {
-                int rr = 0;
-                for (int wi = 0; wi < kAttWarps; ++wi) {
-#pragma unroll 8
-                    for (int ki = 0; ki < kappa; ++ki) rr += (e.wk[wi][ki] > mk) ? 1 : 0;
-                }
-                if (rr == kappa - 1) e.tk = mk;
-            }
-        }
-        __syncthreads();
+        unsigned long long tk = 1ull;
+#pragma unroll
+        for (int wi = 0; wi < kAttWarps; ++wi) tk = max(tk, e.wk[wi][0]);
         // compact the entries at least as good as tau
-        const unsigned long long tk = e.tk;
 #pragma unroll
         for (int u = 0; u <= FR; ++u) {
             if (key[u] && key[u] >= tk) {
