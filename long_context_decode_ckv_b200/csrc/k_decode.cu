@@ -196,7 +196,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, 
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelCand = 1024;     // boundary-bin communities ranked exactly
-enum : int8_t { ST_OUT = 0, ST_IN = 1, ST_CAND = 2 };
 
 // asks L2 to fetch n ints from p on (one prefetch per 128-byte line)
 __device__ __forceinline__ void prefetch_l2_range(const int32_t* p, int n)
@@ -231,7 +230,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     if (d.pdl == 1) pdl_trigger();
     if (*(volatile int*)s.err) return;
     extern __shared__ __align__(16) unsigned char smem_sel[];
-    int8_t* st = reinterpret_cast<int8_t*>(smem_sel);       // [Nc] status of each community
     __shared__ float r_lo[kSelWarps], r_hi[kSelWarps];
     __shared__ int r_w[kSelWarps];
     __shared__ unsigned long long r_kmin[kSelWarps], r_kmax[kSelWarps];
@@ -255,19 +253,21 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
         v[i] = (c < Nc) ? gsc[c] : 0.f;
         co[i] = (c < Nc) ? gco[c] : 0;
     }
+    // status of the thread's communities as bit masks: still a candidate
+    // (cmask), surely kept (imask)
+    unsigned cmask = 0u, imask = 0u;
     float lo = INFINITY, hi = -INFINITY;
     int wsum = 0;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
-        const int c = i * kSelThreads + tid;
         if (w[i] > 0) {
             lo = fminf(lo, v[i]);
             hi = fmaxf(hi, v[i]);
             wsum += w[i];
+            cmask |= 1u << i;
         } else {
             w[i] = 0;
         }
-        if (c < Nc) st[c] = (w[i] > 0) ? ST_CAND : ST_OUT;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
@@ -288,9 +288,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
         wsum += __shfl_xor_sync(kFull, wsum, o);
     }
 
-    // shared memory after the statuses: the passes' histogram and boundary
-    // candidates, later (same bytes) the kept list
-    unsigned char* ub = smem_sel + ((Nc + 15) & ~15);
+    // shared memory: the passes' histogram and boundary candidates, later
+    // (same bytes) the kept list
+    unsigned char* ub = smem_sel;
     unsigned long long* ckey = reinterpret_cast<unsigned long long*>(ub);    // [kSelCand]
     int* hist = reinterpret_cast<int*>(ckey + kSelCand);                      // [kSelBins]
     int* cwt = hist + kSelBins;                                               // [kSelCand]
@@ -298,14 +298,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0;
 
     if (wsum <= budget) {   // every community fits: keep them all
+        imask = cmask;
+        cmask = 0u;
 #pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const int c = i * kSelThreads + tid;
-            if (w[i] > 0) {
-                st[c] = ST_IN;
-                prefetch_l2_range(gpool + co[i], w[i]);
-            }
-        }
+        for (int i = 0; i < E; ++i)
+            if (imask & (1u << i)) prefetch_l2_range(gpool + co[i], w[i]);
     } else {
         // ---- 2./3. bucket passes until the boundary bin is small
         const float scale = (hi > lo) ? (float)kSelBins / (hi - lo) : 0.f;
@@ -323,10 +320,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
                 return (int)((sel_key(v[i], c) >> shift) & (unsigned long long)(kSelBins - 1));
             };
 #pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const int c = i * kSelThreads + tid;
-                if (c < Nc && st[c] == ST_CAND) atomicAdd(&hist[bin_of(i, c)], w[i]);
-            }
+            for (int i = 0; i < E; ++i)
+                if (cmask & (1u << i)) atomicAdd(&hist[bin_of(i, i * kSelThreads + tid)], w[i]);
             __syncthreads();
             // boundary bin: the size summed from the top bin down first exceeds the budget
             const int b0 = kSelBins - 1 - 2 * tid, b1 = b0 - 1;
@@ -345,26 +340,34 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
             above = sh_above;
             hist[b0] = 0;
             hist[b1] = 0;
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                if (!(cmask & (1u << i))) continue;
+                const int c = i * kSelThreads + tid;
+                const int b = bin_of(i, c);
+                if (b > bs) {
+                    imask |= 1u << i;
+                    cmask &= ~(1u << i);
+                    prefetch_l2_range(gpool + co[i], w[i]);   // its members, for the row copy
+                } else if (b < bs) {
+                    cmask &= ~(1u << i);
+                } else {
+                    const int slot = atomicAdd(&sh_n, 1);
+                    if (slot < kSelCand) { ckey[slot] = sel_key(v[i], c); cwt[slot] = w[i]; ccof[slot] = co[i]; }
+                    if (shift < 0) prefetch_l2_range(gpool + co[i], w[i]);   // likely kept too
+                }
+            }
+            __syncthreads();
+            m = sh_n;
+            if (m <= kSelCand) break;                      // uniform
+            // crowded boundary bin: the key range of its communities
             unsigned long long kmn = ~0ull, kmx = 0ull;
 #pragma unroll
             for (int i = 0; i < E; ++i) {
-                const int c = i * kSelThreads + tid;
-                if (c < Nc && st[c] == ST_CAND) {
-                    const int b = bin_of(i, c);
-                    if (b > bs) {
-                        st[c] = ST_IN;
-                        prefetch_l2_range(gpool + co[i], w[i]);   // its members, for the row copy
-                    } else if (b < bs) {
-                        st[c] = ST_OUT;
-                    } else {
-                        const unsigned long long k = sel_key(v[i], c);
-                        kmn = min(kmn, k);
-                        kmx = max(kmx, k);
-                        const int slot = atomicAdd(&sh_n, 1);
-                        if (slot < kSelCand) { ckey[slot] = k; cwt[slot] = w[i]; ccof[slot] = co[i]; }
-                        if (shift < 0) prefetch_l2_range(gpool + co[i], w[i]);   // likely kept too
-                    }
-                }
+                if (!(cmask & (1u << i))) continue;
+                const unsigned long long k = sel_key(v[i], i * kSelThreads + tid);
+                kmn = min(kmn, k);
+                kmx = max(kmx, k);
             }
 #pragma unroll
             for (int o = 16; o; o >>= 1) {
@@ -373,8 +376,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
             }
             if (lane == 0) { r_kmin[warp] = kmn; r_kmax[warp] = kmx; }
             __syncthreads();
-            m = sh_n;
-            if (m <= kSelCand) break;                      // uniform
             kmn = r_kmin[lane];
             kmx = r_kmax[lane];
 #pragma unroll
@@ -411,8 +412,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     }
 #pragma unroll
     for (int i = 0; i < E; ++i) {
-        const int c = i * kSelThreads + tid;
-        const bool kept = c < Nc && st[c] == ST_IN;
+        const bool kept = (imask >> i) & 1u;
         const unsigned bal = __ballot_sync(kFull, kept);
         const int wt = bal ? (int)__reduce_add_sync(kFull, kept ? (unsigned)w[i] : 0u) : 0;
         if (lane == 0) { off_c[i][warp] = __popc(bal); off_w[i][warp] = wt; }
@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
 #pragma unroll
     for (int i = 0; i < E; ++i) {
         const int c = i * kSelThreads + tid;
-        const bool kept = c < Nc && st[c] == ST_IN;
+        const bool kept = (imask >> i) & 1u;
         const unsigned bal = __ballot_sync(kFull, kept);
         if (bal == 0u) continue;                                   // warp-uniform
         const int wk = kept ? w[i] : 0;
@@ -1466,11 +1466,13 @@ void* attend_fn()
 
 size_t select_smem_bytes(int n_comm, int budget)
 {
-    // statuses, then the larger of the passes' arrays and the kept list
+    // the larger of the passes' arrays and the kept list
     const size_t kept_cap = (size_t)std::min(n_comm, budget + 1);
     const size_t passes = (size_t)8 * kSelCand + 4 * kSelBins + 8 * kSelCand;
-    return (size_t)((n_comm + 15) & ~15) + std::max(passes, 4 * (3 * kept_cap + 1));
-}template <int E>
+    return std::max(passes, 4 * (3 * kept_cap + 1));
+}
+
+template <int E>
 static cudaError_t launch_select_e(const DevState& s, const Dims& d, cudaStream_t st)
 {
     return launch_ex(d, k_select<E>, dim3(d.G), dim3(kSelThreads), select_smem_bytes(d.n_comm, d.budget), st, s, d);
