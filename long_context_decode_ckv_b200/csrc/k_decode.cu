@@ -728,7 +728,7 @@ __device__ __forceinline__ void cta_edges(const DevState& st, const Dims& d, int
             for (int h = 0; h < HG; ++h) sw += __expf(r.z[u][h] - sM[h]) * sL[h];
             key[u] = (j < T) ? edge_key(sw, r.t[u]) : 0ull;
         }
-        __syncthreads();   // the running list is complete
+        if (j0 > 0) __syncthreads();   // the running list is complete (round 0: each thread cleared its own)
         // the running list's entry `tid` joins as the thread's extra entry
         key[FR] = (tid < kappa) ? e.lk[tid] : 0ull;
         const int xl = (tid < kappa) ? e.lx[tid] : -1;
@@ -1105,6 +1105,11 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
 
     EdgeRows<HG> er;   // the first round of kept members, loaded under the output merge
     edges_load<HG>(d, zrow, rtok, T, 0, er);
+    float kv = 0.f;    // the new token's key, for the update
+    if (d.fuse_assign && tid < kD) {
+        const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + (n - 1)) * kD;
+        kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
+    }
     // ---- output: every value merged online over the slices; the thread of
     // a head's first value also leaves that head's max and 1 / sum
     for (int i = tid; i < HG * kD; i += NT) {
@@ -1199,11 +1204,9 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
         for (int i = tid; i < size; i += NT) pool[off + i] = pool[old_off + i];
     // running-mean update of the assigned centroid, double math rounded once
     if (tid < kD) {
-        const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + t) * kD;
-        const double kv = d.bf16 ? (double)elem<true>(K, krow + tid) : (double)elem<false>(K, krow + tid);
         float* mu = s.mu + ((int64_t)g * d.Nc + c) * kD;
         const double mv = (double)mu[tid];
-        mu[tid] = __double2float_rn(__dadd_rn(mv, __ddiv_rn(__dsub_rn(kv, mv), (double)(size + 1))));
+        mu[tid] = __double2float_rn(__dadd_rn(mv, __ddiv_rn(__dsub_rn((double)kv, mv), (double)(size + 1))));
     }
     __syncthreads();   // the segment copy is complete before the append
     const int64_t row = (int64_t)g * (d.NM - d.n_init) + (t - d.n_init);
