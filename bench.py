@@ -130,6 +130,30 @@ class Clocks:
                 "samples": len(self.rows)}
 
 
+# ------------------------------------------------------------ ranks (N > 1)
+def rank_env():
+    """(rank, world size, local rank) from the launcher's environment."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def max_over_ranks(dist, value, device):
+    """The largest of every rank's value (each rank's device time: the job
+    takes as long as its slowest replica)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, steps, ms):
+    """Whole-job steps/s: every rank ran `steps` steps of its own replica in
+    at most `ms` milliseconds (weak scaling)."""
+    return world * steps / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ oracle
 def run_oracle_steps(wl, n_steps, graphs=None):
     """Time the CPU oracle (single thread) on `n_steps` decode steps of the
@@ -208,9 +232,7 @@ def main():
     ap.add_argument("--profile-steps", type=int, default=40,
                     help="further steps replayed with per-kernel events (0 = none)")
     args = ap.parse_args()
-    rank = int(os.environ.get("RANK", 0))
-    world = int(os.environ.get("WORLD_SIZE", 1))
-    local = int(os.environ.get("LOCAL_RANK", 0))
+    rank, world, local = rank_env()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
@@ -345,10 +367,7 @@ def main():
         assert ckv.ckv_last_error(r["ctx"]) == ckv.CKV_OK
     ckv.ckv_get_step_debug(reps[(args.warmup + args.steps - 1) % L]["ctx"], n_tok_sel=sel_tok)
     T_mean = float(sel_tok.mean())
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(pg, ms, dev)
 
     # end-to-end through the host-buffer entry point: per step H2D of q and
     # the new token's K/V rows from pinned memory, D2H of the output
@@ -375,12 +394,9 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         ems = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([ems], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(pg, ems, dev)
         eb = 2
-        e2e = {"value": world * args.e2e_steps / (ems / 1e3), "unit": "steps/s",
+        e2e = {"value": job_rate(world, args.e2e_steps, ems), "unit": "steps/s",
                "h2d_bytes_per_step": cfg.batch * (cfg.n_q_heads + 2 * cfg.n_kv_heads) * 128 * eb,
                "d2h_bytes_per_step": cfg.batch * cfg.n_q_heads * 128 * 4}
 
@@ -392,7 +408,7 @@ def main():
     if rank != 0:
         return 0
 
-    steps_per_s = world * args.steps / (ms / 1e3)
+    steps_per_s = job_rate(world, args.steps, ms)
     per_graph = algorithmic_bytes(cfg, T_mean)
     step_bytes = per_graph * cfg.n_graphs
     gbs = step_bytes * args.steps / (ms / 1e3) / 1e9
