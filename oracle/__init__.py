@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
                                        ctypes.POINTER(StepInfo)]
         L.ckvo_row_ptr.restype = i64
         L.ckvo_row_ptr.argtypes = [i64, i32, i32]
+        L.ckvo_dense_stats.argtypes = [i32, i32, P, i32, P, i32, i32, P, P]
         L.ckvo_prefill_rows.argtypes = [i32, i32, i32, i32, P, P, i32, P, i32, P, P, P, P]
         _lib = L
     return _lib
@@ -234,6 +235,25 @@ class Graph:
         k_t = np.ascontiguousarray(k_t)
         if lib().ckvo_update(self.h, c, t, _p(k_t), _dtype_code(k_t)) != 0:
             raise ValueError("bad community id")
+
+
+def dense_stats(q: np.ndarray, K: np.ndarray, n: int):
+    """Dense softmax statistics of q [H][D] over rows [0, n) of K: (m [H], l [H])."""
+    q = np.ascontiguousarray(q)
+    H, D = q.shape
+    m = np.empty(H, np.float64)
+    l = np.empty(H, np.float64)
+    lib().ckvo_dense_stats(H, D, _p(q), _dtype_code(q), _p(np.ascontiguousarray(K)), _dtype_code(K), n,
+                           _p(m), _p(l))
+    return m, l
+
+
+def recall(m_sel, l_sel, m_den, l_den):
+    """Attention-mass recall per head: the dense softmax mass of the attended
+    rows, l_sel * exp(m_sel - m_den) / l_den (Figure 3 right, reading in
+    ckv_oracle.c)."""
+    m_sel, l_sel, m_den, l_den = (np.asarray(x, np.float64) for x in (m_sel, l_sel, m_den, l_den))
+    return l_sel * np.exp(m_sel - m_den) / l_den
 
 
 @dataclass

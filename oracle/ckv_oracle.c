@@ -249,6 +249,36 @@ void ckvo_attend(int n_heads, int D, const void* q, int q_dtype,
     free(z);
 }
 
+/* ---- NEXT f3: attention-mass recall of the retrieved set ---------------- */
+/* Figure 3 (right) caption: the share of the full attention mass that the
+ * retrieved set captures.  Reading: per query head, with the dense softmax
+ * over every cached position [0, n) (the new token included), recall =
+ * sum over the step's attended rows (sinks, kept members, the new token) of
+ * the dense probabilities = l_sel * exp(m_sel - m_den) / l_den, where
+ * (m_sel, l_sel) are the subset softmax statistics of ckvo_attend.  This
+ * function returns the dense statistics (m_den, l_den), in double. */
+void ckvo_dense_stats(int n_heads, int D, const void* q, int q_dtype, const void* K, int kv_dtype, int n,
+                      double* m_out, double* l_out)
+{
+    double* z = (double*)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    for (int h = 0; h < n_heads; ++h) {
+        double m = -INFINITY;
+        for (int j = 0; j < n; ++j) {
+            double dot = 0.0;
+            for (int i = 0; i < D; ++i)
+                dot += elem(q, q_dtype, (int64_t)h * D + i) * elem(K, kv_dtype, (int64_t)j * D + i);
+            z[j] = dot * inv_sqrt_d;
+            if (z[j] > m) m = z[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        m_out[h] = m;
+        l_out[h] = l;
+    }
+    free(z);
+}
+
 /* ---- a4: top-kappa edges ------------------------------------------------ */
 typedef struct { float w; int32_t tok; int32_t idx; } cand;
 

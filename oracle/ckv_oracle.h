@@ -123,6 +123,11 @@ void ckvo_prefill_rows(int n, int D, int n_sinks, int kappa, const void* Q, cons
                        int dtype, const int32_t* rows, int n_rows,
                        int32_t* col, float* w, int32_t* deg, float* gap);
 
+/* Dense softmax statistics over every position [0, n) of K, per head (the
+ * denominator of the attention-mass recall; see ckv_oracle.c). */
+void ckvo_dense_stats(int n_heads, int D, const void* q, int q_dtype, const void* K, int kv_dtype, int n,
+                      double* m_out, double* l_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -337,3 +337,80 @@ def test_row_ptr_closed_form(oracle_lib):
             a = max(0, min(i, S + kap + 1) - S - 1)          # rows with degree < kappa
             closed = a * (a + 1) // 2 + max(0, i - (S + kap + 1)) * kap
             assert oracle.row_ptr(i, S, kap) == closed
+
+
+# ------------------------------------------------ NEXT f3 attention-mass recall
+def test_dense_stats_match_library_logsumexp(oracle_lib):
+    rng = np.random.default_rng(11)
+    n, D, H = 131, 128, 3
+    K = rng.standard_normal((n, D)).astype(np.float32)
+    q = (rng.standard_normal((H, D)) * 3).astype(np.float32)
+    for cut in (1, 7, n):
+        m, l = oracle.dense_stats(q, K, cut)
+        z = torch.from_numpy(q.astype(np.float64)) @ torch.from_numpy(K[:cut].astype(np.float64)).T
+        z = z / math.sqrt(D)
+        np.testing.assert_allclose(m, z.max(1).values.numpy(), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(m + np.log(l), torch.logsumexp(z, 1).numpy(), rtol=0, atol=1e-12)
+    # identical keys: m is the single logit, l counts the rows
+    Kc = np.tile(K[:1], (9, 1))
+    m, l = oracle.dense_stats(q, Kc, 9)
+    np.testing.assert_allclose(m, q.astype(np.float64) @ K[0].astype(np.float64) / math.sqrt(D), atol=1e-12)
+    np.testing.assert_allclose(l, 9.0, rtol=1e-15)
+    # bf16 operands widen exactly
+    qb, Kb = synth.to_bf16_bits(q), synth.to_bf16_bits(K)
+    mb, lb = oracle.dense_stats(qb, Kb, n)
+    m2, l2 = oracle.dense_stats(_f32(qb), _f32(Kb), n)
+    np.testing.assert_array_equal(mb, m2)
+    np.testing.assert_array_equal(lb, l2)
+
+
+@pytest.mark.parametrize("budget", [40, 160, 10 ** 6])
+def test_recall_is_dense_mass_of_attended_rows(oracle_lib, budget):
+    cfg = synth.scaled(synth.TINY, n0=512, n_clusters=24, steps=4, budget=budget, bf16=True)
+    w = synth.make_workload(cfg)
+    K, V = w.K[0, 0], w.V[0, 0]
+    g = oracle.Graph(cfg.n_comm, 128, cfg.n_max)
+    g.init(cfg.n0, cfg.n_sinks, w.labels[0], K)
+    for step in range(cfg.steps):
+        n = cfg.n0 + step + 1
+        q = np.ascontiguousarray(w.q[step, 0])                        # [H][D], one head
+        sizes_before, mem_before = g.sizes(), g.members()           # state before the step
+        r = oracle.decode_step(g, q, K, V, n, cfg.n_sinks, cfg.kappa, cfg.budget)
+        g_rows = _attended_rows_from(sizes_before, mem_before, r.sel, n, cfg.n_sinks)
+        rec = oracle.recall(r.m, r.l, *oracle.dense_stats(q, K, n))
+        ref = _probs64(_f32(q), _f32(K[:n]))[:, g_rows].sum(1)      # brute force, library softmax
+        np.testing.assert_allclose(rec, ref, rtol=1e-12, atol=0)
+        assert np.all(rec <= 1.0 + 1e-12) and np.all(rec > 0)
+        if budget >= n:
+            assert len(g_rows) == n
+            np.testing.assert_allclose(rec, 1.0, rtol=1e-12)
+
+
+def _attended_rows_from(sizes, mem, sel, n, n_sinks):
+    start = np.concatenate([[0], np.cumsum(sizes)])
+    rows = list(range(n_sinks)) + [n - 1]
+    for c in sel:
+        rows += mem[start[c]:start[c + 1]].tolist()
+    assert len(set(rows)) == len(rows)
+    return np.array(sorted(rows), np.int64)
+
+
+def test_recall_grows_with_budget(oracle_lib):
+    """A larger budget keeps a longer prefix of the same order, so the
+    attended set only grows and recall never falls."""
+    cfg0 = synth.scaled(synth.TINY, n0=600, n_clusters=30, steps=1, budget=1, bf16=True)
+    w = synth.make_workload(cfg0)
+    K, V = w.K[0, 0], w.V[0, 0]
+    q = np.ascontiguousarray(w.q[0, 0])
+    n = cfg0.n0 + 1
+    den = oracle.dense_stats(q, K, n)
+    prev = None
+    for budget in (1, 20, 50, 100, 200, 400, 600):
+        g = oracle.Graph(cfg0.n_comm, 128, cfg0.n_max)
+        g.init(cfg0.n0, cfg0.n_sinks, w.labels[0], K)
+        r = oracle.decode_step(g, q, K, V, n, cfg0.n_sinks, cfg0.kappa, budget)
+        rec = oracle.recall(r.m, r.l, *den)
+        if prev is not None:
+            assert np.all(rec >= prev - 1e-12)
+        prev = rec
+    np.testing.assert_allclose(prev, 1.0, rtol=1e-12)
