@@ -172,6 +172,35 @@ ckv_status ckv_last_error(ckv_ctx* ctx);
 ckv_status ckv_get_step_debug(ckv_ctx* ctx, int32_t* n_sel, int32_t* sel, int32_t* n_tok_sel,
                               int32_t* n_edges, int32_t* edges, float* edge_w, int32_t* assigned);
 
+/* Attention-mass recall of the last decode step -- Figure 3 (right), the
+ * share of the full attention mass that the retrieved set captures.  Per
+ * query head: the dense softmax of q over every position [0, n) of K,
+ * summed over the rows that step attended (sinks, kept members, the new
+ * token); computed as l_sel * exp(m_sel - m) / l from the step's own
+ * softmax max and sum over its attended rows (left by ckv_decode_step) and
+ * the dense max and sum over [0, n) (one pass over K here).
+ * q, K: the query and key cache the step with this n was given (q
+ * [B][H_q][D], K [B][H_kv][n_max][D], kv_dtype).  recall: [B][H_q] float32,
+ * device.  Valid after ckv_decode_step(n), before or after its
+ * ckv_assign_update, until the next decode step.  Reads K once; allocates
+ * nothing.  Asynchronous.  Supported for H_q/H_kv <= 32 (bf16) or <= 8
+ * (float32).
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no decode step with this n
+ * since init or import), sticky device errors, CKV_ERR_CUDA. */
+ckv_status ckv_step_recall(ckv_ctx* ctx, const void* q, const void* K, int n, float* recall, void* stream);
+
+/* Dense decode attention, the comparator for the sparse step: every query
+ * head attends over every position [0, n) of its KV head,
+ * out = softmax(q K^T / sqrt(D)) V and lse = m + ln(l) per head.
+ * q, K, V as in ckv_decode_step; out [B][H_q][D] float32 and lse [B][H_q]
+ * float32 (may be NULL), device.  Uses the context's dimensions and
+ * scratch only (no community state; allowed before init).  Asynchronous.
+ * Supported for H_q/H_kv <= 8.
+ * Errors: CKV_ERR_INVALID_ARG (bad pointer, n outside [1, n_max], group
+ * too large), CKV_ERR_CUDA. */
+ckv_status ckv_dense_decode(ckv_ctx* ctx, const void* q, const void* K, const void* V, int n, float* out,
+                            float* lse, void* stream);
+
 /* Per-kernel device time of the decode steps, in the spirit of the pages'
  * Table 10 split of a step into retrieval and attention.  After
  * ckv_profile_begin, every ckv_decode_step / ckv_assign_update records CUDA

@@ -90,6 +90,10 @@ def lib() -> ctypes.CDLL:
     L.ckv_aux_bytes.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.ckv_attend_rows_static.restype = st
     L.ckv_attend_rows_static.argtypes = [ctypes.POINTER(ckv_config), P, P, P, I, P, P, I, P, P]
+    L.ckv_step_recall.restype = st
+    L.ckv_step_recall.argtypes = [P, P, P, I, P, P]
+    L.ckv_dense_decode.restype = st
+    L.ckv_dense_decode.argtypes = [P, P, P, P, I, P, P, P]
     L.ckv_status_string.restype = ctypes.c_char_p
     L.ckv_status_string.argtypes = [I]
     _lib = L
@@ -214,6 +218,17 @@ def ckv_attend_rows_static(cfg, q, K, V, n, rows_host, n_rows_host, max_rows, ou
     _check("ckv_attend_rows_static", lib().ckv_attend_rows_static(
         ctypes.byref(cfg), _ptr(q), _ptr(K), _ptr(V), n, _ptr(rows_host), _ptr(n_rows_host), max_rows,
         _ptr(out), _stream(stream)))
+
+
+def ckv_step_recall(ctx, q, K, n, recall, stream=None):
+    """Attention-mass recall [B][H_q] of the last decode step (n), per query head."""
+    _check("ckv_step_recall", lib().ckv_step_recall(ctx, _ptr(q), _ptr(K), n, _ptr(recall), _stream(stream)))
+
+
+def ckv_dense_decode(ctx, q, K, V, n, out, lse=None, stream=None):
+    """Dense decode attention over [0, n): out [B][H_q][D], lse [B][H_q] (optional)."""
+    _check("ckv_dense_decode", lib().ckv_dense_decode(ctx, _ptr(q), _ptr(K), _ptr(V), n, _ptr(out), _ptr(lse),
+                                                      _stream(stream)))
 
 
 def ckv_aux_bytes(ctx):

@@ -36,6 +36,9 @@ struct ckv_ctx {
     int n_tok;                   // positions covered: sinks + assigned tokens
     int pending;                 // a decode step awaits its assign/update
     int pending_n;
+    int last_n;                  // n of the last decode step (0: none since init)
+    float* dense_part;           // k_dense piece slots
+    unsigned* dense_cnt;         // k_dense arrivals per unit
     ckv_status sticky;
     // profiling: one event per kernel boundary of each profiled step
     int profiling;
@@ -295,8 +298,12 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(e_tok, G * kap);
     ALLOC(e_w, G * kap);
     ALLOC(e_comm, G * kap);
+    ALLOC(sel_ml, (size_t)d.B * d.Hq * 2);
     ALLOC(err, 1);
 #undef ALLOC
+    if (e == cudaSuccess) e = dalloc(x, &x->dense_part, ckv::dense_part_floats(d));
+    if (e == cudaSuccess) e = dalloc(x, &x->dense_cnt, (size_t)d.B * d.Hkv);
+    if (e == cudaSuccess) e = cudaMemset(x->dense_cnt, 0, (size_t)d.B * d.Hkv * sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemset(s.bar, 0, G * 2 * sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemset(s.err, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(s.meta, 0, G * ckv::M_COUNT * sizeof(int32_t));
@@ -326,6 +333,7 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
     CKV_CUDA(cudaStreamSynchronize(st));
     x->initialized = 0;
     x->pending = 0;
+    x->last_n = 0;
     x->sticky = CKV_OK;
     Dims& d = x->d;
     DevState& s = x->s;
@@ -393,6 +401,7 @@ CKV_API ckv_status ckv_decode_step(ckv_ctx* x, const void* q, const void* K, con
     CKV_CUDA(prof_mark(x, 3, st));
     x->pending = 1;
     x->pending_n = n;
+    x->last_n = n;
     return CKV_OK;
 }
 
@@ -449,6 +458,31 @@ CKV_API ckv_status ckv_decode_host(ckv_ctx* x, const void* q_host, const void* k
     CKV_CUDA(cudaMemcpyAsync(out_host, dout, (size_t)d.B * d.Hq * ckv::kD * sizeof(float),
                              cudaMemcpyDeviceToHost, st));
     CKV_CUDA(cudaStreamSynchronize(st));
+    return CKV_OK;
+}
+
+CKV_API ckv_status ckv_step_recall(ckv_ctx* x, const void* q, const void* K, int n, float* recall, void* stream)
+{
+    ckv_status cs = check_ctx(x);
+    if (cs != CKV_OK) return cs;
+    if (!q || !K || !recall) return CKV_ERR_INVALID_ARG;
+    if (!ckv::dense_supported(x->d, false)) return CKV_ERR_INVALID_ARG;
+    if (!x->initialized || x->last_n == 0 || n != x->last_n) return CKV_ERR_STATE;
+    CKV_CUDA(cudaSetDevice(x->cfg.device));
+    const ckv::DenseIO io{nullptr, nullptr, x->s.sel_ml, recall};
+    CKV_CUDA(ckv::launch_dense(x->d, q, K, nullptr, n, x->dense_part, x->dense_cnt, io, (cudaStream_t)stream));
+    return CKV_OK;
+}
+
+CKV_API ckv_status ckv_dense_decode(ckv_ctx* x, const void* q, const void* K, const void* V, int n, float* out,
+                                    float* lse, void* stream)
+{
+    if (!x) return CKV_ERR_INVALID_ARG;
+    if (!q || !K || !V || !out) return CKV_ERR_INVALID_ARG;
+    if (n < 1 || n > x->d.NM || !ckv::dense_supported(x->d, true)) return CKV_ERR_INVALID_ARG;
+    CKV_CUDA(cudaSetDevice(x->cfg.device));
+    const ckv::DenseIO io{out, lse, nullptr, nullptr};
+    CKV_CUDA(ckv::launch_dense(x->d, q, K, V, n, x->dense_part, x->dense_cnt, io, (cudaStream_t)stream));
     return CKV_OK;
 }
 
@@ -676,6 +710,7 @@ CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t byt
     d.n_init = n_init;
     x->n_tok = n_tok;
     x->pending = 0;
+    x->last_n = 0;
     x->sticky = CKV_OK;
     x->initialized = 1;
     return CKV_OK;

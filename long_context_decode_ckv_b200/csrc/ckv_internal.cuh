@@ -19,6 +19,11 @@
 //   part_o    float [G][KC][HG][D] per-CTA P.V per head, relative to its max
 //   bar       uint  [G][2]         arrivals of a graph's slices (slot 0)
 //   e_*       [G][kappa]           the step's edges (rank order) for the update
+//   sel_ml    float [B][Hq][2]     softmax max and sum of each query head over the
+//                                  step's attended rows (for the attention-mass recall)
+// Dense statistics scratch (k_dense.cu; U = B*Hkv units):
+//   dense_part float [U + grid][..] per-piece (m, l[, o]) of each unit's heads
+//   dense_cnt  uint  [U]           arrivals of a unit's pieces
 #pragma once
 
 #include <cuda_runtime.h>
@@ -60,6 +65,7 @@ struct DevState {
     int32_t* e_tok;
     float* e_w;
     int32_t* e_comm;
+    float* sel_ml;           // may be null (then the attention kernel does not write it)
     int* err;                // sticky device error word (ckv_status)
 };
 
@@ -87,6 +93,21 @@ size_t select_smem_bytes(int n_comm, int budget);
 cudaError_t prepare_kernels(const Dims& d);
 int attend_grid(const Dims& d, int sms);
 constexpr int kMaxCommunities = 16384;   // k_select holds 16 of a graph's communities per thread
+
+// dense decode statistics over a whole cache (k_dense.cu): with V, the dense
+// attention output and log-sum-exp per query head; with sel_ml, the
+// attention-mass recall of the attended rows
+struct DenseIO {
+    float* out;              // [B][Hq][D] (with V)
+    float* lse;              // [B][Hq] or null
+    const float* sel_ml;     // [B][Hq][2] or null
+    float* recall;           // [B][Hq] or null (needs sel_ml)
+};
+constexpr int kDenseMaxCtasPerSM = 4;
+bool dense_supported(const Dims& d, bool with_v);
+size_t dense_part_floats(const Dims& d);
+cudaError_t launch_dense(const Dims& d, const void* q, const void* K, const void* V, int n, float* part,
+                         unsigned* cnt, const DenseIO& io, cudaStream_t st);
 
 // init kernels (k_init.cu)
 cudaError_t launch_init_count(const DevState& s, const Dims& d, const int32_t* labels, int n,

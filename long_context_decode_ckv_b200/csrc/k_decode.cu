@@ -33,15 +33,11 @@
 
 #include "ckv_internal.cuh"
 #include "dev_async.cuh"
+#include "warp_mma.cuh"
 
 namespace ckv {
 
 namespace {
-
-constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 template <bool BF16>
 __device__ __forceinline__ float elem(const void* p, int64_t i)
@@ -69,7 +65,6 @@ __device__ __forceinline__ uint32_t ord_u(float f)
     uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-
 
 // ---------------------------------------------------------------- k_score
 // Work unit = 32 consecutive communities of one graph (16 KB of centroids,
@@ -546,91 +541,6 @@ struct AttLayout {
     static_assert(kAttWarps * HG * RSTR * 4 <= kAttWarps * WBUF, "reduction must fit");
     static_assert(kAttWarps * 6 * (kMaxKappa + 128) * 4 <= kAttWarps * WBUF, "edge lists must fit");
 };
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-// 16 bytes, or 16 zero bytes when !valid (nothing is read then)
-__device__ __forceinline__ void cp_async16z(uint32_t dst, const void* src, bool valid)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-
-// four 8x8 b16 matrices; lanes 8i..8i+7 give the row addresses of matrix i
-__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4])
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4])
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-// c += a . b  (16x16 bf16, row-major) x (16x8 bf16, column-major), fp32
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-                 "{%0,%1,%2,%3};\n"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-// transpose of the warp's 8x8 b16 matrix held in fragment layout
-__device__ __forceinline__ uint32_t movtrans(uint32_t x)
-{
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-    return y;
-}
-// (lo, hi) -> bf16 pair, round to nearest even; lo in the low half
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
-{
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-// Butterfly transpose-reduce of NV values per lane (NV a power of two
-// <= 32): afterwards every lane holds the warp-wide sum of value index
-// tr_index<NV>(lane); lanes that differ only in the bits below the last
-// halving offset hold the same value.
-template <int NV>
-__device__ __forceinline__ int tr_index(int lane)
-{
-    int idx = 0;
-#pragma unroll
-    for (int s = 0, len = NV; len > 1; ++s, len >>= 1)
-        idx += ((lane >> (4 - s)) & 1) * (len >> 1);
-    return idx;
-}
-
-template <int NV>
-__device__ __forceinline__ float transpose_reduce(float (&v)[NV], int lane)
-{
-#pragma unroll
-    for (int s = 0, len = NV; len > 1; ++s, len >>= 1) {
-        const int off = 16 >> s;
-        const bool up = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < (len >> 1); ++i) {
-            const float send = up ? v[i] : v[i + (len >> 1)];
-            const float keep = up ? v[i + (len >> 1)] : v[i];
-            v[i] = keep + __shfl_xor_sync(kFull, send, off);
-        }
-    }
-    float r = v[0];
-    constexpr int levels = (NV >= 32) ? 5 : (NV >= 16) ? 4 : (NV >= 8) ? 3 : (NV >= 4) ? 2 : (NV >= 2) ? 1 : 0;
-#pragma unroll
-    for (int off = 16 >> levels; off >= 1 && levels < 5; off >>= 1) r += __shfl_xor_sync(kFull, r, off);
-    return r;
-}
 
 // HG logits of one kept-member row (16-, 8- or 4-byte aligned by HG)
 template <int HG>
@@ -1136,7 +1046,11 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
             }
         }
         out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o / Ls;
-        if (i % kD == 0) { sM[h] = M; sL[h] = 1.f / Ls; }
+        if (i % kD == 0) {
+            sM[h] = M;
+            sL[h] = 1.f / Ls;
+            if (s.sel_ml) *reinterpret_cast<float2*>(s.sel_ml + 2 * ((int64_t)b * d.Hq + h0 + h)) = make_float2(M, Ls);
+        }
     }
     __syncthreads();
     // ---- edges: the top kappa of w = sum_h exp(z - M_h) / L_h over the kept members
@@ -1565,7 +1479,6 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
                          out);
     });
 }
-
 
 cudaError_t launch_append_rows(const Dims& d, const void* knew, const void* vnew, void* K, void* V, int row,
                                cudaStream_t st)

@@ -11,7 +11,10 @@ contract, readings listed in the design doc):
   the GPU state is re-synchronised from the oracle's state;
 * edge weights: relative 2e-5 (float logits against the double oracle);
 * community state (centroids bit-exact, sizes, ascending members, edge rows)
-  through the library's checkpoint record.
+  through the library's checkpoint record;
+* optionally (recall_every > 0) the attention-mass recall of the step per
+  query head against the oracle's (attended-row softmax statistics over
+  dense ones): |r_gpu - r_ref| <= 1e-3 r_ref + 1e-6.
 """
 from __future__ import annotations
 
@@ -27,6 +30,10 @@ from long_context_decode_ckv_b200 import synth
 OUT_RTOL = 2e-3
 GAP_EXEMPT = 1e-5
 W_RTOL = 2e-5
+# recall = l_sel exp(m_sel - m) / l from fp32 sums of exps of fp32 logits;
+# a logit carries at most ~D 2^-23 |z| <= 3e-4 of accumulation error for the
+# workloads' |z| <= 20, which moves a probability by the same relative amount
+RECALL_RTOL, RECALL_ATOL = 1e-3, 1e-6
 
 
 @dataclass
@@ -34,6 +41,8 @@ class StepLog:
     step: int
     exempt: list = field(default_factory=list)      # (graph, what, gap)
     max_out_err: float = 0.0
+    max_recall_err: float = 0.0
+    recalls: list = field(default_factory=list)      # oracle recall per checked head
 
 
 def _torch_view(a, dev):
@@ -58,9 +67,11 @@ def config_for(cfg: synth.DecodeConfig, device: int = 0, slack: int = 16,
 
 
 class Lockstep:
-    def __init__(self, wl: synth.Workload, tracked=None, device: int = 0, slack: int = 16):
+    def __init__(self, wl: synth.Workload, tracked=None, device: int = 0, slack: int = 16,
+                 recall_every: int = 0):
         import torch
         self.wl, self.cfg = wl, wl.cfg
+        self.recall_every = recall_every
         cfg = self.cfg
         self.dev = torch.device("cuda", device)
         self.K = _torch_view(wl.K, self.dev)
@@ -105,6 +116,11 @@ class Lockstep:
         n_tok_sel = np.zeros(G, np.int32)
         ckv.ckv_get_step_debug(self.ctx, n_sel, sel, n_tok_sel, n_edges, edges, edge_w, assigned)
         out = self.out.cpu().numpy()
+        rec = None
+        if self.recall_every and i % self.recall_every == 0:
+            rec_t = torch.full((cfg.batch, cfg.n_q_heads), -1.0, dtype=torch.float32, device=self.dev)
+            ckv.ckv_step_recall(self.ctx, self.q[i], self.K, n, rec_t)
+            rec = rec_t.cpu().numpy()
         log = StepLog(i)
         resync = False
         for g in self.tracked:
@@ -129,6 +145,15 @@ class Lockstep:
                 err = float(np.max(np.abs(out[b, h] - ref)) / max(np.max(np.abs(ref)), 1e-30))
                 log.max_out_err = max(log.max_out_err, err)
                 assert err <= OUT_RTOL, f"step {i} graph {g} head {h}: out rel err {err:.3g}"
+            if rec is not None:
+                q_g = np.ascontiguousarray(self.wl.q[i, b, heads])
+                ref_r = oracle.recall(r.m, r.l, *oracle.dense_stats(q_g, self.wl.K[b, kvh], n))
+                for h_i, h in enumerate(heads):
+                    err = abs(float(rec[b, h]) - ref_r[h_i])
+                    log.max_recall_err = max(log.max_recall_err, err)
+                    log.recalls.append(float(ref_r[h_i]))
+                    assert err <= RECALL_RTOL * ref_r[h_i] + RECALL_ATOL, (
+                        f"step {i} graph {g} head {h}: recall {rec[b, h]} vs oracle {ref_r[h_i]}")
             E = int(n_edges[g])
             ge, gw = edges[g, :E], edge_w[g, :E]
             assert E == len(r.edge_col), f"step {i} graph {g}: {E} edges vs {len(r.edge_col)}"
