@@ -13,6 +13,11 @@ The timed loop rotates over `--replicas` independent copies of the layer
 (separate K/V caches and community state, > 18 GB in total), so no step finds
 its working set in the 126 MB L2: inputs larger than L2, no flush.
 
+After the timed steps it also reports, outside the timed region, the
+attention-mass recall of each replica's last step (Figure 3 right: the dense
+softmax mass of the attended rows, per query head) and the time of a dense
+decode attention over the whole cache (the comparator of the sparse step).
+
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle
 (test infrastructure; the only other code here that runs it is the
 cpu_baseline leg) on the same workload instead.
@@ -62,15 +67,28 @@ def kernel_bytes(cfg, T):
 
 # DRAM bytes read + written per launch from one ncu capture (profiles/,
 # k_score_k_select_k_attend_qwen3_8b_n131072_full.md), valid only for the
-# kernel source they were taken on (sha256 prefix of csrc/k_decode.cu)
-PROFILED_TRAFFIC = {"source_sha256": "74f2c59478a341ad", "k_score": 139.442176e6, "k_attend": 69.224448e6}
+# kernel sources they were taken on (bench.source_hash of csrc/)
+PROFILED_TRAFFIC = {"source_sha256": "872a0dc9f517f7db", "k_score": 139.358208e6, "k_attend": 69.187584e6,
+                    "k_dense_stats": 1077.576416e6, "k_dense_attention": 2151.696384e6}
+
+
+def source_hash():
+    """First 16 hex digits of the SHA-256 over every CUDA source of the library
+    (sorted .cu / .cuh of csrc/): the build a capture was taken on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "long_context_decode_ckv_b200", "csrc", "*.cu*"))):
+        h.update(os.path.basename(f).encode())
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel):
-    import hashlib
-    src = os.path.join(ROOT, "long_context_decode_ckv_b200", "csrc", "k_decode.cu")
+    """DRAM bytes per launch from the ncu capture, only while the sources
+    are the ones it was taken on."""
     try:
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        h = source_hash()
     except OSError:
         return None
     return PROFILED_TRAFFIC.get(kernel) if h == PROFILED_TRAFFIC["source_sha256"] else None
@@ -218,6 +236,58 @@ def reference_arm(args, rank, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+def recall_sweep(args, budgets):
+    """Figure 3 (right): attention-mass recall of the retrieved set versus the
+    token budget, on the throughput workload, every 8th of --steps steps."""
+    import torch
+    import long_context_decode_ckv_b200 as ckv
+    from long_context_decode_ckv_b200 import build as ckv_build
+    cfg = CFG
+    wl = synth.make_workload(cfg, workers=max(1, min(16, os.cpu_count() or 1)))
+    ckv_build.build()
+    dev = torch.device("cuda", 0)
+
+    def upload(a):
+        t = torch.from_numpy(a)
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).to(dev)
+
+    K, V, q = upload(wl.K), upload(wl.V), upload(wl.q)
+    out = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
+    rec = torch.empty((cfg.batch, cfg.n_q_heads), dtype=torch.float32, device=dev)
+    steps = min(args.steps, cfg.steps)
+    rows = []
+    for budget in budgets:
+        c = ckv.ckv_config()
+        c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, 128
+        c.n_max, c.max_communities, c.n_sinks = cfg.n_max, cfg.n_comm, cfg.n_sinks
+        c.kappa, c.budget, c.slack = cfg.kappa, budget, 16
+        c.kv_dtype, c.mode, c.device, c.pool_capacity = ckv.CKV_BF16, ckv.CKV_QUERY_GROUP, 0, 0
+        ctx = ckv.ckv_create(c)
+        Kr, Vr = K.clone(), V.clone()        # the steps' community updates stay per budget
+        ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, Kr, cfg.n0)
+        vals, kept = [], []
+        sel_tok = np.zeros(cfg.n_graphs, np.int32)
+        for i in range(steps):
+            n = cfg.n0 + i + 1
+            ckv.ckv_decode_step(ctx, q[i], Kr, Vr, n, out)
+            ckv.ckv_assign_update(ctx, Kr, n)
+            if i % 8 == 0:
+                ckv.ckv_step_recall(ctx, q[i], Kr, n, rec)
+                vals.append(rec.cpu().numpy().copy())
+                ckv.ckv_get_step_debug(ctx, n_tok_sel=sel_tok)
+                kept.append(float(sel_tok.mean()))
+        assert ckv.ckv_last_error(ctx) == ckv.CKV_OK
+        ckv.ckv_destroy(ctx)
+        del Kr, Vr
+        v = np.stack(vals)
+        rows.append({"budget": budget, "mean_tokens_kept": float(np.mean(kept)), "recall_mean": float(v.mean()),
+                     "recall_p10": float(np.quantile(v, 0.1)), "recall_min": float(v.min()),
+                     "checks": int(v.size)})
+    print(json.dumps({"recall_vs_budget": rows, "workload": WORKLOAD, "steps": steps,
+                      "data": "synthetic clustered keys (not a model's attention)"}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -231,12 +301,19 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
     ap.add_argument("--profile-steps", type=int, default=40,
                     help="further steps replayed with per-kernel events (0 = none)")
+    ap.add_argument("--recall-sweep", default="",
+                    help="comma-separated budgets: print the mean attention-mass recall per budget "
+                         "over --steps decode steps instead of timing")
+    ap.add_argument("--dense-steps", type=int, default=20,
+                    help="dense decode comparator launches timed after the sparse steps (0 = none)")
     args = ap.parse_args()
     rank, world, local = rank_env()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         return reference_arm(args, rank, world)
+    if args.recall_sweep:
+        return recall_sweep(args, [int(b) for b in args.recall_sweep.split(",")])
 
     # host-side generation first (spawned pool, before any CUDA call)
     workers = max(1, min(16, (os.cpu_count() or 1) // max(1, world)))
@@ -400,6 +477,52 @@ def main():
                "h2d_bytes_per_step": cfg.batch * (cfg.n_q_heads + 2 * cfg.n_kv_heads) * 128 * eb,
                "d2h_bytes_per_step": cfg.batch * cfg.n_q_heads * 128 * 4}
 
+    # attention-mass recall of each replica's last step (Figure 3 right),
+    # one dense statistics pass over K per replica
+    rec_t = torch.empty((cfg.batch, cfg.n_q_heads), dtype=torch.float32, device=dev)
+    recalls, rec_ms = [], 0.0
+    for r in reps:
+        i = r["i"] - 1
+        # a first call loads the kernel and sizes its grid; the second is timed
+        ckv.ckv_step_recall(r["ctx"], q[i], r["K"], cfg.n0 + i + 1, rec_t, stream)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        ckv.ckv_step_recall(r["ctx"], q[i], r["K"], cfg.n0 + i + 1, rec_t, stream)
+        r1.record(stream)
+        torch.cuda.synchronize(dev)
+        rec_ms += r0.elapsed_time(r1)
+        recalls.append(rec_t.cpu().numpy().copy())
+    recalls = np.stack(recalls)
+    recall = {"mean": float(recalls.mean()), "min": float(recalls.min()), "heads": int(recalls.size),
+              "budget": cfg.budget, "n": int(cfg.n0 + reps[0]["i"]),
+              "kernel_ms": rec_ms / len(reps), "kernel": "k_dense (statistics only)",
+              "achieved_gbs": cfg.batch * cfg.n_kv_heads * (cfg.n0 + reps[0]["i"]) * 256 / (rec_ms / len(reps) / 1e3) / 1e9,
+              "traffic": profiled_traffic("k_dense_stats")}
+
+    # dense decode comparator: every head over the whole cache, same replicas
+    dense = None
+    if args.dense_steps:
+        dout = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
+        for s in range(3):
+            r = reps[s % L]
+            ckv.ckv_dense_decode(r["ctx"], q[r["i"] - 1], r["K"], r["V"], cfg.n0 + r["i"], dout, None, stream)
+        torch.cuda.synchronize(dev)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for s in range(args.dense_steps):
+            r = reps[s % L]
+            ckv.ckv_dense_decode(r["ctx"], q[r["i"] - 1], r["K"], r["V"], cfg.n0 + r["i"], dout, None, stream)
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        dms = d0.elapsed_time(d1) / args.dense_steps
+        n_d = cfg.n0 + reps[0]["i"]
+        dbytes = cfg.batch * cfg.n_kv_heads * n_d * 128 * 2 * 2 + cfg.batch * cfg.n_q_heads * 128 * (2 + 4)
+        dense = {"kernel": "k_dense", "ms_per_step": dms, "steps_per_s": 1e3 / dms,
+                 "algorithmic_bytes": dbytes, "achieved_gbs": dbytes / (dms / 1e3) / 1e9,
+                 "frac": dbytes / (dms / 1e3) / 1e9 / measured_peaks()[0],
+                 "traffic": profiled_traffic("k_dense_attention"),
+                 "sparse_step_speedup": dms / (ms / args.steps)}
+
     for r in reps:
         ckv.ckv_destroy(r["ctx"])
     if pg:
@@ -445,6 +568,7 @@ def main():
         "algorithmic_bytes_per_step": step_bytes, "mean_tokens_kept": T_mean,
         "kernel_ms_per_step": avg,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "recall": recall, "dense_decode": dense,
         "gpu_launches": 3 * args.steps, "clocks": clk.summary(),
         "gen_seconds": t_gen,
     }
