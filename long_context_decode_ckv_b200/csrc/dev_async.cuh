@@ -70,6 +70,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
         : "memory");
 }
 
+// the same with an L2 cache policy (createpolicy) for the source lines
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, unsigned bytes, unsigned long long* bar,
+                                              uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+
 // Programmatic dependent launch.  pdl_wait blocks until the grid this one
 // was launched behind has completed and its memory is visible (a no-op for
 // an ordinary launch); pdl_trigger lets the grid launched behind this one

@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, 
     volatile int* abort_flag = &sm.abort;
     if (warp == 0) {
         if (lane == 0) {
+            const uint64_t pol = l2_evict_first();   // the centroids are streamed once per step
             int issued = 0;
             for (int u = 0; u < nu; ++u) {
                 const int st = u % kScoreNST;
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, 
                 const int g = (int)(gu / upg), c0 = (int)(gu % upg) * 32;
                 const int rows = min(32, d.n_comm - c0);
                 mbar_expect_tx(&sm.full[st], rows * kD * 4);
-                bulk_g2s(sm.ring[st], s.mu + ((int64_t)g * d.Nc + c0) * kD, rows * kD * 4, &sm.full[st]);
+                bulk_g2s_hint(sm.ring[st], s.mu + ((int64_t)g * d.Nc + c0) * kD, rows * kD * 4, &sm.full[st], pol);
                 issued = u + 1;
             }
             // nothing may still be landing when the CTA exits
@@ -746,6 +747,7 @@ __device__ __forceinline__ void warp_rows_mma(const WarpRows& a, const uint32_t*
         qf[ks][1] = (gid < HG) ? q2[(gid * kD + 16 * ks + 2 * tig + 8) / 2] : 0u;
     }
     const int nb = (a.a1 - a.a0 + NB - 1) / NB;
+    const uint64_t pol = l2_evict_first();   // gathered rows are read once per step
     int tok_base = -L::TOKW;
     auto issue = [&](int bb) {
         if (bb < nb) {
@@ -762,8 +764,8 @@ __device__ __forceinline__ void warp_rows_mma(const WarpRows& a, const uint32_t*
                 const bool ok = rbase + row < a.a1;
                 const int64_t src = ok ? (int64_t)tokw[rbase - tok_base + row] * 256 + ch * 16 : 0;
                 const uint32_t so = row * 256 + ((ch ^ (row & 7)) << 4);
-                cp_async16z(dst + so, a.Kb + src, ok);
-                cp_async16z(dst + NB * 256 + so, a.Vb + src, ok);
+                cp_async16z_ef(dst + so, a.Kb + src, ok, pol);
+                cp_async16z_ef(dst + NB * 256 + so, a.Vb + src, ok, pol);
             }
         }
         cp_async_commit();
@@ -1021,35 +1023,53 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
         kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
     }
     // ---- output: every value merged online over the slices; the thread of
-    // a head's first value also leaves that head's max and 1 / sum
-    for (int i = tid; i < HG * kD; i += NT) {
-        const int h = i / kD;
-        float M = -INFINITY, Ls = 0.f, o = 0.f;
-        for (int j0 = 0; j0 < nc; j0 += 8) {   // 8 slices' loads in flight at once
-            float2 mj[8];
-            float oj[8];
+    // a head's first value also leaves that head's max and 1 / sum.  A
+    // thread's IPT values take their loads of a batch of slices together.
+    {
+        constexpr int IPT = (HG * kD + NT - 1) / NT;              // values per thread
+        constexpr int U = (8 / IPT > 1) ? 8 / IPT : 2;            // slices per batch
+        float M[IPT], Ls[IPT], o[IPT];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const bool ok = j0 + u < nc;
-                mj[u] = ok ? __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)(j0 + u) * HG + h) * 2))
-                           : make_float2(-INFINITY, 0.f);
-                oj[u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
+        for (int it = 0; it < IPT; ++it) { M[it] = -INFINITY; Ls[it] = 0.f; o[it] = 0.f; }
+        for (int j0 = 0; j0 < nc; j0 += U) {
+            float2 mj[IPT][U];
+            float oj[IPT][U];
+#pragma unroll
+            for (int it = 0; it < IPT; ++it) {
+                const int i = tid + it * NT;
+                const int h = i / kD;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const bool ok = j0 + u < nc && i < HG * kD;
+                    mj[it][u] = ok ? __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)(j0 + u) * HG + h) * 2))
+                                   : make_float2(-INFINITY, 0.f);
+                    oj[it][u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
+                }
             }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (mj[u].x == -INFINITY) continue;
-                const float mn = fmaxf(M, mj[u].x);
-                const float a = (M == -INFINITY) ? 0.f : __expf(M - mn), c = __expf(mj[u].x - mn);
-                o = o * a + oj[u] * c;
-                Ls = Ls * a + mj[u].y * c;
-                M = mn;
-            }
+            for (int it = 0; it < IPT; ++it)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (mj[it][u].x == -INFINITY) continue;
+                    const float mn = fmaxf(M[it], mj[it][u].x);
+                    const float a = (M[it] == -INFINITY) ? 0.f : __expf(M[it] - mn), c = __expf(mj[it][u].x - mn);
+                    o[it] = o[it] * a + oj[it][u] * c;
+                    Ls[it] = Ls[it] * a + mj[it][u].y * c;
+                    M[it] = mn;
+                }
         }
-        out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o / Ls;
-        if (i % kD == 0) {
-            sM[h] = M;
-            sL[h] = 1.f / Ls;
-            if (s.sel_ml) *reinterpret_cast<float2*>(s.sel_ml + 2 * ((int64_t)b * d.Hq + h0 + h)) = make_float2(M, Ls);
+#pragma unroll
+        for (int it = 0; it < IPT; ++it) {
+            const int i = tid + it * NT;
+            if (i >= HG * kD) continue;
+            const int h = i / kD;
+            out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o[it] / Ls[it];
+            if (i % kD == 0) {
+                sM[h] = M[it];
+                sL[h] = 1.f / Ls[it];
+                if (s.sel_ml)
+                    *reinterpret_cast<float2*>(s.sel_ml + 2 * ((int64_t)b * d.Hq + h0 + h)) = make_float2(M[it], Ls[it]);
+            }
         }
     }
     __syncthreads();
@@ -1183,16 +1203,39 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
     int* tokw = reinterpret_cast<int*>(smem + L::off_tokw) + warp * L::TOKW;
     float* red = reinterpret_cast<float*>(smem + L::off_buf);          // [warps][HG][RSTR]
 
-    // ---- this CTA's pieces.  The graphs' rows and the error word in one
-    // round of loads; then warp 0 lists the pieces, kMaxPieces at a time
-    // (a later round reloads the rows: the staging area is reused)
+    // ---- this CTA's pieces.  Graph-aligned split (at least as many CTAs as
+    // graphs): graph g owns CTAs [g P / G, (g + 1) P / G), each one slice of
+    // its rows, so a CTA needs only its own graph's row count.  Otherwise the
+    // graphs' rows laid end to end are split evenly: all graphs' row counts
+    // and the error word in one round of loads, then warp 0 lists the pieces,
+    // kMaxPieces at a time (a later round reloads the rows: the staging area
+    // is reused).
+    const bool aligned = d.att_aligned && (int)gridDim.x >= G;
     int* sR = reinterpret_cast<int*>(smem + L::off_buf);
-    for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
+    if (aligned) {
+        if (tid == 0) {
+            const int Pa = (int)gridDim.x;
+            const int g = (int)(((long long)(blockIdx.x + 1) * G - 1) / Pa);
+            const int fa = (int)((long long)g * Pa / G), fb = (int)((long long)(g + 1) * Pa / G);
+            Piece pc;
+            pc.g = g;
+            pc.k = (int)blockIdx.x - fa;
+            pc.nc = fb - fa;
+            pc.R = __ldcg(s.meta + (int64_t)g * M_COUNT + M_ROWS);
+            pc.r0 = (int)((int64_t)pc.k * pc.R / pc.nc);
+            pc.r1 = (int)((int64_t)(pc.k + 1) * pc.R / pc.nc);
+            sp[0] = pc;
+            *snp = 1;
+            *snf = 0;
+        }
+    } else {
+        for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
+    }
     const int errv = *(volatile int*)s.err;
     __syncthreads();
     if (errv) return;
     for (int done = 0;; done += kMaxPieces) {
-        if (warp == 0) {
+        if (!aligned && warp == 0) {
             auto rows_of = [&](int g) -> int {
                 return done == 0 ? sR[g] : __ldcg(s.meta + (int64_t)g * M_COUNT + M_ROWS);
             };
@@ -1202,14 +1245,9 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
             for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(kFull, tot, o);
             const int P = (int)min((long long)gridDim.x, tot);
             const long long A = (long long)blockIdx.x * tot / P, B = (long long)(blockIdx.x + 1) * tot / P;
-            // graph-aligned split (at least as many CTAs as graphs): graph g gets
-            // CTAs [f(g), f(g+1)), f(g) = g + floor(P_g * (P - G) / tot), and
-            // each of them one slice of it
-            const bool aligned = d.att_aligned && (int)gridDim.x >= G;
-            const int Pa = (int)gridDim.x;
             int np = 0;                            // pieces seen so far
             long long carry = 0;
-            for (int g0 = 0; g0 < G && (aligned || (int)blockIdx.x < P); g0 += 32) {
+            for (int g0 = 0; g0 < G && (int)blockIdx.x < P; g0 += 32) {
                 const int g = g0 + lane;
                 const int R = (g < G) ? rows_of(g) : 0;
                 long long incl = R;
@@ -1219,31 +1257,18 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
                     if (lane >= o) incl += t;
                 }
                 const long long Pg = carry + incl - R;
-                int fa = 0, fb = 0;
-                if (aligned) {
-                    fa = g + (int)(Pg * (Pa - G) / tot);
-                    fb = g + 1 + (int)((Pg + R) * (Pa - G) / tot);
-                }
-                const bool mine = g < G && (aligned ? ((int)blockIdx.x >= fa && (int)blockIdx.x < fb)
-                                                    : (Pg < B && Pg + R > A));
+                const bool mine = g < G && Pg < B && Pg + R > A;
                 const unsigned bal = __ballot_sync(kFull, mine);
                 if (mine) {
                     const int slot = np + __popc(bal & ((1u << lane) - 1u)) - done;
                     if (slot >= 0 && slot < kMaxPieces) {
                         Piece pc;
                         pc.g = g;
-                        if (aligned) {
-                            pc.k = (int)blockIdx.x - fa;
-                            pc.nc = fb - fa;
-                            pc.r0 = (int)((int64_t)pc.k * R / pc.nc);
-                            pc.r1 = (int)((int64_t)(pc.k + 1) * R / pc.nc);
-                        } else {
-                            pc.r0 = (int)(max(A, Pg) - Pg);
-                            pc.r1 = (int)(min(B, Pg + R) - Pg);
-                            const int f = share_of(Pg, tot, P);
-                            pc.k = (int)blockIdx.x - f;
-                            pc.nc = share_of(Pg + R - 1, tot, P) - f + 1;
-                        }
+                        pc.r0 = (int)(max(A, Pg) - Pg);
+                        pc.r1 = (int)(min(B, Pg + R) - Pg);
+                        const int f = share_of(Pg, tot, P);
+                        pc.k = (int)blockIdx.x - f;
+                        pc.nc = share_of(Pg + R - 1, tot, P) - f + 1;
                         pc.R = R;
                         sp[slot] = pc;
                     }

@@ -84,6 +84,7 @@ __device__ __forceinline__ void warp_tiles_bf16(const char* __restrict__ Kb, con
     const int gid = lane >> 2;
     const int first = t0 + warp;
     const int nb = (t1 > first) ? (t1 - first + kDnWarps - 1) / kDnWarps : 0;
+    const uint64_t pol = l2_evict_first();   // the cache is streamed once
     auto issue = [&](int bb) {
         if (bb < nb) {
             const uint32_t dst = smem_u32(wbuf + (bb % kDnBuf) * STAGE);
@@ -95,8 +96,8 @@ __device__ __forceinline__ void warp_tiles_bf16(const char* __restrict__ Kb, con
                 const bool ok = rbase + row < n;
                 const int64_t src = ok ? (int64_t)(rbase + row) * 256 + ch * 16 : 0;
                 const uint32_t so = row * 256 + ((ch ^ (row & 7)) << 4);
-                cp_async16z(dst + so, Kb + src, ok);
-                if (WV) cp_async16z(dst + kTileBytes + so, Vb + src, ok);
+                cp_async16z_ef(dst + so, Kb + src, ok, pol);
+                if (WV) cp_async16z_ef(dst + kTileBytes + so, Vb + src, ok, pol);
             }
         }
         cp_async_commit();
@@ -200,6 +201,7 @@ __device__ __forceinline__ void warp_tiles_f32(const char* __restrict__ Kb, cons
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int first = t0 + warp;
     const int nb = (t1 > first) ? (t1 - first + kDnWarps - 1) / kDnWarps : 0;
+    const uint64_t pol = l2_evict_first();   // the cache is streamed once
     auto issue = [&](int bb) {
         if (bb < nb) {
             const uint32_t dst = smem_u32(wbuf + (bb % kDnBuf) * STAGE);
@@ -208,8 +210,8 @@ __device__ __forceinline__ void warp_tiles_f32(const char* __restrict__ Kb, cons
             for (int row = 0; row < 8; ++row) {
                 const bool ok = rbase + row < n;
                 const int64_t src = ok ? (int64_t)(rbase + row) * 512 + lane * 16 : 0;
-                cp_async16z(dst + row * 512 + lane * 16, Kb + src, ok);
-                if (WV) cp_async16z(dst + kTileBytes + row * 512 + lane * 16, Vb + src, ok);
+                cp_async16z_ef(dst + row * 512 + lane * 16, Kb + src, ok, pol);
+                if (WV) cp_async16z_ef(dst + kTileBytes + row * 512 + lane * 16, Vb + src, ok, pol);
             }
         }
         cp_async_commit();
