@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
                                        ctypes.POINTER(StepInfo)]
         L.ckvo_row_ptr.restype = i64
         L.ckvo_row_ptr.argtypes = [i64, i32, i32]
+        L.ckvo_prefill_rows_grouped.argtypes = [i32, i32, i32, i32, i32, P, P, i32, P, i32, P, P, P, P]
         L.ckvo_dense_stats.argtypes = [i32, i32, P, i32, P, i32, i32, P, P]
         L.ckvo_prefill_rows.argtypes = [i32, i32, i32, i32, P, P, i32, P, i32, P, P, P, P]
         _lib = L
@@ -180,6 +181,23 @@ def prefill_rows(Q: np.ndarray, K: np.ndarray, rows, n_sinks: int, kappa: int):
     gap = np.empty(R, np.float32)
     lib().ckvo_prefill_rows(n, D, n_sinks, kappa, _p(Q), _p(K), _dtype_code(Q),
                             _p(rows), R, _p(col), _p(w), _p(deg), _p(gap))
+    return col, w, deg, gap
+
+
+def prefill_rows_grouped(Q: np.ndarray, K: np.ndarray, rows, n_sinks: int, kappa: int):
+    """Query-group aggregated prefill rows: Q [nh][n][D] (the group's heads),
+    K [n][D].  Returns (col [R][kappa], w [R][kappa], deg [R], gap [R])."""
+    Q = np.ascontiguousarray(Q)
+    K = np.ascontiguousarray(K)
+    rows = np.ascontiguousarray(rows, np.int32)
+    nh, n, D = Q.shape
+    R = len(rows)
+    col = np.full((R, kappa), -1, np.int32)
+    w = np.zeros((R, kappa), np.float32)
+    deg = np.empty(R, np.int32)
+    gap = np.empty(R, np.float32)
+    lib().ckvo_prefill_rows_grouped(n, D, n_sinks, kappa, nh, _p(Q), _p(K), _dtype_code(Q),
+                                    _p(rows), R, _p(col), _p(w), _p(deg), _p(gap))
     return col, w, deg, gap
 
 

@@ -486,3 +486,62 @@ void ckvo_prefill_rows(int n, int D, int n_sinks, int kappa, const void* Q, cons
     }
     free(z);
 }
+
+/* ---- NEXT f2: query-group aggregated prefill graph ---------------------- */
+/* The abstract contrasts one graph per query head with query-group graph
+ * aggregation.  Reading for the prefill graph of a group: one graph per KV
+ * head, shared by its nh query heads; for row i every head h has its own
+ * causal softmax p_hij over j in [0, i] (z_hij = q_hi.k_j / sqrt(D)), the
+ * edge weight is their sum w_ij = sum_h p_hij (rounded to float, the value
+ * ranked), and the row's edges are the top-kappa j in [S, i-1] by
+ * (w desc, j asc) -- the prefill counterpart of the decode edge rule.
+ * Q holds the group's heads [nh][n][D]; K is the KV head's keys [n][D]. */
+void ckvo_prefill_rows_grouped(int n, int D, int n_sinks, int kappa, int nh, const void* Q, const void* K,
+                               int dtype, const int32_t* rows, int n_rows,
+                               int32_t* col, float* w, int32_t* deg, float* gap)
+{
+    double* z = (double*)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    double* ws = (double*)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    for (int rr = 0; rr < n_rows; ++rr) {
+        const int i = rows[rr];
+        for (int j = 0; j <= i; ++j) ws[j] = 0.0;
+        for (int h = 0; h < nh; ++h) {
+            const int64_t qrow = ((int64_t)h * n + i) * D;
+            double m = -INFINITY;
+            for (int j = 0; j <= i; ++j) {
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += elem(Q, dtype, qrow + d) * elem(K, dtype, (int64_t)j * D + d);
+                z[j] = dot * inv_sqrt_d;
+                if (z[j] > m) m = z[j];
+            }
+            double l = 0.0;
+            for (int j = 0; j <= i; ++j) l += exp(z[j] - m);
+            for (int j = 0; j <= i; ++j) ws[j] += exp(z[j] - m) / l;
+        }
+        float bw[CKVO_KMAX + 1];
+        int32_t bj[CKVO_KMAX + 1];
+        int nb = 0;
+        for (int j = n_sinks; j < i; ++j) {
+            const float wf = (float)ws[j];
+            int pos = nb;
+            while (pos > 0 && bw[pos - 1] < wf) --pos;   /* equal w: earlier j stays ahead */
+            if (pos > kappa) continue;
+            int last = nb < kappa + 1 ? nb : kappa;
+            for (int k = last; k > pos; --k) { bw[k] = bw[k - 1]; bj[k] = bj[k - 1]; }
+            bw[pos] = wf;
+            bj[pos] = j;
+            if (nb < kappa + 1) ++nb;
+        }
+        int e = nb < kappa ? nb : kappa;
+        deg[rr] = e;
+        for (int k = 0; k < e; ++k) {
+            col[(size_t)rr * kappa + k] = bj[k];
+            w[(size_t)rr * kappa + k] = bw[k];
+        }
+        gap[rr] = (nb > kappa) ? (float)relgap(bw[kappa - 1], bw[kappa]) : INFINITY;
+    }
+    free(ws);
+    free(z);
+}

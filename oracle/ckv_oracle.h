@@ -128,6 +128,13 @@ void ckvo_prefill_rows(int n, int D, int n_sinks, int kappa, const void* Q, cons
 void ckvo_dense_stats(int n_heads, int D, const void* q, int q_dtype, const void* K, int kv_dtype, int n,
                       double* m_out, double* l_out);
 
+/* Query-group aggregated prefill rows: the group's nh heads (Q [nh][n][D])
+ * share one graph over K [n][D]; w_ij = sum_h p_hij, top-kappa of j in
+ * [S, i-1] by (w desc, j asc).  Outputs as ckvo_prefill_rows. */
+void ckvo_prefill_rows_grouped(int n, int D, int n_sinks, int kappa, int nh, const void* Q, const void* K,
+                               int dtype, const int32_t* rows, int n_rows,
+                               int32_t* col, float* w, int32_t* deg, float* gap);
+
 #ifdef __cplusplus
 }
 #endif

@@ -414,3 +414,59 @@ def test_recall_grows_with_budget(oracle_lib):
             assert np.all(rec >= prev - 1e-12)
         prev = rec
     np.testing.assert_allclose(prev, 1.0, rtol=1e-12)
+
+
+# ------------------------------------- NEXT f2 query-group aggregated prefill
+def _grouped_brute(Q, K, S, kap):
+    """Library softmax per head (torch, float64, causal), summed over the
+    heads, rounded to float32; lexsort by (w desc, j asc) per row."""
+    nh, n, D = Q.shape
+    Qt = torch.from_numpy(_f32(Q).astype(np.float64))
+    Kt = torch.from_numpy(_f32(K).astype(np.float64))
+    z = Qt @ Kt.T / math.sqrt(D)                                          # [nh][n][n]
+    z = z.masked_fill(torch.triu(torch.ones(n, n, dtype=torch.bool), 1), -math.inf)
+    wsum = torch.softmax(z, dim=2).sum(0).numpy().astype(np.float32)      # [n][n]
+    out = []
+    for i in range(n):
+        cand = np.arange(S, i)
+        order = cand[np.lexsort((cand, -wsum[i, cand]))][:kap]
+        out.append((order, wsum[i, order]))
+    return out
+
+
+@pytest.mark.parametrize("nh,bf16", [(1, False), (2, True), (4, True), (4, False)])
+def test_grouped_prefill_matches_library_softmax(oracle_lib, nh, bf16):
+    rng = np.random.default_rng(40 + nh)
+    n, D, S, kap = 70, 128, 4, 8
+    Q = (rng.standard_normal((nh, n, D)) * 1.5).astype(np.float32)
+    K = rng.standard_normal((n, D)).astype(np.float32)
+    if bf16:
+        Q, K = synth.to_bf16_bits(Q), synth.to_bf16_bits(K)
+    col, w, deg, _ = oracle.prefill_rows_grouped(Q, K, np.arange(n), S, kap)
+    ref = _grouped_brute(Q, K, S, kap)
+    for i in range(n):
+        order, wr = ref[i]
+        assert deg[i] == min(kap, max(0, i - S))
+        assert list(col[i, :deg[i]]) == list(order), i
+        np.testing.assert_allclose(w[i, :deg[i]], wr, rtol=1e-6, atol=0)
+        assert w[i, :deg[i]].sum() <= nh * (1 + 1e-6)
+
+
+def test_grouped_prefill_special_cases(oracle_lib):
+    rng = np.random.default_rng(9)
+    n, D, S, kap = 90, 128, 3, 6
+    q = (rng.standard_normal((n, D)) * 2).astype(np.float32)
+    K = rng.standard_normal((n, D)).astype(np.float32)
+    rows = np.arange(n)
+    # one head: the per-head prefill graph (weights are that head's p)
+    c1, w1, d1, g1 = oracle.prefill_rows(q, K, rows, S, kap)
+    cg, wg, dg, _ = oracle.prefill_rows_grouped(q[None], K, rows, S, kap)
+    np.testing.assert_array_equal(dg, d1)
+    for i in range(n):
+        if g1[i] > 1e-5:                      # no near-tie at the cutoff
+            assert set(cg[i, :dg[i]].tolist()) == set(c1[i, :d1[i]].tolist())
+    np.testing.assert_allclose(np.sort(wg, 1), np.sort(w1, 1), rtol=1e-6)
+    # the same head twice: the same edges, every weight doubled
+    c2, w2, d2, _ = oracle.prefill_rows_grouped(np.stack([q, q]), K, rows, S, kap)
+    np.testing.assert_array_equal(c2, cg)
+    np.testing.assert_allclose(w2, 2 * wg, rtol=1e-6)
