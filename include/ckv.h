@@ -109,6 +109,28 @@ ckv_status ckv_build_graph(int n_heads, int n, int head_dim, int n_sinks, int ka
                            ckv_dtype dtype, const void* Q, const void* K,
                            int64_t* row_ptr, int32_t* col, float* w, void* stream);
 
+/* Query-group aggregated prefill graph -- the abstract's query-group graph
+ * aggregation applied to Figure 1, step (1): one graph per KV head, shared
+ * by its `group` query heads.  For row i every head h of the group has its
+ * own causal softmax p_hij over j in [0, i] (z_hij = q_hi.k_j / sqrt(D));
+ * the edge weight is w_ij = sum_h p_hij and the row's edges are its
+ * top-kappa j in [S, i-1] by (w desc, j asc).  With group = 1 this is
+ * ckv_build_graph with the weights ranked instead of the scores.
+ * Q: [n_kv_heads * group][n][D] bf16 (query heads u*group .. u*group+group-1
+ * belong to KV head u), K: [n_kv_heads][n][D] bf16, device.  group is 1, 2
+ * or 4.  workspace: device scratch of ckv_build_graph_grouped_workspace()
+ * bytes, 16-byte aligned, owned by the caller (per-head row statistics of
+ * the first pass; undefined afterwards).  Outputs as ckv_build_graph, per
+ * KV head: row_ptr [n_kv_heads][n+1], col and w [n_kv_heads][E].  Two
+ * kernels (row statistics, then the grouped graph on the tensor cores); the
+ * n x n matrices are never stored.  Asynchronous.  A bounded wait that runs
+ * out marks row_ptr[u][0] = -1.
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_CUDA. */
+size_t ckv_build_graph_grouped_workspace(int n_kv_heads, int group, int n);
+ckv_status ckv_build_graph_grouped(int n_kv_heads, int group, int n, int head_dim, int n_sinks, int kappa,
+                                   ckv_dtype dtype, const void* Q, const void* K, void* workspace,
+                                   int64_t* row_ptr, int32_t* col, float* w, void* stream);
+
 /* Initial partition -- Figure 1, step (2): community c of graph g holds the
  * positions j in [S, n) with labels[g][j] == c (ascending); its centroid is
  * the mean of those keys (float, summed in double).  labels: int32

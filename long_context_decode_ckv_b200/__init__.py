@@ -90,6 +90,10 @@ def lib() -> ctypes.CDLL:
     L.ckv_aux_bytes.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.ckv_attend_rows_static.restype = st
     L.ckv_attend_rows_static.argtypes = [ctypes.POINTER(ckv_config), P, P, P, I, P, P, I, P, P]
+    L.ckv_build_graph_grouped_workspace.restype = sz
+    L.ckv_build_graph_grouped_workspace.argtypes = [I, I, I]
+    L.ckv_build_graph_grouped.restype = st
+    L.ckv_build_graph_grouped.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P]
     L.ckv_step_recall.restype = st
     L.ckv_step_recall.argtypes = [P, P, P, I, P, P]
     L.ckv_dense_decode.restype = st
@@ -153,6 +157,17 @@ def ckv_build_graph(n_heads, n, head_dim, n_sinks, kappa, dtype, Q, K, row_ptr, 
     _check("ckv_build_graph", lib().ckv_build_graph(
         n_heads, n, head_dim, n_sinks, kappa, dtype, _ptr(Q), _ptr(K), _ptr(row_ptr), _ptr(col),
         _ptr(w), _stream(stream)))
+
+
+def ckv_build_graph_grouped_workspace(n_kv_heads, group, n) -> int:
+    return lib().ckv_build_graph_grouped_workspace(n_kv_heads, group, n)
+
+
+def ckv_build_graph_grouped(n_kv_heads, group, n, head_dim, n_sinks, kappa, dtype, Q, K, workspace, row_ptr, col, w,
+                            stream=None):
+    _check("ckv_build_graph_grouped", lib().ckv_build_graph_grouped(
+        n_kv_heads, group, n, head_dim, n_sinks, kappa, dtype, _ptr(Q), _ptr(K), _ptr(workspace), _ptr(row_ptr),
+        _ptr(col), _ptr(w), _stream(stream)))
 
 
 def ckv_init_communities(ctx, labels, labels_on_device, n_communities, K, n, stream=None):

@@ -742,3 +742,29 @@ CKV_API ckv_status ckv_build_graph(int n_heads, int n, int head_dim, int n_sinks
     CKV_CUDA(ckv::launch_build_graph(n_heads, n, n_sinks, kappa, Q, K, row_ptr, col, w, (cudaStream_t)stream));
     return CKV_OK;
 }
+
+CKV_API size_t ckv_build_graph_grouped_workspace(int n_kv_heads, int group, int n)
+{
+    if (n_kv_heads < 1 || group < 1 || n < 1) return 0;
+    return ckv::build_graph_grouped_stats_floats(n_kv_heads, group, n) * sizeof(float);
+}
+
+CKV_API ckv_status ckv_build_graph_grouped(int n_kv_heads, int group, int n, int head_dim, int n_sinks, int kappa,
+                                           ckv_dtype dtype, const void* Q, const void* K, void* workspace,
+                                           int64_t* row_ptr, int32_t* col, float* w, void* stream)
+{
+    if (n_kv_heads < 1 || (group != 1 && group != 2 && group != 4) || n < 1 || head_dim != ckv::kD ||
+        n_sinks < 0 || kappa < 1 || kappa > ckv::kMaxKappa || dtype != CKV_BF16 || !Q || !K || !workspace ||
+        !row_ptr || !col || !w)
+        return CKV_ERR_INVALID_ARG;
+    if ((int64_t)n_kv_heads * group * n > INT32_MAX / 2) return CKV_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15) return CKV_ERR_INVALID_ARG;
+    cudaPointerAttributes a;
+    CKV_CUDA(cudaPointerGetAttributes(&a, Q));
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return CKV_ERR_INVALID_ARG;
+    CKV_CUDA(cudaSetDevice(a.device));
+    CKV_CUDA(ckv::launch_build_graph_grouped(n_kv_heads, group, n, n_sinks, kappa, Q, K,
+                                             static_cast<float*>(workspace), row_ptr, col, w,
+                                             (cudaStream_t)stream));
+    return CKV_OK;
+}

@@ -121,6 +121,11 @@ cudaError_t launch_init_centroids(const DevState& s, const Dims& d, const void* 
 // prefill (k_prefill.cu)
 cudaError_t launch_build_graph(int H, int n, int S, int kappa, const void* Q, const void* K,
                                int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st);
+// query-group aggregated prefill graph: per-head row statistics into stats
+// (build_graph_grouped_stats_floats floats), then one graph per KV head
+size_t build_graph_grouped_stats_floats(int Hkv, int group, int n);
+cudaError_t launch_build_graph_grouped(int Hkv, int group, int n, int S, int kappa, const void* Q, const void* K,
+                                       float* stats, int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st);
 
 // device error word: first error wins
 __device__ __forceinline__ void set_error(int* err, int code) { atomicCAS(err, 0, code); }

@@ -118,17 +118,21 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr)
     return d;
 }
 
-// instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kBM >> 4) << 24);
+// instruction descriptor: D f32, A and B bf16, both K-major, M = 128, N = n
+constexpr uint32_t idesc_n(int n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+constexpr uint32_t kIdesc = idesc_n(kBN);
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum)
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum,
+                                          uint32_t idesc = kIdesc)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum)
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
         : "memory");
 }
 
@@ -173,11 +177,15 @@ __device__ __forceinline__ int64_t row_offset(int64_t i, int S, int kappa)
     return a * (a + 1) / 2 + max((int64_t)0, i - (S + kappa + 1)) * kappa;
 }
 
-template <int KM>
+// STATS: no edges; each row's (max of z log2(e), sum of 2^(z log2(e) - max))
+// go to stats[h][i][2] instead (the first pass of the query-group graph),
+// and a bounded wait that runs out sets the int word after them.
+// group: query heads per KV head (the K rows of head h are those of h / group).
+template <int KM, bool STATS>
 __global__ void __launch_bounds__(kThreads, 1)
 k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int H, int n,
-               int S, int kappa, int64_t* __restrict__ row_ptr, int32_t* __restrict__ col,
-               float* __restrict__ w)
+               int S, int kappa, int group, int64_t* __restrict__ row_ptr, int32_t* __restrict__ col,
+               float* __restrict__ w, float* __restrict__ stats)
 {
     extern __shared__ unsigned char smem_raw[];
     PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>(
@@ -218,8 +226,8 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 const int s = t % kStages;
                 if (!mbar_wait(&sm.bar_kempty[s], ((t / kStages) & 1) ^ 1, abort)) break;
                 mbar_expect_tx(&sm.bar_kfull[s], kTileBytes);
-                tma_load_3d(sm.k[s], &tmK, &sm.bar_kfull[s], 0, t * kBN, h);
-                tma_load_3d(sm.k[s] + kHalfBytes, &tmK, &sm.bar_kfull[s], 64, t * kBN, h);
+                tma_load_3d(sm.k[s], &tmK, &sm.bar_kfull[s], 0, t * kBN, h / group);
+                tma_load_3d(sm.k[s] + kHalfBytes, &tmK, &sm.bar_kfull[s], 64, t * kBN, h / group);
                 issued = t + 1;
             }
             // do not leave with copies in flight: the last load of every stage has landed
@@ -295,11 +303,222 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                 for (int k = 0; k < 32; ++k) ps += ex2(fmaf(v[k], kLog2eOverSqrtD, -m2));
                 l += ps;
-                // top-KM candidates j in [S, i-1], ranked by the raw score
+                if constexpr (!STATS) {
+                    // top-KM candidates j in [S, i-1], ranked by the raw score
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int j = j0 + k;
+                        const float a = v[k];
+                        if (a > vals[KM - 1] && j >= S && j < i) {
+#pragma unroll
+                            for (int p = KM - 1; p > 0; --p) {
+                                const float up = vals[p - 1];
+                                const int upi = idx[p - 1];
+                                const bool shift = up < a;
+                                const bool land = !shift && vals[p] < a;
+                                vals[p] = shift ? up : (land ? a : vals[p]);
+                                idx[p] = shift ? upi : (land ? j : idx[p]);
+                            }
+                            if (vals[0] < a) { vals[0] = a; idx[0] = j; }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.bar_aempty[b]);
+        }
+        if (STATS && row_ok && !*abort) {
+            stats[((int64_t)h * n + i) * 2] = m2;
+            stats[((int64_t)h * n + i) * 2 + 1] = l;
+        } else if (row_ok && !*abort) {
+            const int64_t base = (int64_t)h * E + row_offset(i, S, kappa);
+            const int deg = (int)min((int64_t)kappa, max((int64_t)0, (int64_t)i - S));
+            const float inv_l = 1.f / l;
+#pragma unroll
+            for (int k = 0; k < KM; ++k) {
+                if (k < deg) {
+                    col[base + k] = idx[k];
+                    w[base + k] = ex2(fmaf(vals[k], kLog2eOverSqrtD, -m2)) * inv_l;
+                }
+            }
+            row_ptr[(int64_t)h * (n + 1) + i] = row_offset(i, S, kappa);
+            if (i == n - 1) row_ptr[(int64_t)h * (n + 1) + n] = E;
+        }
+    }
+    __syncthreads();
+    if (*abort && threadIdx.x == 0) {
+        // the grouped pass reads the failure word after the statistics
+        if (STATS) atomicExch(reinterpret_cast<int*>(stats + (int64_t)H * n * 2), 1);
+        else row_ptr[(int64_t)h * (n + 1)] = -1;
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+    }
+}
+
+// ---- query-group aggregated graph, second pass --------------------------
+// One CTA per (KV head u, 128-row query block), heaviest blocks first.  The
+// group's NH query blocks stay in shared memory; every K tile (BN rows)
+// feeds NH MMAs, one TMEM accumulator per head, double buffered
+// (2 x NH x BN <= 512 columns).  Epilogue thread = one row: it adds the
+// heads' probabilities 2^(z log2(e) - c_h), c_h = max_h + log2(sum_h) from
+// the first pass, and keeps the row's top-KM by that sum.
+template <int NH>
+struct __align__(1024) GroupSmem {
+    static constexpr int BN = (NH >= 4) ? 64 : 128;            // K rows per tile
+    static constexpr int KT = BN * 256;                         // one K tile (two 64-column halves)
+    unsigned char q[NH][kTileBytes];
+    unsigned char k[kStages][KT];
+    unsigned long long bar_q;
+    unsigned long long bar_kfull[kStages];
+    unsigned long long bar_kempty[kStages];
+    unsigned long long bar_afull[2];
+    unsigned long long bar_aempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int KM, int NH>
+__global__ void __launch_bounds__(kThreads, 1)
+k_prefill_group(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int Hkv, int n,
+                int S, int kappa, const float* __restrict__ stats, int64_t* __restrict__ row_ptr,
+                int32_t* __restrict__ col, float* __restrict__ w)
+{
+    using GS = GroupSmem<NH>;
+    constexpr int BN = GS::BN, KT = GS::KT, KH = BN * 128;
+    constexpr uint32_t TCOLS = (2 * NH * BN <= 256) ? 256u : 512u;
+    constexpr uint32_t IDESC = idesc_n(BN);
+    static_assert(2 * NH * BN <= 512, "accumulators must fit the tensor memory");
+    extern __shared__ unsigned char smem_raw[];
+    GS& sm = *reinterpret_cast<GS*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nqb = (n + kBM - 1) / kBM;
+    const int qb = nqb - 1 - (int)(blockIdx.x / Hkv);
+    const int u = (int)(blockIdx.x % Hkv);
+    const int i0 = qb * kBM;
+    const int ntiles = min(i0 + kBM - 1, n - 1) / BN + 1;       // tiles holding a column <= the block's last row
+    const int64_t E = row_offset(n, S, kappa);
+    const int Hq = Hkv * NH;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_q, 1);
+        for (int s = 0; s < kStages; ++s) { mbar_init(&sm.bar_kfull[s], 1); mbar_init(&sm.bar_kempty[s], 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&sm.bar_afull[b], 1); mbar_init(&sm.bar_aempty[b], 4); }
+        // a first pass that gave up leaves its failure word set
+        sm.abort = *reinterpret_cast<const volatile int*>(stats + (int64_t)Hq * n * 2) != 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&sm.tmem_base)), "r"(TCOLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int* abort = &sm.abort;
+    const bool failed = *abort != 0;
+
+    if (failed) {
+        // nothing to do: the cleanup below reports the failure
+    } else if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_expect_tx(&sm.bar_q, NH * kTileBytes);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                tma_load_3d(sm.q[h], &tmQ, &sm.bar_q, 0, i0, u * NH + h);
+                tma_load_3d(sm.q[h] + kHalfBytes, &tmQ, &sm.bar_q, 64, i0, u * NH + h);
+            }
+            int issued = 0;
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % kStages;
+                if (!mbar_wait(&sm.bar_kempty[s], ((t / kStages) & 1) ^ 1, abort)) break;
+                mbar_expect_tx(&sm.bar_kfull[s], KT);
+                tma_load_3d(sm.k[s], &tmK, &sm.bar_kfull[s], 0, t * BN, u);
+                tma_load_3d(sm.k[s] + KH, &tmK, &sm.bar_kfull[s], 64, t * BN, u);
+                issued = t + 1;
+            }
+            for (int t = max(0, issued - kStages); t < issued; ++t)
+                mbar_wait(&sm.bar_kfull[t % kStages], (t / kStages) & 1, abort);
+            mbar_wait(&sm.bar_q, 0, abort);
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------- MMA
+        if (lane == 0) {
+            int committed = 0;
+            if (mbar_wait(&sm.bar_q, 0, abort)) {
+                for (int t = 0; t < ntiles; ++t) {
+                    const int s = t % kStages, b = t & 1;
+                    if (!mbar_wait(&sm.bar_kfull[s], (t / kStages) & 1, abort)) break;
+                    if (!mbar_wait(&sm.bar_aempty[b], ((t >> 1) & 1) ^ 1, abort)) break;
+                    tc_fence_after();
+                    const uint32_t ka = smem_u32(sm.k[s]);
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        const uint32_t qa = smem_u32(sm.q[h]);
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                umma_bf16(tmem + (uint32_t)((b * NH + h) * BN), umma_desc(qa + c * kHalfBytes + k * 32),
+                                          umma_desc(ka + c * KH + k * 32), (c | k) != 0, IDESC);
+                    }
+                    umma_commit(&sm.bar_kempty[s]);
+                    umma_commit(&sm.bar_afull[b]);
+                    committed = t + 1;
+                }
+            }
+            if (committed > 0) {
+                const int t = committed - 1;
+                mbar_wait(&sm.bar_afull[t & 1], (t >> 1) & 1, abort);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const int i = i0 + r;
+        const bool row_ok = i < n;
+        float ch[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+            ch[h] = 0.f;
+            if (row_ok) {
+                const float2 ml = *reinterpret_cast<const float2*>(stats + ((int64_t)(u * NH + h) * n + i) * 2);
+                ch[h] = ml.x + __log2f(ml.y);
+            }
+        }
+        float vals[KM];
+        int idx[KM];
+#pragma unroll
+        for (int k = 0; k < KM; ++k) { vals[k] = -INFINITY; idx[k] = -1; }
+        for (int t = 0; t < ntiles; ++t) {
+            const int b = t & 1;
+            if (!mbar_wait(&sm.bar_afull[b], (t >> 1) & 1, abort)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                float ws[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) ws[k] = 0.f;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    float v[32];
+                    __syncwarp();   // tcgen05.ld is warp-collective
+                    tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((b * NH + h) * BN + cc * 32), v);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) ws[k] += ex2(fmaf(v[k], kLog2eOverSqrtD, -ch[h]));
+                }
+                if (!row_ok) continue;
+                const int j0 = t * BN + cc * 32;
+                // top-KM candidates j in [S, i-1] by the summed probability
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
                     const int j = j0 + k;
-                    const float a = v[k];
+                    const float a = ws[k];
                     if (a > vals[KM - 1] && j >= S && j < i) {
 #pragma unroll
                         for (int p = KM - 1; p > 0; --p) {
@@ -319,25 +538,24 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (lane == 0) mbar_arrive(&sm.bar_aempty[b]);
         }
         if (row_ok && !*abort) {
-            const int64_t base = (int64_t)h * E + row_offset(i, S, kappa);
+            const int64_t base = (int64_t)u * E + row_offset(i, S, kappa);
             const int deg = (int)min((int64_t)kappa, max((int64_t)0, (int64_t)i - S));
-            const float inv_l = 1.f / l;
 #pragma unroll
             for (int k = 0; k < KM; ++k) {
                 if (k < deg) {
                     col[base + k] = idx[k];
-                    w[base + k] = ex2(fmaf(vals[k], kLog2eOverSqrtD, -m2)) * inv_l;
+                    w[base + k] = vals[k];
                 }
             }
-            row_ptr[(int64_t)h * (n + 1) + i] = row_offset(i, S, kappa);
-            if (i == n - 1) row_ptr[(int64_t)h * (n + 1) + n] = E;
+            row_ptr[(int64_t)u * (n + 1) + i] = row_offset(i, S, kappa);
+            if (i == n - 1) row_ptr[(int64_t)u * (n + 1) + n] = E;
         }
     }
     __syncthreads();
-    if (*abort && threadIdx.x == 0) row_ptr[(int64_t)h * (n + 1)] = -1;
+    if (*abort && threadIdx.x == 0) row_ptr[(int64_t)u * (n + 1)] = -1;
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS) : "memory");
     }
 }
 
@@ -354,31 +572,56 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode()
     return fn;
 }
 
-// [H][n][128] bf16 viewed as a 3-D tensor, box = 64 columns x 128 rows x 1 head
-bool make_map(CUtensorMap* m, const void* base, int H, int n)
+// [H][n][128] bf16 viewed as a 3-D tensor, box = 64 columns x box_rows rows x 1 head
+bool make_map(CUtensorMap* m, const void* base, int H, int n, int box_rows = 128)
 {
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[3] = {128, (cuuint64_t)n, (cuuint64_t)H};
     cuuint64_t strides[2] = {128 * 2, (cuuint64_t)n * 128 * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KM>
-cudaError_t launch_km(const CUtensorMap& mq, const CUtensorMap& mk, int H, int n, int S, int kappa,
-                      int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st)
+template <int KM, bool STATS>
+cudaError_t launch_km(const CUtensorMap& mq, const CUtensorMap& mk, int H, int n, int S, int kappa, int group,
+                      int64_t* row_ptr, int32_t* col, float* w, float* stats, cudaStream_t st)
 {
     const size_t smem = sizeof(PrefillSmem) + 1024;
-    auto kern = k_prefill_topk<KM>;
+    auto kern = k_prefill_topk<KM, STATS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int nqb = (n + kBM - 1) / kBM;
-    kern<<<H * nqb, kThreads, smem, st>>>(mq, mk, H, n, S, kappa, row_ptr, col, w);
+    kern<<<H * nqb, kThreads, smem, st>>>(mq, mk, H, n, S, kappa, group, row_ptr, col, w, stats);
     return cudaGetLastError();
+}
+
+template <int KM, int NH>
+cudaError_t launch_group(const CUtensorMap& mq, const CUtensorMap& mk, int Hkv, int n, int S, int kappa,
+                         const float* stats, int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st)
+{
+    const size_t smem = sizeof(GroupSmem<NH>) + 1024;
+    auto kern = k_prefill_group<KM, NH>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int nqb = (n + kBM - 1) / kBM;
+    kern<<<Hkv * nqb, kThreads, smem, st>>>(mq, mk, Hkv, n, S, kappa, stats, row_ptr, col, w);
+    return cudaGetLastError();
+}
+
+template <int KM>
+cudaError_t launch_group_nh(int nh, const CUtensorMap& mq, const CUtensorMap& mk, int Hkv, int n, int S, int kappa,
+                            const float* stats, int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st)
+{
+    switch (nh) {
+        case 1: return launch_group<KM, 1>(mq, mk, Hkv, n, S, kappa, stats, row_ptr, col, w, st);
+        case 2: return launch_group<KM, 2>(mq, mk, Hkv, n, S, kappa, stats, row_ptr, col, w, st);
+        case 4: return launch_group<KM, 4>(mq, mk, Hkv, n, S, kappa, stats, row_ptr, col, w, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -389,9 +632,35 @@ cudaError_t launch_build_graph(int H, int n, int S, int kappa, const void* Q, co
     if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K)) & 15) return cudaErrorInvalidValue;
     CUtensorMap mq, mk;
     if (!make_map(&mq, Q, H, n) || !make_map(&mk, K, H, n)) return cudaErrorInvalidValue;
-    if (kappa <= 8) return launch_km<8>(mq, mk, H, n, S, kappa, row_ptr, col, w, st);
-    if (kappa <= 16) return launch_km<16>(mq, mk, H, n, S, kappa, row_ptr, col, w, st);
-    return launch_km<32>(mq, mk, H, n, S, kappa, row_ptr, col, w, st);
+    if (kappa <= 8) return launch_km<8, false>(mq, mk, H, n, S, kappa, 1, row_ptr, col, w, nullptr, st);
+    if (kappa <= 16) return launch_km<16, false>(mq, mk, H, n, S, kappa, 1, row_ptr, col, w, nullptr, st);
+    return launch_km<32, false>(mq, mk, H, n, S, kappa, 1, row_ptr, col, w, nullptr, st);
+}
+
+size_t build_graph_grouped_stats_floats(int Hkv, int group, int n)
+{
+    return (size_t)Hkv * group * n * 2 + 4;   // (max, sum) per query head and row, then the failure word
+}
+
+cudaError_t launch_build_graph_grouped(int Hkv, int group, int n, int S, int kappa, const void* Q, const void* K,
+                                       float* stats, int64_t* row_ptr, int32_t* col, float* w, cudaStream_t st)
+{
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K)) & 15) return cudaErrorInvalidValue;
+    if (group != 1 && group != 2 && group != 4) return cudaErrorInvalidValue;
+    const int Hq = Hkv * group;
+    const int bn = (group >= 4) ? 64 : 128;
+    CUtensorMap mq, mk, mkg;
+    if (!make_map(&mq, Q, Hq, n) || !make_map(&mk, K, Hkv, n) || !make_map(&mkg, K, Hkv, n, bn))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(stats + (size_t)Hq * n * 2, 0, 4 * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    // first pass: every query head's row statistics
+    e = launch_km<8, true>(mq, mk, Hq, n, S, kappa, group, row_ptr, col, w, stats, st);
+    if (e != cudaSuccess) return e;
+    // second pass: one graph per KV head, ranked by the summed probabilities
+    if (kappa <= 8) return launch_group_nh<8>(group, mq, mkg, Hkv, n, S, kappa, stats, row_ptr, col, w, st);
+    if (kappa <= 16) return launch_group_nh<16>(group, mq, mkg, Hkv, n, S, kappa, stats, row_ptr, col, w, st);
+    return launch_group_nh<32>(group, mq, mkg, Hkv, n, S, kappa, stats, row_ptr, col, w, st);
 }
 
 }  // namespace ckv
