@@ -236,6 +236,62 @@ def reference_arm(args, rank, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+def prefill_bench(args):
+    """Figure 1 step (1): the prefill top-kappa graph of the 8-head n=16384
+    workload, per head (ckv_build_graph) and per KV head of 4 query heads
+    (ckv_build_graph_grouped); device time per call with CUDA events, and
+    the causal Q K^T flops it implies against the measured bf16 peak."""
+    import torch
+    import long_context_decode_ckv_b200 as ckv
+    from long_context_decode_ckv_b200 import build as ckv_build
+    P = synth.PREFILL
+    Q, K = synth.make_prefill(P)
+    ckv_build.build()
+    dev = torch.device("cuda", 0)
+    q = torch.from_numpy(Q).view(torch.bfloat16).to(dev)
+    k = torch.from_numpy(K).view(torch.bfloat16).to(dev)
+    n, H, S, kap = P.n, P.n_heads, P.n_sinks, P.kappa
+    E = int(np.clip(np.arange(n) - S, 0, kap).sum())
+    causal_flops = 2.0 * 128 * n * (n + 1) / 2 * H          # one Q K^T over the causal triangle, all heads
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    rp = torch.empty((H, n + 1), dtype=torch.int64, device=dev)
+    col = torch.empty((H, E), dtype=torch.int32, device=dev)
+    w = torch.empty((H, E), dtype=torch.float32, device=dev)
+    ms_head = timed(lambda: ckv.ckv_build_graph(H, n, 128, S, kap, ckv.CKV_BF16, q, k, rp, col, w))
+    Hkv, g = H // 4, 4
+    ws = torch.empty(ckv.ckv_build_graph_grouped_workspace(Hkv, g, n), dtype=torch.uint8, device=dev)
+    kk = k[:Hkv].contiguous()
+    ms_group = timed(lambda: ckv.ckv_build_graph_grouped(Hkv, g, n, 128, S, kap, ckv.CKV_BF16, q, kk, ws,
+                                                         rp[:Hkv], col[:Hkv], w[:Hkv]))
+    peak = None
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        peak = float(json.load(open(pp)).get("bf16_tflops", 0)) or None
+    tf_head = causal_flops / (ms_head / 1e3) / 1e12
+    tf_group = 2 * causal_flops / (ms_group / 1e3) / 1e12   # statistics pass + grouped pass
+    print(json.dumps({
+        "metric": "prefill graph ms", "workload": "prefill_8h_n16384_k8_s4_bf16", "steps": args.steps,
+        "warmup": args.warmup,
+        "per_head": {"ms": ms_head, "tflops": tf_head, "frac_of_bf16_peak": tf_head / peak if peak else None},
+        "query_group_4": {"ms": ms_group, "tflops_both_passes": tf_group,
+                          "frac_of_bf16_peak": tf_group / peak if peak else None},
+        "bf16_peak_tflops": peak, "exp2_count": n * (n + 1) / 2 * H,
+    }), flush=True)
+    return 0
+
+
 def recall_sweep(args, budgets):
     """Figure 3 (right): attention-mass recall of the retrieved set versus the
     token budget, on the throughput workload, every 8th of --steps steps."""
@@ -304,6 +360,8 @@ def main():
     ap.add_argument("--recall-sweep", default="",
                     help="comma-separated budgets: print the mean attention-mass recall per budget "
                          "over --steps decode steps instead of timing")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the prefill graph construction (per-head and query-group) instead")
     ap.add_argument("--dense-steps", type=int, default=20,
                     help="dense decode comparator launches timed after the sparse steps (0 = none)")
     args = ap.parse_args()
@@ -314,6 +372,8 @@ def main():
         return reference_arm(args, rank, world)
     if args.recall_sweep:
         return recall_sweep(args, [int(b) for b in args.recall_sweep.split(",")])
+    if args.prefill:
+        return prefill_bench(args)
 
     # host-side generation first (spawned pool, before any CUDA call)
     workers = max(1, min(16, (os.cpu_count() or 1) // max(1, world)))

@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "ckv_internal.cuh"
@@ -35,10 +36,13 @@ namespace {
 
 constexpr int kBM = 128, kBN = 128;
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;                        // the grouped kernel: producer, MMA, 4 epilogue warps
+constexpr int kEpiWarps = 8;                         // per-head kernel: two epilogue warps per TMEM lane quarter
+constexpr int kThreadsH = 64 + 32 * kEpiWarps;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kMaxKM = 32;
 constexpr int kHalfBytes = kBM * 64 * 2;            // one 64-column half of a 128-row tile
 constexpr int kTileBytes = 2 * kHalfBytes;           // 32 KB
-constexpr unsigned kWaitLimit = 1u << 22;
 constexpr float kLog2eOverSqrtD = 0.12751743082459868f;   // log2(e) / sqrt(128)
 
 struct __align__(1024) PrefillSmem {
@@ -51,6 +55,10 @@ struct __align__(1024) PrefillSmem {
     unsigned long long bar_aempty[2];
     uint32_t tmem_base;
     int abort;
+    // the second half's row state, merged into the first half's at the end
+    float xm[kBM][2];
+    float xv[kBM][kMaxKM];
+    int xi[kBM][kMaxKM];   // xv and xi together also stage the epilogue's gated chunks (256 threads x 32 words)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
@@ -74,21 +82,26 @@ __device__ __forceinline__ void mbar_arrive(unsigned long long* b)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 
-// bounded wait for the phase with the given parity to complete
+// bounded wait for the phase with the given parity to complete.  Each poll
+// may suspend the thread for up to kSuspendNs (it wakes as soon as the phase
+// completes), so a waiting role issues few instructions; at most
+// kWaitPolls polls, about a second, before the CTA gives up.
+constexpr unsigned kSuspendNs = 4000;
+constexpr unsigned kWaitPolls = 1u << 18;
 __device__ __forceinline__ bool mbar_wait(unsigned long long* b, unsigned parity, volatile int* abort)
 {
     const uint32_t a = smem_u32(b);
-    for (unsigned it = 0; it < kWaitLimit; ++it) {
+    for (unsigned it = 0; it < kWaitPolls; ++it) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(done)
-            : "r"(a), "r"(parity)
+            : "r"(a), "r"(parity), "r"(kSuspendNs)
             : "memory");
         if (done) return true;
-        if ((it & 1023) == 1023 && *abort) return false;
+        if ((it & 63) == 63 && *abort) return false;
     }
     *abort = 1;
     return false;
@@ -163,6 +176,97 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
+// 32 columns of this warp's TMEM lanes, without waiting (tmem_wait_tie does)
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+// waits for this thread's outstanding tcgen05.ld and ties r to the wait, so
+// that no use of r is scheduled before it
+__device__ __forceinline__ void tmem_wait_tie(uint32_t (&r)[32], bool wait)
+{
+    if (wait) asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                   "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                   "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+// Insert the chunk's candidates (columns j0 + k, k in the bit mask) into the
+// sorted top-KM list.  Candidates are rare after a row's first columns, so
+// the loop over them stays rolled and only one copy of the insertion
+// network is emitted (an unrolled copy per column thrashed the
+// instruction cache).  Ties keep the earlier column ahead.
+template <int KM>
+__device__ __forceinline__ void insert_candidates(unsigned cm, const float (&v)[32], int j0, float (&vals)[KM],
+                                                  int (&idx)[KM])
+{
+#pragma unroll 1
+    while (cm) {
+        const int k = __ffs(cm) - 1;
+        cm &= cm - 1;
+        float a = v[0];
+#pragma unroll
+        for (int kk = 1; kk < 32; ++kk) a = (k == kk) ? v[kk] : a;
+        if (!(a > vals[KM - 1])) continue;      // the list rose past it since the mask was taken
+        const int j = j0 + k;
+#pragma unroll
+        for (int p = KM - 1; p > 0; --p) {
+            const float up = vals[p - 1];
+            const int upi = idx[p - 1];
+            const bool shift = up < a;
+            const bool land = !shift && vals[p] < a;
+            vals[p] = shift ? up : (land ? a : vals[p]);
+            idx[p] = shift ? upi : (land ? j : idx[p]);
+        }
+        if (vals[0] < a) { vals[0] = a; idx[0] = j; }
+    }
+}
+
+// The same with the chunk's values staged in shared memory (column k of
+// this thread at stage[k * stride]): a candidate is one load instead of a
+// select over 32 registers.
+template <int KM>
+__device__ __forceinline__ void insert_staged(unsigned cm, const float* stage, int stride, int j0, float (&vals)[KM],
+                                              int (&idx)[KM])
+{
+#pragma unroll 1
+    while (cm) {
+        const int k = __ffs(cm) - 1;
+        cm &= cm - 1;
+        const float a = stage[k * stride];
+        if (!(a > vals[KM - 1])) continue;      // the list rose past it since the mask was taken
+        const int j = j0 + k;
+#pragma unroll
+        for (int p = KM - 1; p > 0; --p) {
+            const float up = vals[p - 1];
+            const int upi = idx[p - 1];
+            const bool shift = up < a;
+            const bool land = !shift && vals[p] < a;
+            vals[p] = shift ? up : (land ? a : vals[p]);
+            idx[p] = shift ? upi : (land ? j : idx[p]);
+        }
+        if (vals[0] < a) { vals[0] = a; idx[0] = j; }
+    }
+}
+
+// barrier 1 among the per-head kernel's epilogue warps only
+__device__ __forceinline__ void epi_sync()
+{
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x)
 {
     float y;
@@ -181,8 +285,12 @@ __device__ __forceinline__ int64_t row_offset(int64_t i, int S, int kappa)
 // go to stats[h][i][2] instead (the first pass of the query-group graph),
 // and a bounded wait that runs out sets the int word after them.
 // group: query heads per KV head (the K rows of head h are those of h / group).
+static_assert(offsetof(PrefillSmem, xi) == offsetof(PrefillSmem, xv) + sizeof(float) * kBM * kMaxKM &&
+                  2 * kBM * kMaxKM >= kEpiThreads * 32,
+              "the staging area spans xv and xi");
+
 template <int KM, bool STATS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsH, 1)
 k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int H, int n,
                int S, int kappa, int group, int64_t* __restrict__ row_ptr, int32_t* __restrict__ col,
                float* __restrict__ w, float* __restrict__ stats)
@@ -201,7 +309,7 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
         for (int s = 0; s < kStages; ++s) { mbar_init(&sm.bar_kfull[s], 1); mbar_init(&sm.bar_kempty[s], 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(&sm.bar_afull[b], 1); mbar_init(&sm.bar_aempty[b], 4); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&sm.bar_afull[b], 1); mbar_init(&sm.bar_aempty[b], kEpiWarps); }
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -267,7 +375,10 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
     } else {
         // ---------------------------------------------------- epilogue
+        // two warps per TMEM lane quarter: thread = one row, half = which
+        // 32-column chunks of every tile it takes (half, half + 2)
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
+        const int half = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
         const int i = i0 + r;
         const bool row_ok = i < n;
@@ -276,74 +387,134 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         int idx[KM];
 #pragma unroll
         for (int k = 0; k < KM; ++k) { vals[k] = -INFINITY; idx[k] = -1; }
+        // a gated chunk's values, column k of epilogue thread e at stage[k * kEpiThreads + e]; the
+        // merge scratch is free until the loop ends
+        float* stage = &sm.xv[0][0] + (threadIdx.x - 64);
+        auto chunk = [&](const uint32_t (&rv)[32], int j0, bool diag) {
+            // causal mask: only the diagonal tile reaches past i
+            float v[32];
+            // four independent chains for the max and the sum (latency, not issue, bounds a single chain)
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (diag) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    v[k] = (j0 + k > i) ? -INFINITY : __uint_as_float(rv[k]);
+                    mq[k & 3] = fmaxf(mq[k & 3], v[k]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    v[k] = __uint_as_float(rv[k]);
+                    mq[k & 3] = fmaxf(mq[k & 3], v[k]);
+                }
+            }
+            const float mc = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            if (!row_ok || mc == -INFINITY) return;   // no column of this chunk is at or before i
+            const float mcs = mc * kLog2eOverSqrtD;
+            if (mcs > m2) {
+                l *= ex2(m2 - mcs);
+                m2 = mcs;
+            }
+            float pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 32; ++k) pq[k & 3] += ex2(fmaf(v[k], kLog2eOverSqrtD, -m2));
+            l += (pq[0] + pq[1]) + (pq[2] + pq[3]);
+            if constexpr (!STATS) {
+                // top-KM candidates j in [S, i-1], ranked by the raw score
+                const float thr = vals[KM - 1];
+                if (mc > thr) {   // some column may enter the list
+                    unsigned cm = 0u;
+                    if (diag || j0 < S) {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            cm |= (v[k] > thr && j0 + k >= S && j0 + k < i) ? (1u << k) : 0u;
+                    } else {   // every column is in [S, i-1]
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) cm |= (v[k] > thr) ? (1u << k) : 0u;
+                    }
+                    if (__popc(cm) > 1) {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) stage[k * kEpiThreads] = v[k];
+                        insert_staged<KM>(cm, stage, kEpiThreads, j0, vals, idx);
+                    } else {
+                        insert_candidates<KM>(cm, v, j0, vals, idx);
+                    }
+                }
+            }
+        };
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
             if (!mbar_wait(&sm.bar_afull[b], (t >> 1) & 1, abort)) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < kBN / 32; ++ch) {
-                float v[32];
-                __syncwarp();   // tcgen05.ld is warp-collective
-                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + b * kBN + ch * 32, v);
-                const int j0 = t * kBN + ch * 32;
-                // causal mask (only the diagonal tile reaches past i)
-                float mc = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    if (j0 + k > i) v[k] = -INFINITY;
-                    mc = fmaxf(mc, v[k]);
-                }
-                if (!row_ok) continue;
-                const float mcs = mc * kLog2eOverSqrtD;
-                if (mcs > m2) {
-                    l *= ex2(m2 - mcs);
-                    m2 = mcs;
-                }
-                float ps = 0.f;
-#pragma unroll
-                for (int k = 0; k < 32; ++k) ps += ex2(fmaf(v[k], kLog2eOverSqrtD, -m2));
-                l += ps;
-                if constexpr (!STATS) {
-                    // top-KM candidates j in [S, i-1], ranked by the raw score
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int j = j0 + k;
-                        const float a = v[k];
-                        if (a > vals[KM - 1] && j >= S && j < i) {
-#pragma unroll
-                            for (int p = KM - 1; p > 0; --p) {
-                                const float up = vals[p - 1];
-                                const int upi = idx[p - 1];
-                                const bool shift = up < a;
-                                const bool land = !shift && vals[p] < a;
-                                vals[p] = shift ? up : (land ? a : vals[p]);
-                                idx[p] = shift ? upi : (land ? j : idx[p]);
-                            }
-                            if (vals[0] < a) { vals[0] = a; idx[0] = j; }
-                        }
-                    }
-                }
-            }
+            uint32_t ra[32], rb[32];
+            __syncwarp();   // tcgen05.ld is warp-collective
+            tmem_ld32_async(lane_addr + b * kBN + half * 32, ra);
+            tmem_ld32_async(lane_addr + b * kBN + (half + 2) * 32, rb);
+            tmem_wait_tie(ra, true);
+            tmem_wait_tie(rb, false);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.bar_aempty[b]);
+            if (lane == 0) mbar_arrive(&sm.bar_aempty[b]);   // the accumulator is read: the MMA may refill it
+            const bool diag = t == ntiles - 1;      // the tile holding the block's diagonal
+            chunk(ra, t * kBN + half * 32, diag);
+            chunk(rb, t * kBN + (half + 2) * 32, diag);
         }
-        if (STATS && row_ok && !*abort) {
-            stats[((int64_t)h * n + i) * 2] = m2;
-            stats[((int64_t)h * n + i) * 2 + 1] = l;
-        } else if (row_ok && !*abort) {
-            const int64_t base = (int64_t)h * E + row_offset(i, S, kappa);
-            const int deg = (int)min((int64_t)kappa, max((int64_t)0, (int64_t)i - S));
-            const float inv_l = 1.f / l;
+        // the second half hands its row state to the first half
+        epi_sync();
+        if (half == 1) {
+            sm.xm[r][0] = m2;
+            sm.xm[r][1] = l;
+            if constexpr (!STATS) {
 #pragma unroll
-            for (int k = 0; k < KM; ++k) {
-                if (k < deg) {
-                    col[base + k] = idx[k];
-                    w[base + k] = ex2(fmaf(vals[k], kLog2eOverSqrtD, -m2)) * inv_l;
+                for (int k = 0; k < KM; ++k) { sm.xv[r][k] = vals[k]; sm.xi[r][k] = idx[k]; }
+            }
+        }
+        epi_sync();
+        if (half == 0) {
+            const float mo = sm.xm[r][0], lo = sm.xm[r][1];
+            const float mn = fmaxf(m2, mo);
+            if (mn != -INFINITY) {
+                l = (m2 == -INFINITY ? 0.f : l * ex2(m2 - mn)) + (mo == -INFINITY ? 0.f : lo * ex2(mo - mn));
+                m2 = mn;
+            }
+            if constexpr (!STATS) {
+                // insert the second half's list, ranked by (score desc, j asc)
+                auto before = [](float a, int ja, float b, int jb) { return a > b || (a == b && ja < jb); };
+#pragma unroll 1
+                for (int k = 0; k < KM; ++k) {
+                    const float a = sm.xv[r][k];
+                    const int j = sm.xi[r][k];
+                    if (j < 0 || !before(a, j, vals[KM - 1], idx[KM - 1])) break;   // the rest rank lower
+#pragma unroll
+                    for (int p = KM - 1; p > 0; --p) {
+                        const float up = vals[p - 1];
+                        const int upi = idx[p - 1];
+                        const bool shift = before(a, j, up, upi);
+                        const bool land = !shift && before(a, j, vals[p], idx[p]);
+                        vals[p] = shift ? up : (land ? a : vals[p]);
+                        idx[p] = shift ? upi : (land ? j : idx[p]);
+                    }
+                    if (before(a, j, vals[0], idx[0])) { vals[0] = a; idx[0] = j; }
                 }
             }
-            row_ptr[(int64_t)h * (n + 1) + i] = row_offset(i, S, kappa);
-            if (i == n - 1) row_ptr[(int64_t)h * (n + 1) + n] = E;
+            if (STATS && row_ok && !*abort) {
+                stats[((int64_t)h * n + i) * 2] = m2;
+                stats[((int64_t)h * n + i) * 2 + 1] = l;
+            } else if (row_ok && !*abort) {
+                const int64_t base = (int64_t)h * E + row_offset(i, S, kappa);
+                const int deg = (int)min((int64_t)kappa, max((int64_t)0, (int64_t)i - S));
+                const float inv_l = 1.f / l;
+#pragma unroll
+                for (int k = 0; k < KM; ++k) {
+                    if (k < deg) {
+                        col[base + k] = idx[k];
+                        w[base + k] = ex2(fmaf(vals[k], kLog2eOverSqrtD, -m2)) * inv_l;
+                    }
+                }
+                row_ptr[(int64_t)h * (n + 1) + i] = row_offset(i, S, kappa);
+                if (i == n - 1) row_ptr[(int64_t)h * (n + 1) + n] = E;
+            }
         }
     }
     __syncthreads();
@@ -515,22 +686,17 @@ k_prefill_group(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (!row_ok) continue;
                 const int j0 = t * BN + cc * 32;
                 // top-KM candidates j in [S, i-1] by the summed probability
+                const float thr = vals[KM - 1];
+                float mq[4] = {ws[0], ws[1], ws[2], ws[3]};
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int j = j0 + k;
-                    const float a = ws[k];
-                    if (a > vals[KM - 1] && j >= S && j < i) {
+                for (int k = 4; k < 32; ++k) mq[k & 3] = fmaxf(mq[k & 3], ws[k]);
+                const float mc = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+                if (mc > thr) {   // some column may enter the list
+                    unsigned cm = 0u;
 #pragma unroll
-                        for (int p = KM - 1; p > 0; --p) {
-                            const float up = vals[p - 1];
-                            const int upi = idx[p - 1];
-                            const bool shift = up < a;
-                            const bool land = !shift && vals[p] < a;
-                            vals[p] = shift ? up : (land ? a : vals[p]);
-                            idx[p] = shift ? upi : (land ? j : idx[p]);
-                        }
-                        if (vals[0] < a) { vals[0] = a; idx[0] = j; }
-                    }
+                    for (int k = 0; k < 32; ++k)
+                        cm |= (ws[k] > thr && j0 + k >= S && j0 + k < i) ? (1u << k) : 0u;
+                    insert_candidates<KM>(cm, ws, j0, vals, idx);
                 }
             }
             tc_fence_before();
@@ -595,7 +761,7 @@ cudaError_t launch_km(const CUtensorMap& mq, const CUtensorMap& mk, int H, int n
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int nqb = (n + kBM - 1) / kBM;
-    kern<<<H * nqb, kThreads, smem, st>>>(mq, mk, H, n, S, kappa, group, row_ptr, col, w, stats);
+    kern<<<H * nqb, kThreadsH, smem, st>>>(mq, mk, H, n, S, kappa, group, row_ptr, col, w, stats);
     return cudaGetLastError();
 }
 
