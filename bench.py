@@ -65,33 +65,44 @@ def kernel_bytes(cfg, T):
     }
 
 
-# DRAM bytes read + written per launch from one ncu capture (profiles/,
-# k_score_k_select_k_attend_qwen3_8b_n131072_full.md), valid only for the
-# kernel sources they were taken on (bench.source_hash of csrc/)
-PROFILED_TRAFFIC = {"source_sha256": "872a0dc9f517f7db", "k_score": 139.358208e6, "k_attend": 69.187584e6,
-                    "k_dense_stats": 1077.576416e6, "k_dense_attention": 2151.696384e6}
+# DRAM bytes read + written per launch from one ncu capture (profiles/), each
+# valid only while the sources that define that kernel are the ones the
+# capture was taken on (source_hash over KERNEL_SOURCES of the kernel)
+KERNEL_SOURCES = {
+    "k_score": ("k_decode.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
+    "k_attend": ("k_decode.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
+    "k_dense_stats": ("k_dense.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
+    "k_dense_attention": ("k_dense.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
+}
+PROFILED_TRAFFIC = {
+    "k_score": ("f92868379799ae92", 139.236864e6),
+    "k_attend": ("f92868379799ae92", 68.953856e6),
+    "k_dense_stats": ("b8df1d15a63cd101", 1079.294656e6),
+}
 
 
-def source_hash():
-    """First 16 hex digits of the SHA-256 over every CUDA source of the library
-    (sorted .cu / .cuh of csrc/): the build a capture was taken on."""
-    import glob
+def source_hash(files):
+    """First 16 hex digits of the SHA-256 over the given CUDA sources of the
+    library (in order, each with its name)."""
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "long_context_decode_ckv_b200", "csrc", "*.cu*"))):
-        h.update(os.path.basename(f).encode())
-        h.update(open(f, "rb").read())
+    for f in files:
+        h.update(f.encode())
+        h.update(open(os.path.join(ROOT, "long_context_decode_ckv_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel):
-    """DRAM bytes per launch from the ncu capture, only while the sources
-    are the ones it was taken on."""
+    """DRAM bytes per launch from the ncu capture, only while the kernel's
+    sources are the ones it was taken on."""
+    if kernel not in PROFILED_TRAFFIC:
+        return None
     try:
-        h = source_hash()
+        h = source_hash(KERNEL_SOURCES[kernel])
     except OSError:
         return None
-    return PROFILED_TRAFFIC.get(kernel) if h == PROFILED_TRAFFIC["source_sha256"] else None
+    sha, traffic = PROFILED_TRAFFIC[kernel]
+    return traffic if h == sha else None
 
 
 def measured_peaks():
