@@ -26,6 +26,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ckv_oracle.c")
+_SRC2 = os.path.join(_HERE, "leiden_oracle.c")
 _HDR = os.path.join(_HERE, "ckv_oracle.h")
 _LIB = os.path.join(_HERE, "libckv_oracle.so")
 
@@ -35,12 +36,12 @@ KMAX = 64
 
 def build(force: bool = False) -> str:
     """Compile the C oracle into oracle/libckv_oracle.so (gcc, -O2, no FMA)."""
-    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC2), os.path.getmtime(_HDR))
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call([
             "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
-            "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm",
+            "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, _SRC2, "-lm",
         ])
         os.replace(tmp, _LIB)
     return _LIB
@@ -93,6 +94,10 @@ def lib() -> ctypes.CDLL:
         L.ckvo_row_ptr.restype = i64
         L.ckvo_row_ptr.argtypes = [i64, i32, i32]
         L.ckvo_prefill_rows_grouped.argtypes = [i32, i32, i32, i32, i32, P, P, i32, P, i32, P, P, P, P]
+        L.ckvo_leiden.restype = i32
+        L.ckvo_leiden.argtypes = [i32, P, P, P, ctypes.c_double, i32, P]
+        L.ckvo_modularity.restype = ctypes.c_double
+        L.ckvo_modularity.argtypes = [i32, P, P, P, P, ctypes.c_double]
         L.ckvo_dense_stats.argtypes = [i32, i32, P, i32, P, i32, i32, P, P]
         L.ckvo_prefill_rows.argtypes = [i32, i32, i32, i32, P, P, i32, P, i32, P, P, P, P]
         _lib = L
@@ -199,6 +204,25 @@ def prefill_rows_grouped(Q: np.ndarray, K: np.ndarray, rows, n_sinks: int, kappa
     lib().ckvo_prefill_rows_grouped(n, D, n_sinks, kappa, nh, _p(Q), _p(K), _dtype_code(Q),
                                     _p(rows), R, _p(col), _p(w), _p(deg), _p(gap))
     return col, w, deg, gap
+
+
+def leiden(row_ptr, col, w, n: int, gamma: float = 1.0, max_levels: int = 64):
+    """Leiden partition (deterministic variant of leiden_oracle.c) of the
+    directed top-kappa CSR read as an undirected graph: (labels [n], C)."""
+    row_ptr = np.ascontiguousarray(row_ptr, np.int64)
+    col = np.ascontiguousarray(col, np.int32)
+    w = np.ascontiguousarray(w, np.float32)
+    labels = np.empty(max(n, 1), np.int32)
+    C = lib().ckvo_leiden(n, _p(row_ptr), _p(col), _p(w), float(gamma), max_levels, _p(labels))
+    return labels[:n].copy(), C
+
+
+def modularity(row_ptr, col, w, labels, gamma: float = 1.0) -> float:
+    row_ptr = np.ascontiguousarray(row_ptr, np.int64)
+    col = np.ascontiguousarray(col, np.int32)
+    w = np.ascontiguousarray(w, np.float32)
+    labels = np.ascontiguousarray(labels, np.int32)
+    return lib().ckvo_modularity(len(row_ptr) - 1, _p(row_ptr), _p(col), _p(w), _p(labels), float(gamma))
 
 
 # ---------------------------------------------------------------- state

@@ -135,6 +135,18 @@ void ckvo_prefill_rows_grouped(int n, int D, int n_sinks, int kappa, int nh, con
                                int dtype, const int32_t* rows, int n_rows,
                                int32_t* col, float* w, int32_t* deg, float* gap);
 
+/* Leiden partition of a top-kappa token graph (leiden_oracle.c): the
+ * directed CSR (row_ptr [n+1], col, w) read as an undirected weighted graph;
+ * modularity quality with resolution gamma; the deterministic variant
+ * described in leiden_oracle.c.  labels [n] get community ids 0..C-1 by
+ * first appearance; returns C. */
+int ckvo_leiden(int n, const int64_t* row_ptr, const int32_t* col, const float* w, double gamma, int max_levels,
+                int32_t* labels);
+/* Modularity with resolution gamma of a labelling of the same graph:
+ * (in - gamma sum_c K_c^2 / (4m)) / m. */
+double ckvo_modularity(int n, const int64_t* row_ptr, const int32_t* col, const float* w, const int32_t* labels,
+                       double gamma);
+
 #ifdef __cplusplus
 }
 #endif
