@@ -303,6 +303,48 @@ def prefill_bench(args):
     return 0
 
 
+def leiden_bench(args):
+    """Figure 1 step (2) and Figure 2: the prefill graph (GPU, ckv_build_graph)
+    of the 8-head workload at growing n, partitioned by the host Leiden
+    (ckv_leiden, gamma 1); community count, mean size, modularity (GPU,
+    ckv_modularity) and the host time per graph."""
+    import torch
+    import long_context_decode_ckv_b200 as ckv
+    from long_context_decode_ckv_b200 import build as ckv_build
+    P = synth.PREFILL
+    ckv_build.build()
+    dev = torch.device("cuda", 0)
+    rows = []
+    for n in (1024, 2048, 4096, 8192, 16384):
+        Q, K = synth.make_prefill(P, n=n)
+        q = torch.from_numpy(Q).view(torch.bfloat16).to(dev)
+        k = torch.from_numpy(K).view(torch.bfloat16).to(dev)
+        H, S, kap = P.n_heads, P.n_sinks, P.kappa
+        E = int(np.clip(np.arange(n) - S, 0, kap).sum())
+        rp = torch.empty((H, n + 1), dtype=torch.int64, device=dev)
+        col = torch.empty((H, E), dtype=torch.int32, device=dev)
+        w = torch.empty((H, E), dtype=torch.float32, device=dev)
+        ckv.ckv_build_graph(H, n, 128, S, kap, ckv.CKV_BF16, q, k, rp, col, w)
+        torch.cuda.synchronize(dev)
+        counts, qs, secs = [], [], []
+        for h in range(H):
+            rph, colh, wh = rp[h].cpu().numpy(), col[h].cpu().numpy(), w[h].cpu().numpy()
+            labels = np.empty(n, np.int32)
+            t0 = time.perf_counter()
+            C = ckv.ckv_leiden(n, rph, colh, wh, 1.0, labels)
+            secs.append(time.perf_counter() - t0)
+            ws = torch.empty(ckv.ckv_modularity_workspace(C), dtype=torch.uint8, device=dev)
+            qs.append(ckv.ckv_modularity(n, rp[h], col[h], w[h], torch.from_numpy(labels).to(dev), C, 1.0, ws))
+            counts.append(C)
+        rows.append({"n": n, "communities_mean": float(np.mean(counts)),
+                     "communities_over_sqrt_n": float(np.mean(counts) / np.sqrt(n)),
+                     "mean_size": float(n / np.mean(counts)), "modularity_mean": float(np.mean(qs)),
+                     "leiden_host_ms_per_graph": 1e3 * float(np.mean(secs))})
+    print(json.dumps({"leiden_vs_n": rows, "workload": "prefill_8h_k8_s4_bf16 (per-head graphs, gamma 1)",
+                      "data": "synthetic clustered keys (2048 clusters)"}), flush=True)
+    return 0
+
+
 def recall_sweep(args, budgets):
     """Figure 3 (right): attention-mass recall of the retrieved set versus the
     token budget, on the throughput workload, every 8th of --steps steps."""
@@ -371,6 +413,9 @@ def main():
     ap.add_argument("--recall-sweep", default="",
                     help="comma-separated budgets: print the mean attention-mass recall per budget "
                          "over --steps decode steps instead of timing")
+    ap.add_argument("--leiden", action="store_true",
+                    help="partition prefill graphs of growing n with the host Leiden and report the community "
+                         "count and modularity instead")
     ap.add_argument("--prefill", action="store_true",
                     help="time the prefill graph construction (per-head and query-group) instead")
     ap.add_argument("--dense-steps", type=int, default=20,
@@ -385,6 +430,8 @@ def main():
         return recall_sweep(args, [int(b) for b in args.recall_sweep.split(",")])
     if args.prefill:
         return prefill_bench(args)
+    if args.leiden:
+        return leiden_bench(args)
 
     # host-side generation first (spawned pool, before any CUDA call)
     workers = max(1, min(16, (os.cpu_count() or 1) // max(1, world)))

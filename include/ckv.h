@@ -131,6 +131,42 @@ ckv_status ckv_build_graph_grouped(int n_kv_heads, int group, int n, int head_di
                                    ckv_dtype dtype, const void* Q, const void* K, void* workspace,
                                    int64_t* row_ptr, int32_t* col, float* w, void* stream);
 
+/* Leiden partition of a prefill token graph -- Figure 1, step (2) ("the
+ * token graph is partitioned with Leiden"), run on the host as the pages
+ * do.  Input: one graph of ckv_build_graph's output copied to host memory
+ * (row_ptr_host [n+1], col_host and w_host [row_ptr_host[n]]), read as an
+ * undirected weighted graph: an edge i -> j of weight w adds w between i
+ * and j.  Quality: modularity with resolution gamma > 0.  The algorithm is
+ * Leiden's local moving, refinement and aggregation, repeated from its own
+ * result until it no longer changes, with every choice deterministic:
+ *   - nodes go through the queue and the refinement in ascending id;
+ *   - a node moves to the neighbouring community of largest gain, ties to
+ *     staying, then to the lower id;
+ *   - the refinement takes the largest positive gain (zero randomness);
+ *   - all sums are taken in a fixed order.
+ * Output: labels_host [n], community ids 0..C-1 by first appearance, and
+ * *n_communities = C; the labels feed ckv_init_communities (sinks' labels
+ * are ignored there).  Synchronous, host only.
+ * Errors: CKV_ERR_INVALID_ARG (n < 1, gamma <= 0, row_ptr not monotone,
+ * a column outside [0, n), a negative or NaN weight), CKV_ERR_OOM. */
+ckv_status ckv_leiden(int n, const int64_t* row_ptr_host, const int32_t* col_host, const float* w_host,
+                      double gamma, int32_t* labels_host, int* n_communities);
+
+/* Modularity of a partition of that graph -- Figure 3 (left) tracks it over
+ * generation.  Q = (in - gamma * sum_c K_c^2 / (4m)) / m over the graph read
+ * as in ckv_leiden: m is the total edge weight, in the weight of edges
+ * whose ends share a label, K_c the summed degree of community c.
+ * row_ptr, col, w, labels [n] (each in [0, n_communities)) are device
+ * memory; workspace: ckv_modularity_workspace(n_communities) bytes of
+ * device scratch, 8-byte aligned.  Computed on the device in double; the
+ * call synchronises `stream` and writes Q to *q_host.
+ * Errors: CKV_ERR_INVALID_ARG (including a label or column out of range,
+ * found on the device), CKV_ERR_CUDA. */
+size_t ckv_modularity_workspace(int n_communities);
+ckv_status ckv_modularity(int n, const int64_t* row_ptr, const int32_t* col, const float* w,
+                          const int32_t* labels, int n_communities, double gamma, void* workspace,
+                          double* q_host, void* stream);
+
 /* Initial partition -- Figure 1, step (2): community c of graph g holds the
  * positions j in [S, n) with labels[g][j] == c (ascending); its centroid is
  * the mean of those keys (float, summed in double).  labels: int32

@@ -94,6 +94,12 @@ def lib() -> ctypes.CDLL:
     L.ckv_build_graph_grouped_workspace.argtypes = [I, I, I]
     L.ckv_build_graph_grouped.restype = st
     L.ckv_build_graph_grouped.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P]
+    L.ckv_leiden.restype = st
+    L.ckv_leiden.argtypes = [I, P, P, P, ctypes.c_double, P, ctypes.POINTER(ctypes.c_int)]
+    L.ckv_modularity_workspace.restype = sz
+    L.ckv_modularity_workspace.argtypes = [I]
+    L.ckv_modularity.restype = st
+    L.ckv_modularity.argtypes = [I, P, P, P, P, I, ctypes.c_double, P, ctypes.POINTER(ctypes.c_double), P]
     L.ckv_step_recall.restype = st
     L.ckv_step_recall.argtypes = [P, P, P, I, P, P]
     L.ckv_dense_decode.restype = st
@@ -168,6 +174,25 @@ def ckv_build_graph_grouped(n_kv_heads, group, n, head_dim, n_sinks, kappa, dtyp
     _check("ckv_build_graph_grouped", lib().ckv_build_graph_grouped(
         n_kv_heads, group, n, head_dim, n_sinks, kappa, dtype, _ptr(Q), _ptr(K), _ptr(workspace), _ptr(row_ptr),
         _ptr(col), _ptr(w), _stream(stream)))
+
+
+def ckv_leiden(n, row_ptr_host, col_host, w_host, gamma, labels_host) -> int:
+    """Leiden partition on the host (numpy arrays); returns the community count."""
+    c = ctypes.c_int(0)
+    _check("ckv_leiden", lib().ckv_leiden(n, _ptr(row_ptr_host), _ptr(col_host), _ptr(w_host), float(gamma),
+                                          _ptr(labels_host), ctypes.byref(c)))
+    return c.value
+
+
+def ckv_modularity_workspace(n_communities) -> int:
+    return lib().ckv_modularity_workspace(n_communities)
+
+
+def ckv_modularity(n, row_ptr, col, w, labels, n_communities, gamma, workspace, stream=None) -> float:
+    q = ctypes.c_double(0.0)
+    _check("ckv_modularity", lib().ckv_modularity(n, _ptr(row_ptr), _ptr(col), _ptr(w), _ptr(labels), n_communities,
+                                                  float(gamma), _ptr(workspace), ctypes.byref(q), _stream(stream)))
+    return q.value
 
 
 def ckv_init_communities(ctx, labels, labels_on_device, n_communities, K, n, stream=None):

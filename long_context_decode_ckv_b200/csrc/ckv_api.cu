@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "ckv_internal.cuh"
+#include "leiden.h"
 
 #define CKV_API extern "C" __attribute__((visibility("default")))
 
@@ -740,6 +741,51 @@ CKV_API ckv_status ckv_build_graph(int n_heads, int n, int head_dim, int n_sinks
     if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return CKV_ERR_INVALID_ARG;
     CKV_CUDA(cudaSetDevice(a.device));
     CKV_CUDA(ckv::launch_build_graph(n_heads, n, n_sinks, kappa, Q, K, row_ptr, col, w, (cudaStream_t)stream));
+    return CKV_OK;
+}
+
+CKV_API ckv_status ckv_leiden(int n, const int64_t* row_ptr_host, const int32_t* col_host, const float* w_host,
+                              double gamma, int32_t* labels_host, int* n_communities)
+{
+    if (n < 1 || !row_ptr_host || !labels_host || !n_communities || !(gamma > 0.0)) return CKV_ERR_INVALID_ARG;
+    if (row_ptr_host[0] != 0) return CKV_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
+        if (row_ptr_host[i + 1] < row_ptr_host[i]) return CKV_ERR_INVALID_ARG;
+    const int64_t E = row_ptr_host[n];
+    if (E > 0 && (!col_host || !w_host)) return CKV_ERR_INVALID_ARG;
+    for (int64_t e = 0; e < E; ++e)
+        if (col_host[e] < 0 || col_host[e] >= n || !(w_host[e] >= 0.0f)) return CKV_ERR_INVALID_ARG;
+    try {
+        *n_communities = ckv::leiden_partition(n, row_ptr_host, col_host, w_host, gamma, 64, labels_host);
+    } catch (...) {
+        return CKV_ERR_OOM;
+    }
+    return CKV_OK;
+}
+
+CKV_API size_t ckv_modularity_workspace(int n_communities)
+{
+    return n_communities < 1 ? 0 : ckv::modularity_scratch_doubles(n_communities) * sizeof(double) + sizeof(double);
+}
+
+CKV_API ckv_status ckv_modularity(int n, const int64_t* row_ptr, const int32_t* col, const float* w,
+                                  const int32_t* labels, int n_communities, double gamma, void* workspace,
+                                  double* q_host, void* stream)
+{
+    if (n < 1 || n_communities < 1 || !row_ptr || !labels || !workspace || !q_host || !(gamma > 0.0))
+        return CKV_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 7) return CKV_ERR_INVALID_ARG;
+    cudaPointerAttributes a;
+    CKV_CUDA(cudaPointerGetAttributes(&a, row_ptr));
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return CKV_ERR_INVALID_ARG;
+    CKV_CUDA(cudaSetDevice(a.device));
+    double* scratch = static_cast<double*>(workspace);
+    double* q_dev = scratch + ckv::modularity_scratch_doubles(n_communities);
+    cudaStream_t st = (cudaStream_t)stream;
+    CKV_CUDA(ckv::launch_modularity(n, row_ptr, col, w, labels, n_communities, gamma, scratch, q_dev, st));
+    CKV_CUDA(cudaMemcpyAsync(q_host, q_dev, sizeof(double), cudaMemcpyDeviceToHost, st));
+    CKV_CUDA(cudaStreamSynchronize(st));
+    if (*q_host != *q_host) return CKV_ERR_INVALID_ARG;   // a label or column out of range
     return CKV_OK;
 }
 
