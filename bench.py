@@ -345,6 +345,98 @@ def leiden_bench(args):
     return 0
 
 
+def refresh_bench(args):
+    """Tables 8-9 and Figure 3 (left), mechanics: two contexts decode the same
+    steps from the same Leiden partition of the prefill graph; one updates
+    incrementally only, the other also refreshes (ckv_refresh) every R steps.
+    Every R/2 steps both report the modularity of their partition on the
+    token graph (ckv_graph_modularity).  Workload: batch 1, 8 query heads
+    over 2 KV heads, per-head graphs, n0 = 8192, budget 1024; the prefill
+    graph is the keys over themselves (the synthetic workload has no
+    prefill queries)."""
+    import torch
+    import long_context_decode_ckv_b200 as ckv
+    from long_context_decode_ckv_b200 import build as ckv_build
+    R = args.refresh
+    steps = min(args.steps, 4 * R) if args.steps else 4 * R
+    cfg = synth.scaled(synth.LLAMA, batch=1, n_q_heads=8, n_kv_heads=2, n0=8192, n_clusters=512, steps=steps,
+                       budget=1024)
+    wl = synth.make_workload(cfg, workers=max(1, min(16, os.cpu_count() or 1)))
+    ckv_build.build()
+    dev = torch.device("cuda", 0)
+
+    def upload(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)
+
+    K, V, q = upload(wl.K), upload(wl.V), upload(wl.q)
+    S, kap, n0, G = cfg.n_sinks, cfg.kappa, cfg.n0, cfg.n_graphs
+    E = int(np.clip(np.arange(n0) - S, 0, kap).sum())
+    graphs, labels = [], np.empty((G, n0), np.int32)
+    t0 = time.perf_counter()
+    for kvh in range(cfg.n_kv_heads):
+        kk = K[0, kvh, :n0][None].contiguous()
+        rp = torch.empty((1, n0 + 1), dtype=torch.int64, device=dev)
+        col = torch.empty((1, E), dtype=torch.int32, device=dev)
+        w = torch.empty((1, E), dtype=torch.float32, device=dev)
+        ckv.ckv_build_graph(1, n0, 128, S, kap, ckv.CKV_BF16, kk, kk, rp, col, w)
+        graphs.append((rp[0].cpu().numpy(), col[0].cpu().numpy(), w[0].cpu().numpy()))
+    lab_kv = []
+    for rp, col, w in graphs:
+        lab = np.empty(n0, np.int32)
+        ckv.ckv_leiden(n0, rp, col, w, 1.0, lab)
+        lab_kv.append(lab)
+    init_s = time.perf_counter() - t0
+    nc0 = 0
+    for g in range(G):
+        labels[g] = lab_kv[cfg.graph_heads(g)[1]]
+        nc0 = max(nc0, int(labels[g].max()) + 1)
+    Nc = max(4 * nc0, 256)
+    c = ckv.ckv_config()
+    c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim = 1, cfg.n_q_heads, cfg.n_kv_heads, 128
+    c.n_max, c.max_communities, c.n_sinks = cfg.n_max, Nc, S
+    c.kappa, c.budget, c.slack = kap, cfg.budget, 16
+    c.kv_dtype, c.mode, c.device, c.pool_capacity = ckv.CKV_BF16, ckv.CKV_PER_HEAD, 0, 0
+    rp_all = np.stack([graphs[cfg.graph_heads(g)[1]][0] for g in range(G)])
+    col_all = np.stack([graphs[cfg.graph_heads(g)[1]][1] for g in range(G)])
+    w_all = np.stack([graphs[cfg.graph_heads(g)[1]][2] for g in range(G)])
+    arms = {}
+    for name in ("incremental", "refresh"):
+        ctx = ckv.ckv_create(c)
+        ckv.ckv_init_communities(ctx, labels, 0, nc0, K, n0)
+        ckv.ckv_set_token_graph(ctx, rp_all, col_all, w_all, n0)
+        arms[name] = ctx
+    out = torch.empty((1, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
+    qv = np.zeros(G)
+    traj = {"incremental": [], "refresh": []}
+    refresh_ms, counts = [], []
+    cnt = np.zeros(G, np.int32)
+    for i in range(steps + 1):
+        if i % max(1, R // 2) == 0:
+            for name, ctx in arms.items():
+                ckv.ckv_graph_modularity(ctx, 1.0, qv)
+                traj[name].append({"generated": i, "modularity_mean": float(qv.mean()),
+                                   "modularity_min": float(qv.min())})
+        if i == steps:
+            break
+        if i and i % R == 0:
+            t1 = time.perf_counter()
+            ckv.ckv_refresh(arms["refresh"], K, 1.0, cnt)
+            refresh_ms.append(1e3 * (time.perf_counter() - t1))
+            counts.append(float(cnt.mean()))
+        n = n0 + i + 1
+        for ctx in arms.values():
+            ckv.ckv_decode_step(ctx, q[i], K, V, n, out)
+            ckv.ckv_assign_update(ctx, K, n)
+    for ctx in arms.values():
+        assert ckv.ckv_last_error(ctx) == ckv.CKV_OK
+        ckv.ckv_destroy(ctx)
+    print(json.dumps({"refresh_period": R, "steps": steps, "n0": n0, "graphs": G,
+                      "initial_communities": nc0, "prefill_graph_and_leiden_s": init_s,
+                      "modularity": traj, "refresh_ms": refresh_ms, "communities_after_refresh": counts,
+                      "data": "synthetic clustered keys; prefill graph = keys over keys"}), flush=True)
+    return 0
+
+
 def recall_sweep(args, budgets):
     """Figure 3 (right): attention-mass recall of the retrieved set versus the
     token budget, on the throughput workload, every 8th of --steps steps."""
@@ -413,6 +505,9 @@ def main():
     ap.add_argument("--recall-sweep", default="",
                     help="comma-separated budgets: print the mean attention-mass recall per budget "
                          "over --steps decode steps instead of timing")
+    ap.add_argument("--refresh", type=int, default=0,
+                    help="refresh period R: decode with and without a refresh every R steps and report the "
+                         "modularity over generation instead (Tables 8-9, Figure 3 left)")
     ap.add_argument("--leiden", action="store_true",
                     help="partition prefill graphs of growing n with the host Leiden and report the community "
                          "count and modularity instead")
@@ -432,6 +527,8 @@ def main():
         return prefill_bench(args)
     if args.leiden:
         return leiden_bench(args)
+    if args.refresh:
+        return refresh_bench(args)
 
     # host-side generation first (spawned pool, before any CUDA call)
     workers = max(1, min(16, (os.cpu_count() or 1) // max(1, world)))

@@ -167,6 +167,41 @@ ckv_status ckv_modularity(int n, const int64_t* row_ptr, const int32_t* col, con
                           const int32_t* labels, int n_communities, double gamma, void* workspace,
                           double* q_host, void* stream);
 
+/* Token graph of the context, for refresh and modularity.  Registers each
+ * graph's token graph over positions [0, n) on the host (copied): the
+ * prefill graph in the layout of ckv_build_graph, row_ptr_host [G][n+1]
+ * (each starting at 0) and col_host, w_host [G][E] with E = row_ptr_host[n]
+ * (graph 0's count, the stride of every graph).  Allowed right after
+ * ckv_init_communities(..., n) and before any decode step (n must be the
+ * init's n).  Synchronous, host only.
+ * Errors: CKV_ERR_INVALID_ARG (layout, a column outside [0, n), a negative
+ * weight), CKV_ERR_STATE. */
+ckv_status ckv_set_token_graph(ckv_ctx* ctx, const int64_t* row_ptr_host, const int32_t* col_host,
+                               const float* w_host, int n);
+
+/* Refresh -- Tables 8-9 compare periodic re-partitioning with the
+ * incremental update of step (3).  Each graph's token graph is extended by
+ * the decode-time rows the context recorded since the last init (the new
+ * tokens' top-kappa edges).  It is then partitioned again with ckv_leiden
+ * (gamma; the graphs on parallel host threads), and the communities are
+ * re-initialised from the new labels over [0, n_tok) with the keys K, as
+ * ckv_init_communities does.  Decoding continues with the next n.
+ * n_communities_host [G] (may be NULL) gets each graph's count.  Requires a
+ * registered token graph covering [0, n_init) (ckv_set_token_graph, or the
+ * previous refresh).  Synchronous.
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no token graph, a step half
+ * done), CKV_ERR_CAPACITY (more communities than max_communities: the state
+ * is kept), CKV_ERR_OOM, CKV_ERR_CUDA, sticky device errors. */
+ckv_status ckv_refresh(ckv_ctx* ctx, const void* K, double gamma, int32_t* n_communities_host, void* stream);
+
+/* Modularity (ckv_modularity, on the device) of each graph's current
+ * partition on its current token graph: the registered rows plus the
+ * decode-time rows, with the community of every position the incremental
+ * update gave it (sinks alone).  q_host [G].  Synchronous (allocates and
+ * frees device scratch).
+ * Errors: as ckv_refresh, CKV_ERR_CUDA. */
+ckv_status ckv_graph_modularity(ckv_ctx* ctx, double gamma, double* q_host, void* stream);
+
 /* Initial partition -- Figure 1, step (2): community c of graph g holds the
  * positions j in [S, n) with labels[g][j] == c (ascending); its centroid is
  * the mean of those keys (float, summed in double).  labels: int32

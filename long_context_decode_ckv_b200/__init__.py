@@ -100,6 +100,12 @@ def lib() -> ctypes.CDLL:
     L.ckv_modularity_workspace.argtypes = [I]
     L.ckv_modularity.restype = st
     L.ckv_modularity.argtypes = [I, P, P, P, P, I, ctypes.c_double, P, ctypes.POINTER(ctypes.c_double), P]
+    L.ckv_set_token_graph.restype = st
+    L.ckv_set_token_graph.argtypes = [P, P, P, P, I]
+    L.ckv_refresh.restype = st
+    L.ckv_refresh.argtypes = [P, P, ctypes.c_double, P, P]
+    L.ckv_graph_modularity.restype = st
+    L.ckv_graph_modularity.argtypes = [P, ctypes.c_double, P, P]
     L.ckv_step_recall.restype = st
     L.ckv_step_recall.argtypes = [P, P, P, I, P, P]
     L.ckv_dense_decode.restype = st
@@ -193,6 +199,18 @@ def ckv_modularity(n, row_ptr, col, w, labels, n_communities, gamma, workspace, 
     _check("ckv_modularity", lib().ckv_modularity(n, _ptr(row_ptr), _ptr(col), _ptr(w), _ptr(labels), n_communities,
                                                   float(gamma), _ptr(workspace), ctypes.byref(q), _stream(stream)))
     return q.value
+
+
+def ckv_set_token_graph(ctx, row_ptr_host, col_host, w_host, n):
+    _check("ckv_set_token_graph", lib().ckv_set_token_graph(ctx, _ptr(row_ptr_host), _ptr(col_host), _ptr(w_host), n))
+
+
+def ckv_refresh(ctx, K, gamma, n_communities_host=None, stream=None):
+    _check("ckv_refresh", lib().ckv_refresh(ctx, _ptr(K), float(gamma), _ptr(n_communities_host), _stream(stream)))
+
+
+def ckv_graph_modularity(ctx, gamma, q_host, stream=None):
+    _check("ckv_graph_modularity", lib().ckv_graph_modularity(ctx, float(gamma), _ptr(q_host), _stream(stream)))
 
 
 def ckv_init_communities(ctx, labels, labels_on_device, n_communities, K, n, stream=None):

@@ -14,6 +14,7 @@
 #include <algorithm>
 #include <array>
 #include <new>
+#include <thread>
 #include <vector>
 
 #include "ckv_internal.cuh"
@@ -46,6 +47,16 @@ struct ckv_ctx {
     std::vector<cudaEvent_t> ev_pool;   // all events ever created (reused)
     size_t ev_used;
     std::vector<std::array<cudaEvent_t, 6>> ev_steps;
+    // token graph of every graph on the host (rows [0, tg_rows)): the
+    // prefill graph the caller registered, extended by decode-time rows at
+    // each refresh
+    struct TokenGraph {
+        std::vector<int64_t> rp;
+        std::vector<int32_t> col;
+        std::vector<float> w;
+    };
+    std::vector<TokenGraph> tg;
+    int tg_rows;
 };
 
 namespace {
@@ -786,6 +797,177 @@ CKV_API ckv_status ckv_modularity(int n, const int64_t* row_ptr, const int32_t* 
     CKV_CUDA(cudaMemcpyAsync(q_host, q_dev, sizeof(double), cudaMemcpyDeviceToHost, st));
     CKV_CUDA(cudaStreamSynchronize(st));
     if (*q_host != *q_host) return CKV_ERR_INVALID_ARG;   // a label or column out of range
+    return CKV_OK;
+}
+
+// ---------------------------------------------------------------- refresh
+CKV_API ckv_status ckv_set_token_graph(ckv_ctx* x, const int64_t* row_ptr_host, const int32_t* col_host,
+                                       const float* w_host, int n)
+{
+    ckv_status cs = check_ctx(x);
+    if (cs != CKV_OK) return cs;
+    if (!row_ptr_host || !col_host || !w_host) return CKV_ERR_INVALID_ARG;
+    if (!x->initialized || x->pending || n != x->d.n_init || n != x->n_tok) return CKV_ERR_STATE;
+    const int G = x->d.G;
+    const int64_t E = row_ptr_host[n];                         // edge stride of every graph
+    std::vector<ckv_ctx::TokenGraph> tg((size_t)G);
+    for (int g = 0; g < G; ++g) {
+        const int64_t* rp = row_ptr_host + (size_t)g * (n + 1);
+        if (rp[0] != 0 || rp[n] > E) return CKV_ERR_INVALID_ARG;
+        for (int i = 0; i < n; ++i)
+            if (rp[i + 1] < rp[i]) return CKV_ERR_INVALID_ARG;
+        const int32_t* col = col_host + (size_t)g * E;
+        const float* w = w_host + (size_t)g * E;
+        for (int64_t e = 0; e < rp[n]; ++e)
+            if (col[e] < 0 || col[e] >= n || !(w[e] >= 0.0f)) return CKV_ERR_INVALID_ARG;
+        tg[(size_t)g].rp.assign(rp, rp + n + 1);
+        tg[(size_t)g].col.assign(col, col + rp[n]);
+        tg[(size_t)g].w.assign(w, w + rp[n]);
+    }
+    x->tg.swap(tg);
+    x->tg_rows = n;
+    return CKV_OK;
+}
+
+namespace {
+
+// the decode-time rows [n_init, n_tok) of every graph, from the device
+cudaError_t fetch_decode_rows(ckv_ctx* x, std::vector<int32_t>& deg, std::vector<int32_t>& col,
+                              std::vector<float>& w)
+{
+    const Dims& d = x->d;
+    const size_t rows = (size_t)(x->n_tok - d.n_init), G = d.G, er = (size_t)x->edge_rows;
+    deg.assign(G * rows, 0);
+    col.assign(G * rows * d.kappa, 0);
+    w.assign(G * rows * d.kappa, 0.f);
+    if (!rows) return cudaSuccess;
+    cudaError_t e;
+    for (size_t g = 0; g < G; ++g) {
+        if ((e = cudaMemcpy(&deg[g * rows], x->s.edge_deg + g * er, rows * 4, cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return e;
+        if ((e = cudaMemcpy(&col[g * rows * d.kappa], x->s.edge_col + g * er * d.kappa, rows * d.kappa * 4,
+                            cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return e;
+        if ((e = cudaMemcpy(&w[g * rows * d.kappa], x->s.edge_w + g * er * d.kappa, rows * d.kappa * 4,
+                            cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
+// graph g's token graph over [0, n_tok): the host rows, then the decode rows
+ckv_ctx::TokenGraph combined_graph(const ckv_ctx* x, int g, const std::vector<int32_t>& deg,
+                                   const std::vector<int32_t>& col, const std::vector<float>& w)
+{
+    const Dims& d = x->d;
+    const size_t rows = (size_t)(x->n_tok - d.n_init);
+    ckv_ctx::TokenGraph t = x->tg[(size_t)g];
+    for (size_t r = 0; r < rows; ++r) {
+        const int nd = deg[(size_t)g * rows + r];
+        for (int k = 0; k < nd; ++k) {
+            t.col.push_back(col[((size_t)g * rows + r) * d.kappa + k]);
+            t.w.push_back(w[((size_t)g * rows + r) * d.kappa + k]);
+        }
+        t.rp.push_back((int64_t)t.col.size());
+    }
+    return t;
+}
+
+}  // namespace
+
+CKV_API ckv_status ckv_refresh(ckv_ctx* x, const void* K, double gamma, int32_t* n_communities_host, void* stream)
+{
+    ckv_status cs = check_ctx(x);
+    if (cs != CKV_OK) return cs;
+    if (!K || !(gamma > 0.0)) return CKV_ERR_INVALID_ARG;
+    if (!x->initialized || x->pending || x->tg.empty() || x->tg_rows != x->d.n_init) return CKV_ERR_STATE;
+    CKV_CUDA(cudaSetDevice(x->cfg.device));
+    CKV_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+    cs = read_device_error(x);
+    if (cs != CKV_OK) { x->sticky = cs; return cs; }
+    std::vector<int32_t> deg, col;
+    std::vector<float> w;
+    CKV_CUDA(fetch_decode_rows(x, deg, col, w));
+    const int G = x->d.G, n = x->n_tok;
+    std::vector<ckv_ctx::TokenGraph> next((size_t)G);
+    std::vector<int32_t> labels((size_t)G * n), counts((size_t)G, 0);
+    // the graphs are independent: partition them on several host threads
+    const int nthr = std::max(1, std::min(G, (int)std::thread::hardware_concurrency()));
+    std::vector<std::thread> pool;
+    std::vector<char> failed((size_t)nthr + 1, 0);
+    auto work = [&](int t) {
+        try {
+            for (int g = t; g < G; g += nthr) {
+                next[(size_t)g] = combined_graph(x, g, deg, col, w);
+                counts[(size_t)g] = ckv::leiden_partition(n, next[(size_t)g].rp.data(), next[(size_t)g].col.data(),
+                                                          next[(size_t)g].w.data(), gamma, 64, &labels[(size_t)g * n]);
+            }
+        } catch (...) {
+            failed[(size_t)t] = 1;
+        }
+    };
+    try {
+        for (int t = 1; t < nthr; ++t) pool.emplace_back(work, t);
+    } catch (...) {
+        failed[(size_t)nthr] = 1;   // fewer threads: this one still covers its own share below
+    }
+    work(0);
+    for (auto& th : pool) th.join();
+    if (failed[(size_t)nthr]) {     // a thread could not start: finish its graphs here
+        for (int t = (int)pool.size() + 1; t < nthr; ++t) work(t);
+    }
+    for (int t = 0; t < nthr; ++t)
+        if (failed[(size_t)t]) return CKV_ERR_OOM;
+    const int nc = *std::max_element(counts.begin(), counts.end());
+    if (nc > x->d.Nc) return CKV_ERR_CAPACITY;   // the state is unchanged
+    cs = ckv_init_communities(x, labels.data(), 0, nc, K, n, stream);
+    if (cs != CKV_OK) return cs;
+    x->tg.swap(next);
+    x->tg_rows = n;
+    if (n_communities_host)
+        for (int g = 0; g < G; ++g) n_communities_host[g] = counts[(size_t)g];
+    return CKV_OK;
+}
+
+CKV_API ckv_status ckv_graph_modularity(ckv_ctx* x, double gamma, double* q_host, void* stream)
+{
+    ckv_status cs = check_ctx(x);
+    if (cs != CKV_OK) return cs;
+    if (!q_host || !(gamma > 0.0)) return CKV_ERR_INVALID_ARG;
+    if (!x->initialized || x->pending || x->tg.empty() || x->tg_rows != x->d.n_init) return CKV_ERR_STATE;
+    cudaStream_t st = (cudaStream_t)stream;
+    CKV_CUDA(cudaSetDevice(x->cfg.device));
+    CKV_CUDA(cudaStreamSynchronize(st));
+    std::vector<int32_t> deg, col;
+    std::vector<float> w;
+    CKV_CUDA(fetch_decode_rows(x, deg, col, w));
+    const Dims& d = x->d;
+    const int n = x->n_tok;
+    std::vector<int32_t> lab((size_t)n);
+    for (int g = 0; g < d.G; ++g) {
+        const ckv_ctx::TokenGraph t = combined_graph(x, g, deg, col, w);
+        CKV_CUDA(cudaMemcpy(lab.data(), x->s.tok_comm + (size_t)g * d.NM, (size_t)n * 4, cudaMemcpyDeviceToHost));
+        for (int32_t& l : lab) l = (l < 0) ? d.n_comm : l;      // sinks (no edges): one extra label
+        const size_t E = t.col.size();
+        void* buf = nullptr;
+        const size_t bytes = (size_t)(n + 1) * 8 + E * 8 + (size_t)n * 4 + ckv_modularity_workspace(d.n_comm + 1) + 64;
+        CKV_CUDA(cudaMalloc(&buf, bytes));
+        char* p = static_cast<char*>(buf);
+        int64_t* drp = reinterpret_cast<int64_t*>(p);
+        int32_t* dcol = reinterpret_cast<int32_t*>(p + (size_t)(n + 1) * 8);
+        float* dw = reinterpret_cast<float*>(p + (size_t)(n + 1) * 8 + E * 4);
+        int32_t* dlab = reinterpret_cast<int32_t*>(p + (size_t)(n + 1) * 8 + E * 8);
+        void* ws = reinterpret_cast<void*>(((uintptr_t)(p + (size_t)(n + 1) * 8 + E * 8 + (size_t)n * 4) + 15) & ~(uintptr_t)15);
+        cudaError_t e = cudaMemcpy(drp, t.rp.data(), (size_t)(n + 1) * 8, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && E) e = cudaMemcpy(dcol, t.col.data(), E * 4, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && E) e = cudaMemcpy(dw, t.w.data(), E * 4, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) e = cudaMemcpy(dlab, lab.data(), (size_t)n * 4, cudaMemcpyHostToDevice);
+        ckv_status r = (e == cudaSuccess) ? ckv_modularity(n, drp, dcol, dw, dlab, d.n_comm + 1, gamma, ws,
+                                                           &q_host[g], stream)
+                                          : CKV_ERR_CUDA;
+        cudaFree(buf);
+        if (r != CKV_OK) return r;
+    }
     return CKV_OK;
 }
 
