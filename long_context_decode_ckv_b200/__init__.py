@@ -182,8 +182,33 @@ def ckv_build_graph_grouped(n_kv_heads, group, n, head_dim, n_sinks, kappa, dtyp
         _ptr(col), _ptr(w), _stream(stream)))
 
 
+def _host_in(a, dtype):
+    """A host array for an input argument: C-contiguous, of exactly `dtype`."""
+    import numpy as np
+    a = np.asarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected a {np.dtype(dtype).name} array, got {a.dtype}")
+    return np.ascontiguousarray(a)
+
+
+def _host_out(a, dtype):
+    """A host array the library writes: C-contiguous, writable, exactly `dtype`."""
+    import numpy as np
+    if not isinstance(a, np.ndarray) or a.dtype != dtype or not a.flags["C_CONTIGUOUS"] or not a.flags["WRITEABLE"]:
+        raise TypeError(f"expected a writable C-contiguous {np.dtype(dtype).name} numpy array")
+    return a
+
+
 def ckv_leiden(n, row_ptr_host, col_host, w_host, gamma, labels_host) -> int:
     """Leiden partition on the host (numpy arrays); returns the community count."""
+    import numpy as np
+    row_ptr_host = _host_in(row_ptr_host, np.int64)
+    col_host = _host_in(col_host, np.int32)
+    w_host = _host_in(w_host, np.float32)
+    labels_host = _host_out(labels_host, np.int32)
+    if len(row_ptr_host) < n + 1 or len(labels_host) < n or len(col_host) < row_ptr_host[n] or \
+            len(w_host) < row_ptr_host[n]:
+        raise ValueError("array shorter than the graph")
     c = ctypes.c_int(0)
     _check("ckv_leiden", lib().ckv_leiden(n, _ptr(row_ptr_host), _ptr(col_host), _ptr(w_host), float(gamma),
                                           _ptr(labels_host), ctypes.byref(c)))
@@ -202,14 +227,23 @@ def ckv_modularity(n, row_ptr, col, w, labels, n_communities, gamma, workspace, 
 
 
 def ckv_set_token_graph(ctx, row_ptr_host, col_host, w_host, n):
+    import numpy as np
+    row_ptr_host = _host_in(row_ptr_host, np.int64)
+    col_host = _host_in(col_host, np.int32)
+    w_host = _host_in(w_host, np.float32)
     _check("ckv_set_token_graph", lib().ckv_set_token_graph(ctx, _ptr(row_ptr_host), _ptr(col_host), _ptr(w_host), n))
 
 
 def ckv_refresh(ctx, K, gamma, n_communities_host=None, stream=None):
+    import numpy as np
+    if n_communities_host is not None:
+        n_communities_host = _host_out(n_communities_host, np.int32)
     _check("ckv_refresh", lib().ckv_refresh(ctx, _ptr(K), float(gamma), _ptr(n_communities_host), _stream(stream)))
 
 
 def ckv_graph_modularity(ctx, gamma, q_host, stream=None):
+    import numpy as np
+    q_host = _host_out(q_host, np.float64)
     _check("ckv_graph_modularity", lib().ckv_graph_modularity(ctx, float(gamma), _ptr(q_host), _stream(stream)))
 
 

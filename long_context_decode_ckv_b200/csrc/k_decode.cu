@@ -516,12 +516,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
 //
 // Each warp keeps an online softmax (running max and sum per head) and
 // spills the kept members' logits to L2.  The CTA combines its warps into
-// one (m, l, o) partial per head and publishes it; once all slices of the
-// graph have published (a per-graph arrival counter: the grid is
-// co-resident by cooperative launch, and the wait is bounded), every slice
-// derives the graph's exact softmax statistics, writes its share of the
-// output and ranks its own kept members' edge weights w_j; the last slice
-// to finish merges the slices' candidate lists into the top-kappa edges.
+// one (m, l, o) partial per head, publishes it and counts itself in on the
+// graph's arrival counter; no CTA waits.  The slice that arrives last
+// finishes the graph (finish_graph):
+// - it merges the partials into the output and the softmax statistics;
+// - it ranks the kept members' edge weights w_j into the top-kappa edges;
+// - it votes on the new token's community and updates that community.
 constexpr int kAttNBuf = 3;        // batches per warp pipeline
 
 template <bool BF16, int HG>

@@ -80,3 +80,15 @@ def test_arguments_checked():
         with pytest.raises(ckv.CkvError) as e:
             ckv.ckv_leiden(*args, lab)
         assert e.value.status == ckv.CKV_ERR_INVALID_ARG
+
+
+def test_binding_checks_host_arrays():
+    rp = np.array([0, 1, 1], np.int64)
+    col = np.array([0], np.int32)
+    w = np.array([1.0], np.float32)
+    with pytest.raises(TypeError):
+        ckv.ckv_leiden(2, rp.astype(np.int32), col, w, 1.0, np.zeros(2, np.int32))   # wrong row_ptr dtype
+    with pytest.raises(TypeError):
+        ckv.ckv_leiden(2, rp, col, w, 1.0, np.zeros(2, np.int64))                  # wrong labels dtype
+    with pytest.raises(ValueError):
+        ckv.ckv_leiden(3, rp, col, w, 1.0, np.zeros(3, np.int32))                  # row_ptr too short
