@@ -155,6 +155,17 @@ cudaError_t alloc_edges(ckv_ctx* x, int64_t rows)
     return cudaSuccess;
 }
 
+// empty score range and zero total size for every graph (k_score accumulates
+// into it, k_select resets it after reading)
+cudaError_t reset_srange(ckv_ctx* x, cudaStream_t st)
+{
+    std::vector<uint32_t> h((size_t)x->d.G * 4, 0u);
+    for (size_t g = 0; g < (size_t)x->d.G; ++g) h[4 * g] = 0xffffffffu;
+    cudaError_t e = cudaMemcpyAsync(x->s.srange, h.data(), h.size() * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e;
+}
+
 ckv_status read_device_error(ckv_ctx* x)
 {
     int err = 0;
@@ -311,6 +322,7 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(e_w, G * kap);
     ALLOC(e_comm, G * kap);
     ALLOC(sel_ml, (size_t)d.B * d.Hq * 2);
+    ALLOC(srange, G * 4);
     ALLOC(err, 1);
 #undef ALLOC
     if (e == cudaSuccess) e = dalloc(x, &x->dense_part, ckv::dense_part_floats(d));
@@ -319,6 +331,7 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     if (e == cudaSuccess) e = cudaMemset(s.bar, 0, G * 2 * sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemset(s.err, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(s.meta, 0, G * ckv::M_COUNT * sizeof(int32_t));
+    if (e == cudaSuccess) e = reset_srange(x, 0);
     const size_t qb = (size_t)d.B * d.Hq * ckv::kD;
     x->stage_bytes = qb * elem_bytes(cfg->kv_dtype) + 2 * (size_t)d.B * d.Hkv * ckv::kD * elem_bytes(cfg->kv_dtype) +
                      qb * sizeof(float) + 64;
@@ -369,6 +382,7 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
     step(cudaMemsetAsync(s.tok_comm, 0xff, G * d.NM * sizeof(int32_t), st));
     step(cudaMemsetAsync(s.bar, 0, G * 2 * sizeof(unsigned), st));
     step(cudaMemsetAsync(s.mu, 0, G * d.Nc * ckv::kD * sizeof(float), st));
+    step(reset_srange(x, st));
     step(ckv::launch_init_count(s, d, dlabels, n, st));
     int err = 0;
     step(cudaMemcpyAsync(&err, s.err, sizeof(int), cudaMemcpyDeviceToHost, st));
@@ -717,6 +731,7 @@ CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t byt
     }
     CKV_CUDA(cudaMemset(s.err, 0, sizeof(int)));
     CKV_CUDA(cudaMemset(s.bar, 0, G * 2 * sizeof(unsigned)));
+    CKV_CUDA(reset_srange(x, 0));
     CKV_CUDA(cudaDeviceSynchronize());
     d.n_comm = Nc;
     d.n_init = n_init;

@@ -19,6 +19,7 @@
 //   part_o    float [G][KC][HG][D] per-CTA P.V per head, relative to its max
 //   bar       uint  [G][2]         arrivals of a graph's slices (slot 0)
 //   e_*       [G][kappa]           the step's edges (rank order) for the update
+//   srange    uint  [G][4]         score range keys and total size of the step (k_score -> k_select)
 //   sel_ml    float [B][Hq][2]     softmax max and sum of each query head over the
 //                                  step's attended rows (for the attention-mass recall)
 // Dense statistics scratch (k_dense.cu; U = B*Hkv units):
@@ -66,6 +67,8 @@ struct DevState {
     float* e_w;
     int32_t* e_comm;
     float* sel_ml;           // may be null (then the attention kernel does not write it)
+    uint32_t* srange;        // [G][4] min and max score key of the non-empty communities, their total
+                             // size, pad: accumulated by k_score, read and reset by k_select
     int* err;                // sticky device error word (ckv_status)
 };
 

@@ -127,10 +127,32 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, 
     const int c = warp - 1;
     int gq = -1;
     float qs[4] = {0.f, 0.f, 0.f, 0.f};
+    // the graph's score range over its non-empty communities and their
+    // total size, for the selection: each lane keeps its own while the warp
+    // stays on one graph, then one reduction and three atomics per graph
+    uint32_t rmin = 0xffffffffu, rmax = 0u;
+    int rsum = 0;
+    auto flush_range = [&](int gf) {
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            rmin = min(rmin, __shfl_xor_sync(kFull, rmin, o));
+            rmax = max(rmax, __shfl_xor_sync(kFull, rmax, o));
+            rsum += __shfl_xor_sync(kFull, rsum, o);
+        }
+        if (lane == 0 && gf >= 0 && rmax != 0u) {
+            atomicMin(s.srange + 4 * gf, rmin);
+            atomicMax(s.srange + 4 * gf + 1, rmax);
+            atomicAdd(s.srange + 4 * gf + 2, (unsigned)rsum);
+        }
+        rmin = 0xffffffffu;
+        rmax = 0u;
+        rsum = 0;
+    };
     for (int u = c; u < nu; u += kScoreCW) {
         const int64_t gu = u0 + u;
         const int g = (int)(gu / upg), c0 = (int)(gu % upg) * 32;
         if (g != gq) {   // sum of the graph's query heads, this lane's 4 dims
+            flush_range(gq);
             int b, h0, kvh;
             graph_heads(d, g, b, h0, kvh);
 #pragma unroll
@@ -168,15 +190,23 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, 
             }
         }
         if (lane < rows) s.score[gi] = (sz > 0) ? part[0] : -INFINITY;
+        if (lane < rows && sz > 0) {   // this lane's running range and size (order-preserving keys; +0 for -0)
+            const uint32_t k = ord_u(part[0] + 0.0f);
+            rmin = min(rmin, k);
+            rmax = max(rmax, k);
+            rsum += sz;
+        }
     }
+    flush_range(gq);
     if (*abort_flag && c == 0 && lane == 0) set_error(s.err, CKV_ERR_TIMEOUT);
 }
 
 // --------------------------------------------------------------- k_select
 // One CTA of 1024 threads per graph.  Thread t owns communities t, t + 1024,
-// ... (E of them, scores and sizes in registers); its status lives in
-// shared memory.  Exact budgeted top-C in (score desc, id asc) order:
-//   1. one round of loads; the score range and the total size;
+// ... (E of them, scores and sizes in registers, their status in register
+// bit masks).  Exact budgeted top-C in (score desc, id asc) order:
+//   1. one round of loads; the score range and the total size come from
+//      k_score (order-preserving keys reduced by atomics per graph);
 //   2. a size-weighted histogram over kSelBins bins, linear in the score
 //      (bins are monotone in the score, so every community of a higher bin
 //      ranks before every one of a lower bin); the boundary bin is where the
@@ -188,7 +218,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, 
 //      size of the better ones, and is kept iff the sizes through it fit;
 //   5. the kept ids in ascending order with the prefix of their sizes, by
 //      ballots per 32 ids and one scan over the (round, warp) counts;
-//   6. each kept community's owner copies its members into the row list.
+//   6. warps copy the kept communities' member segments into the row list,
+//      eight communities' loads in flight per warp.
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelCand = 1024;     // boundary-bin communities ranked exactly
@@ -226,7 +257,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
     if (d.pdl == 1) pdl_trigger();
     if (*(volatile int*)s.err) return;
     extern __shared__ __align__(16) unsigned char smem_sel[];
-    __shared__ float r_lo[kSelWarps], r_hi[kSelWarps];
     __shared__ int r_w[kSelWarps];
     __shared__ unsigned long long r_kmin[kSelWarps], r_kmax[kSelWarps];
     __shared__ int off_c[E][kSelWarps], off_w[E][kSelWarps];
@@ -249,40 +279,23 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
         v[i] = (c < Nc) ? gsc[c] : 0.f;
         co[i] = (c < Nc) ? gco[c] : 0;
     }
+    // the score range and the total size, left by k_score
+    const uint4 rg = __ldcg(reinterpret_cast<const uint4*>(s.srange + 4 * g));
     // status of the thread's communities as bit masks: still a candidate
     // (cmask), surely kept (imask)
     unsigned cmask = 0u, imask = 0u;
-    float lo = INFINITY, hi = -INFINITY;
-    int wsum = 0;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
-        if (w[i] > 0) {
-            lo = fminf(lo, v[i]);
-            hi = fmaxf(hi, v[i]);
-            wsum += w[i];
-            cmask |= 1u << i;
-        } else {
-            w[i] = 0;
-        }
+        if (w[i] > 0) cmask |= 1u << i;
+        else w[i] = 0;
     }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        lo = fminf(lo, __shfl_xor_sync(kFull, lo, o));
-        hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, o));
-        wsum += __shfl_xor_sync(kFull, wsum, o);
-    }
-    if (lane == 0) { r_lo[warp] = lo; r_hi[warp] = hi; r_w[warp] = wsum; }
+    auto from_ord = [](uint32_t u) { return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u); };
+    const bool any = rg.y != 0u;
+    const float lo = any ? from_ord(rg.x) : INFINITY, hi = any ? from_ord(rg.y) : -INFINITY;
+    const int wsum = (int)rg.z;
     if (tid == 0) { sh_n = 0; sh_above = 0; sh_bn = 0; sh_bt = 0; }
     __syncthreads();
-    lo = r_lo[lane];
-    hi = r_hi[lane];
-    wsum = r_w[lane];
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        lo = fminf(lo, __shfl_xor_sync(kFull, lo, o));
-        hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, o));
-        wsum += __shfl_xor_sync(kFull, wsum, o);
-    }
+    if (tid == 0) *reinterpret_cast<uint4*>(s.srange + 4 * g) = make_uint4(0xffffffffu, 0u, 0u, 0u);   // for the next step
 
     // shared memory: the passes' histogram and boundary candidates, later
     // (same bytes) the kept list
@@ -326,8 +339,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
             const int incl = warp_incl(x, lane);
             if (lane == 31) r_w[warp] = incl;
             __syncthreads();
-            int wpre = 0;
-            for (int j = 0; j < warp; ++j) wpre += r_w[j];
+            const int rw = r_w[lane];   // kSelWarps == 32
+            const int wpre = __shfl_sync(kFull, warp_incl(rw, lane) - rw, warp);
             const int bef = above + wpre + incl - x;
             if (bef <= budget && bef + h0 > budget) { sh_b = b0; sh_above = bef; }
             else if (bef + h0 <= budget && bef + h0 + h1 > budget) { sh_b = b1; sh_above = bef + h0; }
