@@ -75,9 +75,9 @@ KERNEL_SOURCES = {
     "k_dense_attention": ("k_dense.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
 }
 PROFILED_TRAFFIC = {
-    "k_score": ("f92868379799ae92", 139.236864e6),
-    "k_attend": ("f92868379799ae92", 68.953856e6),
-    "k_dense_stats": ("b8df1d15a63cd101", 1079.294656e6),
+    "k_score": ("50d47023298fccf9", 139.16185e6),
+    "k_attend": ("50d47023298fccf9", 69.00096e6),
+    "k_dense_stats": ("1674ed41fb19dce3", 1079.90176e6),
 }
 
 
