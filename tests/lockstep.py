@@ -1,8 +1,9 @@
 """Lockstep parity checker: the CUDA library against the CPU oracle, step by
 step, on the same seeded workload.
 
-Per decode step and tracked graph it compares (rules of the north-star
-contract, readings listed in the design doc):
+Per decode step and tracked graph it compares ("CommunityKV: Efficient
+Long-Context Decoding via Graph Partitioning", Figure 1 caption step (3);
+tolerances: bf16 inputs with fp32 accumulation, decisions on the float value):
 
 * attention output: max |o_gpu - o_ref| / max |o_ref| <= 2e-3 per (batch, head);
 * kept communities, edge set and assigned community: bit-exact, except where
