@@ -69,6 +69,28 @@ def test_same_labels_on_prefill_graph(oracle_lib):
     assert oracle.modularity(rp, cc, ww, lab) > 0.3
 
 
+def test_edge_cases_match_oracle(oracle_lib):
+    empty = (np.zeros(0, np.int32), np.zeros(0, np.float32))
+    cases = [
+        (1, np.array([0, 0], np.int64), *empty),                                  # one node
+        (5, np.zeros(6, np.int64), *empty),                                       # no edges
+        (5, np.array([0, 1, 1, 1, 2, 2], np.int64), np.array([3, 0], np.int32),  # isolated nodes
+         np.array([1.0, 2.0], np.float32)),
+        (2, np.array([0, 1, 2], np.int64), np.array([0, 0], np.int32),           # a self-loop
+         np.array([1.0, 1.0], np.float32)),
+        (2, np.array([0, 1, 2], np.int64), np.array([1, 0], np.int32),           # zero weights
+         np.array([0.0, 0.0], np.float32)),
+    ]
+    expect = {0: [0], 1: [0, 1, 2, 3, 4], 2: [0, 1, 2, 0, 3], 4: [0, 1]}       # hand-derived
+    for k, (n, rp, col, w) in enumerate(cases):
+        lab, C = _lib_leiden(rp, col, w, n, 1.0)
+        ref, Cr = oracle.leiden(rp, col, w, n, 1.0)
+        assert C == Cr
+        np.testing.assert_array_equal(lab, ref)
+        if k in expect:
+            assert list(lab) == expect[k] and C == max(expect[k]) + 1
+
+
 def test_arguments_checked():
     rp = np.array([0, 1, 1], np.int64)
     lab = np.zeros(2, np.int32)
@@ -76,10 +98,15 @@ def test_arguments_checked():
                  (2, rp, np.array([0], np.int32), np.array([-1.0], np.float32), 1.0),     # negative weight
                  (2, rp, np.array([0], np.int32), np.array([1.0], np.float32), 0.0),      # gamma
                  (2, np.array([0, 2, 1], np.int64), np.array([0, 1], np.int32),
-                  np.array([1.0, 1.0], np.float32), 1.0)):                                # row_ptr not monotone
+                  np.array([1.0, 1.0], np.float32), 1.0),                                 # row_ptr not monotone
+                 (2, rp, np.array([0], np.int32), np.array([np.nan], np.float32), 1.0)):  # NaN weight
         with pytest.raises(ckv.CkvError) as e:
             ckv.ckv_leiden(*args, lab)
         assert e.value.status == ckv.CKV_ERR_INVALID_ARG
+    with pytest.raises(ckv.CkvError) as e:                                          # n < 1
+        ckv.ckv_leiden(0, np.zeros(1, np.int64), np.zeros(0, np.int32), np.zeros(0, np.float32), 1.0,
+                       np.zeros(0, np.int32))
+    assert e.value.status == ckv.CKV_ERR_INVALID_ARG
 
 
 def test_binding_checks_host_arrays():
