@@ -684,6 +684,7 @@ def main():
         kh = torch.from_numpy(np.ascontiguousarray(wl.K[:, :, cfg.n0:])).pin_memory()
         vh = torch.from_numpy(np.ascontiguousarray(wl.V[:, :, cfg.n0:])).pin_memory()
         oh = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32).pin_memory()
+        qstep = [qh[i] for i in range(cfg.steps)]   # each step's pinned host buffers
         kstep = [kh[:, :, i].contiguous() for i in range(cfg.steps)]
         vstep = [vh[:, :, i].contiguous() for i in range(cfg.steps)]
         s0 = s_prof + args.profile_steps
@@ -695,7 +696,7 @@ def main():
         for s in range(s0, s0 + args.e2e_steps):
             r = reps[s % L]
             i = r["i"]
-            ckv.ckv_decode_host(r["ctx"], qh[i], kstep[i], vstep[i], r["K"], r["V"], cfg.n0 + i + 1,
+            ckv.ckv_decode_host(r["ctx"], qstep[i], kstep[i], vstep[i], r["K"], r["V"], cfg.n0 + i + 1,
                                 oh, stream)
             r["i"] = i + 1
         e1.record(stream)
