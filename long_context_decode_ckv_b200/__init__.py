@@ -3,8 +3,10 @@ attention for B200 (sm_100a).
 
 Argument marshalling only: every function below calls the C entry point of
 the same name in libckv.so (declared in include/ckv.h), passing device
-pointers of torch tensors and the raw CUDA stream.  No step of the method
-runs in Python.  If the compiled library is missing, the first call raises
+pointers of torch tensors and the raw CUDA stream.  A device argument must be
+a CUDA tensor (or a raw int address) and a host argument a numpy array or CPU
+tensor; the wrong kind raises TypeError before the call.  No step of the
+method runs in Python.  If the compiled library is missing, the first call raises
 ``RuntimeError`` -- there is no fallback.
 
 Method: "CommunityKV: Efficient Long-Context Decoding via Graph
@@ -116,17 +118,32 @@ def lib() -> ctypes.CDLL:
     return L
 
 
-def _ptr(x) -> int | None:
-    """Device/host address of a torch tensor, numpy array, int or None."""
-    if x is None:
-        return None
-    if isinstance(x, int):
+def _dev(x) -> int | None:
+    """Address of a device-memory argument: a CUDA torch tensor, a raw int
+    address (taken as device memory) or None.  Host memory is refused here,
+    before the call, since a kernel cannot dereference it."""
+    if x is None or isinstance(x, int):
         return x
-    if hasattr(x, "data_ptr"):
+    if hasattr(x, "is_cuda"):
+        if not x.is_cuda:
+            raise TypeError("expected device memory (a CUDA tensor), got a CPU tensor")
+        return x.data_ptr()
+    raise TypeError(f"expected device memory (a CUDA tensor), got {type(x).__name__}")
+
+
+def _hostp(x) -> int | None:
+    """Address of a host-memory argument: a numpy array, a CPU torch tensor,
+    a raw int address (taken as host memory) or None.  A CUDA tensor is
+    refused."""
+    if x is None or isinstance(x, int):
+        return x
+    if hasattr(x, "is_cuda"):
+        if x.is_cuda:
+            raise TypeError("expected host memory, got a CUDA tensor")
         return x.data_ptr()
     if hasattr(x, "ctypes"):
         return x.ctypes.data
-    raise TypeError(f"cannot take the address of {type(x)}")
+    raise TypeError(f"expected host memory (a numpy array or CPU tensor), got {type(x).__name__}")
 
 
 def _stream(s) -> int | None:
@@ -167,8 +184,8 @@ def ckv_destroy(ctx: int) -> None:
 
 def ckv_build_graph(n_heads, n, head_dim, n_sinks, kappa, dtype, Q, K, row_ptr, col, w, stream=None):
     _check("ckv_build_graph", lib().ckv_build_graph(
-        n_heads, n, head_dim, n_sinks, kappa, dtype, _ptr(Q), _ptr(K), _ptr(row_ptr), _ptr(col),
-        _ptr(w), _stream(stream)))
+        n_heads, n, head_dim, n_sinks, kappa, dtype, _dev(Q), _dev(K), _dev(row_ptr), _dev(col),
+        _dev(w), _stream(stream)))
 
 
 def ckv_build_graph_grouped_workspace(n_kv_heads, group, n) -> int:
@@ -178,8 +195,8 @@ def ckv_build_graph_grouped_workspace(n_kv_heads, group, n) -> int:
 def ckv_build_graph_grouped(n_kv_heads, group, n, head_dim, n_sinks, kappa, dtype, Q, K, workspace, row_ptr, col, w,
                             stream=None):
     _check("ckv_build_graph_grouped", lib().ckv_build_graph_grouped(
-        n_kv_heads, group, n, head_dim, n_sinks, kappa, dtype, _ptr(Q), _ptr(K), _ptr(workspace), _ptr(row_ptr),
-        _ptr(col), _ptr(w), _stream(stream)))
+        n_kv_heads, group, n, head_dim, n_sinks, kappa, dtype, _dev(Q), _dev(K), _dev(workspace), _dev(row_ptr),
+        _dev(col), _dev(w), _stream(stream)))
 
 
 def _host_in(a, dtype):
@@ -210,8 +227,8 @@ def ckv_leiden(n, row_ptr_host, col_host, w_host, gamma, labels_host) -> int:
             len(w_host) < row_ptr_host[n]:
         raise ValueError("array shorter than the graph")
     c = ctypes.c_int(0)
-    _check("ckv_leiden", lib().ckv_leiden(n, _ptr(row_ptr_host), _ptr(col_host), _ptr(w_host), float(gamma),
-                                          _ptr(labels_host), ctypes.byref(c)))
+    _check("ckv_leiden", lib().ckv_leiden(n, _hostp(row_ptr_host), _hostp(col_host), _hostp(w_host), float(gamma),
+                                          _hostp(labels_host), ctypes.byref(c)))
     return c.value
 
 
@@ -221,8 +238,8 @@ def ckv_modularity_workspace(n_communities) -> int:
 
 def ckv_modularity(n, row_ptr, col, w, labels, n_communities, gamma, workspace, stream=None) -> float:
     q = ctypes.c_double(0.0)
-    _check("ckv_modularity", lib().ckv_modularity(n, _ptr(row_ptr), _ptr(col), _ptr(w), _ptr(labels), n_communities,
-                                                  float(gamma), _ptr(workspace), ctypes.byref(q), _stream(stream)))
+    _check("ckv_modularity", lib().ckv_modularity(n, _dev(row_ptr), _dev(col), _dev(w), _dev(labels), n_communities,
+                                                  float(gamma), _dev(workspace), ctypes.byref(q), _stream(stream)))
     return q.value
 
 
@@ -231,39 +248,40 @@ def ckv_set_token_graph(ctx, row_ptr_host, col_host, w_host, n):
     row_ptr_host = _host_in(row_ptr_host, np.int64)
     col_host = _host_in(col_host, np.int32)
     w_host = _host_in(w_host, np.float32)
-    _check("ckv_set_token_graph", lib().ckv_set_token_graph(ctx, _ptr(row_ptr_host), _ptr(col_host), _ptr(w_host), n))
+    _check("ckv_set_token_graph", lib().ckv_set_token_graph(ctx, _hostp(row_ptr_host), _hostp(col_host), _hostp(w_host),
+                                                            n))
 
 
 def ckv_refresh(ctx, K, gamma, n_communities_host=None, stream=None):
     import numpy as np
     if n_communities_host is not None:
         n_communities_host = _host_out(n_communities_host, np.int32)
-    _check("ckv_refresh", lib().ckv_refresh(ctx, _ptr(K), float(gamma), _ptr(n_communities_host), _stream(stream)))
+    _check("ckv_refresh", lib().ckv_refresh(ctx, _dev(K), float(gamma), _hostp(n_communities_host), _stream(stream)))
 
 
 def ckv_graph_modularity(ctx, gamma, q_host, stream=None):
     import numpy as np
     q_host = _host_out(q_host, np.float64)
-    _check("ckv_graph_modularity", lib().ckv_graph_modularity(ctx, float(gamma), _ptr(q_host), _stream(stream)))
+    _check("ckv_graph_modularity", lib().ckv_graph_modularity(ctx, float(gamma), _hostp(q_host), _stream(stream)))
 
 
 def ckv_init_communities(ctx, labels, labels_on_device, n_communities, K, n, stream=None):
     _check("ckv_init_communities", lib().ckv_init_communities(
-        ctx, _ptr(labels), int(labels_on_device), n_communities, _ptr(K), n, _stream(stream)))
+        ctx, (_dev(labels) if labels_on_device else _hostp(labels)), int(labels_on_device), n_communities, _dev(K), n, _stream(stream)))
 
 
 def ckv_decode_step(ctx, q, K, V, n, out, stream=None):
-    _check("ckv_decode_step", lib().ckv_decode_step(ctx, _ptr(q), _ptr(K), _ptr(V), n, _ptr(out),
+    _check("ckv_decode_step", lib().ckv_decode_step(ctx, _dev(q), _dev(K), _dev(V), n, _dev(out),
                                                     _stream(stream)))
 
 
 def ckv_assign_update(ctx, K, n, stream=None):
-    _check("ckv_assign_update", lib().ckv_assign_update(ctx, _ptr(K), n, _stream(stream)))
+    _check("ckv_assign_update", lib().ckv_assign_update(ctx, _dev(K), n, _stream(stream)))
 
 
 def ckv_decode_host(ctx, q_host, k_new_host, v_new_host, K, V, n, out_host, stream=None):
     _check("ckv_decode_host", lib().ckv_decode_host(
-        ctx, _ptr(q_host), _ptr(k_new_host), _ptr(v_new_host), _ptr(K), _ptr(V), n, _ptr(out_host),
+        ctx, _hostp(q_host), _hostp(k_new_host), _hostp(v_new_host), _dev(K), _dev(V), n, _hostp(out_host),
         _stream(stream)))
 
 
@@ -274,8 +292,8 @@ def ckv_last_error(ctx) -> int:
 def ckv_get_step_debug(ctx, n_sel=None, sel=None, n_tok_sel=None, n_edges=None, edges=None,
                        edge_w=None, assigned=None):
     _check("ckv_get_step_debug", lib().ckv_get_step_debug(
-        ctx, _ptr(n_sel), _ptr(sel), _ptr(n_tok_sel), _ptr(n_edges), _ptr(edges), _ptr(edge_w),
-        _ptr(assigned)))
+        ctx, _hostp(n_sel), _hostp(sel), _hostp(n_tok_sel), _hostp(n_edges), _hostp(edges), _hostp(edge_w),
+        _hostp(assigned)))
 
 
 def ckv_profile_begin(ctx) -> None:
@@ -308,18 +326,18 @@ def ckv_attend_rows_static(cfg, q, K, V, n, rows_host, n_rows_host, max_rows, ou
     in the library's static device array); rows_host / n_rows_host are host
     arrays."""
     _check("ckv_attend_rows_static", lib().ckv_attend_rows_static(
-        ctypes.byref(cfg), _ptr(q), _ptr(K), _ptr(V), n, _ptr(rows_host), _ptr(n_rows_host), max_rows,
-        _ptr(out), _stream(stream)))
+        ctypes.byref(cfg), _dev(q), _dev(K), _dev(V), n, _hostp(rows_host), _hostp(n_rows_host), max_rows,
+        _dev(out), _stream(stream)))
 
 
 def ckv_step_recall(ctx, q, K, n, recall, stream=None):
     """Attention-mass recall [B][H_q] of the last decode step (n), per query head."""
-    _check("ckv_step_recall", lib().ckv_step_recall(ctx, _ptr(q), _ptr(K), n, _ptr(recall), _stream(stream)))
+    _check("ckv_step_recall", lib().ckv_step_recall(ctx, _dev(q), _dev(K), n, _dev(recall), _stream(stream)))
 
 
 def ckv_dense_decode(ctx, q, K, V, n, out, lse=None, stream=None):
     """Dense decode attention over [0, n): out [B][H_q][D], lse [B][H_q] (optional)."""
-    _check("ckv_dense_decode", lib().ckv_dense_decode(ctx, _ptr(q), _ptr(K), _ptr(V), n, _ptr(out), _ptr(lse),
+    _check("ckv_dense_decode", lib().ckv_dense_decode(ctx, _dev(q), _dev(K), _dev(V), n, _dev(out), _dev(lse),
                                                       _stream(stream)))
 
 

@@ -108,3 +108,43 @@ def test_checkpoint_record_roundtrip():
         np.testing.assert_array_equal(getattr(t, f), getattr(s, f))
     with pytest.raises(ValueError):
         ckv_state.parse(b"\0" * 64)
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor on a machine without one (never dereferenced)."""
+    is_cuda = True
+
+    def data_ptr(self):
+        return 0x1000
+
+
+def test_binding_refuses_the_wrong_memory_kind():
+    # device arguments take CUDA tensors only, host arguments never a CUDA
+    # tensor: both are refused before the C call, so no kernel is handed a
+    # host address
+    import torch
+    dev = _FakeCudaTensor()
+    host = np.zeros(4, np.float32)
+    calls = [
+        lambda: ckv.ckv_decode_step(None, host, dev, dev, 1, dev),                 # numpy for q
+        lambda: ckv.ckv_decode_step(None, dev, torch.zeros(4), dev, 1, dev),       # CPU tensor for K
+        lambda: ckv.ckv_assign_update(None, host, 1),
+        lambda: ckv.ckv_decode_host(None, dev, host, host, dev, dev, 1, host),     # CUDA tensor for q_host
+        lambda: ckv.ckv_decode_host(None, host, host, host, host, dev, 1, host),   # numpy for K
+        lambda: ckv.ckv_get_step_debug(None, n_sel=dev),
+        lambda: ckv.ckv_init_communities(None, host, 1, 1, dev, 4),                # host labels said on device
+        lambda: ckv.ckv_init_communities(None, dev, 0, 1, dev, 4),                 # device labels said on host
+        lambda: ckv.ckv_build_graph(1, 8, 128, 4, 8, ckv.CKV_BF16, host, dev, dev, dev, dev),
+        lambda: ckv.ckv_modularity(4, dev, dev, dev, host, 1, 1.0, dev),
+        lambda: ckv.ckv_step_recall(None, dev, dev, 1, host),
+        lambda: ckv.ckv_dense_decode(None, dev, dev, dev, 1, dev, host),
+        lambda: ckv.ckv_refresh(None, host, 1.0),
+        lambda: ckv.ckv_graph_modularity(None, 1.0, dev),
+    ]
+    for fn in calls:
+        with pytest.raises(TypeError):
+            fn()
+    # the right kinds reach the C entry point, which rejects the null context
+    with pytest.raises(ckv.CkvError) as e:
+        ckv.ckv_decode_step(None, dev, dev, dev, 1, dev)
+    assert e.value.status == ckv.CKV_ERR_INVALID_ARG
