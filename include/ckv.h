@@ -147,8 +147,9 @@ ckv_status ckv_build_graph_grouped(int n_kv_heads, int group, int n, int head_di
  * Output: labels_host [n], community ids 0..C-1 by first appearance, and
  * *n_communities = C; the labels feed ckv_init_communities (sinks' labels
  * are ignored there).  Synchronous, host only.
- * Errors: CKV_ERR_INVALID_ARG (n < 1, gamma <= 0, row_ptr not monotone,
- * a column outside [0, n), a negative or NaN weight), CKV_ERR_OOM. */
+ * Errors: CKV_ERR_INVALID_ARG (n < 1, gamma not finite and positive,
+ * row_ptr not monotone, a column outside [0, n), a weight not finite and
+ * non-negative), CKV_ERR_OOM. */
 ckv_status ckv_leiden(int n, const int64_t* row_ptr_host, const int32_t* col_host, const float* w_host,
                       double gamma, int32_t* labels_host, int* n_communities);
 
@@ -174,8 +175,8 @@ ckv_status ckv_modularity(int n, const int64_t* row_ptr, const int32_t* col, con
  * (graph 0's count, the stride of every graph).  Allowed right after
  * ckv_init_communities(..., n) and before any decode step (n must be the
  * init's n).  Synchronous, host only.
- * Errors: CKV_ERR_INVALID_ARG (layout, a column outside [0, n), a negative
- * weight), CKV_ERR_STATE. */
+ * Errors: CKV_ERR_INVALID_ARG (layout, a column outside [0, n), a weight
+ * not finite and non-negative), CKV_ERR_STATE. */
 ckv_status ckv_set_token_graph(ckv_ctx* ctx, const int64_t* row_ptr_host, const int32_t* col_host,
                                const float* w_host, int n);
 

@@ -7,6 +7,7 @@
 // used for end-to-end timing.  Every step of the method runs in the CUDA
 // kernels of k_decode.cu, k_init.cu and k_prefill.cu.
 #include <cuda_runtime.h>
+#include <float.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -62,6 +63,11 @@ struct ckv_ctx {
 namespace {
 
 constexpr uint32_t kMagic = 0x31564B43u;   // "CKV1"
+
+// a resolution is a finite positive number; an edge weight a finite
+// non-negative one (NaN fails both comparisons)
+bool valid_gamma(double g) { return g > 0.0 && g <= DBL_MAX; }
+bool valid_weight(float w) { return w >= 0.0f && w <= FLT_MAX; }
 
 ckv_status cuda_status(cudaError_t e)
 {
@@ -773,14 +779,14 @@ CKV_API ckv_status ckv_build_graph(int n_heads, int n, int head_dim, int n_sinks
 CKV_API ckv_status ckv_leiden(int n, const int64_t* row_ptr_host, const int32_t* col_host, const float* w_host,
                               double gamma, int32_t* labels_host, int* n_communities)
 {
-    if (n < 1 || !row_ptr_host || !labels_host || !n_communities || !(gamma > 0.0)) return CKV_ERR_INVALID_ARG;
+    if (n < 1 || !row_ptr_host || !labels_host || !n_communities || !valid_gamma(gamma)) return CKV_ERR_INVALID_ARG;
     if (row_ptr_host[0] != 0) return CKV_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i)
         if (row_ptr_host[i + 1] < row_ptr_host[i]) return CKV_ERR_INVALID_ARG;
     const int64_t E = row_ptr_host[n];
     if (E > 0 && (!col_host || !w_host)) return CKV_ERR_INVALID_ARG;
     for (int64_t e = 0; e < E; ++e)
-        if (col_host[e] < 0 || col_host[e] >= n || !(w_host[e] >= 0.0f)) return CKV_ERR_INVALID_ARG;
+        if (col_host[e] < 0 || col_host[e] >= n || !valid_weight(w_host[e])) return CKV_ERR_INVALID_ARG;
     try {
         *n_communities = ckv::leiden_partition(n, row_ptr_host, col_host, w_host, gamma, 64, labels_host);
     } catch (...) {
@@ -798,7 +804,7 @@ CKV_API ckv_status ckv_modularity(int n, const int64_t* row_ptr, const int32_t* 
                                   const int32_t* labels, int n_communities, double gamma, void* workspace,
                                   double* q_host, void* stream)
 {
-    if (n < 1 || n_communities < 1 || !row_ptr || !labels || !workspace || !q_host || !(gamma > 0.0))
+    if (n < 1 || n_communities < 1 || !row_ptr || !labels || !workspace || !q_host || !valid_gamma(gamma))
         return CKV_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) & 7) return CKV_ERR_INVALID_ARG;
     cudaPointerAttributes a;
@@ -834,7 +840,7 @@ CKV_API ckv_status ckv_set_token_graph(ckv_ctx* x, const int64_t* row_ptr_host, 
         const int32_t* col = col_host + (size_t)g * E;
         const float* w = w_host + (size_t)g * E;
         for (int64_t e = 0; e < rp[n]; ++e)
-            if (col[e] < 0 || col[e] >= n || !(w[e] >= 0.0f)) return CKV_ERR_INVALID_ARG;
+            if (col[e] < 0 || col[e] >= n || !valid_weight(w[e])) return CKV_ERR_INVALID_ARG;
         tg[(size_t)g].rp.assign(rp, rp + n + 1);
         tg[(size_t)g].col.assign(col, col + rp[n]);
         tg[(size_t)g].w.assign(w, w + rp[n]);
@@ -894,7 +900,7 @@ CKV_API ckv_status ckv_refresh(ckv_ctx* x, const void* K, double gamma, int32_t*
 {
     ckv_status cs = check_ctx(x);
     if (cs != CKV_OK) return cs;
-    if (!K || !(gamma > 0.0)) return CKV_ERR_INVALID_ARG;
+    if (!K || !valid_gamma(gamma)) return CKV_ERR_INVALID_ARG;
     if (!x->initialized || x->pending || x->tg.empty() || x->tg_rows != x->d.n_init) return CKV_ERR_STATE;
     CKV_CUDA(cudaSetDevice(x->cfg.device));
     CKV_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
@@ -948,7 +954,7 @@ CKV_API ckv_status ckv_graph_modularity(ckv_ctx* x, double gamma, double* q_host
 {
     ckv_status cs = check_ctx(x);
     if (cs != CKV_OK) return cs;
-    if (!q_host || !(gamma > 0.0)) return CKV_ERR_INVALID_ARG;
+    if (!q_host || !valid_gamma(gamma)) return CKV_ERR_INVALID_ARG;
     if (!x->initialized || x->pending || x->tg.empty() || x->tg_rows != x->d.n_init) return CKV_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     CKV_CUDA(cudaSetDevice(x->cfg.device));

@@ -99,7 +99,10 @@ def test_arguments_checked():
                  (2, rp, np.array([0], np.int32), np.array([1.0], np.float32), 0.0),      # gamma
                  (2, np.array([0, 2, 1], np.int64), np.array([0, 1], np.int32),
                   np.array([1.0, 1.0], np.float32), 1.0),                                 # row_ptr not monotone
-                 (2, rp, np.array([0], np.int32), np.array([np.nan], np.float32), 1.0)):  # NaN weight
+                 (2, rp, np.array([0], np.int32), np.array([np.nan], np.float32), 1.0),   # NaN weight
+                 (2, rp, np.array([0], np.int32), np.array([np.inf], np.float32), 1.0),   # infinite weight
+                 (2, rp, np.array([0], np.int32), np.array([1.0], np.float32), np.inf),   # infinite gamma
+                 (2, rp, np.array([0], np.int32), np.array([1.0], np.float32), np.nan)):  # NaN gamma
         with pytest.raises(ckv.CkvError) as e:
             ckv.ckv_leiden(*args, lab)
         assert e.value.status == ckv.CKV_ERR_INVALID_ARG
