@@ -122,3 +122,12 @@ def test_binding_checks_host_arrays():
         ckv.ckv_leiden(2, rp, col, w, 1.0, np.zeros(2, np.int64))                  # wrong labels dtype
     with pytest.raises(ValueError):
         ckv.ckv_leiden(3, rp, col, w, 1.0, np.zeros(3, np.int32))                  # row_ptr too short
+
+
+def test_two_triangles(oracle_lib):
+    # the oracle's closed-form case: the library finds the same two triangles
+    rp = np.array([0, 0, 1, 3, 4, 5, 7], np.int64)
+    col = np.array([0, 0, 1, 2, 3, 3, 4], np.int32)
+    w = np.ones(7, np.float32)
+    lab, C = _lib_leiden(rp, col, w, 6, 1.0)
+    assert C == 2 and list(lab) == [0, 0, 0, 1, 1, 1]

@@ -151,3 +151,18 @@ def test_edge_cases(oracle_lib):
     labels, C = oracle.leiden(rp, col, w, 4)
     assert C == 3 and labels[1] == labels[2] and len({labels[0], labels[1], labels[3]}) == 3
     assert oracle.modularity(rp, col, w, labels) == pytest.approx(0.0, abs=1e-12)  # one edge inside: 1 - 1
+
+
+def test_two_triangles_closed_form(oracle_lib):
+    # two triangles {0,1,2} and {3,4,5} joined by the edge 2-3, unit weights:
+    # m = 7; each triangle holds 3 edges and a degree sum of 7, so
+    # Q = 2 * (3/7 - (7/14)^2) = 5/14 at gamma = 1, and at gamma:
+    # Q = 6/7 - gamma / 2
+    edges = [(1, 0, 1.0), (2, 0, 1.0), (2, 1, 1.0), (3, 2, 1.0), (4, 3, 1.0), (5, 3, 1.0), (5, 4, 1.0)]
+    rp, col, w = _csr(6, edges)
+    labels, C = oracle.leiden(rp, col, w, 6, 1.0)
+    assert C == 2 and list(labels) == [0, 0, 0, 1, 1, 1]
+    assert oracle.modularity(rp, col, w, labels) == pytest.approx(5 / 14, abs=1e-12)
+    assert oracle.modularity(rp, col, w, labels, 0.5) == pytest.approx(6 / 7 - 0.25, abs=1e-12)
+    # everything in one community: Q = 1 - gamma
+    assert oracle.modularity(rp, col, w, np.zeros(6, np.int32)) == pytest.approx(0.0, abs=1e-12)
