@@ -23,6 +23,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <utility>
 #include <vector>
 
 #include "leiden.h"
@@ -40,30 +41,69 @@ struct Adj {
     std::vector<double> k;       // degree: sum of wt + 2 loop
 };
 
-struct Half {                    // one endpoint's view of an edge before merging
-    int32_t to;
-    int64_t order;
-    double w;
+// Half-edges of every node, grouped by node: node v's are he[hoff[v] ..
+// hoff[v + 1]) in the order they were added (their `order`), so a stable
+// sort of a group by neighbour gives the (neighbour, order) order.
+struct Halves {
+    std::vector<int64_t> hoff;   // [n + 1]
+    std::vector<int32_t> to;
+    std::vector<double> w;
 };
 
-// merges each node's half-edges (sorted by (to, order)) into adjacency lists
-Adj merge_halves(int n, std::vector<std::vector<Half>>& halves, const std::vector<double>& loop)
+// Collects half-edges in two passes: `emit(sink)` calls sink(node, to, w) for
+// every half-edge in increasing order, once to count and once to place.
+template <typename Emit>
+Halves collect_halves(int n, Emit emit)
+{
+    Halves h;
+    h.hoff.assign((size_t)n + 1, 0);
+    emit([&](int a, int32_t, double) { ++h.hoff[(size_t)a + 1]; });
+    for (int v = 0; v < n; ++v) h.hoff[(size_t)v + 1] += h.hoff[(size_t)v];
+    h.to.resize((size_t)h.hoff[(size_t)n]);
+    h.w.resize((size_t)h.hoff[(size_t)n]);
+    std::vector<int64_t> pos(h.hoff.begin(), h.hoff.end() - 1);
+    emit([&](int a, int32_t b, double x) {
+        const int64_t p = pos[(size_t)a]++;
+        h.to[(size_t)p] = b;
+        h.w[(size_t)p] = x;
+    });
+    return h;
+}
+
+// merges each node's half-edges, summed in (neighbour, order) order, into
+// adjacency lists
+Adj merge_halves(int n, const Halves& h, const std::vector<double>& loop)
 {
     Adj a;
     a.n = n;
     a.off.assign((size_t)n + 1, 0);
     a.loop = loop;
     a.k.assign((size_t)n, 0.0);
+    a.to.reserve(h.to.size());
+    a.wt.reserve(h.to.size());
+    // (neighbour, position in the group) of each half-edge: unique keys, so
+    // any sort by them is the stable sort by neighbour
+    std::vector<std::pair<int32_t, int32_t>> key;
     for (int v = 0; v < n; ++v) {
-        auto& h = halves[(size_t)v];
-        std::sort(h.begin(), h.end(), [](const Half& x, const Half& y) {
-            return x.to != y.to ? x.to < y.to : x.order < y.order;
-        });
+        const int64_t b = h.hoff[(size_t)v], e = h.hoff[(size_t)v + 1];
+        const size_t d = (size_t)(e - b);
+        key.resize(d);
+        for (size_t i = 0; i < d; ++i) key[i] = {h.to[(size_t)b + i], (int32_t)i};
+        if (d <= 32) {
+            for (size_t i = 1; i < d; ++i) {   // insertion sort (already ordered by position)
+                const auto x = key[i];
+                size_t j = i;
+                for (; j > 0 && key[j - 1].first > x.first; --j) key[j] = key[j - 1];
+                key[j] = x;
+            }
+        } else {
+            std::sort(key.begin(), key.end());
+        }
         size_t i = 0;
-        while (i < h.size()) {
+        while (i < d) {
             double s = 0.0;
-            const int32_t t = h[i].to;
-            for (; i < h.size() && h[i].to == t; ++i) s += h[i].w;
+            const int32_t t = key[i].first;
+            for (; i < d && key[i].first == t; ++i) s += h.w[(size_t)b + (size_t)key[i].second];
             a.to.push_back(t);
             a.wt.push_back(s);
         }
@@ -79,19 +119,21 @@ Adj merge_halves(int n, std::vector<std::vector<Half>>& halves, const std::vecto
 
 Adj from_topk(int n, const int64_t* rp, const int32_t* col, const float* w)
 {
-    std::vector<std::vector<Half>> halves((size_t)n);
     std::vector<double> loop((size_t)n, 0.0);
-    int64_t order = 0;
     for (int i = 0; i < n; ++i)
-        for (int64_t e = rp[i]; e < rp[i + 1]; ++e) {
-            const int32_t j = col[e];
-            const double x = (double)w[e];
-            if (j == i) { loop[(size_t)i] += x; continue; }
-            halves[(size_t)i].push_back({j, order, x});
-            halves[(size_t)j].push_back({i, order, x});
-            ++order;
-        }
-    return merge_halves(n, halves, loop);
+        for (int64_t e = rp[i]; e < rp[i + 1]; ++e)
+            if (col[e] == i) loop[(size_t)i] += (double)w[e];
+    const Halves h = collect_halves(n, [&](auto&& sink) {
+        for (int i = 0; i < n; ++i)
+            for (int64_t e = rp[i]; e < rp[i + 1]; ++e) {
+                const int32_t j = col[e];
+                if (j == i) continue;
+                const double x = (double)w[e];
+                sink(i, j, x);
+                sink(j, i, x);
+            }
+    });
+    return merge_halves(n, h, loop);
 }
 
 // first-appearance renumbering; returns the number of communities
@@ -194,9 +236,11 @@ std::vector<int> refinement(const Adj& g, const std::vector<int>& comm, int nc, 
             if (comm[(size_t)g.to[(size_t)e]] == comm[(size_t)v]) s += g.wt[(size_t)e];
         ext[(size_t)v] = single_ext[(size_t)v] = s;
     }
-    std::vector<int> byc((size_t)n);
-    for (int v = 0; v < n; ++v) byc[(size_t)v] = v;
-    std::stable_sort(byc.begin(), byc.end(), [&](int a, int b) { return comm[(size_t)a] < comm[(size_t)b]; });
+    // nodes by community, ascending node order within one (a stable counting sort)
+    std::vector<int> byc((size_t)n), cstart((size_t)nc + 1, 0);
+    for (int v = 0; v < n; ++v) ++cstart[(size_t)comm[(size_t)v] + 1];
+    for (int c = 0; c < nc; ++c) cstart[(size_t)c + 1] += cstart[(size_t)c];
+    for (int v = 0; v < n; ++v) byc[(size_t)cstart[(size_t)comm[(size_t)v]]++] = v;
     NeighbourWeights nb((size_t)n);
     for (int v : byc) {
         const int c = comm[(size_t)v];
@@ -241,19 +285,23 @@ Adj coarsen(const Adj& g, const std::vector<int>& ref, std::vector<int>& node_of
     int nn = 0;
     for (int r = 0; r < n; ++r)
         if (present[(size_t)r]) node_of_ref[(size_t)r] = nn++;
-    std::vector<std::vector<Half>> halves((size_t)nn);
     std::vector<double> loop((size_t)nn, 0.0);
-    int64_t order = 0;
     for (int u = 0; u < n; ++u) {
         const int a = node_of_ref[(size_t)ref[(size_t)u]];
         loop[(size_t)a] += g.loop[(size_t)u];
-        for (int64_t e = g.off[(size_t)u]; e < g.off[(size_t)u + 1]; ++e) {
-            const int b = node_of_ref[(size_t)ref[(size_t)g.to[(size_t)e]]];
-            if (a == b) loop[(size_t)a] += g.wt[(size_t)e] / 2.0;
-            else halves[(size_t)a].push_back({b, order++, g.wt[(size_t)e]});
-        }
+        for (int64_t e = g.off[(size_t)u]; e < g.off[(size_t)u + 1]; ++e)
+            if (node_of_ref[(size_t)ref[(size_t)g.to[(size_t)e]]] == a) loop[(size_t)a] += g.wt[(size_t)e] / 2.0;
     }
-    Adj h = merge_halves(nn, halves, loop);
+    const Halves hv = collect_halves(nn, [&](auto&& sink) {
+        for (int u = 0; u < n; ++u) {
+            const int a = node_of_ref[(size_t)ref[(size_t)u]];
+            for (int64_t e = g.off[(size_t)u]; e < g.off[(size_t)u + 1]; ++e) {
+                const int b = node_of_ref[(size_t)ref[(size_t)g.to[(size_t)e]]];
+                if (a != b) sink(a, b, g.wt[(size_t)e]);
+            }
+        }
+    });
+    Adj h = merge_halves(nn, hv, loop);
     std::fill(h.k.begin(), h.k.end(), 0.0);
     for (int u = 0; u < n; ++u) h.k[(size_t)node_of_ref[(size_t)ref[(size_t)u]]] += g.k[(size_t)u];
     return h;

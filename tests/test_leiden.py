@@ -39,6 +39,19 @@ def test_same_labels_as_oracle_on_random_graphs(oracle_lib, seed, gamma):
     np.testing.assert_array_equal(lab, ref)
 
 
+@pytest.mark.parametrize("seed", range(3))
+def test_same_labels_on_larger_graphs(oracle_lib, seed):
+    # coarse levels whose nodes have hundreds of neighbours (the adjacency
+    # merge's sorted path as well as its insertion-sort path)
+    n = [3000, 6000, 12000][seed]
+    rp, col, w = _random_knn(n, 8, 100 + seed)
+    for gamma in (0.7, 1.0):
+        lab, C = _lib_leiden(rp, col, w, n, gamma)
+        ref, Cr = oracle.leiden(rp, col, w, n, gamma)
+        assert C == Cr
+        np.testing.assert_array_equal(lab, ref)
+
+
 def test_same_labels_on_equal_weights(oracle_lib):
     # every weight 1: gains tie everywhere, so the tie rules decide
     rng = np.random.default_rng(3)
