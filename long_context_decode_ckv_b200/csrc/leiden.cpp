@@ -41,9 +41,8 @@ struct Adj {
     std::vector<double> k;       // degree: sum of wt + 2 loop
 };
 
-// Half-edges of every node, grouped by node: node v's are he[hoff[v] ..
-// hoff[v + 1]) in the order they were added (their `order`), so a stable
-// sort of a group by neighbour gives the (neighbour, order) order.
+// Half-edges of every node, grouped by node: node v's are [hoff[v],
+// hoff[v + 1]) in the order they were emitted.
 struct Halves {
     std::vector<int64_t> hoff;   // [n + 1]
     std::vector<int32_t> to;
@@ -70,44 +69,64 @@ Halves collect_halves(int n, Emit emit)
     return h;
 }
 
-// merges each node's half-edges, summed in (neighbour, order) order, into
-// adjacency lists
-Adj merge_halves(int n, const Halves& h, const std::vector<double>& loop)
+// Adjacency lists from each node's half-edges: each(v, add) calls add(to, w)
+// for node v's half-edges in their order.  A neighbour's weights are summed
+// in that order (the same sums as summing after a stable sort by
+// neighbour), and the distinct (node, neighbour) pairs are put in ascending
+// neighbour order by two counting-sort transpositions: node -> neighbour
+// lists scattered by neighbour (nodes ascending), then back.
+template <typename Each>
+Adj merge_adj(int n, Each each, const std::vector<double>& loop)
 {
     Adj a;
     a.n = n;
-    a.off.assign((size_t)n + 1, 0);
     a.loop = loop;
     a.k.assign((size_t)n, 0.0);
-    a.to.reserve(h.to.size());
-    a.wt.reserve(h.to.size());
-    // (neighbour, position in the group) of each half-edge: unique keys, so
-    // any sort by them is the stable sort by neighbour
-    std::vector<std::pair<int32_t, int32_t>> key;
+    std::vector<int32_t> slot((size_t)n, -1);
+    std::vector<int64_t> uoff((size_t)n + 1, 0);
+    std::vector<int32_t> uto;
+    std::vector<double> uw;
     for (int v = 0; v < n; ++v) {
-        const int64_t b = h.hoff[(size_t)v], e = h.hoff[(size_t)v + 1];
-        const size_t d = (size_t)(e - b);
-        key.resize(d);
-        for (size_t i = 0; i < d; ++i) key[i] = {h.to[(size_t)b + i], (int32_t)i};
-        if (d <= 32) {
-            for (size_t i = 1; i < d; ++i) {   // insertion sort (already ordered by position)
-                const auto x = key[i];
-                size_t j = i;
-                for (; j > 0 && key[j - 1].first > x.first; --j) key[j] = key[j - 1];
-                key[j] = x;
+        const int64_t u0 = (int64_t)uto.size();
+        each(v, [&](int32_t t, double x) {
+            if (slot[(size_t)t] < 0) {
+                slot[(size_t)t] = (int32_t)(uto.size() - (size_t)u0);
+                uto.push_back(t);
+                uw.push_back(0.0);
             }
-        } else {
-            std::sort(key.begin(), key.end());
-        }
-        size_t i = 0;
-        while (i < d) {
-            double s = 0.0;
-            const int32_t t = key[i].first;
-            for (; i < d && key[i].first == t; ++i) s += h.w[(size_t)b + (size_t)key[i].second];
-            a.to.push_back(t);
-            a.wt.push_back(s);
-        }
-        a.off[(size_t)v + 1] = (int64_t)a.to.size();
+            uw[(size_t)u0 + (size_t)slot[(size_t)t]] += x;
+        });
+        for (int64_t i = u0; i < (int64_t)uto.size(); ++i) slot[(size_t)uto[(size_t)i]] = -1;
+        uoff[(size_t)v + 1] = (int64_t)uto.size();
+    }
+    const size_t U = uto.size();
+    // transpose: by neighbour, nodes ascending
+    std::vector<int64_t> toff((size_t)n + 1, 0);
+    for (size_t i = 0; i < U; ++i) ++toff[(size_t)uto[i] + 1];
+    for (int v = 0; v < n; ++v) toff[(size_t)v + 1] += toff[(size_t)v];
+    std::vector<int32_t> tfrom(U);
+    std::vector<double> tw(U);
+    {
+        std::vector<int64_t> pos(toff.begin(), toff.end() - 1);
+        for (int v = 0; v < n; ++v)
+            for (int64_t i = uoff[(size_t)v]; i < uoff[(size_t)v + 1]; ++i) {
+                const int64_t p = pos[(size_t)uto[(size_t)i]]++;
+                tfrom[(size_t)p] = v;
+                tw[(size_t)p] = uw[(size_t)i];
+            }
+    }
+    // and back: every node's neighbours ascending
+    a.to.resize(U);
+    a.wt.resize(U);
+    a.off = uoff;
+    {
+        std::vector<int64_t> pos(uoff.begin(), uoff.end() - 1);
+        for (int t = 0; t < n; ++t)
+            for (int64_t i = toff[(size_t)t]; i < toff[(size_t)t + 1]; ++i) {
+                const int64_t p = pos[(size_t)tfrom[(size_t)i]]++;
+                a.to[(size_t)p] = t;
+                a.wt[(size_t)p] = tw[(size_t)i];
+            }
     }
     for (int v = 0; v < n; ++v) {
         double s = 0.0;
@@ -133,7 +152,9 @@ Adj from_topk(int n, const int64_t* rp, const int32_t* col, const float* w)
                 sink(j, i, x);
             }
     });
-    return merge_halves(n, h, loop);
+    return merge_adj(n, [&](int v, auto&& add) {
+        for (int64_t i = h.hoff[(size_t)v]; i < h.hoff[(size_t)v + 1]; ++i) add(h.to[(size_t)i], h.w[(size_t)i]);
+    }, loop);
 }
 
 // first-appearance renumbering; returns the number of communities
@@ -285,23 +306,34 @@ Adj coarsen(const Adj& g, const std::vector<int>& ref, std::vector<int>& node_of
     int nn = 0;
     for (int r = 0; r < n; ++r)
         if (present[(size_t)r]) node_of_ref[(size_t)r] = nn++;
-    std::vector<double> loop((size_t)nn, 0.0);
-    for (int u = 0; u < n; ++u) {
-        const int a = node_of_ref[(size_t)ref[(size_t)u]];
-        loop[(size_t)a] += g.loop[(size_t)u];
-        for (int64_t e = g.off[(size_t)u]; e < g.off[(size_t)u + 1]; ++e)
-            if (node_of_ref[(size_t)ref[(size_t)g.to[(size_t)e]]] == a) loop[(size_t)a] += g.wt[(size_t)e] / 2.0;
+    // coarse node of every node, and each coarse node's members ascending (a
+    // stable counting sort): a coarse node's half-edges are its members'
+    // edges in ascending member order, as they come in one pass over the nodes
+    std::vector<int> cn((size_t)n), mstart((size_t)nn + 1, 0), mem((size_t)n);
+    for (int u = 0; u < n; ++u) cn[(size_t)u] = node_of_ref[(size_t)ref[(size_t)u]];
+    for (int u = 0; u < n; ++u) ++mstart[(size_t)cn[(size_t)u] + 1];
+    for (int a = 0; a < nn; ++a) mstart[(size_t)a + 1] += mstart[(size_t)a];
+    {
+        std::vector<int> pos(mstart.begin(), mstart.end() - 1);
+        for (int u = 0; u < n; ++u) mem[(size_t)pos[(size_t)cn[(size_t)u]]++] = u;
     }
-    const Halves hv = collect_halves(nn, [&](auto&& sink) {
-        for (int u = 0; u < n; ++u) {
-            const int a = node_of_ref[(size_t)ref[(size_t)u]];
+    std::vector<double> loop((size_t)nn, 0.0);
+    for (int a = 0; a < nn; ++a)
+        for (int i = mstart[(size_t)a]; i < mstart[(size_t)a + 1]; ++i) {
+            const int u = mem[(size_t)i];
+            loop[(size_t)a] += g.loop[(size_t)u];
+            for (int64_t e = g.off[(size_t)u]; e < g.off[(size_t)u + 1]; ++e)
+                if (cn[(size_t)g.to[(size_t)e]] == a) loop[(size_t)a] += g.wt[(size_t)e] / 2.0;
+        }
+    Adj h = merge_adj(nn, [&](int a, auto&& add) {
+        for (int i = mstart[(size_t)a]; i < mstart[(size_t)a + 1]; ++i) {
+            const int u = mem[(size_t)i];
             for (int64_t e = g.off[(size_t)u]; e < g.off[(size_t)u + 1]; ++e) {
-                const int b = node_of_ref[(size_t)ref[(size_t)g.to[(size_t)e]]];
-                if (a != b) sink(a, b, g.wt[(size_t)e]);
+                const int b = cn[(size_t)g.to[(size_t)e]];
+                if (b != a) add(b, g.wt[(size_t)e]);
             }
         }
-    });
-    Adj h = merge_halves(nn, hv, loop);
+    }, loop);
     std::fill(h.k.begin(), h.k.end(), 0.0);
     for (int u = 0; u < n; ++u) h.k[(size_t)node_of_ref[(size_t)ref[(size_t)u]]] += g.k[(size_t)u];
     return h;
