@@ -89,6 +89,39 @@ def test_null_arguments_rejected(L):
     ckv.ckv_destroy(None)   # ignored
 
 
+def test_newer_entry_points_check_arguments_on_host(L):
+    # every check below runs before any device call
+    p = ctypes.c_void_p(16)
+    q = ctypes.c_double(0.0)
+    one = ctypes.c_double(1.0)
+    bad = ckv.CKV_ERR_INVALID_ARG
+    # query-group prefill graph: pointers, group (1, 2, 4 or 8 heads), kappa, bf16 only
+    assert L.ckv_build_graph_grouped(2, 4, 64, 128, 4, 8, ckv.CKV_BF16, None, None, None, None, None, None, None) == bad
+    assert L.ckv_build_graph_grouped(2, 3, 64, 128, 4, 8, ckv.CKV_BF16, p, p, p, p, p, p, None) == bad
+    assert L.ckv_build_graph_grouped(2, 4, 64, 128, 4, 0, ckv.CKV_BF16, p, p, p, p, p, p, None) == bad
+    assert L.ckv_build_graph_grouped(2, 4, 64, 128, 4, 8, ckv.CKV_F32, p, p, p, p, p, p, None) == bad
+    assert L.ckv_build_graph_grouped_workspace(0, 4, 64) == 0
+    # modularity: n, pointers, resolution
+    assert L.ckv_modularity(0, p, p, p, p, 1, one, p, ctypes.byref(q), None) == bad
+    assert L.ckv_modularity(4, None, p, p, p, 1, one, p, ctypes.byref(q), None) == bad
+    assert L.ckv_modularity(4, p, p, p, p, 1, ctypes.c_double(0.0), p, ctypes.byref(q), None) == bad
+    assert L.ckv_modularity(4, p, p, p, p, 1, ctypes.c_double(float("inf")), p, ctypes.byref(q), None) == bad
+    assert L.ckv_modularity_workspace(0) == 0
+    # calls on a context refuse a null one
+    assert L.ckv_step_recall(None, p, p, 1, p, None) == bad
+    assert L.ckv_dense_decode(None, p, p, p, 1, p, None, None) == bad
+    assert L.ckv_set_token_graph(None, p, p, p, 4) == bad
+    assert L.ckv_refresh(None, p, one, None, None) == bad
+    assert L.ckv_graph_modularity(None, one, ctypes.byref(q), None) == bad
+    assert L.ckv_init_communities(None, None, 0, 1, None, 4, None) == bad
+    assert L.ckv_decode_host(None, None, None, None, None, None, 1, None, None) == bad
+    assert L.ckv_get_step_debug(None, None, None, None, None, None, None, None) == bad
+    assert L.ckv_export_state(None, None, None) == bad
+    assert L.ckv_profile_begin(None) == bad
+    assert L.ckv_aux_bytes(None, None, None) == bad
+    assert L.ckv_attend_rows_static(None, p, p, p, 5, p, p, 4, p, None) == bad
+
+
 def test_checkpoint_record_roundtrip():
     rng = np.random.default_rng(0)
     G, Nc, D, S, kap, n_init, n_tok = 3, 5, 128, 4, 8, 40, 43
