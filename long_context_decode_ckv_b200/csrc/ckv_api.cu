@@ -877,6 +877,23 @@ cudaError_t fetch_decode_rows(ckv_ctx* x, std::vector<int32_t>& deg, std::vector
 }
 
 // graph g's token graph over [0, n_tok): the host rows, then the decode rows
+// the decode-time rows read back from the device are well formed: degrees
+// in [0, kappa], columns in [0, n_tok), finite non-negative weights (host
+// code indexes by them)
+bool valid_decode_rows(const ckv_ctx* x, const std::vector<int32_t>& deg, const std::vector<int32_t>& col,
+                       const std::vector<float>& w)
+{
+    const int kap = x->d.kappa;
+    for (size_t r = 0; r < deg.size(); ++r) {
+        if (deg[r] < 0 || deg[r] > kap) return false;
+        for (int k = 0; k < deg[r]; ++k) {
+            const size_t i = r * (size_t)kap + (size_t)k;
+            if (col[i] < 0 || col[i] >= x->n_tok || !valid_weight(w[i])) return false;
+        }
+    }
+    return true;
+}
+
 ckv_ctx::TokenGraph combined_graph(const ckv_ctx* x, int g, const std::vector<int32_t>& deg,
                                    const std::vector<int32_t>& col, const std::vector<float>& w)
 {
@@ -909,6 +926,7 @@ CKV_API ckv_status ckv_refresh(ckv_ctx* x, const void* K, double gamma, int32_t*
     std::vector<int32_t> deg, col;
     std::vector<float> w;
     CKV_CUDA(fetch_decode_rows(x, deg, col, w));
+    if (!valid_decode_rows(x, deg, col, w)) return CKV_ERR_STATE;
     const int G = x->d.G, n = x->n_tok;
     std::vector<ckv_ctx::TokenGraph> next((size_t)G);
     std::vector<int32_t> labels((size_t)G * n), counts((size_t)G, 0);
@@ -962,6 +980,7 @@ CKV_API ckv_status ckv_graph_modularity(ckv_ctx* x, double gamma, double* q_host
     std::vector<int32_t> deg, col;
     std::vector<float> w;
     CKV_CUDA(fetch_decode_rows(x, deg, col, w));
+    if (!valid_decode_rows(x, deg, col, w)) return CKV_ERR_STATE;
     const Dims& d = x->d;
     const int n = x->n_tok;
     std::vector<int32_t> lab((size_t)n);
