@@ -321,7 +321,11 @@ ckv_status ckv_profile_end(ckv_ctx* ctx, float* ms /* [4] */, int* steps);
  * n_tok = positions covered (sinks + assigned tokens).  Export: pass
  * host_buf = NULL to get the size in *bytes; otherwise *bytes is the
  * buffer's capacity on entry and the bytes written on return.  Import
- * validates the record against the context and replaces the state.
+ * validates the record against the context (dimensions; sizes summing to
+ * n_tok - S; every position in [S, n_tok) a member exactly once, ascending
+ * within its community; edge degrees in [0, kappa] and columns in
+ * [0, n_tok); finite centroids; finite non-negative edge weights) and
+ * replaces the state.
  * Both are synchronous.  Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no
  * state yet), CKV_ERR_OOM, CKV_ERR_CUDA. */
 ckv_status ckv_export_state(ckv_ctx* ctx, void* host_buf, size_t* bytes);

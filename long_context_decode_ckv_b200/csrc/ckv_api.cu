@@ -8,6 +8,7 @@
 // kernels of k_decode.cu, k_init.cu and k_prefill.cu.
 #include <cuda_runtime.h>
 #include <float.h>
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -704,12 +705,15 @@ CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t byt
         if (total != (int64_t)nmem) return CKV_ERR_INVALID_ARG;
         top[g] = (int32_t)o;
         memcpy(&mu[g * d.Nc * D], &mu_in[g * Nc * D], (size_t)Nc * D * 4);
+        for (size_t i = 0; i < (size_t)Nc * D; ++i)
+            if (!(std::fabs(mu_in[g * Nc * D + i]) <= FLT_MAX)) return CKV_ERR_INVALID_ARG;   // finite centroids
         for (size_t r = 0; r < rows; ++r) {
             const int32_t dg = deg_in[g * rows + r];
             if (dg < 0 || dg > d.kappa) return CKV_ERR_INVALID_ARG;
             for (int e = 0; e < dg; ++e) {
                 const int32_t c = col_in[(g * rows + r) * d.kappa + e];
-                if (c < 0 || c >= n_tok) return CKV_ERR_INVALID_ARG;
+                if (c < 0 || c >= n_tok || !valid_weight(w_in[(g * rows + r) * d.kappa + e]))
+                    return CKV_ERR_INVALID_ARG;
             }
         }
     }
