@@ -258,6 +258,23 @@ ckv_status ckv_decode_host(ckv_ctx* ctx, const void* q_host, const void* k_new_h
  * (CKV_OK if none). */
 ckv_status ckv_last_error(ckv_ctx* ctx);
 
+/* Kernel launches of one decode step (ckv_decode_step plus
+ * ckv_assign_update) of this context: 1 with the fused step kernel (the
+ * default), 3 when the environment variable CKV_STEP=split was set at
+ * ckv_create (scoring, selection, attention as separate kernels).  -1 for
+ * NULL. */
+int ckv_step_launches(const ckv_ctx* ctx);
+
+/* Failure detection: the bound of the fused step's one cross-CTA wait (an
+ * attention item waiting for its graph's selection), in polls of about
+ * 64 ns each; 0 restores the default (2^22 polls).  A wait that runs out
+ * stops the step and sets CKV_ERR_TIMEOUT in the error word (read by
+ * ckv_last_error); the context is then failed until ckv_init_communities()
+ * or ckv_import_state().  A limit of 1 poll makes any step whose selection
+ * is not already published time out, which is how the tests drive it.
+ * Errors: CKV_ERR_INVALID_ARG (NULL). */
+ckv_status ckv_set_wait_limit(ckv_ctx* ctx, unsigned polls);
+
 /* Read back the last completed step's decisions into host buffers (any may
  * be NULL).  n_sel [G]; sel [G][max_communities] (kept community ids of
  * each graph, ascending id); n_tok_sel [G] (member tokens kept); n_edges

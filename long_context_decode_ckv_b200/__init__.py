@@ -78,6 +78,10 @@ def lib() -> ctypes.CDLL:
     L.ckv_decode_host.argtypes = [P, P, P, P, P, P, I, P, P]
     L.ckv_last_error.restype = st
     L.ckv_last_error.argtypes = [P]
+    L.ckv_step_launches.restype = I
+    L.ckv_step_launches.argtypes = [P]
+    L.ckv_set_wait_limit.restype = st
+    L.ckv_set_wait_limit.argtypes = [P, ctypes.c_uint]
     L.ckv_get_step_debug.restype = st
     L.ckv_get_step_debug.argtypes = [P, P, P, P, P, P, P, P]
     L.ckv_profile_begin.restype = st
@@ -287,6 +291,14 @@ def ckv_decode_host(ctx, q_host, k_new_host, v_new_host, K, V, n, out_host, stre
 
 def ckv_last_error(ctx) -> int:
     return lib().ckv_last_error(ctx)
+
+
+def ckv_step_launches(ctx) -> int:
+    return lib().ckv_step_launches(ctx)
+
+
+def ckv_set_wait_limit(ctx, polls: int):
+    _check("ckv_set_wait_limit", lib().ckv_set_wait_limit(ctx, int(polls)))
 
 
 def ckv_get_step_debug(ctx, n_sel=None, sel=None, n_tok_sel=None, n_edges=None, edges=None,

@@ -301,6 +301,18 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     }
     d.nCTA = ckv::attend_grid(d, sms);
     if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
+    {   // the decode step: one fused kernel unless CKV_STEP=split (the
+        // three-kernel path: scoring, selection, attention)
+        const char* v = getenv("CKV_STEP");
+        d.fused = !(v && v[0] == 's');
+    }
+    d.api = ckv::step_api(d.S, d.budget);
+    d.spg = 1;
+    d.rows_given = 0;
+    d.rtok_stride = d.NM;
+    d.wait_polls = ckv::kStepWaitPolls;
+    if (ckv::prepare_step(d, sms, &d.nStep) != cudaSuccess || d.nStep < 2) { delete x; return CKV_ERR_CUDA; }
+    d.n_workers = std::min(std::min(d.G, ckv::kStepWorkers), d.nStep / 2);
     d.n_comm = 0;
     d.n_init = 0;
 
@@ -315,7 +327,7 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(pool, G * (size_t)d.P);
     ALLOC(pool_top, G);
     ALLOC(tok_comm, G * NM);
-    const size_t KC = d.nCTA, kap = d.kappa;
+    const size_t KC = std::max(d.nCTA, d.api), kap = d.kappa;
     ALLOC(score, G * Nc);
     ALLOC(sel, G * Nc);
     ALLOC(meta, G * ckv::M_COUNT);
@@ -330,8 +342,17 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(e_comm, G * kap);
     ALLOC(sel_ml, (size_t)d.B * d.Hq * 2);
     ALLOC(srange, G * 4);
+    ALLOC(step_ctr, 2);
+    ALLOC(gcnt, G * 4);
+    ALLOC(shist, G * ckv::step_hist_bins());
+    ALLOC(sel_row, G * 3 * (Nc + 1));
+    ALLOC(kinfo, G * Nc * 4);
     ALLOC(err, 1);
 #undef ALLOC
+    s.rows_T = nullptr;
+    if (e == cudaSuccess) e = cudaMemset(s.step_ctr, 0, 2 * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemset(s.gcnt, 0, G * 4 * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemset(s.shist, 0, G * ckv::step_hist_bins() * sizeof(unsigned));
     if (e == cudaSuccess) e = dalloc(x, &x->dense_part, ckv::dense_part_floats(d));
     if (e == cudaSuccess) e = dalloc(x, &x->dense_cnt, (size_t)d.B * d.Hkv);
     if (e == cudaSuccess) e = cudaMemset(x->dense_cnt, 0, (size_t)d.B * d.Hkv * sizeof(unsigned));
@@ -370,6 +391,7 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
     Dims& d = x->d;
     DevState& s = x->s;
     d.n_comm = n_communities;
+    d.spg = (n_communities + ckv::step_cpi() - 1) / ckv::step_cpi();
     d.n_init = n;
     const size_t G = d.G;
     const int32_t* dlabels = labels;
@@ -388,6 +410,9 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
     step(cudaMemsetAsync(s.ccap, 0, G * d.Nc * sizeof(int32_t), st));
     step(cudaMemsetAsync(s.tok_comm, 0xff, G * d.NM * sizeof(int32_t), st));
     step(cudaMemsetAsync(s.bar, 0, G * 2 * sizeof(unsigned), st));
+    step(cudaMemsetAsync(s.step_ctr, 0, 2 * sizeof(unsigned), st));
+    step(cudaMemsetAsync(s.gcnt, 0, G * 4 * sizeof(unsigned), st));
+    step(cudaMemsetAsync(s.shist, 0, G * ckv::step_hist_bins() * sizeof(unsigned), st));
     step(cudaMemsetAsync(s.mu, 0, G * d.Nc * ckv::kD * sizeof(float), st));
     step(reset_srange(x, st));
     step(ckv::launch_init_count(s, d, dlabels, n, st));
@@ -426,11 +451,17 @@ CKV_API ckv_status ckv_decode_step(ckv_ctx* x, const void* q, const void* K, con
     cudaStream_t st = (cudaStream_t)stream;
     CKV_CUDA(cudaSetDevice(x->cfg.device));
     CKV_CUDA(prof_mark(x, 0, st));
-    CKV_CUDA(ckv::launch_score(x->s, x->d, q, st));
-    CKV_CUDA(prof_mark(x, 1, st));
-    CKV_CUDA(ckv::launch_select(x->s, x->d, st));
-    CKV_CUDA(prof_mark(x, 2, st));
-    CKV_CUDA(ckv::launch_attend(x->s, x->d, q, K, V, n, out, st));
+    if (x->d.fused) {
+        CKV_CUDA(ckv::launch_step(x->s, x->d, q, K, V, n, out, st));
+        CKV_CUDA(prof_mark(x, 1, st));
+        CKV_CUDA(prof_mark(x, 2, st));
+    } else {
+        CKV_CUDA(ckv::launch_score(x->s, x->d, q, st));
+        CKV_CUDA(prof_mark(x, 1, st));
+        CKV_CUDA(ckv::launch_select(x->s, x->d, st));
+        CKV_CUDA(prof_mark(x, 2, st));
+        CKV_CUDA(ckv::launch_attend(x->s, x->d, q, K, V, n, out, st));
+    }
     CKV_CUDA(prof_mark(x, 3, st));
     x->pending = 1;
     x->pending_n = n;
@@ -526,6 +557,15 @@ CKV_API ckv_status ckv_last_error(ckv_ctx* x)
     ckv_status e = read_device_error(x);
     if (e != CKV_OK) x->sticky = e;
     return e;
+}
+
+CKV_API int ckv_step_launches(const ckv_ctx* x) { return x ? (x->d.fused ? 1 : 3) : -1; }
+
+CKV_API ckv_status ckv_set_wait_limit(ckv_ctx* x, unsigned polls)
+{
+    if (!x) return CKV_ERR_INVALID_ARG;
+    x->d.wait_polls = polls ? polls : ckv::kStepWaitPolls;
+    return CKV_OK;
 }
 
 CKV_API ckv_status ckv_profile_begin(ckv_ctx* x)
@@ -741,9 +781,13 @@ CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t byt
     }
     CKV_CUDA(cudaMemset(s.err, 0, sizeof(int)));
     CKV_CUDA(cudaMemset(s.bar, 0, G * 2 * sizeof(unsigned)));
+    CKV_CUDA(cudaMemset(s.step_ctr, 0, 2 * sizeof(unsigned)));
+    CKV_CUDA(cudaMemset(s.gcnt, 0, G * 4 * sizeof(unsigned)));
+    CKV_CUDA(cudaMemset(s.shist, 0, G * ckv::step_hist_bins() * sizeof(unsigned)));
     CKV_CUDA(reset_srange(x, 0));
     CKV_CUDA(cudaDeviceSynchronize());
     d.n_comm = Nc;
+    d.spg = (Nc + ckv::step_cpi() - 1) / ckv::step_cpi();
     d.n_init = n_init;
     x->n_tok = n_tok;
     x->pending = 0;

@@ -68,7 +68,16 @@ struct DevState {
     int32_t* e_comm;
     float* sel_ml;           // may be null (then the attention kernel does not write it)
     uint32_t* srange;        // [G][4] min and max score key of the non-empty communities, their total
-                             // size, pad: accumulated by k_score, read and reset by k_select
+                             // size, pad: accumulated by the scoring, read and reset by the selection
+    // fused step kernel (k_step.cu)
+    unsigned* step_ctr;      // [2] queue head and CTAs done; reset by the last CTA to leave
+    unsigned* gcnt;          // [G][4] score items done, selection done, attention items done, pad
+    unsigned* shist;         // [G][step_hist_bins()] sizes per coarse score bin, filled by the score
+                             // items, read and cleared by the selection
+    int32_t* sel_row;        // [G][3 (Nc + 1)] kept list (ids, row starts, segments) when it
+                             // does not fit shared memory
+    int32_t* kinfo;          // [G][Nc][4] each kept community's id, row start, size, segment start
+    const int32_t* rows_T;   // [G] kept rows of each graph when the rows are given (else null)
     int* err;                // sticky device error word (ckv_status)
 };
 
@@ -82,6 +91,15 @@ struct Dims {
     int fuse_assign;         // the attention kernel also assigns the new token and updates
     int att_aligned;         // attention CTAs split graph by graph (else the rows evenly)
     int pdl;                 // programmatic dependent launch: 0 off, 1 trigger at kernel start, 2 after the main work
+    // fused step kernel (k_step.cu)
+    int spg;                 // score items per graph
+    int api;                 // attention items per graph
+    int rows_given;          // attention over given rows: no scoring, selection, edges or update
+    unsigned wait_polls;     // polls of an attention item's wait for its graph's selection
+    int nStep;               // CTAs of the step grid (co-resident)
+    int rtok_stride;         // entries per graph of the kept-row list rtok (n_max, or the given rows' capacity)
+    int n_workers;           // CTAs of the step grid that run the selections and finishes
+    int fused;               // ckv_decode_step runs the fused kernel (else the three kernels)
 };
 
 // kernel launchers (k_decode.cu)
@@ -96,6 +114,17 @@ size_t select_smem_bytes(int n_comm, int budget);
 cudaError_t prepare_kernels(const Dims& d);
 int attend_grid(const Dims& d, int sms);
 constexpr int kMaxCommunities = 16384;   // k_select holds 16 of a graph's communities per thread
+
+// the fused step (k_step.cu): scoring, selection, attention, edges, vote
+// and update of every graph in one persistent cooperative launch
+int step_cpi();                                  // communities per score item
+int step_hist_bins();                            // coarse score bins per graph
+int step_api(int S, int rows);                   // attention items for up to `rows` kept rows
+cudaError_t prepare_step(const Dims& d, int sms, int* grid);
+cudaError_t launch_step(const DevState& s, const Dims& d, const void* q, const void* K, const void* V, int n,
+                        float* out, cudaStream_t st);
+constexpr unsigned kStepWaitPolls = 1u << 22;    // default bound of a cross-CTA wait (polls with 64 ns naps)
+constexpr int kStepWorkers = 16;                 // selection / finish CTAs of the step grid, at most
 
 // dense decode statistics over a whole cache (k_dense.cu): with V, the dense
 // attention output and log-sum-exp per query head; with sel_ml, the

@@ -4,19 +4,20 @@
 // Some hosts cannot call cudaMalloc where this runs: plugin-style
 // integrations (an inference engine's custom-op execute path, for example)
 // that forbid device allocation after set-up and hand the op no workspace.
-// For them ckv_attend_rows_static runs the library's gather-attention
-// kernel (the one ckv_decode_step uses) with its scratch -- row list,
-// logits, per-CTA softmax statistics and P.V partials, arrival counter,
-// edge ranking -- in the file-scope device array below instead of memory
-// from a context.
+// For them ckv_attend_rows_static runs the attention items of the library's
+// fused decode kernel (the gather, the tensor-core contractions and the
+// merge of the partials that ckv_decode_step uses) with its scratch -- the
+// row lists, per-item softmax statistics and P.V partials, the queue and
+// arrival counters -- in the file-scope device array below instead of
+// memory from a context.
 //
 // The array is kStaticScratchBytes per device and stays resident on every
 // GPU that loads the library until the process exits.  Every call shares
-// it: the call clears the counter and error word it needs, copies its row
-// list in, and launches on `stream`; calls whose work overlaps on the GPU
-// (different streams, or different host threads) race on it and must be
-// serialised by the caller.  The first call on a device looks up the
-// array's device address; make that first call before any stream capture.
+// it: the call clears the counters it needs, copies the row lists in, and
+// launches on `stream`; calls whose work overlaps on the GPU (different
+// streams, or different host threads) race on it and must be serialised by
+// the caller.  The first call on a device looks up the array's device
+// address and sets the kernel's launch attributes.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -34,26 +35,30 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
+struct DeviceSetup {
+    void* addr;     // device address of g_static_scratch
+    int sms;
+};
 std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices];   // device address of g_static_scratch, per device
-
-// Device address of the scratch array on `dev` (the current device).  The
-// host-side name g_static_scratch is only a stand-in; a kernel must get the
-// address returned by cudaGetSymbolAddress.
-cudaError_t scratch_address(int dev, void** out)
-{
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
-    return cudaSuccess;
-}
+DeviceSetup g_setup[kMaxDevices];
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Restores the caller's current device when the call returns.
+struct DeviceGuard {
+    int prev = -1;
+    cudaError_t enter(int dev)
+    {
+        cudaError_t e = cudaGetDevice(&prev);
+        if (e != cudaSuccess) { prev = -1; return e; }
+        return prev == dev ? cudaSuccess : cudaSetDevice(dev);
+    }
+    ~DeviceGuard()
+    {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
 
 }  // namespace
 
@@ -65,14 +70,20 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     if (!cfg || !q || !K || !V || !out || !rows_host || !n_rows_host) return CKV_ERR_INVALID_ARG;
     if (cfg->batch < 1 || cfg->n_q_heads < 1 || cfg->n_kv_heads < 1 || cfg->n_q_heads % cfg->n_kv_heads ||
         cfg->head_dim != kD || cfg->n_max < 1 || cfg->n_sinks < 0 || cfg->device < 0 ||
-        cfg->device >= kMaxDevices || (cfg->kv_dtype != CKV_F32 && cfg->kv_dtype != CKV_BF16) ||
+        (cfg->kv_dtype != CKV_F32 && cfg->kv_dtype != CKV_BF16) ||
         (cfg->mode != CKV_PER_HEAD && cfg->mode != CKV_QUERY_GROUP))
+        return CKV_ERR_INVALID_ARG;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || cfg->device >= ndev || cfg->device >= kMaxDevices)
         return CKV_ERR_INVALID_ARG;
     const int Gq = cfg->n_q_heads / cfg->n_kv_heads;
     const int HG = cfg->mode == CKV_QUERY_GROUP ? Gq : 1;
     if (HG != 1 && HG != 2 && HG != 4 && HG != 8) return CKV_ERR_INVALID_ARG;
     if (n < cfg->n_sinks + 1 || n > cfg->n_max || max_rows < 0) return CKV_ERR_INVALID_ARG;
-    const int G = cfg->mode == CKV_QUERY_GROUP ? cfg->batch * cfg->n_kv_heads : cfg->batch * cfg->n_q_heads;
+    const int64_t G64 = cfg->mode == CKV_QUERY_GROUP ? (int64_t)cfg->batch * cfg->n_kv_heads
+                                                     : (int64_t)cfg->batch * cfg->n_q_heads;
+    if (G64 > (1 << 20)) return CKV_ERR_INVALID_ARG;
+    const int G = (int)G64;
     // every row must be an ordinary past position: not a sink, not the new token
     for (int g = 0; g < G; ++g) {
         const int T = n_rows_host[g];
@@ -82,79 +93,72 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
             if (j < cfg->n_sinks || j >= n - 1) return CKV_ERR_INVALID_ARG;
         }
     }
-    int sms = 0;
-    cudaError_t e = cudaSetDevice(cfg->device);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, cfg->device);
-    void* base = nullptr;
-    if (e == cudaSuccess) e = scratch_address(cfg->device, &base);
-    if (e != cudaSuccess) return CKV_ERR_CUDA;
 
-    // one graph per launch, so the scratch holds a single graph's rows
     ckv::Dims d{};
-    d.B = 1;
-    d.Hkv = 1;
-    d.Hq = HG;
-    d.Gq = HG;
-    d.G = 1;
+    d.B = cfg->batch;
+    d.Hq = cfg->n_q_heads;
+    d.Hkv = cfg->n_kv_heads;
+    d.Gq = Gq;
+    d.G = G;
     d.HG = HG;
     d.NM = cfg->n_max;
     d.S = cfg->n_sinks;
-    d.kappa = 1;          // the kernel also ranks one edge; this call discards it
-    d.mode = CKV_QUERY_GROUP;
+    d.kappa = 1;
+    d.mode = cfg->mode;
     d.bf16 = cfg->kv_dtype == CKV_BF16;
-    const int grid = ckv::attend_grid(d, sms);
-    if (grid < 1) return CKV_ERR_CUDA;
-    // at most one CTA per 64 rows of the largest graph
-    const int64_t rows_max = (int64_t)d.S + max_rows + 1;
-    d.nCTA = (int)((rows_max + 63) / 64 < grid ? (rows_max + 63) / 64 : grid);
-    // scratch layout: meta | bar | err | edges | row list | logits | partials
-    const size_t KC = d.nCTA;
+    d.rows_given = 1;
+    d.rtok_stride = max_rows;
+    d.api = ckv::step_api(d.S, max_rows);
+    d.wait_polls = ckv::kStepWaitPolls;
+    // scratch layout: counters (queue head, CTAs done, error word, pad,
+    // graphs' arrivals) | kept-row counts | row lists | partials
+    const size_t A = (size_t)d.api;
     size_t off = 0;
-    const size_t o_meta = off;  off = align256(off + ckv::M_COUNT * 4);
-    const size_t o_bar = off;   off = align256(off + 2 * 4);
-    const size_t o_err = off;   off = align256(off + 4);
-    const size_t o_e = off;     off = align256(off + 3 * 4);
-    // (graph index 0 in every launch: the row list holds max_rows entries and
-    // the spill logits rows_max rows, whatever the cache length)
-    const size_t o_rtok = off;  off = align256(off + (size_t)max_rows * 4);
-    const size_t o_zrow = off;  off = align256(off + (size_t)rows_max * HG * 4);
-    const size_t o_pml = off;   off = align256(off + KC * HG * 2 * 4);
-    const size_t o_po = off;    off = align256(off + KC * HG * kD * 4);
-    if (off > kStaticScratchBytes) return CKV_ERR_CAPACITY;   // max_rows too large for the array
-    unsigned char* sb = static_cast<unsigned char*>(base);
+    const size_t o_ctr = off;   off = align256(off + (4 + 4 * (size_t)G) * 4);
+    const size_t o_rT = off;    off = align256(off + (size_t)G * 4);
+    const size_t o_rtok = off;  off = align256(off + (size_t)G * max_rows * 4);
+    const size_t o_pml = off;   off = align256(off + (size_t)G * A * HG * 2 * 4);
+    const size_t o_po = off;    off = align256(off + (size_t)G * A * HG * kD * 4);
+    if (off > kStaticScratchBytes) return CKV_ERR_CAPACITY;   // the rows and partials do not fit the array
+
+    DeviceGuard guard;
+    if (guard.enter(cfg->device) != cudaSuccess) return CKV_ERR_CUDA;
+    DeviceSetup su;
+    {
+        std::lock_guard<std::mutex> lock(g_setup_mutex);
+        DeviceSetup& ds = g_setup[cfg->device];
+        if (!ds.addr) {
+            // the host-side name g_static_scratch is only a stand-in: a
+            // kernel must be given the address this returns
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return CKV_ERR_CUDA;
+            if (cudaDeviceGetAttribute(&ds.sms, cudaDevAttrMultiProcessorCount, cfg->device) != cudaSuccess)
+                return CKV_ERR_CUDA;
+            ds.addr = p;
+        }
+        su = ds;
+    }
+    int grid = 0;
+    if (ckv::prepare_step(d, su.sms, &grid) != cudaSuccess || grid < 1) return CKV_ERR_CUDA;
+    d.nStep = grid;
+    unsigned char* sb = static_cast<unsigned char*>(su.addr);
     ckv::DevState s{};
-    s.meta = reinterpret_cast<int32_t*>(sb + o_meta);
-    s.bar = reinterpret_cast<unsigned int*>(sb + o_bar);
-    s.err = reinterpret_cast<int*>(sb + o_err);
-    s.e_tok = reinterpret_cast<int32_t*>(sb + o_e);
-    s.e_w = reinterpret_cast<float*>(sb + o_e + 4);
-    s.e_comm = reinterpret_cast<int32_t*>(sb + o_e + 8);
+    s.step_ctr = reinterpret_cast<unsigned*>(sb + o_ctr);
+    s.err = reinterpret_cast<int*>(sb + o_ctr + 8);
+    s.gcnt = reinterpret_cast<unsigned*>(sb + o_ctr + 16);
+    s.rows_T = reinterpret_cast<const int32_t*>(sb + o_rT);
     s.rtok = reinterpret_cast<int32_t*>(sb + o_rtok);
-    s.rcomm = s.rtok;     // community of a row: only read for the edges, which this call discards
-    s.zrow = reinterpret_cast<float*>(sb + o_zrow);
     s.part_ml = reinterpret_cast<float*>(sb + o_pml);
     s.part_o = reinterpret_cast<float*>(sb + o_po);
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t eb = d.bf16 ? 2 : 4;
-    for (int g = 0; g < G; ++g) {
-        int b, h0, kvh;
-        if (cfg->mode == CKV_QUERY_GROUP) { b = g / cfg->n_kv_heads; kvh = g % cfg->n_kv_heads; h0 = kvh * Gq; }
-        else { b = g / cfg->n_q_heads; h0 = g % cfg->n_q_heads; kvh = h0 / Gq; }
-        const int T = n_rows_host[g];
-        int32_t meta[ckv::M_COUNT] = {0};
-        meta[ckv::M_T] = T;
-        meta[ckv::M_ROWS] = d.S + T + 1;
-        const char* qg = static_cast<const char*>(q) + ((int64_t)b * cfg->n_q_heads + h0) * kD * eb;
-        const char* Kg = static_cast<const char*>(K) + ((int64_t)b * cfg->n_kv_heads + kvh) * cfg->n_max * kD * eb;
-        const char* Vg = static_cast<const char*>(V) + ((int64_t)b * cfg->n_kv_heads + kvh) * cfg->n_max * kD * eb;
-        float* og = out + ((int64_t)b * cfg->n_q_heads + h0) * kD;
-        e = cudaMemcpyAsync(s.meta, meta, sizeof meta, cudaMemcpyHostToDevice, st);
-        if (e == cudaSuccess && T > 0)
-            e = cudaMemcpyAsync(s.rtok, rows_host + (int64_t)g * max_rows, (size_t)T * 4, cudaMemcpyHostToDevice, st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(sb + o_bar, 0, 256 + 256, st);   // arrival counters, error word
-        if (e == cudaSuccess) e = ckv::launch_attend(s, d, qg, Kg, Vg, n, og, st);
-        if (e != cudaSuccess) return CKV_ERR_CUDA;
-    }
-    return CKV_OK;
+    cudaError_t e = cudaMemsetAsync(sb + o_ctr, 0, (4 + 4 * (size_t)G) * 4, st);
+    // host -> device copies straight from the caller's buffers (pageable
+    // memory is staged before these calls return)
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(sb + o_rT, n_rows_host, (size_t)G * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess && max_rows > 0)
+        e = cudaMemcpyAsync(sb + o_rtok, rows_host, (size_t)G * max_rows * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = ckv::launch_step(s, d, q, K, V, n, out, st);
+    return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
 }

@@ -270,7 +270,10 @@ def test_per_kernel_profile_eager_and_captured(captured):
         torch.cuda.synchronize()
         ms, n = ckv.ckv_profile_end(ctx)
         assert n == cfg.steps
-        assert all(m > 0.0 for m in ms) and sum(ms) < 1000.0 * n
+        # the fused step has one kernel: its time is ms[0], the selection
+        # and attention spans are then empty
+        timed = ms[:1] if ckv.ckv_step_launches(ctx) == 1 else ms[:3]
+        assert all(m > 0.0 for m in timed) and all(m >= 0.0 for m in ms) and sum(ms) < 1000.0 * n
         for i in steps:
             ckv.ckv_decode_step(ref_ctx, q[i], K, V, cfg.n0 + i + 1, ref)
             ckv.ckv_assign_update(ref_ctx, K, cfg.n0 + i + 1)
