@@ -259,9 +259,9 @@ ckv_status ckv_decode_host(ckv_ctx* ctx, const void* q_host, const void* k_new_h
 ckv_status ckv_last_error(ckv_ctx* ctx);
 
 /* Kernel launches of one decode step (ckv_decode_step plus
- * ckv_assign_update) of this context: 1 with the fused step kernel (the
- * default), 3 when the environment variable CKV_STEP=split was set at
- * ckv_create (scoring, selection, attention as separate kernels).  -1 for
+ * ckv_assign_update) of this context: 3 by default (scoring, selection,
+ * attention as separate kernels), 1 when the environment variable
+ * CKV_STEP=fused was set at ckv_create (one persistent kernel).  -1 for
  * NULL. */
 int ckv_step_launches(const ckv_ctx* ctx);
 

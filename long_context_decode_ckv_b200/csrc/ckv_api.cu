@@ -301,10 +301,10 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     }
     d.nCTA = ckv::attend_grid(d, sms);
     if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
-    {   // the decode step: one fused kernel unless CKV_STEP=split (the
-        // three-kernel path: scoring, selection, attention)
+    {   // the decode step: three kernels (scoring, selection, attention)
+        // unless CKV_STEP=fused (one persistent kernel)
         const char* v = getenv("CKV_STEP");
-        d.fused = !(v && v[0] == 's');
+        d.fused = v && v[0] == 'f';
     }
     d.api = ckv::step_api(d.S, d.budget);
     d.spg = 1;
