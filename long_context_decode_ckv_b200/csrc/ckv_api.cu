@@ -310,9 +310,14 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     d.spg = 1;
     d.rows_given = 0;
     d.rtok_stride = d.NM;
+    d.nsu = (d.Nc + 15) / 16;
     d.wait_polls = ckv::kStepWaitPolls;
     if (ckv::prepare_step(d, sms, &d.nStep) != cudaSuccess || d.nStep < 2) { delete x; return CKV_ERR_CUDA; }
-    d.n_workers = std::min(std::min(d.G, ckv::kStepWorkers), d.nStep / 2);
+    {   // worker CTAs of the fused step (CKV_STEP_WORKERS overrides the default, for measurements)
+        const char* v = getenv("CKV_STEP_WORKERS");
+        const int want = (v && atoi(v) > 0) ? atoi(v) : ckv::kStepWorkers;
+        d.n_workers = std::min(std::min(d.G, want), d.nStep / 2);
+    }
     d.n_comm = 0;
     d.n_init = 0;
 
@@ -347,6 +352,7 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     ALLOC(shist, G * ckv::step_hist_bins());
     ALLOC(sel_row, G * 3 * (Nc + 1));
     ALLOC(kinfo, G * Nc * 4);
+    ALLOC(smax, G * ((Nc + 15) / 16));
     ALLOC(err, 1);
 #undef ALLOC
     s.rows_T = nullptr;

@@ -77,6 +77,7 @@ struct DevState {
     int32_t* sel_row;        // [G][3 (Nc + 1)] kept list (ids, row starts, segments) when it
                              // does not fit shared memory
     int32_t* kinfo;          // [G][Nc][4] each kept community's id, row start, size, segment start
+    unsigned* smax;          // [G][nsu] each 16-community slot's largest score key (0: all empty)
     const int32_t* rows_T;   // [G] kept rows of each graph when the rows are given (else null)
     int* err;                // sticky device error word (ckv_status)
 };
@@ -99,6 +100,7 @@ struct Dims {
     int nStep;               // CTAs of the step grid (co-resident)
     int rtok_stride;         // entries per graph of the kept-row list rtok (n_max, or the given rows' capacity)
     int n_workers;           // CTAs of the step grid that run the selections and finishes
+    int nsu;                 // 16-community slots per graph (max_communities / 16, rounded up)
     int fused;               // ckv_decode_step runs the fused kernel (else the three kernels)
 };
 
@@ -124,7 +126,7 @@ cudaError_t prepare_step(const Dims& d, int sms, int* grid);
 cudaError_t launch_step(const DevState& s, const Dims& d, const void* q, const void* K, const void* V, int n,
                         float* out, cudaStream_t st);
 constexpr unsigned kStepWaitPolls = 1u << 22;    // default bound of a cross-CTA wait (polls with 64 ns naps)
-constexpr int kStepWorkers = 16;                 // selection / finish CTAs of the step grid, at most
+constexpr int kStepWorkers = 8;                  // selection / finish CTAs of the step grid, at most
 
 // dense decode statistics over a whole cache (k_dense.cu): with V, the dense
 // attention output and log-sum-exp per query head; with sel_ml, the

@@ -141,6 +141,8 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
     int grid = 0;
     if (ckv::prepare_step(d, su.sms, &grid) != cudaSuccess || grid < 1) return CKV_ERR_CUDA;
     d.nStep = grid;
+    d.n_workers = G < ckv::kStepWorkers ? G : ckv::kStepWorkers;
+    if (d.n_workers > grid / 2) d.n_workers = grid / 2;
     unsigned char* sb = static_cast<unsigned char*>(su.addr);
     ckv::DevState s{};
     s.step_ctr = reinterpret_cast<unsigned*>(sb + o_ctr);

@@ -50,11 +50,13 @@ namespace ckv {
 
 namespace {
 
-constexpr int kW = 4;                           // warps per CTA
-constexpr int kT = 32 * kW;                     // threads per CTA
+constexpr int kW = 4;                           // warps of a streaming half
+constexpr int kT = 32 * kW;                     // threads of a streaming half
+constexpr int kWW = 2 * kW;                     // warps of a CTA (a worker uses them all)
+constexpr int kWT = 32 * kWW;                   // threads of a CTA
 constexpr int kSlot = 8192;                     // bytes of one pipeline slot
 constexpr int kNSlot = 3;                       // slots per warp
-constexpr int kRing = kW * kNSlot * kSlot;      // the CTA's rings, 96 KB
+constexpr int kRing = kW * kNSlot * kSlot;      // a half's rings, 96 KB
 constexpr int kSubC = 16;                       // communities per score slot (8 KB)
 constexpr int kSubPW = 4;                       // score slots per warp and item
 constexpr int kCPI = kW * kSubPW * kSubC;       // communities per score item
@@ -65,23 +67,32 @@ constexpr int kCoarseShift = 20;                // coarse bin of a score: the to
 constexpr int kCoarse = 1 << (32 - kCoarseShift);
 
 struct Misc {
-    int item;                  // the CTA's next item (thread 0 -> all)
+    int item;                  // the half's next item (its thread 0 -> all)
     int flag;                  // a broadcast decision
     int abort[kW];             // per warp: a bounded wait ran out
     float sM[8], sL[8];        // finish: each head's max and 1 / sum
     int sflag[8];              // finish: the assignment's decisions
-    int scan_i[2 * kW];        // block scans
-    unsigned long long red_k[2 * kW];
+    int scan_i[4 * kWW];       // block scans (workers)
+    unsigned long long red_k[2 * kWW];
 };
 
-constexpr int kXS = 14464;                      // after the rings: the selection's bitmaps and lists
-constexpr int kOffX = kRing;
-constexpr int kOffTok = kOffX + kXS;
-constexpr int kOffBar = kOffTok + kW * kTokW * 4;
-constexpr int kOffMisc = kOffBar + ((kW * kNSlot * 8 + 127) / 128) * 128;
-constexpr int kSmemBytes = kOffMisc + ((int)sizeof(Misc) + 127) / 128 * 128;
-// two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
-static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs must fit one SM");
+// shared memory: two halves, each rings | row-token windows | mbarriers |
+// Misc.  A worker CTA uses half 0's rings for its staging and half 1's
+// rings for the selection's bitmaps and lists, with half 0's Misc.
+constexpr int kHOffTok = kRing;
+constexpr int kHOffBar = kHOffTok + kW * kTokW * 4;
+constexpr int kHOffMisc = kHOffBar + ((kW * kNSlot * 8 + 127) / 128) * 128;
+constexpr int kHalf = kHOffMisc + ((int)sizeof(Misc) + 127) / 128 * 128;
+constexpr int kSmemBytes = 2 * kHalf;
+constexpr int kOffX = kHalf;                    // the selection's bitmaps and lists (in half 1's rings)
+constexpr int kXS = kRing;
+static_assert(kSmemBytes <= 232448, "the CTA's shared memory must fit");
+
+// barrier of the calling thread's half (4 warps): named barrier 1 + half
+__device__ __forceinline__ void hsync()
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + (int)(threadIdx.x >> 7)), "r"(kT) : "memory");
+}
 
 template <bool BF16>
 __device__ __forceinline__ float elem(const void* p, int64_t i)
@@ -150,7 +161,7 @@ __device__ __forceinline__ int cta_excl(int x, int* scan, int* tot)
     __syncthreads();
     int before = 0, all = 0;
 #pragma unroll
-    for (int w = 0; w < kW; ++w) {
+    for (int w = 0; w < kWW; ++w) {
         const int v = scan[w];
         before += (w < warp) ? v : 0;
         all += v;
@@ -203,13 +214,15 @@ __device__ __forceinline__ void set_flag(unsigned* flag)
 // Every non-empty community also adds its size to bin (key >> 20) of the
 // graph's coarse histogram in global memory (key: the order-preserving bits
 // of its score, so the bins order the communities by score and need no
-// score range): the selection starts from it.
+// score range), and each slot publishes its largest key: the selection
+// starts from the histogram and looks only at slots that reach its
+// boundary.
 template <bool BF16>
 __device__ __forceinline__ void score_item(const DevState& s, const Dims& d, const void* __restrict__ q, int g,
                                            int p, unsigned char* smem, unsigned long long* bars, unsigned& fills,
                                            Misc& mi)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = (threadIdx.x >> 5) & (kW - 1);
     int b, h0, kvh;
     graph_heads(d, g, b, h0, kvh);
     unsigned char* ring = smem + warp * (kNSlot * kSlot);
@@ -263,10 +276,14 @@ __device__ __forceinline__ void score_item(const DevState& s, const Dims& d, con
             issue(j + kNSlot);
         }
         const float v = transpose_reduce<kSubC>(part, lane);   // lane 2r: community c0 + r
+        const bool live = (lane & 1) == 0 && row < rows && sz > 0;
         if ((lane & 1) == 0 && row < rows) {
             s.score[gi] = (sz > 0) ? v : -INFINITY;
             if (sz > 0) atomicAdd(hist + (ord_u(v + 0.0f) >> kCoarseShift), (unsigned)sz);
         }
+        // the slot's largest key (0: no non-empty community), for the selection
+        const unsigned smk = __reduce_max_sync(kFull, live ? ord_u(v + 0.0f) : 0u);
+        if (lane == 0) s.smax[(int64_t)g * d.nsu + c0 / kSubC] = smk;
     }
     if (j < nsub) {
         // a copy never completed: report it, and wait (bounded) for the
@@ -292,7 +309,7 @@ __device__ __forceinline__ void score_item(const DevState& s, const Dims& d, con
 constexpr int kSelCache = 8192;    // communities staged in shared memory (the rest read from L2)
 constexpr int kSelB = 1024;        // bins of a refinement pass
 constexpr int kSelCap = 256;       // boundary communities ranked exactly
-constexpr int kSelCapW = 128;      // boundary communities each warp lists
+constexpr int kSelCapW = 64;       // boundary communities each warp lists
 constexpr int kKeepCap = (kSelCache - 1) / 3;   // kept-list entries in the scores' bytes
 
 struct SelSmem {                   // in the rings
@@ -303,24 +320,25 @@ struct SelSmem {                   // in the rings
 static_assert(sizeof(SelSmem) <= kRing, "selection staging must fit the rings");
 struct SelX {                      // in the region after the rings
     int hist[kSelB];
-    unsigned long long wkey[kW * kSelCapW];    // boundary candidates: per warp, or (refinement) flat
-    int ww[kW * kSelCapW];
+    unsigned long long wkey[kWW * kSelCapW];    // boundary candidates: per warp, or (refinement) flat
+    int ww[kWW * kSelCapW];
     unsigned keep[kMaxCommunities / 32];       // kept bitmap
     unsigned cand[kMaxCommunities / 32];       // still-a-candidate bitmap
-    int nw[kW];                                // candidates each warp listed
+    int nw[kWW];                                // candidates each warp listed
     int n_cand, b_bin, b_above;
 };
-static_assert(kW * kSelCapW >= kSelCap, "the flat candidate list must fit");
+static_assert(kWW * kSelCapW >= kSelCap, "the flat candidate list must fit");
+static_assert(sizeof(SelX) <= kXS, "the selection's lists must fit half 1's rings");
 
-// Boundary of a histogram of NB bins held top-first, PB = NB / kT bins per
+// Boundary of a histogram of NB bins held top-first, PB = NB / kWT bins per
 // thread (thread t: bins NB-1-PB t .. NB-PB(t+1)): the bin where `above`
 // plus the sizes summed from the top first exceeds the budget, and the sizes
-// above it.  The caller guarantees above plus the whole histogram exceeds
-// the budget.
+// above it, set only when above plus the whole histogram exceeds the
+// budget.  Returns the histogram's total.
 template <int PB>
-__device__ __forceinline__ void sel_boundary(const int (&loc)[PB], SelX& x, Misc& mi, int above, int budget)
+__device__ __forceinline__ int sel_boundary(const int (&loc)[PB], SelX& x, Misc& mi, int above, int budget)
 {
-    constexpr int NB = PB * kT;
+    constexpr int NB = PB * kWT;
     const int t = threadIdx.x;
     int tsum = 0;
 #pragma unroll
@@ -336,6 +354,7 @@ __device__ __forceinline__ void sel_boundary(const int (&loc)[PB], SelX& x, Misc
         acc += loc[k];
     }
     __syncthreads();
+    return tot;   // the histogram's total
 }
 
 __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& sm, SelX& x, Misc& mi)
@@ -353,7 +372,7 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
     // ---- round 1: the coarse histogram (this thread's 32 bins, top first;
     // cleared for the next step) and the staged scores, sizes and segment
     // starts (16-byte copies when each graph's rows are 16-byte aligned)
-    constexpr int PB = kCoarse / kT;
+    constexpr int PB = kCoarse / kWT;
     int loc[PB];
     {
         uint4* gh = reinterpret_cast<uint4*>(s.shist + (int64_t)g * kCoarse) + (kCoarse - PB * (tid + 1)) / 4;
@@ -362,13 +381,13 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
         for (int i = 0; i < PB / 4; ++i) h4[i] = __ldcg(gh + i);
         if ((d.Nc & 3) == 0) {
             const int nch = (NS + 3) / 4;
-            for (int i = tid; i < nch; i += kT) {
+            for (int i = tid; i < nch; i += kWT) {
                 cp_async16(sm.cs + 4 * i, gsc + 4 * i);
                 cp_async16(sm.cz + 4 * i, gsz + 4 * i);
                 cp_async16(sm.co + 4 * i, gco + 4 * i);
             }
         } else {
-            for (int c = tid; c < NS; c += kT) {
+            for (int c = tid; c < NS; c += kWT) {
                 cp_async4(sm.cs + c, gsc + c);
                 cp_async4(sm.cz + c, gsz + c);
                 cp_async4(sm.co + c, gco + c);
@@ -385,20 +404,23 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
             loc[PB - 4 - 4 * i] = (int)h4[i].w;
         }
     }
-    for (int i = tid; i < NWd; i += kT) x.cand[i] = 0u;
-    // ---- the total size decides whether everything fits; else the
-    // boundary bin
-    int wsum;
-    {
-        int t4 = 0;
+    // the slots' largest keys (this thread: slots tid + kWT j)
+    constexpr int SJ = (kMaxCommunities / kSubC + kWT - 1) / kWT;
+    static_assert(SJ * kWW <= 4 * kWW && kMaxCommunities / kSubC <= kSelB, "live-slot scan and list sizes");
+    const int NSU = (Nc + kSubC - 1) / kSubC;
+    unsigned smk[SJ];
 #pragma unroll
-        for (int k = 0; k < PB; ++k) t4 += loc[k];
-        cta_excl(t4, mi.scan_i, &wsum);
+    for (int j = 0; j < SJ; ++j) {
+        const int su = tid + kWT * j;
+        smk[j] = (su < NSU) ? __ldcg(s.smax + (int64_t)g * d.nsu + su) : 0u;
     }
+    for (int i = tid; i < NWd; i += kWT) { x.cand[i] = 0u; x.keep[i] = 0u; }
+    // ---- the boundary bin, and from the same scan the total size: when
+    // everything fits there is no boundary
+    const int wsum = sel_boundary<PB>(loc, x, mi, 0, budget);
     const bool all = wsum <= budget;
     int above = 0, b0 = -1;
     if (!all) {
-        sel_boundary<PB>(loc, x, mi, 0, budget);
         b0 = x.b_bin;
         above = x.b_above;
     }
@@ -408,80 +430,97 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
         if (c < kSelCache) { v = sm.cs[c]; w = sm.cz[c]; }
         else { v = __ldcg(gsc + c); w = gsz[c]; }
     };
-    // ---- classify, 4 communities (one 16-byte chunk) a load: above the
-    // boundary bin kept, in it a candidate.  Chunk i's 4 bits go to bitmap
-    // word i / 8 through the 8 lanes that share it (consecutive threads hold
-    // consecutive chunks); each warp lists its candidates by ballot prefix.
-    const int nch = (Nc + 3) / 4;
-    if (tid < 4 * nch - Nc && Nc + tid < kSelCache) sm.cz[Nc + tid] = 0;   // the last chunk's padding
-    __syncthreads();
+    // ---- the live slots: those whose largest key reaches the boundary bin
+    // (with everything kept, every slot with a non-empty community), listed
+    // in ascending order (slot tid + kWT j goes j-major, warp by warp)
+    int* lsl = reinterpret_cast<int*>(x.hist);   // the live slots (the refinement's bins come later)
+    {
+        unsigned bl[SJ];
+        int cntw = 0;
+#pragma unroll
+        for (int j = 0; j < SJ; ++j) {
+            const bool lv = smk[j] != 0u && (all || (int)(smk[j] >> kCoarseShift) >= b0);
+            bl[j] = __ballot_sync(kFull, lv);
+            if (lane == 0) mi.scan_i[j * kWW + warp] = __popc(bl[j]);
+            cntw += __popc(bl[j]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < SJ; ++j) {
+            int base = 0;
+            for (int q = 0; q < j * kWW + warp; ++q) base += mi.scan_i[q];
+            if ((bl[j] >> lane) & 1u) lsl[base + __popc(bl[j] & lt)] = tid + kWT * j;
+        }
+        int nl = 0;
+        for (int q = 0; q < SJ * kWW; ++q) nl += mi.scan_i[q];
+        __syncthreads();
+        if (tid == 0) x.n_cand = nl;   // (the live count, kept until the ranking resets it)
+        __syncthreads();
+    }
+    const int NLV = x.n_cand;
+    // ---- classify the live slots, one 16-byte chunk (4 communities) a
+    // thread: above the boundary bin kept, in it a candidate.  The 4 chunks
+    // of a slot sit in 4 consecutive lanes, which assemble its 16 bits; each
+    // warp lists its candidates by ballot prefix.
     int ncw = 0;   // candidates this warp has met (uniform in the warp)
-    constexpr int CU = 4;
-    for (int i0 = 0; i0 < nch; i0 += CU * kT) {
-        float4 v[CU];
-        int4 w[CU];
+    for (int t0 = 0; t0 < 4 * NLV; t0 += kWT) {
+        const int t = t0 + tid;
+        const bool on = t < 4 * NLV;
+        const int su = on ? lsl[t >> 2] : 0, qc = t & 3;
+        const int i = 4 * su + qc;   // chunk
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        int4 w = make_int4(0, 0, 0, 0);
+        if (on) {
+            if (4 * i < kSelCache) {
+                v = reinterpret_cast<const float4*>(sm.cs)[i];
+                w = reinterpret_cast<const int4*>(sm.cz)[i];
+            } else {   // beyond the staged communities: from L2
 #pragma unroll
-        for (int u = 0; u < CU; ++u) {
-            const int i = i0 + u * kT + tid;
-            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            w[u] = make_int4(0, 0, 0, 0);
-            if (i < nch) {
-                if (4 * i < kSelCache) {
-                    v[u] = reinterpret_cast<const float4*>(sm.cs)[i];
-                    w[u] = reinterpret_cast<const int4*>(sm.cz)[i];
-                } else {   // beyond the staged communities: from L2
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 4 * i + e;
-                        (&v[u].x)[e] = (c < Nc) ? __ldcg(gsc + c) : 0.f;
-                        (&w[u].x)[e] = (c < Nc) ? gsz[c] : 0;
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 4 * i + e;
+                    (&v.x)[e] = (c < Nc) ? __ldcg(gsc + c) : 0.f;
+                    (&w.x)[e] = (c < Nc) ? gsz[c] : 0;
                 }
             }
         }
+        unsigned kb = 0u, cb = 0u;
 #pragma unroll
-        for (int u = 0; u < CU; ++u) {
-            const int i = i0 + u * kT + tid;
-            unsigned kb = 0u, cb = 0u;
+        for (int e = 0; e < 4; ++e) {
+            const int bn = ((&w.x)[e] <= 0 || 4 * i + e >= Nc) ? -1 : all ? kCoarse : bin_of((&v.x)[e]);
+            kb |= (bn > b0 ? 1u : 0u) << e;
+            cb |= (bn == b0 ? 1u : 0u) << e;
+        }
+        unsigned kw = kb << (4 * qc), cw = cb << (4 * qc);
+        kw |= __shfl_xor_sync(kFull, kw, 1);
+        cw |= __shfl_xor_sync(kFull, cw, 1);
+        kw |= __shfl_xor_sync(kFull, kw, 2);
+        cw |= __shfl_xor_sync(kFull, cw, 2);
+        if (on && qc == 0) {
+            if (kw) atomicOr(&x.keep[su >> 1], kw << (16 * (su & 1)));
+            if (cw) atomicOr(&x.cand[su >> 1], cw << (16 * (su & 1)));
+        }
+        if (__any_sync(kFull, cb != 0u)) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int bn = ((&w[u].x)[e] <= 0) ? -1 : all ? kCoarse : bin_of((&v[u].x)[e]);
-                kb |= (bn > b0 ? 1u : 0u) << e;
-                cb |= (bn == b0 ? 1u : 0u) << e;
-            }
-            unsigned kw = kb << (4 * (lane & 7)), cw = cb << (4 * (lane & 7));
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1) {
-                kw |= __shfl_xor_sync(kFull, kw, o);
-                cw |= __shfl_xor_sync(kFull, cw, o);
-            }
-            if ((lane & 7) == 0 && i < nch) {
-                x.keep[i >> 3] = kw;
-                x.cand[i >> 3] = cw;
-            }
-            if (__any_sync(kFull, cb != 0u)) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const unsigned me = __ballot_sync(kFull, (cb >> e) & 1u);
-                    if ((cb >> e) & 1u) {
-                        const int slot = ncw + __popc(me & lt);
-                        if (slot < kSelCapW) {
-                            x.wkey[warp * kSelCapW + slot] = sel_key((&v[u].x)[e], 4 * i + e);
-                            x.ww[warp * kSelCapW + slot] = (&w[u].x)[e];
-                        }
+                const unsigned me = __ballot_sync(kFull, (cb >> e) & 1u);
+                if ((cb >> e) & 1u) {
+                    const int slot = ncw + __popc(me & lt);
+                    if (slot < kSelCapW) {
+                        x.wkey[warp * kSelCapW + slot] = sel_key((&v.x)[e], 4 * i + e);
+                        x.ww[warp * kSelCapW + slot] = (&w.x)[e];
                     }
-                    ncw += __popc(me);
                 }
+                ncw += __popc(me);
             }
         }
     }
     if (lane == 0) x.nw[warp] = ncw;
     __syncthreads();
     if (!all) {
-        int nwl[kW], m = 0;
+        int nwl[kWW], m = 0;
         bool over = false;
 #pragma unroll
-        for (int w = 0; w < kW; ++w) {
+        for (int w = 0; w < kWW; ++w) {
             nwl[w] = x.nw[w];
             m += nwl[w];
             over |= nwl[w] > kSelCapW;
@@ -491,7 +530,7 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
             // radix passes over the candidates' keys, 10 bits below their
             // highest differing bit each time; the final candidates end in
             // the flat list
-            for (int w = 0; w < kW; ++w) nwl[w] = 0;
+            for (int w = 0; w < kWW; ++w) nwl[w] = 0;
             for (int pass = 0; m > kSelCap || over; ++pass) {
                 over = false;
                 if (pass == 8) {   // 64 key bits take at most 7 passes: unreachable
@@ -499,7 +538,7 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
                     return;
                 }
                 unsigned long long kmn = ~0ull, kmx = 0ull;
-                for (int i = tid; i < NWd; i += kT) {
+                for (int i = tid; i < NWd; i += kWT) {
                     unsigned bits = x.cand[i];
                     while (bits) {
                         const int c = 32 * i + __ffs(bits) - 1;
@@ -517,19 +556,19 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
                     kmn = min(kmn, __shfl_xor_sync(kFull, kmn, o));
                     kmx = max(kmx, __shfl_xor_sync(kFull, kmx, o));
                 }
-                if (lane == 0) { mi.red_k[warp] = kmn; mi.red_k[kW + warp] = kmx; }
-                for (int i = tid; i < kSelB; i += kT) x.hist[i] = 0;
+                if (lane == 0) { mi.red_k[warp] = kmn; mi.red_k[kWW + warp] = kmx; }
+                for (int i = tid; i < kSelB; i += kWT) x.hist[i] = 0;
                 __syncthreads();
                 kmn = mi.red_k[0];
-                kmx = mi.red_k[kW];
+                kmx = mi.red_k[kWW];
 #pragma unroll
-                for (int w = 1; w < kW; ++w) {
+                for (int w = 1; w < kWW; ++w) {
                     kmn = min(kmn, mi.red_k[w]);
-                    kmx = max(kmx, mi.red_k[kW + w]);
+                    kmx = max(kmx, mi.red_k[kWW + w]);
                 }
                 const int shift = max(0, 63 - __clzll((long long)(kmn ^ kmx)) - 9);
                 auto digit = [&](unsigned long long k) { return (int)((k >> shift) & (unsigned long long)(kSelB - 1)); };
-                for (int i = tid; i < NWd; i += kT) {
+                for (int i = tid; i < NWd; i += kWT) {
                     unsigned bits = x.cand[i];
                     while (bits) {
                         const int c = 32 * i + __ffs(bits) - 1;
@@ -542,7 +581,7 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
                 }
                 __syncthreads();
                 {
-                    constexpr int RB = kSelB / kT;
+                    constexpr int RB = kSelB / kWT;
                     int rl[RB];
 #pragma unroll
                     for (int k = 0; k < RB; ++k) rl[k] = x.hist[kSelB - 1 - (RB * tid + k)];
@@ -552,7 +591,7 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
                 above = x.b_above;
                 if (tid == 0) x.n_cand = 0;
                 __syncthreads();
-                for (int i = tid; i < NWd; i += kT) {
+                for (int i = tid; i < NWd; i += kWT) {
                     unsigned bits = x.cand[i], nc = 0u, nk = 0u;
                     while (bits) {
                         const int bit = __ffs(bits) - 1;
@@ -580,24 +619,31 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
         }
         // ---- the boundary communities ranked exactly: each sums the sizes
         // of the better ones and is kept iff the sizes through it fit
-        for (int i = tid; i < m; i += kT) {
-            int li = i, wl = 0;   // list and index of candidate i
-            while (wl < kW - 1 && li >= nwl[wl]) { li -= nwl[wl]; ++wl; }
-            const unsigned long long k = x.wkey[wl * kSelCapW + li];
-            const int w = x.ww[wl * kSelCapW + li];
-            int bp[4] = {0, 0, 0, 0};
+        // the lists made one (in the refinement bins' bytes), then thread i
+        // ranks candidate i against all of them
+        unsigned long long* fk = reinterpret_cast<unsigned long long*>(x.hist);   // [kSelCap]
+        int* fw = reinterpret_cast<int*>(fk + kSelCap);                          // [kSelCap]
+        static_assert(kSelCap * 12 <= (int)sizeof(x.hist), "the flat candidates must fit the bins");
+        {
+            int base = 0;
 #pragma unroll
-            for (int l = 0; l < kW; ++l) {
-                const unsigned long long* kl = x.wkey + l * kSelCapW;
-                const int* wl = x.ww + l * kSelCapW;
-                const int nl = nwl[l];
-                int t = 0;
-                for (; t + 4 <= nl; t += 4) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) bp[q] += (kl[t + q] > k) ? wl[t + q] : 0;
-                }
-                for (; t < nl; ++t) bp[0] += (kl[t] > k) ? wl[t] : 0;
+            for (int l = 0; l < kWW; ++l) base += (l < warp) ? nwl[l] : 0;
+            for (int t = lane; t < nwl[warp]; t += 32) {
+                fk[base + t] = x.wkey[warp * kSelCapW + t];
+                fw[base + t] = x.ww[warp * kSelCapW + t];
             }
+        }
+        __syncthreads();
+        for (int i = tid; i < m; i += kWT) {
+            const unsigned long long k = fk[i];
+            const int w = fw[i];
+            int bp[4] = {0, 0, 0, 0};
+            int t = 0;
+            for (; t + 4 <= m; t += 4) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) bp[q] += (fk[t + q] > k) ? fw[t + q] : 0;
+            }
+            for (; t < m; ++t) bp[0] += (fk[t] > k) ? fw[t] : 0;
             const int bpre = bp[0] + bp[1] + bp[2] + bp[3];
             if (above + bpre + w <= budget || (above == 0 && bpre == 0)) {
                 const int c = (int)~(uint32_t)(k & 0xffffffffull);
@@ -610,7 +656,7 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
     // owns the bitmap words [t WPT, (t + 1) WPT); one scan of (count, sizes)
     auto size_of = [&](int c) { return (c < kSelCache) ? sm.cz[c] : gsz[c]; };
     auto off_of = [&](int c) { return (c < kSelCache) ? sm.co[c] : gco[c]; };
-    const int WPT = (NWd + kT - 1) / kT;
+    const int WPT = (NWd + kWT - 1) / kWT;
     const int wa = min(NWd, tid * WPT), wb = min(NWd, (tid + 1) * WPT);
     int cnt = 0, tsz = 0;
     for (int i = wa; i < wb; ++i) {
@@ -626,14 +672,14 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
     {
         const int ic = warp_incl(cnt, lane), is = warp_incl(tsz, lane);
         __syncthreads();
-        if (lane == 31) { mi.scan_i[warp] = ic; mi.scan_i[kW + warp] = is; }
+        if (lane == 31) { mi.scan_i[warp] = ic; mi.scan_i[kWW + warp] = is; }
         __syncthreads();
         int bc = 0, bs = 0;
         C = 0;
         T = 0;
 #pragma unroll
-        for (int w = 0; w < kW; ++w) {
-            const int vc = mi.scan_i[w], vs = mi.scan_i[kW + w];
+        for (int w = 0; w < kWW; ++w) {
+            const int vc = mi.scan_i[w], vs = mi.scan_i[kWW + w];
             bc += (w < warp) ? vc : 0;
             bs += (w < warp) ? vs : 0;
             C += vc;
@@ -675,48 +721,31 @@ __device__ void select_graph(const DevState& s, const Dims& d, int g, SelSmem& s
         meta[M_ROWS] = d.S + T + 1;
     }
     __syncthreads();   // the kept list is complete
-    // ---- round 2: the kept members' rows.  Thread t copies rows
-    // [t RPT, (t + 1) RPT): the kept community of its first row by binary
-    // search, then a walk (row r is member r - krow[k] of kept community k);
-    // all of its pool loads are issued before any store.
+    // ---- round 2: the kept members' rows.  Warp w copies kept communities
+    // w, w + 8, ... (lane = member), 32 communities' loads in flight.
     int32_t* rtok = s.rtok + (int64_t)g * d.rtok_stride;
-    constexpr int RU = 32;
-    const int RPT = (T + kT - 1) / kT;
-    for (int c0 = 0; c0 < RPT; c0 += RU) {
-        const int ra = min(T, tid * RPT + c0), rb = min(T, min(tid * RPT + c0 + RU, (tid + 1) * RPT));
-        int a = 0;
-        if (ra < rb) {
-            int top = 1;
-            while (2 * top < C) top *= 2;
-            for (int step = top; step > 0; step >>= 1) {
-                const int t = a + step;
-                if (t < C && krow[t] <= ra) a = t;
-            }
-        }
-        int src[RU];
+    constexpr int KU = 32;
+    for (int k0 = warp; k0 < C; k0 += KU * kWW) {
+        int rs[KU], sz[KU], of[KU], tk[KU];
 #pragma unroll
-        for (int u = 0; u < RU; ++u) {
-            const int r = ra + u;
-            src[u] = -1;
-            if (r < rb) {
-                while (krow[a + 1] <= r) ++a;   // krow[C] = T > r
-                src[u] = koff[a] + (r - krow[a]);
-            }
-        }
-        int tk[RU];
-#pragma unroll
-        for (int u = 0; u < RU; ++u) {
-            const bool ok = src[u] >= 0 && (int64_t)src[u] < d.P;
-            tk[u] = ok ? gpool[src[u]] : 0;
+        for (int u = 0; u < KU; ++u) {
+            const int k = k0 + u * kWW;
+            const bool on = k < C;
+            rs[u] = on ? krow[k] : 0;
+            sz[u] = on ? krow[k + 1] - rs[u] : 0;
+            of[u] = on ? koff[k] : 0;
+            if (of[u] < 0 || (int64_t)of[u] + sz[u] > d.P) sz[u] = -1;   // a corrupt segment: read nothing
         }
 #pragma unroll
-        for (int u = 0; u < RU; ++u) {
-            const int r = ra + u;
-            if (r < rb) {
-                if (src[u] < 0 || (int64_t)src[u] >= d.P) set_error(s.err, CKV_ERR_STATE);   // a corrupt segment
-                rtok[r] = tk[u];
-            }
+        for (int u = 0; u < KU; ++u) tk[u] = (lane < sz[u]) ? gpool[of[u] + lane] : 0;
+#pragma unroll
+        for (int u = 0; u < KU; ++u) {
+            if (lane < sz[u]) rtok[rs[u] + lane] = tk[u];
+            if (sz[u] < 0 && lane == 0) set_error(s.err, CKV_ERR_STATE);
         }
+#pragma unroll
+        for (int u = 0; u < KU; ++u)   // communities longer than a warp: the rest
+            for (int r = 32 + lane; r < sz[u]; r += 32) rtok[rs[u] + r] = gpool[of[u] + r];
     }
 }
 
@@ -781,7 +810,7 @@ __device__ __forceinline__ void warp_rows_mma(const WarpRows& a, const uint32_t*
 {
     using L = AttL<true, HG>;
     constexpr int NB = L::NB;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = (threadIdx.x >> 5) & (kW - 1);
     const int gid = lane >> 2, tig = lane & 3;
     // B operand Q^T (dims x heads): lane holds head gid, dims 16ks + 2tig (+1, +8, +9)
     uint32_t qf[8][2];
@@ -902,7 +931,7 @@ __device__ __forceinline__ void warp_rows_mma(const WarpRows& a, const uint32_t*
         l[jj] += __shfl_xor_sync(kFull, l[jj], 8);
         l[jj] += __shfl_xor_sync(kFull, l[jj], 16);
     }
-    __syncthreads();   // every warp is done with its pipeline: red overlays them
+    hsync();   // every warp of the half is done with its pipeline: red overlays them
     float* rw = red + warp * HG * L::RSTR;
 #pragma unroll
     for (int jj = 0; jj < 2; ++jj) {
@@ -927,7 +956,7 @@ __device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __
     using L = AttL<false, HG>;
     constexpr int NB = L::NB, RB = L::RB, NV = 4 * HG;
     static_assert(L::BATCH + NB * HG * 4 <= kSlot, "batch and exchange must fit a slot");
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = (threadIdx.x >> 5) & (kW - 1);
     float qv[HG][4];
 #pragma unroll
     for (int h = 0; h < HG; ++h)
@@ -1036,7 +1065,7 @@ __device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __
         __syncwarp();
     }
     cp_async_wait<0>();
-    __syncthreads();   // every warp is done with its pipeline: red overlays them
+    hsync();   // every warp of the half is done with its pipeline: red overlays them
 #pragma unroll
     for (int h = 0; h < HG; ++h) {
         float* rw = red + (warp * HG + h) * L::RSTR;
@@ -1052,11 +1081,26 @@ __device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __
 // extra entries of threads 0 .. kappa-1.  Per round: tau = the kappa-th
 // best of each warp's lane-bests is a lower bound of the answer (that warp
 // holds kappa keys at least as good), so only entries >= the largest such
-// tau -- at most kW * kappa * (FR + 1), the capacity of ck / cx -- are
+// tau -- at most kWW * kappa * (FR + 1), the capacity of ck / cx -- are
 // compacted and ranked by counting.  The list keeps each entry's kept-member
 // row for the assignment.
 constexpr int kFinMaxRows = 16;                                 // rows per thread and round
-constexpr int kFinCand = kW * kMaxKappa * (kFinMaxRows + 1);    // compacted entries, at most
+constexpr int kFinCand = kWW * kMaxKappa * (kFinMaxRows + 1);    // compacted entries, at most
+
+// An edge weight (a sum of at most 8 probabilities, so below 8, with every
+// vote's total below 8 too) as fixed point in units of 2^-59: exact for
+// weights of at least 2^-36, and sums of them exact.  The votes are then
+// exact sums; a double-precision sum in any order differs from them by at
+// most a few units of 2^-53 relative.
+__device__ __forceinline__ unsigned long long weight_fix(float w)
+{
+    const uint32_t b = __float_as_uint(w);
+    const int e = (int)((b >> 23) & 255u);
+    if (e == 0) return 0ull;                         // zero (and subnormals, far below 2^-36)
+    const unsigned long long m = (unsigned long long)((b & 0x7fffffu) | 0x800000u);
+    const int sh = e - 127 - 23 + 59;                // value = m 2^(e - 127 - 23)
+    return sh >= 0 ? (m << sh) : (sh > -64 ? (m >> -sh) : 0ull);
+}
 
 // 64-bit order-preserving key of an edge candidate: larger = ranked first
 // (w desc, token asc; w >= 0); 0 marks an empty slot
@@ -1070,16 +1114,16 @@ __device__ __forceinline__ int key_t(unsigned long long k) { return (int)~(uint3
 struct EdgeScratch {
     unsigned long long lk[kMaxKappa];            // running list (rank order)
     int lx[kMaxKappa];                           // kept-member row of each entry
-    unsigned long long wk[kW];                   // each warp's tau
+    unsigned long long wk[kWW];                   // each warp's tau
     int m;                                       // compacted entries
 };
-// the finish's shared memory (in the rings): item weights | edge scratch |
-// staged logits, tokens and kept-community table (when they fit) |
-// compaction slots (keys, then rows)
+// the finish's shared memory: half 0's rings hold the staged logits,
+// tokens and kept-community table (when they fit); half 1's rings the item
+// weights, the edge scratch and the compaction slots (keys, then rows)
 constexpr int kFinWgt = 0;                       // [nc][HG] floats, nc <= kMaxApi
 constexpr int kFinScr = kMaxApi * 8 * 4;
-constexpr int kFinStage = kFinScr + ((int)sizeof(EdgeScratch) + 127) / 128 * 128;
-static_assert(kFinStage + kFinCand * 12 <= kRing, "edge scratch must fit the rings");
+constexpr int kFinCk = kFinScr + ((int)sizeof(EdgeScratch) + 127) / 128 * 128;
+static_assert(kFinCk + kFinCand * 12 <= kRing, "edge scratch must fit the rings");
 
 template <int HG>
 struct EdgeRows {
@@ -1117,13 +1161,13 @@ __device__ __forceinline__ void load_logits(const float* p, float (&z)[HG])
     }
 }
 
-// one round's logits and tokens of this thread: rows j0 + tid + u * kT
+// one round's logits and tokens of this thread: rows j0 + tid + u * kWT
 template <int HG>
 __device__ __forceinline__ void edges_load(const EdgeSrc& src, int T, int j0, EdgeRows<HG>& r)
 {
 #pragma unroll
     for (int u = 0; u < EdgeRows<HG>::FR; ++u) {
-        const int j = j0 + threadIdx.x + u * kT;
+        const int j = j0 + threadIdx.x + u * kWT;
         r.t[u] = 0;
         if (j < T) {
             if (src.staged) {
@@ -1145,14 +1189,14 @@ __device__ __forceinline__ void cta_edges(const Dims& d, const EdgeSrc& src, int
     constexpr int FR = EdgeRows<HG>::FR;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kappa = d.kappa;
-    const int cap = kW * kappa * (FR + 1);
+    const int cap = kWW * kappa * (FR + 1);
     if (tid < kMaxKappa) { e.lk[tid] = 0ull; e.lx[tid] = -1; }
-    for (int j0 = 0; j0 < max(T, 1); j0 += FR * kT) {
+    for (int j0 = 0; j0 < max(T, 1); j0 += FR * kWT) {
         if (j0 > 0) edges_load<HG>(src, T, j0, r);
         unsigned long long key[FR + 1];
 #pragma unroll
         for (int u = 0; u < FR; ++u) {
-            const int j = j0 + tid + u * kT;
+            const int j = j0 + tid + u * kWT;
             float sw = 0.f;
 #pragma unroll
             for (int h = 0; h < HG; ++h) sw += __expf(r.z[u][h] - sM[h]) * sL[h];
@@ -1174,21 +1218,21 @@ __device__ __forceinline__ void cta_edges(const Dims& d, const EdgeSrc& src, int
         __syncthreads();
         unsigned long long tk = 1ull;
 #pragma unroll
-        for (int wi = 0; wi < kW; ++wi) tk = max(tk, e.wk[wi]);
+        for (int wi = 0; wi < kWW; ++wi) tk = max(tk, e.wk[wi]);
 #pragma unroll
         for (int u = 0; u <= FR; ++u) {
             if (key[u] && key[u] >= tk) {
                 const int slot = atomicAdd(&e.m, 1);
                 if (slot < cap) {
                     ck[slot] = key[u];
-                    cx[slot] = (u < FR) ? j0 + tid + u * kT : xl;
+                    cx[slot] = (u < FR) ? j0 + tid + u * kWT : xl;
                 }
             }
         }
         __syncthreads();
         // rank them; the first kappa become the running list
         const int m = min(e.m, cap);
-        for (int i = tid; i < m; i += kT) {
+        for (int i = tid; i < m; i += kWT) {
             const unsigned long long mk = ck[i];
             int rr = 0;
 #pragma unroll 8
@@ -1198,7 +1242,7 @@ __device__ __forceinline__ void cta_edges(const Dims& d, const EdgeSrc& src, int
                 e.lx[rr] = cx[i];
             }
         }
-        for (int i = m + tid; i < kappa; i += kT) { e.lk[i] = 0ull; e.lx[i] = -1; }
+        for (int i = m + tid; i < kappa; i += kWT) { e.lk[i] = 0ull; e.lx[i] = -1; }
     }
     __syncthreads();
 }
@@ -1224,7 +1268,8 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
     const bool full = !d.rows_given;
     const float* pmg = s.part_ml + (int64_t)g * nc * HG * 2;
     const float* pog = s.part_o + (int64_t)g * nc * HG * kD;
-    float* wgt = reinterpret_cast<float*>(scratch + kFinWgt);   // [nc][HG] item weights
+    unsigned char* scratch1 = scratch + kHalf;
+    float* wgt = reinterpret_cast<float*>(scratch1 + kFinWgt);   // [nc][HG] item weights
     int C = 0;
     EdgeSrc src;
     unsigned long long* ck = nullptr;
@@ -1238,29 +1283,28 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
         const int64_t ze = ((int64_t)g * d.NM + d.S) * HG, te = (int64_t)g * d.rtok_stride;
         const int zpad = (int)(ze & 3), tpad = (int)(te & 3);
         const int zc = (zpad + T * HG + 3) & ~3, tc = (tpad + T + 3) & ~3;   // elements copied
-        const int cap = kW * d.kappa * (EdgeRows<HG>::FR + 1);
+        const int cap = kWW * d.kappa * (EdgeRows<HG>::FR + 1);
         const int4* kig = reinterpret_cast<const int4*>(s.kinfo) + (int64_t)g * d.Nc;
-        src.staged = (int64_t)kFinStage + 4 * ((int64_t)zc + tc) + 16 * (int64_t)C + 12 * (int64_t)cap <= kRing;
+        src.staged = 4 * ((int64_t)zc + tc) + 16 * (int64_t)C <= kRing;
         if (src.staged) {
-            float* zs = reinterpret_cast<float*>(scratch + kFinStage);
+            float* zs = reinterpret_cast<float*>(scratch);
             int32_t* ts = reinterpret_cast<int32_t*>(zs + zc);
             int4* ks = reinterpret_cast<int4*>(ts + tc);
             const float* zg = s.zrow + (ze - zpad);
             const int32_t* tg = s.rtok + (te - tpad);
-            for (int i = tid; i < zc / 4; i += kT) cp_async16(zs + 4 * i, zg + 4 * i);
-            for (int i = tid; i < tc / 4; i += kT) cp_async16(ts + 4 * i, tg + 4 * i);
-            for (int i = tid; i < C; i += kT) cp_async16(ks + i, kig + i);
+            for (int i = tid; i < zc / 4; i += kWT) cp_async16(zs + 4 * i, zg + 4 * i);
+            for (int i = tid; i < tc / 4; i += kWT) cp_async16(ts + 4 * i, tg + 4 * i);
+            for (int i = tid; i < C; i += kWT) cp_async16(ks + i, kig + i);
             cp_async_commit();
             src.z = zs + zpad;
             src.t = ts + tpad;
             src.ki = ks;
-            ck = reinterpret_cast<unsigned long long*>(ks + C);
         } else {
             src.z = s.zrow + ze;
             src.t = s.rtok + te;
             src.ki = kig;
-            ck = reinterpret_cast<unsigned long long*>(scratch + kFinStage);
         }
+        ck = reinterpret_cast<unsigned long long*>(scratch1 + kFinCk);
         cx = reinterpret_cast<int*>(ck + cap);
     }
     EdgeRows<HG> er;   // the first round of kept members
@@ -1269,7 +1313,7 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
         const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + (n - 1)) * kD;
         kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
     }
-    constexpr bool kPre = HG * (kD / 4) <= kT;
+    constexpr bool kPre = HG * (kD / 4) <= kWT;
     const bool pre = kPre && nc <= 16;
     float4 ov[kPre ? 16 : 1];
     if constexpr (kPre) {
@@ -1283,8 +1327,8 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
         }
     }
     if (full && !src.staged) edges_load<HG>(src, T, 0, er);
-    // ---- the heads' max and sum over the items: warp h % kW takes head h
-    for (int h = warp; h < HG; h += kW) {
+    // ---- the heads' max and sum over the items: warp h % kWW takes head h
+    for (int h = warp; h < HG; h += kWW) {
         float M = -INFINITY, Lsum = 0.f;
         for (int k0 = 0; k0 < nc; k0 += 32) {
             const int k = k0 + lane;
@@ -1331,7 +1375,7 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
             }
             *reinterpret_cast<float4*>(out + ((int64_t)b * d.Hq + h0 + h) * kD + 4 * d4) = o;
         }
-    } else for (int i4 = tid; i4 < HG * (kD / 4); i4 += kT) {
+    } else for (int i4 = tid; i4 < HG * (kD / 4); i4 += kWT) {
         const int h = i4 / (kD / 4), d4 = i4 % (kD / 4);
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k0 = 0; k0 < nc; k0 += 16) {
@@ -1358,7 +1402,7 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
         __syncthreads();
         edges_load<HG>(src, T, 0, er);
     }
-    EdgeScratch& es = *reinterpret_cast<EdgeScratch*>(scratch + kFinScr);
+    EdgeScratch& es = *reinterpret_cast<EdgeScratch*>(scratch1 + kFinScr);
     cta_edges<HG>(d, src, T, mi.sM, mi.sL, es, ck, cx, er);
     // ---- the assignment: each edge's kept community (the last with row
     // start <= its row), then the weighted plurality of their ids
@@ -1390,19 +1434,23 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
             s.e_comm[(int64_t)g * d.kappa + lane] = cm;
         }
         if (lane == 0) s.meta[(int64_t)g * M_COUNT + M_NEDGE] = ne;
-        // each lane sums its community's weights in rank order (double),
+        // each lane sums its community's weights exactly, in fixed point
+        // (the order of the sum does not matter then); the largest sum wins,
         // ties to the lower id
-        double v = 0.0;
+        const unsigned long long fw = real ? weight_fix(lw) : 0ull;
+        unsigned long long v = 0ull;
+#pragma unroll 8
         for (int e = 0; e < ne; ++e) {
             const int ce = __shfl_sync(kFull, cm, e);
-            const float we = __shfl_sync(kFull, lw, e);
-            if (ce == cm) v += (double)we;
+            const unsigned long long we = __shfl_sync(kFull, fw, e);
+            v += (ce == cm) ? we : 0ull;
         }
-        double bv = real ? v : -1.0;
+        // (vote + 1, inverted id): the largest key is the winner; no edge: 0
+        unsigned long long bv = real ? v + 1ull : 0ull;
         int bc = real ? cm : 0x7fffffff;
 #pragma unroll
         for (int o = 16; o; o >>= 1) {
-            const double v2 = __shfl_xor_sync(kFull, bv, o);
+            const unsigned long long v2 = __shfl_xor_sync(kFull, bv, o);
             const int c2 = __shfl_xor_sync(kFull, bc, o);
             if (v2 > bv || (v2 == bv && c2 < bc)) { bv = v2; bc = c2; }
         }
@@ -1445,7 +1493,7 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
     const int t = n - 1;
     int32_t* pool = s.pool + (int64_t)g * d.P;
     if (off != old_off)
-        for (int i = tid; i < size; i += kT) pool[off + i] = pool[old_off + i];
+        for (int i = tid; i < size; i += kWT) pool[off + i] = pool[old_off + i];
     // running-mean update of the assigned centroid, double math rounded once
     if (tid < kD) {
         const double mv = (double)mval;
@@ -1471,159 +1519,161 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
 }
 
 // ------------------------------------------------------------ the kernel
+// One CTA of 256 threads per SM.  The first n_workers CTAs are workers:
+// all 8 warps run every selection and then every finish, graph g on worker
+// g mod n_workers (two warps per scheduler hide each other's latency in
+// that serial code).  Every other CTA runs as two independent halves of 4
+// warps, each with its own rings, barriers and named barrier, streaming
+// items from the queue: while one half waits (a ring ramping up, a
+// selection not yet published) the other keeps the SM's loads in flight.
 template <bool BF16, int HG>
-__global__ void __launch_bounds__(kT, 2) k_step(DevState s, Dims d, const void* __restrict__ q,
-                                                const void* __restrict__ K, const void* __restrict__ V, int n,
-                                                float* __restrict__ out)
+__global__ void __launch_bounds__(kWT, 1) k_step(DevState s, Dims d, const void* __restrict__ q,
+                                                 const void* __restrict__ K, const void* __restrict__ V, int n,
+                                                 float* __restrict__ out)
 {
     using L = AttL<BF16, HG>;
     extern __shared__ __align__(128) unsigned char smem[];
-    Misc& mi = *reinterpret_cast<Misc*>(smem + kOffMisc);
-    unsigned long long* bars = reinterpret_cast<unsigned long long*>(smem + kOffBar);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    int* tokw = reinterpret_cast<int*>(smem + kOffTok) + warp * kTokW;
-    float* red = reinterpret_cast<float*>(smem);
+    const int half = threadIdx.x >> 7, ht = threadIdx.x & (kT - 1), hwarp = ht >> 5;
+    unsigned char* hb = smem + half * kHalf;
+    Misc& mh = *reinterpret_cast<Misc*>(hb + kHOffMisc);
+    unsigned long long* bars = reinterpret_cast<unsigned long long*>(hb + kHOffBar);
+    int* tokw = reinterpret_cast<int*>(hb + kHOffTok) + hwarp * kTokW;
+    float* red = reinterpret_cast<float*>(hb);
     const int NS = d.rows_given ? 0 : d.G * d.spg;
     const int total = NS + d.G * d.api;
     unsigned* qctr = s.step_ctr;
-    // worker CTAs (the first n_workers) run every selection and then every
-    // finish, graph g on worker g mod n_workers, so their code stays in
-    // those SMs' instruction caches; the other CTAs stream the queue
-    const int NWk = d.rows_given ? 0 : d.n_workers;
+    const int NWk = d.n_workers;
     const bool worker = (int)blockIdx.x < NWk;
-    if (tid == 0) {
+    if (ht == 0) {
         for (int i = 0; i < kW * kNSlot; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
-        mi.item = (worker || *(volatile int*)s.err) ? total : (int)atomicAdd(qctr, 1u);
+        mh.item = (worker || *(volatile int*)s.err) ? total : (int)atomicAdd(qctr, 1u);
     }
-    if (tid < kW) mi.abort[tid] = 0;
+    if (ht < kW) mh.abort[ht] = 0;
     __syncthreads();
     if (worker) {
+        Misc& mw = *reinterpret_cast<Misc*>(smem + kHOffMisc);   // half 0's
         bool ok = true;
-        for (int g = blockIdx.x; ok && g < d.G; g += NWk) {
+        for (int g = blockIdx.x; ok && !d.rows_given && g < d.G; g += NWk) {
             // ---------------- selection of g once its score items are done
-            if (tid == 0) mi.flag = wait_count(s.gcnt + 4 * g, (unsigned)d.spg, s.err, d.wait_polls);
+            if (threadIdx.x == 0) mw.flag = wait_count(s.gcnt + 4 * g, (unsigned)d.spg, s.err, d.wait_polls);
             __syncthreads();
-            ok = mi.flag;
+            ok = mw.flag;
             if (!ok) break;
             __threadfence();
-            select_graph(s, d, g, *reinterpret_cast<SelSmem*>(smem), *reinterpret_cast<SelX*>(smem + kOffX), mi);
+            select_graph(s, d, g, *reinterpret_cast<SelSmem*>(smem), *reinterpret_cast<SelX*>(smem + kOffX), mw);
             __threadfence();
             __syncthreads();
-            if (tid == 0) set_flag(s.gcnt + 4 * g + 1);
+            if (threadIdx.x == 0) set_flag(s.gcnt + 4 * g + 1);
         }
         for (int g = blockIdx.x; ok && g < d.G; g += NWk) {
             // ---------------- finish of g once its attention items are done
-            if (tid == 0) mi.flag = wait_count(s.gcnt + 4 * g + 2, (unsigned)d.api, s.err, d.wait_polls);
+            if (threadIdx.x == 0) mw.flag = wait_count(s.gcnt + 4 * g + 2, (unsigned)d.api, s.err, d.wait_polls);
             __syncthreads();
-            ok = mi.flag;
+            ok = mw.flag;
             if (!ok) break;
             __threadfence();
-            const int R = __ldcg(s.meta + (int64_t)g * M_COUNT + M_ROWS);
-            finish_graph<HG>(s, d, g, R, K, n, out, smem, mi);
-            __syncthreads();
-        }
-        if (!ok && tid == 0) set_error(s.err, CKV_ERR_TIMEOUT);
-    }
-    int item = mi.item;
-    unsigned fills = 0;   // score slots this warp has used (uniform in the warp)
-    while (item < total) {
-        if (item < NS) {
-            // ---------------- score item
-            const int g = item / d.spg, p = item % d.spg;
-            score_item<BF16>(s, d, q, g, p, smem, bars, fills, mi);
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) atomicAdd(s.gcnt + 4 * g, 1u);
-        } else {
-            // ---------------- attention item (with given rows, the last of
-            // a graph's items merges the graph's output)
-            const int j = item - NS;
-            const int g = j / d.api, k = j % d.api;
-            if (!d.rows_given) {
-                if (tid == 0) mi.flag = wait_count(s.gcnt + 4 * g + 1, 1u, s.err, d.wait_polls);
-                __syncthreads();
-                if (!mi.flag) {
-                    if (tid == 0) set_error(s.err, CKV_ERR_TIMEOUT);
-                    break;
-                }
-            }
-            int b, h0, kvh;
-            graph_heads(d, g, b, h0, kvh);
             const int R = d.rows_given ? d.S + s.rows_T[g] + 1 : __ldcg(s.meta + (int64_t)g * M_COUNT + M_ROWS);
-            const int r0 = (int)((int64_t)k * R / d.api), r1 = (int)((int64_t)(k + 1) * R / d.api);
-            const int nrows = r1 - r0;
-            const int64_t kvbase = ((int64_t)b * d.Hkv + kvh) * d.NM;
-            WarpRows a;
-            a.Kb = reinterpret_cast<const char*>(K) + kvbase * L::RB;
-            a.Vb = reinterpret_cast<const char*>(V) + kvbase * L::RB;
-            a.rtok = s.rtok + (int64_t)g * d.rtok_stride;
-            a.zrow = d.rows_given ? nullptr : s.zrow + (int64_t)g * d.NM * HG;
-            a.a0 = r0 + (int)((int64_t)warp * nrows / kW);
-            a.a1 = r0 + (int)((int64_t)(warp + 1) * nrows / kW);
-            a.S = d.S;
-            a.T = R - d.S - 1;
-            a.R = R;
-            a.t_new = n - 1;
-            a.err = s.err;
-            unsigned char* wbuf = smem + warp * (kNSlot * kSlot);
-            if constexpr (BF16) {
-                const uint32_t* q2 = reinterpret_cast<const uint32_t*>(q) + ((int64_t)b * d.Hq + h0) * kD / 2;
-                warp_rows_mma<HG>(a, q2, wbuf, tokw, red);
-            } else {
-                const float* qg = reinterpret_cast<const float*>(q) + ((int64_t)b * d.Hq + h0) * kD;
-                warp_rows_fma<HG>(a, qg, wbuf, tokw, red);
-            }
+            finish_graph<HG>(s, d, g, R, K, n, out, smem, mw);
             __syncthreads();
-            // combine the warps: (m, l, acc) -> this item's partial per head
-            float* po = s.part_o + ((int64_t)g * d.api + k) * HG * kD;
-            float* pm = s.part_ml + ((int64_t)g * d.api + k) * HG * 2;
-            for (int i = tid; i < HG * kD; i += kT) {
-                const int h = i / kD, dd = i % kD;
-                float mw[kW];
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < kW; ++w) {
-                    mw[w] = red[(w * HG + h) * L::RSTR + kD];
-                    M = fmaxf(M, mw[w]);
-                }
-                float o = 0.f, l = 0.f;
-#pragma unroll
-                for (int w = 0; w < kW; ++w) {
-                    const float* rw = red + (w * HG + h) * L::RSTR;
-                    const float f = (mw[w] == -INFINITY) ? 0.f : __expf(mw[w] - M);
-                    o = fmaf(rw[dd], f, o);
-                    l = fmaf(rw[kD + 1], f, l);
-                }
-                po[i] = o;
-                if (dd == 0) *reinterpret_cast<float2*>(pm + h * 2) = make_float2(M, l);
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) mi.flag = (atomicAdd(s.gcnt + 4 * g + 2, 1u) == (unsigned)d.api - 1);
-            __syncthreads();
-            if (d.rows_given && mi.flag) {
-                __threadfence();
-                finish_graph<HG>(s, d, g, R, K, n, out, smem, mi);
-            }
         }
-        __syncthreads();
-        if (tid == 0) mi.item = (*(volatile int*)s.err) ? total : (int)atomicAdd(qctr, 1u);
-        __syncthreads();
-        item = mi.item;
+        if (!ok && threadIdx.x == 0) set_error(s.err, CKV_ERR_TIMEOUT);
+    } else {
+        int item = mh.item;
+        unsigned fills = 0;   // score slots this warp has used (uniform in the warp)
+        while (item < total) {
+            if (item < NS) {
+                // ---------------- score item
+                const int g = item / d.spg, p = item % d.spg;
+                score_item<BF16>(s, d, q, g, p, hb, bars, fills, mh);
+                __threadfence();
+                hsync();
+                if (ht == 0) atomicAdd(s.gcnt + 4 * g, 1u);
+            } else {
+                // ---------------- attention item
+                const int j = item - NS;
+                const int g = j / d.api, k = j % d.api;
+                if (!d.rows_given) {
+                    if (ht == 0) mh.flag = wait_count(s.gcnt + 4 * g + 1, 1u, s.err, d.wait_polls);
+                    hsync();
+                    if (!mh.flag) {
+                        if (ht == 0) set_error(s.err, CKV_ERR_TIMEOUT);
+                        break;
+                    }
+                }
+                int b, h0, kvh;
+                graph_heads(d, g, b, h0, kvh);
+                const int R = d.rows_given ? d.S + s.rows_T[g] + 1 : __ldcg(s.meta + (int64_t)g * M_COUNT + M_ROWS);
+                const int r0 = (int)((int64_t)k * R / d.api), r1 = (int)((int64_t)(k + 1) * R / d.api);
+                const int nrows = r1 - r0;
+                const int64_t kvbase = ((int64_t)b * d.Hkv + kvh) * d.NM;
+                WarpRows a;
+                a.Kb = reinterpret_cast<const char*>(K) + kvbase * L::RB;
+                a.Vb = reinterpret_cast<const char*>(V) + kvbase * L::RB;
+                a.rtok = s.rtok + (int64_t)g * d.rtok_stride;
+                a.zrow = d.rows_given ? nullptr : s.zrow + (int64_t)g * d.NM * HG;
+                a.a0 = r0 + (int)((int64_t)hwarp * nrows / kW);
+                a.a1 = r0 + (int)((int64_t)(hwarp + 1) * nrows / kW);
+                a.S = d.S;
+                a.T = R - d.S - 1;
+                a.R = R;
+                a.t_new = n - 1;
+                a.err = s.err;
+                unsigned char* wbuf = hb + hwarp * (kNSlot * kSlot);
+                if constexpr (BF16) {
+                    const uint32_t* q2 = reinterpret_cast<const uint32_t*>(q) + ((int64_t)b * d.Hq + h0) * kD / 2;
+                    warp_rows_mma<HG>(a, q2, wbuf, tokw, red);
+                } else {
+                    const float* qg = reinterpret_cast<const float*>(q) + ((int64_t)b * d.Hq + h0) * kD;
+                    warp_rows_fma<HG>(a, qg, wbuf, tokw, red);
+                }
+                hsync();
+                // combine the warps: (m, l, acc) -> this item's partial per head
+                float* po = s.part_o + ((int64_t)g * d.api + k) * HG * kD;
+                float* pm = s.part_ml + ((int64_t)g * d.api + k) * HG * 2;
+                for (int i = ht; i < HG * kD; i += kT) {
+                    const int h = i / kD, dd = i % kD;
+                    float mwv[kW];
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < kW; ++w) {
+                        mwv[w] = red[(w * HG + h) * L::RSTR + kD];
+                        M = fmaxf(M, mwv[w]);
+                    }
+                    float o = 0.f, l = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kW; ++w) {
+                        const float* rw = red + (w * HG + h) * L::RSTR;
+                        const float f = (mwv[w] == -INFINITY) ? 0.f : __expf(mwv[w] - M);
+                        o = fmaf(rw[dd], f, o);
+                        l = fmaf(rw[kD + 1], f, l);
+                    }
+                    po[i] = o;
+                    if (dd == 0) *reinterpret_cast<float2*>(pm + h * 2) = make_float2(M, l);
+                }
+                __threadfence();
+                hsync();
+                if (ht == 0) atomicAdd(s.gcnt + 4 * g + 2, 1u);
+            }
+            hsync();
+            if (ht == 0) mh.item = (*(volatile int*)s.err) ? total : (int)atomicAdd(qctr, 1u);
+            hsync();
+            item = mh.item;
+        }
     }
     // ---- the last CTA to leave resets the queue and the graphs' counters
     // for the next step
+    Misc& m0 = *reinterpret_cast<Misc*>(smem + kHOffMisc);
     __syncthreads();
-    if (tid == 0) {
+    if (threadIdx.x == 0) {
         __threadfence();
-        mi.flag = (atomicAdd(qctr + 1, 1u) == gridDim.x - 1);
+        m0.flag = (atomicAdd(qctr + 1, 1u) == gridDim.x - 1);
     }
     __syncthreads();
-    if (mi.flag) {
+    if (m0.flag) {
         __threadfence();
-        for (int i = tid; i < 4 * d.G; i += kT) s.gcnt[i] = 0u;
-        if (tid == 0) { qctr[0] = 0u; qctr[1] = 0u; }
+        for (int i = threadIdx.x; i < 4 * d.G; i += kWT) s.gcnt[i] = 0u;
+        if (threadIdx.x == 0) { qctr[0] = 0u; qctr[1] = 0u; }
     }
 }
 
@@ -1668,11 +1718,11 @@ cudaError_t prepare_step(const Dims& d, int sms, int* grid)
         constexpr int HG = decltype(hgc)::value;
         const void* fn = d.bf16 ? step_fn<true, HG>() : step_fn<false, HG>();
         cudaError_t r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        // two CTAs per SM need the largest shared-memory share of the L1
+        // the CTA's ~197 KB need the largest shared-memory share of the L1
         if (r == cudaSuccess)
             r = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (r != cudaSuccess) return r;
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kT, kSmemBytes);
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kWT, kSmemBytes);
     });
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorLaunchOutOfResources;
@@ -1687,7 +1737,7 @@ cudaError_t launch_step(const DevState& s, const Dims& d, const void* q, const v
         constexpr int HG = decltype(hgc)::value;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(d.nStep);
-        cfg.blockDim = dim3(kT);
+        cfg.blockDim = dim3(kWT);
         cfg.dynamicSmemBytes = kSmemBytes;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
