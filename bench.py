@@ -184,25 +184,86 @@ def job_rate(world, steps, ms):
 
 
 # ------------------------------------------------------------------ oracle
-def run_oracle_steps(wl, n_steps, graphs=None):
-    """Time the CPU oracle (single thread) on `n_steps` decode steps of the
-    workload; returns (seconds, graph-steps done)."""
+def host_cores():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+class OracleSteps:
+    """The CPU oracle on the decode workload, graph by graph.  The graphs of
+    a step are independent, so with threads > 1 they run on a thread pool
+    (each oracle call is one C call that releases the GIL); a step ends when
+    all its graphs are done."""
+
+    def __init__(self, wl, threads=1, graphs=None):
+        import oracle
+        from concurrent.futures import ThreadPoolExecutor
+        self.oracle, self.wl, self.cfg = oracle, wl, wl.cfg
+        cfg = wl.cfg
+        self.graphs = list(range(cfg.n_graphs)) if graphs is None else list(graphs)
+        self.og = {}
+        for g in self.graphs:
+            b, kvh, _ = cfg.graph_heads(g)
+            self.og[g] = oracle.Graph(cfg.n_comm, cfg.head_dim, cfg.n_max)
+            self.og[g].init(cfg.n0, cfg.n_sinks, wl.labels[g], wl.K[b, kvh])
+        self.threads = max(1, min(threads, len(self.graphs)))
+        self.pool = ThreadPoolExecutor(self.threads) if self.threads > 1 else None
+
+    def _one(self, i, g):
+        cfg, wl = self.cfg, self.wl
+        b, kvh, heads = cfg.graph_heads(g)
+        self.oracle.decode_step(self.og[g], np.ascontiguousarray(wl.q[i, b, heads]), wl.K[b, kvh],
+                                wl.V[b, kvh], cfg.n0 + i + 1, cfg.n_sinks, cfg.kappa, cfg.budget)
+
+    def step(self, i):
+        if self.pool is None:
+            for g in self.graphs:
+                self._one(i, g)
+        else:
+            list(self.pool.map(lambda g: self._one(i, g), self.graphs))
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.shutdown()
+
+
+def run_oracle_steps(wl, n_steps, threads=1, first=0):
+    """Time the CPU oracle on decode steps [first, first + n_steps) of the
+    workload (steps before `first` run untimed); returns seconds."""
+    o = OracleSteps(wl, threads)
+    try:
+        for i in range(first):
+            o.step(i)
+        t0 = time.perf_counter()
+        for i in range(first, first + n_steps):
+            o.step(i)
+        return time.perf_counter() - t0
+    finally:
+        o.close()
+
+
+def prefill_oracle_time(P, Q, K, rows_per_head=2048, threads=1):
+    """The prefill oracle (top-kappa rows of every head) on a bounded sample:
+    `rows_per_head` rows spread evenly over [0, n) of each head, split over
+    `threads` threads.  A row i costs (i + 1) key dots, so the time is scaled
+    to all n rows by the ratio of summed row lengths.  Returns (seconds
+    measured, seconds extrapolated to the whole prefill, sample note)."""
     import oracle
-    cfg = wl.cfg
-    graphs = list(range(cfg.n_graphs)) if graphs is None else graphs
-    og = {}
-    for g in graphs:
-        b, kvh, _ = cfg.graph_heads(g)
-        og[g] = oracle.Graph(cfg.n_comm, cfg.head_dim, cfg.n_max)
-        og[g].init(cfg.n0, cfg.n_sinks, wl.labels[g], wl.K[b, kvh])
+    from concurrent.futures import ThreadPoolExecutor
+    n, H = P.n, P.n_heads
+    rows = np.unique(np.linspace(0, n - 1, rows_per_head).round().astype(np.int32))
+    chunks = [(h, c) for h in range(H) for c in np.array_split(rows, max(1, threads // H + 1))]
+
+    def work(hc):
+        h, r = hc
+        oracle.prefill_rows(Q[h], K[h], r, P.n_sinks, P.kappa)
+
     t0 = time.perf_counter()
-    for i in range(n_steps):
-        n = cfg.n0 + i + 1
-        for g in graphs:
-            b, kvh, heads = cfg.graph_heads(g)
-            oracle.decode_step(og[g], np.ascontiguousarray(wl.q[i, b, heads]), wl.K[b, kvh],
-                               wl.V[b, kvh], n, cfg.n_sinks, cfg.kappa, cfg.budget)
-    return time.perf_counter() - t0, n_steps * len(graphs)
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(work, chunks))
+    secs = time.perf_counter() - t0
+    scale = (n * (n + 1) / 2) / float((rows.astype(np.float64) + 1).sum())
+    return secs, secs * scale, (f"{len(rows)} rows evenly spread over n={n} x {H} heads, "
+                                f"{threads} threads, scaled x{scale:.2f} by summed row length")
 
 
 def reference_arm(args, rank, world):
@@ -212,35 +273,18 @@ def reference_arm(args, rank, world):
     steps = args.warmup + args.steps
     if steps > CFG.steps:
         raise SystemExit(f"--impl reference supports at most {CFG.steps} steps")
-    import oracle
-    cfg = CFG
-    og = {}
-    for g in range(cfg.n_graphs):
-        b, kvh, _ = cfg.graph_heads(g)
-        og[g] = oracle.Graph(cfg.n_comm, cfg.head_dim, cfg.n_max)
-        og[g].init(cfg.n0, cfg.n_sinks, wl.labels[g], wl.K[b, kvh])
-
-    def one(i):
-        n = cfg.n0 + i + 1
-        for g in range(cfg.n_graphs):
-            b, kvh, heads = cfg.graph_heads(g)
-            oracle.decode_step(og[g], np.ascontiguousarray(wl.q[i, b, heads]), wl.K[b, kvh],
-                               wl.V[b, kvh], n, cfg.n_sinks, cfg.kappa, cfg.budget)
-
-    for i in range(args.warmup):
-        one(i)
-    t0 = time.perf_counter()
-    for i in range(args.warmup, steps):
-        one(i)
-    dt = time.perf_counter() - t0
+    cores = host_cores()
+    dt = run_oracle_steps(wl, args.steps, threads=cores, first=args.warmup)
     v = args.steps / dt
-    sample = f"{args.steps} full decode steps (all 32 graphs) after {args.warmup} warm-up steps"
+    sample = (f"{args.steps} full decode steps (all {CFG.n_graphs} graphs, one thread per graph on "
+              f"{min(cores, CFG.n_graphs)} of {cores} host cores) after {args.warmup} warm-up steps")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": WORKLOAD},
-        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": min(cores, CFG.n_graphs), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
     return 0
@@ -258,35 +302,45 @@ def upload_graph(g, stream):
     stream.synchronize()
 
 
-def prefill_bench(args):
+def bf16_peak_tflops():
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        v = float(json.load(open(pp)).get("bf16_tflops", 0) or 0)
+        if v:
+            return v, "measured"
+    return 1590.0, "fallback"
+
+
+def prefill_measure(steps, warmup, P=synth.PREFILL):
     """Figure 1 step (1): the prefill top-kappa graph of the 8-head n=16384
     workload, per head (ckv_build_graph) and per KV head of 4 query heads
-    (ckv_build_graph_grouped); device time per call with CUDA events, and
-    the causal Q K^T flops it implies against the measured bf16 peak."""
+    (ckv_build_graph_grouped); device time per call with CUDA events over
+    `steps` calls after `warmup`, and the causal Q K^T flops it implies
+    against the measured bf16 peak (burst: each call is timed alone)."""
     import torch
     import long_context_decode_ckv_b200 as ckv
     from long_context_decode_ckv_b200 import build as ckv_build
-    P = synth.PREFILL
     Q, K = synth.make_prefill(P)
     ckv_build.build()
-    dev = torch.device("cuda", 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
     q = torch.from_numpy(Q).view(torch.bfloat16).to(dev)
     k = torch.from_numpy(K).view(torch.bfloat16).to(dev)
     n, H, S, kap = P.n, P.n_heads, P.n_sinks, P.kappa
     E = int(np.clip(np.arange(n) - S, 0, kap).sum())
     causal_flops = 2.0 * 128 * n * (n + 1) / 2 * H          # one Q K^T over the causal triangle, all heads
+    stream = torch.cuda.current_stream(dev)
 
     def timed(fn):
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             fn()
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.steps):
+        e0.record(stream)
+        for _ in range(steps):
             fn()
-        e1.record()
+        e1.record(stream)
         torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / args.steps
+        return e0.elapsed_time(e1) / steps
 
     rp = torch.empty((H, n + 1), dtype=torch.int64, device=dev)
     col = torch.empty((H, E), dtype=torch.int32, device=dev)
@@ -297,20 +351,181 @@ def prefill_bench(args):
     kk = k[:Hkv].contiguous()
     ms_group = timed(lambda: ckv.ckv_build_graph_grouped(Hkv, g, n, 128, S, kap, ckv.CKV_BF16, q, kk, ws,
                                                          rp[:Hkv], col[:Hkv], w[:Hkv]))
-    peak = None
-    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(pp):
-        peak = float(json.load(open(pp)).get("bf16_tflops", 0)) or None
+    peak, peak_kind = bf16_peak_tflops()
     tf_head = causal_flops / (ms_head / 1e3) / 1e12
     tf_group = 2 * causal_flops / (ms_group / 1e3) / 1e12   # statistics pass + grouped pass
-    print(json.dumps({
-        "metric": "prefill graph ms", "workload": "prefill_8h_n16384_k8_s4_bf16", "steps": args.steps,
-        "warmup": args.warmup,
-        "per_head": {"ms": ms_head, "tflops": tf_head, "frac_of_bf16_peak": tf_head / peak if peak else None},
-        "query_group_4": {"ms": ms_group, "tflops_both_passes": tf_group,
-                          "frac_of_bf16_peak": tf_group / peak if peak else None},
-        "bf16_peak_tflops": peak, "exp2_count": n * (n + 1) / 2 * H,
-    }), flush=True)
+    res = {
+        "workload": "prefill_8h_n16384_k8_s4_bf16", "steps": steps, "warmup": warmup,
+        "ms": ms_head, "kernel": "k_prefill_topk",
+        "roofline": {"bound": "tensor", "achieved": tf_head, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tf_head / peak, "peak_kind": peak_kind + " bf16 burst",
+                     "flops_per_launch": causal_flops},
+        "query_group_4": {"ms": ms_group, "tflops_both_passes": tf_group, "frac": tf_group / peak},
+        "exp2_count": n * (n + 1) / 2 * H,
+    }
+    del q, k, rp, col, w, ws, kk
+    torch.cuda.empty_cache()
+    return res, (Q, K)
+
+
+def prefill_bench(args):
+    res, _ = prefill_measure(args.steps, args.warmup)
+    print(json.dumps({"metric": "prefill graph ms", **res}), flush=True)
+    return 0
+
+
+def decode_rate(cfg, wl, warmup, steps, replicas, profile_steps=0):
+    """Decode steps/s of one more workload (cfg, wl already drawn): `replicas`
+    independent layer copies rotated (inputs larger than L2), `warmup`
+    eager steps, then `steps` steps captured into a CUDA graph and timed
+    with events on the launching stream; optionally `profile_steps` more
+    with per-kernel events.  Returns a dict with the rate, GB/s and the
+    dominant kernel's roofline."""
+    import torch
+    import long_context_decode_ckv_b200 as ckv
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    L = replicas
+    if -(-(warmup + steps + profile_steps) // L) > cfg.steps:
+        raise SystemExit(f"{cfg.name}: not enough decode tokens for these steps")
+
+    def upload(a):
+        t = torch.from_numpy(a)
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).to(dev)
+
+    K0, V0, q = upload(wl.K), upload(wl.V), upload(wl.q)
+    reps = []
+    c = ckv.ckv_config()
+    c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    c.n_max, c.max_communities, c.n_sinks = cfg.n_max, cfg.n_comm, cfg.n_sinks
+    c.kappa, c.budget, c.slack = cfg.kappa, cfg.budget, 16
+    c.kv_dtype = ckv.CKV_BF16 if cfg.bf16 else ckv.CKV_F32
+    c.mode = ckv.CKV_QUERY_GROUP if cfg.mode == synth.QUERY_GROUP else ckv.CKV_PER_HEAD
+    c.device, c.pool_capacity = dev.index, 0
+    try:
+        for r in range(L):
+            K = K0 if r == 0 else K0.clone()
+            V = V0 if r == 0 else V0.clone()
+            ctx = ckv.ckv_create(c)
+            reps.append({"ctx": ctx, "K": K, "V": V, "i": 0})
+            ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        aux, kvb = ckv.ckv_aux_bytes(reps[0]["ctx"])
+        out = torch.empty((cfg.batch, cfg.n_q_heads, cfg.head_dim), dtype=torch.float32, device=dev)
+
+        def step(s, st):
+            r = reps[s % L]
+            i = r["i"]
+            ckv.ckv_decode_step(r["ctx"], q[i], r["K"], r["V"], cfg.n0 + i + 1, out, st)
+            ckv.ckv_assign_update(r["ctx"], r["K"], cfg.n0 + i + 1, st)
+            r["i"] = i + 1
+
+        def graph_of(first, count):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                cap = torch.cuda.current_stream(dev)
+                for s in range(first, first + count):
+                    step(s, cap)
+            upload_graph(g, stream)
+            return g
+
+        for s in range(warmup):
+            step(s, stream)
+        torch.cuda.synchronize(dev)
+        g = graph_of(warmup, steps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / steps
+        del g
+        avg = None
+        if profile_steps:
+            for r in reps:
+                ckv.ckv_profile_begin(r["ctx"])
+            g = graph_of(warmup + steps, profile_steps)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            tot, ks = [0.0] * 4, 0
+            for r in reps:
+                m, k = ckv.ckv_profile_end(r["ctx"])
+                tot = [a + b for a, b in zip(tot, m)]
+                ks += k
+            del g
+            avg = [t / ks for t in tot] if ks else None
+        for r in reps:
+            assert ckv.ckv_last_error(r["ctx"]) == ckv.CKV_OK
+        launches = ckv.ckv_step_launches(reps[0]["ctx"])
+        sel_tok = np.zeros(cfg.n_graphs, np.int32)
+        ckv.ckv_get_step_debug(reps[(warmup + steps - 1) % L]["ctx"], n_tok_sel=sel_tok)
+    finally:
+        for r in reps:
+            ckv.ckv_destroy(r["ctx"])
+        del reps
+        torch.cuda.empty_cache()
+    T_mean = float(sel_tok.mean())
+    step_bytes = algorithmic_bytes(cfg, T_mean) * cfg.n_graphs
+    peak, peak_kind = measured_peaks()
+    res = {"workload": cfg.name, "steps_per_s": 1e3 / ms, "ms_per_step": ms, "steps": steps,
+           "warmup": warmup, "layer_replicas": L, "graphs": cfg.n_graphs, "mean_tokens_kept": T_mean,
+           "algorithmic_bytes_per_step": step_bytes, "hbm_gbs": step_bytes / (ms / 1e3) / 1e9,
+           "hbm_frac_of_measured": step_bytes / (ms / 1e3) / 1e9 / peak, "gpu_launches": launches * steps,
+           "aux_bytes": aux, "kv_bytes": kvb, "aux_over_kv": aux / kvb}
+    if avg is not None:
+        res["kernel_ms_per_step"] = dict(zip(["score", "select", "attend_edges_update", "step_close"], avg)) \
+            if launches == 3 else {"step": avg[0], "step_close": avg[3]}
+        res["roofline"] = roofline_of(cfg, T_mean, avg, launches, peak, peak_kind)
+    return res
+
+
+def roofline_of(cfg, T_mean, avg, launches, peak, peak_kind):
+    """The dominant kernel's algorithmic bytes over its average event time.
+    avg: per-kernel ms per step (score, select, attend, close) or, for the
+    single-launch step, the step kernel's in avg[0]."""
+    if launches == 1:
+        kb = algorithmic_bytes(cfg, T_mean) * cfg.n_graphs
+        kname, t = "k_step", avg[0]
+    else:
+        dom = 0 if avg[0] >= avg[2] else 2
+        kb = kernel_bytes(cfg, T_mean)["score" if dom == 0 else "attend"] * cfg.n_graphs
+        kname, t = ("k_score" if dom == 0 else "k_attend"), avg[dom]
+    achieved = kb / (t / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": peak_kind, "traffic": profiled_traffic(kname),
+            "algorithmic_bytes_per_launch": kb, "avg_launch_ms": t}
+
+
+def sweep_bench(args):
+    """The batch-16 Qwen3-4B-shaped sweep: decode steps/s at every (n, budget)
+    point (n in 8K/32K/128K, budget 128..4096), one JSON line per point plus
+    a summary line.  The workload of one n serves its four budgets."""
+    import torch
+    from long_context_decode_ckv_b200 import build as ckv_build
+    ckv_build.build()
+    torch.cuda.set_device(0)
+    workers = max(1, min(16, os.cpu_count() or 1))
+    rows = []
+    with Clocks(0) as clk:
+        for n in (8192, 32768, 131072):
+            base = synth.make_workload(synth.sweep_config(n, 128), workers=workers)
+            for t in (128, 512, 1024, 4096):
+                cfg = synth.sweep_config(n, t)
+                wl = synth.Workload(cfg, base.K, base.V, base.q, base.labels)
+                # enough replicas that the rotated step data exceeds L2 4 times over
+                sb = algorithmic_bytes(cfg, min(t, cfg.n0)) * cfg.n_graphs
+                kvb = cfg.batch * cfg.n_kv_heads * cfg.n_max * cfg.head_dim * 2 * 2
+                L = int(min(max(2, -(-4 * 126e6 // sb)), max(1, 48e9 // kvb)))
+                L = max(L, -(-(args.warmup + args.steps) // cfg.steps))
+                r = decode_rate(cfg, wl, args.warmup, args.steps, L, profile_steps=0)
+                r.update(n=n, budget=t)
+                rows.append(r)
+                print(json.dumps({"sweep_point": r}), flush=True)
+            del base
+    print(json.dumps({"metric": "decode steps/s (sweep)", "points": len(rows),
+                      "table": [{k: r[k] for k in ("n", "budget", "steps_per_s", "ms_per_step", "hbm_gbs",
+                                                    "mean_tokens_kept", "layer_replicas")} for r in rows],
+                      "clocks": clk.summary()}), flush=True)
     return 0
 
 
@@ -526,6 +741,10 @@ def main():
                     help="time the prefill graph construction (per-head and query-group) instead")
     ap.add_argument("--dense-steps", type=int, default=20,
                     help="dense decode comparator launches timed after the sparse steps (0 = none)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="decode steps/s at every point of the batch-16 (n, budget) sweep instead")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the prefill and Llama per-head measurements of the default line")
     args = ap.parse_args()
     rank, world, local = rank_env()
     if args.warmup < 3:
@@ -536,6 +755,8 @@ def main():
         return recall_sweep(args, [int(b) for b in args.recall_sweep.split(",")])
     if args.prefill:
         return prefill_bench(args)
+    if args.sweep:
+        return sweep_bench(args)
     if args.leiden:
         return leiden_bench(args)
     if args.refresh:
@@ -545,6 +766,7 @@ def main():
     workers = max(1, min(16, (os.cpu_count() or 1) // max(1, world)))
     t_gen = time.perf_counter()
     wl = synth.make_workload(CFG, workers=workers)
+    wl_llama = synth.make_workload(synth.LLAMA, workers=workers) if not args.no_extras else None
     t_gen = time.perf_counter() - t_gen
 
     import torch
@@ -673,6 +895,7 @@ def main():
     for r in reps:
         assert ckv.ckv_last_error(r["ctx"]) == ckv.CKV_OK
     launches_per_step = ckv.ckv_step_launches(reps[0]["ctx"])
+    aux_b, kv_b = ckv.ckv_aux_bytes(reps[0]["ctx"])
     ckv.ckv_get_step_debug(reps[(args.warmup + args.steps - 1) % L]["ctx"], n_tok_sel=sel_tok)
     T_mean = float(sel_tok.mean())
     ms = max_over_ranks(pg, ms, dev)
@@ -757,11 +980,22 @@ def main():
 
     for r in reps:
         ckv.ckv_destroy(r["ctx"])
+    del reps, K0, V0
+    torch.cuda.empty_cache()
     if pg:
         pg.barrier()
         pg.destroy_process_group()
     if rank != 0:
         return 0
+
+    # the other headline numbers, each timed on its own after the step:
+    # the Llama-3.1-8B per-head decode workload and the prefill graph
+    llama, prefill, prefill_qk = None, None, None
+    if not args.no_extras:
+        lc = synth.LLAMA
+        llama = decode_rate(lc, wl_llama, 5, 40, max(4, -(-(5 + 40 + 16) // lc.steps)), profile_steps=16)
+        del wl_llama
+        prefill, prefill_qk = prefill_measure(10, 3)
 
     steps_per_s = job_rate(world, args.steps, ms)
     per_graph = algorithmic_bytes(cfg, T_mean)
@@ -769,32 +1003,31 @@ def main():
     gbs = step_bytes * args.steps / (ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     avg, roofline = None, None
-    if kern_ms is not None and kern_steps and launches_per_step == 1:
-        # the fused step kernel moves every algorithmic byte of the step
-        avg = {"step": kern_ms[0] / kern_steps, "step_close": kern_ms[3] / kern_steps}
-        achieved = step_bytes / (avg["step"] / 1e3) / 1e9
-        roofline = {"bound": "hbm", "kernel": "k_step", "achieved": achieved, "peak": peak,
-                    "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                    "traffic": profiled_traffic("k_step"), "algorithmic_bytes_per_launch": step_bytes,
-                    "avg_launch_ms": avg["step"]}
-    elif kern_ms is not None and kern_steps:
-        names = ["score", "select", "attend_edges_update", "step_close"]
-        avg = {nm: kern_ms[k] / kern_steps for k, nm in enumerate(names)}
-        dom = max(("score", "attend_edges_update"), key=lambda nm: avg[nm])
-        kb = kernel_bytes(cfg, T_mean)["attend" if dom != "score" else "score"] * cfg.n_graphs
-        achieved = kb / (avg[dom] / 1e3) / 1e9
-        kname = "k_score" if dom == "score" else "k_attend"
-        roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
-                    "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                    "traffic": profiled_traffic(kname), "algorithmic_bytes_per_launch": kb,
-                    "avg_launch_ms": avg[dom]}
+    if kern_ms is not None and kern_steps:
+        per = [k / kern_steps for k in kern_ms]
+        avg = ({"step": per[0], "step_close": per[3]} if launches_per_step == 1 else
+               dict(zip(["score", "select", "attend_edges_update", "step_close"], per)))
+        roofline = roofline_of(cfg, T_mean, per, launches_per_step, peak, peak_kind)
 
+    # the oracle on the host: all cores (one thread per graph), one core,
+    # and the prefill oracle on sampled rows
     cpu = None
     if not args.no_cpu:
-        secs, gsteps = run_oracle_steps(wl, args.cpu_steps)
-        cpu = {"value": (gsteps / cfg.n_graphs) / secs, "unit": "steps/s", "cores": 1, "kind": "oracle",
-               "sample": f"{args.cpu_steps} decode steps x {cfg.n_graphs} graphs of the same workload, "
-                         f"single-threaded C oracle ({secs:.1f} s)"}
+        cores = host_cores()
+        secs = run_oracle_steps(wl, args.cpu_steps, threads=cores)
+        secs1 = run_oracle_steps(wl, max(1, args.cpu_steps // 4), threads=1)
+        cpu = {"value": args.cpu_steps / secs, "unit": "steps/s", "cores": min(cores, cfg.n_graphs),
+               "kind": "oracle",
+               "sample": f"{args.cpu_steps} decode steps x {cfg.n_graphs} graphs of the same workload, C oracle, "
+                         f"one thread per graph on {min(cores, cfg.n_graphs)} of {cores} host cores ({secs:.1f} s)",
+               "single_core": {"value": max(1, args.cpu_steps // 4) / secs1, "unit": "steps/s", "cores": 1,
+                               "sample": f"{max(1, args.cpu_steps // 4)} decode steps x {cfg.n_graphs} graphs, "
+                                         f"one thread ({secs1:.1f} s)"}}
+        if prefill_qk is not None:
+            pm, pe, note = prefill_oracle_time(synth.PREFILL, *prefill_qk, threads=cores)
+            cpu["prefill"] = {"value": pe * 1e3, "unit": "ms (extrapolated)", "cores": cores,
+                              "measured_s": pm, "sample": note,
+                              "gpu_over_cpu": (pe * 1e3) / prefill["ms"] if prefill else None}
     line = {
         "metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -808,6 +1041,8 @@ def main():
         "algorithmic_bytes_per_step": step_bytes, "mean_tokens_kept": T_mean,
         "kernel_ms_per_step": avg,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "aux_bytes": aux_b, "kv_bytes": kv_b, "aux_over_kv": aux_b / kv_b,
+        "prefill": prefill, "llama_per_head": llama,
         "recall": recall, "dense_decode": dense,
         "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
         "gen_seconds": t_gen,

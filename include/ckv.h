@@ -28,6 +28,11 @@
  *    ckv_last_error(), and every later call of that context then returns
  *    the same error until ckv_init_communities() or ckv_import_state().
  *  - No call aborts, traps or prints.
+ *  - Calls that allocate device memory (ckv_create, ckv_init_communities,
+ *    ckv_import_state, ckv_refresh, ckv_graph_modularity) allocate before
+ *    they change the context, so CKV_ERR_OOM leaves its state as it was.
+ *    For tests of that path, CKV_FAULT_ALLOC=k in the environment makes the
+ *    k-th device allocation inside each such call fail as out of memory.
  *  - A context is not thread-safe; use one context per host thread.
  */
 #ifndef CKV_H
@@ -265,9 +270,10 @@ ckv_status ckv_last_error(ckv_ctx* ctx);
  * NULL. */
 int ckv_step_launches(const ckv_ctx* ctx);
 
-/* Failure detection: the bound of the fused step's one cross-CTA wait (an
- * attention item waiting for its graph's selection), in polls of about
- * 64 ns each; 0 restores the default (2^22 polls).  A wait that runs out
+/* Failure detection: the bound of the fused step's cross-CTA waits (a
+ * selection waiting for its graph's score items, an attention item for its
+ * graph's selection, a finish for its graph's attention items), in polls
+ * of about 64 ns each; 0 restores the default (2^22 polls).  A wait that runs out
  * stops the step and sets CKV_ERR_TIMEOUT in the error word (read by
  * ckv_last_error); the context is then failed until ckv_init_communities()
  * or ckv_import_state().  A limit of 1 poll makes any step whose selection
@@ -364,11 +370,16 @@ ckv_status ckv_import_state(ckv_ctx* ctx, const void* host_buf, size_t bytes);
  * library keeps until exit; a call needs about max_rows * (4 + 4 * heads
  * per graph) bytes plus its split partials, so max_rows up to about 800,000
  * for a group of 4 heads; a larger max_rows returns CKV_ERR_CAPACITY.
- * Every call shares the array, so calls that overlap on the GPU race;
- * serialise them.  The first call on a device looks up the array's device
- * address; make it before any stream capture.  Asynchronous on `stream`.
- * Errors: CKV_ERR_INVALID_ARG (bad pointer, size or row), CKV_ERR_CAPACITY,
- * CKV_ERR_CUDA. */
+ * Every call shares the array, so calls from different host threads race;
+ * serialise them.  The call runs on `stream` and is synchronous: it copies
+ * the row lists in, launches one kernel, reads the kernel's error word back
+ * and waits for the stream, so rows_host and n_rows_host (pageable or
+ * page-locked) may be reused on return, and the call cannot be captured
+ * into a CUDA graph.  The caller's current device is restored on return.
+ * Errors: CKV_ERR_INVALID_ARG (bad pointer, size, row or device),
+ * CKV_ERR_CAPACITY (max_rows too large for the array), CKV_ERR_STATE (the
+ * kernel found a row outside the cache), CKV_ERR_TIMEOUT (a bounded wait
+ * inside the kernel ran out), CKV_ERR_CUDA. */
 ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, const void* K, const void* V,
                                   int n, const int32_t* rows_host, const int32_t* n_rows_host,
                                   int max_rows, float* out, void* stream);

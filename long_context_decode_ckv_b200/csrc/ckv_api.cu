@@ -78,6 +78,29 @@ ckv_status cuda_status(cudaError_t e)
     return CKV_ERR_CUDA;
 }
 
+// Forced allocation failure for the failure-handling tests: with
+// CKV_FAULT_ALLOC=k in the environment, the k-th device allocation made
+// inside one library call fails as if the device were out of memory.  Each
+// call that allocates arms the count on entry (FaultScope); dev_malloc is
+// the only allocator of the context code.
+thread_local int t_fault_left = 0;
+
+struct FaultScope {
+    FaultScope()
+    {
+        const char* v = getenv("CKV_FAULT_ALLOC");
+        t_fault_left = v ? atoi(v) : 0;
+    }
+    ~FaultScope() { t_fault_left = 0; }
+};
+
+cudaError_t dev_malloc(void** p, size_t bytes)
+{
+    *p = nullptr;
+    if (t_fault_left > 0 && --t_fault_left == 0) return cudaErrorMemoryAllocation;
+    return cudaMalloc(p, bytes);
+}
+
 #define CKV_CUDA(call)                                      \
     do {                                                    \
         cudaError_t e_ = (call);                            \
@@ -120,7 +143,7 @@ template <typename T>
 cudaError_t dalloc(ckv_ctx* x, T** p, size_t count)
 {
     void* v = nullptr;
-    cudaError_t e = cudaMalloc(&v, count * sizeof(T) + 16);
+    cudaError_t e = dev_malloc(&v, count * sizeof(T) + 16);
     if (e != cudaSuccess) return e;
     x->allocs.push_back(v);
     *p = static_cast<T*>(v);
@@ -146,20 +169,43 @@ void free_edges(ckv_ctx* x)
     x->s.edge_deg = nullptr;
 }
 
-cudaError_t alloc_edges(ckv_ctx* x, int64_t rows)
+// a new edge store for `rows` decode rows per graph, allocated before the
+// old one is released: on failure the context keeps its store
+struct EdgeStore {
+    void* p[3] = {nullptr, nullptr, nullptr};
+    int64_t rows = 0;
+    void release()
+    {
+        for (void*& q : p) {
+            if (q) cudaFree(q);
+            q = nullptr;
+        }
+    }
+};
+
+cudaError_t new_edges(const ckv_ctx* x, int64_t rows, EdgeStore& es)
 {
-    free_edges(x);
     const int64_t G = x->d.G, k = x->d.kappa;
     const int64_t r = rows > 0 ? rows : 1;
     cudaError_t e;
-    if ((e = cudaMalloc(&x->edge_alloc[0], (size_t)(G * r * k) * 4)) != cudaSuccess) return e;
-    if ((e = cudaMalloc(&x->edge_alloc[1], (size_t)(G * r * k) * 4)) != cudaSuccess) return e;
-    if ((e = cudaMalloc(&x->edge_alloc[2], (size_t)(G * r) * 4)) != cudaSuccess) return e;
+    es.rows = rows;
+    if ((e = dev_malloc(&es.p[0], (size_t)(G * r * k) * 4)) == cudaSuccess &&
+        (e = dev_malloc(&es.p[1], (size_t)(G * r * k) * 4)) == cudaSuccess &&
+        (e = dev_malloc(&es.p[2], (size_t)(G * r) * 4)) == cudaSuccess)
+        return cudaSuccess;
+    es.release();
+    return e;
+}
+
+void install_edges(ckv_ctx* x, EdgeStore& es)
+{
+    free_edges(x);
+    for (int i = 0; i < 3; ++i) x->edge_alloc[i] = es.p[i];
     x->s.edge_col = static_cast<int32_t*>(x->edge_alloc[0]);
     x->s.edge_w = static_cast<float*>(x->edge_alloc[1]);
     x->s.edge_deg = static_cast<int32_t*>(x->edge_alloc[2]);
-    x->edge_rows = rows;
-    return cudaSuccess;
+    x->edge_rows = es.rows;
+    es = EdgeStore{};
 }
 
 // empty score range and zero total size for every graph (k_score accumulates
@@ -255,6 +301,7 @@ CKV_API void ckv_destroy(ckv_ctx* x)
 
 CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
 {
+    FaultScope fault;
     if (!out) return CKV_ERR_INVALID_ARG;
     *out = nullptr;
     if (!valid_config(cfg)) return CKV_ERR_INVALID_ARG;
@@ -369,7 +416,7 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
     const size_t qb = (size_t)d.B * d.Hq * ckv::kD;
     x->stage_bytes = qb * elem_bytes(cfg->kv_dtype) + 2 * (size_t)d.B * d.Hkv * ckv::kD * elem_bytes(cfg->kv_dtype) +
                      qb * sizeof(float) + 64;
-    if (e == cudaSuccess) e = cudaMalloc(&x->stage, x->stage_bytes);
+    if (e == cudaSuccess) e = dev_malloc(&x->stage, x->stage_bytes);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         ckv_status st = cuda_status(e);
@@ -387,9 +434,22 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
     if (!x || !labels || !K) return CKV_ERR_INVALID_ARG;
     if (n < x->d.S || n > x->d.NM || n_communities < 1 || n_communities > x->d.Nc)
         return CKV_ERR_INVALID_ARG;
+    FaultScope fault;
     cudaStream_t st = (cudaStream_t)stream;
     CKV_CUDA(cudaSetDevice(x->cfg.device));
     CKV_CUDA(cudaStreamSynchronize(st));
+    // everything the call allocates comes first: when an allocation fails
+    // the context keeps its state
+    EdgeStore es;
+    void* tmp = nullptr;
+    {
+        cudaError_t ea = new_edges(x, (int64_t)x->d.NM - n, es);
+        if (ea == cudaSuccess && !labels_on_device) ea = dev_malloc(&tmp, x->d.G * (size_t)n * sizeof(int32_t) + 16);
+        if (ea != cudaSuccess) {
+            es.release();
+            return cuda_status(ea);
+        }
+    }
     x->initialized = 0;
     x->pending = 0;
     x->last_n = 0;
@@ -401,11 +461,9 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
     d.n_init = n;
     const size_t G = d.G;
     const int32_t* dlabels = labels;
-    void* tmp = nullptr;
     if (!labels_on_device) {
-        CKV_CUDA(cudaMalloc(&tmp, G * (size_t)n * sizeof(int32_t) + 16));
         cudaError_t e = cudaMemcpyAsync(tmp, labels, G * (size_t)n * sizeof(int32_t), cudaMemcpyHostToDevice, st);
-        if (e != cudaSuccess) { cudaFree(tmp); return cuda_status(e); }
+        if (e != cudaSuccess) { cudaFree(tmp); es.release(); return cuda_status(e); }
         dlabels = static_cast<const int32_t*>(tmp);
     }
     cudaError_t e = cudaSuccess;
@@ -434,13 +492,13 @@ CKV_API ckv_status ckv_init_communities(ckv_ctx* x, const int32_t* labels, int l
         step(cudaStreamSynchronize(st));
     }
     if (tmp) cudaFree(tmp);
-    if (e != cudaSuccess) return cuda_status(e);
+    if (e != cudaSuccess) { es.release(); return cuda_status(e); }
     if (err != 0) {
+        es.release();
         cudaMemset(s.err, 0, sizeof(int));
         return (ckv_status)err;
     }
-    e = alloc_edges(x, (int64_t)d.NM - n);
-    if (e != cudaSuccess) return cuda_status(e);
+    install_edges(x, es);
     x->n_tok = n;
     x->initialized = 1;
     return CKV_OK;
@@ -695,6 +753,7 @@ CKV_API ckv_status ckv_export_state(ckv_ctx* x, void* host_buf, size_t* bytes)
 
 CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t bytes)
 {
+    FaultScope fault;
     if (!x || !host_buf || bytes < 36) return CKV_ERR_INVALID_ARG;
     int32_t hdr[9];
     memcpy(hdr, host_buf, sizeof hdr);
@@ -756,17 +815,22 @@ CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t byt
         for (size_t r = 0; r < rows; ++r) {
             const int32_t dg = deg_in[g * rows + r];
             if (dg < 0 || dg > d.kappa) return CKV_ERR_INVALID_ARG;
+            // the token at n_init + r links to earlier ordinary positions
             for (int e = 0; e < dg; ++e) {
                 const int32_t c = col_in[(g * rows + r) * d.kappa + e];
-                if (c < 0 || c >= n_tok || !valid_weight(w_in[(g * rows + r) * d.kappa + e]))
+                if (c < d.S || c >= n_init + (int64_t)r || !valid_weight(w_in[(g * rows + r) * d.kappa + e]))
                     return CKV_ERR_INVALID_ARG;
             }
         }
     }
     CKV_CUDA(cudaSetDevice(x->cfg.device));
     CKV_CUDA(cudaDeviceSynchronize());
-    cudaError_t e = alloc_edges(x, (int64_t)d.NM - n_init);
-    if (e != cudaSuccess) return cuda_status(e);
+    {
+        EdgeStore es;
+        const cudaError_t e = new_edges(x, (int64_t)d.NM - n_init, es);
+        if (e != cudaSuccess) return cuda_status(e);   // the context keeps its state
+        install_edges(x, es);
+    }
     DevState& s = x->s;
     CKV_CUDA(cudaMemcpy(s.mu, mu.data(), mu.size() * 4, cudaMemcpyHostToDevice));
     CKV_CUDA(cudaMemcpy(s.csize, size.data(), size.size() * 4, cudaMemcpyHostToDevice));
@@ -932,17 +996,20 @@ cudaError_t fetch_decode_rows(ckv_ctx* x, std::vector<int32_t>& deg, std::vector
 
 // graph g's token graph over [0, n_tok): the host rows, then the decode rows
 // the decode-time rows read back from the device are well formed: degrees
-// in [0, kappa], columns in [0, n_tok), finite non-negative weights (host
-// code indexes by them)
+// in [0, kappa], the row of position n_init + r linking only to ordinary
+// positions in [S, n_init + r), finite non-negative weights (host code
+// indexes by them)
 bool valid_decode_rows(const ckv_ctx* x, const std::vector<int32_t>& deg, const std::vector<int32_t>& col,
                        const std::vector<float>& w)
 {
     const int kap = x->d.kappa;
-    for (size_t r = 0; r < deg.size(); ++r) {
-        if (deg[r] < 0 || deg[r] > kap) return false;
-        for (int k = 0; k < deg[r]; ++k) {
-            const size_t i = r * (size_t)kap + (size_t)k;
-            if (col[i] < 0 || col[i] >= x->n_tok || !valid_weight(w[i])) return false;
+    const size_t rows = (size_t)(x->n_tok - x->d.n_init);
+    for (size_t i0 = 0; i0 < deg.size(); ++i0) {
+        if (deg[i0] < 0 || deg[i0] > kap) return false;
+        const int64_t hi = (int64_t)x->d.n_init + (int64_t)(rows ? i0 % rows : 0);
+        for (int k = 0; k < deg[i0]; ++k) {
+            const size_t i = i0 * (size_t)kap + (size_t)k;
+            if (col[i] < x->d.S || col[i] >= hi || !valid_weight(w[i])) return false;
         }
     }
     return true;
@@ -1024,6 +1091,7 @@ CKV_API ckv_status ckv_refresh(ckv_ctx* x, const void* K, double gamma, int32_t*
 
 CKV_API ckv_status ckv_graph_modularity(ckv_ctx* x, double gamma, double* q_host, void* stream)
 {
+    FaultScope fault;
     ckv_status cs = check_ctx(x);
     if (cs != CKV_OK) return cs;
     if (!q_host || !valid_gamma(gamma)) return CKV_ERR_INVALID_ARG;
@@ -1045,7 +1113,7 @@ CKV_API ckv_status ckv_graph_modularity(ckv_ctx* x, double gamma, double* q_host
         const size_t E = t.col.size();
         void* buf = nullptr;
         const size_t bytes = (size_t)(n + 1) * 8 + E * 8 + (size_t)n * 4 + ckv_modularity_workspace(d.n_comm + 1) + 64;
-        CKV_CUDA(cudaMalloc(&buf, bytes));
+        CKV_CUDA(dev_malloc(&buf, bytes));
         char* p = static_cast<char*>(buf);
         int64_t* drp = reinterpret_cast<int64_t*>(p);
         int32_t* dcol = reinterpret_cast<int32_t*>(p + (size_t)(n + 1) * 8);

@@ -13,11 +13,12 @@
 //
 // The array is kStaticScratchBytes per device and stays resident on every
 // GPU that loads the library until the process exits.  Every call shares
-// it: the call clears the counters it needs, copies the row lists in, and
-// launches on `stream`; calls whose work overlaps on the GPU (different
-// streams, or different host threads) race on it and must be serialised by
-// the caller.  The first call on a device looks up the array's device
-// address and sets the kernel's launch attributes.
+// it: the call clears the counters it needs, copies the row lists in,
+// launches on `stream`, reads the kernel's error word back and waits for
+// the stream, so it is synchronous and cannot be captured into a graph;
+// calls from different host threads race on the array and must be
+// serialised by the caller.  The first call on a device looks up the
+// array's device address and sets the kernel's launch attributes.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -155,12 +156,19 @@ CKV_API ckv_status ckv_attend_rows_static(const ckv_config* cfg, const void* q, 
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(sb + o_ctr, 0, (4 + 4 * (size_t)G) * 4, st);
-    // host -> device copies straight from the caller's buffers (pageable
-    // memory is staged before these calls return)
+    // host -> device copies straight from the caller's buffers; the call
+    // waits for the stream before it returns, so the buffers (pageable or
+    // page-locked) may be reused as soon as it does
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(sb + o_rT, n_rows_host, (size_t)G * 4, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess && max_rows > 0)
         e = cudaMemcpyAsync(sb + o_rtok, rows_host, (size_t)G * max_rows * 4, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = ckv::launch_step(s, d, q, K, V, n, out, st);
-    return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+    // the kernel's own checks (a row outside the cache, a wait that ran
+    // out) land in the error word
+    int err = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&err, s.err, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return CKV_ERR_CUDA;
+    return err ? (ckv_status)err : CKV_OK;
 }

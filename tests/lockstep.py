@@ -13,12 +13,18 @@ tolerances: bf16 inputs with fp32 accumulation, decisions on the float value):
 * edge weights: relative 2e-5 (float logits against the double oracle);
 * community state (centroids bit-exact, sizes, ascending members, edge rows)
   through the library's checkpoint record;
+* the number of exempt near-ties over a run is capped (max_exempt): a
+  systematic drift would otherwise be absorbed one re-synchronisation per
+  step;
 * optionally (recall_every > 0) the attention-mass recall of the step per
   query head against the oracle's (attended-row softmax statistics over
   dense ones): |r_gpu - r_ref| <= 1e-3 r_ref + 1e-6.
 """
 from __future__ import annotations
 
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -35,6 +41,14 @@ W_RTOL = 2e-5
 # a logit carries at most ~D 2^-23 |z| <= 3e-4 of accumulation error for the
 # workloads' |z| <= 20, which moves a probability by the same relative amount
 RECALL_RTOL, RECALL_ATOL = 1e-3, 1e-6
+# near-tie exemptions allowed per run: fp32 scores and logits flip a
+# decision only where the float gap is ~1e-6 relative, a few percent of the
+# graph-steps at most; anything above this is a real divergence
+EXEMPT_FRAC, EXEMPT_MIN = 0.05, 4
+
+
+def exempt_cap(graph_steps: int) -> int:
+    return max(EXEMPT_MIN, math.ceil(EXEMPT_FRAC * graph_steps))
 
 
 @dataclass
@@ -92,11 +106,27 @@ class Lockstep:
         self.oracle_edges = {g: [] for g in self.tracked}   # per decode row: (col, w)
         self.n = cfg.n0
         self.logs: list[StepLog] = []
+        # the tracked graphs' oracle steps are independent C calls (ctypes
+        # drops the GIL): run them on the host's cores
+        cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+        self.pool = ThreadPoolExecutor(max(1, min(len(self.tracked), cores)))
 
     def close(self):
         if getattr(self, "ctx", None):
             ckv.ckv_destroy(self.ctx)
             self.ctx = None
+        if getattr(self, "pool", None):
+            self.pool.shutdown()
+            self.pool = None
+
+    def n_exempt(self) -> int:
+        return sum(len(l.exempt) for l in self.logs)
+
+    def check_exempt_cap(self):
+        n_ex, gs = self.n_exempt(), len(self.logs) * len(self.tracked)
+        print(f"{self.cfg.name}: {len(self.logs)} steps x {len(self.tracked)} graphs, "
+              f"exempt near-ties {n_ex} (cap {exempt_cap(gs)})")
+        assert n_ex <= exempt_cap(gs), f"{n_ex} near-tie exemptions in {gs} graph-steps"
 
     # ---------------------------------------------------------------- step
     def step(self, i: int) -> StepLog:
@@ -124,11 +154,16 @@ class Lockstep:
             rec = rec_t.cpu().numpy()
         log = StepLog(i)
         resync = False
+
+        def oracle_step(g):
+            b, kvh, heads = cfg.graph_heads(g)
+            return oracle.decode_step(self.og[g], np.ascontiguousarray(self.wl.q[i, b, heads]),
+                                      self.wl.K[b, kvh], self.wl.V[b, kvh], n, cfg.n_sinks, kap,
+                                      cfg.budget)
+        ref_steps = dict(zip(self.tracked, self.pool.map(oracle_step, self.tracked)))
         for g in self.tracked:
             b, kvh, heads = cfg.graph_heads(g)
-            r = oracle.decode_step(self.og[g], np.ascontiguousarray(self.wl.q[i, b, heads]),
-                                   self.wl.K[b, kvh], self.wl.V[b, kvh], n, cfg.n_sinks, kap,
-                                   cfg.budget)
+            r = ref_steps[g]
             self.oracle_edges[g].append((r.edge_col.copy(), r.edge_w.copy()))
             gsel = set(sel[g, :n_sel[g]].tolist())
             if gsel != set(r.sel.tolist()):
