@@ -1027,7 +1027,7 @@ def main():
             pm, pe, note = prefill_oracle_time(synth.PREFILL, *prefill_qk, threads=cores)
             cpu["prefill"] = {"value": pe * 1e3, "unit": "ms (extrapolated)", "cores": cores,
                               "measured_s": pm, "sample": note,
-                              "gpu_over_cpu": (pe * 1e3) / prefill["ms"] if prefill else None}
+                              "gpu_speedup": (pe * 1e3) / prefill["ms"] if prefill else None}
     line = {
         "metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,

@@ -20,8 +20,11 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libckv.so")
+# CKV_DEBUG_BOUNDS=1 in the environment selects the range-checked build
+DEBUG_BOUNDS = os.environ.get("CKV_DEBUG_BOUNDS") == "1"
+LIB_PATH = os.path.join(HERE, "libckv_debug.so" if DEBUG_BOUNDS else "libckv.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "ckv.h")
+HEADER_DEBUG = os.path.join(os.path.dirname(HERE), "include", "ckv_debug.h")
 
 CKV_OK, CKV_ERR_INVALID_ARG, CKV_ERR_CAPACITY, CKV_ERR_OOM = 0, 1, 2, 3
 CKV_ERR_CUDA, CKV_ERR_TIMEOUT, CKV_ERR_STATE = 4, 5, 6
@@ -44,9 +47,9 @@ class CkvError(RuntimeError):
 _lib = None
 
 
-def declared_functions():
-    """Names of every function declared in include/ckv.h."""
-    text = open(HEADER).read()
+def declared_functions(header: str = HEADER):
+    """Names of every function declared in a header (default include/ckv.h)."""
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(ckv_[a-z_0-9]+)\s*\(", text)))
 
@@ -56,7 +59,7 @@ def lib() -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"libckv.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+        raise RuntimeError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run __graft_entry__.build()")
     L = ctypes.CDLL(LIB_PATH)
     P, I, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_int
     sz = ctypes.c_size_t
@@ -351,6 +354,19 @@ def ckv_dense_decode(ctx, q, K, V, n, out, lse=None, stream=None):
     """Dense decode attention over [0, n): out [B][H_q][D], lse [B][H_q] (optional)."""
     _check("ckv_dense_decode", lib().ckv_dense_decode(ctx, _dev(q), _dev(K), _dev(V), n, _dev(out), _dev(lse),
                                                       _stream(stream)))
+
+
+def ckv_debug_poke(ctx, what: int, g: int, c: int, r: int, value: int):
+    """Overwrite one int32 of the device community state (range-checked
+    build only): what 0 = member r of community c, 1 = community c's segment
+    offset."""
+    L = lib()
+    if not hasattr(L, "ckv_debug_poke"):
+        raise RuntimeError("ckv_debug_poke needs the range-checked build (CKV_DEBUG_BOUNDS=1)")
+    fn = L.ckv_debug_poke
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int32]
+    _check("ckv_debug_poke", fn(ctx, int(what), int(g), int(c), int(r), int(value)))
 
 
 def ckv_aux_bytes(ctx):

@@ -21,6 +21,9 @@
 
 #include "ckv_internal.cuh"
 #include "leiden.h"
+#ifdef CKV_DEBUG_BOUNDS
+#include "ckv_debug.h"
+#endif
 
 #define CKV_API extern "C" __attribute__((visibility("default")))
 
@@ -724,7 +727,8 @@ CKV_API ckv_status ckv_export_state(ckv_ctx* x, void* host_buf, size_t* bytes)
         size_t k = 0;
         for (size_t c = 0; c < Nc; ++c) {
             const int32_t sz = size[g * d.Nc + c], o = off[g * d.Nc + c];
-            if (k + sz > nmem) return CKV_ERR_STATE;
+            // the segment read back must lie inside the pool before host code reads it
+            if (sz < 0 || o < 0 || (int64_t)o + sz > d.P || k + sz > nmem) return CKV_ERR_STATE;
             memcpy(p + (k * 4), &pool[g * d.P + o], (size_t)sz * 4);
             k += sz;
         }
@@ -866,6 +870,30 @@ CKV_API ckv_status ckv_import_state(ckv_ctx* x, const void* host_buf, size_t byt
     x->initialized = 1;
     return CKV_OK;
 }
+
+#ifdef CKV_DEBUG_BOUNDS
+// Fault injection of the debug build only: overwrite one int32 of the
+// device community state, bypassing every host check, so that a test can
+// show the kernels' range checks turning a corrupt entry into CKV_ERR_STATE.
+CKV_API ckv_status ckv_debug_poke(ckv_ctx* x, int what, int g, int c, int r, int32_t value)
+{
+    if (!x || !x->initialized || g < 0 || g >= x->d.G || c < 0 || c >= x->d.n_comm) return CKV_ERR_INVALID_ARG;
+    if (what != 0 && what != 1) return CKV_ERR_INVALID_ARG;
+    CKV_CUDA(cudaSetDevice(x->cfg.device));
+    CKV_CUDA(cudaDeviceSynchronize());
+    const int64_t gi = (int64_t)g * x->d.Nc + c;
+    if (what == 1) {
+        CKV_CUDA(cudaMemcpy(x->s.coff + gi, &value, sizeof value, cudaMemcpyHostToDevice));
+        return CKV_OK;
+    }
+    int32_t size = 0, off = 0;
+    CKV_CUDA(cudaMemcpy(&size, x->s.csize + gi, sizeof size, cudaMemcpyDeviceToHost));
+    CKV_CUDA(cudaMemcpy(&off, x->s.coff + gi, sizeof off, cudaMemcpyDeviceToHost));
+    if (r < 0 || r >= size || off < 0 || (int64_t)off + r >= x->d.P) return CKV_ERR_INVALID_ARG;
+    CKV_CUDA(cudaMemcpy(x->s.pool + (int64_t)g * x->d.P + off + r, &value, sizeof value, cudaMemcpyHostToDevice));
+    return CKV_OK;
+}
+#endif
 
 CKV_API ckv_status ckv_aux_bytes(const ckv_ctx* x, size_t* aux_bytes, size_t* kv_bytes)
 {

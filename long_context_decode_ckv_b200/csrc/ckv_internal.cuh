@@ -164,4 +164,24 @@ cudaError_t launch_build_graph_grouped(int Hkv, int group, int n, int S, int kap
 // device error word: first error wins
 __device__ __forceinline__ void set_error(int* err, int code) { atomicCAS(err, 0, code); }
 
+// Range checks of the debug build (libckv_debug.so, compiled with
+// -DCKV_DEBUG_BOUNDS): CKV_IN_RANGE(i, lo, hi, err) is true when lo <= i <
+// hi and otherwise sets CKV_ERR_STATE in the error word and is false, so the
+// caller skips the access or redirects it in bounds.  They cover the
+// community segments (offset + size inside the member pool) wherever a
+// kernel reads or moves one, and the community an update writes.  In the
+// release build they compile to `true`.  Gathered token rows are checked in
+// both builds.
+__device__ __forceinline__ bool in_range_or_flag(int64_t i, int64_t lo, int64_t hi, int* err)
+{
+    if (i >= lo && i < hi) return true;
+    set_error(err, CKV_ERR_STATE);
+    return false;
+}
+#ifdef CKV_DEBUG_BOUNDS
+#define CKV_IN_RANGE(i, lo, hi, err) ::ckv::in_range_or_flag((int64_t)(i), (int64_t)(lo), (int64_t)(hi), (err))
+#else
+#define CKV_IN_RANGE(i, lo, hi, err) true
+#endif
+
 }  // namespace ckv

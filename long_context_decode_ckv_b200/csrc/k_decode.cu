@@ -225,8 +225,12 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelCand = 1024;     // boundary-bin communities ranked exactly
 
 // asks L2 to fetch n ints from p on (one prefetch per 128-byte line)
-__device__ __forceinline__ void prefetch_l2_range(const int32_t* p, int n)
+__device__ __forceinline__ void prefetch_l2_range(const int32_t* pool, int off, int n, int64_t P)
 {
+#ifdef CKV_DEBUG_BOUNDS
+    if (off < 0 || (int64_t)off + n > P) return;   // a bad segment: the row copy reports it
+#endif
+    const int32_t* p = pool + off;
     const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~(uintptr_t)127;
     const uintptr_t a1 = reinterpret_cast<uintptr_t>(p + n);
     for (uintptr_t a = a0; a < a1; a += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
         cmask = 0u;
 #pragma unroll
         for (int i = 0; i < E; ++i)
-            if (imask & (1u << i)) prefetch_l2_range(gpool + co[i], w[i]);
+            if (imask & (1u << i)) prefetch_l2_range(gpool, co[i], w[i], d.P);
     } else {
         // ---- 2./3. bucket passes until the boundary bin is small
         const float scale = (hi > lo) ? (float)kSelBins / (hi - lo) : 0.f;
@@ -357,13 +361,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
                 if (b > bs) {
                     imask |= 1u << i;
                     cmask &= ~(1u << i);
-                    prefetch_l2_range(gpool + co[i], w[i]);   // its members, for the row copy
+                    prefetch_l2_range(gpool, co[i], w[i], d.P);   // its members, for the row copy
                 } else if (b < bs) {
                     cmask &= ~(1u << i);
                 } else {
                     const int slot = atomicAdd(&sh_n, 1);
                     if (slot < kSelCand) { ckey[slot] = sel_key(v[i], c); cwt[slot] = w[i]; ccof[slot] = co[i]; }
-                    if (shift < 0) prefetch_l2_range(gpool + co[i], w[i]);   // likely kept too
+                    if (shift < 0) prefetch_l2_range(gpool, co[i], w[i], d.P);   // likely kept too
                 }
             }
             __syncthreads();
@@ -496,16 +500,20 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int k = k0 + u * kSelWarps;
-            tk[u] = (k < C && lane < pre[k + 1] - pre[k]) ? pool[cof[k] + lane] : 0;
+            const int sz = k < C ? pre[k + 1] - pre[k] : 0;
+            // the segment inside the pool (debug build; a bad one reads token 0)
+            const bool in = k < C && CKV_IN_RANGE(cof[k], 0, (int64_t)d.P - sz + 1, s.err);
+            tk[u] = (in && lane < sz) ? pool[cof[k] + lane] : 0;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int k = k0 + u * kSelWarps;
             if (k >= C) break;
             const int r0 = pre[k], sz = pre[k + 1] - r0, cc = cid[k];
+            const bool in = CKV_IN_RANGE(cof[k], 0, (int64_t)d.P - sz + 1, s.err);
             if (lane < sz) { rtok[r0 + lane] = tk[u]; rcomm[r0 + lane] = cc; }
             for (int j = 32 + lane; j < sz; j += 32) {   // communities longer than a warp
-                rtok[r0 + j] = pool[cof[k] + j];
+                rtok[r0 + j] = in ? pool[cof[k] + j] : 0;
                 rcomm[r0 + j] = cc;
             }
         }
@@ -719,6 +727,7 @@ struct WarpRows {
     const char* Vb;
     const int32_t* rtok;     // token of each kept-member row
     float* zrow;             // logits of the kept members, [row][HG]
+    int* err;                // the step's error word
     int a0, a1, S, T, R, t_new;
 };
 
@@ -729,7 +738,9 @@ __device__ __forceinline__ int row_token(const WarpRows& a, int r)
     return a.rtok[r - a.S];
 }
 
-// tokens of rows r .. r + TOKW - 1 of this warp into its smem window
+// tokens of rows r .. r + TOKW - 1 of this warp into its smem window (a
+// token outside [0, n) -- a corrupt row list -- sets the error word and
+// gathers row 0 instead, so no address outside the cache is formed)
 template <int TOKW>
 __device__ __forceinline__ void tokens_from(const WarpRows& a, int r, int* tokw, int lane)
 {
@@ -737,7 +748,12 @@ __device__ __forceinline__ void tokens_from(const WarpRows& a, int r, int* tokw,
 #pragma unroll
     for (int i = 0; i < TOKW / 32; ++i) {
         const int rr = r + 32 * i + lane;
-        tokw[32 * i + lane] = (rr < a.a1) ? row_token(a, rr) : 0;
+        int t = (rr < a.a1) ? row_token(a, rr) : 0;
+        if ((unsigned)t > (unsigned)a.t_new) {
+            set_error(a.err, CKV_ERR_STATE);
+            t = 0;
+        }
+        tokw[32 * i + lane] = t;
     }
     __syncwarp();
 }
@@ -1131,13 +1147,17 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
                 const int off0 = ne ? es.loff[src] : s.coff[gi];
                 const int top = s.pool_top[g];
                 int ok = 1, off = off0;
-                if (size == cp) {   // segment full: move it to the pool top with twice the room
+                // the community and its segment inside the pool (debug build)
+                if (!CKV_IN_RANGE(c, 0, d.Nc, s.err) || !CKV_IN_RANGE(size, 0, (int64_t)cp + 1, s.err) ||
+                    !CKV_IN_RANGE(off0, 0, d.P - cp + 1, s.err))
+                    ok = -1;
+                if (ok > 0 && size == cp) {   // segment full: move it to the pool top with twice the room
                     const int ncap = max(16, 2 * cp);
                     if ((int64_t)top + ncap > d.P) ok = 0;
                     else { s.pool_top[g] = top + ncap; off = top; }
                 }
                 if (!ok) set_error(s.err, CKV_ERR_CAPACITY);
-                sflag[0] = c; sflag[1] = ok; sflag[2] = off; sflag[3] = size; sflag[4] = off0; sflag[5] = ne;
+                sflag[0] = c; sflag[1] = ok > 0; sflag[2] = off; sflag[3] = size; sflag[4] = off0; sflag[5] = ne;
             }
         }
     }
@@ -1306,6 +1326,7 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
             a.Vb = reinterpret_cast<const char*>(V) + kvbase * RB;
             a.rtok = s.rtok + (int64_t)g * d.NM;
             a.zrow = s.zrow + (int64_t)g * d.NM * HG;
+            a.err = s.err;
             a.a0 = pc.r0 + (int)((int64_t)warp * nrows / kAttWarps);
             a.a1 = pc.r0 + (int)((int64_t)(warp + 1) * nrows / kAttWarps);
             a.S = d.S;

@@ -1479,13 +1479,17 @@ __device__ void finish_graph(const DevState& s, const Dims& d, int g, int R, con
         const int size = ne ? mi.sflag[3] : s.csize[gi];
         const int off0 = ne ? mi.sflag[4] : s.coff[gi];
         int ok = 1, off = off0;
-        if (size == cp) {   // segment full: move it to the pool top with twice the room
+        // the community and its segment inside the pool (debug build)
+        if (!CKV_IN_RANGE(c, 0, d.Nc, s.err) || !CKV_IN_RANGE(size, 0, (int64_t)cp + 1, s.err) ||
+            !CKV_IN_RANGE(off0, 0, d.P - cp + 1, s.err))
+            ok = -1;
+        if (ok > 0 && size == cp) {   // segment full: move it to the pool top with twice the room
             const int ncap = max(16, 2 * cp);
             if ((int64_t)top + ncap > d.P) ok = 0;
             else { s.pool_top[g] = top + ncap; off = top; }
         }
         if (!ok) set_error(s.err, CKV_ERR_CAPACITY);
-        mi.sflag[1] = ok; mi.sflag[2] = off; mi.sflag[3] = size; mi.sflag[4] = off0; mi.sflag[6] = cp;
+        mi.sflag[1] = ok > 0; mi.sflag[2] = off; mi.sflag[3] = size; mi.sflag[4] = off0; mi.sflag[6] = cp;
     }
     __syncthreads();
     if (!mi.sflag[1]) return;

@@ -43,8 +43,9 @@ W_RTOL = 2e-5
 RECALL_RTOL, RECALL_ATOL = 1e-3, 1e-6
 # near-tie exemptions allowed per run: fp32 scores and logits flip a
 # decision only where the float gap is ~1e-6 relative, a few percent of the
-# graph-steps at most; anything above this is a real divergence
-EXEMPT_FRAC, EXEMPT_MIN = 0.05, 4
+# graph-steps at most (the sweep and Qwen3-8B runs see 0-1 in 512-1024);
+# anything above this is a real divergence
+EXEMPT_FRAC, EXEMPT_MIN = 0.01, 2
 
 
 def exempt_cap(graph_steps: int) -> int:

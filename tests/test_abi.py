@@ -25,10 +25,25 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(raw, name), f"libckv.so does not export {name}"
 
 
+def _exports(path):
+    out = os.popen(f"nm -D --defined-only {path}").read().split("\n")
+    return {ln.split()[-1] for ln in out if " T ckv_" in ln}
+
+
 def test_exports_nothing_undeclared(L):
-    out = os.popen(f"nm -D --defined-only {ckv.LIB_PATH}").read().split("\n")
-    ours = {ln.split()[-1] for ln in out if " T ckv_" in ln}
-    assert ours == set(ckv.declared_functions())
+    assert _exports(ckv_build.LIB) == set(ckv.declared_functions())
+
+
+def test_range_checked_build_exports_both_headers():
+    # libckv_debug.so: every ckv.h entry point plus the fault injection of
+    # ckv_debug.h, which the release library does not export
+    ckv_build.build(debug=True)
+    dbg = set(ckv.declared_functions(ckv.HEADER_DEBUG)) - set(ckv.declared_functions())
+    assert dbg == {"ckv_debug_poke"}
+    assert _exports(ckv_build.LIB_DEBUG) == set(ckv.declared_functions()) | dbg
+    assert not (_exports(ckv_build.LIB) & dbg)
+    raw = ctypes.CDLL(ckv_build.LIB_DEBUG)
+    assert hasattr(raw, "ckv_debug_poke")
 
 
 def good_config():
