@@ -291,6 +291,51 @@ def reference_arm(args, rank, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+class Stepper:
+    """Decode steps over layer replicas: ckv_decode_step on the caller's
+    stream, ckv_assign_update (the edges, assignment and update kernel) on a
+    side stream, so that it overlaps the next replica's step the way a
+    decoder overlaps it with the next layer; a replica's next step waits for
+    its previous update (events; also inside CUDA graph capture)."""
+
+    def __init__(self, reps, q, out, cfg, dev, side=True):
+        import torch
+        import long_context_decode_ckv_b200 as ckv
+        self.ckv, self.reps, self.q, self.out, self.cfg = ckv, reps, q, out, cfg
+        self.side = torch.cuda.Stream(device=dev) if side else None
+        self.ev_a = [torch.cuda.Event() for _ in reps]
+        self.ev_u = [torch.cuda.Event() for _ in reps]
+        self.pending = [False] * len(reps)
+
+    def step(self, s, st):
+        ckv, cfg = self.ckv, self.cfg
+        r = s % len(self.reps)
+        rep = self.reps[r]
+        i = rep["i"]
+        n = cfg.n0 + i + 1
+        if self.side is None:   # both calls on the caller's stream
+            ckv.ckv_decode_step(rep["ctx"], self.q[i], rep["K"], rep["V"], n, self.out, st)
+            ckv.ckv_assign_update(rep["ctx"], rep["K"], n, st)
+            rep["i"] = i + 1
+            return
+        if self.pending[r]:
+            st.wait_event(self.ev_u[r])
+        ckv.ckv_decode_step(rep["ctx"], self.q[i], rep["K"], rep["V"], n, self.out, st)
+        self.ev_a[r].record(st)
+        self.side.wait_event(self.ev_a[r])
+        ckv.ckv_assign_update(rep["ctx"], rep["K"], n, self.side)
+        self.ev_u[r].record(self.side)
+        self.pending[r] = True
+        rep["i"] = i + 1
+
+    def join(self, st):
+        """The caller's stream waits for every update still outstanding."""
+        for r, p in enumerate(self.pending):
+            if p:
+                st.wait_event(self.ev_u[r])
+                self.pending[r] = False
+
+
 def upload_graph(g, stream):
     """Uploads an instantiated CUDA graph to the device ahead of its first
     launch (a one-time setup cost, like the instantiation), so that the
@@ -411,25 +456,21 @@ def decode_rate(cfg, wl, warmup, steps, replicas, profile_steps=0):
             ckv.ckv_init_communities(ctx, wl.labels, 0, cfg.n_comm, K, cfg.n0)
         aux, kvb = ckv.ckv_aux_bytes(reps[0]["ctx"])
         out = torch.empty((cfg.batch, cfg.n_q_heads, cfg.head_dim), dtype=torch.float32, device=dev)
-
-        def step(s, st):
-            r = reps[s % L]
-            i = r["i"]
-            ckv.ckv_decode_step(r["ctx"], q[i], r["K"], r["V"], cfg.n0 + i + 1, out, st)
-            ckv.ckv_assign_update(r["ctx"], r["K"], cfg.n0 + i + 1, st)
-            r["i"] = i + 1
+        stepper = Stepper(reps, q, out, cfg, dev)
 
         def graph_of(first, count):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, capture_error_mode="relaxed"):
                 cap = torch.cuda.current_stream(dev)
                 for s in range(first, first + count):
-                    step(s, cap)
+                    stepper.step(s, cap)
+                stepper.join(cap)
             upload_graph(g, stream)
             return g
 
         for s in range(warmup):
-            step(s, stream)
+            stepper.step(s, stream)
+        stepper.join(stream)
         torch.cuda.synchronize(dev)
         g = graph_of(warmup, steps)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -473,10 +514,18 @@ def decode_rate(cfg, wl, warmup, steps, replicas, profile_steps=0):
            "hbm_frac_of_measured": step_bytes / (ms / 1e3) / 1e9 / peak, "gpu_launches": launches * steps,
            "aux_bytes": aux, "kv_bytes": kvb, "aux_over_kv": aux / kvb}
     if avg is not None:
-        res["kernel_ms_per_step"] = dict(zip(["score", "select", "attend_edges_update", "step_close"], avg)) \
-            if launches == 3 else {"step": avg[0], "step_close": avg[3]}
+        res["kernel_ms_per_step"] = {k: v for k, v in zip(kernel_names(launches), avg) if k != "-"}
         res["roofline"] = roofline_of(cfg, T_mean, avg, launches, peak, peak_kind)
     return res
+
+
+def kernel_names(launches):
+    """Names of the four per-kernel spans ckv_profile_end reports."""
+    if launches == 1:
+        return ["step", "-", "-", "step_close"]
+    if launches == 4:
+        return ["score", "select", "attend_output", "edges_assign_update"]
+    return ["score", "select", "attend_edges_update", "step_close"]
 
 
 def roofline_of(cfg, T_mean, avg, launches, peak, peak_kind):
@@ -743,6 +792,9 @@ def main():
                     help="dense decode comparator launches timed after the sparse steps (0 = none)")
     ap.add_argument("--sweep", action="store_true",
                     help="decode steps/s at every point of the batch-16 (n, budget) sweep instead")
+    ap.add_argument("--update-stream", default="side", choices=["side", "main"],
+                    help="stream of ckv_assign_update: a side stream overlapping the next replica's step "
+                         "(default), or the step's own stream")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the prefill and Llama per-head measurements of the default line")
     args = ap.parse_args()
@@ -809,17 +861,12 @@ def main():
     out = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     sel_tok = np.zeros(cfg.n_graphs, np.int32)
-
-    def step(s, st):
-        r = reps[s % L]
-        i = r["i"]
-        n = cfg.n0 + i + 1
-        ckv.ckv_decode_step(r["ctx"], q[i], r["K"], r["V"], n, out, st)
-        ckv.ckv_assign_update(r["ctx"], r["K"], n, st)
-        r["i"] = i + 1
+    stepper = Stepper(reps, q, out, cfg, dev, side=args.update_stream == "side")
+    step = stepper.step
 
     for s in range(args.warmup):
         step(s, stream)
+    stepper.join(stream)
     torch.cuda.synchronize(dev)
 
     def capture(first, count):
@@ -834,6 +881,7 @@ def main():
                 cap = torch.cuda.current_stream(dev)
                 for s in range(first, first + count):
                     step(s, cap)
+                stepper.join(cap)
             try:
                 upload_graph(g, stream)
             except Exception as exc:   # the first replay then uploads it
@@ -843,6 +891,7 @@ def main():
             print(f"CUDA graph capture failed ({exc}); timing eager launches", file=sys.stderr)
             for r, i in zip(reps, saved):
                 r["i"] = i
+            stepper.pending = [False] * len(reps)
             return None
 
     def run(first, count, g):
@@ -851,6 +900,7 @@ def main():
         else:
             for s in range(first, first + count):
                 step(s, stream)
+            stepper.join(stream)
 
     # timed steps: no profiling events inside
     s_timed = args.warmup
@@ -1005,8 +1055,7 @@ def main():
     avg, roofline = None, None
     if kern_ms is not None and kern_steps:
         per = [k / kern_steps for k in kern_ms]
-        avg = ({"step": per[0], "step_close": per[3]} if launches_per_step == 1 else
-               dict(zip(["score", "select", "attend_edges_update", "step_close"], per)))
+        avg = {k: v for k, v in zip(kernel_names(launches_per_step), per) if k != "-"}
         roofline = roofline_of(cfg, T_mean, per, launches_per_step, peak, peak_kind)
 
     # the oracle on the host: all cores (one thread per graph), one core,
@@ -1036,7 +1085,10 @@ def main():
         "config": {"workload": WORKLOAD, "graphs": cfg.n_graphs, "layer_replicas": L,
                    "l2": f"{L} layer replicas rotated (inputs larger than L2), no flush",
                    "parallelism": "replicas" if world > 1 else "single",
-                   "launch": launch_mode},
+                   "launch": launch_mode,
+                   "update": ("inside the step's last kernel" if launches_per_step != 4 else
+                              "side stream: each ckv_assign_update overlaps the next replica's step"
+                              if args.update_stream == "side" else "own kernel on the step's stream")},
         "hbm_gbs": gbs, "hbm_frac_of_8000": gbs / NOMINAL_HBM_GBS, "hbm_frac_of_measured": gbs / peak,
         "algorithmic_bytes_per_step": step_bytes, "mean_tokens_kept": T_mean,
         "kernel_ms_per_step": avg,

@@ -242,10 +242,20 @@ ckv_status ckv_init_communities(ckv_ctx* ctx, const int32_t* labels, int labels_
 ckv_status ckv_decode_step(ckv_ctx* ctx, const void* q, const void* K, const void* V, int n,
                            float* out, void* stream);
 
-/* Closes the decode step begun by ckv_decode_step with the same n (the
- * edges, assignment and update already ran inside that call's last kernel;
- * this call launches nothing).  K must be non-NULL.
- * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no preceding decode step). */
+/* Closes the decode step begun by ckv_decode_step with the same n: the new
+ * token's top-kappa edges over the kept members, its community by the
+ * weighted vote of their communities, and the centroid update and append
+ * (Figure 1 caption, step (3); abstract, "a local update rule").  Launches
+ * one kernel (one CTA per graph) on `stream` at the lowest stream priority;
+ * it reads the new token's key from row n-1 of K and what the step's
+ * attention kernel left.  The step's output needs none of it, so a caller
+ * may run this call on a second stream, overlapping the next layer's work;
+ * it must then make the context's next ckv_decode_step wait for it (an
+ * event recorded on that stream after this call).  With CKV_STEP=fused or
+ * CKV_UPDATE=inline in the environment at ckv_create, the step's last
+ * kernel already did this work and the call launches nothing.
+ * Errors: CKV_ERR_INVALID_ARG, CKV_ERR_STATE (no preceding decode step),
+ * CKV_ERR_CUDA; a step that failed on the device changes no state here. */
 ckv_status ckv_assign_update(ckv_ctx* ctx, const void* K, int n, void* stream);
 
 /* One whole decode step from host memory: copies the new token's key and
@@ -264,10 +274,11 @@ ckv_status ckv_decode_host(ckv_ctx* ctx, const void* q_host, const void* k_new_h
 ckv_status ckv_last_error(ckv_ctx* ctx);
 
 /* Kernel launches of one decode step (ckv_decode_step plus
- * ckv_assign_update) of this context: 3 by default (scoring, selection,
- * attention as separate kernels), 1 when the environment variable
- * CKV_STEP=fused was set at ckv_create (one persistent kernel).  -1 for
- * NULL. */
+ * ckv_assign_update) of this context: 4 by default (scoring, selection,
+ * attention, then edges/assignment/update), 3 with CKV_UPDATE=inline (the
+ * attention kernel also runs the last part), 1 when CKV_STEP=fused (one
+ * persistent kernel); the environment variables are read at ckv_create.
+ * -1 for NULL. */
 int ckv_step_launches(const ckv_ctx* ctx);
 
 /* Failure detection: the bound of the fused step's cross-CTA waits (a
@@ -323,10 +334,11 @@ ckv_status ckv_dense_decode(ckv_ctx* ctx, const void* q, const void* K, const vo
  * ckv_profile_begin, every ckv_decode_step / ckv_assign_update records CUDA
  * events on its stream around each of its kernels; ckv_profile_end
  * synchronises, writes the summed milliseconds of ms[0] centroid scoring,
- * ms[1] community selection, ms[2] gather + attention + edges + assignment
- * + update (one kernel) and ms[3] the rest of the step (ckv_assign_update,
- * which launches nothing), and the number of steps they cover, and stops
- * recording.  Both are host calls; begin is not
+ * ms[1] community selection, ms[2] gather + attention + output (with
+ * CKV_UPDATE=inline also the edges, assignment and update) and ms[3]
+ * ckv_assign_update's edges + assignment + update kernel (0 when it
+ * launches nothing); with CKV_STEP=fused ms[0] is the whole step.  Also
+ * the number of steps they cover; stops recording.  Both are host calls; begin is not
  * allowed while a step is half done.  Errors: CKV_ERR_INVALID_ARG,
  * CKV_ERR_STATE, CKV_ERR_CUDA. */
 ckv_status ckv_profile_begin(ckv_ctx* ctx);

@@ -356,6 +356,12 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
         const char* v = getenv("CKV_STEP");
         d.fused = v && v[0] == 'f';
     }
+    {   // the three-kernel step leaves the edges, assignment and update to
+        // ckv_assign_update's own kernel, unless CKV_UPDATE=inline (then the
+        // attention kernel's last slice of each graph runs them)
+        const char* v = getenv("CKV_UPDATE");
+        d.defer_update = !d.fused && !(v && v[0] == 'i');
+    }
     d.api = ckv::step_api(d.S, d.budget);
     d.spg = 1;
     d.rows_given = 0;
@@ -544,9 +550,10 @@ CKV_API ckv_status ckv_assign_update(ckv_ctx* x, const void* K, int n, void* str
     if (!x->pending || n != x->pending_n) return CKV_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     CKV_CUDA(cudaSetDevice(x->cfg.device));
-    // the attention kernel of ckv_decode_step already assigned the token and
-    // updated its community (it reads the new key from the same K)
+    // the edges, assignment and update: their own kernel, or already done by
+    // the step's last kernel (the fused step, or CKV_UPDATE=inline)
     CKV_CUDA(prof_mark(x, 4, st));
+    if (x->d.defer_update) CKV_CUDA(ckv::launch_update(x->s, x->d, K, n, st));
     CKV_CUDA(prof_mark(x, 5, st));
     x->pending = 0;
     x->n_tok = n;
@@ -626,7 +633,10 @@ CKV_API ckv_status ckv_last_error(ckv_ctx* x)
     return e;
 }
 
-CKV_API int ckv_step_launches(const ckv_ctx* x) { return x ? (x->d.fused ? 1 : 3) : -1; }
+CKV_API int ckv_step_launches(const ckv_ctx* x)
+{
+    return x ? (x->d.fused ? 1 : 3 + (x->d.defer_update ? 1 : 0)) : -1;
+}
 
 CKV_API ckv_status ckv_set_wait_limit(ckv_ctx* x, unsigned polls)
 {

@@ -89,6 +89,7 @@ struct Dims {
     int nSM;                 // multiprocessors of the device
     int n_comm;              // communities in use (set at init)
     int n_init;              // first decode position (edge store row 0)
+    int defer_update;        // edges, assignment and update run in k_update (ckv_assign_update)
     int fuse_assign;         // the attention kernel also assigns the new token and updates
     int att_aligned;         // attention CTAs split graph by graph (else the rows evenly)
     int pdl;                 // programmatic dependent launch: 0 off, 1 trigger at kernel start, 2 after the main work
@@ -107,9 +108,13 @@ struct Dims {
 // kernel launchers (k_decode.cu)
 cudaError_t launch_score(const DevState& s, const Dims& d, const void* q, cudaStream_t st);
 cudaError_t launch_select(const DevState& s, const Dims& d, cudaStream_t st);
-// attention, edges and (d.fuse_assign) the assignment and update of the step
+// attention and output, then (unless d.defer_update) the edges and (with
+// d.fuse_assign) the assignment and update of the step
 cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const void* K,
                           const void* V, int n, float* out, cudaStream_t st);
+// the step's edges, assignment and update when d.defer_update (one CTA per
+// graph, at the lowest stream priority)
+cudaError_t launch_update(const DevState& s, const Dims& d, const void* K, int n, cudaStream_t st);
 size_t select_smem_bytes(int n_comm, int budget);
 // sets the kernels' shared-memory limits on the current device; then the
 // number of co-resident CTAs of the attention kernel (0 on error)

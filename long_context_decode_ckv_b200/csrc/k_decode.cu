@@ -84,12 +84,23 @@ struct ScoreSmem {
     int abort;
 };
 
+// whether the step already failed, read once for the whole CTA (every
+// thread then takes the same branch; another CTA may set the word meanwhile)
+__device__ __forceinline__ bool step_failed(const int* err)
+{
+    __shared__ int e;
+    __syncthreads();
+    if (threadIdx.x == 0) e = *(volatile const int*)err;
+    __syncthreads();
+    return e != 0;
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kScoreThreads, 1) k_score(DevState s, Dims d, const void* __restrict__ q)
 {
     pdl_wait();
     if (d.pdl) pdl_trigger();
-    if (*(volatile int*)s.err) return;
+    if (step_failed(s.err)) return;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -259,7 +270,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
 {
     pdl_wait();
     if (d.pdl == 1) pdl_trigger();
-    if (*(volatile int*)s.err) return;
+    if (step_failed(s.err)) return;
     extern __shared__ __align__(16) unsigned char smem_sel[];
     __shared__ int r_w[kSelWarps];
     __shared__ unsigned long long r_kmin[kSelWarps], r_kmax[kSelWarps];
@@ -1029,80 +1040,20 @@ __device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __
 // A graph's last slice to finish: merge the slices' partials, rank the
 // edges, and (when fused) assign the new token and update its community.
 // Runs with the whole CTA; red / smem scratch is free.
+// The new token's edges (the top kappa of w = sum_h exp(z - M_h) / L_h over
+// the kept members), its assignment and the community update, for graph g
+// of the step whose output merge left sM (max) and sL (1 / sum) per head.
+// er: the first round of kept members' logits, loaded by the caller; kv:
+// this thread's value of the new token's key (threads < D).
 template <int HG>
-__device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, int g, int nc, int R,
-                                             const void* __restrict__ K, int n, float* __restrict__ out,
-                                             unsigned char* scratch, float* sM, float* sL, int* sflag)
+__device__ __forceinline__ void edges_assign_update(const DevState& s, const Dims& d, int g, int T, int n, float kv,
+                                                    EdgeRows<HG>& er, unsigned char* scratch, const float* sM,
+                                                    const float* sL, int* sflag)
 {
     constexpr int NT = kAttWarps * 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int b, h0, kvh;
-    graph_heads(d, g, b, h0, kvh);
-    const int T = R - d.S - 1;
     const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
     const float* zrow = s.zrow + (int64_t)g * d.NM * HG;
-    const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
-    const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
-
-    EdgeRows<HG> er;   // the first round of kept members, loaded under the output merge
-    edges_load<HG>(d, zrow, rtok, T, 0, er);
-    float kv = 0.f;    // the new token's key, for the update
-    if (d.fuse_assign && tid < kD) {
-        const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + (n - 1)) * kD;
-        kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
-    }
-    // ---- output: every value merged online over the slices; the thread of
-    // a head's first value also leaves that head's max and 1 / sum.  A
-    // thread's IPT values take their loads of a batch of slices together.
-    {
-        constexpr int IPT = (HG * kD + NT - 1) / NT;              // values per thread
-        constexpr int U = (8 / IPT > 1) ? 8 / IPT : 2;            // slices per batch
-        float M[IPT], Ls[IPT], o[IPT];
-#pragma unroll
-        for (int it = 0; it < IPT; ++it) { M[it] = -INFINITY; Ls[it] = 0.f; o[it] = 0.f; }
-        for (int j0 = 0; j0 < nc; j0 += U) {
-            float2 mj[IPT][U];
-            float oj[IPT][U];
-#pragma unroll
-            for (int it = 0; it < IPT; ++it) {
-                const int i = tid + it * NT;
-                const int h = i / kD;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const bool ok = j0 + u < nc && i < HG * kD;
-                    mj[it][u] = ok ? __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)(j0 + u) * HG + h) * 2))
-                                   : make_float2(-INFINITY, 0.f);
-                    oj[it][u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
-                }
-            }
-#pragma unroll
-            for (int it = 0; it < IPT; ++it)
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    if (mj[it][u].x == -INFINITY) continue;
-                    const float mn = fmaxf(M[it], mj[it][u].x);
-                    const float a = (M[it] == -INFINITY) ? 0.f : __expf(M[it] - mn), c = __expf(mj[it][u].x - mn);
-                    o[it] = o[it] * a + oj[it][u] * c;
-                    Ls[it] = Ls[it] * a + mj[it][u].y * c;
-                    M[it] = mn;
-                }
-        }
-#pragma unroll
-        for (int it = 0; it < IPT; ++it) {
-            const int i = tid + it * NT;
-            if (i >= HG * kD) continue;
-            const int h = i / kD;
-            out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o[it] / Ls[it];
-            if (i % kD == 0) {
-                sM[h] = M[it];
-                sL[h] = 1.f / Ls[it];
-                if (s.sel_ml)
-                    *reinterpret_cast<float2*>(s.sel_ml + 2 * ((int64_t)b * d.Hq + h0 + h)) = make_float2(M[it], Ls[it]);
-            }
-        }
-    }
-    __syncthreads();
-    // ---- edges: the top kappa of w = sum_h exp(z - M_h) / L_h over the kept members
     EdgeScratch& es = *reinterpret_cast<EdgeScratch*>(scratch);
     cta_edges<HG>(s, d, g, zrow, rtok, T, sM, sL, es, er, d.fuse_assign != 0);
     if (warp == 0) {
@@ -1194,6 +1145,86 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
     }
 }
 
+
+template <int HG>
+__device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, int g, int nc, int R,
+                                             const void* __restrict__ K, int n, float* __restrict__ out,
+                                             unsigned char* scratch, float* sM, float* sL, int* sflag)
+{
+    constexpr int NT = kAttWarps * 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int b, h0, kvh;
+    graph_heads(d, g, b, h0, kvh);
+    const int T = R - d.S - 1;
+    const int32_t* rtok = s.rtok + (int64_t)g * d.NM;
+    const float* zrow = s.zrow + (int64_t)g * d.NM * HG;
+    const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
+    const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
+
+    // inline update: the first round of kept members and the new token's
+    // key are loaded under the output merge (deferred: k_update loads them)
+    const bool upd = !d.defer_update;
+    EdgeRows<HG> er;
+    if (upd) edges_load<HG>(d, zrow, rtok, T, 0, er);
+    float kv = 0.f;
+    if (upd && d.fuse_assign && tid < kD) {
+        const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + (n - 1)) * kD;
+        kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
+    }
+    // ---- output: every value merged online over the slices; the thread of
+    // a head's first value also leaves that head's max and 1 / sum.  A
+    // thread's IPT values take their loads of a batch of slices together.
+    {
+        constexpr int IPT = (HG * kD + NT - 1) / NT;              // values per thread
+        constexpr int U = (8 / IPT > 1) ? 8 / IPT : 2;            // slices per batch
+        float M[IPT], Ls[IPT], o[IPT];
+#pragma unroll
+        for (int it = 0; it < IPT; ++it) { M[it] = -INFINITY; Ls[it] = 0.f; o[it] = 0.f; }
+        for (int j0 = 0; j0 < nc; j0 += U) {
+            float2 mj[IPT][U];
+            float oj[IPT][U];
+#pragma unroll
+            for (int it = 0; it < IPT; ++it) {
+                const int i = tid + it * NT;
+                const int h = i / kD;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const bool ok = j0 + u < nc && i < HG * kD;
+                    mj[it][u] = ok ? __ldcg(reinterpret_cast<const float2*>(pmg + ((int64_t)(j0 + u) * HG + h) * 2))
+                                   : make_float2(-INFINITY, 0.f);
+                    oj[it][u] = ok ? __ldcg(pog + (int64_t)(j0 + u) * HG * kD + i) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int it = 0; it < IPT; ++it)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (mj[it][u].x == -INFINITY) continue;
+                    const float mn = fmaxf(M[it], mj[it][u].x);
+                    const float a = (M[it] == -INFINITY) ? 0.f : __expf(M[it] - mn), c = __expf(mj[it][u].x - mn);
+                    o[it] = o[it] * a + oj[it][u] * c;
+                    Ls[it] = Ls[it] * a + mj[it][u].y * c;
+                    M[it] = mn;
+                }
+        }
+#pragma unroll
+        for (int it = 0; it < IPT; ++it) {
+            const int i = tid + it * NT;
+            if (i >= HG * kD) continue;
+            const int h = i / kD;
+            out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o[it] / Ls[it];
+            if (i % kD == 0) {
+                sM[h] = M[it];
+                sL[h] = 1.f / Ls[it];
+                if (s.sel_ml)
+                    *reinterpret_cast<float2*>(s.sel_ml + 2 * ((int64_t)b * d.Hq + h0 + h)) = make_float2(M[it], Ls[it]);
+            }
+        }
+    }
+    __syncthreads();
+    if (upd) edges_assign_update<HG>(s, d, g, T, n, kv, er, scratch, sM, sL, sflag);
+}
+
 // CTA work: the graphs' rows laid end to end (graph-major, each graph's
 // rows in its own order) are split evenly over the CTAs; a CTA's share is
 // one or more pieces, each a contiguous run of one graph's rows.
@@ -1264,9 +1295,7 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
     } else {
         for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
     }
-    const int errv = *(volatile int*)s.err;
-    __syncthreads();
-    if (errv) return;
+    if (step_failed(s.err)) return;
     for (int done = 0;; done += kMaxPieces) {
         if (!aligned && warp == 0) {
             auto rows_of = [&](int g) -> int {
@@ -1388,6 +1417,41 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
     }
 }
 
+// The deferred part of a decode step, launched by ckv_assign_update: one CTA
+// per graph computes the new token's edges, assignment and community update
+// from what the step's attention kernel left -- each head's softmax max and
+// sum over the attended rows (sel_ml), the kept members' logits (zrow) and
+// rows (rtok, rcomm).  A step that already failed changes no state.
+template <int HG>
+__global__ void __launch_bounds__(kAttWarps * 32, 1) k_update(DevState s, Dims d, const void* __restrict__ K, int n)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    float* sM = reinterpret_cast<float*>(smem + sizeof(EdgeScratch));   // [8]
+    float* sL = sM + 8;                                                  // [8]
+    int* sflag = reinterpret_cast<int*>(sL + 8);                         // [8]
+    const int g = blockIdx.x, tid = threadIdx.x;
+    if (step_failed(s.err)) return;
+    int b, h0, kvh;
+    graph_heads(d, g, b, h0, kvh);
+    const int T = __ldcg(s.meta + (int64_t)g * M_COUNT + M_ROWS) - d.S - 1;
+    EdgeRows<HG> er;
+    edges_load<HG>(d, s.zrow + (int64_t)g * d.NM * HG, s.rtok + (int64_t)g * d.NM, T, 0, er);
+    float kv = 0.f;
+    if (tid < kD) {
+        const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + (n - 1)) * kD;
+        kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
+    }
+    if (tid < HG) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(s.sel_ml) + ((int64_t)b * d.Hq + h0 + tid));
+        sM[tid] = ml.x;
+        sL[tid] = 1.f / ml.y;
+    }
+    __syncthreads();
+    edges_assign_update<HG>(s, d, g, T, n, kv, er, smem, sM, sL, sflag);
+}
+
+constexpr size_t kUpdateSmem = sizeof(EdgeScratch) + 24 * 4;
+
 // new token's K and V rows: staging [B][H_kv][D] -> cache row `row`
 __global__ void k_append(const uint32_t* __restrict__ knew, const uint32_t* __restrict__ vnew,
                          uint32_t* __restrict__ K, uint32_t* __restrict__ V, int64_t NM, int row, int words)
@@ -1400,9 +1464,26 @@ __global__ void k_append(const uint32_t* __restrict__ knew, const uint32_t* __re
     }
 }
 
-// Launch with programmatic stream serialization (when d.pdl): the kernel may
-// begin launching while the previous kernel of the stream finishes; every
-// decode kernel starts with pdl_wait.  Cooperative when asked.
+// the stream priority range {lowest, highest} (the same on every device)
+struct PriorityRange {
+    int lo = 0, hi = 0;
+    PriorityRange()
+    {
+        if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) lo = hi = 0;
+    }
+};
+inline void priority_range(int& lo, int& hi)
+{
+    static const PriorityRange r;   // fetched once, on first use
+    lo = r.lo;
+    hi = r.hi;
+}
+
+// The decode kernels run at the highest priority (the step's output waits
+// on them; the deferred update runs at the lowest), with programmatic
+// stream serialization when d.pdl: the kernel may begin launching while
+// the previous kernel of the stream finishes; every decode kernel starts
+// with pdl_wait.
 template <typename... P, typename... A>
 cudaError_t launch_ex(const Dims& d, void (*fn)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                       A&&... args)
@@ -1412,11 +1493,15 @@ cudaError_t launch_ex(const Dims& d, void (*fn)(P...), dim3 grid, dim3 block, si
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int lo = 0, hi = 0;
+    priority_range(lo, hi);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributePriority;
+    attr[0].val.priority = hi;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = d.pdl ? 1 : 0;
+    cfg.numAttrs = d.pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, fn, std::forward<A>(args)...);
 }
 
@@ -1436,6 +1521,12 @@ template <bool BF16, int HG>
 void* attend_fn()
 {
     return reinterpret_cast<void*>(k_attend<BF16, HG>);
+}
+
+template <int HG>
+void* update_fn()
+{
+    return reinterpret_cast<void*>(k_update<HG>);
 }
 
 }  // namespace
@@ -1506,7 +1597,10 @@ cudaError_t prepare_kernels(const Dims& d)
         constexpr int HG = decltype(hgc)::value;
         void* fn = d.bf16 ? attend_fn<true, HG>() : attend_fn<false, HG>();
         const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
-        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaError_t e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e2 == cudaSuccess)
+            e2 = cudaFuncSetAttribute(update_fn<HG>(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUpdateSmem);
+        return e2;
     });
 }
 
@@ -1536,6 +1630,28 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
                              out);
         return launch_ex(d, k_attend<false, HG>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K, V, n,
                          out);
+    });
+}
+
+cudaError_t launch_update(const DevState& s, const Dims& d, const void* K, int n, cudaStream_t st)
+{
+    return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
+        constexpr int HG = decltype(hgc)::value;
+        // the lowest stream priority: where it shares the GPU with the next
+        // step's kernels, those get the SMs first
+        int lo = 0, hi = 0;
+        priority_range(lo, hi);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(d.G);
+        cfg.blockDim = dim3(kAttWarps * 32);
+        cfg.dynamicSmemBytes = kUpdateSmem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributePriority;
+        attr[0].val.priority = lo;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, k_update<HG>, s, d, K, n);
     });
 }
 

@@ -91,7 +91,7 @@ def test_corrupt_state_reports_error_without_fault():
     line = [ln for ln in p.stdout.splitlines() if ln.startswith("RESULT ")][-1]
     res = json.loads(line[len("RESULT "):])
     OK, STATE = ckv.CKV_OK, ckv.CKV_ERR_STATE
-    assert res["split_launches"] == 3 and res["fused_launches"] == 1
+    assert res["split_launches"] == 4 and res["fused_launches"] == 1
     for mode in ("split", "fused"):
         for what in (0, 1):
             assert res[f"{mode}_{what}"] == [OK, STATE], (mode, what, res)

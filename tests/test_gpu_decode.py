@@ -294,8 +294,10 @@ def test_per_kernel_profile_eager_and_captured(captured):
         ms, n = ckv.ckv_profile_end(ctx)
         assert n == cfg.steps
         # the fused step has one kernel: its time is ms[0], the selection
-        # and attention spans are then empty
-        timed = ms[:1] if ckv.ckv_step_launches(ctx) == 1 else ms[:3]
+        # and attention spans are then empty; ms[3] is the update kernel's
+        # when ckv_assign_update launches one
+        launches = ckv.ckv_step_launches(ctx)
+        timed = ms[:1] if launches == 1 else ms[:launches]
         assert all(m > 0.0 for m in timed) and all(m >= 0.0 for m in ms) and sum(ms) < 1000.0 * n
         for i in steps:
             ckv.ckv_decode_step(ref_ctx, q[i], K, V, cfg.n0 + i + 1, ref)
@@ -306,3 +308,48 @@ def test_per_kernel_profile_eager_and_captured(captured):
     finally:
         ckv.ckv_destroy(ctx)
         ckv.ckv_destroy(ref_ctx)
+
+
+def test_update_on_a_second_stream_matches_inline(monkeypatch):
+    """ckv_assign_update's kernel run on a second stream, each step of the
+    context waiting for the previous update by an event (as a decoder
+    overlapping it with the next layer does), gives bit for bit the outputs
+    and state of the inline update (CKV_UPDATE=inline: the attention
+    kernel's last slice runs the edges, assignment and update)."""
+    import torch
+    cfg = synth.scaled(synth.LLAMA, batch=2, n_q_heads=8, n_kv_heads=2, n0=4000, n_clusters=125,
+                       budget=300, steps=8, mode=synth.QUERY_GROUP)
+    wl = synth.make_workload(cfg)
+    dev = torch.device("cuda", 0)
+    K, V, q = _torch_view(wl.K, dev), _torch_view(wl.V, dev), _torch_view(wl.q, dev)
+    deferred = ckv.ckv_create(config_for(cfg))
+    monkeypatch.setenv("CKV_UPDATE", "inline")
+    inline = ckv.ckv_create(config_for(cfg))
+    try:
+        assert ckv.ckv_step_launches(deferred) == 4 and ckv.ckv_step_launches(inline) == 3
+        for c in (deferred, inline):
+            ckv.ckv_init_communities(c, wl.labels, 0, cfg.n_comm, K, cfg.n0)
+        main, side = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_a, ev_u = torch.cuda.Event(), torch.cuda.Event()
+        out_d = torch.empty((cfg.batch, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
+        out_i = torch.empty_like(out_d)
+        for i in range(cfg.steps):
+            n = cfg.n0 + i + 1
+            if i:
+                main.wait_event(ev_u)
+            ckv.ckv_decode_step(deferred, q[i], K, V, n, out_d, main.cuda_stream)
+            ev_a.record(main)
+            side.wait_event(ev_a)
+            ckv.ckv_assign_update(deferred, K, n, side.cuda_stream)
+            ev_u.record(side)
+            ckv.ckv_decode_step(inline, q[i], K, V, n, out_i)
+            ckv.ckv_assign_update(inline, K, n)
+            main.synchronize()
+            torch.cuda.synchronize()
+            assert torch.equal(out_d, out_i), f"step {i}: outputs differ"
+        torch.cuda.synchronize()
+        assert ckv.ckv_last_error(deferred) == ckv.CKV_OK and ckv.ckv_last_error(inline) == ckv.CKV_OK
+        assert ckv.ckv_export_state(deferred) == ckv.ckv_export_state(inline)
+    finally:
+        ckv.ckv_destroy(deferred)
+        ckv.ckv_destroy(inline)
