@@ -75,8 +75,8 @@ KERNEL_SOURCES = {
     "k_dense_attention": ("k_dense.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
 }
 PROFILED_TRAFFIC = {
-    "k_score": ("50d47023298fccf9", 139.16185e6),
-    "k_attend": ("50d47023298fccf9", 69.00096e6),
+    "k_score": ("0e2dc2dc48a06a69", 138.51443e6),
+    "k_attend": ("0e2dc2dc48a06a69", 67.85408e6),
     "k_dense_stats": ("1674ed41fb19dce3", 1079.90176e6),
 }
 
