@@ -11,14 +11,18 @@
 //
 // One CTA per (head, 128-row query block), heaviest (longest causal row
 // range) blocks first.  Warp roles:
-//   warp 0      TMA producer: Q block once, then K tiles through a 4-stage
+//   warp 0      TMA producer: Q block once, then K tiles through a 3-stage
 //               ring (128-byte swizzled, the layout tcgen05 reads).
 //   warp 1      allocates 256 TMEM columns (two 128 x 128 fp32
 //               accumulators) and issues tcgen05.mma (kind::f16, bf16 in,
 //               fp32 accumulate, M = N = 128, K = 16 x 8) from one thread.
-//   warps 2..5  epilogue: thread = one query row (its TMEM lane); reads the
-//               row's 128 scores with tcgen05.ld, keeps the online softmax
-//               (max, sum of exp2) and a sorted register top-KM list.
+//   warps 2..17 epilogue, four warps per TMEM lane quarter: thread = one
+//               query row (its TMEM lane) and one 32-column chunk of every
+//               tile; it reads the chunk with tcgen05.ld and keeps the
+//               online softmax (max, sum of exp2) and a sorted register
+//               top-KM list; the four parts of a row merge at the end.
+//               Four warps per quarter keep more independent rows in
+//               flight: the per-row work is a chain of dependent steps.
 // Every mbarrier wait is bounded; a wait that runs out marks row_ptr[h][0]
 // = -1 (an impossible offset), every role leaves its loop, and the TMEM is
 // freed before the CTA exits.
@@ -35,9 +39,11 @@ namespace ckv {
 namespace {
 
 constexpr int kBM = 128, kBN = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 4;                           // K ring of the grouped kernel
 constexpr int kThreads = 192;                        // the grouped kernel: producer, MMA, 4 epilogue warps
-constexpr int kEpiWarps = 8;                         // per-head kernel: two epilogue warps per TMEM lane quarter
+constexpr int kStagesH = 3;                          // K ring of the per-head kernel
+constexpr int kParts = 4;                            // per-head kernel: epilogue warps per TMEM lane quarter
+constexpr int kEpiWarps = 4 * kParts;
 constexpr int kThreadsH = 64 + 32 * kEpiWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kMaxKM = 32;
@@ -47,18 +53,23 @@ constexpr float kLog2eOverSqrtD = 0.12751743082459868f;   // log2(e) / sqrt(128)
 
 struct __align__(1024) PrefillSmem {
     unsigned char q[kTileBytes];
-    unsigned char k[kStages][kTileBytes];
+    unsigned char k[kStagesH][kTileBytes];
     unsigned long long bar_q;
-    unsigned long long bar_kfull[kStages];
-    unsigned long long bar_kempty[kStages];
+    unsigned long long bar_kfull[kStagesH];
+    unsigned long long bar_kempty[kStagesH];
     unsigned long long bar_afull[2];
     unsigned long long bar_aempty[2];
     uint32_t tmem_base;
     int abort;
-    // the second half's row state, merged into the first half's at the end
+    // a part's row state, merged into part 0's at the end
     float xm[kBM][2];
-    float xv[kBM][kMaxKM];
-    int xi[kBM][kMaxKM];   // xv and xi together also stage the epilogue's gated chunks (256 threads x 32 words)
+    union {
+        float stage[32 * kEpiThreads];   // during the loop: a gated chunk's values, column k of thread e at [k * kEpiThreads + e]
+        struct {
+            float v[kBM][kMaxKM];
+            int i[kBM][kMaxKM];
+        } x;                             // at the end: a part's top-KM list per row
+    } u;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
@@ -285,9 +296,7 @@ __device__ __forceinline__ int64_t row_offset(int64_t i, int S, int kappa)
 // go to stats[h][i][2] instead (the first pass of the query-group graph),
 // and a bounded wait that runs out sets the int word after them.
 // group: query heads per KV head (the K rows of head h are those of h / group).
-static_assert(offsetof(PrefillSmem, xi) == offsetof(PrefillSmem, xv) + sizeof(float) * kBM * kMaxKM &&
-                  2 * kBM * kMaxKM >= kEpiThreads * 32,
-              "the staging area spans xv and xi");
+static_assert(sizeof(PrefillSmem) + 1024 <= 227 * 1024, "the per-head kernel's shared memory fits one CTA");
 
 template <int KM, bool STATS>
 __global__ void __launch_bounds__(kThreadsH, 1)
@@ -308,7 +317,7 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < kStages; ++s) { mbar_init(&sm.bar_kfull[s], 1); mbar_init(&sm.bar_kempty[s], 1); }
+        for (int s = 0; s < kStagesH; ++s) { mbar_init(&sm.bar_kfull[s], 1); mbar_init(&sm.bar_kempty[s], 1); }
         for (int b = 0; b < 2; ++b) { mbar_init(&sm.bar_afull[b], 1); mbar_init(&sm.bar_aempty[b], kEpiWarps); }
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -331,16 +340,16 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_load_3d(sm.q + kHalfBytes, &tmQ, &sm.bar_q, 64, i0, h);
             int issued = 0;
             for (int t = 0; t < ntiles; ++t) {
-                const int s = t % kStages;
-                if (!mbar_wait(&sm.bar_kempty[s], ((t / kStages) & 1) ^ 1, abort)) break;
+                const int s = t % kStagesH;
+                if (!mbar_wait(&sm.bar_kempty[s], ((t / kStagesH) & 1) ^ 1, abort)) break;
                 mbar_expect_tx(&sm.bar_kfull[s], kTileBytes);
                 tma_load_3d(sm.k[s], &tmK, &sm.bar_kfull[s], 0, t * kBN, h / group);
                 tma_load_3d(sm.k[s] + kHalfBytes, &tmK, &sm.bar_kfull[s], 64, t * kBN, h / group);
                 issued = t + 1;
             }
             // do not leave with copies in flight: the last load of every stage has landed
-            for (int t = max(0, issued - kStages); t < issued; ++t)
-                mbar_wait(&sm.bar_kfull[t % kStages], (t / kStages) & 1, abort);
+            for (int t = max(0, issued - kStagesH); t < issued; ++t)
+                mbar_wait(&sm.bar_kfull[t % kStagesH], (t / kStagesH) & 1, abort);
             mbar_wait(&sm.bar_q, 0, abort);
         }
     } else if (warp == 1) {
@@ -350,8 +359,8 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (mbar_wait(&sm.bar_q, 0, abort)) {
                 const uint32_t qa = smem_u32(sm.q);
                 for (int t = 0; t < ntiles; ++t) {
-                    const int s = t % kStages, b = t & 1;
-                    if (!mbar_wait(&sm.bar_kfull[s], (t / kStages) & 1, abort)) break;
+                    const int s = t % kStagesH, b = t & 1;
+                    if (!mbar_wait(&sm.bar_kfull[s], (t / kStagesH) & 1, abort)) break;
                     if (!mbar_wait(&sm.bar_aempty[b], ((t >> 1) & 1) ^ 1, abort)) break;
                     tc_fence_after();
                     const uint32_t ka = smem_u32(sm.k[s]);
@@ -375,10 +384,10 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
     } else {
         // ---------------------------------------------------- epilogue
-        // two warps per TMEM lane quarter: thread = one row, half = which
-        // 32-column chunks of every tile it takes (half, half + 2)
+        // kParts warps per TMEM lane quarter: thread = one row, part = the
+        // 32-column chunk of every tile it takes
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
-        const int half = (warp - 2) >> 2;
+        const int part = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
         const int i = i0 + r;
         const bool row_ok = i < n;
@@ -389,7 +398,7 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int k = 0; k < KM; ++k) { vals[k] = -INFINITY; idx[k] = -1; }
         // a gated chunk's values, column k of epilogue thread e at stage[k * kEpiThreads + e]; the
         // merge scratch is free until the loop ends
-        float* stage = &sm.xv[0][0] + (threadIdx.x - 64);
+        float* stage = sm.u.stage + (threadIdx.x - 64);
         auto chunk = [&](const uint32_t (&rv)[32], int j0, bool diag) {
             // causal mask: only the diagonal tile reaches past i
             float v[32];
@@ -447,31 +456,29 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const int b = t & 1;
             if (!mbar_wait(&sm.bar_afull[b], (t >> 1) & 1, abort)) break;
             tc_fence_after();
-            uint32_t ra[32], rb[32];
+            uint32_t ra[32];
             __syncwarp();   // tcgen05.ld is warp-collective
-            tmem_ld32_async(lane_addr + b * kBN + half * 32, ra);
-            tmem_ld32_async(lane_addr + b * kBN + (half + 2) * 32, rb);
+            tmem_ld32_async(lane_addr + b * kBN + part * 32, ra);
             tmem_wait_tie(ra, true);
-            tmem_wait_tie(rb, false);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.bar_aempty[b]);   // the accumulator is read: the MMA may refill it
             const bool diag = t == ntiles - 1;      // the tile holding the block's diagonal
-            chunk(ra, t * kBN + half * 32, diag);
-            chunk(rb, t * kBN + (half + 2) * 32, diag);
+            chunk(ra, t * kBN + part * 32, diag);
         }
-        // the second half hands its row state to the first half
-        epi_sync();
-        if (half == 1) {
-            sm.xm[r][0] = m2;
-            sm.xm[r][1] = l;
-            if constexpr (!STATS) {
+        // parts 1 .. kParts-1 hand their row state to part 0 in turn
+        for (int src = 1; src < kParts; ++src) {
+            epi_sync();   // the staging area (first round) or the previous hand-off is free
+            if (part == src) {
+                sm.xm[r][0] = m2;
+                sm.xm[r][1] = l;
+                if constexpr (!STATS) {
 #pragma unroll
-                for (int k = 0; k < KM; ++k) { sm.xv[r][k] = vals[k]; sm.xi[r][k] = idx[k]; }
+                    for (int k = 0; k < KM; ++k) { sm.u.x.v[r][k] = vals[k]; sm.u.x.i[r][k] = idx[k]; }
+                }
             }
-        }
-        epi_sync();
-        if (half == 0) {
+            epi_sync();
+            if (part != 0) continue;
             const float mo = sm.xm[r][0], lo = sm.xm[r][1];
             const float mn = fmaxf(m2, mo);
             if (mn != -INFINITY) {
@@ -479,12 +486,12 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 m2 = mn;
             }
             if constexpr (!STATS) {
-                // insert the second half's list, ranked by (score desc, j asc)
+                // insert the other part's list, ranked by (score desc, j asc)
                 auto before = [](float a, int ja, float b, int jb) { return a > b || (a == b && ja < jb); };
 #pragma unroll 1
                 for (int k = 0; k < KM; ++k) {
-                    const float a = sm.xv[r][k];
-                    const int j = sm.xi[r][k];
+                    const float a = sm.u.x.v[r][k];
+                    const int j = sm.u.x.i[r][k];
                     if (j < 0 || !before(a, j, vals[KM - 1], idx[KM - 1])) break;   // the rest rank lower
 #pragma unroll
                     for (int p = KM - 1; p > 0; --p) {
@@ -498,6 +505,8 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     if (before(a, j, vals[0], idx[0])) { vals[0] = a; idx[0] = j; }
                 }
             }
+        }
+        if (part == 0) {
             if (STATS && row_ok && !*abort) {
                 stats[((int64_t)h * n + i) * 2] = m2;
                 stats[((int64_t)h * n + i) * 2 + 1] = l;
