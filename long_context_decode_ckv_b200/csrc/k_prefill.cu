@@ -61,6 +61,9 @@ struct __align__(1024) PrefillSmem {
     unsigned long long bar_aempty[2];
     uint32_t tmem_base;
     int abort;
+    // each part's current KM-th best score of each row (a lower bound of the
+    // row's final KM-th: every part gates its candidates by the largest)
+    float thr[kBM][kParts];
     // a part's row state, merged into part 0's at the end
     float xm[kBM][2];
     union {
@@ -272,10 +275,37 @@ __device__ __forceinline__ void insert_staged(unsigned cm, const float* stage, i
     }
 }
 
+// Insert one candidate (value a, column j) into the sorted top-KM list
+// (callers know a ranks above the list's last entry).
+template <int KM>
+__device__ __forceinline__ void insert_one(float a, int j, float (&vals)[KM], int (&idx)[KM])
+{
+#pragma unroll
+    for (int p = KM - 1; p > 0; --p) {
+        const float up = vals[p - 1];
+        const int upi = idx[p - 1];
+        const bool shift = up < a;
+        const bool land = !shift && vals[p] < a;
+        vals[p] = shift ? up : (land ? a : vals[p]);
+        idx[p] = shift ? upi : (land ? j : idx[p]);
+    }
+    if (vals[0] < a) { vals[0] = a; idx[0] = j; }
+}
+
 // barrier 1 among the per-head kernel's epilogue warps only
 __device__ __forceinline__ void epi_sync()
 {
     asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
+}
+
+// the largest float below x (x finite or -inf): "v >= x" is "v > below(x)"
+__device__ __forceinline__ float below(float x)
+{
+    if (x == -INFINITY) return x;
+    const int b = __float_as_int(x);
+    if (x > 0.f) return __int_as_float(b - 1);
+    if (x < 0.f) return __int_as_float(b + 1);
+    return -1.4e-45f;   // below +-0: the negative subnormal of least magnitude
 }
 
 __device__ __forceinline__ float ex2(float x)
@@ -297,6 +327,7 @@ __device__ __forceinline__ int64_t row_offset(int64_t i, int S, int kappa)
 // and a bounded wait that runs out sets the int word after them.
 // group: query heads per KV head (the K rows of head h are those of h / group).
 static_assert(sizeof(PrefillSmem) + 1024 <= 227 * 1024, "the per-head kernel's shared memory fits one CTA");
+static_assert(kParts == 4, "the gate reads a row's four part thresholds");
 
 template <int KM, bool STATS>
 __global__ void __launch_bounds__(kThreadsH, 1)
@@ -399,6 +430,9 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // a gated chunk's values, column k of epilogue thread e at stage[k * kEpiThreads + e]; the
         // merge scratch is free until the loop ends
         float* stage = sm.u.stage + (threadIdx.x - 64);
+        volatile float* thr_row = &sm.thr[r][0];   // the parts of row r (read while others write)
+        thr_row[part] = -INFINITY;
+        epi_sync();
         auto chunk = [&](const uint32_t (&rv)[32], int j0, bool diag) {
             // causal mask: only the diagonal tile reaches past i
             float v[32];
@@ -429,8 +463,13 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int k = 0; k < 32; ++k) pq[k & 3] += ex2(fmaf(v[k], kLog2eOverSqrtD, -m2));
             l += (pq[0] + pq[1]) + (pq[2] + pq[3]);
             if constexpr (!STATS) {
-                // top-KM candidates j in [S, i-1], ranked by the raw score
-                const float thr = vals[KM - 1];
+                // top-KM candidates j in [S, i-1], ranked by the raw score:
+                // above this part's KM-th (a later column loses a tie) and not
+                // below another part's KM-th (KM scores of the row rank at
+                // least that high already; a tie there may still win on j)
+                const float own = vals[KM - 1];
+                const float gate = fmaxf(fmaxf(thr_row[0], thr_row[1]), fmaxf(thr_row[2], thr_row[3]));
+                const float thr = gate > own ? below(gate) : own;
                 if (mc > thr) {   // some column may enter the list
                     unsigned cm = 0u;
                     if (diag || j0 < S) {
@@ -445,9 +484,13 @@ k_prefill_topk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                         for (int k = 0; k < 32; ++k) stage[k * kEpiThreads] = v[k];
                         insert_staged<KM>(cm, stage, kEpiThreads, j0, vals, idx);
-                    } else {
-                        insert_candidates<KM>(cm, v, j0, vals, idx);
+                    } else if (cm) {
+                        if (diag || j0 < S)   // the max may be a masked column (a sink, i itself)
+                            insert_candidates<KM>(cm, v, j0, vals, idx);
+                        else                  // every column is a candidate: the one is the max
+                            insert_one<KM>(mc, j0 + __ffs(cm) - 1, vals, idx);
                     }
+                    thr_row[part] = vals[KM - 1];
                 }
             }
         };
