@@ -349,8 +349,6 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
         const char* v = getenv("CKV_PDL");
         d.pdl = (v && (v[0] == '1' || v[0] == '2')) ? v[0] - '0' : 0;
     }
-    d.nCTA = ckv::attend_grid(d, sms);
-    if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
     {   // the decode step: three kernels (scoring, selection, attention)
         // unless CKV_STEP=fused (one persistent kernel)
         const char* v = getenv("CKV_STEP");
@@ -362,6 +360,8 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
         const char* v = getenv("CKV_UPDATE");
         d.defer_update = !d.fused && !(v && v[0] == 'i');
     }
+    d.nCTA = ckv::attend_grid(d, sms);
+    if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
     d.api = ckv::step_api(d.S, d.budget);
     d.spg = 1;
     d.rows_given = 0;

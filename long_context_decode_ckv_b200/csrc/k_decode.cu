@@ -1037,9 +1037,6 @@ __device__ __forceinline__ void warp_rows_fma(const WarpRows& a, const float* __
     }
 }
 
-// A graph's last slice to finish: merge the slices' partials, rank the
-// edges, and (when fused) assign the new token and update its community.
-// Runs with the whole CTA; red / smem scratch is free.
 // The new token's edges (the top kappa of w = sum_h exp(z - M_h) / L_h over
 // the kept members), its assignment and the community update, for graph g
 // of the step whose output merge left sM (max) and sL (1 / sum) per head.
@@ -1146,13 +1143,17 @@ __device__ __forceinline__ void edges_assign_update(const DevState& s, const Dim
 }
 
 
-template <int HG>
+// A graph's last slice to finish: merge the slices' partials into the
+// output and each head's (m, l); with UPD also rank the edges, assign the
+// new token and update its community.  Runs with the whole CTA; red / smem
+// scratch is free.
+template <int HG, bool UPD>
 __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, int g, int nc, int R,
                                              const void* __restrict__ K, int n, float* __restrict__ out,
                                              unsigned char* scratch, float* sM, float* sL, int* sflag)
 {
     constexpr int NT = kAttWarps * 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     int b, h0, kvh;
     graph_heads(d, g, b, h0, kvh);
     const int T = R - d.S - 1;
@@ -1161,15 +1162,16 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
     const float* pmg = s.part_ml + (int64_t)g * d.nCTA * HG * 2;
     const float* pog = s.part_o + (int64_t)g * d.nCTA * HG * kD;
 
-    // inline update: the first round of kept members and the new token's
-    // key are loaded under the output merge (deferred: k_update loads them)
-    const bool upd = !d.defer_update;
+    // inline update (UPD): the first round of kept members and the new
+    // token's key are loaded under the output merge (else k_update runs it)
     EdgeRows<HG> er;
-    if (upd) edges_load<HG>(d, zrow, rtok, T, 0, er);
     float kv = 0.f;
-    if (upd && d.fuse_assign && tid < kD) {
-        const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + (n - 1)) * kD;
-        kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
+    if constexpr (UPD) {
+        edges_load<HG>(d, zrow, rtok, T, 0, er);
+        if (d.fuse_assign && tid < kD) {
+            const int64_t krow = (((int64_t)b * d.Hkv + kvh) * d.NM + (n - 1)) * kD;
+            kv = d.bf16 ? elem<true>(K, krow + tid) : elem<false>(K, krow + tid);
+        }
     }
     // ---- output: every value merged online over the slices; the thread of
     // a head's first value also leaves that head's max and 1 / sum.  A
@@ -1222,7 +1224,7 @@ __device__ __forceinline__ void finish_graph(const DevState& s, const Dims& d, i
         }
     }
     __syncthreads();
-    if (upd) edges_assign_update<HG>(s, d, g, T, n, kv, er, scratch, sM, sL, sflag);
+    if constexpr (UPD) edges_assign_update<HG>(s, d, g, T, n, kv, er, scratch, sM, sL, sflag);
 }
 
 // CTA work: the graphs' rows laid end to end (graph-major, each graph's
@@ -1242,7 +1244,7 @@ __device__ __forceinline__ int share_of(long long x, long long tot, int P)
     return (int)(((x + 1) * P - 1) / tot);
 }
 
-template <bool BF16, int HG>
+template <bool BF16, int HG, bool UPD>
 __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d, const void* __restrict__ q,
                                                              const void* __restrict__ K,
                                                              const void* __restrict__ V, int n,
@@ -1409,7 +1411,7 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         for (int f = 0; f < nfin; ++f) {
             const Piece pc = sp[sfin[f]];
             __syncthreads();   // the scratch is free
-            finish_graph<HG>(s, d, pc.g, pc.nc, pc.R, K, n, out, smem + L::off_buf, sM, sL, sflag);
+            finish_graph<HG, UPD>(s, d, pc.g, pc.nc, pc.R, K, n, out, smem + L::off_buf, sM, sL, sflag);
             if (tid == 0) s.bar[pc.g * 2] = 0u;
         }
         if (npieces < kMaxPieces) break;
@@ -1517,10 +1519,16 @@ cudaError_t dispatch_hg(int hg, F&& f)
     }
 }
 
-template <bool BF16, int HG>
-void* attend_fn()
+// the attention kernel of a context: fp32 or bf16 rows, HG heads per graph,
+// with the edges, assignment and update inline or left to k_update
+template <int HG>
+void* attend_fn(const Dims& d)
 {
-    return reinterpret_cast<void*>(k_attend<BF16, HG>);
+    if (d.bf16)
+        return d.defer_update ? reinterpret_cast<void*>(k_attend<true, HG, false>)
+                              : reinterpret_cast<void*>(k_attend<true, HG, true>);
+    return d.defer_update ? reinterpret_cast<void*>(k_attend<false, HG, false>)
+                          : reinterpret_cast<void*>(k_attend<false, HG, true>);
 }
 
 template <int HG>
@@ -1595,7 +1603,7 @@ cudaError_t prepare_kernels(const Dims& d)
     if (e != cudaSuccess) return e;
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
-        void* fn = d.bf16 ? attend_fn<true, HG>() : attend_fn<false, HG>();
+        void* fn = attend_fn<HG>(d);
         const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
         cudaError_t e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e2 == cudaSuccess)
@@ -1611,7 +1619,7 @@ int attend_grid(const Dims& d, int sms)
     if (e == cudaSuccess)
         e = dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
             constexpr int HG = decltype(hgc)::value;
-            void* fn = d.bf16 ? attend_fn<true, HG>() : attend_fn<false, HG>();
+            void* fn = attend_fn<HG>(d);
             const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
             return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kAttWarps * 32, bytes);
         });
@@ -1625,11 +1633,18 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
         const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
-        if (d.bf16)
-            return launch_ex(d, k_attend<true, HG>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K, V, n,
-                             out);
-        return launch_ex(d, k_attend<false, HG>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K, V, n,
-                         out);
+        if (d.bf16) {
+            if (d.defer_update)
+                return launch_ex(d, k_attend<true, HG, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d,
+                                 q, K, V, n, out);
+            return launch_ex(d, k_attend<true, HG, true>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K,
+                             V, n, out);
+        }
+        if (d.defer_update)
+            return launch_ex(d, k_attend<false, HG, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q,
+                             K, V, n, out);
+        return launch_ex(d, k_attend<false, HG, true>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K, V,
+                         n, out);
     });
 }
 
