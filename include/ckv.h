@@ -261,9 +261,12 @@ ckv_status ckv_assign_update(ckv_ctx* ctx, const void* K, int n, void* stream);
 /* One whole decode step from host memory: copies the new token's key and
  * value (k_new_host, v_new_host: [B][H_kv][D]) into row n-1 of the device
  * caches K and V, copies q_host ([B][H_q][D]) to the device, runs
- * ckv_decode_step and ckv_assign_update, copies the output to out_host
- * ([B][H_q][D] float32) and synchronises the stream.  Host buffers should
- * be page-locked for the copies to be asynchronous.
+ * ckv_decode_step, copies the output to out_host ([B][H_q][D] float32),
+ * launches ckv_assign_update's kernel and returns once the output has
+ * arrived; the update finishes on `stream` behind it (the next call on the
+ * stream is ordered after it; its device errors surface at the next
+ * ckv_last_error).  Host buffers should be page-locked for the copies to
+ * be asynchronous; all of them may be reused on return.
  * Errors: as the two calls above, plus CKV_ERR_CUDA. */
 ckv_status ckv_decode_host(ckv_ctx* ctx, const void* q_host, const void* k_new_host,
                            const void* v_new_host, void* K, void* V, int n, float* out_host,

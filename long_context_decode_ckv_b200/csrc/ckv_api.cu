@@ -50,6 +50,7 @@ struct ckv_ctx {
     // profiling: one event per kernel boundary of each profiled step
     int profiling;
     std::vector<cudaEvent_t> ev_pool;   // all events ever created (reused)
+    cudaEvent_t host_done;              // ckv_decode_host: its output has reached the host
     size_t ev_used;
     std::vector<std::array<cudaEvent_t, 6>> ev_steps;
     // token graph of every graph on the host (rows [0, tg_rows)): the
@@ -296,6 +297,7 @@ CKV_API void ckv_destroy(ckv_ctx* x)
     cudaSetDevice(x->cfg.device);
     cudaDeviceSynchronize();
     for (cudaEvent_t e : x->ev_pool) cudaEventDestroy(e);
+    if (x->host_done) cudaEventDestroy(x->host_done);
     free_edges(x);
     for (void* p : x->allocs) cudaFree(p);
     if (x->stage) cudaFree(x->stage);
@@ -591,11 +593,15 @@ CKV_API ckv_status ckv_decode_host(ckv_ctx* x, const void* q_host, const void* k
     CKV_CUDA(ckv::launch_append_rows(d, dk, dv, K, V, n - 1, st));
     cs = ckv_decode_step(x, dq, K, V, n, dout, stream);
     if (cs != CKV_OK) return cs;
-    cs = ckv_assign_update(x, K, n, stream);
-    if (cs != CKV_OK) return cs;
+    // the output goes back first; the call returns when it has arrived, and
+    // the update kernel finishes behind it on the stream
     CKV_CUDA(cudaMemcpyAsync(out_host, dout, (size_t)d.B * d.Hq * ckv::kD * sizeof(float),
                              cudaMemcpyDeviceToHost, st));
-    CKV_CUDA(cudaStreamSynchronize(st));
+    if (!x->host_done) CKV_CUDA(cudaEventCreateWithFlags(&x->host_done, cudaEventDisableTiming));
+    CKV_CUDA(cudaEventRecord(x->host_done, st));
+    cs = ckv_assign_update(x, K, n, stream);
+    if (cs != CKV_OK) return cs;
+    CKV_CUDA(cudaEventSynchronize(x->host_done));
     return CKV_OK;
 }
 

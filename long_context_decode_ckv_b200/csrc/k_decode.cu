@@ -1278,8 +1278,10 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
     // is reused).
     const bool aligned = d.att_aligned && (int)gridDim.x >= G;
     int* sR = reinterpret_cast<int*>(smem + L::off_buf);
+    __shared__ int s_failed;   // the step already failed (read with the row count: one round trip)
     if (aligned) {
         if (tid == 0) {
+            const int failed = *(volatile const int*)s.err;
             const int Pa = (int)gridDim.x;
             const int g = (int)(((long long)(blockIdx.x + 1) * G - 1) / Pa);
             const int fa = (int)((long long)g * Pa / G), fb = (int)((long long)(g + 1) * Pa / G);
@@ -1293,11 +1295,14 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
             sp[0] = pc;
             *snp = 1;
             *snf = 0;
+            s_failed = failed;
         }
     } else {
+        if (tid == 0) s_failed = *(volatile const int*)s.err;
         for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
     }
-    if (step_failed(s.err)) return;
+    __syncthreads();
+    if (s_failed) return;
     for (int done = 0;; done += kMaxPieces) {
         if (!aligned && warp == 0) {
             auto rows_of = [&](int g) -> int {
