@@ -362,12 +362,6 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
         const char* v = getenv("CKV_UPDATE");
         d.defer_update = !d.fused && !(v && v[0] == 'i');
     }
-    {   // the selection: one CTA per graph, or with CKV_SELECT=cluster a
-        // cluster of four CTAs per graph where the clusters fit (measured
-        // slower on the Qwen3-8B workload, so not the default)
-        const char* v = getenv("CKV_SELECT");
-        d.sel_cluster = (v && v[0] == 'c') && ckv::select_on_clusters(d, sms);
-    }
     d.nCTA = ckv::attend_grid(d, sms);
     if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
     d.api = ckv::step_api(d.S, d.budget);

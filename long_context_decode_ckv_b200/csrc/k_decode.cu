@@ -23,7 +23,6 @@
 //             to finish merges the (m, l, o) partials, ranks the kept
 //             members' edge weights, assigns the new token by weighted
 //             plurality and updates that community's running mean.
-#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -526,397 +525,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(DevState s, Dims d)
             if (lane < sz) { rtok[r0 + lane] = tk[u]; rcomm[r0 + lane] = cc; }
             for (int j = 32 + lane; j < sz; j += 32) {   // communities longer than a warp
                 rtok[r0 + j] = in ? pool[cof[k] + j] : 0;
-                rcomm[r0 + j] = cc;
-            }
-        }
-    }
-}
-
-// ------------------------------------------------------------ k_select_cl
-// The same selection as k_select -- size-weighted histogram passes, the
-// boundary bin's communities ranked exactly, the kept ids in ascending order
-// and then the boundary's kept ones in rank order, the kept members' rows --
-// with a graph's communities split over the kSCL CTAs of one thread-block
-// cluster: CTA r of the cluster holds the contiguous ids [r Q, (r + 1) Q).
-// The CTAs sum their histograms, gather their candidates and their kept
-// counts through distributed shared memory between cluster barriers, so one
-// SM does a quarter of a graph's per-community work (k_select's time is set
-// by its instruction count on one SM per graph).
-constexpr int kSCL = 4;
-constexpr int kSCThreads = 256;
-constexpr int kSCWarps = kSCThreads / 32;
-constexpr int kSCBinsPT = kSelBins / kSCThreads;   // histogram bins per thread in the boundary scan
-
-template <int E>
-struct SelClLayout {
-    static constexpr int Q = E * kSCThreads;          // communities per CTA
-    static constexpr int LK = Q + kSelCand;           // own kept entries, at most
-    static constexpr size_t off_ckey = 0;                                           // u64 [kSelCand] own candidates
-    static constexpr size_t off_akey = off_ckey + 8 * kSelCand;                      // u64 [kSelCand] every candidate
-    static constexpr size_t off_cwt = off_akey + 8 * kSelCand;                       // int [kSelCand]
-    static constexpr size_t off_ccof = off_cwt + 4 * kSelCand;                       // int [kSelCand]
-    static constexpr size_t off_awt = off_ccof + 4 * kSelCand;                       // int [kSelCand]
-    static constexpr size_t off_kst = off_awt + 4 * kSelCand;                        // int [LK] row start
-    static constexpr size_t off_ksz = off_kst + 4 * (size_t)LK;                      // int [LK] size
-    static constexpr size_t off_kid = off_ksz + 4 * (size_t)LK;                      // int [LK] community
-    static constexpr size_t off_kof = off_kid + 4 * (size_t)LK;                      // int [LK] segment start
-    static constexpr size_t bytes = off_kof + 4 * (size_t)LK;
-};
-
-struct SelClShared {
-    int hist[kSelBins];
-    int n_cand;                     // this CTA's boundary-bin candidates
-    int cnt[4];                     // surely kept: count, sizes; kept boundary candidates: count, sizes
-    int failed;
-    int sh_b, sh_above;
-    int r_w[kSCWarps];
-    unsigned long long kmin, kmax;
-    unsigned long long r_kmin[kSCWarps], r_kmax[kSCWarps];
-};
-
-template <int E>
-__global__ void __cluster_dims__(kSCL, 1, 1) __launch_bounds__(kSCThreads, 1) k_select_cl(DevState s, Dims d)
-{
-    namespace cg = cooperative_groups;
-    using L = SelClLayout<E>;
-    pdl_wait();
-    if (d.pdl == 1) pdl_trigger();
-    cg::cluster_group cl = cg::this_cluster();
-    extern __shared__ __align__(16) unsigned char smem_sel[];
-    __shared__ SelClShared x;
-    __shared__ int off_c[E][kSCWarps], off_w[E][kSCWarps];
-    const int rank = (int)cl.block_rank();
-    const int g = (int)blockIdx.x / kSCL;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int Nc = d.n_comm, budget = d.budget;
-    unsigned long long* ckey = reinterpret_cast<unsigned long long*>(smem_sel + L::off_ckey);
-    unsigned long long* akey = reinterpret_cast<unsigned long long*>(smem_sel + L::off_akey);
-    int* cwt = reinterpret_cast<int*>(smem_sel + L::off_cwt);
-    int* ccof = reinterpret_cast<int*>(smem_sel + L::off_ccof);
-    int* awt = reinterpret_cast<int*>(smem_sel + L::off_awt);
-    int* kst = reinterpret_cast<int*>(smem_sel + L::off_kst);
-    int* ksz = reinterpret_cast<int*>(smem_sel + L::off_ksz);
-    int* kid = reinterpret_cast<int*>(smem_sel + L::off_kid);
-    int* kof = reinterpret_cast<int*>(smem_sel + L::off_kof);
-
-    // ---- 1. this CTA's scores, sizes and segment starts; the graph's score
-    // range and total size (left by k_score); the step's error word, read by
-    // rank 0 for the whole cluster
-    const int c_lo = rank * L::Q;
-    const float* gsc = s.score + (int64_t)g * d.Nc;
-    const int32_t* gsz = s.csize + (int64_t)g * d.Nc;
-    const int32_t* gco = s.coff + (int64_t)g * d.Nc;
-    const int32_t* gpool = s.pool + (int64_t)g * d.P;
-    float v[E];
-    int w[E], co[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        const int c = c_lo + i * kSCThreads + tid;
-        w[i] = (c < Nc) ? gsz[c] : 0;
-        v[i] = (c < Nc) ? gsc[c] : 0.f;
-        co[i] = (c < Nc) ? gco[c] : 0;
-    }
-    const uint4 rg = __ldcg(reinterpret_cast<const uint4*>(s.srange + 4 * g));
-    if (tid == 0) {
-        x.failed = (rank == 0) ? *(volatile const int*)s.err : 0;
-        x.n_cand = 0;
-        x.cnt[0] = x.cnt[1] = x.cnt[2] = x.cnt[3] = 0;
-    }
-#pragma unroll
-    for (int j = 0; j < kSCBinsPT; ++j) x.hist[tid * kSCBinsPT + j] = 0;
-    unsigned cmask = 0u, imask = 0u;
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        if (w[i] > 0) cmask |= 1u << i;
-        else w[i] = 0;
-    }
-    auto from_ord = [](uint32_t u) { return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u); };
-    const bool any = rg.y != 0u;
-    const float lo = any ? from_ord(rg.x) : INFINITY, hi = any ? from_ord(rg.y) : -INFINITY;
-    const int wsum = (int)rg.z;
-    cl.sync();                                             // every CTA read the range; rank 0 the error word
-    if (*cl.map_shared_rank(&x.failed, 0)) {               // the same answer in every CTA
-        cl.sync();                                         // no CTA leaves while a peer reads it
-        return;
-    }
-    if (rank == 0 && tid == 0)
-        *reinterpret_cast<uint4*>(s.srange + 4 * g) = make_uint4(0xffffffffu, 0u, 0u, 0u);   // for the next step
-
-    int m = 0;                                             // boundary-bin candidates of the cluster
-    if (wsum <= budget) {                                  // every community fits: keep them all
-        imask = cmask;
-        cmask = 0u;
-#pragma unroll
-        for (int i = 0; i < E; ++i)
-            if (imask & (1u << i)) prefetch_l2_range(gpool, co[i], w[i], d.P);
-    } else {
-        // ---- 2./3. bucket passes until the boundary bin is small
-        const float scale = (hi > lo) ? (float)kSelBins / (hi - lo) : 0.f;
-        int above = 0;      // size of the communities known to be kept
-        int shift = -1;     // -1: linear in the score; else radix window of the key
-        __syncthreads();    // hist zeroed
-        for (int pass = 0;; ++pass) {
-            if (pass == 8) {   // 64 key bits take at most 6 radix passes: unreachable
-                if (rank == 0 && tid == 0) set_error(s.err, CKV_ERR_STATE);
-                cl.sync();
-                return;
-            }
-            auto bin_of = [&](int i, int c) -> int {
-                if (shift < 0) return min(kSelBins - 1, (int)((v[i] - lo) * scale));
-                return (int)((sel_key(v[i], c) >> shift) & (unsigned long long)(kSelBins - 1));
-            };
-#pragma unroll
-            for (int i = 0; i < E; ++i)
-                if (cmask & (1u << i)) atomicAdd(&x.hist[bin_of(i, c_lo + i * kSCThreads + tid)], w[i]);
-            cl.sync();                                     // every CTA's histogram is complete
-            // boundary bin: the size summed from the top bin down first
-            // exceeds the budget.  Thread t sums bins 2047 - 8t - j over the
-            // cluster (top first).
-            int hb[kSCBinsPT];
-            int xs = 0;
-#pragma unroll
-            for (int j = 0; j < kSCBinsPT; ++j) hb[j] = 0;
-#pragma unroll
-            for (int r = 0; r < kSCL; ++r) {
-                const int* hr = cl.map_shared_rank(x.hist, r);
-#pragma unroll
-                for (int j = 0; j < kSCBinsPT; ++j) hb[j] += hr[kSelBins - 1 - kSCBinsPT * tid - j];
-            }
-#pragma unroll
-            for (int j = 0; j < kSCBinsPT; ++j) xs += hb[j];
-            const int incl = warp_incl(xs, lane);
-            if (lane == 31) x.r_w[warp] = incl;
-            __syncthreads();
-            int wpre = 0;
-#pragma unroll
-            for (int k = 0; k < kSCWarps; ++k) wpre += (k < warp) ? x.r_w[k] : 0;
-            int run = above + wpre + incl - xs;
-#pragma unroll
-            for (int j = 0; j < kSCBinsPT; ++j) {
-                if (run <= budget && run + hb[j] > budget) {
-                    x.sh_b = kSelBins - 1 - kSCBinsPT * tid - j;
-                    x.sh_above = run;
-                }
-                run += hb[j];
-            }
-            cl.sync();                                     // every CTA has read every histogram
-            const int bs = x.sh_b;
-            above = x.sh_above;
-#pragma unroll
-            for (int j = 0; j < kSCBinsPT; ++j) x.hist[tid * kSCBinsPT + j] = 0;
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                if (!(cmask & (1u << i))) continue;
-                const int c = c_lo + i * kSCThreads + tid;
-                const int b = bin_of(i, c);
-                if (b > bs) {
-                    imask |= 1u << i;
-                    cmask &= ~(1u << i);
-                    prefetch_l2_range(gpool, co[i], w[i], d.P);   // its members, for the row copy
-                } else if (b < bs) {
-                    cmask &= ~(1u << i);
-                } else {
-                    const int slot = atomicAdd(&x.n_cand, 1);
-                    if (slot < kSelCand) { ckey[slot] = sel_key(v[i], c); cwt[slot] = w[i]; ccof[slot] = co[i]; }
-                    if (shift < 0) prefetch_l2_range(gpool, co[i], w[i], d.P);   // likely kept too
-                }
-            }
-            // the same kept size and boundary bin in every CTA; the local
-            // histograms are zero again
-            x.sh_above = above;
-            __syncthreads();
-            cl.sync();                                     // every CTA's candidate count is final
-            m = 0;
-#pragma unroll
-            for (int r = 0; r < kSCL; ++r) m += *cl.map_shared_rank(&x.n_cand, r);
-            if (m <= kSelCand) break;                      // uniform
-            // crowded boundary bin: the key range of its communities
-            unsigned long long kmn = ~0ull, kmx = 0ull;
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                if (!(cmask & (1u << i))) continue;
-                const unsigned long long k = sel_key(v[i], c_lo + i * kSCThreads + tid);
-                kmn = min(kmn, k);
-                kmx = max(kmx, k);
-            }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                kmn = min(kmn, __shfl_xor_sync(kFull, kmn, o));
-                kmx = max(kmx, __shfl_xor_sync(kFull, kmx, o));
-            }
-            if (lane == 0) { x.r_kmin[warp] = kmn; x.r_kmax[warp] = kmx; }
-            __syncthreads();
-            if (tid == 0) {
-                unsigned long long a = ~0ull, b = 0ull;
-                for (int k = 0; k < kSCWarps; ++k) { a = min(a, x.r_kmin[k]); b = max(b, x.r_kmax[k]); }
-                x.kmin = a;
-                x.kmax = b;
-            }
-            cl.sync();                                     // every CTA's key range is published
-            kmn = ~0ull;
-            kmx = 0ull;
-#pragma unroll
-            for (int r = 0; r < kSCL; ++r) {
-                kmn = min(kmn, *cl.map_shared_rank(&x.kmin, r));
-                kmx = max(kmx, *cl.map_shared_rank(&x.kmax, r));
-            }
-            // the candidates share every key bit above the highest differing one
-            shift = max(0, 63 - __clzll((long long)(kmn ^ kmx)) - 10);
-            cl.sync();                                     // every CTA has read the counts and ranges
-            if (tid == 0) x.n_cand = 0;
-            __syncthreads();
-        }
-    }
-    // ---- 4. every candidate of the cluster, gathered into each CTA; its
-    // own candidates ranked exactly (each counts the better ones and their
-    // sizes; kept iff the sizes through it fit)
-    const int above = (wsum <= budget) ? 0 : x.sh_above;
-    {
-        int base = 0;
-#pragma unroll
-        for (int r = 0; r < kSCL; ++r) {
-            const int nr = (wsum <= budget) ? 0 : *cl.map_shared_rank(&x.n_cand, r);
-            const unsigned long long* kr = cl.map_shared_rank(ckey, r);
-            const int* wr = cl.map_shared_rank(cwt, r);
-            for (int t = tid; t < nr; t += kSCThreads) {
-                akey[base + t] = kr[t];
-                awt[base + t] = wr[t];
-            }
-            base += nr;
-        }
-    }
-    __syncthreads();
-    const int nloc = (wsum <= budget) ? 0 : x.n_cand;
-    unsigned long long bkey = 0ull;
-    int brank = 0, bpre = 0, bw = 0, bco = 0;
-    bool bkeep = false;
-    if (tid < nloc) {
-        bkey = ckey[tid];
-        bw = cwt[tid];
-        bco = ccof[tid];
-        for (int t = 0; t < m; ++t) {
-            const bool better = akey[t] > bkey;
-            brank += better ? 1 : 0;
-            bpre += better ? awt[t] : 0;
-        }
-        bkeep = (above + bpre + bw <= budget) || (above == 0 && bpre == 0);
-        if (bkeep) { atomicAdd(&x.cnt[2], 1); atomicAdd(&x.cnt[3], bw); }
-    }
-    // ---- 5. this CTA's surely kept ids in ascending order: ballots per 32
-    // ids and one scan of (round, warp) totals
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        const bool kept = (imask >> i) & 1u;
-        const unsigned bal = __ballot_sync(kFull, kept);
-        const int wt = bal ? (int)__reduce_add_sync(kFull, kept ? (unsigned)w[i] : 0u) : 0;
-        if (lane == 0) { off_c[i][warp] = __popc(bal); off_w[i][warp] = wt; }
-    }
-    __syncthreads();
-    if (warp == 0) {   // exclusive offsets in (round, warp) order; lane owns E * kSCWarps / 32 entries
-        constexpr int PL = (E * kSCWarps + 31) / 32;
-        int sc = 0, sw = 0;
-        for (int j = 0; j < PL; ++j) {
-            const int e = lane * PL + j;
-            if (e < E * kSCWarps) {
-                sc += off_c[e / kSCWarps][e % kSCWarps];
-                sw += off_w[e / kSCWarps][e % kSCWarps];
-            }
-        }
-        const int ic = warp_incl(sc, lane), iw = warp_incl(sw, lane);
-        int pc = ic - sc, pw = iw - sw;
-        for (int j = 0; j < PL; ++j) {
-            const int e = lane * PL + j;
-            if (e < E * kSCWarps) {
-                const int a = off_c[e / kSCWarps][e % kSCWarps], b = off_w[e / kSCWarps][e % kSCWarps];
-                off_c[e / kSCWarps][e % kSCWarps] = pc;
-                off_w[e / kSCWarps][e % kSCWarps] = pw;
-                pc += a;
-                pw += b;
-            }
-        }
-        if (lane == 31) { x.cnt[0] = ic; x.cnt[1] = iw; }
-    }
-    __syncthreads();
-    cl.sync();                                             // every CTA's counts are final
-    int Cpre = 0, Tpre = 0, C0 = 0, T0 = 0, BN = 0, BT = 0;
-#pragma unroll
-    for (int r = 0; r < kSCL; ++r) {
-        const int* cr = cl.map_shared_rank(x.cnt, r);
-        const int c0 = cr[0], t0 = cr[1];
-        Cpre += (r < rank) ? c0 : 0;
-        Tpre += (r < rank) ? t0 : 0;
-        C0 += c0;
-        T0 += t0;
-        BN += cr[2];
-        BT += cr[3];
-    }
-    cl.sync();                                             // no CTA reads a peer's shared memory after this
-    const int C = C0 + BN, T = T0 + BT;
-    // ---- 6. the kept list: this CTA's entries (its surely kept ids, then its
-    // kept boundary candidates) with their place in the graph's list
-    int32_t* gsel = s.sel + (int64_t)g * d.Nc;
-    const int C0r = x.cnt[0];
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        const int c = c_lo + i * kSCThreads + tid;
-        const bool kept = (imask >> i) & 1u;
-        const unsigned bal = __ballot_sync(kFull, kept);
-        if (bal == 0u) continue;                                   // warp-uniform
-        const int wk = kept ? w[i] : 0;
-        const int wx = (bal & (bal - 1u)) ? warp_incl(wk, lane) - wk : 0;   // exclusive prefix
-        if (kept) {
-            const int lp = off_c[i][warp] + __popc(bal & ((1u << lane) - 1u));
-            kst[lp] = Tpre + off_w[i][warp] + wx;
-            ksz[lp] = w[i];
-            kid[lp] = c;
-            kof[lp] = co[i];
-            gsel[Cpre + lp] = c;
-        }
-    }
-    if (tid == 0) x.n_cand = C0r;                         // next local slot for kept boundary candidates
-    __syncthreads();
-    if (bkeep) {
-        const int lp = atomicAdd(&x.n_cand, 1);
-        const int c = (int)~(uint32_t)(bkey & 0xffffffffull);
-        kst[lp] = T0 + bpre;
-        ksz[lp] = bw;
-        kid[lp] = c;
-        kof[lp] = bco;
-        gsel[C0 + brank] = c;
-    }
-    if (rank == 0 && tid == 0) {
-        int32_t* meta = s.meta + (int64_t)g * M_COUNT;
-        meta[M_C] = C;
-        meta[M_T] = T;
-        meta[M_ROWS] = d.S + T + 1;
-    }
-    if (d.pdl == 2) pdl_trigger();
-    __syncthreads();
-    // ---- 7. the kept members' rows: warp k copies this CTA's kept entries
-    // k, k + 8, ... (contiguous segments, eight entries' loads in flight)
-    const int nk = x.n_cand;
-    const int32_t* pool = gpool;
-    int32_t* rtok = s.rtok + (int64_t)g * d.NM;
-    int32_t* rcomm = s.rcomm + (int64_t)g * d.NM;
-    for (int k0 = warp; k0 < nk; k0 += 8 * kSCWarps) {
-        int tk[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int k = k0 + u * kSCWarps;
-            const int sz = k < nk ? ksz[k] : 0;
-            // the segment inside the pool (debug build; a bad one reads token 0)
-            const bool in = k < nk && CKV_IN_RANGE(kof[k], 0, (int64_t)d.P - sz + 1, s.err);
-            tk[u] = (in && lane < sz) ? pool[kof[k] + lane] : 0;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int k = k0 + u * kSCWarps;
-            if (k >= nk) break;
-            const int r0 = kst[k], sz = ksz[k], cc = kid[k];
-            const bool in = CKV_IN_RANGE(kof[k], 0, (int64_t)d.P - sz + 1, s.err);
-            if (lane < sz) { rtok[r0 + lane] = tk[u]; rcomm[r0 + lane] = cc; }
-            for (int j = 32 + lane; j < sz; j += 32) {   // communities longer than a warp
-                rtok[r0 + j] = in ? pool[kof[k] + j] : 0;
                 rcomm[r0 + j] = cc;
             }
         }
@@ -1956,36 +1564,8 @@ static cudaError_t launch_select_e(const DevState& s, const Dims& d, cudaStream_
     return launch_ex(d, d.bf16 ? k_score<true> : k_score<false>, dim3(grid), dim3(kScoreThreads), smem, st, s, d, q);
 }
 
-template <int E>
-static cudaError_t launch_select_cl_e(const DevState& s, const Dims& d, cudaStream_t st)
-{
-    return launch_ex(d, k_select_cl<E>, dim3(d.G * kSCL), dim3(kSCThreads), SelClLayout<E>::bytes, st, s, d);
-}
-
-template <int... Es>
-static cudaError_t launch_select_cl_any(int e, const DevState& s, const Dims& d, cudaStream_t st,
-                                        std::integer_sequence<int, Es...>)
-{
-    cudaError_t r = cudaErrorInvalidValue;
-    ((e == Es + 1 ? (r = launch_select_cl_e<Es + 1>(s, d, st), true) : false) || ...);
-    return r;
-}
-
-template <int... Es>
-static cudaError_t prepare_select_cl(std::integer_sequence<int, Es...>)
-{
-    cudaError_t r = cudaSuccess;
-    ((r == cudaSuccess ? (r = cudaFuncSetAttribute(k_select_cl<Es + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)SelClLayout<Es + 1>::bytes)) : r), ...);
-    return r;
-}
-
 cudaError_t launch_select(const DevState& s, const Dims& d, cudaStream_t st)
 {
-    if (d.sel_cluster) {
-        const int e = (d.n_comm + kSCL * kSCThreads - 1) / (kSCL * kSCThreads);
-        return launch_select_cl_any(e < 1 ? 1 : e, s, d, st, std::make_integer_sequence<int, 16>{});
-    }
     switch ((d.n_comm + kSelThreads - 1) / kSelThreads) {
         case 0:
         case 1: return launch_select_e<1>(s, d, st);
@@ -2021,7 +1601,6 @@ cudaError_t prepare_kernels(const Dims& d)
                              (const void*)k_select<16>};
     for (const void* f : sel_fns)
         if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_bytes);
-    if (e == cudaSuccess) e = prepare_select_cl(std::make_integer_sequence<int, 16>{});
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_score<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScoreSmem));
     if (e == cudaSuccess)
@@ -2036,13 +1615,6 @@ cudaError_t prepare_kernels(const Dims& d)
             e2 = cudaFuncSetAttribute(update_fn<HG>(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUpdateSmem);
         return e2;
     });
-}
-
-bool select_on_clusters(const Dims& d, int sms)
-{
-    // a cluster of kSCL CTAs per graph while the clusters fit about two per
-    // SM at once (beyond that the one-CTA selection spreads as well)
-    return (int64_t)d.G * kSCL <= 2 * (int64_t)sms && d.n_comm <= 16 * kSCL * kSCThreads;
 }
 
 int attend_grid(const Dims& d, int sms)

@@ -354,25 +354,3 @@ def test_update_on_a_second_stream_matches_inline(monkeypatch):
         ckv.ckv_destroy(deferred)
         ckv.ckv_destroy(inline)
 
-
-@pytest.mark.parametrize("kw", [
-    dict(),                                                  # linear histogram pass
-    dict(n0=24000, n_clusters=1500, budget=6000, steps=3),   # with zero queries: radix passes
-    dict(budget=8),                                          # forced C = 1
-    dict(budget=10 ** 6),                                    # every community kept
-])
-def test_cluster_selection(kw, monkeypatch):
-    """The selection on a cluster of four CTAs per graph (CKV_SELECT=cluster)
-    keeps exactly the oracle's communities, like the one-CTA selection."""
-    monkeypatch.setenv("CKV_SELECT", "cluster")
-    cfg = synth.scaled(synth.TINY, **kw)
-    wl = synth.make_workload(cfg, workers=WORKERS)
-    if "n_clusters" in kw:
-        wl.q[:] = 0
-    ls = Lockstep(wl)
-    try:
-        for i in range(cfg.steps):
-            ls.step(i)
-        ls.compare_state()
-    finally:
-        ls.close()
