@@ -93,6 +93,15 @@ def test_small_gqa_both_modes(mode):
     run_lockstep(cfg)
 
 
+@pytest.mark.parametrize("group,bf16", [(2, True), (8, True), (4, False), (8, False)])
+def test_query_group_sizes(group, bf16):
+    # query groups of 2 and 8 heads per graph (the tensor-core path) and the
+    # fp32 CUDA-core path with 4 and 8 heads per graph
+    cfg = synth.scaled(synth.LLAMA, batch=2, n_q_heads=2 * group, n_kv_heads=2, n0=3000, n_clusters=100,
+                       budget=300, steps=10, mode=synth.QUERY_GROUP, bf16=bf16)
+    run_lockstep(cfg)
+
+
 def test_llama_per_head_full():
     run_lockstep(synth.LLAMA, compare_every=16)
 
