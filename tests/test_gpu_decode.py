@@ -102,6 +102,21 @@ def test_query_group_sizes(group, bf16):
     run_lockstep(cfg)
 
 
+@pytest.mark.parametrize("name", ["tiny_fp32", "gqa_bf16", "qwen8b_sampled"])
+def test_single_launch_step(name, monkeypatch):
+    """The whole step as one persistent kernel (CKV_STEP=fused: score items,
+    selection and finish workers, attention items) in lockstep with the
+    oracle."""
+    monkeypatch.setenv("CKV_STEP", "fused")
+    if name == "tiny_fp32":
+        run_lockstep(synth.TINY)
+    elif name == "gqa_bf16":
+        run_lockstep(synth.scaled(synth.LLAMA, batch=2, n_q_heads=8, n_kv_heads=2, n0=4000, n_clusters=125,
+                                  budget=300, steps=12, mode=synth.QUERY_GROUP))
+    else:
+        run_lockstep(synth.scaled(synth.QWEN8B, steps=16), tracked=[0, 13, 26, 31], compare_every=0)
+
+
 def test_llama_per_head_full():
     run_lockstep(synth.LLAMA, compare_every=16)
 
