@@ -7,7 +7,7 @@
 // assign it to a community in constant time; Table 1: O(sqrt(n) d)
 // retrieval, O(d) update.
 //
-// Three kernels per step:
+// Four kernels per step:
 //   k_score   centroid GEMV (HBM-bound): a persistent TMA ring of 16 KB
 //             units (32 communities), lane = 4 dims, the 32 partial dots
 //             reduced by a butterfly transpose.
@@ -20,9 +20,13 @@
 //             gathers its own run of K and V rows (16-byte cp.async) and,
 //             for bf16, runs both contractions on the tensor cores
 //             (mma.sync) with an online softmax; the last slice of a graph
-//             to finish merges the (m, l, o) partials, ranks the kept
-//             members' edge weights, assigns the new token by weighted
-//             plurality and updates that community's running mean.
+//             to finish merges the (m, l, o) partials into the output and
+//             each head's (m, l).
+//   k_update  (ckv_assign_update, lowest priority) one CTA per graph ranks
+//             the kept members' edge weights, assigns the new token by
+//             weighted plurality and updates that community's running
+//             mean.  With d.defer_update off, k_attend's last slice runs
+//             the same code instead.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
