@@ -75,8 +75,8 @@ KERNEL_SOURCES = {
     "k_dense_attention": ("k_dense.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
 }
 PROFILED_TRAFFIC = {
-    "k_score": ("9a882f3338174ae7", 138.430464e6),
-    "k_attend": ("9a882f3338174ae7", 67.989504e6),
+    "k_score": ("4200f03a029f82d5", 138.430464e6),
+    "k_attend": ("4200f03a029f82d5", 67.989504e6),
     "k_dense_stats": ("1674ed41fb19dce3", 1079.90176e6),
 }
 
