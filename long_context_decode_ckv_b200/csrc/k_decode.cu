@@ -80,6 +80,11 @@ constexpr int kScoreCW = 8;
 constexpr int kScoreThreads = 32 * (1 + kScoreCW);
 constexpr int kScoreNST = 8;
 constexpr int kScoreStage = 32 * kD * 4;
+// unit u goes through slot u % kScoreNST and is read by warp u % kScoreCW:
+// every slot must belong to one consumer warp, so that its mbarrier phases
+// complete in the order that warp waits for them (a parity wait on a phase
+// two generations ahead would pass at once)
+static_assert(kScoreNST % kScoreCW == 0, "each ring slot is read by a single consumer warp");
 
 struct ScoreSmem {
     unsigned char ring[kScoreNST][kScoreStage];
