@@ -362,6 +362,13 @@ CKV_API ckv_status ckv_create(const ckv_config* cfg, ckv_ctx** out)
         const char* v = getenv("CKV_UPDATE");
         d.defer_update = !d.fused && !(v && v[0] == 'i');
     }
+    {   // with the deferred update and at most a quarter as many graphs as
+        // SMs, the attention runs as one cluster of four CTAs per graph
+        // whose slices merge in distributed shared memory, unless
+        // CKV_ATT_CLUSTER=0
+        const char* v = getenv("CKV_ATT_CLUSTER");
+        d.att_cluster = !(v && v[0] == '0') && !d.fused && ckv::attend_on_clusters(d, sms);
+    }
     d.nCTA = ckv::attend_grid(d, sms);
     if (d.nCTA < 1) { delete x; return CKV_ERR_CUDA; }
     d.api = ckv::step_api(d.S, d.budget);

@@ -90,6 +90,7 @@ struct Dims {
     int n_comm;              // communities in use (set at init)
     int n_init;              // first decode position (edge store row 0)
     int defer_update;        // edges, assignment and update run in k_update (ckv_assign_update)
+    int att_cluster;         // the attention runs as one cluster of 4 CTAs per graph (merge in shared memory)
     int fuse_assign;         // the attention kernel also assigns the new token and updates
     int att_aligned;         // attention CTAs split graph by graph (else the rows evenly)
     int pdl;                 // programmatic dependent launch: 0 off, 1 trigger at kernel start, 2 after the main work
@@ -120,6 +121,7 @@ size_t select_smem_bytes(int n_comm, int budget);
 // number of co-resident CTAs of the attention kernel (0 on error)
 cudaError_t prepare_kernels(const Dims& d);
 int attend_grid(const Dims& d, int sms);
+bool attend_on_clusters(const Dims& d, int sms);
 constexpr int kMaxCommunities = 16384;   // k_select holds 16 of a graph's communities per thread
 
 // the fused step (k_step.cu): scoring, selection, attention, edges, vote

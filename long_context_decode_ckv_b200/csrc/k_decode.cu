@@ -27,6 +27,7 @@
 //             weighted plurality and updates that community's running
 //             mean.  With d.defer_update off, k_attend's last slice runs
 //             the same code instead.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -1253,7 +1254,14 @@ __device__ __forceinline__ int share_of(long long x, long long tot, int P)
     return (int)(((x + 1) * P - 1) / tot);
 }
 
-template <bool BF16, int HG, bool UPD>
+// kAttCluster CTAs per graph, one thread-block cluster, when CL: each CTA
+// leaves its slice's partial in its own shared memory and the cluster's
+// rank 0 merges the four through distributed shared memory (no partials in
+// global memory, no arrival counter)
+constexpr int kAttCluster = 4;
+constexpr int kAttClPart = 64 * 1024;   // the cluster partial's offset in the (free) pipeline area
+
+template <bool BF16, int HG, bool UPD, bool CL>
 __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d, const void* __restrict__ q,
                                                              const void* __restrict__ K,
                                                              const void* __restrict__ V, int n,
@@ -1292,8 +1300,9 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         if (tid == 0) {
             const int failed = *(volatile const int*)s.err;
             const int Pa = (int)gridDim.x;
-            const int g = (int)(((long long)(blockIdx.x + 1) * G - 1) / Pa);
-            const int fa = (int)((long long)g * Pa / G), fb = (int)((long long)(g + 1) * Pa / G);
+            const int g = CL ? (int)blockIdx.x / kAttCluster : (int)(((long long)(blockIdx.x + 1) * G - 1) / Pa);
+            const int fa = CL ? g * kAttCluster : (int)((long long)g * Pa / G);
+            const int fb = CL ? fa + kAttCluster : (int)((long long)(g + 1) * Pa / G);
             Piece pc;
             pc.g = g;
             pc.k = (int)blockIdx.x - fa;
@@ -1311,7 +1320,9 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
         for (int g = tid; g < G; g += NT) sR[g] = s.meta[(int64_t)g * M_COUNT + M_ROWS];
     }
     __syncthreads();
-    if (s_failed) return;
+    // (CL: no early exit -- every CTA of a cluster must reach its barriers;
+    // a failed step's rows are checked tokens of a consistent row list)
+    if (!CL && s_failed) return;
     for (int done = 0;; done += kMaxPieces) {
         if (!aligned && warp == 0) {
             auto rows_of = [&](int g) -> int {
@@ -1389,8 +1400,10 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
             }
             __syncthreads();
             // combine the warps: (m, l, acc) -> this slice's partial per head
-            float* po = s.part_o + ((int64_t)g * d.nCTA + k) * HG * kD;
-            float* pm = s.part_ml + ((int64_t)g * d.nCTA + k) * HG * 2;
+            // (CL: into this CTA's shared memory, past the reduction area)
+            float* po = CL ? reinterpret_cast<float*>(smem + L::off_buf + kAttClPart)
+                           : s.part_o + ((int64_t)g * d.nCTA + k) * HG * kD;
+            float* pm = CL ? po + HG * kD : s.part_ml + ((int64_t)g * d.nCTA + k) * HG * 2;
             for (int i = tid; i < HG * kD; i += NT) {
                 const int h = i / kD, dd = i % kD;
                 float mw[kAttWarps];
@@ -1410,6 +1423,45 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
                 }
                 po[i] = o;
                 if (dd == 0) *reinterpret_cast<float2*>(pm + h * 2) = make_float2(M, l);
+            }
+            if constexpr (CL) {
+                static_assert(kAttWarps * HG * L::RSTR * 4 <= kAttClPart &&
+                                  kAttClPart + (HG * kD + 2 * HG) * 4 <= kAttWarps * L::WBUF,
+                              "the cluster partial lies in the pipelines, past the reduction");
+                // ---- the cluster's four partials merged by its rank 0
+                namespace cg = cooperative_groups;
+                cg::cluster_group cl = cg::this_cluster();
+                cl.sync();                                   // every slice's partial is in place
+                if (cl.block_rank() == 0) {
+                    int b, h0, kvh;
+                    graph_heads(d, g, b, h0, kvh);
+                    for (int i = tid; i < HG * kD; i += NT) {
+                        const int h = i / kD;
+                        float mr[kAttCluster], orr[kAttCluster], lr[kAttCluster];
+                        float M = -INFINITY;
+#pragma unroll
+                        for (int r = 0; r < kAttCluster; ++r) {
+                            const float* pr = cl.map_shared_rank(po, r);
+                            const float2 ml = *reinterpret_cast<const float2*>(pr + HG * kD + h * 2);
+                            mr[r] = ml.x;
+                            lr[r] = ml.y;
+                            orr[r] = pr[i];
+                            M = fmaxf(M, mr[r]);
+                        }
+                        float o = 0.f, l = 0.f;
+#pragma unroll
+                        for (int r = 0; r < kAttCluster; ++r) {
+                            const float f = (mr[r] == -INFINITY) ? 0.f : __expf(mr[r] - M);
+                            o = fmaf(orr[r], f, o);
+                            l = fmaf(lr[r], f, l);
+                        }
+                        out[((int64_t)b * d.Hq + h0 + h) * kD + i % kD] = o / l;
+                        if (i % kD == 0 && s.sel_ml)
+                            *reinterpret_cast<float2*>(s.sel_ml + 2 * ((int64_t)b * d.Hq + h0 + h)) = make_float2(M, l);
+                    }
+                }
+                cl.sync();                                   // no slice leaves before rank 0 has read it
+                return;
             }
             // ---- the last slice of a graph to arrive finishes it
             __threadfence();
@@ -1538,11 +1590,14 @@ cudaError_t dispatch_hg(int hg, F&& f)
 template <int HG>
 void* attend_fn(const Dims& d)
 {
+    if (d.att_cluster)
+        return d.bf16 ? reinterpret_cast<void*>(k_attend<true, HG, false, true>)
+                      : reinterpret_cast<void*>(k_attend<false, HG, false, true>);
     if (d.bf16)
-        return d.defer_update ? reinterpret_cast<void*>(k_attend<true, HG, false>)
-                              : reinterpret_cast<void*>(k_attend<true, HG, true>);
-    return d.defer_update ? reinterpret_cast<void*>(k_attend<false, HG, false>)
-                          : reinterpret_cast<void*>(k_attend<false, HG, true>);
+        return d.defer_update ? reinterpret_cast<void*>(k_attend<true, HG, false, false>)
+                              : reinterpret_cast<void*>(k_attend<true, HG, true, false>);
+    return d.defer_update ? reinterpret_cast<void*>(k_attend<false, HG, false, false>)
+                          : reinterpret_cast<void*>(k_attend<false, HG, true, false>);
 }
 
 template <int HG>
@@ -1626,6 +1681,11 @@ cudaError_t prepare_kernels(const Dims& d)
     });
 }
 
+bool attend_on_clusters(const Dims& d, int sms)
+{
+    return d.defer_update && d.att_aligned && (int64_t)d.G * kAttCluster <= sms;
+}
+
 int attend_grid(const Dims& d, int sms)
 {
     int occ = 0;
@@ -1647,18 +1707,38 @@ cudaError_t launch_attend(const DevState& s, const Dims& d, const void* q, const
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
         const int bytes = d.bf16 ? AttLayout<true, HG>::bytes : AttLayout<false, HG>::bytes;
+        if (d.att_cluster) {   // kAttCluster CTAs per graph in one cluster
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(d.G * kAttCluster);
+            cfg.blockDim = dim3(kAttWarps * 32);
+            cfg.dynamicSmemBytes = bytes;
+            cfg.stream = st;
+            int lo = 0, hi = 0;
+            priority_range(lo, hi);
+            cudaLaunchAttribute attr[2];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = kAttCluster;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            attr[1].id = cudaLaunchAttributePriority;
+            attr[1].val.priority = hi;
+            cfg.attrs = attr;
+            cfg.numAttrs = 2;
+            if (d.bf16) return cudaLaunchKernelEx(&cfg, k_attend<true, HG, false, true>, s, d, q, K, V, n, out);
+            return cudaLaunchKernelEx(&cfg, k_attend<false, HG, false, true>, s, d, q, K, V, n, out);
+        }
         if (d.bf16) {
             if (d.defer_update)
-                return launch_ex(d, k_attend<true, HG, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d,
-                                 q, K, V, n, out);
-            return launch_ex(d, k_attend<true, HG, true>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K,
-                             V, n, out);
+                return launch_ex(d, k_attend<true, HG, false, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st,
+                                 s, d, q, K, V, n, out);
+            return launch_ex(d, k_attend<true, HG, true, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s,
+                             d, q, K, V, n, out);
         }
         if (d.defer_update)
-            return launch_ex(d, k_attend<false, HG, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q,
-                             K, V, n, out);
-        return launch_ex(d, k_attend<false, HG, true>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q, K, V,
-                         n, out);
+            return launch_ex(d, k_attend<false, HG, false, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s,
+                             d, q, K, V, n, out);
+        return launch_ex(d, k_attend<false, HG, true, false>, dim3(d.nCTA), dim3(kAttWarps * 32), bytes, st, s, d, q,
+                         K, V, n, out);
     });
 }
 
