@@ -75,8 +75,8 @@ KERNEL_SOURCES = {
     "k_dense_attention": ("k_dense.cu", "warp_mma.cuh", "dev_async.cuh", "ckv_internal.cuh"),
 }
 PROFILED_TRAFFIC = {
-    "k_score": ("df382b38a1c852de", 138.591232e6),
-    "k_attend": ("df382b38a1c852de", 67.92192e6),
+    "k_score": ("88429c0b21494fe5", 138.591232e6),
+    "k_attend": ("88429c0b21494fe5", 67.92192e6),
     "k_dense_stats": ("1674ed41fb19dce3", 1079.90176e6),
 }
 

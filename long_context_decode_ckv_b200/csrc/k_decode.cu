@@ -1489,9 +1489,12 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_attend(DevState s, Dims d
 // per graph computes the new token's edges, assignment and community update
 // from what the step's attention kernel left -- each head's softmax max and
 // sum over the attended rows (sel_ml), the kept members' logits (zrow) and
-// rows (rtok, rcomm).  A step that already failed changes no state.
+// rows (rtok, rcomm).  A step that already failed changes no state.  It
+// runs beside the next step's scan: at most 96 registers a thread, so that
+// one update CTA (two warps per SM sub-partition) and one scan CTA (three
+// warps on one sub-partition) fit in a sub-partition's 16 K registers.
 template <int HG>
-__global__ void __launch_bounds__(kAttWarps * 32, 1) k_update(DevState s, Dims d, const void* __restrict__ K, int n)
+__global__ void __maxnreg__(96) k_update(DevState s, Dims d, const void* __restrict__ K, int n)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     float* sM = reinterpret_cast<float*>(smem + sizeof(EdgeScratch));   // [8]
@@ -1519,6 +1522,7 @@ __global__ void __launch_bounds__(kAttWarps * 32, 1) k_update(DevState s, Dims d
 }
 
 constexpr size_t kUpdateSmem = sizeof(EdgeScratch) + 24 * 4;
+static_assert(sizeof(ScoreSmem) + kUpdateSmem + 2 * 1024 <= 228 * 1024, "a scan CTA and an update CTA share an SM");
 
 // new token's K and V rows: staging [B][H_kv][D] -> cache row `row`
 __global__ void k_append(const uint32_t* __restrict__ knew, const uint32_t* __restrict__ vnew,
@@ -1665,10 +1669,14 @@ cudaError_t prepare_kernels(const Dims& d)
                              (const void*)k_select<16>};
     for (const void* f : sel_fns)
         if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_bytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_score<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScoreSmem));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_score<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScoreSmem));
+    // the scan and the update kernel (side stream) share SMs: both ask for
+    // the largest shared-memory carveout, so that a scan CTA never waits
+    // for an SM's update CTA to leave (their registers fit together too)
+    for (const void* f : {(const void*)k_score<true>, (const void*)k_score<false>}) {
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScoreSmem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    }
     if (e != cudaSuccess) return e;
     return dispatch_hg(d.HG, [&](auto hgc) -> cudaError_t {
         constexpr int HG = decltype(hgc)::value;
@@ -1677,6 +1685,9 @@ cudaError_t prepare_kernels(const Dims& d)
         cudaError_t e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e2 == cudaSuccess)
             e2 = cudaFuncSetAttribute(update_fn<HG>(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUpdateSmem);
+        if (e2 == cudaSuccess)
+            e2 = cudaFuncSetAttribute(update_fn<HG>(), cudaFuncAttributePreferredSharedMemoryCarveout,
+                                      cudaSharedmemCarveoutMaxShared);
         return e2;
     });
 }
