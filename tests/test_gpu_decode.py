@@ -80,6 +80,42 @@ def test_tied_scores_take_the_radix_passes():
         ls.close()
 
 
+def test_one_community_far_above_the_rest():
+    # one community's keys far along the query direction: its score sits far
+    # above every other, so the upper half of the score range holds only it
+    # (less than the budget) and the linear histogram crowds every other
+    # community into its lowest bins; the boundary lies among them.
+    cfg = synth.scaled(synth.TINY, n0=8000, n_clusters=400, budget=600, steps=4)
+    wl = synth.make_workload(cfg, workers=WORKERS)
+    S, D = cfg.n_sinks, cfg.head_dim
+    rng = np.random.default_rng(synth.BASE_SEED + 91)
+    u = rng.standard_normal(D)
+    u /= np.linalg.norm(u)
+    lab = wl.labels[0]
+    c_star = int(lab[S])
+    members = np.nonzero(lab[S:cfg.n0] == c_star)[0] + S
+    wl.K[0, 0, members] = (30.0 * u).astype(np.float32)
+    wl.q[:, 0, 0] = (u + 0.01 * rng.standard_normal((cfg.steps, D))).astype(np.float32)
+    # the case holds at the first step: the initial centroids (member means)
+    # that score in the upper half of the range hold no more than the budget
+    pos = np.arange(S, cfg.n0)
+    mu = np.zeros((cfg.n_comm, D))
+    size = np.zeros(cfg.n_comm, np.int64)
+    np.add.at(mu, lab[pos], wl.K[0, 0, pos].astype(np.float64))
+    np.add.at(size, lab[pos], 1)
+    live = size > 0
+    sc = (mu[live] / size[live, None]) @ wl.q[0, 0, 0].astype(np.float64)
+    upper = sc >= sc.min() + 0.5 * (sc.max() - sc.min())
+    assert size[live][upper].sum() <= cfg.budget < size.sum()
+    ls = Lockstep(wl)
+    try:
+        for i in range(cfg.steps):
+            ls.step(i)
+        ls.compare_state()
+    finally:
+        ls.close()
+
+
 def test_small_slack_relocates_segments():
     # slack 0: every append past the initial size moves the community segment
     cfg = synth.scaled(synth.TINY, n0=512, n_clusters=2, steps=40)
